@@ -1,0 +1,224 @@
+"""Oracle of the sparse MoE layer forward (test infrastructure only; see package docstring).
+
+Notation: T tokens, H hidden (5120 in [P1] "Status": router GEMM (5120, 256)), E routed
+experts (256), k chosen per token (8; [P2] "Overview"), I expert intermediate size.
+
+Steps, in order ([P1] "Status"/"Remaining work", [P2] "Overview"/"Variants", [P3]
+"Agents worked on the serving path"):
+  1. router logits l = x W_r^T, x BF16 and W_r FP32 taken exactly, accumulated in FP64
+  2. p = softmax over all E logits
+  3. the k experts of largest p (equal p: lower expert index first), in descending p
+  4. w_j = p_j / sum of the chosen p (renormalisation over the chosen k)
+  5. token -> expert histogram, exclusive prefix sum (offsets), and the permutation
+     that lists the rows of expert e in [offsets[e], offsets[e+1]) in ascending token order
+  6. A1 = Q(x, alpha_a1)                              (NVFP4 activation, W4A4)
+  7. G = deq(A1) deq(W_gate)^T, U = deq(A1) deq(W_up)^T  per expert (FP64)
+  8. h = G * sigmoid(G) * U                           (SwiGLU), rounded to FP32
+  9. A2 = Q(h, alpha_a2)
+ 10. y = deq(A2) deq(W_down)^T                        (FP64)
+ 11. m = sum_j w_j y_j                                (weighted un-permute, MoE finalize)
+ 12. n = m / sqrt(mean(m^2) + eps) * gamma            (post-RMSNorm of the sandwich norm)
+ 13. out = bf16_rne(residual + n)                     (residual add)
+Readings where the pages are silent: gate rows are the first I rows of the stored
+gate/up weight, up rows the last I; no bias, no clamp, no shared expert; RMSNorm is the
+plain gamma * x_hat form; the output is rounded to BF16 once, from the exact sum.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .nvfp4 import dequantize_nvfp4, quantize_nvfp4, tensor_scale
+
+
+# ----------------------------------------------------------------------------- routing
+def router_logits(x: np.ndarray, router_w: np.ndarray) -> np.ndarray:
+    """Step 1: l[t, e] = sum_h x[t, h] * W_r[e, h] in FP64 ([P1] "Status": (5120, 256))."""
+    return np.asarray(x, np.float64) @ np.asarray(router_w, np.float64).T
+
+
+def route_topk(logits: np.ndarray, k: int):
+    """Steps 2-4 ([P2] "Overview": each token goes to 8 of 256 experts).
+
+    Returns ids [T, k] (int64, descending p, ties to the lower index), w [T, k] (FP64,
+    renormalised over the chosen k) and p [T, E] (softmax over all experts).
+    """
+    l = np.asarray(logits, np.float64)
+    z = np.exp(l - l.max(axis=1, keepdims=True))
+    p = z / z.sum(axis=1, keepdims=True)
+    # A stable sort of -p keeps equal probabilities in ascending index order.
+    order = np.argsort(-p, axis=1, kind="stable")
+    ids = order[:, :k]
+    psel = np.take_along_axis(p, ids, axis=1)
+    w = psel / psel.sum(axis=1, keepdims=True)
+    return ids.astype(np.int64), w, p
+
+
+def near_tie_mask(logits: np.ndarray, k: int, rel: float = 1e-5) -> np.ndarray:
+    """Tokens whose k-th and (k+1)-th largest logits differ by less than
+    rel * max(|l_k|, |l_k+1|, 1); their choice of expert is not unique at FP32-class
+    precision, so exact-match checks of routing skip and count them."""
+    l = np.asarray(logits, np.float64)
+    if k >= l.shape[1]:
+        return np.zeros(l.shape[0], dtype=bool)
+    srt = -np.sort(-l, axis=1)
+    a, b = srt[:, k - 1], srt[:, k]
+    return (a - b) < rel * np.maximum(np.maximum(np.abs(a), np.abs(b)), 1.0)
+
+
+def permute(ids: np.ndarray, num_experts: int):
+    """Step 5: histogram, exclusive scan and the stable (expert, token) permutation.
+
+    Returns counts [E], offsets [E+1], perm_src [T*k] (token of permuted row r),
+    perm_slot [T*k] (slot j of that row) and inv [T, k] (permuted row of (t, j)).
+    """
+    ids = np.asarray(ids, np.int64)
+    t_count, k = ids.shape
+    flat_e = ids.reshape(-1)
+    flat_t = np.repeat(np.arange(t_count), k)
+    flat_j = np.tile(np.arange(k), t_count)
+    counts = np.bincount(flat_e, minlength=num_experts).astype(np.int64)
+    offsets = np.zeros(num_experts + 1, np.int64)
+    offsets[1:] = np.cumsum(counts)
+    # Sort by expert, then by token (lexsort: last key is primary).
+    order = np.lexsort((flat_t, flat_e))
+    perm_src = flat_t[order]
+    perm_slot = flat_j[order]
+    inv = np.empty((t_count, k), np.int64)
+    inv[perm_src, perm_slot] = np.arange(t_count * k)
+    return dict(counts=counts, offsets=offsets, perm_src=perm_src, perm_slot=perm_slot, inv=inv)
+
+
+# ----------------------------------------------------------------------------- experts
+def quantize_expert(w_gu: np.ndarray, w_d: np.ndarray):
+    """NVFP4 weights of one expert ([P2] "Variants": routed experts are NVFP4).
+
+    w_gu: FP32 [2I, H] (rows 0..I-1 gate, I..2I-1 up); w_d: FP32 [H, I].
+    One tensor scale for gate+up together and one for down, each amax / 2688.
+    """
+    a_gu = tensor_scale(w_gu)
+    a_d = tensor_scale(w_d)
+    gu_p, gu_s = quantize_nvfp4(w_gu, a_gu)
+    d_p, d_s = quantize_nvfp4(w_d, a_d)
+    return dict(w_gu=gu_p, w_gu_sf=gu_s, w_gu_alpha=a_gu, w_d=d_p, w_d_sf=d_s, w_d_alpha=a_d)
+
+
+def dequantize_expert(q):
+    """FP64 gate/up [2I, H] and down [H, I] of a quantised expert."""
+    return (
+        dequantize_nvfp4(q["w_gu"], q["w_gu_sf"], q["w_gu_alpha"]),
+        dequantize_nvfp4(q["w_d"], q["w_d_sf"], q["w_d_alpha"]),
+    )
+
+
+def swiglu(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """Step 8 before rounding: silu(g) * u = g * sigmoid(g) * u, FP64."""
+    return g / (1.0 + np.exp(-g)) * u
+
+
+def expert_forward(a1_packed, a1_sf, alpha_a1, deq_w, alpha_a2):
+    """Steps 7-10 for the rows routed to one expert.
+
+    a1_packed/a1_sf: NVFP4 rows of that expert's inputs; deq_w: (gate/up, down) in FP64.
+    Returns dict(h32 [R, I] FP32, a2_packed, a2_sf, y [R, H] FP64).
+    """
+    w_gu, w_d = deq_w
+    inter = w_gu.shape[0] // 2
+    a1 = dequantize_nvfp4(a1_packed, a1_sf, alpha_a1)
+    g = a1 @ w_gu[:inter].T
+    u = a1 @ w_gu[inter:].T
+    h32 = swiglu(g, u).astype(np.float32)
+    a2_packed, a2_sf = quantize_nvfp4(h32, alpha_a2)
+    a2 = dequantize_nvfp4(a2_packed, a2_sf, alpha_a2)
+    y = a2 @ w_d.T
+    return dict(h32=h32, a2_packed=a2_packed, a2_sf=a2_sf, y=y)
+
+
+# ----------------------------------------------------------------------------- finalize
+def bf16_round(z: np.ndarray) -> np.ndarray:
+    """Round FP64 values to the nearest BF16 (8 significant bits), ties to even; returns
+    the rounded values as FP64 (finite inputs within the BF16 range)."""
+    z = np.asarray(z, np.float64)
+    f, ex = np.frexp(z)  # z = f * 2**ex, |f| in [0.5, 1)
+    q = np.ldexp(1.0, ex - 8)  # step of an 8-bit significand in that binade
+    out = np.rint(z / q) * q
+    # BF16 keeps the FP32 exponent range; below 2^-126 the step stays 2^-133.
+    tiny = np.abs(z) < 2.0 ** -126
+    if np.any(tiny):
+        out[tiny] = np.rint(z[tiny] / 2.0 ** -133) * 2.0 ** -133
+    return out
+
+
+def finalize(y_sel: np.ndarray, w: np.ndarray, residual: np.ndarray, gamma: np.ndarray, eps: float):
+    """Steps 11-13 ([P1] "Remaining work": MoE finalize; "Status": sandwich norms).
+
+    y_sel: [T, k, H] expert outputs of each token's chosen experts, w: [T, k].
+    Returns (pre-rounding FP64 output [T, H], BF16-rounded output as FP64 [T, H], m).
+    """
+    m = np.einsum("tk,tkh->th", np.asarray(w, np.float64), np.asarray(y_sel, np.float64))
+    rms = np.sqrt(np.mean(m * m, axis=1, keepdims=True) + eps)
+    n = m / rms * np.asarray(gamma, np.float64)[None, :]
+    pre = np.asarray(residual, np.float64) + n
+    return pre, bf16_round(pre), m
+
+
+# ----------------------------------------------------------------------------- forward
+class ExpertCache:
+    """Quantises (with this oracle's quantiser) and dequantises experts on first use.
+
+    get_fp32(e) must return the FP32 weights (w_gu [2I, H], w_d [H, I]) of expert e.
+    """
+
+    def __init__(self, get_fp32, keep: int = 64):
+        self.get_fp32 = get_fp32
+        self.keep = keep
+        self._deq = {}
+        self._q = {}
+
+    def quantized(self, e: int):
+        if e not in self._q:
+            w_gu, w_d = self.get_fp32(e)
+            self._q[e] = quantize_expert(w_gu, w_d)
+        return self._q[e]
+
+    def dequantized(self, e: int):
+        if e not in self._deq:
+            if len(self._deq) >= self.keep:
+                self._deq.pop(next(iter(self._deq)))
+            self._deq[e] = dequantize_expert(self.quantized(e))
+        return self._deq[e]
+
+
+def moe_forward_tokens(x, residual, router_w, gamma, experts: ExpertCache, top_k, alpha_a1, alpha_a2,
+                       eps=1e-6):
+    """Steps 1-4 and 6-13 for a set of tokens (each token's output depends on that token
+    only, so any subset of a batch gives the same rows as the whole batch).
+
+    x, residual: FP64 [T, H] (exact BF16 values).  Returns dict with logits, ids, w,
+    near_tie, a1 (packed, sf), h32 [T, k, I], y [T, k, H], out_pre, out (BF16 as FP64).
+    """
+    x = np.asarray(x, np.float64)
+    t_count, hidden = x.shape
+    logits = router_logits(x, router_w)
+    ids, w, _ = route_topk(logits, top_k)
+    a1_packed, a1_sf = quantize_nvfp4(x.astype(np.float32), alpha_a1)
+    y = np.zeros((t_count, top_k, hidden), np.float64)
+    h32 = None
+    for e in np.unique(ids):
+        tt, jj = np.nonzero(ids == e)
+        r = expert_forward(a1_packed[tt], a1_sf[tt], alpha_a1, experts.dequantized(int(e)), alpha_a2)
+        if h32 is None:
+            h32 = np.zeros((t_count, top_k, r["h32"].shape[1]), np.float32)
+        h32[tt, jj] = r["h32"]
+        y[tt, jj] = r["y"]
+    out_pre, out, m = finalize(y, w, residual, gamma, eps)
+    return dict(logits=logits, ids=ids, w=w, near_tie=near_tie_mask(logits, top_k),
+                a1_packed=a1_packed, a1_sf=a1_sf, h32=h32, y=y, m=m, out_pre=out_pre, out=out)
+
+
+def moe_forward(x, residual, router_w, gamma, experts: ExpertCache, num_experts, top_k, alpha_a1, alpha_a2,
+                eps=1e-6):
+    """The whole layer for a batch: moe_forward_tokens plus the permutation of step 5."""
+    r = moe_forward_tokens(x, residual, router_w, gamma, experts, top_k, alpha_a1, alpha_a2, eps)
+    r.update(permute(r["ids"], num_experts))
+    return r
