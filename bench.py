@@ -1,0 +1,382 @@
+#!/usr/bin/env python
+"""Benchmark of the Beam-style sparse MoE layer forward (libbeam_moe) on B200 GPUs.
+
+One step = one whole layer forward (router, top-k, permutation, NVFP4 quantisation, the
+two grouped NVFP4 GEMMs, finalize) over one synthetic batch of the chosen workload.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode8] [--impl ours|reference]
+
+N > 1 runs under torchrun, one rank per GPU: token data parallel replicas (each rank a
+full copy of the layer and its own batch, no collective on the data path; the process
+group only carries the barrier and the max-over-ranks of the timing), so scaling is weak.
+Rank 0 prints one JSON line.  --impl reference times the CPU oracle (FP64) instead, on
+bounded samples of the same workload, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "moe_layer_tokens_per_s"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 512 << 20  # written between timed steps (L2 is 126 MB)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------------ algorithmic work
+def kernel_work(shape: mi.LayerShape, T: int, counts: np.ndarray) -> dict:
+    """Algorithmic bytes and FLOPs of each kernel for one forward (T tokens).
+
+    NVFP4 costs 0.5 B per value plus one scale byte per 16 values (0.5625 B/value).  Only
+    the experts that received tokens have their weights read."""
+    H, I, E, k = shape.hidden, shape.inter, shape.experts, shape.top_k
+    R = T * k
+    used = int((counts > 0).sum())
+    q = 0.5625
+    return {
+        "router": dict(bytes=E * H * 4 + T * H * 2 + T * E * 4, flops=2 * T * H * E),
+        "topk": dict(bytes=T * E * 4 + R * 8, flops=0),
+        "chunk_hist": dict(bytes=R * 4, flops=0),
+        "scan": dict(bytes=E * 16, flops=0),
+        "scatter": dict(bytes=R * 12, flops=0),
+        "quant_a1": dict(bytes=T * H * 2 + R * H * q, flops=0),
+        "gemm_gate_up": dict(bytes=used * 2 * I * H * q + R * H * q + R * I * q, flops=2 * R * 2 * I * H),
+        "gemm_down": dict(bytes=used * H * I * q + R * I * q + R * H * 2, flops=2 * R * H * I),
+        "finalize": dict(bytes=R * H * 2 + 2 * T * H * 2 + H * 2, flops=0),
+        "_used_experts": used,
+    }
+
+
+def read_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        tab = json.load(f)
+    ent = tab.get(f"{kernel}@{workload}")
+    if not ent:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "sparse_moe_layer_fp32_b200", "csrc", ent["source"])
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return ent["bytes_per_launch"] if digest == ent["source_sha256_16"] else None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [c.strip() for c in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        finally:
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def oracle_sample(shape: mi.LayerShape, tokens, seed=0):
+    """Inputs and quantised experts the oracle needs for a token sample (prepared untimed)."""
+    from oracle import moe
+    xs, rs = [], []
+    for t in tokens:
+        xb, rb = mi.tokens(shape, seed, t, t + 1)
+        xs.append(xb[0])
+        rs.append(rb[0])
+    x = mi.bf16_bits_to_f32(np.stack(xs)).astype(np.float64)
+    res = mi.bf16_bits_to_f32(np.stack(rs)).astype(np.float64)
+    wr = mi.router_weight(shape, seed)
+    g = mi.bf16_bits_to_f32(mi.gamma(shape, seed)).astype(np.float64)
+    ids, _, _ = moe.route_topk(moe.router_logits(x, wr), shape.top_k)
+    quantised = {int(e): moe.quantize_expert(*mi.expert_weights(shape, seed, int(e))) for e in np.unique(ids)}
+    return x, res, wr, g, quantised
+
+
+def oracle_step(shape, sample):
+    """One oracle forward of the sample: routing, experts (dequantised from the stored
+    NVFP4 weights, FP64 matmuls), finalize.  Returns tokens processed."""
+    from oracle import moe
+    x, res, wr, g, quantised = sample
+    a1, a2 = mi.activation_scales(shape)
+    cache = moe.ExpertCache(lambda e: None, keep=2)
+    cache._q = dict(quantised)
+    moe.moe_forward_tokens(x, res, wr, g, cache, shape.top_k, a1, a2, shape.rms_eps)
+    return x.shape[0]
+
+
+def cpu_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_sample_tokens(shape):
+    return [0] if shape.tokens <= 64 else [0, shape.tokens // 2]
+
+
+def cpu_baseline(shape, budget_s=25.0):
+    toks = cpu_sample_tokens(shape)
+    sample = oracle_sample(shape, toks)
+    t0 = time.perf_counter()
+    n = 0
+    reps = 0
+    while True:
+        n += oracle_step(shape, sample)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s or reps >= 3:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{len(toks)} token(s) of the {shape.name} batch x {reps} repeats: FP64 router, "
+                      f"NVFP4 experts dequantised from stored codes, finalize; weights pre-quantised untimed"}
+
+
+def run_reference(args, shape, rank, world):
+    if rank != 0:
+        return
+    sample = oracle_sample(shape, cpu_sample_tokens(shape))
+    for _ in range(args.warmup):
+        oracle_step(shape, sample)
+    t0 = time.perf_counter()
+    n = sum(oracle_step(shape, sample) for _ in range(args.steps))
+    dt = time.perf_counter() - t0
+    value = n / dt
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(shape),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{len(cpu_sample_tokens(shape))} token(s) of the {shape.name} batch per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(shape):
+    return {"workload": shape.name, "tokens": shape.tokens, "hidden": shape.hidden, "experts": shape.experts,
+            "top_k": shape.top_k, "inter": shape.inter, "routing": "zipf-skewed" if shape.skew else "uniform",
+            "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MiB write between timed steps"}
+
+
+# ------------------------------------------------------------------ GPU leg
+def run_ours(args, shape, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import sparse_moe_layer_fp32_b200 as bm
+    from sparse_moe_layer_fp32_b200 import synthetic
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    weights = synthetic.make_weights(shape, 0, device=dev)
+    layer = synthetic.make_layer(shape, weights)
+    x, res = synthetic.make_batch(shape, seed=rank)  # each replica its own batch
+    x, res = x.to(dev), res.to(dev)
+    out = torch.empty_like(res)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    T = shape.tokens
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 3)):
+        layer.forward(x, res, out)
+        flush.zero_()
+    layer.check()
+    torch.cuda.synchronize()
+    barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize()
+        barrier()
+        for i in range(args.steps):
+            starts[i].record(stream)
+            layer.forward(x, res, out)
+            ends[i].record(stream)
+            flush.zero_()
+        torch.cuda.synchronize()
+        barrier()
+    launches = layer.launches() * args.steps
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(step_ms) / args.steps
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    value = world * T / (ms / 1e3)
+    layer.check()
+
+    # ---- per-kernel durations (CUDA events inside the library, same stream), separate pass
+    layer.profile(True)
+    acc = {}
+    reps = max(args.steps, 5)
+    for _ in range(reps):
+        layer.forward(x, res, out)
+        for name, kms in layer.kernel_times():
+            acc.setdefault(name, []).append(kms)
+        flush.zero_()
+    layer.profile(False)
+    kern = {n: sum(v) / len(v) for n, v in acc.items()}
+    offsets = np.frombuffer(layer.debug(bm.BUF_OFFSETS).cpu().numpy().tobytes(), np.int32)
+    counts = np.diff(offsets)
+    work = kernel_work(shape, T, counts)
+    top = max(kern, key=kern.get)
+    pk = peaks()
+    wk = work[top]
+    if wk["flops"] > 0 and wk["flops"] / max(wk["bytes"], 1) > (4 * pk["bf16_sus"] * 1e12) / (pk["hbm"] * 1e9):
+        bound, achieved, peak, unit = ("tensor", wk["flops"] / (kern[top] / 1e3) / 1e12, 4 * pk["bf16_sus"],
+                                       "TFLOP/s")
+        peak_note = f"NVFP4 dense = 4 x {pk['src']} sustained BF16 cuBLAS peak (nominal 9 / 2.25 PF ratio)"
+    else:
+        bound, achieved, peak, unit = "hbm", wk["bytes"] / (kern[top] / 1e3) / 1e9, pk["hbm"], "GB/s"
+        peak_note = f"{pk['src']} copy bandwidth"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": read_traffic(top, shape.name), "kernel": top, "kernel_ms": kern[top],
+                "peak_source": peak_note}
+
+    # ---- end to end through the host-buffer entry point (copies inside the timed region)
+    xh = x.cpu().pin_memory()
+    rh = res.cpu().pin_memory()
+    oh = torch.empty_like(rh).pin_memory()
+    for _ in range(3):
+        layer.forward_host(xh, rh, oh)
+    torch.cuda.synchronize()
+    barrier()
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        e_s[i].record(stream)
+        layer.forward_host(xh, rh, oh)
+        e_e[i].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)) / args.steps
+    t = torch.tensor([e2e_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+    assert torch.equal(oh.to(dev), layer.forward(x, res)), "host-buffer path differs from device path"
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) experts, fp32 router and accumulation",
+            "data": "synthetic (seeded; random-init weights of the layer's shapes)",
+            "config": dict(workload_config(shape), parallelism=f"token-dp replicas x{world}"),
+            "roofline": roofline,
+            "kernels_ms": kern,
+            "used_experts": work["_used_experts"],
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": 2 * T * shape.hidden * 2,
+                    "d2h_bytes_per_step": T * shape.hidden * 2},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+    layer.close()
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode8", choices=sorted(mi.SHAPES))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    shape = mi.SHAPES[args.workload]
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, shape, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, shape, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(shape)
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

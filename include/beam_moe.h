@@ -1,0 +1,184 @@
+/*
+ * beam_moe.h — C ABI of libbeam_moe.so: the forward pass of one Beam-style sparse
+ * mixture-of-experts layer on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources are web pages, cited by title and section):
+ *   - router GEMM from hidden 5120 to 256 expert logits, computed in FP32
+ *     (vLLM PR "Day-0 support for Reflection's Beam-1.0", section "Status": router GEMM
+ *     kernels for (5120, 256); news article "vLLM adds day-zero Reflection Beam serving",
+ *     section "Agents worked on the serving path": a specialised FP32 router kernel);
+ *   - softmax over all experts, the top 8 of 256 (vLLM recipe
+ *     "reflection/Beam-1.0-501B-A23B", section "Overview"), weights renormalised over
+ *     the chosen 8;
+ *   - routed experts in NVFP4, W4A4 on Blackwell (recipe, section "Variants"), SwiGLU;
+ *   - MoE finalize: weighted un-permute, post-RMSNorm of the sandwich norm (eps 1e-6)
+ *     and residual add (PR, sections "Status" and "Remaining work").
+ *
+ * Conventions for every entry point:
+ *   - Pointers are device pointers unless the name says _host.  `stream` is a
+ *     cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - Work is enqueued asynchronously on `stream`; nothing synchronises the host except
+ *     beam_moe_create, beam_moe_check and beam_moe_destroy, which say so.
+ *   - Errors are returned as a beam_moe_status and never thrown.  Argument errors are
+ *     found on the host before anything is enqueued.  Faults found on the device (a wait
+ *     that ran out of time, an index out of range) set a device error word that
+ *     beam_moe_check reports.
+ *   - BF16 tensors are passed as raw 16-bit patterns (uint16_t / void*).
+ *   - Activation and weight tensors must start on a 16-byte boundary (the kernels use
+ *     16-byte vector accesses); a misaligned pointer is rejected with INVALID_ARG.
+ *   - NVFP4 data: two 4-bit E2M1 codes per byte, element 2i in the low nibble; one
+ *     unsigned E4M3 scale byte per 16 consecutive elements of a row; one FP32 tensor
+ *     scale alpha per tensor; value = e2m1 * e4m3 * alpha.
+ */
+#ifndef BEAM_MOE_H_
+#define BEAM_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BEAM_MOE_API __attribute__((visibility("default")))
+#else
+#define BEAM_MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BEAM_MOE_OK = 0,
+  BEAM_MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, tokens > max_tokens ...  */
+  BEAM_MOE_ERR_UNSUPPORTED = 2, /* a shape this build does not handle (see create)      */
+  BEAM_MOE_ERR_CUDA = 3,        /* a CUDA runtime call failed                           */
+  BEAM_MOE_ERR_OOM = 4,         /* device allocation failed                              */
+  BEAM_MOE_ERR_TIMEOUT = 5,     /* a bounded device wait gave up (reported by check)    */
+  BEAM_MOE_ERR_DEVICE = 6       /* a device-side range check failed (reported by check) */
+} beam_moe_status;
+
+/* Layer shape and the static activation scales.  Supported: hidden % 256 == 0,
+ * inter % 128 == 0, 1 <= top_k <= 16, top_k <= num_experts <= 1024,
+ * num_experts % 32 == 0 or num_experts < 32, max_tokens >= 1. */
+typedef struct {
+  int32_t max_tokens;  /* largest num_tokens a forward may be called with              */
+  int32_t hidden;      /* H (5120)                                                    */
+  int32_t num_experts; /* E (256)                                                     */
+  int32_t top_k;       /* k (8)                                                       */
+  int32_t inter;       /* I, expert intermediate size                                 */
+  float rms_eps;       /* post-RMSNorm epsilon (1e-6)                                 */
+  float alpha_a1;      /* FP32 tensor scale of the NVFP4 expert inputs (> 0)          */
+  float alpha_a2;      /* FP32 tensor scale of the NVFP4 SwiGLU outputs (> 0)         */
+} beam_moe_config;
+
+/* Layer weights (device pointers, read only during beam_moe_create; the caller keeps
+ * ownership and may free them after create returns). */
+typedef struct {
+  const float* router_w;     /* [E][H] FP32, row e = expert e                           */
+  const uint8_t* w_gu;       /* [E][2I][H/2] NVFP4 codes; rows 0..I-1 gate, I..2I-1 up  */
+  const uint8_t* w_gu_sf;    /* [E][2I][H/16] E4M3 scales, row-major                     */
+  const float* w_gu_alpha;   /* [E] tensor scale of each expert's gate+up                */
+  const uint8_t* w_d;        /* [E][H][I/2] NVFP4 codes of the down projection          */
+  const uint8_t* w_d_sf;     /* [E][H][I/16] E4M3 scales                                 */
+  const float* w_d_alpha;    /* [E] tensor scale of each expert's down                   */
+  const uint16_t* gamma;     /* [H] BF16 RMSNorm weight                                  */
+} beam_moe_weights;
+
+typedef struct beam_moe_ctx* beam_moe_t;
+
+/* Validates cfg, allocates the handle's device memory (repacked weights and a workspace
+ * sized for cfg->max_tokens), repacks the weights into the tensor-core layout on `stream`
+ * and synchronises `stream` before returning.  On success *out owns all of it until
+ * beam_moe_destroy.  Returns INVALID_ARG / UNSUPPORTED / OOM / CUDA. */
+BEAM_MOE_API beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weights* weights, void* stream,
+                                beam_moe_t* out);
+
+/* out[T][H] = residual + RMSNorm(sum_j w_j * expert_{id_j}(x)) * gamma, rounded to BF16.
+ * x, residual, out: [num_tokens][H] BF16 row-major, caller-owned, device memory.
+ * out may equal residual (in-place residual update); no other aliasing.  0 <= num_tokens
+ * <= max_tokens (0 enqueues nothing).  Uses the handle's workspace, so calls on one
+ * handle must be ordered (same stream, or synchronised). */
+BEAM_MOE_API beam_moe_status beam_moe_forward(beam_moe_t h, const void* x, const void* residual, void* out, int32_t num_tokens,
+                                 void* stream);
+
+/* Same as beam_moe_forward with HOST buffers: copies x and residual to the handle's
+ * device staging buffers, runs the forward, copies out back, all enqueued on `stream`
+ * (cudaMemcpyAsync; pinned host memory makes the copies asynchronous).  The caller
+ * synchronises `stream` before reading out_host. */
+BEAM_MOE_API beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const void* residual_host, void* out_host,
+                                      int32_t num_tokens, void* stream);
+
+/* Bytes of logits_ws that beam_moe_route needs for this shape (the logits may be held as
+ * partial sums over slices of H).  0 for empty shapes. */
+BEAM_MOE_API int64_t beam_moe_route_workspace_bytes(int32_t num_tokens, int32_t hidden, int32_t num_experts);
+
+/* Routing alone, on caller buffers: logits[T][E] = x W_r^T (FP32 arithmetic), then the
+ * top-k of the softmax (ties: lower expert index) in descending weight and the weights
+ * renormalised over the chosen k.  x [T][H] BF16, router_w [E][H] FP32; logits_ws is
+ * caller scratch of beam_moe_route_workspace_bytes(T, H, E) bytes; ids [T][k] int32 and
+ * w [T][k] FP32 are outputs.  Same shape limits as beam_moe_config. */
+BEAM_MOE_API beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num_tokens, int32_t hidden,
+                               int32_t num_experts, int32_t top_k, float* logits_ws, int32_t* ids, float* w,
+                               void* stream);
+
+/* NVFP4 quantiser Q (weights or activations): src [rows][cols] FP32 row-major, cols %
+ * 16 == 0.  codes [rows][cols/2], sf [rows][cols/16] (row-major scale bytes).  alpha >
+ * 0 uses that tensor scale; alpha <= 0 computes alpha = amax(src) / 2688 on the device
+ * first.  If alpha_out is not NULL the scale used is written there (device FP32). */
+BEAM_MOE_API beam_moe_status beam_moe_quantize_nvfp4(const float* src, int64_t rows, int64_t cols, float alpha, uint8_t* codes,
+                                        uint8_t* sf, float* alpha_out, void* stream);
+
+/* Internal buffers of the last forward, for tests (layouts in the comment of each id). */
+typedef enum {
+  BEAM_MOE_BUF_LOGITS = 0,   /* [T][E] FP32                                                */
+  BEAM_MOE_BUF_IDS = 1,      /* [T][k] int32                                               */
+  BEAM_MOE_BUF_WEIGHTS = 2,  /* [T][k] FP32                                                */
+  BEAM_MOE_BUF_OFFSETS = 3,  /* [E+1] int32: rows of expert e are [off[e], off[e+1])       */
+  BEAM_MOE_BUF_PERM = 4,     /* [T*k] int32: token of permuted row r                        */
+  BEAM_MOE_BUF_INV = 5,      /* [T][k] int32: permuted row of (token, slot)                */
+  BEAM_MOE_BUF_SFBLOCK = 6,  /* [E+1] int32: first 128-row scale block of each expert      */
+  BEAM_MOE_BUF_A1 = 7,       /* [T*k][H/2] NVFP4 codes of the permuted expert inputs       */
+  BEAM_MOE_BUF_A1_SF = 8,    /* scale blocks: [nblk][H/64][512], see below                 */
+  BEAM_MOE_BUF_A2 = 9,       /* [T*k][Ip/2] codes of the SwiGLU outputs, Ip = ceil(I/256)*256 */
+  BEAM_MOE_BUF_A2_SF = 10,   /* [nblk][Ip/64][512]                                          */
+  BEAM_MOE_BUF_Y = 11        /* [T*k][H] BF16 expert outputs in permuted row order          */
+} beam_moe_buffer;
+/* Scale blocks: the rows of expert e, local row i = r - off[e], live in block
+ * sfblock[e] + i/128, row m = i%128; for scale s of that row the byte is at
+ * ((block * (K/64) + s/4) * 512) + (m%32)*16 + (m/32)*4 + s%4. */
+
+/* Copies min(bytes, size of the buffer) bytes of internal buffer `which` to dst (device),
+ * enqueued on `stream`.  *size_out (host, may be NULL) receives the buffer's size for the
+ * last forward's num_tokens. */
+BEAM_MOE_API beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, void* dst, size_t bytes, size_t* size_out,
+                                    void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word.  Returns OK,
+ * TIMEOUT or DEVICE. */
+BEAM_MOE_API beam_moe_status beam_moe_check(beam_moe_t h, void* stream);
+
+/* Per-kernel timing.  While enabled (enable != 0), beam_moe_forward records a CUDA event
+ * on `stream` before its first kernel and after each kernel it enqueues.  Creating the
+ * events is the only allocation; enable once, outside any timed region. */
+BEAM_MOE_API beam_moe_status beam_moe_profile_enable(beam_moe_t h, int32_t enable);
+
+/* Waits for the events of the last profiled forward and writes the duration in ms of each
+ * of its kernels, in launch order, to ms[0 .. min(capacity, count)); *count (host) gets
+ * the number of kernels.  Names of the kernels: beam_moe_kernel_name. */
+BEAM_MOE_API beam_moe_status beam_moe_profile_read(beam_moe_t h, float* ms, int32_t capacity, int32_t* count);
+
+/* Name of the index-th kernel of the last forward ("router", "topk", ...), or NULL. */
+BEAM_MOE_API const char* beam_moe_kernel_name(beam_moe_t h, int32_t index);
+
+/* Number of kernels the last beam_moe_forward enqueued. */
+BEAM_MOE_API int32_t beam_moe_last_launch_count(beam_moe_t h);
+
+BEAM_MOE_API const char* beam_moe_status_string(beam_moe_status s);
+
+/* Synchronises the device, then frees everything the handle owns.  NULL is a no-op. */
+BEAM_MOE_API void beam_moe_destroy(beam_moe_t h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BEAM_MOE_H_ */

@@ -1,0 +1,228 @@
+"""Python binding of libbeam_moe.so: the Beam-style sparse MoE layer forward on a B200.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+PyTorch provides device memory and streams.  The functions keep the C names
+(beam_moe_create, beam_moe_forward, ...); ``MoELayer`` wraps a handle.  Importing this
+package never falls back to anything: if the library is missing it raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbeam_moe.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_OOM, ERR_TIMEOUT, ERR_DEVICE = range(7)
+(BUF_LOGITS, BUF_IDS, BUF_WEIGHTS, BUF_OFFSETS, BUF_PERM, BUF_INV, BUF_SFBLOCK, BUF_A1, BUF_A1_SF, BUF_A2,
+ BUF_A2_SF, BUF_Y) = range(12)
+
+EXPORTED = [
+    "beam_moe_create", "beam_moe_forward", "beam_moe_forward_host", "beam_moe_route",
+    "beam_moe_route_workspace_bytes", "beam_moe_quantize_nvfp4", "beam_moe_debug_copy", "beam_moe_check",
+    "beam_moe_last_launch_count", "beam_moe_status_string", "beam_moe_destroy", "beam_moe_profile_enable",
+    "beam_moe_profile_read", "beam_moe_kernel_name",
+]
+
+
+class BeamMoeConfig(ctypes.Structure):
+    _fields_ = [("max_tokens", ctypes.c_int32), ("hidden", ctypes.c_int32), ("num_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("inter", ctypes.c_int32), ("rms_eps", ctypes.c_float),
+                ("alpha_a1", ctypes.c_float), ("alpha_a2", ctypes.c_float)]
+
+
+class BeamMoeWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("router_w", "w_gu", "w_gu_sf", "w_gu_alpha", "w_d", "w_d_sf", "w_d_alpha", "gamma")]
+
+
+class BeamMoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run sparse_moe_layer_fp32_b200.build.build() "
+                          "(needs nvcc with sm_100a support)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "beam_moe_create": (i32, [ctypes.POINTER(BeamMoeConfig), ctypes.POINTER(BeamMoeWeights), vp,
+                                  ctypes.POINTER(vp)]),
+        "beam_moe_forward": (i32, [vp, vp, vp, vp, i32, vp]),
+        "beam_moe_forward_host": (i32, [vp, vp, vp, vp, i32, vp]),
+        "beam_moe_route": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp]),
+        "beam_moe_route_workspace_bytes": (i64, [i32, i32, i32]),
+        "beam_moe_quantize_nvfp4": (i32, [vp, i64, i64, f32, vp, vp, vp, vp]),
+        "beam_moe_debug_copy": (i32, [vp, i32, vp, sz, ctypes.POINTER(sz), vp]),
+        "beam_moe_check": (i32, [vp, vp]),
+        "beam_moe_last_launch_count": (i32, [vp]),
+        "beam_moe_status_string": (ctypes.c_char_p, [i32]),
+        "beam_moe_destroy": (None, [vp]),
+        "beam_moe_profile_enable": (i32, [vp, i32]),
+        "beam_moe_profile_read": (i32, [vp, ctypes.POINTER(f32), i32, ctypes.POINTER(i32)]),
+        "beam_moe_kernel_name": (ctypes.c_char_p, [vp, i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.beam_moe_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise BeamMoeError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ------------------------------------------------------------------ C names
+def beam_moe_create(cfg: BeamMoeConfig, weights: BeamMoeWeights, stream=None) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_lib.beam_moe_create(ctypes.byref(cfg), ctypes.byref(weights), _stream(stream), ctypes.byref(h)),
+           "beam_moe_create")
+    return h
+
+
+def beam_moe_forward(h, x, residual, out, num_tokens: int, stream=None):
+    _check(_lib.beam_moe_forward(h, _ptr(x), _ptr(residual), _ptr(out), int(num_tokens), _stream(stream)),
+           "beam_moe_forward")
+
+
+def beam_moe_forward_host(h, x_host, residual_host, out_host, num_tokens: int, stream=None):
+    _check(_lib.beam_moe_forward_host(h, _ptr(x_host), _ptr(residual_host), _ptr(out_host), int(num_tokens),
+                                      _stream(stream)), "beam_moe_forward_host")
+
+
+def beam_moe_route_workspace_bytes(num_tokens: int, hidden: int, num_experts: int) -> int:
+    return int(_lib.beam_moe_route_workspace_bytes(num_tokens, hidden, num_experts))
+
+
+def beam_moe_route(x, router_w, top_k: int, stream=None):
+    """Returns (ids [T, k] int32, w [T, k] float32) for x [T, H] bf16, router_w [E, H] fp32."""
+    t_count, hidden = x.shape
+    experts = router_w.shape[0]
+    ws = torch.empty(max(beam_moe_route_workspace_bytes(t_count, hidden, experts) // 4, 1), dtype=torch.float32,
+                     device=x.device)
+    ids = torch.empty((t_count, top_k), dtype=torch.int32, device=x.device)
+    w = torch.empty((t_count, top_k), dtype=torch.float32, device=x.device)
+    _check(_lib.beam_moe_route(_ptr(x), _ptr(router_w), t_count, hidden, experts, top_k, _ptr(ws), _ptr(ids),
+                               _ptr(w), _stream(stream)), "beam_moe_route")
+    return ids, w
+
+
+def beam_moe_quantize_nvfp4(src, alpha: float | None = None, stream=None):
+    """NVFP4 of a 2-D FP32 CUDA tensor: (codes uint8 [r, c/2], scales uint8 [r, c/16], alpha fp32 [1])."""
+    rows, cols = src.shape
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=src.device)
+    sf = torch.empty((rows, cols // 16), dtype=torch.uint8, device=src.device)
+    alpha_out = torch.empty(1, dtype=torch.float32, device=src.device)
+    a = -1.0 if alpha is None else float(alpha)
+    _check(_lib.beam_moe_quantize_nvfp4(_ptr(src.contiguous()), rows, cols, ctypes.c_float(a), _ptr(codes),
+                                        _ptr(sf), _ptr(alpha_out), _stream(stream)), "beam_moe_quantize_nvfp4")
+    return codes, sf, alpha_out
+
+
+def beam_moe_debug_copy(h, which: int, stream=None) -> torch.Tensor:
+    size = ctypes.c_size_t(0)
+    _check(_lib.beam_moe_debug_copy(h, which, None, 0, ctypes.byref(size), _stream(stream)), "beam_moe_debug_copy")
+    out = torch.empty(max(size.value, 1), dtype=torch.uint8, device="cuda")
+    _check(_lib.beam_moe_debug_copy(h, which, _ptr(out), size.value, None, _stream(stream)), "beam_moe_debug_copy")
+    return out[: size.value]
+
+
+def beam_moe_check(h, stream=None):
+    _check(_lib.beam_moe_check(h, _stream(stream)), "beam_moe_check")
+
+
+def beam_moe_last_launch_count(h) -> int:
+    return int(_lib.beam_moe_last_launch_count(h))
+
+
+def beam_moe_destroy(h):
+    _lib.beam_moe_destroy(h)
+
+
+def beam_moe_profile_enable(h, enable: bool = True):
+    _check(_lib.beam_moe_profile_enable(h, 1 if enable else 0), "beam_moe_profile_enable")
+
+
+def beam_moe_profile_read(h):
+    """[(kernel name, ms)] of the last profiled forward, in launch order."""
+    buf = (ctypes.c_float * 32)()
+    n = ctypes.c_int32(0)
+    _check(_lib.beam_moe_profile_read(h, buf, 32, ctypes.byref(n)), "beam_moe_profile_read")
+    return [(_lib.beam_moe_kernel_name(h, i).decode(), float(buf[i])) for i in range(n.value)]
+
+
+# ------------------------------------------------------------------ handle wrapper
+class MoELayer:
+    """Owns a beam_moe handle.  Weight tensors are CUDA tensors in the C-ABI layout."""
+
+    def __init__(self, *, max_tokens, hidden, num_experts, top_k, inter, alpha_a1, alpha_a2, router_w, w_gu,
+                 w_gu_sf, w_gu_alpha, w_d, w_d_sf, w_d_alpha, gamma, rms_eps=1e-6, stream=None):
+        self.cfg = BeamMoeConfig(max_tokens, hidden, num_experts, top_k, inter, rms_eps, float(alpha_a1),
+                                 float(alpha_a2))
+        ws = [router_w, w_gu, w_gu_sf, w_gu_alpha, w_d, w_d_sf, w_d_alpha, gamma]
+        wts = BeamMoeWeights(*[t.data_ptr() for t in ws])
+        self.hidden, self.top_k = hidden, top_k
+        self.handle = beam_moe_create(self.cfg, wts, stream)
+
+    def forward(self, x, residual, out=None, stream=None):
+        out = torch.empty_like(residual) if out is None else out
+        beam_moe_forward(self.handle, x, residual, out, x.shape[0], stream)
+        return out
+
+    def forward_host(self, x_host, residual_host, out_host, stream=None):
+        beam_moe_forward_host(self.handle, x_host, residual_host, out_host, x_host.shape[0], stream)
+        return out_host
+
+    def debug(self, which: int, stream=None) -> torch.Tensor:
+        return beam_moe_debug_copy(self.handle, which, stream)
+
+    def check(self, stream=None):
+        beam_moe_check(self.handle, stream)
+
+    def launches(self) -> int:
+        return beam_moe_last_launch_count(self.handle)
+
+    def profile(self, enable: bool = True):
+        beam_moe_profile_enable(self.handle, enable)
+
+    def kernel_times(self):
+        return beam_moe_profile_read(self.handle)
+
+    def close(self):
+        if self.handle:
+            beam_moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,477 @@
+// C ABI of libbeam_moe: handle, device memory, TMA descriptors and the forward sequence.
+// The operation and its sources are described in include/beam_moe.h.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/beam_moe.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace beam;
+
+struct beam_moe_ctx {
+  beam_moe_config cfg;
+  int H, E, k, I, Ip, Tmax;
+  int64_t Rmax, nblk_max, n_chunks_max;
+  int num_sms;
+  // weights (owned, repacked)
+  float* router_w;
+  uint8_t *w_gu, *w_gu_sf, *w_d, *w_d_sf;
+  float *w_gu_alpha, *w_d_alpha;
+  uint16_t* gamma;
+  // workspace
+  float* logits;
+  int64_t logits_floats;
+  int32_t *ids, *chunk_counts, *chunk_base, *offsets, *sf_block, *num_mblocks, *perm, *inv;
+  float* w;
+  MBlock* mblocks;
+  uint8_t *a1, *a1_sf, *a2, *a2_sf;
+  uint16_t* y;
+  uint32_t* err;
+  uint16_t *stage_x, *stage_res, *stage_out;
+  CUtensorMap map_a1, map_wgu, map_a2, map_wd;
+  int last_T;
+  int last_launches;
+  std::vector<void*> allocs;
+  // optional per-kernel timing
+  static constexpr int kMaxEvents = 17;
+  bool profiling;
+  bool profiled_last;
+  cudaEvent_t events[kMaxEvents];
+  const char* names[kMaxEvents];
+};
+
+namespace {
+
+beam_moe_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return BEAM_MOE_OK;
+  if (e == cudaErrorMemoryAllocation) return BEAM_MOE_ERR_OOM;
+  return BEAM_MOE_ERR_CUDA;
+}
+
+#define BEAM_TRY(call)                              \
+  do {                                              \
+    cudaError_t e_ = (call);                        \
+    if (e_ != cudaSuccess) return cuda_status(e_);  \
+  } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes]; boxes of 128 bytes x box_rows, 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+cudaError_t dalloc(beam_moe_ctx* h, T** p, size_t bytes) {
+  void* q = nullptr;
+  cudaError_t e = cudaMalloc(&q, std::max<size_t>(bytes, 16));
+  if (e != cudaSuccess) return e;
+  h->allocs.push_back(q);
+  *p = static_cast<T*>(q);
+  return cudaSuccess;
+}
+
+void free_all(beam_moe_ctx* h) {
+  for (void* p : h->allocs) cudaFree(p);
+  h->allocs.clear();
+}
+
+beam_moe_status check_shape(int H, int E, int k) {
+  if (H <= 0 || E <= 0 || k <= 0) return BEAM_MOE_ERR_INVALID_ARG;
+  if (H % 256 != 0 || k > 16 || k > E || E > 1024 || (E >= 32 && E % 32 != 0)) return BEAM_MOE_ERR_UNSUPPORTED;
+  return BEAM_MOE_OK;
+}
+
+int64_t route_ws_floats(int T, int H, int E) {
+  return static_cast<int64_t>(router_split_count(T, H, E)) * T * E;
+}
+
+__global__ void store_f32_kernel(float* p, float v) { *p = v; }
+
+// Kernels use 16-byte vector accesses on these pointers.
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* beam_moe_status_string(beam_moe_status s) {
+  switch (s) {
+    case BEAM_MOE_OK: return "ok";
+    case BEAM_MOE_ERR_INVALID_ARG: return "invalid argument";
+    case BEAM_MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case BEAM_MOE_ERR_CUDA: return "CUDA runtime error";
+    case BEAM_MOE_ERR_OOM: return "out of device memory";
+    case BEAM_MOE_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case BEAM_MOE_ERR_DEVICE: return "device-side range check failed";
+  }
+  return "unknown status";
+}
+
+int64_t beam_moe_route_workspace_bytes(int32_t num_tokens, int32_t hidden, int32_t num_experts) {
+  if (num_tokens <= 0 || hidden <= 0 || num_experts <= 0) return 0;
+  return route_ws_floats(num_tokens, hidden, num_experts) * static_cast<int64_t>(sizeof(float));
+}
+
+beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weights* wts, void* stream,
+                                beam_moe_t* out) {
+  if (!cfg || !wts || !out) return BEAM_MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!wts->router_w || !wts->w_gu || !wts->w_gu_sf || !wts->w_gu_alpha || !wts->w_d || !wts->w_d_sf ||
+      !wts->w_d_alpha || !wts->gamma)
+    return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned(wts->w_gu, 16) || !aligned(wts->w_d, 16) || !aligned(wts->gamma, 16))
+    return BEAM_MOE_ERR_INVALID_ARG;
+  if (cfg->max_tokens <= 0 || !(cfg->alpha_a1 > 0.0f) || !(cfg->alpha_a2 > 0.0f) || !(cfg->rms_eps >= 0.0f))
+    return BEAM_MOE_ERR_INVALID_ARG;
+  beam_moe_status st = check_shape(cfg->hidden, cfg->num_experts, cfg->top_k);
+  if (st != BEAM_MOE_OK) return st;
+  if (cfg->inter <= 0) return BEAM_MOE_ERR_INVALID_ARG;
+  if (cfg->inter % 128 != 0) return BEAM_MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(cfg->max_tokens) * cfg->top_k > (1ll << 30)) return BEAM_MOE_ERR_UNSUPPORTED;
+  if (!tensor_map_encoder()) return BEAM_MOE_ERR_CUDA;
+
+  beam_moe_ctx* h = new (std::nothrow) beam_moe_ctx();
+  if (!h) return BEAM_MOE_ERR_OOM;
+  h->cfg = *cfg;
+  h->H = cfg->hidden;
+  h->E = cfg->num_experts;
+  h->k = cfg->top_k;
+  h->I = cfg->inter;
+  h->Ip = (cfg->inter + 255) / 256 * 256;
+  h->Tmax = cfg->max_tokens;
+  h->Rmax = static_cast<int64_t>(h->Tmax) * h->k;
+  h->nblk_max = (h->Rmax + 127) / 128 + h->E;
+  h->n_chunks_max = (h->Tmax + kChunkTokens - 1) / kChunkTokens;
+  h->last_T = 0;
+  h->last_launches = 0;
+  h->profiling = false;
+  h->profiled_last = false;
+  for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i) {
+    h->events[i] = nullptr;
+    h->names[i] = nullptr;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int H = h->H, E = h->E, I = h->I, Ip = h->Ip;
+
+  auto fail = [&](cudaError_t e) {
+    cudaStreamSynchronize(s);
+    free_all(h);
+    delete h;
+    return cuda_status(e);
+  };
+#define CREATE_TRY(call)                    \
+  do {                                      \
+    cudaError_t e_ = (call);                \
+    if (e_ != cudaSuccess) return fail(e_); \
+  } while (0)
+
+  int dev = 0;
+  CREATE_TRY(cudaGetDevice(&dev));
+  CREATE_TRY(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
+
+  // ---- weights
+  CREATE_TRY(dalloc(h, &h->router_w, sizeof(float) * E * H));
+  CREATE_TRY(dalloc(h, &h->w_gu, static_cast<size_t>(E) * 2 * I * (H / 2)));
+  CREATE_TRY(dalloc(h, &h->w_gu_sf, static_cast<size_t>(E) * 2 * I * (H / 16)));
+  CREATE_TRY(dalloc(h, &h->w_d, static_cast<size_t>(E) * H * (Ip / 2)));
+  CREATE_TRY(dalloc(h, &h->w_d_sf, static_cast<size_t>(E) * H * (Ip / 16)));
+  CREATE_TRY(dalloc(h, &h->w_gu_alpha, sizeof(float) * E));
+  CREATE_TRY(dalloc(h, &h->w_d_alpha, sizeof(float) * E));
+  CREATE_TRY(dalloc(h, &h->gamma, sizeof(uint16_t) * H));
+  CREATE_TRY(cudaMemcpyAsync(h->router_w, wts->router_w, sizeof(float) * E * H, cudaMemcpyDeviceToDevice, s));
+  CREATE_TRY(cudaMemcpyAsync(h->w_gu_alpha, wts->w_gu_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
+  CREATE_TRY(cudaMemcpyAsync(h->w_d_alpha, wts->w_d_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
+  CREATE_TRY(cudaMemcpyAsync(h->gamma, wts->gamma, sizeof(uint16_t) * H, cudaMemcpyDeviceToDevice, s));
+  CREATE_TRY(launch_repack_gate_up(wts->w_gu, wts->w_gu_sf, E, I, H, h->w_gu, h->w_gu_sf, s));
+  CREATE_TRY(launch_repack_down(wts->w_d, wts->w_d_sf, E, I, Ip, H, h->w_d, h->w_d_sf, s));
+
+  // ---- workspace
+  int64_t lf = 0;
+  for (int T = 1; T <= h->Tmax; T = (T < 64 ? T + 1 : T + 64)) lf = std::max(lf, route_ws_floats(T, H, E));
+  lf = std::max(lf, route_ws_floats(h->Tmax, H, E));
+  h->logits_floats = lf;
+  const int64_t R = h->Rmax;
+  CREATE_TRY(dalloc(h, &h->logits, sizeof(float) * lf));
+  CREATE_TRY(dalloc(h, &h->ids, sizeof(int32_t) * R));
+  CREATE_TRY(dalloc(h, &h->w, sizeof(float) * R));
+  CREATE_TRY(dalloc(h, &h->chunk_counts, sizeof(int32_t) * h->n_chunks_max * E));
+  CREATE_TRY(dalloc(h, &h->chunk_base, sizeof(int32_t) * h->n_chunks_max * E));
+  CREATE_TRY(dalloc(h, &h->offsets, sizeof(int32_t) * (E + 1)));
+  CREATE_TRY(dalloc(h, &h->sf_block, sizeof(int32_t) * (E + 1)));
+  CREATE_TRY(dalloc(h, &h->num_mblocks, sizeof(int32_t)));
+  CREATE_TRY(dalloc(h, &h->mblocks, sizeof(MBlock) * h->nblk_max));
+  CREATE_TRY(dalloc(h, &h->perm, sizeof(int32_t) * R));
+  CREATE_TRY(dalloc(h, &h->inv, sizeof(int32_t) * R));
+  CREATE_TRY(dalloc(h, &h->a1, static_cast<size_t>(R) * (H / 2)));
+  CREATE_TRY(dalloc(h, &h->a1_sf, static_cast<size_t>(h->nblk_max) * (H / 64) * 512));
+  CREATE_TRY(dalloc(h, &h->a2, static_cast<size_t>(R) * (Ip / 2)));
+  CREATE_TRY(dalloc(h, &h->a2_sf, static_cast<size_t>(h->nblk_max) * (Ip / 64) * 512));
+  CREATE_TRY(dalloc(h, &h->y, sizeof(uint16_t) * static_cast<size_t>(R) * H));
+  CREATE_TRY(dalloc(h, &h->err, sizeof(uint32_t)));
+  CREATE_TRY(dalloc(h, &h->stage_x, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
+  CREATE_TRY(dalloc(h, &h->stage_res, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
+  CREATE_TRY(dalloc(h, &h->stage_out, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
+  // The SwiGLU outputs beyond I (when I is not a multiple of 256) are never written: their
+  // codes and scales must read as zero in the down GEMM.  Scale blocks of unused rows are
+  // also defined this way.
+  CREATE_TRY(cudaMemsetAsync(h->a2, 0, static_cast<size_t>(R) * (Ip / 2), s));
+  CREATE_TRY(cudaMemsetAsync(h->a2_sf, 0, static_cast<size_t>(h->nblk_max) * (Ip / 64) * 512, s));
+  CREATE_TRY(cudaMemsetAsync(h->a1_sf, 0, static_cast<size_t>(h->nblk_max) * (H / 64) * 512, s));
+  CREATE_TRY(cudaMemsetAsync(h->err, 0, sizeof(uint32_t), s));
+
+  if (!make_map_u8(&h->map_a1, h->a1, H / 2, R, 128) || !make_map_u8(&h->map_wgu, h->w_gu, H / 2,
+                                                                       static_cast<uint64_t>(E) * 2 * I, 256) ||
+      !make_map_u8(&h->map_a2, h->a2, Ip / 2, R, 128) ||
+      !make_map_u8(&h->map_wd, h->w_d, Ip / 2, static_cast<uint64_t>(E) * H, 256))
+    return fail(cudaErrorInvalidValue);
+  CREATE_TRY(cudaStreamSynchronize(s));
+  CREATE_TRY(cudaGetLastError());
+#undef CREATE_TRY
+  *out = h;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num_tokens, int32_t hidden,
+                               int32_t num_experts, int32_t top_k, float* logits_ws, int32_t* ids, float* w,
+                               void* stream) {
+  beam_moe_status st = check_shape(hidden, num_experts, top_k);
+  if (st != BEAM_MOE_OK) return st;
+  if (num_tokens < 0) return BEAM_MOE_ERR_INVALID_ARG;
+  if (num_tokens == 0) return BEAM_MOE_OK;
+  if (!x || !router_w || !logits_ws || !ids || !w) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(router_w, 16) || !aligned(logits_ws, 4) || !aligned(ids, 4) || !aligned(w, 4))
+    return BEAM_MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  BEAM_TRY(launch_router_logits(static_cast<const uint16_t*>(x), router_w, num_tokens, hidden, num_experts,
+                                logits_ws, s));
+  BEAM_TRY(launch_topk(logits_ws, router_split_count(num_tokens, hidden, num_experts), num_tokens, num_experts,
+                       top_k, ids, w, s));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_forward(beam_moe_t h, const void* x, const void* residual, void* out, int32_t num_tokens,
+                                 void* stream) {
+  if (!h) return BEAM_MOE_ERR_INVALID_ARG;
+  if (num_tokens < 0 || num_tokens > h->Tmax) return BEAM_MOE_ERR_INVALID_ARG;
+  if (num_tokens == 0) {
+    h->last_T = 0;
+    h->last_launches = 0;
+    return BEAM_MOE_OK;
+  }
+  if (!x || !residual || !out) return BEAM_MOE_ERR_INVALID_ARG;
+  if (x == out) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(residual, 16) || !aligned(out, 16)) return BEAM_MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int T = num_tokens, H = h->H, E = h->E, k = h->k;
+  const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  int launches = 0;
+  const bool prof = h->profiling;
+  auto mark = [&](const char* name) -> cudaError_t {
+    if (!prof) return cudaSuccess;
+    h->names[launches] = name;
+    return cudaEventRecord(h->events[launches + 1], s);
+  };
+  if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
+  BEAM_TRY(launch_router_logits(xb, h->router_w, T, H, E, h->logits, s));
+  BEAM_TRY(mark("router"));
+  ++launches;
+  BEAM_TRY(launch_topk(h->logits, router_split_count(T, H, E), T, E, k, h->ids, h->w, s));
+  BEAM_TRY(mark("topk"));
+  ++launches;
+  BEAM_TRY(launch_chunk_hist(h->ids, T, k, E, h->chunk_counts, s));
+  BEAM_TRY(mark("chunk_hist"));
+  ++launches;
+  BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
+                       h->num_mblocks, s));
+  BEAM_TRY(mark("scan"));
+  ++launches;
+  BEAM_TRY(launch_scatter(h->ids, h->chunk_base, T, k, E, h->perm, h->inv, s));
+  BEAM_TRY(mark("scatter"));
+  ++launches;
+  BEAM_TRY(launch_quant_a1(xb, h->ids, h->inv, h->offsets, h->sf_block, T, H, k, h->cfg.alpha_a1, h->a1,
+                           h->a1_sf, s));
+  BEAM_TRY(mark("quant_a1"));
+  ++launches;
+
+  GemmArgs g{};
+  g.mblocks = h->mblocks;
+  g.num_mblocks = h->num_mblocks;
+  g.err = h->err;
+  // gate/up: 256 B rows per tile = 128 gate + 128 up features
+  g.n_tiles = h->I / 128;
+  g.k_tiles = H / 256;
+  g.n_rows_b = 2 * h->I;
+  g.sfa = h->a1_sf;
+  g.sfb = h->w_gu_sf;
+  g.alpha_b = h->w_gu_alpha;
+  g.alpha_a = h->cfg.alpha_a1;
+  g.a2 = h->a2;
+  g.a2_sf = h->a2_sf;
+  g.a2_row_bytes = h->Ip / 2;
+  g.a2_kgroups = h->Ip / 64;
+  g.alpha_a2 = h->cfg.alpha_a2;
+  BEAM_TRY(launch_gemm_gate_up(h->map_a1, h->map_wgu, g, h->num_sms, s));
+  BEAM_TRY(mark("gemm_gate_up"));
+  ++launches;
+  // down
+  g.n_tiles = H / 256;
+  g.k_tiles = h->Ip / 256;
+  g.n_rows_b = H;
+  g.sfa = h->a2_sf;
+  g.sfb = h->w_d_sf;
+  g.alpha_b = h->w_d_alpha;
+  g.alpha_a = h->cfg.alpha_a2;
+  g.y = h->y;
+  g.y_cols = H;
+  BEAM_TRY(launch_gemm_down(h->map_a2, h->map_wd, g, h->num_sms, s));
+  BEAM_TRY(mark("gemm_down"));
+  ++launches;
+  BEAM_TRY(launch_finalize(h->y, h->w, h->inv, static_cast<const uint16_t*>(residual), h->gamma, T, H, k,
+                           h->cfg.rms_eps, static_cast<uint16_t*>(out), s));
+  BEAM_TRY(mark("finalize"));
+  ++launches;
+  h->last_T = T;
+  h->last_launches = launches;
+  h->profiled_last = prof;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const void* residual_host, void* out_host,
+                                      int32_t num_tokens, void* stream) {
+  if (!h) return BEAM_MOE_ERR_INVALID_ARG;
+  if (num_tokens < 0 || num_tokens > h->Tmax) return BEAM_MOE_ERR_INVALID_ARG;
+  if (num_tokens == 0) return beam_moe_forward(h, nullptr, nullptr, nullptr, 0, stream);
+  if (!x_host || !residual_host || !out_host) return BEAM_MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = sizeof(uint16_t) * static_cast<size_t>(num_tokens) * h->H;
+  BEAM_TRY(cudaMemcpyAsync(h->stage_x, x_host, bytes, cudaMemcpyHostToDevice, s));
+  BEAM_TRY(cudaMemcpyAsync(h->stage_res, residual_host, bytes, cudaMemcpyHostToDevice, s));
+  beam_moe_status st = beam_moe_forward(h, h->stage_x, h->stage_res, h->stage_out, num_tokens, stream);
+  if (st != BEAM_MOE_OK) return st;
+  BEAM_TRY(cudaMemcpyAsync(out_host, h->stage_out, bytes, cudaMemcpyDeviceToHost, s));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_quantize_nvfp4(const float* src, int64_t rows, int64_t cols, float alpha, uint8_t* codes,
+                                        uint8_t* sf, float* alpha_out, void* stream) {
+  if (rows < 0 || cols < 0 || cols % 16 != 0) return BEAM_MOE_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return BEAM_MOE_OK;
+  if (!src || !codes || !sf) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!(alpha > 0.0f) && !alpha_out) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned(src, 16) || !aligned(codes, 8) || (alpha_out && !aligned(alpha_out, 4))) return BEAM_MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (alpha > 0.0f) {
+    BEAM_TRY(launch_quantize_rows(src, rows, cols, alpha, nullptr, codes, sf, s));
+    if (alpha_out) {
+      store_f32_kernel<<<1, 1, 0, s>>>(alpha_out, alpha);
+      BEAM_TRY(cudaGetLastError());
+    }
+    return BEAM_MOE_OK;
+  }
+  // alpha_out first holds amax (as FP32 bits), then the scale amax / 2688
+  BEAM_TRY(launch_amax(src, rows * cols, alpha_out, s));
+  BEAM_TRY(launch_quantize_rows(src, rows, cols, 0.0f, alpha_out, codes, sf, s));
+  BEAM_TRY(launch_amax_to_alpha(alpha_out, s));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, void* dst, size_t bytes, size_t* size_out,
+                                    void* stream) {
+  if (!h) return BEAM_MOE_ERR_INVALID_ARG;
+  const int64_t T = h->last_T, R = T * h->k;
+  const void* src = nullptr;
+  size_t n = 0;
+  switch (which) {
+    case BEAM_MOE_BUF_LOGITS: src = h->logits; n = sizeof(float) * route_ws_floats(static_cast<int>(T), h->H, h->E); break;
+    case BEAM_MOE_BUF_IDS: src = h->ids; n = sizeof(int32_t) * R; break;
+    case BEAM_MOE_BUF_WEIGHTS: src = h->w; n = sizeof(float) * R; break;
+    case BEAM_MOE_BUF_OFFSETS: src = h->offsets; n = sizeof(int32_t) * (h->E + 1); break;
+    case BEAM_MOE_BUF_PERM: src = h->perm; n = sizeof(int32_t) * R; break;
+    case BEAM_MOE_BUF_INV: src = h->inv; n = sizeof(int32_t) * R; break;
+    case BEAM_MOE_BUF_SFBLOCK: src = h->sf_block; n = sizeof(int32_t) * (h->E + 1); break;
+    case BEAM_MOE_BUF_A1: src = h->a1; n = static_cast<size_t>(R) * (h->H / 2); break;
+    case BEAM_MOE_BUF_A1_SF: src = h->a1_sf; n = static_cast<size_t>(h->nblk_max) * (h->H / 64) * 512; break;
+    case BEAM_MOE_BUF_A2: src = h->a2; n = static_cast<size_t>(R) * (h->Ip / 2); break;
+    case BEAM_MOE_BUF_A2_SF: src = h->a2_sf; n = static_cast<size_t>(h->nblk_max) * (h->Ip / 64) * 512; break;
+    case BEAM_MOE_BUF_Y: src = h->y; n = sizeof(uint16_t) * static_cast<size_t>(R) * h->H; break;
+    default: return BEAM_MOE_ERR_INVALID_ARG;
+  }
+  if (T == 0) n = 0;
+  if (size_out) *size_out = n;
+  if (!dst || bytes == 0 || n == 0) return BEAM_MOE_OK;
+  BEAM_TRY(cudaMemcpyAsync(dst, src, std::min(bytes, n), cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_check(beam_moe_t h, void* stream) {
+  if (!h) return BEAM_MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  BEAM_TRY(cudaStreamSynchronize(s));
+  uint32_t err = 0;
+  BEAM_TRY(cudaMemcpy(&err, h->err, sizeof(err), cudaMemcpyDeviceToHost));
+  if (err == 0) return BEAM_MOE_OK;
+  BEAM_TRY(cudaMemset(h->err, 0, sizeof(uint32_t)));
+  if (err & (kErrTimeoutProducer | kErrTimeoutMma | kErrTimeoutEpilogue)) return BEAM_MOE_ERR_TIMEOUT;
+  return BEAM_MOE_ERR_DEVICE;
+}
+
+int32_t beam_moe_last_launch_count(beam_moe_t h) { return h ? h->last_launches : 0; }
+
+beam_moe_status beam_moe_profile_enable(beam_moe_t h, int32_t enable) {
+  if (!h) return BEAM_MOE_ERR_INVALID_ARG;
+  if (enable && !h->events[0])
+    for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i) BEAM_TRY(cudaEventCreate(&h->events[i]));
+  h->profiling = enable != 0;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_profile_read(beam_moe_t h, float* ms, int32_t capacity, int32_t* count) {
+  if (!h || !count || (capacity > 0 && !ms)) return BEAM_MOE_ERR_INVALID_ARG;
+  *count = h->profiled_last ? h->last_launches : 0;
+  if (!h->profiled_last) return BEAM_MOE_OK;
+  BEAM_TRY(cudaEventSynchronize(h->events[h->last_launches]));
+  for (int i = 0; i < h->last_launches && i < capacity; ++i)
+    BEAM_TRY(cudaEventElapsedTime(&ms[i], h->events[i], h->events[i + 1]));
+  return BEAM_MOE_OK;
+}
+
+const char* beam_moe_kernel_name(beam_moe_t h, int32_t index) {
+  if (!h || index < 0 || index >= h->last_launches) return nullptr;
+  return h->names[index];
+}
+
+void beam_moe_destroy(beam_moe_t h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i)
+    if (h->events[i]) cudaEventDestroy(h->events[i]);
+  free_all(h);
+  delete h;
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// MoE finalize: weighted top-k un-permute, post-RMSNorm of the sandwich norm, residual add.
+//
+//   m[t]   = sum_j w[t][j] * y[inv[t][j]]              (FP32)
+//   out[t] = bf16( residual[t] + m[t] / sqrt(mean(m[t]^2) + eps) * gamma )
+//
+// The pages name this step (vLLM PR "Day-0 support for Reflection's Beam-1.0", sections
+// "Status" and "Remaining work": moe_finalize.cu, fused with the sandwich norms; news
+// article "vLLM adds day-zero Reflection Beam serving": fused normalisation and residual
+// kernels).  One CTA per token; every global access is a 16-byte vector (8 BF16), and a
+// warp's accesses are contiguous, so the k row gathers of y stream at full HBM width.
+#include "common.cuh"
+#include "internal.h"
+
+namespace beam {
+
+__device__ __forceinline__ void unpack8(const uint4 v, float (&f)[8]) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = bf16_bits_to_f32(u[i] & 0xFFFFu);
+    f[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);  // a -> low half
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+constexpr int kFinThreads = 128;
+
+__global__ void __launch_bounds__(kFinThreads) finalize_kernel(const uint16_t* __restrict__ y,
+                                                               const float* __restrict__ w,
+                                                               const int32_t* __restrict__ inv,
+                                                               const uint16_t* residual,
+                                                               const uint16_t* __restrict__ gamma, int H, int k,
+                                                               float eps, uint16_t* out) {
+  extern __shared__ float m_s[];  // [H]
+  __shared__ int s_row[16];
+  __shared__ float s_w[16];
+  __shared__ float s_red[kFinThreads / 32];
+  const int t = blockIdx.x;
+  if (threadIdx.x < k) {
+    s_row[threadIdx.x] = inv[static_cast<size_t>(t) * k + threadIdx.x];
+    s_w[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
+  }
+  __syncthreads();
+  const int nchunks = H / 8;
+  float ss = 0.0f;
+  for (int c = threadIdx.x; c < nchunks; c += kFinThreads) {
+    float acc[8] = {};
+    for (int j = 0; j < k; ++j) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j]) * H) + c);
+      float f[8];
+      unpack8(v, f);
+      const float wj = s_w[j];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      m_s[c * 8 + i] = acc[i];
+      ss = fmaf(acc[i], acc[i], ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kFinThreads / 32; ++i) tot += s_red[i];
+  const float rinv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+  for (int c = threadIdx.x; c < nchunks; c += kFinThreads) {
+    float r[8], g[8];
+    unpack8(reinterpret_cast<const uint4*>(residual + static_cast<size_t>(t) * H)[c], r);  // out may alias residual
+    unpack8(__ldg(reinterpret_cast<const uint4*>(gamma) + c), g);
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = r[2 * i] + m_s[c * 8 + 2 * i] * rinv * g[2 * i];
+      const float b = r[2 * i + 1] + m_s[c * 8 + 2 * i + 1] * rinv * g[2 * i + 1];
+      o[i] = pack_bf16x2(a, b);
+    }
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
+                            const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(H) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e =
+        cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  finalize_kernel<<<T, kFinThreads, smem, s>>>(y, w, inv, residual, gamma, H, k, eps, out);
+  return cudaGetLastError();
+}
+
+}  // namespace beam

@@ -1,0 +1,217 @@
+// Token -> expert histogram, prefix scan, permutation, and the NVFP4 quantisation of the
+// expert inputs fused into the permute.
+//
+// The permuted order lists the (token, slot) pairs of expert e in rows
+// [offsets[e], offsets[e+1]), in ascending token order.  It is deterministic: the rank
+// of token t among the tokens of its chunk that chose expert e is a popcount of a
+// per-warp bitmask (OR is order-independent), and chunk bases come from a sequential
+// per-expert scan over chunks.  Each expert's rows are also cut into 128-row work blocks
+// (the M tiles of the grouped GEMMs), each with its own scale block so the tensor-core
+// scale layout stays aligned to 128 rows whatever offsets[e] is.
+//
+// A1 = Q(x, alpha_a1): x rows are quantised once per token (16-value blocks along H) and
+// the codes are written to the token's k permuted rows (the NVFP4 W4A4 experts of the
+// recipe "reflection/Beam-1.0-501B-A23B", section "Variants").
+#include "common.cuh"
+#include "internal.h"
+
+namespace beam {
+
+// chunk_counts[c][e] = number of (t, j) in chunk c with ids[t][j] == e
+__global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
+                                                         int32_t* __restrict__ chunk_counts) {
+  extern __shared__ int32_t cnt[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kChunkTokens;
+  const int n = min(kChunkTokens, T - t0) * k;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = ids[static_cast<size_t>(t0) * k + i];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
+}
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += u;
+  }
+  if (lane == 31) warp_sums[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < nwarps ? warp_sums[lane] : 0;
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += u;
+    }
+    if (lane < nwarps) warp_sums[lane] = si - s;  // exclusive prefix of warp totals
+    if (lane == 31) warp_sums[32] = si;           // grand total
+  }
+  __syncthreads();
+  total = warp_sums[32];
+  const int r = warp_sums[warp] + inc - v;
+  __syncthreads();
+  return r;
+}
+
+// One CTA, one thread per expert.
+__global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chunks, int E,
+                            int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
+                            int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks,
+                            int32_t* __restrict__ num_mblocks) {
+  __shared__ int warp_sums[33];
+  const int e = threadIdx.x;
+  int cnt = 0;
+  if (e < E) {
+    for (int c = 0; c < n_chunks; ++c) {
+      const size_t i = static_cast<size_t>(c) * E + e;
+      const int v = chunk_counts[i];
+      chunk_base[i] = cnt;
+      cnt += v;
+    }
+  }
+  const int nblk = (cnt + 127) / 128;
+  int total_rows, total_blk;
+  const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
+  const int blk = block_exclusive_scan(nblk, warp_sums, total_blk);
+  if (e < E) {
+    offsets[e] = off;
+    sf_block[e] = blk;
+    for (int c = 0; c < n_chunks; ++c) chunk_base[static_cast<size_t>(c) * E + e] += off;
+    for (int i = 0; i < nblk; ++i) {
+      MBlock m;
+      m.expert = e;
+      m.row_begin = off + 128 * i;
+      m.rows = min(128, cnt - 128 * i);
+      m.sf_block = blk + i;
+      mblocks[blk + i] = m;
+    }
+  }
+  if (e == 0) {
+    offsets[E] = total_rows;
+    sf_block[E] = total_blk;
+    *num_mblocks = total_blk;
+  }
+}
+
+// perm_src[r] = t and inv[t][j] = r for every (t, j) of one chunk of 256 tokens.
+__global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ ids,
+                                                      const int32_t* __restrict__ chunk_base, int T, int k, int E,
+                                                      int32_t* __restrict__ perm_src, int32_t* __restrict__ inv) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* mask = sm;                                    // [8][E]
+  int32_t* pre = reinterpret_cast<int32_t*>(sm + 8 * E);  // [8][E]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) mask[i] = 0;
+  __syncthreads();
+  const int chunk = blockIdx.x;
+  const int t = chunk * kChunkTokens + warp * 32 + lane;
+  if (t < T)
+    for (int j = 0; j < k; ++j) atomicOr(&mask[warp * E + ids[static_cast<size_t>(t) * k + j]], 1u << lane);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      pre[w * E + e] = run;
+      run += __popc(mask[w * E + e]);
+    }
+  }
+  __syncthreads();
+  if (t < T) {
+    const uint32_t below = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[static_cast<size_t>(t) * k + j];
+      const int rank = pre[warp * E + e] + __popc(mask[warp * E + e] & below);
+      const int r = chunk_base[static_cast<size_t>(chunk) * E + e] + rank;
+      perm_src[r] = t;
+      inv[static_cast<size_t>(t) * k + j] = r;
+    }
+  }
+}
+
+// One warp per token: quantise x[t] once, write it to the token's k permuted rows.
+__global__ void __launch_bounds__(256) quant_a1_kernel(const uint16_t* __restrict__ x,
+                                                       const int32_t* __restrict__ ids,
+                                                       const int32_t* __restrict__ inv,
+                                                       const int32_t* __restrict__ offsets,
+                                                       const int32_t* __restrict__ sf_block, int T, int H, int k,
+                                                       float alpha, uint8_t* __restrict__ a1,
+                                                       uint8_t* __restrict__ a1_sf) {
+  __shared__ int s_r[8][16], s_blk[8][16], s_m[8][16];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  // lane j < k: the permuted row of slot j and where its scales live
+  if (lane < k) {
+    const int r = inv[static_cast<size_t>(t) * k + lane];
+    const int e = ids[static_cast<size_t>(t) * k + lane];
+    const int li = r - offsets[e];
+    s_r[warp][lane] = r;
+    s_blk[warp][lane] = sf_block[e] + (li >> 7);
+    s_m[warp][lane] = li & 127;
+  }
+  __syncwarp();
+  const float six_alpha = __fmul_rn(6.0f, alpha);
+  const int nb = H / 16, kgroups = H / 64;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+  for (int b = lane; b < nb; b += 32) {
+    const uint4 p0 = __ldg(xr + 2 * b), p1 = __ldg(xr + 2 * b + 1);
+    const uint32_t u[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = bf16_bits_to_f32(u[i] & 0xFFFFu);
+      v[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+    }
+    uint32_t lo, hi;
+    const uint32_t sc = quant_block16(v, alpha, six_alpha, lo, hi);
+    for (int j = 0; j < k; ++j) {
+      const int r = s_r[warp][j], blk = s_blk[warp][j], m = s_m[warp][j];
+      *reinterpret_cast<uint2*>(a1 + static_cast<size_t>(r) * (H / 2) + b * 8) = make_uint2(lo, hi);
+      a1_sf[sf_atom_offset(blk, kgroups, m, b)] = static_cast<uint8_t>(sc);
+    }
+  }
+}
+
+cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s) {
+  const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
+  chunk_hist_kernel<<<n_chunks, 256, E * sizeof(int32_t), s>>>(ids, T, k, E, chunk_counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
+                        int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, cudaStream_t s) {
+  const int threads = ((E + 31) / 32) * 32;
+  scan_kernel<<<1, threads, 0, s>>>(chunk_counts, n_chunks, E, chunk_base, offsets, sf_block, mblocks, num_mblocks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, int T, int k, int E, int32_t* perm_src,
+                           int32_t* inv, cudaStream_t s) {
+  const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
+  const size_t smem = static_cast<size_t>(16) * E * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  scatter_kernel<<<n_chunks, 256, smem, s>>>(ids, chunk_base, T, k, E, perm_src, inv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* ids, const int32_t* inv, const int32_t* offsets,
+                            const int32_t* sf_block, int T, int H, int k, float alpha, uint8_t* a1, uint8_t* a1_sf,
+                            cudaStream_t s) {
+  quant_a1_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, ids, inv, offsets, sf_block, T, H, k, alpha, a1, a1_sf);
+  return cudaGetLastError();
+}
+
+}  // namespace beam

@@ -1,0 +1,95 @@
+"""Helpers of the GPU parity tests: reading the library's internal buffers back into the
+oracle's layouts, and the output comparison at the layer's tolerances."""
+
+import numpy as np
+import torch
+
+import moe_inputs as mi
+import sparse_moe_layer_fp32_b200 as bm
+from oracle import moe, nvfp4
+
+# Output tolerance of the layer against the oracle: relative L2 1e-2 and per-element
+# absolute 5e-2 (tokens whose 8th/9th logit gap is a near-tie are excluded and counted).
+REL_L2 = 1e-2
+ABS_MAX = 5e-2
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def buf(layer, which, dtype):
+    return to_np(layer.debug(which)).view(dtype)
+
+
+def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int) -> np.ndarray:
+    """Scale blocks (beam_moe.h layout) -> row-major scales [rows, kcols/16] in permuted row order."""
+    experts = len(offsets) - 1
+    rows = int(offsets[-1])
+    kgroups = kcols // 64
+    out = np.zeros((rows, kcols // 16), np.uint8)
+    s = np.arange(kcols // 16)
+    for e in range(experts):
+        n = int(offsets[e + 1] - offsets[e])
+        if n == 0:
+            continue
+        i = np.arange(n)
+        blk = sf_block[e] + i // 128
+        m = i % 128
+        off = ((blk[:, None] * kgroups + s[None, :] // 4) * 512 + (m[:, None] % 32) * 16 + (m[:, None] // 32) * 4
+               + s[None, :] % 4)
+        out[offsets[e]:offsets[e + 1]] = sf_buf[off]
+    return out
+
+
+def norm_zero(packed: np.ndarray) -> np.ndarray:
+    """Map the E2M1 negative zero (code 8) to +0 in packed bytes (+-0 are equal values)."""
+    c = nvfp4.unpack_nibbles(packed)
+    c[c == 8] = 0
+    return nvfp4.pack_nibbles(c)
+
+
+def compare_outputs(gpu_out: np.ndarray, ref_pre: np.ndarray, skip=None):
+    """Returns (rel_l2, max_abs) of the GPU output against the oracle's, rows in skip excluded."""
+    keep = np.ones(gpu_out.shape[0], bool) if skip is None else ~np.asarray(skip, bool)
+    g, r = gpu_out[keep], ref_pre[keep]
+    if g.size == 0:
+        return 0.0, 0.0
+    rel = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30))
+    return rel, float(np.max(np.abs(g - r)))
+
+
+def ids_match(gpu_ids: np.ndarray, ref_ids: np.ndarray, logits: np.ndarray, near: np.ndarray, rel=1e-5):
+    """Routing equality except at near-ties.  Slots whose logits are within the near-tie
+    gap of a neighbour may swap order; everything else must match exactly."""
+    bad = []
+    for t in range(ref_ids.shape[0]):
+        if near[t]:
+            continue
+        if set(gpu_ids[t].tolist()) != set(ref_ids[t].tolist()):
+            bad.append(t)
+            continue
+        if not np.array_equal(gpu_ids[t], ref_ids[t]):
+            lv = logits[t, ref_ids[t]]
+            gap = np.abs(np.diff(lv))
+            tol = rel * np.maximum(np.maximum(np.abs(lv[:-1]), np.abs(lv[1:])), 1.0)
+            # every position that differs must sit next to a near-equal neighbour
+            diff = np.nonzero(gpu_ids[t] != ref_ids[t])[0]
+            if not all((j > 0 and gap[j - 1] < tol[j - 1]) or (j < len(gap) and gap[j] < tol[j]) for j in diff):
+                bad.append(t)
+    return bad
+
+
+def oracle_layer_inputs(shape: mi.LayerShape, seed: int, weights_fp32=None, tokens=None):
+    """Oracle-side inputs of a workload: x, residual (FP64 of BF16), W_r, gamma, expert cache."""
+    xb, rb = mi.tokens(shape, seed) if tokens is None else tokens
+    x = mi.bf16_bits_to_f32(xb).astype(np.float64)
+    res = mi.bf16_bits_to_f32(rb).astype(np.float64)
+    wr = mi.router_weight(shape, seed)
+    g = mi.bf16_bits_to_f32(mi.gamma(shape, seed)).astype(np.float64)
+    getter = weights_fp32 or (lambda e: mi.expert_weights(shape, seed, e))
+    return x, res, wr, g, moe.ExpertCache(getter, keep=16)

@@ -1,0 +1,154 @@
+"""Whole-layer GPU forward (beam_moe_forward through the C ABI) against the oracle, stage by
+stage and end to end, on small shapes that still span several tiles and ragged tails.
+
+Each stage is checked on the GPU's own previous-stage output, so one stage's rounding does
+not cascade into the next check:
+  routing ids/w      exact except near-ties
+  offsets/perm/inv   bit-exact vs the oracle permutation of the GPU ids
+  A1 codes/scales    bit-exact vs the oracle quantiser on the permuted x rows
+  A2 (SwiGLU NVFP4)  code mismatch rate (GPU FP32 h vs oracle FP64 h may straddle a
+                     rounding boundary) and dequantised relative L2
+  y                  relative L2 vs the oracle down GEMM of the GPU's A2
+  out                vs the oracle finalize of the GPU's y, and end to end vs the oracle
+Sources: router 5120 -> 256 and the fused finalize/sandwich norm (vLLM PR "Day-0 support
+for Reflection's Beam-1.0", section "Status"); 8 of 256 experts and NVFP4 W4A4 experts
+(recipe "reflection/Beam-1.0-501B-A23B", sections "Overview" and "Variants")."""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+import moe_inputs as mi  # noqa: E402
+from oracle import moe, nvfp4  # noqa: E402
+from tests.gpu_util import (ABS_MAX, REL_L2, bf16_to_f64, buf, compare_outputs, ids_match, norm_zero,  # noqa: E402
+                            oracle_layer_inputs, sf_rows, to_np)
+
+
+@pytest.fixture(scope="module")
+def bm():
+    import sparse_moe_layer_fp32_b200 as m
+    return m
+
+
+# (name, shape) — tiny is the workload of the same name; "mid" spans 2-3 output tiles and
+# 2 K tiles per GEMM with an intermediate size that needs K padding (384 -> 512).
+SHAPES = {
+    "tiny": mi.SHAPES["tiny"],
+    "mid": mi.LayerShape("mid", 0, 512, 32, 4, 384),
+}
+
+
+def _scales(shape, x, res, wr, g, cache):
+    a1 = np.float32(np.float32(np.abs(x).max()) / np.float32(2688))
+    r = moe.moe_forward_tokens(x, res, wr, g, cache, shape.top_k, a1, np.float32(1.0))
+    return a1, np.float32(np.float32(np.abs(r["h32"]).max()) / np.float32(2688))
+
+
+def _run(bm, shape, tokens, seed, max_tokens=None):
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(shape, tokens=tokens)
+    x, res, wr, g, cache = oracle_layer_inputs(shape, seed)
+    a1, a2 = _scales(shape, x, res, wr, g, cache)
+    weights = synthetic.make_weights(shape, seed, threads=4)
+    layer = bm.MoELayer(max_tokens=max_tokens or max(tokens, 1), hidden=shape.hidden, num_experts=shape.experts,
+                        top_k=shape.top_k, inter=shape.inter, alpha_a1=float(a1), alpha_a2=float(a2), **weights)
+    xd, rd = synthetic.make_batch(shape, seed)
+    out = layer.forward(xd, rd)
+    layer.check()
+    ref = moe.moe_forward(x, res, wr, g, cache, shape.experts, shape.top_k, a1, a2, shape.rms_eps)
+    return shape, layer, weights, out, ref, (x, res, wr, g, cache, a1, a2)
+
+
+@pytest.mark.parametrize("name,tokens,seed", [("tiny", 4, 0), ("tiny", 1, 1), ("tiny", 37, 2), ("tiny", 1500, 3),
+                                              ("mid", 200, 4), ("mid", 7, 5)])
+def test_forward_stages_and_end_to_end(bm, name, tokens, seed):
+    shape, layer, weights, out, ref, (x, res, wr, g, cache, a1, a2) = _run(bm, SHAPES[name], tokens, seed)
+    T, E, k, H, I = tokens, shape.experts, shape.top_k, shape.hidden, shape.inter
+    Ip = (I + 255) // 256 * 256
+    # ---- routing
+    ids = buf(layer, bm.BUF_IDS, np.int32).reshape(T, k)
+    w = buf(layer, bm.BUF_WEIGHTS, np.float32).reshape(T, k)
+    near = ref["near_tie"]
+    assert not ids_match(ids, ref["ids"], ref["logits"], near)
+    np.testing.assert_allclose(w.sum(1), 1.0, atol=1e-5)
+    # ---- permutation of the GPU ids: bit-exact
+    pm = moe.permute(ids.astype(np.int64), E)
+    offsets = buf(layer, bm.BUF_OFFSETS, np.int32)
+    perm = buf(layer, bm.BUF_PERM, np.int32)
+    inv = buf(layer, bm.BUF_INV, np.int32).reshape(T, k)
+    sfb = buf(layer, bm.BUF_SFBLOCK, np.int32)
+    np.testing.assert_array_equal(offsets, pm["offsets"])
+    np.testing.assert_array_equal(perm, pm["perm_src"])
+    np.testing.assert_array_equal(inv, pm["inv"])
+    nblk = np.array([(c + 127) // 128 for c in pm["counts"]])
+    np.testing.assert_array_equal(sfb, np.concatenate([[0], np.cumsum(nblk)]))
+    # ---- A1: bit-exact
+    a1p = buf(layer, bm.BUF_A1, np.uint8).reshape(T * k, H // 2)
+    a1s = sf_rows(buf(layer, bm.BUF_A1_SF, np.uint8), sfb, offsets, H)
+    rp, rs = nvfp4.quantize_nvfp4(x[perm].astype(np.float32), a1)
+    np.testing.assert_array_equal(a1s, rs)
+    np.testing.assert_array_equal(norm_zero(a1p), norm_zero(rp))
+    # ---- A2 and y from the GPU's own inputs
+    a2p = buf(layer, bm.BUF_A2, np.uint8).reshape(T * k, Ip // 2)[:, : I // 2]
+    a2s = sf_rows(buf(layer, bm.BUF_A2_SF, np.uint8), sfb, offsets, Ip)[:, : I // 16]
+    y = to_np(layer.debug(bm.BUF_Y).view(torch.bfloat16).float()).reshape(T * k, H).astype(np.float64)
+    mism, n_codes = 0, 0
+    y_ref = np.zeros_like(y)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if lo == hi:
+            continue
+        deq = cache.dequantized(e)
+        r = moe.expert_forward(a1p[lo:hi], a1s[lo:hi], a1, deq, a2)
+        c_gpu = nvfp4.unpack_nibbles(norm_zero(a2p[lo:hi]))
+        c_ref = nvfp4.unpack_nibbles(norm_zero(r["a2_packed"]))
+        mism += int((c_gpu != c_ref).sum()) + int((a2s[lo:hi] != r["a2_sf"]).sum())
+        n_codes += c_gpu.size
+        y_ref[lo:hi] = nvfp4.dequantize_nvfp4(a2p[lo:hi], a2s[lo:hi], a2) @ deq[1].T
+        d_gpu = nvfp4.dequantize_nvfp4(a2p[lo:hi], a2s[lo:hi], a2)
+        d_ref = nvfp4.dequantize_nvfp4(r["a2_packed"], r["a2_sf"], a2)
+        assert np.linalg.norm(d_gpu - d_ref) <= 1e-2 * max(np.linalg.norm(d_ref), 1e-30)
+    assert mism <= max(2, 1e-3 * n_codes), f"A2 mismatches {mism} of {n_codes}"
+    rel_y = np.linalg.norm(y - y_ref) / max(np.linalg.norm(y_ref), 1e-30)
+    assert rel_y < 5e-3, rel_y
+    # ---- finalize of the GPU's own y, w, inv
+    out_np = bf16_to_f64(out)
+    pre, _, _ = moe.finalize(y[inv], w.astype(np.float64), res, g, shape.rms_eps)
+    assert np.all(np.abs(out_np - pre) <= 2.0 ** -8 * np.maximum(np.abs(pre), 1.0))
+    # ---- end to end
+    rel, mx = compare_outputs(out_np, ref["out_pre"], skip=near)
+    assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
+    assert layer.launches() > 0
+    layer.close()
+
+
+def test_forward_edge_cases(bm):
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(SHAPES["tiny"], tokens=6)
+    weights = synthetic.make_weights(shape, 0, threads=2)
+    layer = bm.MoELayer(max_tokens=6, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                        inter=shape.inter, alpha_a1=0.0012, alpha_a2=0.00012, **weights)
+    x, r = synthetic.make_batch(shape, 0)
+    out = layer.forward(x, r)
+    # in place: out == residual
+    r2 = r.clone()
+    layer.forward(x, r2, out=r2)
+    torch.cuda.synchronize()
+    assert torch.equal(out, r2)
+    # zero tokens is a no-op; more than max_tokens is rejected before launching
+    layer.forward(x[:0], r[:0])
+    with pytest.raises(bm.BeamMoeError) as ei:
+        bm.beam_moe_forward(layer.handle, torch.cat([x, x[:1]]), torch.cat([r, r[:1]]), torch.empty_like(
+            torch.cat([r, r[:1]])), 7)
+    assert ei.value.status == bm.ERR_INVALID_ARG
+    # repeated calls are deterministic
+    o1 = layer.forward(x, r)
+    o2 = layer.forward(x, r)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    layer.check()
+    layer.close()
