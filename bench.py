@@ -69,20 +69,22 @@ def kernel_work(shape: mi.LayerShape, T: int, counts: np.ndarray) -> dict:
     }
 
 
-def read_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+def read_traffic(kernel: str, used_experts: int):
+    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json), scaled
+    by the experts that received tokens; None when the kernel's source changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        tab = json.load(f)
-    ent = tab.get(f"{kernel}@{workload}")
+        ent = json.load(f).get(kernel)
     if not ent:
         return None
     import hashlib
     src = os.path.join(ROOT, "sparse_moe_layer_fp32_b200", "csrc", ent["source"])
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return ent["bytes_per_launch"] if digest == ent["source_sha256_16"] else None
+    if digest != ent["source_sha256_16"]:
+        return None
+    return ent["bytes_per_used_expert"] * used_experts
 
 
 # ------------------------------------------------------------------ clocks
@@ -234,6 +236,8 @@ def run_ours(args, shape, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     weights = synthetic.make_weights(shape, 0, device=dev)
     layer = synthetic.make_layer(shape, weights)
+    del weights  # the handle holds its own repacked copy
+    torch.cuda.empty_cache()
     x, res = synthetic.make_batch(shape, seed=rank)  # each replica its own batch
     x, res = x.to(dev), res.to(dev)
     out = torch.empty_like(res)
@@ -297,7 +301,7 @@ def run_ours(args, shape, rank, world, local_rank):
         bound, achieved, peak, unit = "hbm", wk["bytes"] / (kern[top] / 1e3) / 1e9, pk["hbm"], "GB/s"
         peak_note = f"{pk['src']} copy bandwidth"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": read_traffic(top, shape.name), "kernel": top, "kernel_ms": kern[top],
+                "traffic": read_traffic(top, work["_used_experts"]), "kernel": top, "kernel_ms": kern[top],
                 "peak_source": peak_note}
 
     # ---- end to end through the host-buffer entry point (copies inside the timed region)

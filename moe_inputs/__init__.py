@@ -56,6 +56,9 @@ SHAPES = {
         LayerShape("prefill32k_skew", 32768, 5120, 256, 8, 1536, skew=True),
         # intermediate size implied by the pages' checkpoint sizes (a labelled extra)
         LayerShape("decode8_i2560", 8, 5120, 256, 8, 2560),
+        # profiling case: the decode step's per-expert shapes with 32 experts, so that a
+        # multi-pass profiler capture holds a few GB (weights still far larger than L2)
+        LayerShape("decode8_e32", 8, 5120, 32, 8, 1536),
     ]
 }
 
@@ -134,5 +137,8 @@ def activation_scales(shape: LayerShape):
     with open(_SCALES_FILE) as f:
         table = json.load(f)
     key = f"h{shape.hidden}_e{shape.experts}_k{shape.top_k}_i{shape.inter}"
+    if key not in table:
+        # the scales depend on the x and weight distributions, not on the expert count
+        key = next(k for k in table if k.startswith(f"h{shape.hidden}_") and k.endswith(f"_k{shape.top_k}_i{shape.inter}"))
     a1, a2 = table[key]["alpha_a1"], table[key]["alpha_a2"]
     return np.float32(a1), np.float32(a2)
