@@ -120,6 +120,28 @@ BEAM_MOE_API beam_moe_status beam_moe_route(const void* x, const float* router_w
                                int32_t num_experts, int32_t top_k, float* logits_ws, int32_t* ids, float* w,
                                void* stream);
 
+/* Routing without any device allocation.  The pages have no counterpart of this entry
+ * point: it exists for callers that cannot call cudaMalloc, such as plugins inside a host
+ * engine that owns all device memory and hands them only their inputs and outputs, or
+ * latency-critical loops where an allocation (and the device synchronisation it can
+ * imply) is not allowed after start-up.  Same result as beam_moe_route (same kernels),
+ * but the logits scratch is a fixed 8 MiB array compiled into this library: every GPU
+ * that loads the library holds it until the process exits.
+ *   - Accepts exactly the shapes whose beam_moe_route_workspace_bytes(T, H, E) is at
+ *     most 8 MiB (at H = 5120, E = 256: T <= 4096 and 4736 <= T <= 8192); larger shapes
+ *     return BEAM_MOE_ERR_UNSUPPORTED before anything is enqueued.
+ *   - The first call on each device looks up the array's device address (with that
+ *     device current) and caches it; make that first call before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's contents
+ *     (every element a call reads it first writes, so nothing needs clearing).  Calls
+ *     that overlap on the GPU (different streams, or different host threads) race on it:
+ *     order them.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ * Arguments and outputs as beam_moe_route, without logits_ws. */
+BEAM_MOE_API beam_moe_status beam_moe_route_static(const void* x, const float* router_w, int32_t num_tokens,
+                                                   int32_t hidden, int32_t num_experts, int32_t top_k, int32_t* ids,
+                                                   float* w, void* stream);
+
 /* NVFP4 quantiser Q (weights or activations): src [rows][cols] FP32 row-major, cols %
  * 16 == 0.  codes [rows][cols/2], sf [rows][cols/16] (row-major scale bytes).  alpha >
  * 0 uses that tensor scale; alpha <= 0 computes alpha = amax(src) / 2688 on the device

@@ -24,7 +24,7 @@ EXPORTED = [
     "beam_moe_create", "beam_moe_forward", "beam_moe_forward_host", "beam_moe_route",
     "beam_moe_route_workspace_bytes", "beam_moe_quantize_nvfp4", "beam_moe_debug_copy", "beam_moe_check",
     "beam_moe_last_launch_count", "beam_moe_status_string", "beam_moe_destroy", "beam_moe_profile_enable",
-    "beam_moe_profile_read", "beam_moe_kernel_name",
+    "beam_moe_profile_read", "beam_moe_kernel_name", "beam_moe_route_static",
 ]
 
 
@@ -67,6 +67,7 @@ def _load():
         "beam_moe_profile_enable": (i32, [vp, i32]),
         "beam_moe_profile_read": (i32, [vp, ctypes.POINTER(f32), i32, ctypes.POINTER(i32)]),
         "beam_moe_kernel_name": (ctypes.c_char_p, [vp, i32]),
+        "beam_moe_route_static": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
