@@ -215,13 +215,38 @@ def run_reference(args, shape, rank, world):
                          "sample": f"{len(cpu_sample_tokens(shape))} token(s) of the {shape.name} batch per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    emit(line, rank)
 
 
 def workload_config(shape):
     return {"workload": shape.name, "tokens": shape.tokens, "hidden": shape.hidden, "experts": shape.experts,
             "top_k": shape.top_k, "inter": shape.inter, "routing": "zipf-skewed" if shape.skew else "uniform",
             "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MiB write between timed steps"}
+
+
+# ------------------------------------------------------------------ multi-rank plumbing
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank number over all ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Tokens per second of the whole job: every rank processes its own batch (weak scaling)."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
+def emit(line: dict, rank: int, stream=None) -> bool:
+    """Rank 0 alone prints the JSON line."""
+    if rank != 0:
+        return False
+    print(json.dumps(line), file=stream or sys.stdout, flush=True)
+    return True
 
 
 # ------------------------------------------------------------------ GPU leg
@@ -268,12 +293,8 @@ def run_ours(args, shape, rank, world, local_rank):
         barrier()
     launches = layer.launches() * args.steps
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = sum(step_ms) / args.steps
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    value = world * T / (ms / 1e3)
+    ms = reduce_max(sum(step_ms) / args.steps, world, dev)
+    value = whole_job_rate(T, world, ms)
     layer.check()
 
     # ---- per-kernel durations (CUDA events inside the library, same stream), separate pass
@@ -321,11 +342,7 @@ def run_ours(args, shape, rank, world, local_rank):
         flush.zero_()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)) / args.steps
-    t = torch.tensor([e2e_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)) / args.steps, world, dev)
     assert torch.equal(oh.to(dev), layer.forward(x, res)), "host-buffer path differs from device path"
 
     line = None
@@ -339,7 +356,7 @@ def run_ours(args, shape, rank, world, local_rank):
             "roofline": roofline,
             "kernels_ms": kern,
             "used_experts": work["_used_experts"],
-            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": 2 * T * shape.hidden * 2,
+            "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * T * shape.hidden * 2,
                     "d2h_bytes_per_step": T * shape.hidden * 2},
             "gpu_launches": launches,
             "clocks": clk.summary(),
@@ -376,10 +393,9 @@ def main():
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
-    if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(shape)
-        print(json.dumps(line), flush=True)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(shape)
+    emit(line, rank)
 
 
 if __name__ == "__main__":

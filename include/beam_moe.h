@@ -151,22 +151,25 @@ BEAM_MOE_API beam_moe_status beam_moe_quantize_nvfp4(const float* src, int64_t r
 
 /* Internal buffers of the last forward, for tests (layouts in the comment of each id). */
 typedef enum {
-  BEAM_MOE_BUF_LOGITS = 0,   /* [T][E] FP32                                                */
+  BEAM_MOE_BUF_LOGITS = 0,   /* [S][T][E] FP32 partial sums over S slices of H (S = size/(4TE)) */
   BEAM_MOE_BUF_IDS = 1,      /* [T][k] int32                                               */
   BEAM_MOE_BUF_WEIGHTS = 2,  /* [T][k] FP32                                                */
   BEAM_MOE_BUF_OFFSETS = 3,  /* [E+1] int32: rows of expert e are [off[e], off[e+1])       */
   BEAM_MOE_BUF_PERM = 4,     /* [T*k] int32: token of permuted row r                        */
   BEAM_MOE_BUF_INV = 5,      /* [T][k] int32: permuted row of (token, slot)                */
   BEAM_MOE_BUF_SFBLOCK = 6,  /* [E+1] int32: first 128-row scale block of each expert      */
-  BEAM_MOE_BUF_A1 = 7,       /* [T*k][H/2] NVFP4 codes of the permuted expert inputs       */
+  BEAM_MOE_BUF_A1 = 7,       /* activation tiles (below) of the permuted expert inputs, K = H */
   BEAM_MOE_BUF_A1_SF = 8,    /* scale blocks: [nblk][H/64][512], see below                 */
-  BEAM_MOE_BUF_A2 = 9,       /* [T*k][Ip/2] codes of the SwiGLU outputs, Ip = ceil(I/256)*256 */
+  BEAM_MOE_BUF_A2 = 9,       /* activation tiles of the SwiGLU outputs, K = Ip = ceil(I/256)*256 */
   BEAM_MOE_BUF_A2_SF = 10,   /* [nblk][Ip/64][512]                                          */
   BEAM_MOE_BUF_Y = 11        /* [T*k][H] BF16 expert outputs in permuted row order          */
 } beam_moe_buffer;
-/* Scale blocks: the rows of expert e, local row i = r - off[e], live in block
- * sfblock[e] + i/128, row m = i%128; for scale s of that row the byte is at
- * ((block * (K/64) + s/4) * 512) + (m%32)*16 + (m/32)*4 + s%4. */
+/* Blocks: the rows of expert e, local row i = r - off[e], live in block
+ * blk = sfblock[e] + i/128, row m = i%128.
+ * Scale blocks: scale s of that row is the byte at
+ * ((blk * (K/64) + s/4) * 512) + (m%32)*16 + (m/32)*4 + s%4.
+ * Activation tiles: codes byte j of that row (values 2j, 2j+1) is at
+ * ((blk * (K/256) + j/128) * 16384) + m*128 + ((((j%128)/16) ^ (m%8)) * 16) + j%16. */
 
 /* Copies min(bytes, size of the buffer) bytes of internal buffer `which` to dst (device),
  * enqueued on `stream`.  *size_out (host, may be NULL) receives the buffer's size for the
@@ -190,6 +193,12 @@ BEAM_MOE_API beam_moe_status beam_moe_profile_read(beam_moe_t h, float* ms, int3
 
 /* Name of the index-th kernel of the last forward ("router", "topk", ...), or NULL. */
 BEAM_MOE_API const char* beam_moe_kernel_name(beam_moe_t h, int32_t index);
+
+/* Failure-detection check: enqueues one CTA that waits, with the same bounded mbarrier
+ * wait as the GEMM kernels, on a barrier nothing completes.  After limit_ns (1 ns .. 2 s)
+ * it gives up, sets the timeout bit of the device error word and exits normally, so the
+ * next beam_moe_check returns BEAM_MOE_ERR_TIMEOUT and the context stays usable. */
+BEAM_MOE_API beam_moe_status beam_moe_debug_wait_timeout(beam_moe_t h, int64_t limit_ns, void* stream);
 
 /* Number of kernels the last beam_moe_forward enqueued. */
 BEAM_MOE_API int32_t beam_moe_last_launch_count(beam_moe_t h);

@@ -59,6 +59,8 @@ SHAPES = {
         # profiling case: the decode step's per-expert shapes with 32 experts, so that a
         # multi-pass profiler capture holds a few GB (weights still far larger than L2)
         LayerShape("decode8_e32", 8, 5120, 32, 8, 1536),
+        # profiling case: the 8 x 2K prefill's rows per expert (512) with 32 experts
+        LayerShape("prefill2k_e32", 2048, 5120, 32, 8, 1536),
     ]
 }
 

@@ -24,7 +24,7 @@ EXPORTED = [
     "beam_moe_create", "beam_moe_forward", "beam_moe_forward_host", "beam_moe_route",
     "beam_moe_route_workspace_bytes", "beam_moe_quantize_nvfp4", "beam_moe_debug_copy", "beam_moe_check",
     "beam_moe_last_launch_count", "beam_moe_status_string", "beam_moe_destroy", "beam_moe_profile_enable",
-    "beam_moe_profile_read", "beam_moe_kernel_name", "beam_moe_route_static",
+    "beam_moe_profile_read", "beam_moe_kernel_name", "beam_moe_route_static", "beam_moe_debug_wait_timeout",
 ]
 
 
@@ -68,6 +68,7 @@ def _load():
         "beam_moe_profile_read": (i32, [vp, ctypes.POINTER(f32), i32, ctypes.POINTER(i32)]),
         "beam_moe_kernel_name": (ctypes.c_char_p, [vp, i32]),
         "beam_moe_route_static": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
+        "beam_moe_debug_wait_timeout": (i32, [vp, i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -166,6 +167,10 @@ def beam_moe_last_launch_count(h) -> int:
 
 def beam_moe_destroy(h):
     _lib.beam_moe_destroy(h)
+
+
+def beam_moe_debug_wait_timeout(h, limit_ns: int, stream=None):
+    _check(_lib.beam_moe_debug_wait_timeout(h, int(limit_ns), _stream(stream)), "beam_moe_debug_wait_timeout")
 
 
 def beam_moe_profile_enable(h, enable: bool = True):

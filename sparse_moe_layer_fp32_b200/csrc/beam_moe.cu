@@ -20,7 +20,8 @@ struct beam_moe_ctx {
   int num_sms;
   // weights (owned, repacked)
   float* router_w;
-  uint8_t *w_gu, *w_gu_sf, *w_d, *w_d_sf;
+  uint16_t* router_w3;  // BF16 split of router_w, tiled for the tensor-core router
+  uint8_t *w_gu_tiles, *w_d_tiles;  // contiguous GEMM weight tiles (codes + scales)
   float *w_gu_alpha, *w_d_alpha;
   uint16_t* gamma;
   // workspace
@@ -32,9 +33,10 @@ struct beam_moe_ctx {
   uint8_t *a1, *a1_sf, *a2, *a2_sf;
   uint16_t* y;
   uint32_t* err;
+  unsigned int* route_counter;  // last-CTA election of the fused small-batch routing kernel
   uint16_t *stage_x, *stage_res, *stage_out;
-  CUtensorMap map_a1, map_wgu, map_a2, map_wd;
   int last_T;
+  int last_splits;  // logits layout of the last forward: [splits][T][E] partial sums
   int last_launches;
   std::vector<void*> allocs;
   // optional per-kernel timing
@@ -71,16 +73,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D byte tensor [rows][row_bytes]; boxes of 128 bytes x box_rows, 128-byte swizzle.
-bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+// 2-D BF16 tensor [rows][cols]; boxes of 32 values (64 bytes) x box_rows, 64-byte swizzle.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {row_bytes, rows};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {128, box_rows};
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -110,6 +112,19 @@ int64_t route_ws_floats(int T, int H, int E) {
 }
 
 __global__ void store_f32_kernel(float* p, float v) { *p = v; }
+
+// One CTA waits, with the kernels' bounded wait, on an mbarrier that nothing will complete.
+__global__ void wait_timeout_probe_kernel(uint64_t limit_ns, uint32_t* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns)) atomicOr(err, kErrTimeoutMma);
+}
 
 // Kernels use 16-byte vector accesses on these pointers.
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -150,7 +165,7 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   beam_moe_status st = check_shape(cfg->hidden, cfg->num_experts, cfg->top_k);
   if (st != BEAM_MOE_OK) return st;
   if (cfg->inter <= 0) return BEAM_MOE_ERR_INVALID_ARG;
-  if (cfg->inter % 128 != 0) return BEAM_MOE_ERR_UNSUPPORTED;
+  if (cfg->inter % 128 != 0 || cfg->hidden > 16384) return BEAM_MOE_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(cfg->max_tokens) * cfg->top_k > (1ll << 30)) return BEAM_MOE_ERR_UNSUPPORTED;
   if (!tensor_map_encoder()) return BEAM_MOE_ERR_CUDA;
 
@@ -167,6 +182,7 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   h->nblk_max = (h->Rmax + 127) / 128 + h->E;
   h->n_chunks_max = (h->Tmax + kChunkTokens - 1) / kChunkTokens;
   h->last_T = 0;
+  h->last_splits = 1;
   h->last_launches = 0;
   h->profiling = false;
   h->profiled_last = false;
@@ -195,19 +211,21 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
 
   // ---- weights
   CREATE_TRY(dalloc(h, &h->router_w, sizeof(float) * E * H));
-  CREATE_TRY(dalloc(h, &h->w_gu, static_cast<size_t>(E) * 2 * I * (H / 2)));
-  CREATE_TRY(dalloc(h, &h->w_gu_sf, static_cast<size_t>(E) * 2 * I * (H / 16)));
-  CREATE_TRY(dalloc(h, &h->w_d, static_cast<size_t>(E) * H * (Ip / 2)));
-  CREATE_TRY(dalloc(h, &h->w_d_sf, static_cast<size_t>(E) * H * (Ip / 16)));
+  CREATE_TRY(dalloc(h, &h->router_w3, sizeof(uint16_t) * 3 * E * H));
+  const size_t gu_tiles = static_cast<size_t>(E) * (2 * I / 256) * (H / 256);
+  const size_t d_tiles = static_cast<size_t>(E) * (H / 256) * (Ip / 256);
+  CREATE_TRY(dalloc(h, &h->w_gu_tiles, gu_tiles * kTileBytes));
+  CREATE_TRY(dalloc(h, &h->w_d_tiles, d_tiles * kTileBytes));
   CREATE_TRY(dalloc(h, &h->w_gu_alpha, sizeof(float) * E));
   CREATE_TRY(dalloc(h, &h->w_d_alpha, sizeof(float) * E));
   CREATE_TRY(dalloc(h, &h->gamma, sizeof(uint16_t) * H));
   CREATE_TRY(cudaMemcpyAsync(h->router_w, wts->router_w, sizeof(float) * E * H, cudaMemcpyDeviceToDevice, s));
+  CREATE_TRY(launch_split_router(h->router_w, E, H, h->router_w3, s));
   CREATE_TRY(cudaMemcpyAsync(h->w_gu_alpha, wts->w_gu_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
   CREATE_TRY(cudaMemcpyAsync(h->w_d_alpha, wts->w_d_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
   CREATE_TRY(cudaMemcpyAsync(h->gamma, wts->gamma, sizeof(uint16_t) * H, cudaMemcpyDeviceToDevice, s));
-  CREATE_TRY(launch_repack_gate_up(wts->w_gu, wts->w_gu_sf, E, I, H, h->w_gu, h->w_gu_sf, s));
-  CREATE_TRY(launch_repack_down(wts->w_d, wts->w_d_sf, E, I, Ip, H, h->w_d, h->w_d_sf, s));
+  CREATE_TRY(launch_repack_tiles(wts->w_gu, wts->w_gu_sf, E, 2 * I, H, H, I, h->w_gu_tiles, s));
+  CREATE_TRY(launch_repack_tiles(wts->w_d, wts->w_d_sf, E, H, I, Ip, 0, h->w_d_tiles, s));
 
   // ---- workspace
   int64_t lf = 0;
@@ -226,28 +244,25 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   CREATE_TRY(dalloc(h, &h->mblocks, sizeof(MBlock) * h->nblk_max));
   CREATE_TRY(dalloc(h, &h->perm, sizeof(int32_t) * R));
   CREATE_TRY(dalloc(h, &h->inv, sizeof(int32_t) * R));
-  CREATE_TRY(dalloc(h, &h->a1, static_cast<size_t>(R) * (H / 2)));
+  CREATE_TRY(dalloc(h, &h->a1, static_cast<size_t>(h->nblk_max) * (H / 2) * 128));
   CREATE_TRY(dalloc(h, &h->a1_sf, static_cast<size_t>(h->nblk_max) * (H / 64) * 512));
-  CREATE_TRY(dalloc(h, &h->a2, static_cast<size_t>(R) * (Ip / 2)));
+  CREATE_TRY(dalloc(h, &h->a2, static_cast<size_t>(h->nblk_max) * (Ip / 2) * 128));
   CREATE_TRY(dalloc(h, &h->a2_sf, static_cast<size_t>(h->nblk_max) * (Ip / 64) * 512));
   CREATE_TRY(dalloc(h, &h->y, sizeof(uint16_t) * static_cast<size_t>(R) * H));
   CREATE_TRY(dalloc(h, &h->err, sizeof(uint32_t)));
+  CREATE_TRY(dalloc(h, &h->route_counter, sizeof(unsigned int)));
+  CREATE_TRY(cudaMemsetAsync(h->route_counter, 0, sizeof(unsigned int), s));
   CREATE_TRY(dalloc(h, &h->stage_x, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   CREATE_TRY(dalloc(h, &h->stage_res, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   CREATE_TRY(dalloc(h, &h->stage_out, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   // The SwiGLU outputs beyond I (when I is not a multiple of 256) are never written: their
   // codes and scales must read as zero in the down GEMM.  Scale blocks of unused rows are
   // also defined this way.
-  CREATE_TRY(cudaMemsetAsync(h->a2, 0, static_cast<size_t>(R) * (Ip / 2), s));
+  CREATE_TRY(cudaMemsetAsync(h->a2, 0, static_cast<size_t>(h->nblk_max) * (Ip / 2) * 128, s));
   CREATE_TRY(cudaMemsetAsync(h->a2_sf, 0, static_cast<size_t>(h->nblk_max) * (Ip / 64) * 512, s));
   CREATE_TRY(cudaMemsetAsync(h->a1_sf, 0, static_cast<size_t>(h->nblk_max) * (H / 64) * 512, s));
   CREATE_TRY(cudaMemsetAsync(h->err, 0, sizeof(uint32_t), s));
 
-  if (!make_map_u8(&h->map_a1, h->a1, H / 2, R, 128) || !make_map_u8(&h->map_wgu, h->w_gu, H / 2,
-                                                                       static_cast<uint64_t>(E) * 2 * I, 256) ||
-      !make_map_u8(&h->map_a2, h->a2, Ip / 2, R, 128) ||
-      !make_map_u8(&h->map_wd, h->w_d, Ip / 2, static_cast<uint64_t>(E) * H, 256))
-    return fail(cudaErrorInvalidValue);
   CREATE_TRY(cudaStreamSynchronize(s));
   CREATE_TRY(cudaGetLastError());
 #undef CREATE_TRY
@@ -297,22 +312,42 @@ beam_moe_status beam_moe_forward(beam_moe_t h, const void* x, const void* residu
     return cudaEventRecord(h->events[launches + 1], s);
   };
   if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
-  BEAM_TRY(launch_router_logits(xb, h->router_w, T, H, E, h->logits, s));
-  BEAM_TRY(mark("router"));
-  ++launches;
-  BEAM_TRY(launch_topk(h->logits, router_split_count(T, H, E), T, E, k, h->ids, h->w, s));
-  BEAM_TRY(mark("topk"));
-  ++launches;
-  BEAM_TRY(launch_chunk_hist(h->ids, T, k, E, h->chunk_counts, s));
-  BEAM_TRY(mark("chunk_hist"));
-  ++launches;
-  BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
-                       h->num_mblocks, s));
-  BEAM_TRY(mark("scan"));
-  ++launches;
-  BEAM_TRY(launch_scatter(h->ids, h->chunk_base, T, k, E, h->perm, h->inv, s));
-  BEAM_TRY(mark("scatter"));
-  ++launches;
+  if (route_small_supported(T, H, E, k)) {
+    // router + top-k + histogram + scan + permutation in one launch
+    BEAM_TRY(launch_route_small(xb, h->router_w, T, H, E, k, h->logits, h->ids, h->w, h->offsets, h->sf_block,
+                                h->mblocks, h->num_mblocks, h->perm, h->inv, h->route_counter, s));
+    BEAM_TRY(mark("route_small"));
+    ++launches;
+    h->last_splits = 1;
+  } else {
+    if (router_tc_supported(T, H, E, k)) {
+      // FP32-class logits on the tensor cores (BF16 x 3-part split), top-k in the epilogue
+      CUtensorMap map_x;
+      if (!make_map_bf16(&map_x, xb, H, T, 128)) return BEAM_MOE_ERR_CUDA;
+      BEAM_TRY(launch_router_tc(map_x, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s));
+      BEAM_TRY(mark("router_tc"));
+      ++launches;
+      h->last_splits = 1;
+    } else {
+      BEAM_TRY(launch_router_logits(xb, h->router_w, T, H, E, h->logits, s));
+      BEAM_TRY(mark("router"));
+      ++launches;
+      h->last_splits = router_split_count(T, H, E);
+      BEAM_TRY(launch_topk(h->logits, h->last_splits, T, E, k, h->ids, h->w, s));
+      BEAM_TRY(mark("topk"));
+      ++launches;
+    }
+    BEAM_TRY(launch_chunk_hist(h->ids, T, k, E, h->chunk_counts, s));
+    BEAM_TRY(mark("chunk_hist"));
+    ++launches;
+    BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
+                         h->num_mblocks, s));
+    BEAM_TRY(mark("scan"));
+    ++launches;
+    BEAM_TRY(launch_scatter(h->ids, h->chunk_base, T, k, E, h->perm, h->inv, s));
+    BEAM_TRY(mark("scatter"));
+    ++launches;
+  }
   BEAM_TRY(launch_quant_a1(xb, h->ids, h->inv, h->offsets, h->sf_block, T, H, k, h->cfg.alpha_a1, h->a1,
                            h->a1_sf, s));
   BEAM_TRY(mark("quant_a1"));
@@ -321,34 +356,35 @@ beam_moe_status beam_moe_forward(beam_moe_t h, const void* x, const void* residu
   GemmArgs g{};
   g.mblocks = h->mblocks;
   g.num_mblocks = h->num_mblocks;
+  g.max_rows_per_expert = T;  // a token chooses an expert at most once
   g.err = h->err;
   // gate/up: 256 B rows per tile = 128 gate + 128 up features
   g.n_tiles = h->I / 128;
   g.k_tiles = H / 256;
-  g.n_rows_b = 2 * h->I;
+  g.a_tiles = h->a1;
+  g.b_tiles = h->w_gu_tiles;
   g.sfa = h->a1_sf;
-  g.sfb = h->w_gu_sf;
   g.alpha_b = h->w_gu_alpha;
   g.alpha_a = h->cfg.alpha_a1;
   g.a2 = h->a2;
   g.a2_sf = h->a2_sf;
-  g.a2_row_bytes = h->Ip / 2;
+  g.a2_k_tiles = h->Ip / 256;
   g.a2_kgroups = h->Ip / 64;
   g.alpha_a2 = h->cfg.alpha_a2;
-  BEAM_TRY(launch_gemm_gate_up(h->map_a1, h->map_wgu, g, h->num_sms, s));
+  BEAM_TRY(launch_gemm_gate_up(g, h->num_sms, s));
   BEAM_TRY(mark("gemm_gate_up"));
   ++launches;
   // down
   g.n_tiles = H / 256;
   g.k_tiles = h->Ip / 256;
-  g.n_rows_b = H;
+  g.a_tiles = h->a2;
+  g.b_tiles = h->w_d_tiles;
   g.sfa = h->a2_sf;
-  g.sfb = h->w_d_sf;
   g.alpha_b = h->w_d_alpha;
   g.alpha_a = h->cfg.alpha_a2;
   g.y = h->y;
   g.y_cols = H;
-  BEAM_TRY(launch_gemm_down(h->map_a2, h->map_wd, g, h->num_sms, s));
+  BEAM_TRY(launch_gemm_down(g, h->num_sms, s));
   BEAM_TRY(mark("gemm_down"));
   ++launches;
   BEAM_TRY(launch_finalize(h->y, h->w, h->inv, static_cast<const uint16_t*>(residual), h->gamma, T, H, k,
@@ -407,16 +443,16 @@ beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, void* dst, size
   const void* src = nullptr;
   size_t n = 0;
   switch (which) {
-    case BEAM_MOE_BUF_LOGITS: src = h->logits; n = sizeof(float) * route_ws_floats(static_cast<int>(T), h->H, h->E); break;
+    case BEAM_MOE_BUF_LOGITS: src = h->logits; n = sizeof(float) * h->last_splits * T * h->E; break;
     case BEAM_MOE_BUF_IDS: src = h->ids; n = sizeof(int32_t) * R; break;
     case BEAM_MOE_BUF_WEIGHTS: src = h->w; n = sizeof(float) * R; break;
     case BEAM_MOE_BUF_OFFSETS: src = h->offsets; n = sizeof(int32_t) * (h->E + 1); break;
     case BEAM_MOE_BUF_PERM: src = h->perm; n = sizeof(int32_t) * R; break;
     case BEAM_MOE_BUF_INV: src = h->inv; n = sizeof(int32_t) * R; break;
     case BEAM_MOE_BUF_SFBLOCK: src = h->sf_block; n = sizeof(int32_t) * (h->E + 1); break;
-    case BEAM_MOE_BUF_A1: src = h->a1; n = static_cast<size_t>(R) * (h->H / 2); break;
+    case BEAM_MOE_BUF_A1: src = h->a1; n = static_cast<size_t>(h->nblk_max) * (h->H / 2) * 128; break;
     case BEAM_MOE_BUF_A1_SF: src = h->a1_sf; n = static_cast<size_t>(h->nblk_max) * (h->H / 64) * 512; break;
-    case BEAM_MOE_BUF_A2: src = h->a2; n = static_cast<size_t>(R) * (h->Ip / 2); break;
+    case BEAM_MOE_BUF_A2: src = h->a2; n = static_cast<size_t>(h->nblk_max) * (h->Ip / 2) * 128; break;
     case BEAM_MOE_BUF_A2_SF: src = h->a2_sf; n = static_cast<size_t>(h->nblk_max) * (h->Ip / 64) * 512; break;
     case BEAM_MOE_BUF_Y: src = h->y; n = sizeof(uint16_t) * static_cast<size_t>(R) * h->H; break;
     default: return BEAM_MOE_ERR_INVALID_ARG;
@@ -441,6 +477,13 @@ beam_moe_status beam_moe_check(beam_moe_t h, void* stream) {
 }
 
 int32_t beam_moe_last_launch_count(beam_moe_t h) { return h ? h->last_launches : 0; }
+
+beam_moe_status beam_moe_debug_wait_timeout(beam_moe_t h, int64_t limit_ns, void* stream) {
+  if (!h || limit_ns <= 0 || limit_ns > static_cast<int64_t>(kWaitLimitNs)) return BEAM_MOE_ERR_INVALID_ARG;
+  wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns), h->err);
+  BEAM_TRY(cudaGetLastError());
+  return BEAM_MOE_OK;
+}
 
 beam_moe_status beam_moe_profile_enable(beam_moe_t h, int32_t enable) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;

@@ -31,6 +31,31 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while the previous
+// kernel in the stream is still running.  pdl_wait() blocks until that kernel has finished
+// and its memory is visible (a no-op for a normal launch); every kernel of the forward
+// calls it before touching memory that another kernel of the stream writes or reads.
+// pdl_trigger() lets the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -58,14 +83,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Waits for the phase with parity `parity` of `bar`.  Returns false (and sets *abort)
 // when the wait ran past kWaitLimitNs or another role already aborted.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         return false;
       }
@@ -88,6 +114,15 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(smem_dst)),
                "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+// Asks L2 to fetch a contiguous range (16-byte aligned, bytes % 16 == 0); no completion.
+__device__ __forceinline__ void prefetch_l2(const void* gsrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes) : "memory");
+}
+// Same for one box of a 2-D tensor map.
+__device__ __forceinline__ void prefetch_l2_tile(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
                : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -168,6 +203,16 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   d |= static_cast<uint64_t>(2u) << 61;                // 128-byte swizzle
   return d;
 }
+// Same for the 64-byte swizzle: rows of 64 bytes, 8-row groups 512 bytes apart, type 4.
+__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(512u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(4u) << 61;
+  return d;
+}
 // Descriptor of a 32-row x 16-byte source for tcgen05.cp: 8-row core matrices of
 // contiguous 16-byte rows, 128 bytes apart, no swizzle.
 __device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr) {
@@ -223,6 +268,15 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float al
   return sc;
 }
 
+// Activation tiles: the codes of each 128-row block are stored as K/256 tiles of 128 rows x
+// 128 bytes (256 values), row m at m * 128 and its 16-byte chunk c at ((c ^ (m % 8)) * 16):
+// the 128-byte swizzle the tensor core reads, so a tile (or its first rows) is one
+// contiguous copy.  Byte offset of 16-byte chunk c of row m of tile (block, kt):
+__device__ __forceinline__ size_t act_tile_offset(size_t block, int k_tiles, int kt, int m, int c) {
+  return (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(kt)) * 16384u +
+         static_cast<size_t>(m * 128 + ((c ^ (m & 7)) << 4));
+}
+
 // Byte offset of scale s of row m (0..127) in a 128-row scale block with K/64 groups.
 __device__ __forceinline__ size_t sf_atom_offset(size_t block, int kgroups, int m, int s) {
   return (block * static_cast<size_t>(kgroups) + static_cast<size_t>(s >> 2)) * 512u +
@@ -230,5 +284,35 @@ __device__ __forceinline__ size_t sf_atom_offset(size_t block, int kgroups, int 
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Exclusive prefix sum of one int per thread over the whole CTA (blockDim.x <= 1024, a
+// multiple of 32); *total gets the sum.  warp_sums: 33 ints of shared memory.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += u;
+  }
+  if (lane == 31) warp_sums[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < nwarps ? warp_sums[lane] : 0;
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += u;
+    }
+    if (lane < nwarps) warp_sums[lane] = si - s;  // exclusive prefix of warp totals
+    if (lane == 31) warp_sums[32] = si;           // grand total
+  }
+  __syncthreads();
+  total = warp_sums[32];
+  const int r = warp_sums[warp] + inc - v;
+  __syncthreads();
+  return r;
+}
 
 }  // namespace beam

@@ -29,7 +29,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 constexpr int kFinThreads = 128;
 
-__global__ void __launch_bounds__(kFinThreads) finalize_kernel(const uint16_t* __restrict__ y,
+// Large batches: CTAs of 128 threads, several chunks per thread, the weighted sums kept in
+// shared memory until the RMS is known; many CTAs per SM hide the gather latency.
+__global__ void __launch_bounds__(kFinThreads) finalize_wide_kernel(const uint16_t* __restrict__ y,
                                                                const float* __restrict__ w,
                                                                const int32_t* __restrict__ inv,
                                                                const uint16_t* residual,
@@ -40,6 +42,8 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(const uint16_t* _
   __shared__ float s_w[16];
   __shared__ float s_red[kFinThreads / 32];
   const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x < k) {
     s_row[threadIdx.x] = inv[static_cast<size_t>(t) * k + threadIdx.x];
     s_w[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
@@ -49,13 +53,20 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(const uint16_t* _
   float ss = 0.0f;
   for (int c = threadIdx.x; c < nchunks; c += kFinThreads) {
     float acc[8] = {};
-    for (int j = 0; j < k; ++j) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j]) * H) + c);
-      float f[8];
-      unpack8(v, f);
-      const float wj = s_w[j];
+    for (int j0 = 0; j0 < k; j0 += 4) {
+      uint4 yv[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+      for (int j = 0; j < 4; ++j)
+        if (j0 + j < k) yv[j] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j0 + j]) * H) + c);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (j0 + j >= k) break;
+        float f[8];
+        unpack8(yv[j], f);
+        const float wj = s_w[j0 + j];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+      }
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -86,16 +97,94 @@ __global__ void __launch_bounds__(kFinThreads) finalize_kernel(const uint16_t* _
   }
 }
 
+// Small batches: one CTA per token, CPT 16-byte chunks (8 values) per thread kept in
+// registers, the k row gathers of a thread issued together, one block reduction.
+template <int CPT>
+__global__ void __launch_bounds__(1024) finalize_kernel(const uint16_t* __restrict__ y, const float* __restrict__ w,
+                                                        const int32_t* __restrict__ inv, const uint16_t* residual,
+                                                        const uint16_t* __restrict__ gamma, int H, int k, float eps,
+                                                        uint16_t* out) {
+  __shared__ int s_row[16];
+  __shared__ float s_w[16];
+  __shared__ float s_red[32];
+  const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x < k) {
+    s_row[threadIdx.x] = inv[static_cast<size_t>(t) * k + threadIdx.x];
+    s_w[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
+  }
+  __syncthreads();
+  const int nchunks = H / 8;
+  float acc[CPT][8];
+  float ss = 0.0f;
+#pragma unroll
+  for (int q = 0; q < CPT; ++q) {
+    const int c = threadIdx.x + q * blockDim.x;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[q][i] = 0.0f;
+    if (c < nchunks) {
+      for (int j0 = 0; j0 < k; j0 += 8) {
+        uint4 yv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)  // up to 8 row gathers in flight together
+          if (j0 + j < k) yv[j] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j0 + j]) * H) + c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j0 + j >= k) break;
+          float f[8];
+          unpack8(yv[j], f);
+          const float wj = s_w[j0 + j];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[q][i] = fmaf(wj, f[i], acc[q][i]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(acc[q][i], acc[q][i], ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.0f;
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) tot += s_red[i];
+  const float rinv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+#pragma unroll
+  for (int q = 0; q < CPT; ++q) {
+    const int c = threadIdx.x + q * blockDim.x;
+    if (c >= nchunks) continue;
+    float r[8], g[8];
+    unpack8(reinterpret_cast<const uint4*>(residual + static_cast<size_t>(t) * H)[c], r);  // out may alias residual
+    unpack8(__ldg(reinterpret_cast<const uint4*>(gamma) + c), g);
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = pack_bf16x2(r[2 * i] + acc[q][2 * i] * rinv * g[2 * i], r[2 * i + 1] + acc[q][2 * i + 1] * rinv * g[2 * i + 1]);
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
                             const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(H) * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e =
-        cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
+  const int nchunks = H / 8;
+  if (T >= 256) {
+    const size_t smem = static_cast<size_t>(H) * sizeof(float);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(finalize_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(finalize_wide_kernel, dim3(T), dim3(kFinThreads), smem, s, y, w, inv, residual, gamma, H, k, eps,
+                      out);
   }
-  finalize_kernel<<<T, kFinThreads, smem, s>>>(y, w, inv, residual, gamma, H, k, eps, out);
-  return cudaGetLastError();
+  if (nchunks <= 1024) {
+    const int threads = ((nchunks + 31) / 32) * 32;
+    return launch_pdl(finalize_kernel<1>, dim3(T), dim3(threads), 0, s, y, w, inv, residual, gamma, H, k, eps, out);
+  }
+  if (nchunks <= 2048)
+    return launch_pdl(finalize_kernel<2>, dim3(T), dim3(1024), 0, s, y, w, inv, residual, gamma, H, k, eps, out);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace beam

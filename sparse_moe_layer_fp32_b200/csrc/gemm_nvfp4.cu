@@ -8,9 +8,12 @@
 //   down:    D[r][n] = A2[r] . Wd[e][n],   K = I; epilogue y = bf16(D * scale)
 //
 // Design (one persistent CTA per SM, 320 threads, warp-specialised):
-//   warp 0      TMA producer: per 256-wide K step, a 128x256 A tile (16 KB), a 256x256 B
-//               tile (32 KB), and the matching E4M3 scale blocks (2 KB + 4 KB, plain bulk
-//               copies) into a 4-stage shared-memory ring, all landing on one mbarrier.
+//   warp 0      producer: per 256-wide K step, bulk copies of the A tile (the valid rows
+//               of a 128-row activation tile, <= 16 KB), the expert's weight tile with its
+//               scales (32 KB + 4 KB) and the A scales (2 KB) into a 4-stage shared-memory
+//               ring, all landing on one mbarrier.  Activations and weights are both stored
+//               as contiguous tiles already in the swizzled shared-memory order, so every
+//               load is one sequential copy.
 //   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scales -> TMEM) and
 //               tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128, N=256, K=64) into a
 //               128x256 FP32 accumulator in TMEM, and tcgen05.commit to free stages.
@@ -29,12 +32,25 @@ namespace beam {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK_BYTES = 128;  // 256 FP4 values per K step (one 128-byte swizzle row)
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK_BYTES;      // 16384
-constexpr int B_BYTES = BN * BK_BYTES;      // 32768
-constexpr int SFA_BYTES = 4 * 512;          // 4 K-groups of 64 values x 128 rows
-constexpr int SFB_BYTES = 2 * 4 * 512;      // 2 row blocks of 128
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 55296 (multiple of 1024)
+constexpr int A_TILE_BYTES = BM * BK_BYTES;  // 16384: one activation tile in global memory
+constexpr int B_BYTES = BN * BK_BYTES;       // 32768
+constexpr int SFA_BYTES = 4 * 512;           // 4 K-groups of 64 values x 128 rows
+constexpr int SFB_BYTES = 2 * 4 * 512;       // 2 row blocks of 128
+static_assert(B_BYTES + SFB_BYTES == kTileBytes, "weight tile = B codes + B scales");
+// Two ring shapes.  Stage layout: A | B | SFB | SFA (B and SFB are one contiguous weight
+// tile).  Full: A holds 128 rows, 4 stages.  Small-M (batches of <= 32 tokens, so every
+// expert has <= 32 rows): A holds 32 rows, which leaves room for a 5th stage of weights in
+// flight.  The MMA still reads 128 rows of A; rows past the region read the stage's B bytes
+// and only feed accumulator rows that are never stored.
+template <int kStages, int kABytes>
+struct Ring {
+  static constexpr int STAGES = kStages;
+  static constexpr int A_BYTES = kABytes;
+  static constexpr int STAGE_BYTES = kABytes + B_BYTES + SFB_BYTES + SFA_BYTES;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for the swizzle");
+};
+using RingFull = Ring<4, A_TILE_BYTES>;
+using RingSmallM = Ring<5, 32 * BK_BYTES>;
 constexpr int NUM_THREADS = 320;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
@@ -48,9 +64,10 @@ constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((
 
 enum Epilogue { kSwiGLU = 0, kStoreBF16 = 1 };
 
+constexpr int kMaxStages = 5;
 struct __align__(8) GemmSmemTail {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
@@ -58,7 +75,11 @@ struct __align__(8) GemmSmemTail {
   int abort_flag;
 };
 
-size_t gemm_smem_bytes() { return static_cast<size_t>(STAGES) * STAGE_BYTES + sizeof(GemmSmemTail) + 1024; }
+template <class R>
+static size_t ring_smem_bytes() {
+  return static_cast<size_t>(R::STAGES) * R::STAGE_BYTES + sizeof(GemmSmemTail) + 1024;
+}
+size_t gemm_smem_bytes() { return ring_smem_bytes<RingFull>(); }
 
 __device__ __forceinline__ float silu_times(float g, float u) { return __fdiv_rn(g, 1.0f + expf(-g)) * u; }
 
@@ -67,10 +88,10 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int EPI>
+template <int EPI, class R>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                      const GemmArgs args) {
+    gemm_nvfp4_kernel(const GemmArgs args) {
+  constexpr int STAGES = R::STAGES, A_BYTES = R::A_BYTES, STAGE_BYTES = R::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmSmemTail* tail = reinterpret_cast<GemmSmemTail*>(smem + STAGES * STAGE_BYTES);
@@ -96,6 +117,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tail->tmem_base;
+  pdl_wait();  // the previous kernel's outputs (block list, activations) are complete
+  pdl_trigger();
 
   const int n_tiles = args.n_tiles, k_tiles = args.k_tiles;
   const int kgroups = k_tiles * 4;
@@ -104,8 +127,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      prefetch_tmap(&map_a);
-      prefetch_tmap(&map_b);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;
@@ -113,10 +134,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const MBlock mb = args.mblocks[tile / n_tiles];
         const int nt = tile % n_tiles;
-        const int b_row = mb.expert * args.n_rows_b + nt * BN;
         const uint8_t* sfa = args.sfa + (static_cast<size_t>(mb.sf_block) * kgroups) * 512;
-        const uint8_t* sfb0 =
-            args.sfb + (static_cast<size_t>(mb.expert) * (args.n_rows_b / 128) + nt * 2) * kgroups * 512;
+        const uint8_t* btile =
+            args.b_tiles + (static_cast<size_t>(mb.expert) * n_tiles + nt) * k_tiles * static_cast<size_t>(kTileBytes);
         for (int kt = 0; kt < k_tiles; ++kt) {
           if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1, abort_flag)) {
             ok = false;
@@ -124,17 +144,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           uint8_t* sa = smem + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
-          uint8_t* ssfa = sb + B_BYTES;
-          uint8_t* ssfb = ssfa + SFA_BYTES;
-          mbar_arrive_expect_tx(&tail->full[stage], STAGE_BYTES);
+          uint8_t* ssfa = sb + B_BYTES + SFB_BYTES;
+          // rows past the block's valid rows are not copied: their stale shared-memory
+          // contents only reach accumulator rows that are never stored
+          uint32_t a_bytes = static_cast<uint32_t>(min(BM, (mb.rows + 7) & ~7)) * BK_BYTES;
+          if (a_bytes > static_cast<uint32_t>(A_BYTES)) {  // cannot happen when the host picks the ring right
+            atomicOr(args.err, kErrRange);
+            a_bytes = A_BYTES;
+          }
+          mbar_arrive_expect_tx(&tail->full[stage], a_bytes + kTileBytes + SFA_BYTES);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          tma_load_2d(sa, &map_a, &tail->full[stage], kt * BK_BYTES, mb.row_begin);
-          tma_load_2d(sb, &map_b, &tail->full[stage], kt * BK_BYTES, b_row);
+          bulk_load(sa, args.a_tiles + (static_cast<size_t>(mb.sf_block) * k_tiles + kt) * A_TILE_BYTES, a_bytes,
+                    &tail->full[stage]);
+          bulk_load(sb, btile + static_cast<size_t>(kt) * kTileBytes, kTileBytes, &tail->full[stage]);
           bulk_load(ssfa, sfa + static_cast<size_t>(kt) * 4 * 512, SFA_BYTES, &tail->full[stage]);
-          bulk_load(ssfb, sfb0 + static_cast<size_t>(kt) * 4 * 512, SFA_BYTES, &tail->full[stage]);
-          bulk_load(ssfb + SFA_BYTES, sfb0 + static_cast<size_t>(kgroups) * 512 + static_cast<size_t>(kt) * 4 * 512,
-                    SFA_BYTES, &tail->full[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -166,8 +190,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t ssfa = sb + B_BYTES;
-          const uint32_t ssfb = ssfa + SFA_BYTES;
+          const uint32_t ssfb = sb + B_BYTES;
+          const uint32_t ssfa = ssfb + SFB_BYTES;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             tc_cp_32x128b_x4(tmem + SFA_COL + kb * 4, sdesc_sf(ssfa + kb * 512));
@@ -224,12 +248,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc_phase ^= 1;
       if (row_in_tile >= mb.rows) continue;
       const size_t r = static_cast<size_t>(mb.row_begin + row_in_tile);
+      (void)r;
       const float scale = args.alpha_a * __ldg(args.alpha_b + mb.expert);
       if constexpr (EPI == kSwiGLU) {
         const float alpha2 = args.alpha_a2;
         const float six_alpha2 = __fmul_rn(6.0f, alpha2);
         const int f0 = nt * 128 + half * 64;  // first feature of this thread's 64
-        uint8_t* dst = args.a2 + r * args.a2_row_bytes + f0 / 2;
+        uint32_t codes[8];
         uint32_t scodes = 0;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
@@ -241,11 +266,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float u = __uint_as_float(v[2 + (c >> 5)][c & 31]) * scale;
             h[i] = silu_times(g, u);
           }
-          uint32_t lo, hi;
-          const uint32_t sc = quant_block16(h, alpha2, six_alpha2, lo, hi);
-          *reinterpret_cast<uint2*>(dst + b * 8) = make_uint2(lo, hi);
+          const uint32_t sc = quant_block16(h, alpha2, six_alpha2, codes[2 * b], codes[2 * b + 1]);
           scodes |= sc << (8 * b);
         }
+        // 64 features = 32 bytes = 16-byte chunks c0, c0 + 1 of K tile f0 / 256 of the A2 tile
+        const int a2_kt = f0 >> 8, c0 = (f0 & 255) >> 5;
+        *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.a2_k_tiles, a2_kt, row_in_tile, c0)) =
+            make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.a2_k_tiles, a2_kt, row_in_tile, c0 + 1)) =
+            make_uint4(codes[4], codes[5], codes[6], codes[7]);
         // the 4 scales of this K-group (features f0..f0+63) are 4 contiguous bytes
         *reinterpret_cast<uint32_t*>(args.a2_sf + sf_atom_offset(mb.sf_block, args.a2_kgroups, row_in_tile,
                                                                  f0 / 16)) = scodes;
@@ -272,24 +301,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-template <int EPI>
-static cudaError_t launch_gemm(const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& a, int grid,
-                               cudaStream_t s) {
-  const size_t smem = gemm_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int EPI, class R>
+static cudaError_t launch_ring(const GemmArgs& a, int grid, cudaStream_t s) {
+  const size_t smem = ring_smem_bytes<R>();
+  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<EPI, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  gemm_nvfp4_kernel<EPI><<<grid, NUM_THREADS, smem, s>>>(map_a, map_b, a);
-  return cudaGetLastError();
+  return launch_pdl(gemm_nvfp4_kernel<EPI, R>, dim3(grid), dim3(NUM_THREADS), smem, s, a);
 }
 
-cudaError_t launch_gemm_gate_up(const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& a, int grid,
-                                cudaStream_t s) {
-  return launch_gemm<kSwiGLU>(map_a, map_b, a, grid, s);
+template <int EPI>
+static cudaError_t launch_gemm(const GemmArgs& a, int grid, cudaStream_t s) {
+  // With at most 32 tokens no expert has more than 32 rows.
+  if (a.max_rows_per_expert <= 32) return launch_ring<EPI, RingSmallM>(a, grid, s);
+  return launch_ring<EPI, RingFull>(a, grid, s);
 }
-cudaError_t launch_gemm_down(const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& a, int grid,
-                             cudaStream_t s) {
-  return launch_gemm<kStoreBF16>(map_a, map_b, a, grid, s);
-}
+
+cudaError_t launch_gemm_gate_up(const GemmArgs& a, int grid, cudaStream_t s) { return launch_gemm<kSwiGLU>(a, grid, s); }
+cudaError_t launch_gemm_down(const GemmArgs& a, int grid, cudaStream_t s) { return launch_gemm<kStoreBF16>(a, grid, s); }
 
 }  // namespace beam

@@ -26,6 +26,23 @@ int router_split_count(int T, int H, int E);
 cudaError_t launch_topk(const float* logits, int splits, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t s);
 
+// ---- router on the tensor cores for large batches (router_tc.cu)
+constexpr int kRouterTcMinTokens = 1024;
+bool router_tc_supported(int T, int H, int E, int k);
+size_t router_tc_smem_bytes(int E);
+cudaError_t launch_split_router(const float* w, int E, int H, uint16_t* out, cudaStream_t s);
+// map_x: x [T][H] BF16, boxes 32 x 128 with the 64-byte swizzle; w_tiles: the split router
+// weights from launch_split_router.  Writes logits [T][E], ids / w [T][k].
+cudaError_t launch_router_tc(const CUtensorMap& map_x, const uint16_t* w_tiles, int T, int H, int E, int k,
+                             float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s);
+
+// ---- routing of a small batch in one launch (route_small.cu)
+bool route_small_supported(int T, int H, int E, int k);
+cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, int E, int k, float* logits,
+                               int32_t* ids, float* wout, int32_t* offsets, int32_t* sf_block, MBlock* mblocks,
+                               int32_t* num_mblocks, int32_t* perm, int32_t* inv, unsigned int* done_counter,
+                               cudaStream_t s);
+
 // ---- permutation and activation quantisation (routing.cu)
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s);
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
@@ -37,33 +54,35 @@ cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* ids, const int32_t
                             cudaStream_t s);
 
 // ---- weight quantiser and repacking (quant.cu)
+// Contiguous weight tiles of the grouped GEMMs: 256 rows x 256 K values of codes in the
+// swizzled shared-memory order, then their scales (see repack_tiles_kernel).
+constexpr int kTileCodeBytes = 256 * 128;
+constexpr int kTileSfBytes = 2 * 4 * 512;
+constexpr int kTileBytes = kTileCodeBytes + kTileSfBytes;  // 36864
+// rows_per_e % 256 == 0; K = logical contraction size, Kp = K rounded up to 256 (zero pad).
+// interleave_inter != 0: gate/up rows, interleaved per 128 features (inter = I).
+cudaError_t launch_repack_tiles(const uint8_t* codes, const uint8_t* sf, int E, int rows_per_e, int K, int Kp,
+                                int interleave_inter, uint8_t* dst, cudaStream_t s);
 cudaError_t launch_quantize_rows(const float* src, int64_t rows, int64_t cols, float alpha, const float* alpha_dev,
                                  uint8_t* codes, uint8_t* sf, cudaStream_t s);
 cudaError_t launch_amax(const float* src, int64_t n, float* amax_bits, cudaStream_t s);
 cudaError_t launch_amax_to_alpha(float* inout, cudaStream_t s);
-// Gate/up: codes [E][2I][H/2] -> rows interleaved per 128-feature block (gate block then
-// up block); scales -> 128-row scale blocks [E][2I/128][H/64][512].
-cudaError_t launch_repack_gate_up(const uint8_t* codes, const uint8_t* sf, int E, int I, int H, uint8_t* codes_out,
-                                  uint8_t* sf_out, cudaStream_t s);
-// Down: codes [E][H][I/2] -> [E][H][Ip/2] (zero padded), scales -> [E][H/128][Ip/64][512].
-cudaError_t launch_repack_down(const uint8_t* codes, const uint8_t* sf, int E, int I, int Ip, int H,
-                               uint8_t* codes_out, uint8_t* sf_out, cudaStream_t s);
-
 // ---- grouped NVFP4 GEMMs (gemm_nvfp4.cu)
 struct GemmArgs {
   const MBlock* mblocks;
   const int32_t* num_mblocks;
+  int max_rows_per_expert;  // an upper bound (the number of tokens) used to pick the ring shape
   int n_tiles;        // output tiles of 256 columns per 128-row block
   int k_tiles;        // K / 256
-  int n_rows_b;       // rows of B per expert
+  const uint8_t* a_tiles;  // activation tiles [blk][k_tiles][16384] (act_tile_offset)
+  const uint8_t* b_tiles;  // weight tiles [E][n_tiles][k_tiles][kTileBytes]
   const uint8_t* sfa; // activation scale blocks [blk][K/64][512]
-  const uint8_t* sfb; // weight scale blocks [E][n_rows_b/128][K/64][512]
   const float* alpha_b;  // [E]
   float alpha_a;
   // gate/up epilogue: SwiGLU + NVFP4 of h
-  uint8_t* a2;        // [rows][Ip/2]
+  uint8_t* a2;        // activation tiles [blk][Ip/256][16384]
   uint8_t* a2_sf;     // [blk][Ip/64][512]
-  int a2_row_bytes;   // Ip/2
+  int a2_k_tiles;     // Ip/256
   int a2_kgroups;     // Ip/64
   float alpha_a2;
   // down epilogue: BF16 rows
@@ -71,10 +90,8 @@ struct GemmArgs {
   int y_cols;         // H
   uint32_t* err;
 };
-cudaError_t launch_gemm_gate_up(const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& a, int grid,
-                                cudaStream_t s);
-cudaError_t launch_gemm_down(const CUtensorMap& map_a, const CUtensorMap& map_b, const GemmArgs& a, int grid,
-                             cudaStream_t s);
+cudaError_t launch_gemm_gate_up(const GemmArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_gemm_down(const GemmArgs& a, int grid, cudaStream_t s);
 size_t gemm_smem_bytes();
 
 // ---- finalize (finalize.cu)

@@ -82,47 +82,59 @@ cudaError_t launch_quantize_rows(const float* src, int64_t rows, int64_t cols, f
 // Gate/up rows are interleaved per 128-feature block b: rows [256b, 256b+128) are gate
 // features [128b, 128b+128) and rows [256b+128, 256b+256) the matching up features, so
 // one 256-row B tile gives an epilogue thread both halves of SwiGLU for 128 features.
+// Returns the source row (rows 0..I-1 gate, I..2I-1 up) of interleaved row lr.
 __device__ __forceinline__ int gate_up_src_row(int lr, int I) {
   const int fb = lr >> 8, g = (lr >> 7) & 1, i = lr & 127;
   return g * I + fb * 128 + i;
 }
 
-__global__ void repack_rows_kernel(const uint8_t* __restrict__ src, int E, int rows_per_e, int src_bytes,
-                                   int dst_bytes, int interleave_inter, uint8_t* __restrict__ dst) {
-  // one thread per 16 bytes of destination
-  const int64_t chunks_per_row = dst_bytes / 16;
-  const int64_t total = static_cast<int64_t>(E) * rows_per_e * chunks_per_row;
+// Weights as contiguous B tiles for the grouped GEMMs.  Tile (e, nt, kt) covers rows
+// [256 nt, 256 nt + 256) of expert e (after the gate/up interleave) and K values
+// [256 kt, 256 kt + 256): kTileCodeBytes of codes laid out exactly as the tensor core
+// reads them from shared memory (row r at r * 128, 16-byte chunk c of the row at
+// ((c ^ (r % 8)) * 16): the 128-byte swizzle), then kTileSfBytes of scales (two 128-row
+// blocks, each 4 K-groups x 512 bytes in the tcgen05 scale-factor layout).  One bulk copy
+// moves a whole tile.
+__global__ void repack_tiles_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, int E,
+                                    int rows_per_e, int K, int Kp, int interleave_inter, uint8_t* __restrict__ dst) {
+  const int n_tiles = rows_per_e / 256, k_tiles = Kp / 256;
+  constexpr int kChunks = kTileBytes / 16;  // 16-byte chunks per tile
+  const int64_t total = static_cast<int64_t>(E) * n_tiles * k_tiles * kChunks;
+  const int src_row_bytes = K / 2, src_scales = K / 16;
   for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < total;
        q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = q / chunks_per_row;
-    const int c = static_cast<int>(q % chunks_per_row);
-    const int e = static_cast<int>(row / rows_per_e), lr = static_cast<int>(row % rows_per_e);
-    const int slr = interleave_inter ? gate_up_src_row(lr, interleave_inter) : lr;
+    const int64_t tile = q / kChunks;
+    const int o = static_cast<int>(q % kChunks) * 16;  // byte offset in the tile
+    const int kt = static_cast<int>(tile % k_tiles);
+    const int nt = static_cast<int>((tile / k_tiles) % n_tiles);
+    const int e = static_cast<int>(tile / (static_cast<int64_t>(k_tiles) * n_tiles));
     uint4 v = make_uint4(0, 0, 0, 0);
-    if (c * 16 < src_bytes)
-      v = *reinterpret_cast<const uint4*>(src + (static_cast<int64_t>(e) * rows_per_e + slr) * src_bytes + c * 16);
-    *reinterpret_cast<uint4*>(dst + row * dst_bytes + c * 16) = v;
-  }
-}
-
-// Scale bytes [E][rows][src_scales] -> 128-row scale blocks [E][rows/128][kgroups][512].
-__global__ void repack_sf_kernel(const uint8_t* __restrict__ src, int E, int rows_per_e, int src_scales,
-                                 int kgroups, int interleave_inter, uint8_t* __restrict__ dst) {
-  const int64_t total = static_cast<int64_t>(E) * (rows_per_e / 128) * kgroups * 512;
-  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < total;
-       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int o = static_cast<int>(q & 511);
-    const int64_t blk_k = q >> 9;
-    const int kg = static_cast<int>(blk_k % kgroups);
-    const int64_t blk = blk_k / kgroups;  // global block index = e * (rows/128) + rb
-    const int e = static_cast<int>(blk / (rows_per_e / 128)), rb = static_cast<int>(blk % (rows_per_e / 128));
-    const int m = (o >> 4) + 32 * ((o & 15) >> 2);
-    const int sidx = kg * 4 + (o & 3);
-    const int lr = rb * 128 + m;
-    const int slr = interleave_inter ? gate_up_src_row(lr, interleave_inter) : lr;
-    uint8_t v = 0;
-    if (sidx < src_scales) v = src[(static_cast<int64_t>(e) * rows_per_e + slr) * src_scales + sidx];
-    dst[q] = v;
+    if (o < kTileCodeBytes) {
+      // shared-memory slot (o >> 4) & 7 of row r holds logical 16-byte chunk slot ^ (r % 8)
+      const int r = o >> 7, c = ((o >> 4) & 7) ^ (r & 7);
+      const int lr = nt * 256 + r;
+      const int slr = interleave_inter ? gate_up_src_row(lr, interleave_inter) : lr;
+      const int byte = kt * 128 + c * 16;  // K/2 is a multiple of 64: a chunk is all in or all out
+      if (byte < src_row_bytes)
+        v = *reinterpret_cast<const uint4*>(codes + (static_cast<int64_t>(e) * rows_per_e + slr) * src_row_bytes + byte);
+    } else {
+      uint8_t b[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int so = o - kTileCodeBytes + i;
+        const int nb = so >> 11, kb = (so >> 9) & 3, a = so & 511;
+        const int m = (a >> 4) + 32 * ((a & 15) >> 2);
+        const int sidx = (kt * 4 + kb) * 4 + (a & 3);
+        const int lr = nt * 256 + nb * 128 + m;
+        const int slr = interleave_inter ? gate_up_src_row(lr, interleave_inter) : lr;
+        b[i] = sidx < src_scales ? sf[(static_cast<int64_t>(e) * rows_per_e + slr) * src_scales + sidx] : 0;
+      }
+      v.x = b[0] | (b[1] << 8) | (b[2] << 16) | (static_cast<uint32_t>(b[3]) << 24);
+      v.y = b[4] | (b[5] << 8) | (b[6] << 16) | (static_cast<uint32_t>(b[7]) << 24);
+      v.z = b[8] | (b[9] << 8) | (b[10] << 16) | (static_cast<uint32_t>(b[11]) << 24);
+      v.w = b[12] | (b[13] << 8) | (b[14] << 16) | (static_cast<uint32_t>(b[15]) << 24);
+    }
+    *reinterpret_cast<uint4*>(dst + tile * kTileBytes + o) = v;
   }
 }
 
@@ -131,26 +143,10 @@ static int grid_for(int64_t work) {
   return static_cast<int>(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
 }
 
-cudaError_t launch_repack_gate_up(const uint8_t* codes, const uint8_t* sf, int E, int I, int H, uint8_t* codes_out,
-                                  uint8_t* sf_out, cudaStream_t s) {
-  const int rows = 2 * I;
-  repack_rows_kernel<<<grid_for(static_cast<int64_t>(E) * rows * (H / 32)), 256, 0, s>>>(codes, E, rows, H / 2,
-                                                                                        H / 2, I, codes_out);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  repack_sf_kernel<<<grid_for(static_cast<int64_t>(E) * rows * (H / 16)), 256, 0, s>>>(sf, E, rows, H / 16, H / 64,
-                                                                                      I, sf_out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_repack_down(const uint8_t* codes, const uint8_t* sf, int E, int I, int Ip, int H,
-                               uint8_t* codes_out, uint8_t* sf_out, cudaStream_t s) {
-  repack_rows_kernel<<<grid_for(static_cast<int64_t>(E) * H * (Ip / 32)), 256, 0, s>>>(codes, E, H, I / 2, Ip / 2,
-                                                                                      0, codes_out);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  repack_sf_kernel<<<grid_for(static_cast<int64_t>(E) * H * (Ip / 16)), 256, 0, s>>>(sf, E, H, I / 16, Ip / 64, 0,
-                                                                                    sf_out);
+cudaError_t launch_repack_tiles(const uint8_t* codes, const uint8_t* sf, int E, int rows_per_e, int K, int Kp,
+                                int interleave_inter, uint8_t* dst, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(E) * (rows_per_e / 256) * (Kp / 256) * (kTileBytes / 16);
+  repack_tiles_kernel<<<grid_for(total), 256, 0, s>>>(codes, sf, E, rows_per_e, K, Kp, interleave_inter, dst);
   return cudaGetLastError();
 }
 

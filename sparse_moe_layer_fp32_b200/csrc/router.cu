@@ -18,6 +18,7 @@
 // chosen logits, so the 256-way sum is not needed.
 #include "common.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace beam {
 
@@ -72,6 +73,8 @@ __global__ void __launch_bounds__(256) router_sgemm_kernel(const uint16_t* __res
   __shared__ __align__(16) float As[RBK][RBM + 4];
   __shared__ __align__(16) float Bs[RBK][RBN + 4];
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const int m0 = blockIdx.y * RBM, n0 = blockIdx.x * RBN;
   const int split = blockIdx.z;
   const int kbeg = split * k_per_split, kend = kbeg + k_per_split;
@@ -144,8 +147,7 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* w, int T, int H
   }
   const int splits = router_split_count(T, H, E);
   dim3 grid((E + RBN - 1) / RBN, (T + RBM - 1) / RBM, splits);
-  router_sgemm_kernel<<<grid, 256, 0, s>>>(x, w, T, H, E, H / splits, logits);
-  return cudaGetLastError();
+  return launch_pdl(router_sgemm_kernel, grid, dim3(256), 0, s, x, w, T, H, E, H / splits, logits);
 }
 
 // ------------------------------------------------------------------ top-k
@@ -154,6 +156,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
                                                    int32_t* __restrict__ ids, float* __restrict__ wout) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
   if (t >= T) return;
   float v[EPL];
 #pragma unroll
@@ -166,56 +170,19 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
     }
     v[i] = a;
   }
-  uint32_t taken = 0;
-  float sel_v[16];
-  int sel_e[16];
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (!((taken >> i) & 1u) && e < E && (v[i] > bv || (v[i] == bv && e < be))) {
-        bv = v[i];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    sel_v[j] = bv;
-    sel_e[j] = be;
-  }
-  // renormalised weights = softmax over the chosen logits (sel_v[0] is the largest)
-  float z[16], sum = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    z[j] = expf(sel_v[j] - sel_v[0]);
-    sum += z[j];
-  }
-  for (int j = lane; j < k; j += 32) {
-    ids[static_cast<size_t>(t) * k + j] = sel_e[j];
-    wout[static_cast<size_t>(t) * k + j] = z[j] / sum;
-  }
+  warp_topk<EPL>(v, E, k, lane, ids + static_cast<size_t>(t) * k, wout + static_cast<size_t>(t) * k);
 }
 
 cudaError_t launch_topk(const float* logits, int splits, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t s) {
   const int blocks = (T + 7) / 8;
   const int epl = (E + 31) / 32;
-  if (epl <= 1) topk_kernel<1><<<blocks, 256, 0, s>>>(logits, splits, T, E, k, ids, w);
-  else if (epl <= 2) topk_kernel<2><<<blocks, 256, 0, s>>>(logits, splits, T, E, k, ids, w);
-  else if (epl <= 4) topk_kernel<4><<<blocks, 256, 0, s>>>(logits, splits, T, E, k, ids, w);
-  else if (epl <= 8) topk_kernel<8><<<blocks, 256, 0, s>>>(logits, splits, T, E, k, ids, w);
-  else if (epl <= 16) topk_kernel<16><<<blocks, 256, 0, s>>>(logits, splits, T, E, k, ids, w);
-  else topk_kernel<32><<<blocks, 256, 0, s>>>(logits, splits, T, E, k, ids, w);
-  return cudaGetLastError();
+  if (epl <= 1) return launch_pdl(topk_kernel<1>, dim3(blocks), dim3(256), 0, s, logits, splits, T, E, k, ids, w);
+  if (epl <= 2) return launch_pdl(topk_kernel<2>, dim3(blocks), dim3(256), 0, s, logits, splits, T, E, k, ids, w);
+  if (epl <= 4) return launch_pdl(topk_kernel<4>, dim3(blocks), dim3(256), 0, s, logits, splits, T, E, k, ids, w);
+  if (epl <= 8) return launch_pdl(topk_kernel<8>, dim3(blocks), dim3(256), 0, s, logits, splits, T, E, k, ids, w);
+  if (epl <= 16) return launch_pdl(topk_kernel<16>, dim3(blocks), dim3(256), 0, s, logits, splits, T, E, k, ids, w);
+  return launch_pdl(topk_kernel<32>, dim3(blocks), dim3(256), 0, s, logits, splits, T, E, k, ids, w);
 }
 
 }  // namespace beam

@@ -11,7 +11,8 @@
 //
 // A1 = Q(x, alpha_a1): x rows are quantised once per token (16-value blocks along H) and
 // the codes are written to the token's k permuted rows (the NVFP4 W4A4 experts of the
-// recipe "reflection/Beam-1.0-501B-A23B", section "Variants").
+// recipe "reflection/Beam-1.0-501B-A23B", section "Variants"), as activation tiles (see
+// act_tile_offset) of the row's 128-row block.
 #include "common.cuh"
 #include "internal.h"
 
@@ -21,6 +22,8 @@ namespace beam {
 __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
                                                          int32_t* __restrict__ chunk_counts) {
   extern __shared__ int32_t cnt[];
+  pdl_wait();
+  pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   const int t0 = blockIdx.x * kChunkTokens;
@@ -33,40 +36,14 @@ __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restri
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
 }
 
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  int inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += u;
-  }
-  if (lane == 31) warp_sums[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    int s = lane < nwarps ? warp_sums[lane] : 0;
-    int si = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, si, o);
-      if (lane >= o) si += u;
-    }
-    if (lane < nwarps) warp_sums[lane] = si - s;  // exclusive prefix of warp totals
-    if (lane == 31) warp_sums[32] = si;           // grand total
-  }
-  __syncthreads();
-  total = warp_sums[32];
-  const int r = warp_sums[warp] + inc - v;
-  __syncthreads();
-  return r;
-}
-
 // One CTA, one thread per expert.
 __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chunks, int E,
                             int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
                             int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks,
                             int32_t* __restrict__ num_mblocks) {
   __shared__ int warp_sums[33];
+  pdl_wait();
+  pdl_trigger();
   const int e = threadIdx.x;
   int cnt = 0;
   if (e < E) {
@@ -109,6 +86,8 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
   uint32_t* mask = sm;                                    // [8][E]
   int32_t* pre = reinterpret_cast<int32_t*>(sm + 8 * E);  // [8][E]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) mask[i] = 0;
   __syncthreads();
   const int chunk = blockIdx.x;
@@ -137,24 +116,81 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
   }
 }
 
-// One warp per token: quantise x[t] once, write it to the token's k permuted rows.
-__global__ void __launch_bounds__(256) quant_a1_kernel(const uint16_t* __restrict__ x,
+// One thread per 16-value block of x: quantise it once and write it to the token's k
+// permuted rows.  The four threads of one 64-value group (one scale word of the
+// tensor-core layout) combine their scale bytes and one of them stores the 32-bit word.
+__global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restrict__ x,
                                                        const int32_t* __restrict__ ids,
                                                        const int32_t* __restrict__ inv,
                                                        const int32_t* __restrict__ offsets,
                                                        const int32_t* __restrict__ sf_block, int T, int H, int k,
                                                        float alpha, uint8_t* __restrict__ a1,
                                                        uint8_t* __restrict__ a1_sf) {
-  __shared__ int s_r[8][16], s_blk[8][16], s_m[8][16];
+  const int nb = H / 16, kgroups = H / 64;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const bool active = gid < static_cast<int64_t>(T) * nb;
+  const int t = active ? static_cast<int>(gid / nb) : 0;
+  const int b = active ? static_cast<int>(gid % nb) : 0;
+  pdl_wait();
+  pdl_trigger();
+  uint32_t lo = 0, hi = 0, sc = 0;
+  int r[16], e[16];
+  if (active) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+    const uint4 p0 = __ldg(xr + 2 * b), p1 = __ldg(xr + 2 * b + 1);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)  // all slot indices in flight together
+      if (j < k) {
+        r[j] = __ldg(inv + static_cast<size_t>(t) * k + j);
+        e[j] = __ldg(ids + static_cast<size_t>(t) * k + j);
+      }
+    const uint32_t u[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = bf16_bits_to_f32(u[i] & 0xFFFFu);
+      v[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+    }
+    sc = quant_block16(v, alpha, __fmul_rn(6.0f, alpha), lo, hi);
+  }
+  // lanes 4q..4q+3 hold blocks 4g..4g+3 of one token (nb is a multiple of 4)
+  const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc, 1);
+  const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
+  const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
+  const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  if (!active) return;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j >= k) break;
+    const int li = r[j] - __ldg(offsets + e[j]);
+    const int blk = __ldg(sf_block + e[j]) + (li >> 7), m = li & 127;
+    // block b of 16 values: 8 bytes, half of 16-byte chunk (b % 16) / 2 of K tile b / 16
+    *reinterpret_cast<uint2*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1) + (b & 1) * 8) =
+        make_uint2(lo, hi);
+    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, kgroups, m, b)) = word;
+  }
+}
+
+// Large batches: one warp per token, quantise x[t] once, write it to the token's k rows.
+__global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __restrict__ x,
+                                                       const int32_t* __restrict__ ids,
+                                                       const int32_t* __restrict__ inv,
+                                                       const int32_t* __restrict__ offsets,
+                                                       const int32_t* __restrict__ sf_block, int T, int H, int k,
+                                                       float alpha, uint8_t* __restrict__ a1,
+                                                       uint8_t* __restrict__ a1_sf) {
+  __shared__ int s_blk[8][16], s_m[8][16];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * 8 + warp;
+  pdl_wait();
+  pdl_trigger();
   if (t >= T) return;
   // lane j < k: the permuted row of slot j and where its scales live
   if (lane < k) {
     const int r = inv[static_cast<size_t>(t) * k + lane];
     const int e = ids[static_cast<size_t>(t) * k + lane];
     const int li = r - offsets[e];
-    s_r[warp][lane] = r;
     s_blk[warp][lane] = sf_block[e] + (li >> 7);
     s_m[warp][lane] = li & 127;
   }
@@ -174,8 +210,9 @@ __global__ void __launch_bounds__(256) quant_a1_kernel(const uint16_t* __restric
     uint32_t lo, hi;
     const uint32_t sc = quant_block16(v, alpha, six_alpha, lo, hi);
     for (int j = 0; j < k; ++j) {
-      const int r = s_r[warp][j], blk = s_blk[warp][j], m = s_m[warp][j];
-      *reinterpret_cast<uint2*>(a1 + static_cast<size_t>(r) * (H / 2) + b * 8) = make_uint2(lo, hi);
+      const int blk = s_blk[warp][j], m = s_m[warp][j];
+      *reinterpret_cast<uint2*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1) + (b & 1) * 8) =
+          make_uint2(lo, hi);
       a1_sf[sf_atom_offset(blk, kgroups, m, b)] = static_cast<uint8_t>(sc);
     }
   }
@@ -183,15 +220,15 @@ __global__ void __launch_bounds__(256) quant_a1_kernel(const uint16_t* __restric
 
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s) {
   const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
-  chunk_hist_kernel<<<n_chunks, 256, E * sizeof(int32_t), s>>>(ids, T, k, E, chunk_counts);
-  return cudaGetLastError();
+  return launch_pdl(chunk_hist_kernel, dim3(n_chunks), dim3(256), E * sizeof(int32_t), s, ids, T, k, E,
+                    chunk_counts);
 }
 
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
-  scan_kernel<<<1, threads, 0, s>>>(chunk_counts, n_chunks, E, chunk_base, offsets, sf_block, mblocks, num_mblocks);
-  return cudaGetLastError();
+  return launch_pdl(scan_kernel, dim3(1), dim3(threads), 0, s, chunk_counts, n_chunks, E, chunk_base, offsets,
+                    sf_block, mblocks, num_mblocks);
 }
 
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, int T, int k, int E, int32_t* perm_src,
@@ -203,15 +240,18 @@ cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, int T,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  scatter_kernel<<<n_chunks, 256, smem, s>>>(ids, chunk_base, T, k, E, perm_src, inv);
-  return cudaGetLastError();
+  return launch_pdl(scatter_kernel, dim3(n_chunks), dim3(256), smem, s, ids, chunk_base, T, k, E, perm_src, inv);
 }
 
 cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* ids, const int32_t* inv, const int32_t* offsets,
                             const int32_t* sf_block, int T, int H, int k, float alpha, uint8_t* a1, uint8_t* a1_sf,
                             cudaStream_t s) {
-  quant_a1_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, ids, inv, offsets, sf_block, T, H, k, alpha, a1, a1_sf);
-  return cudaGetLastError();
+  if (T >= 256)
+    return launch_pdl(quant_a1_wide_kernel, dim3((T + 7) / 8), dim3(256), 0, s, x, ids, inv, offsets, sf_block, T, H,
+                      k, alpha, a1, a1_sf);
+  const int64_t threads = static_cast<int64_t>(T) * (H / 16);
+  return launch_pdl(quant_a1_kernel, dim3(static_cast<unsigned>((threads + 127) / 128)), dim3(128), 0, s, x, ids, inv,
+                    offsets, sf_block, T, H, k, alpha, a1, a1_sf);
 }
 
 }  // namespace beam

@@ -46,6 +46,26 @@ def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols
     return out
 
 
+def tile_rows(tiles: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int) -> np.ndarray:
+    """Activation tiles (beam_moe.h layout) -> packed codes [rows, kcols/2] in permuted row order."""
+    experts = len(offsets) - 1
+    rows = int(offsets[-1])
+    k_tiles = kcols // 256
+    out = np.zeros((rows, kcols // 2), np.uint8)
+    j = np.arange(kcols // 2)
+    for e in range(experts):
+        n = int(offsets[e + 1] - offsets[e])
+        if n == 0:
+            continue
+        i = np.arange(n)
+        blk = (sf_block[e] + i // 128)[:, None]
+        m = (i % 128)[:, None]
+        off = ((blk * k_tiles + j[None, :] // 128) * 16384 + m * 128 + ((((j[None, :] % 128) // 16) ^ (m % 8)) * 16)
+               + j[None, :] % 16)
+        out[offsets[e]:offsets[e + 1]] = tiles[off]
+    return out
+
+
 def norm_zero(packed: np.ndarray) -> np.ndarray:
     """Map the E2M1 negative zero (code 8) to +0 in packed bytes (+-0 are equal values)."""
     c = nvfp4.unpack_nibbles(packed)

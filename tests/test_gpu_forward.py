@@ -25,7 +25,7 @@ pytestmark = pytest.mark.gpu
 import moe_inputs as mi  # noqa: E402
 from oracle import moe, nvfp4  # noqa: E402
 from tests.gpu_util import (ABS_MAX, REL_L2, bf16_to_f64, buf, compare_outputs, ids_match, norm_zero,  # noqa: E402
-                            oracle_layer_inputs, sf_rows, to_np)
+                            oracle_layer_inputs, sf_rows, tile_rows, to_np)
 
 
 @pytest.fixture(scope="module")
@@ -87,13 +87,13 @@ def test_forward_stages_and_end_to_end(bm, name, tokens, seed):
     nblk = np.array([(c + 127) // 128 for c in pm["counts"]])
     np.testing.assert_array_equal(sfb, np.concatenate([[0], np.cumsum(nblk)]))
     # ---- A1: bit-exact
-    a1p = buf(layer, bm.BUF_A1, np.uint8).reshape(T * k, H // 2)
+    a1p = tile_rows(buf(layer, bm.BUF_A1, np.uint8), sfb, offsets, H)
     a1s = sf_rows(buf(layer, bm.BUF_A1_SF, np.uint8), sfb, offsets, H)
     rp, rs = nvfp4.quantize_nvfp4(x[perm].astype(np.float32), a1)
     np.testing.assert_array_equal(a1s, rs)
     np.testing.assert_array_equal(norm_zero(a1p), norm_zero(rp))
     # ---- A2 and y from the GPU's own inputs
-    a2p = buf(layer, bm.BUF_A2, np.uint8).reshape(T * k, Ip // 2)[:, : I // 2]
+    a2p = tile_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, Ip)[:, : I // 2]
     a2s = sf_rows(buf(layer, bm.BUF_A2_SF, np.uint8), sfb, offsets, Ip)[:, : I // 16]
     y = to_np(layer.debug(bm.BUF_Y).view(torch.bfloat16).float()).reshape(T * k, H).astype(np.float64)
     mism, n_codes = 0, 0
@@ -151,4 +151,28 @@ def test_forward_edge_cases(bm):
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
     layer.check()
+    layer.close()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(bm):
+    # Failure detection without a GPU fault: a wait that nothing completes gives up after
+    # 50 ms, the error word says TIMEOUT, and the next forward still runs correctly.
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(SHAPES["tiny"], tokens=4)
+    weights = synthetic.make_weights(shape, 0, threads=2)
+    layer = bm.MoELayer(max_tokens=4, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                        inter=shape.inter, alpha_a1=0.0012, alpha_a2=0.00012, **weights)
+    x, r = synthetic.make_batch(shape, 0)
+    before = layer.forward(x, r)
+    layer.check()
+    bm.beam_moe_debug_wait_timeout(layer.handle, 50_000_000)
+    with pytest.raises(bm.BeamMoeError) as ei:
+        layer.check()
+    assert ei.value.status == bm.ERR_TIMEOUT
+    layer.check()  # the error word was cleared by the check that reported it
+    after = layer.forward(x, r)
+    layer.check()
+    assert torch.equal(before, after)
+    with pytest.raises(bm.BeamMoeError):
+        bm.beam_moe_debug_wait_timeout(layer.handle, 0)
     layer.close()
