@@ -100,6 +100,16 @@ BEAM_MOE_API beam_moe_status beam_moe_create(const beam_moe_config* cfg, const b
 BEAM_MOE_API beam_moe_status beam_moe_forward(beam_moe_t h, const void* x, const void* residual, void* out, int32_t num_tokens,
                                  void* stream);
 
+/* beam_moe_forward fused with the next sublayer's sandwich pre-norm (the PR's sandwich
+ * norms fused with the MoE finalize): besides out, writes
+ *   next_x[T][H] = bf16( out / sqrt(mean(out^2) + next_eps) * next_gamma ),
+ * computed from the BF16 out values.  next_gamma: [H] BF16 device pointer (the next
+ * sublayer's pre-norm weight); next_x must not alias x, residual or out.  Same errors as
+ * beam_moe_forward. */
+BEAM_MOE_API beam_moe_status beam_moe_forward_prenorm(beam_moe_t h, const void* x, const void* residual, void* out,
+                                                      void* next_x, const void* next_gamma, float next_eps,
+                                                      int32_t num_tokens, void* stream);
+
 /* Same as beam_moe_forward with HOST buffers: copies x and residual to the handle's
  * device staging buffers, runs the forward, copies out back, all enqueued on `stream`
  * (cudaMemcpyAsync; pinned host memory makes the copies asynchronous).  The caller

@@ -48,6 +48,7 @@ from .moe import (  # noqa: F401
     permute,
     expert_forward,
     finalize,
+    next_prenorm,
     moe_forward,
     moe_forward_tokens,
 )

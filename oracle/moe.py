@@ -162,6 +162,19 @@ def finalize(y_sel: np.ndarray, w: np.ndarray, residual: np.ndarray, gamma: np.n
     return pre, bf16_round(pre), m
 
 
+def next_prenorm(out_bf16: np.ndarray, gamma_next: np.ndarray, eps: float):
+    """The next sublayer's sandwich pre-norm on the updated residual stream ([PR] "Status":
+    Beam's sandwich norms; "Remaining work": fused with the MoE finalize).
+
+    out_bf16: the layer output as it leaves the layer (BF16 values, as FP64) [T, H].
+    Returns (pre-rounding FP64, BF16-rounded as FP64) of out / sqrt(mean(out^2) + eps) * gamma_next.
+    Reading: the norm reads the BF16 residual the next layer receives, not the FP32 sum.
+    """
+    o = np.asarray(out_bf16, np.float64)
+    pre = o / np.sqrt(np.mean(o * o, axis=1, keepdims=True) + eps) * np.asarray(gamma_next, np.float64)[None, :]
+    return pre, bf16_round(pre)
+
+
 # ----------------------------------------------------------------------------- forward
 class ExpertCache:
     """Quantises (with this oracle's quantiser) and dequantises experts on first use.

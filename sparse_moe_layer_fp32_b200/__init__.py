@@ -25,6 +25,7 @@ EXPORTED = [
     "beam_moe_route_workspace_bytes", "beam_moe_quantize_nvfp4", "beam_moe_debug_copy", "beam_moe_check",
     "beam_moe_last_launch_count", "beam_moe_status_string", "beam_moe_destroy", "beam_moe_profile_enable",
     "beam_moe_profile_read", "beam_moe_kernel_name", "beam_moe_route_static", "beam_moe_debug_wait_timeout",
+    "beam_moe_forward_prenorm",
 ]
 
 
@@ -69,6 +70,7 @@ def _load():
         "beam_moe_kernel_name": (ctypes.c_char_p, [vp, i32]),
         "beam_moe_route_static": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
         "beam_moe_debug_wait_timeout": (i32, [vp, i64, vp]),
+        "beam_moe_forward_prenorm": (i32, [vp, vp, vp, vp, vp, vp, f32, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -113,6 +115,12 @@ def beam_moe_create(cfg: BeamMoeConfig, weights: BeamMoeWeights, stream=None) ->
 def beam_moe_forward(h, x, residual, out, num_tokens: int, stream=None):
     _check(_lib.beam_moe_forward(h, _ptr(x), _ptr(residual), _ptr(out), int(num_tokens), _stream(stream)),
            "beam_moe_forward")
+
+
+def beam_moe_forward_prenorm(h, x, residual, out, next_x, next_gamma, next_eps: float, num_tokens: int, stream=None):
+    _check(_lib.beam_moe_forward_prenorm(h, _ptr(x), _ptr(residual), _ptr(out), _ptr(next_x), _ptr(next_gamma),
+                                         ctypes.c_float(next_eps), int(num_tokens), _stream(stream)),
+           "beam_moe_forward_prenorm")
 
 
 def beam_moe_forward_host(h, x_host, residual_host, out_host, num_tokens: int, stream=None):
@@ -202,6 +210,13 @@ class MoELayer:
         out = torch.empty_like(residual) if out is None else out
         beam_moe_forward(self.handle, x, residual, out, x.shape[0], stream)
         return out
+
+    def forward_prenorm(self, x, residual, next_gamma, next_eps=1e-6, out=None, next_x=None, stream=None):
+        """(out, next_x): the layer output and the next sublayer's pre-normed input."""
+        out = torch.empty_like(residual) if out is None else out
+        next_x = torch.empty_like(residual) if next_x is None else next_x
+        beam_moe_forward_prenorm(self.handle, x, residual, out, next_x, next_gamma, next_eps, x.shape[0], stream)
+        return out, next_x
 
     def forward_host(self, x_host, residual_host, out_host, stream=None):
         beam_moe_forward_host(self.handle, x_host, residual_host, out_host, x_host.shape[0], stream)

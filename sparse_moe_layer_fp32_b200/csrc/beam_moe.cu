@@ -288,8 +288,8 @@ beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num
   return BEAM_MOE_OK;
 }
 
-beam_moe_status beam_moe_forward(beam_moe_t h, const void* x, const void* residual, void* out, int32_t num_tokens,
-                                 void* stream) {
+static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* residual, void* out, void* next_x,
+                                    const void* next_gamma, float next_eps, int32_t num_tokens, void* stream) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;
   if (num_tokens < 0 || num_tokens > h->Tmax) return BEAM_MOE_ERR_INVALID_ARG;
   if (num_tokens == 0) {
@@ -388,13 +388,30 @@ beam_moe_status beam_moe_forward(beam_moe_t h, const void* x, const void* residu
   BEAM_TRY(mark("gemm_down"));
   ++launches;
   BEAM_TRY(launch_finalize(h->y, h->w, h->inv, static_cast<const uint16_t*>(residual), h->gamma, T, H, k,
-                           h->cfg.rms_eps, static_cast<uint16_t*>(out), s));
+                           h->cfg.rms_eps, static_cast<uint16_t*>(out), static_cast<uint16_t*>(next_x),
+                           static_cast<const uint16_t*>(next_gamma), next_eps, s));
   BEAM_TRY(mark("finalize"));
   ++launches;
   h->last_T = T;
   h->last_launches = launches;
   h->profiled_last = prof;
   return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_forward(beam_moe_t h, const void* x, const void* residual, void* out, int32_t num_tokens,
+                                 void* stream) {
+  return forward_impl(h, x, residual, out, nullptr, nullptr, 0.0f, num_tokens, stream);
+}
+
+beam_moe_status beam_moe_forward_prenorm(beam_moe_t h, const void* x, const void* residual, void* out, void* next_x,
+                                         const void* next_gamma, float next_eps, int32_t num_tokens, void* stream) {
+  if (!h || num_tokens < 0) return BEAM_MOE_ERR_INVALID_ARG;
+  if (num_tokens > 0) {
+    if (!next_x || !next_gamma || !(next_eps >= 0.0f)) return BEAM_MOE_ERR_INVALID_ARG;
+    if (!aligned(next_x, 16) || !aligned(next_gamma, 16)) return BEAM_MOE_ERR_INVALID_ARG;
+    if (next_x == x || next_x == residual || next_x == out) return BEAM_MOE_ERR_INVALID_ARG;
+  }
+  return forward_impl(h, x, residual, out, next_x, next_gamma, next_eps, num_tokens, stream);
 }
 
 beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const void* residual_host, void* out_host,

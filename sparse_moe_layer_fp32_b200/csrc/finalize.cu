@@ -29,14 +29,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 constexpr int kFinThreads = 128;
 
+// The next sublayer's sandwich pre-norm, fused: x_next = bf16(out / sqrt(mean(out^2) + eps)
+// * gamma), out being the BF16 values just written.  Disabled when x == nullptr.
+struct NextNorm {
+  uint16_t* x;
+  const uint16_t* gamma;
+  float eps;
+};
+
+// 1 / sqrt(sum / H + eps) of a per-thread partial sum, over the CTA (blockDim % 32 == 0).
+__device__ __forceinline__ float block_rinv(float part, int H, float eps, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  __syncthreads();  // s_red may still be read from a previous reduction
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = part;
+  __syncthreads();
+  float tot = 0.0f;
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) tot += s_red[i];
+  return 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+}
+
 // Large batches: CTAs of 128 threads, several chunks per thread, the weighted sums kept in
 // shared memory until the RMS is known; many CTAs per SM hide the gather latency.
+template <bool PRE>
 __global__ void __launch_bounds__(kFinThreads) finalize_wide_kernel(const uint16_t* __restrict__ y,
                                                                const float* __restrict__ w,
                                                                const int32_t* __restrict__ inv,
                                                                const uint16_t* residual,
                                                                const uint16_t* __restrict__ gamma, int H, int k,
-                                                               float eps, uint16_t* out) {
+                                                               float eps, uint16_t* out, NextNorm nn) {
   extern __shared__ float m_s[];  // [H]
   __shared__ int s_row[16];
   __shared__ float s_w[16];
@@ -82,6 +103,7 @@ __global__ void __launch_bounds__(kFinThreads) finalize_wide_kernel(const uint16
 #pragma unroll
   for (int i = 0; i < kFinThreads / 32; ++i) tot += s_red[i];
   const float rinv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+  float ss2 = 0.0f;
   for (int c = threadIdx.x; c < nchunks; c += kFinThreads) {
     float r[8], g[8];
     unpack8(reinterpret_cast<const uint4*>(residual + static_cast<size_t>(t) * H)[c], r);  // out may alias residual
@@ -93,17 +115,39 @@ __global__ void __launch_bounds__(kFinThreads) finalize_wide_kernel(const uint16
       const float b = r[2 * i + 1] + m_s[c * 8 + 2 * i + 1] * rinv * g[2 * i + 1];
       o[i] = pack_bf16x2(a, b);
     }
-    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = ov;
+    if constexpr (PRE) {  // keep the BF16 output for the next sublayer's pre-norm
+      float f[8];
+      unpack8(ov, f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        m_s[c * 8 + i] = f[i];
+        ss2 = fmaf(f[i], f[i], ss2);
+      }
+    }
+  }
+  if constexpr (PRE) {
+    const float r2 = block_rinv(ss2, H, nn.eps, s_red);
+    for (int c = threadIdx.x; c < nchunks; c += kFinThreads) {
+      float g[8];
+      unpack8(__ldg(reinterpret_cast<const uint4*>(nn.gamma) + c), g);
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o[i] = pack_bf16x2(m_s[c * 8 + 2 * i] * r2 * g[2 * i], m_s[c * 8 + 2 * i + 1] * r2 * g[2 * i + 1]);
+      reinterpret_cast<uint4*>(nn.x + static_cast<size_t>(t) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
 // Small batches: one CTA per token, CPT 16-byte chunks (8 values) per thread kept in
 // registers, the k row gathers of a thread issued together, one block reduction.
-template <int CPT>
+template <int CPT, bool PRE>
 __global__ void __launch_bounds__(1024) finalize_kernel(const uint16_t* __restrict__ y, const float* __restrict__ w,
                                                         const int32_t* __restrict__ inv, const uint16_t* residual,
                                                         const uint16_t* __restrict__ gamma, int H, int k, float eps,
-                                                        uint16_t* out) {
+                                                        uint16_t* out, NextNorm nn) {
   __shared__ int s_row[16];
   __shared__ float s_w[16];
   __shared__ float s_red[32];
@@ -150,6 +194,7 @@ __global__ void __launch_bounds__(1024) finalize_kernel(const uint16_t* __restri
   float tot = 0.0f;
   for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) tot += s_red[i];
   const float rinv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
+  float ss2 = 0.0f;
 #pragma unroll
   for (int q = 0; q < CPT; ++q) {
     const int c = threadIdx.x + q * blockDim.x;
@@ -161,30 +206,62 @@ __global__ void __launch_bounds__(1024) finalize_kernel(const uint16_t* __restri
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       o[i] = pack_bf16x2(r[2 * i] + acc[q][2 * i] * rinv * g[2 * i], r[2 * i + 1] + acc[q][2 * i + 1] * rinv * g[2 * i + 1]);
-    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = ov;
+    if constexpr (PRE) {  // the next pre-norm reads the BF16 values just written
+      unpack8(ov, acc[q]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss2 = fmaf(acc[q][i], acc[q][i], ss2);
+    }
+  }
+  if constexpr (PRE) {
+    const float r2 = block_rinv(ss2, H, nn.eps, s_red);
+#pragma unroll
+    for (int q = 0; q < CPT; ++q) {
+      const int c = threadIdx.x + q * blockDim.x;
+      if (c >= nchunks) continue;
+      float g[8];
+      unpack8(__ldg(reinterpret_cast<const uint4*>(nn.gamma) + c), g);
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(acc[q][2 * i] * r2 * g[2 * i], acc[q][2 * i + 1] * r2 * g[2 * i + 1]);
+      reinterpret_cast<uint4*>(nn.x + static_cast<size_t>(t) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
-cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
-                            const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, cudaStream_t s) {
+template <bool PRE>
+static cudaError_t launch_finalize_t(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
+                                     const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out,
+                                     NextNorm nn, cudaStream_t s) {
   const int nchunks = H / 8;
   if (T >= 256) {
     const size_t smem = static_cast<size_t>(H) * sizeof(float);
     if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(finalize_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaError_t e = cudaFuncSetAttribute(finalize_wide_kernel<PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
       if (e != cudaSuccess) return e;
     }
-    return launch_pdl(finalize_wide_kernel, dim3(T), dim3(kFinThreads), smem, s, y, w, inv, residual, gamma, H, k, eps,
-                      out);
+    return launch_pdl(finalize_wide_kernel<PRE>, dim3(T), dim3(kFinThreads), smem, s, y, w, inv, residual, gamma, H, k,
+                      eps, out, nn);
   }
   if (nchunks <= 1024) {
     const int threads = ((nchunks + 31) / 32) * 32;
-    return launch_pdl(finalize_kernel<1>, dim3(T), dim3(threads), 0, s, y, w, inv, residual, gamma, H, k, eps, out);
+    return launch_pdl(finalize_kernel<1, PRE>, dim3(T), dim3(threads), 0, s, y, w, inv, residual, gamma, H, k, eps,
+                      out, nn);
   }
   if (nchunks <= 2048)
-    return launch_pdl(finalize_kernel<2>, dim3(T), dim3(1024), 0, s, y, w, inv, residual, gamma, H, k, eps, out);
+    return launch_pdl(finalize_kernel<2, PRE>, dim3(T), dim3(1024), 0, s, y, w, inv, residual, gamma, H, k, eps, out,
+                      nn);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
+                            const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, uint16_t* next_x,
+                            const uint16_t* next_gamma, float next_eps, cudaStream_t s) {
+  const NextNorm nn{next_x, next_gamma, next_eps};
+  if (next_x) return launch_finalize_t<true>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, s);
+  return launch_finalize_t<false>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, s);
 }
 
 }  // namespace beam

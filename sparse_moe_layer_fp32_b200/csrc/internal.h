@@ -95,7 +95,9 @@ cudaError_t launch_gemm_down(const GemmArgs& a, int grid, cudaStream_t s);
 size_t gemm_smem_bytes();
 
 // ---- finalize (finalize.cu)
+// next_x != nullptr also writes the next sublayer's pre-norm of out: bf16(out * rinv * next_gamma).
 cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
-                            const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, cudaStream_t s);
+                            const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, uint16_t* next_x,
+                            const uint16_t* next_gamma, float next_eps, cudaStream_t s);
 
 }  // namespace beam

@@ -176,3 +176,29 @@ def test_bounded_wait_reports_timeout_and_context_survives(bm):
     with pytest.raises(bm.BeamMoeError):
         bm.beam_moe_debug_wait_timeout(layer.handle, 0)
     layer.close()
+
+
+@pytest.mark.parametrize("name,tokens,seed", [("tiny", 5, 7), ("tiny", 300, 8), ("mid", 9, 9)])
+def test_forward_with_fused_next_prenorm(bm, name, tokens, seed):
+    # The next sublayer's sandwich pre-norm fused into the finalize: out is unchanged and
+    # next_x = bf16(RMSNorm(out) * gamma_next), checked on the GPU's own out (one BF16
+    # rounding apart) and end to end against the oracle.
+    shape, layer, weights, out_plain, ref, (x, res, wr, g, cache, a1, a2) = _run(bm, SHAPES[name], tokens, seed)
+    from sparse_moe_layer_fp32_b200 import synthetic
+    xd, rd = synthetic.make_batch(shape, seed)
+    g_next_bits = mi.gamma(dataclasses.replace(shape, name="next"), seed + 100)
+    g_next = synthetic.bf16_tensor(g_next_bits)
+    out, next_x = layer.forward_prenorm(xd, rd, g_next, 1e-6)
+    layer.check()
+    torch.cuda.synchronize()
+    assert torch.equal(out, out_plain)
+    gn = mi.bf16_bits_to_f32(g_next_bits).astype(np.float64)
+    pre, _ = moe.next_prenorm(bf16_to_f64(out), gn, 1e-6)
+    nx = bf16_to_f64(next_x)
+    assert np.all(np.abs(nx - pre) <= 2.0 ** -7 * np.maximum(np.abs(pre), 2.0 ** -6))
+    pre_ref, _ = moe.next_prenorm(ref["out"], gn, 1e-6)
+    rel, mx = compare_outputs(nx, pre_ref, skip=ref["near_tie"])
+    assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
+    with pytest.raises(bm.BeamMoeError):
+        layer.forward_prenorm(xd, rd, g_next, 1e-6, next_x=rd)  # next_x may not alias residual
+    layer.close()

@@ -188,6 +188,21 @@ def test_rmsnorm_closed_form_and_bf16():
     np.testing.assert_array_equal(moe.bf16_round(v.astype(np.float64)), ref)
 
 
+def test_next_prenorm_closed_form():
+    # constant rows c -> gamma * sign(c) / sqrt(1 + eps / c^2); the output is rounded to BF16
+    c = np.array([3.0, -0.25])
+    out = np.broadcast_to(c[:, None], (2, 32)).copy()
+    gam = np.linspace(0.5, 2.0, 32)
+    pre, rounded = moe.next_prenorm(out, gam, 1e-6)
+    expect = np.sign(c)[:, None] * gam[None, :] / np.sqrt(1 + 1e-6 / c[:, None] ** 2)
+    np.testing.assert_allclose(pre, expect, rtol=1e-14)
+    assert np.all(np.abs(rounded - pre) <= 2.0 ** -8 * np.abs(pre))  # half a BF16 ulp
+    # scale invariance: RMSNorm(a x) = RMSNorm(x) for a > 0 (eps -> 0)
+    x = np.random.default_rng(8).standard_normal((3, 64))
+    np.testing.assert_allclose(moe.next_prenorm(4.0 * x, np.ones(64), 0.0)[0], moe.next_prenorm(x, np.ones(64), 0.0)[0],
+                               rtol=1e-13)
+
+
 def test_grid_exact_expert_gemms_equal_fp64_matmul():
     # Operands already on the E2M1 x E4M3 grid with power-of-two tensor scales quantise
     # losslessly, so steps 7 and 10 reduce to plain FP64 matmuls of the raw values.
