@@ -62,8 +62,10 @@ def kernel_work(shape: mi.LayerShape, T: int, counts: np.ndarray) -> dict:
         "scan": dict(bytes=E * 16, flops=0),
         "scatter": dict(bytes=R * 12, flops=0),
         "quant_a1": dict(bytes=T * H * 2 + R * H * q, flops=0),
-        "gemm_gate_up": dict(bytes=used * 2 * I * H * q + R * H * q + R * I * q, flops=2 * R * 2 * I * H),
-        "gemm_down": dict(bytes=used * H * I * q + R * I * q + R * H * 2, flops=2 * R * H * I),
+        # gate/up + down in one launch: both weight sets of the used experts, A1 read, the
+        # NVFP4 intermediate A2 written and read back, y written (BF16)
+        "gemm_experts": dict(bytes=used * 3 * I * H * q + R * H * q + 2 * R * I * q + R * H * 2,
+                             flops=2 * R * 3 * I * H),
         "finalize": dict(bytes=R * H * 2 + 2 * T * H * 2 + H * 2, flops=0),
         "_used_experts": used,
     }
@@ -218,10 +220,13 @@ def run_reference(args, shape, rank, world):
     emit(line, rank)
 
 
-def workload_config(shape):
+def workload_config(shape, l2_flush="write"):
+    l2 = f"flushed: {L2_FLUSH_BYTES >> 20} MiB write between timed steps"
+    if l2_flush == "write+read":
+        l2 = f"flushed: {L2_FLUSH_BYTES >> 20} MiB write + {L2_FLUSH_BYTES >> 21} MiB read between timed steps"
     return {"workload": shape.name, "tokens": shape.tokens, "hidden": shape.hidden, "experts": shape.experts,
             "top_k": shape.top_k, "inter": shape.inter, "routing": "zipf-skewed" if shape.skew else "uniform",
-            "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MiB write between timed steps"}
+            "l2": l2}
 
 
 # ------------------------------------------------------------------ multi-rank plumbing
@@ -267,7 +272,17 @@ def run_ours(args, shape, rank, world, local_rank):
     x, res = x.to(dev), res.to(dev)
     out = torch.empty_like(res)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.float32, device=dev) if args.l2_flush == "write+read" \
+        else None
     T = shape.tokens
+
+    def flush_l2():
+        """Between steps, outside the timed region: write a buffer 4x the L2; with
+        write+read, then read another 2x the L2 so the step starts with L2 clean as well
+        as cold (the write-back of the flush's dirty lines is not charged to the step)."""
+        flush.zero_()
+        if clean is not None:
+            clean.sum()
 
     def barrier():
         if world > 1:
@@ -275,7 +290,7 @@ def run_ours(args, shape, rank, world, local_rank):
 
     for _ in range(max(args.warmup, 3)):
         layer.forward(x, res, out)
-        flush.zero_()
+        flush_l2()
     layer.check()
     torch.cuda.synchronize()
     barrier()
@@ -288,7 +303,7 @@ def run_ours(args, shape, rank, world, local_rank):
             starts[i].record(stream)
             layer.forward(x, res, out)
             ends[i].record(stream)
-            flush.zero_()
+            flush_l2()
         torch.cuda.synchronize()
         barrier()
     launches = layer.launches() * args.steps
@@ -305,7 +320,7 @@ def run_ours(args, shape, rank, world, local_rank):
         layer.forward(x, res, out)
         for name, kms in layer.kernel_times():
             acc.setdefault(name, []).append(kms)
-        flush.zero_()
+        flush_l2()
     layer.profile(False)
     kern = {n: sum(v) / len(v) for n, v in acc.items()}
     offsets = np.frombuffer(layer.debug(bm.BUF_OFFSETS).cpu().numpy().tobytes(), np.int32)
@@ -339,7 +354,7 @@ def run_ours(args, shape, rank, world, local_rank):
         e_s[i].record(stream)
         layer.forward_host(xh, rh, oh)
         e_e[i].record(stream)
-        flush.zero_()
+        flush_l2()
     torch.cuda.synchronize()
     barrier()
     e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)) / args.steps, world, dev)
@@ -352,7 +367,7 @@ def run_ours(args, shape, rank, world, local_rank):
             "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) experts, fp32 router and accumulation",
             "data": "synthetic (seeded; random-init weights of the layer's shapes)",
-            "config": dict(workload_config(shape), parallelism=f"token-dp replicas x{world}"),
+            "config": dict(workload_config(shape, args.l2_flush), parallelism=f"token-dp replicas x{world}"),
             "roofline": roofline,
             "kernels_ms": kern,
             "used_experts": work["_used_experts"],
@@ -373,6 +388,9 @@ def main():
     ap.add_argument("--workload", default="decode8", choices=sorted(mi.SHAPES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--l2-flush", default="write+read", choices=["write", "write+read"],
+                    help="between timed steps: write 512 MiB, then (default) read 256 MiB so the step starts "
+                         "with L2 cold and clean")
     args = ap.parse_args()
     shape = mi.SHAPES[args.workload]
     rank = int(os.environ.get("RANK", 0))

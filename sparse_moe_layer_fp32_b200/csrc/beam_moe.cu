@@ -28,12 +28,14 @@ struct beam_moe_ctx {
   float* logits;
   int64_t logits_floats;
   int32_t *ids, *chunk_counts, *chunk_base, *offsets, *sf_block, *num_mblocks, *perm, *inv;
+  int32_t* tile_row;  // [T][k]: 128 x activation block + row in it (where slot (t, j) goes in A1)
   float* w;
   MBlock* mblocks;
   uint8_t *a1, *a1_sf, *a2, *a2_sf;
   uint16_t* y;
   uint32_t* err;
   unsigned int* route_counter;  // last-CTA election of the fused small-batch routing kernel
+  uint32_t* sched;              // tile scheduler of the expert GEMM launch (sched_words(nblk_max))
   uint16_t *stage_x, *stage_res, *stage_out;
   int last_T;
   int last_splits;  // logits layout of the last forward: [splits][T][E] partial sums
@@ -231,6 +233,8 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   int64_t lf = 0;
   for (int T = 1; T <= h->Tmax; T = (T < 64 ? T + 1 : T + 64)) lf = std::max(lf, route_ws_floats(T, H, E));
   lf = std::max(lf, route_ws_floats(h->Tmax, H, E));
+  for (int T = 1; T <= std::min(h->Tmax, kMaxSmallRouterTokens); ++T)
+    if (route_small_supported(T, H, h->E, h->k)) lf = std::max(lf, route_small_ws_floats(T, H, h->E));
   h->logits_floats = lf;
   const int64_t R = h->Rmax;
   CREATE_TRY(dalloc(h, &h->logits, sizeof(float) * lf));
@@ -244,6 +248,7 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   CREATE_TRY(dalloc(h, &h->mblocks, sizeof(MBlock) * h->nblk_max));
   CREATE_TRY(dalloc(h, &h->perm, sizeof(int32_t) * R));
   CREATE_TRY(dalloc(h, &h->inv, sizeof(int32_t) * R));
+  CREATE_TRY(dalloc(h, &h->tile_row, sizeof(int32_t) * R));
   CREATE_TRY(dalloc(h, &h->a1, static_cast<size_t>(h->nblk_max) * (H / 2) * 128));
   CREATE_TRY(dalloc(h, &h->a1_sf, static_cast<size_t>(h->nblk_max) * (H / 64) * 512));
   CREATE_TRY(dalloc(h, &h->a2, static_cast<size_t>(h->nblk_max) * (Ip / 2) * 128));
@@ -252,6 +257,7 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   CREATE_TRY(dalloc(h, &h->err, sizeof(uint32_t)));
   CREATE_TRY(dalloc(h, &h->route_counter, sizeof(unsigned int)));
   CREATE_TRY(cudaMemsetAsync(h->route_counter, 0, sizeof(unsigned int), s));
+  CREATE_TRY(dalloc(h, &h->sched, sizeof(uint32_t) * sched_words(h->nblk_max)));
   CREATE_TRY(dalloc(h, &h->stage_x, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   CREATE_TRY(dalloc(h, &h->stage_res, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   CREATE_TRY(dalloc(h, &h->stage_out, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
@@ -314,11 +320,13 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
   if (route_small_supported(T, H, E, k)) {
     // router + top-k + histogram + scan + permutation in one launch
+    int slices = 1;
     BEAM_TRY(launch_route_small(xb, h->router_w, T, H, E, k, h->logits, h->ids, h->w, h->offsets, h->sf_block,
-                                h->mblocks, h->num_mblocks, h->perm, h->inv, h->route_counter, s));
+                                h->mblocks, h->num_mblocks, h->perm, h->inv, h->tile_row, h->route_counter, h->sched,
+                                static_cast<int>(sched_words(h->nblk_max)), h->err, &slices, s));
     BEAM_TRY(mark("route_small"));
     ++launches;
-    h->last_splits = 1;
+    h->last_splits = slices;
   } else {
     if (router_tc_supported(T, H, E, k)) {
       // FP32-class logits on the tensor cores (BF16 x 3-part split), top-k in the epilogue
@@ -341,55 +349,46 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     BEAM_TRY(mark("chunk_hist"));
     ++launches;
     BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
-                         h->num_mblocks, s));
+                         h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), s));
     BEAM_TRY(mark("scan"));
     ++launches;
-    BEAM_TRY(launch_scatter(h->ids, h->chunk_base, T, k, E, h->perm, h->inv, s));
+    BEAM_TRY(launch_scatter(h->ids, h->chunk_base, h->offsets, h->sf_block, T, k, E, h->perm, h->inv, h->tile_row,
+                            s));
     BEAM_TRY(mark("scatter"));
     ++launches;
   }
-  BEAM_TRY(launch_quant_a1(xb, h->ids, h->inv, h->offsets, h->sf_block, T, H, k, h->cfg.alpha_a1, h->a1,
-                           h->a1_sf, s));
+  BEAM_TRY(launch_quant_a1(xb, h->tile_row, T, H, k, h->cfg.alpha_a1, h->a1, h->a1_sf, s));
   BEAM_TRY(mark("quant_a1"));
   ++launches;
 
-  GemmArgs g{};
+  ExpertGemmArgs g{};
   g.mblocks = h->mblocks;
   g.num_mblocks = h->num_mblocks;
   g.max_rows_per_expert = T;  // a token chooses an expert at most once
-  g.err = h->err;
-  // gate/up: 256 B rows per tile = 128 gate + 128 up features
-  g.n_tiles = h->I / 128;
-  g.k_tiles = H / 256;
-  g.a_tiles = h->a1;
-  g.b_tiles = h->w_gu_tiles;
-  g.sfa = h->a1_sf;
-  g.alpha_b = h->w_gu_alpha;
-  g.alpha_a = h->cfg.alpha_a1;
+  g.gu_n_tiles = h->I / 128;
+  g.gu_k_tiles = H / 256;
+  g.a1 = h->a1;
+  g.a1_sf = h->a1_sf;
+  g.w_gu = h->w_gu_tiles;
+  g.w_gu_alpha = h->w_gu_alpha;
+  g.alpha_a1 = h->cfg.alpha_a1;
   g.a2 = h->a2;
   g.a2_sf = h->a2_sf;
-  g.a2_k_tiles = h->Ip / 256;
-  g.a2_kgroups = h->Ip / 64;
   g.alpha_a2 = h->cfg.alpha_a2;
-  BEAM_TRY(launch_gemm_gate_up(g, h->num_sms, s));
-  BEAM_TRY(mark("gemm_gate_up"));
-  ++launches;
-  // down
-  g.n_tiles = H / 256;
-  g.k_tiles = h->Ip / 256;
-  g.a_tiles = h->a2;
-  g.b_tiles = h->w_d_tiles;
-  g.sfa = h->a2_sf;
-  g.alpha_b = h->w_d_alpha;
-  g.alpha_a = h->cfg.alpha_a2;
+  g.d_n_tiles = H / 256;
+  g.d_k_tiles = h->Ip / 256;
+  g.w_d = h->w_d_tiles;
+  g.w_d_alpha = h->w_d_alpha;
   g.y = h->y;
   g.y_cols = H;
-  BEAM_TRY(launch_gemm_down(g, h->num_sms, s));
-  BEAM_TRY(mark("gemm_down"));
+  g.sched = h->sched;
+  g.err = h->err;
+  BEAM_TRY(launch_gemm_experts(g, h->num_sms, s));
+  BEAM_TRY(mark("gemm_experts"));
   ++launches;
   BEAM_TRY(launch_finalize(h->y, h->w, h->inv, static_cast<const uint16_t*>(residual), h->gamma, T, H, k,
                            h->cfg.rms_eps, static_cast<uint16_t*>(out), static_cast<uint16_t*>(next_x),
-                           static_cast<const uint16_t*>(next_gamma), next_eps, s));
+                           static_cast<const uint16_t*>(next_gamma), next_eps, h->err, s));
   BEAM_TRY(mark("finalize"));
   ++launches;
   h->last_T = T;

@@ -8,6 +8,8 @@
 // article "vLLM adds day-zero Reflection Beam serving": fused normalisation and residual
 // kernels).  One CTA per token; every global access is a 16-byte vector (8 BF16), and a
 // warp's accesses are contiguous, so the k row gathers of y stream at full HBM width.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -141,127 +143,149 @@ __global__ void __launch_bounds__(kFinThreads) finalize_wide_kernel(const uint16
   }
 }
 
-// Small batches: one CTA per token, CPT 16-byte chunks (8 values) per thread kept in
-// registers, the k row gathers of a thread issued together, one block reduction.
-template <int CPT, bool PRE>
-__global__ void __launch_bounds__(1024) finalize_kernel(const uint16_t* __restrict__ y, const float* __restrict__ w,
-                                                        const int32_t* __restrict__ inv, const uint16_t* residual,
-                                                        const uint16_t* __restrict__ gamma, int H, int k, float eps,
-                                                        uint16_t* out, NextNorm nn) {
+// Small batches: one CTA per token, its rows staged in shared memory by bulk copies (a
+// handful of CTAs must move each token's k rows of y, so the loads go through the copy
+// engine rather than per-thread loads).  The residual row and gamma (and the next gamma) do
+// not depend on the GEMM and are copied before the wait for it; inv and w come from the
+// routing, two launches back, and are read first.  Each thread owns 8-value chunks; the
+// weighted sums are recomputed from shared memory in each pass instead of being kept.
+template <bool PRE>
+__global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __restrict__ y,
+                                                              const float* __restrict__ w,
+                                                              const int32_t* __restrict__ inv,
+                                                              const uint16_t* residual,
+                                                              const uint16_t* __restrict__ gamma, int H, int k,
+                                                              float eps, uint16_t* out, NextNorm nn, uint32_t* err) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint16_t* ys = reinterpret_cast<uint16_t*>(smem);  // [k][H]
+  uint16_t* rs = ys + static_cast<size_t>(k) * H;     // [H] residual row
+  uint16_t* gs = rs + H;                              // [H] gamma
+  uint16_t* ngs = gs + H;                             // [H] next gamma (PRE)
+  __shared__ uint64_t bars[2];
   __shared__ int s_row[16];
   __shared__ float s_w[16];
   __shared__ float s_red[32];
+  __shared__ int s_abort;
   const int t = blockIdx.x;
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < k) {
+    s_row[threadIdx.x] = __ldcg(inv + static_cast<size_t>(t) * k + threadIdx.x);
+    s_w[threadIdx.x] = __ldcg(w + static_cast<size_t>(t) * k + threadIdx.x);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bars[0], (PRE ? 3u : 2u) * row_bytes);
+    bulk_load(rs, residual + static_cast<size_t>(t) * H, row_bytes, &bars[0]);  // out may alias residual
+    bulk_load(gs, gamma, row_bytes, &bars[0]);
+    if constexpr (PRE) bulk_load(ngs, nn.gamma, row_bytes, &bars[0]);
+  }
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x < k) {
-    s_row[threadIdx.x] = inv[static_cast<size_t>(t) * k + threadIdx.x];
-    s_w[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bars[1], static_cast<uint32_t>(k) * row_bytes);
+    for (int j = 0; j < k; ++j)
+      bulk_load(ys + static_cast<size_t>(j) * H, y + static_cast<size_t>(s_row[j]) * H, row_bytes, &bars[1]);
   }
-  __syncthreads();
+  const bool ok0 = mbar_wait_bounded(&bars[0], 0, &s_abort);
+  const bool ok1 = mbar_wait_bounded(&bars[1], 0, &s_abort);
+  if (!(ok0 && ok1) && threadIdx.x == 0) atomicOr(err, kErrTimeoutEpilogue);
   const int nchunks = H / 8;
-  float acc[CPT][8];
-  float ss = 0.0f;
+  // m[c] = sum_j w_j y_j over this chunk's 8 values, in slot order
+  auto weighted = [&](int c, float (&m)[8]) {
 #pragma unroll
-  for (int q = 0; q < CPT; ++q) {
-    const int c = threadIdx.x + q * blockDim.x;
+    for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      float f[8];
+      unpack8(reinterpret_cast<const uint4*>(ys + static_cast<size_t>(j) * H)[c], f);
+      const float wj = s_w[j];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[q][i] = 0.0f;
-    if (c < nchunks) {
-      for (int j0 = 0; j0 < k; j0 += 8) {
-        uint4 yv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)  // up to 8 row gathers in flight together
-          if (j0 + j < k) yv[j] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j0 + j]) * H) + c);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j0 + j >= k) break;
-          float f[8];
-          unpack8(yv[j], f);
-          const float wj = s_w[j0 + j];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[q][i] = fmaf(wj, f[i], acc[q][i]);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ss = fmaf(acc[q][i], acc[q][i], ss);
+      for (int i = 0; i < 8; ++i) m[i] = fmaf(wj, f[i], m[i]);
     }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  float tot = 0.0f;
-  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) tot += s_red[i];
-  const float rinv = 1.0f / sqrtf(tot / static_cast<float>(H) + eps);
-  float ss2 = 0.0f;
-#pragma unroll
-  for (int q = 0; q < CPT; ++q) {
-    const int c = threadIdx.x + q * blockDim.x;
-    if (c >= nchunks) continue;
+  };
+  auto out_chunk = [&](int c, float rinv, float (&m)[8]) -> uint4 {
     float r[8], g[8];
-    unpack8(reinterpret_cast<const uint4*>(residual + static_cast<size_t>(t) * H)[c], r);  // out may alias residual
-    unpack8(__ldg(reinterpret_cast<const uint4*>(gamma) + c), g);
+    unpack8(reinterpret_cast<const uint4*>(rs)[c], r);
+    unpack8(reinterpret_cast<const uint4*>(gs)[c], g);
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      o[i] = pack_bf16x2(r[2 * i] + acc[q][2 * i] * rinv * g[2 * i], r[2 * i + 1] + acc[q][2 * i + 1] * rinv * g[2 * i + 1]);
-    const uint4 ov = make_uint4(o[0], o[1], o[2], o[3]);
+      o[i] = pack_bf16x2(r[2 * i] + m[2 * i] * rinv * g[2 * i], r[2 * i + 1] + m[2 * i + 1] * rinv * g[2 * i + 1]);
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  };
+  float ss = 0.0f;
+  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+    float m[8];
+    weighted(c, m);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(m[i], m[i], ss);
+  }
+  const float rinv = block_rinv(ss, H, eps, s_red);
+  float ss2 = 0.0f;
+  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+    float m[8];
+    weighted(c, m);
+    const uint4 ov = out_chunk(c, rinv, m);
     reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = ov;
     if constexpr (PRE) {  // the next pre-norm reads the BF16 values just written
-      unpack8(ov, acc[q]);
+      float f[8];
+      unpack8(ov, f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ss2 = fmaf(acc[q][i], acc[q][i], ss2);
+      for (int i = 0; i < 8; ++i) ss2 = fmaf(f[i], f[i], ss2);
     }
   }
   if constexpr (PRE) {
     const float r2 = block_rinv(ss2, H, nn.eps, s_red);
-#pragma unroll
-    for (int q = 0; q < CPT; ++q) {
-      const int c = threadIdx.x + q * blockDim.x;
-      if (c >= nchunks) continue;
-      float g[8];
-      unpack8(__ldg(reinterpret_cast<const uint4*>(nn.gamma) + c), g);
+    for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+      float m[8], f[8], g[8];
+      weighted(c, m);
+      unpack8(out_chunk(c, rinv, m), f);  // the same BF16 values as stored above
+      unpack8(reinterpret_cast<const uint4*>(ngs)[c], g);
       uint32_t o[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(acc[q][2 * i] * r2 * g[2 * i], acc[q][2 * i + 1] * r2 * g[2 * i + 1]);
+      for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(f[2 * i] * r2 * g[2 * i], f[2 * i + 1] * r2 * g[2 * i + 1]);
       reinterpret_cast<uint4*>(nn.x + static_cast<size_t>(t) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
 }
 
+static size_t finalize_small_smem(int H, int k) { return static_cast<size_t>(k + 3) * H * 2; }
+
 template <bool PRE>
 static cudaError_t launch_finalize_t(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
                                      const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out,
-                                     NextNorm nn, cudaStream_t s) {
+                                     NextNorm nn, uint32_t* err, cudaStream_t s) {
   const int nchunks = H / 8;
-  if (T >= 256) {
-    const size_t smem = static_cast<size_t>(H) * sizeof(float);
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(finalize_wide_kernel<PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-    }
-    return launch_pdl(finalize_wide_kernel<PRE>, dim3(T), dim3(kFinThreads), smem, s, y, w, inv, residual, gamma, H, k,
-                      eps, out, nn);
+  const size_t small = finalize_small_smem(H, k);
+  if (T < 256 && small <= 200 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(finalize_small_kernel<PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(small));
+    if (e != cudaSuccess) return e;
+    const int threads = std::min(1024, ((nchunks + 31) / 32) * 32);
+    return launch_pdl(finalize_small_kernel<PRE>, dim3(T), dim3(threads), small, s, y, w, inv, residual, gamma, H, k,
+                      eps, out, nn, err);
   }
-  if (nchunks <= 1024) {
-    const int threads = ((nchunks + 31) / 32) * 32;
-    return launch_pdl(finalize_kernel<1, PRE>, dim3(T), dim3(threads), 0, s, y, w, inv, residual, gamma, H, k, eps,
-                      out, nn);
+  const size_t smem = static_cast<size_t>(H) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(finalize_wide_kernel<PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
   }
-  if (nchunks <= 2048)
-    return launch_pdl(finalize_kernel<2, PRE>, dim3(T), dim3(1024), 0, s, y, w, inv, residual, gamma, H, k, eps, out,
-                      nn);
-  return cudaErrorInvalidValue;
+  return launch_pdl(finalize_wide_kernel<PRE>, dim3(T), dim3(kFinThreads), smem, s, y, w, inv, residual, gamma, H, k,
+                    eps, out, nn);
 }
 
 cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
                             const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, uint16_t* next_x,
-                            const uint16_t* next_gamma, float next_eps, cudaStream_t s) {
+                            const uint16_t* next_gamma, float next_eps, uint32_t* err, cudaStream_t s) {
   const NextNorm nn{next_x, next_gamma, next_eps};
-  if (next_x) return launch_finalize_t<true>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, s);
-  return launch_finalize_t<false>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, s);
+  if (next_x) return launch_finalize_t<true>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, err, s);
+  return launch_finalize_t<false>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, err, s);
 }
 
 }  // namespace beam

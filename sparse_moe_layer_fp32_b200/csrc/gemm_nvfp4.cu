@@ -1,4 +1,5 @@
-// Grouped NVFP4 x NVFP4 GEMMs of the routed experts on the sm_100a tensor cores.
+// Grouped NVFP4 x NVFP4 GEMMs of the routed experts on the sm_100a tensor cores: the
+// gate/up GEMM and the down GEMM of every expert in ONE persistent launch.
 //
 // NVFP4 routed experts run W4A4 on Blackwell (recipe "reflection/Beam-1.0-501B-A23B",
 // section "Variants"); the experts are SwiGLU MLPs.  Two GEMMs per expert e over the rows
@@ -7,12 +8,24 @@
 //   gate/up: D[r][n] = A1[r] . Wgu[e][n],  K = H; epilogue h = silu(g) * u, A2 = Q(h)
 //   down:    D[r][n] = A2[r] . Wd[e][n],   K = I; epilogue y = bf16(D * scale)
 //
-// Design (one persistent CTA per SM, 320 threads, warp-specialised):
-//   warp 0      producer: per 256-wide K step, bulk copies of the A tile (the valid rows
-//               of a 128-row activation tile, <= 16 KB), the expert's weight tile with its
-//               scales (32 KB + 4 KB) and the A scales (2 KB) into a 4-stage shared-memory
-//               ring, all landing on one mbarrier.  Activations and weights are both stored
-//               as contiguous tiles already in the swizzled shared-memory order, so every
+// Work items are (128-row block of one expert) x (256-column tile).  The tile list holds
+// every gate/up tile, then every down tile; CTAs claim tiles in that order from a global
+// counter, so a CTA that drew cheap tiles takes more, and the down tiles of early blocks
+// fill the tail of the gate/up work instead of waiting for a second launch.  A down tile
+// of block b needs all of block b's A2 columns: every epilogue warp that finishes a
+// gate/up tile of b publishes its stores (proxy fence, release) and bumps ready[b]; the
+// producer that claimed the down tile waits (bounded) until ready[b] counts all of them,
+// then reads A2 with bulk copies.  Claims are in list order and a gate/up tile never
+// waits on anything, so every awaited tile is held by a running CTA: no deadlock, and no
+// need for all CTAs to be resident at once.
+//
+// CTA layout (one persistent CTA per SM, 320 threads, warp-specialised):
+//   warp 0      producer: claims tiles, publishes each tile id through a small shared
+//               ring, and per 256-wide K step bulk-copies the A tile (the valid rows of a
+//               128-row activation tile, <= 16 KB), the expert's weight tile with its
+//               scales (32 KB + 4 KB) and the A scales (2 KB) into the stage ring, all
+//               landing on one mbarrier.  Activations and weights are both stored as
+//               contiguous tiles already in the swizzled shared-memory order, so every
 //               load is one sequential copy.
 //   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scales -> TMEM) and
 //               tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128, N=256, K=64) into a
@@ -20,10 +33,8 @@
 //   warps 2..9  epilogue: tcgen05.ld the accumulator (each warp its 32-lane quarter and
 //               one half of the columns), release it to the MMA warp at once, then do the
 //               FP32 math and the stores while the next tile accumulates.
-// Work items are (128-row block of one expert) x (256-column tile); the block list is
-// built on the device by the permutation step, so the host never synchronises.
-// Every mbarrier wait is bounded (kWaitLimitNs): on expiry the CTA sets the device error
-// word, drains its own copies and MMAs, frees TMEM and exits.
+// Every wait is bounded (kWaitLimitNs): on expiry the CTA sets the device error word,
+// drains its own copies and MMAs, frees TMEM and exits.
 #include "common.cuh"
 #include "internal.h"
 
@@ -53,6 +64,7 @@ using RingFull = Ring<4, A_TILE_BYTES>;
 using RingSmallM = Ring<5, 32 * BK_BYTES>;
 constexpr int NUM_THREADS = 320;
 constexpr int NUM_EPI_WARPS = 8;
+constexpr int kTileSlots = 4;       // tile ids the producer may publish ahead of the epilogue
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;     // 256 FP32 columns
 constexpr uint32_t SFA_COL = 256;   // 4 K-groups x 4 columns
@@ -62,15 +74,16 @@ constexpr uint32_t SFB_COL = 288;   // 4 K-groups x 8 columns
 // operands, N = 256 (n_dim = N/8 at bit 17), M = 128 (m_dim = M/16 at bit 24).
 constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((BM >> 4) << 24);
 
-enum Epilogue { kSwiGLU = 0, kStoreBF16 = 1 };
-
 constexpr int kMaxStages = 5;
 struct __align__(8) GemmSmemTail {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
+  uint64_t tile_full[kTileSlots];   // producer -> MMA + epilogue: tile id published
+  uint64_t tile_empty[kTileSlots];  // MMA + epilogue warps -> producer: slot read
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
+  int tile_ids[kTileSlots];         // claimed tile, -1 = no more work
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -79,7 +92,6 @@ template <class R>
 static size_t ring_smem_bytes() {
   return static_cast<size_t>(R::STAGES) * R::STAGE_BYTES + sizeof(GemmSmemTail) + 1024;
 }
-size_t gemm_smem_bytes() { return ring_smem_bytes<RingFull>(); }
 
 __device__ __forceinline__ float silu_times(float g, float u) { return __fdiv_rn(g, 1.0f + expf(-g)) * u; }
 
@@ -88,9 +100,50 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int EPI, class R>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_nvfp4_kernel(const GemmArgs args) {
+// Waits until *counter >= target (acquire).  Returns false (and sets *abort) when the
+// wait ran past kWaitLimitNs or another role already aborted.
+__device__ __forceinline__ bool wait_counter_bounded(const uint32_t* counter, uint32_t target,
+                                                     volatile int* abort_flag) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Block-list entries are written by the routing kernels; read them from L2.
+__device__ __forceinline__ MBlock load_mblock(const MBlock* p) {
+  const int4 v = __ldcg(reinterpret_cast<const int4*>(p));
+  return MBlock{v.x, v.y, v.z, v.w};
+}
+
+// Position of a tile id in the list [gate/up tiles of every block][down tiles of every block].
+struct TileRef {
+  bool down;
+  int block;  // index into the block list
+  int nt;     // 256-column output tile
+};
+
+__device__ __forceinline__ TileRef tile_ref(int id, int total_gu, int n_gu, int n_d) {
+  TileRef t;
+  t.down = id >= total_gu;
+  const int rel = t.down ? id - total_gu : id;
+  const int n = t.down ? n_d : n_gu;
+  t.block = rel / n;
+  t.nt = rel - t.block * n;
+  return t;
+}
+
+template <class R>
+__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const ExpertGemmArgs args) {
   constexpr int STAGES = R::STAGES, A_BYTES = R::A_BYTES, STAGE_BYTES = R::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -102,6 +155,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&tail->full[s], 1);
       mbar_init(&tail->empty[s], 1);
+    }
+    for (int j = 0; j < kTileSlots; ++j) {
+      mbar_init(&tail->tile_full[j], 1);
+      mbar_init(&tail->tile_empty[j], 1 + NUM_EPI_WARPS);
     }
     mbar_init(&tail->acc_full, 1);
     mbar_init(&tail->acc_empty, NUM_EPI_WARPS);
@@ -117,53 +174,112 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tail->tmem_base;
-  pdl_wait();  // the previous kernel's outputs (block list, activations) are complete
-  pdl_trigger();
+  // The block list and the zeroed scheduler words come from the routing kernels, two or
+  // more launches back, which are complete once this grid runs (every kernel of the forward
+  // triggers its dependents only after its own wait).  Only the activations A1 come from the
+  // previous kernel, so the producer claims tiles and streams the first stages' weights
+  // before it waits; every other thread waits here.
+  const bool producer = warp == 0 && lane == 0;
+  if (!producer) {
+    pdl_wait();
+    pdl_trigger();
+  }
 
-  const int n_tiles = args.n_tiles, k_tiles = args.k_tiles;
-  const int kgroups = k_tiles * 4;
-  const int total = *args.num_mblocks * n_tiles;
+  const int n_gu = args.gu_n_tiles, n_d = args.d_n_tiles;
+  const int num_blocks = __ldcg(args.num_mblocks);
+  const int total_gu = num_blocks * n_gu;
+  const int total = total_gu + num_blocks * n_d;
+  uint32_t* const ready = args.sched + 1;
+  const uint32_t ready_target = static_cast<uint32_t>(n_gu) * NUM_EPI_WARPS;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, slot = 0;
+      uint32_t phase = 0, slot_phase = 0;
       uint32_t armed = 0, armed_parity = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const MBlock mb = args.mblocks[tile / n_tiles];
-        const int nt = tile % n_tiles;
-        const uint8_t* sfa = args.sfa + (static_cast<size_t>(mb.sf_block) * kgroups) * 512;
-        const uint8_t* btile =
-            args.b_tiles + (static_cast<size_t>(mb.expert) * n_tiles + nt) * k_tiles * static_cast<size_t>(kTileBytes);
+      // The next claim is issued while the current tile's last STAGES K steps are still to
+      // be loaded, so its round trip hides behind them instead of opening a gap in the ring.
+      uint32_t claim = atomicAdd(args.sched, 1u);
+      bool waited = false;  // grid dependency resolved: activations may be read
+      for (;;) {
+        if (!mbar_wait_bounded(&tail->tile_empty[slot], slot_phase ^ 1, abort_flag)) break;
+        int id = claim < static_cast<uint32_t>(total) ? static_cast<int>(claim) : -1;
+        tail->tile_ids[slot] = id;
+        mbar_arrive(&tail->tile_full[slot]);
+        if (++slot == kTileSlots) {
+          slot = 0;
+          slot_phase ^= 1;
+        }
+        if (id < 0) break;
+        const TileRef t = tile_ref(id, total_gu, n_gu, n_d);
+        const MBlock mb = load_mblock(args.mblocks + t.block);
+        const int k_tiles = t.down ? args.d_k_tiles : args.gu_k_tiles;
+        const int n_tiles = t.down ? n_d : n_gu;
+        const uint8_t* a_src = (t.down ? args.a2 : args.a1) + static_cast<size_t>(mb.sf_block) * k_tiles * A_TILE_BYTES;
+        const uint8_t* sfa = (t.down ? args.a2_sf : args.a1_sf) + static_cast<size_t>(mb.sf_block) * k_tiles * SFA_BYTES;
+        const uint8_t* btile = (t.down ? args.w_d : args.w_gu) +
+                               (static_cast<size_t>(mb.expert) * n_tiles + t.nt) * k_tiles * static_cast<size_t>(kTileBytes);
+        if (t.down) {
+          // this block's A2 is written by the gate/up epilogues (possibly of other CTAs)
+          if (!wait_counter_bounded(ready + t.block, ready_target, abort_flag)) {
+            atomicOr(args.err, kErrTimeoutProducer);
+            break;
+          }
+          fence_proxy_async_global();
+        }
+        // rows past the block's valid rows are not copied: their stale shared-memory
+        // contents only reach accumulator rows that are never stored
+        uint32_t a_bytes = static_cast<uint32_t>(min(BM, (mb.rows + 7) & ~7)) * BK_BYTES;
+        if (a_bytes > static_cast<uint32_t>(A_BYTES)) {  // cannot happen when the host picks the ring right
+          atomicOr(args.err, kErrRange);
+          a_bytes = A_BYTES;
+        }
+        // A and its scales of K step kk into stage st
+        auto load_a = [&](int st, int kk) {
+          uint8_t* sa = smem + st * STAGE_BYTES;
+          bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, a_bytes, &tail->full[st]);
+          bulk_load(sa + A_BYTES + B_BYTES + SFB_BYTES, sfa + static_cast<size_t>(kk) * SFA_BYTES, SFA_BYTES,
+                    &tail->full[st]);
+        };
+        // Before the wait only the weights are loaded; the first tile starts at stage 0, so
+        // its deferred K steps kk < STAGES sit in stages kk.
+        int deferred = 0;
+        auto resolve = [&]() {
+          pdl_wait();
+          pdl_trigger();
+          waited = true;
+          for (int kk = 0; kk < deferred; ++kk) load_a(kk, kk);
+        };
+        bool ok = true;
+        const int claim_at = max(0, k_tiles - STAGES);
         for (int kt = 0; kt < k_tiles; ++kt) {
+          if (kt == claim_at) claim = atomicAdd(args.sched, 1u);
+          if (!waited && kt == STAGES) resolve();
           if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          uint8_t* ssfa = sb + B_BYTES + SFB_BYTES;
-          // rows past the block's valid rows are not copied: their stale shared-memory
-          // contents only reach accumulator rows that are never stored
-          uint32_t a_bytes = static_cast<uint32_t>(min(BM, (mb.rows + 7) & ~7)) * BK_BYTES;
-          if (a_bytes > static_cast<uint32_t>(A_BYTES)) {  // cannot happen when the host picks the ring right
-            atomicOr(args.err, kErrRange);
-            a_bytes = A_BYTES;
-          }
           mbar_arrive_expect_tx(&tail->full[stage], a_bytes + kTileBytes + SFA_BYTES);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          bulk_load(sa, args.a_tiles + (static_cast<size_t>(mb.sf_block) * k_tiles + kt) * A_TILE_BYTES, a_bytes,
+          bulk_load(smem + stage * STAGE_BYTES + A_BYTES, btile + static_cast<size_t>(kt) * kTileBytes, kTileBytes,
                     &tail->full[stage]);
-          bulk_load(sb, btile + static_cast<size_t>(kt) * kTileBytes, kTileBytes, &tail->full[stage]);
-          bulk_load(ssfa, sfa + static_cast<size_t>(kt) * 4 * 512, SFA_BYTES, &tail->full[stage]);
+          if (waited)
+            load_a(stage, kt);
+          else
+            ++deferred;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
+        if (!waited) resolve();
+        if (!ok) break;
+      }
+      if (!waited) {  // no tile claimed
+        pdl_wait();
+        pdl_trigger();
       }
       // Copies still in flight land before this CTA may exit (bounded).
       for (int s = 0; s < STAGES; ++s)
@@ -176,12 +292,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      int stage = 0, slot = 0;
+      uint32_t phase = 0, acc_phase = 0, slot_phase = 0;
+      for (;;) {
+        if (!mbar_wait_bounded(&tail->tile_full[slot], slot_phase, abort_flag)) break;
+        const int id = tail->tile_ids[slot];
+        mbar_arrive(&tail->tile_empty[slot]);
+        if (++slot == kTileSlots) {
+          slot = 0;
+          slot_phase ^= 1;
+        }
+        if (id < 0) break;
+        const int k_tiles = id >= total_gu ? args.d_k_tiles : args.gu_k_tiles;
         if (!mbar_wait_bounded(&tail->acc_empty, acc_phase ^ 1, abort_flag)) break;
         tc_fence_after();
+        bool ok = true;
         for (int kt = 0; kt < k_tiles; ++kt) {
           if (!mbar_wait_bounded(&tail->full[stage], phase, abort_flag)) {
             ok = false;
@@ -225,14 +350,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (warp - 2) >> 2;       // which half of the 256 accumulator columns
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const MBlock mb = args.mblocks[tile / n_tiles];
-      const int nt = tile % n_tiles;
-      if (!mbar_wait_bounded(&tail->acc_full, acc_phase, abort_flag)) break;
+    const float alpha2 = args.alpha_a2;
+    const float six_alpha2 = __fmul_rn(6.0f, alpha2);
+    int slot = 0;
+    uint32_t acc_phase = 0, slot_phase = 0;
+    for (;;) {
+      // every lane waits; the warp leaves together if any lane gave up, so the warp-wide
+      // operations below never run with part of the warp gone
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->tile_full[slot], slot_phase, abort_flag))) break;
+      const int id = tail->tile_ids[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->tile_empty[slot]);
+      if (++slot == kTileSlots) {
+        slot = 0;
+        slot_phase ^= 1;
+      }
+      if (id < 0) break;
+      const TileRef t = tile_ref(id, total_gu, n_gu, n_d);
+      const MBlock mb = load_mblock(args.mblocks + t.block);
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->acc_full, acc_phase, abort_flag))) break;
       tc_fence_after();
       uint32_t v[4][32];
-      if constexpr (EPI == kSwiGLU) {
+      if (!t.down) {  // gate columns [half*64, +64) and the matching up columns
         tmem_ld_32x32b_x32(t_lane + ACC_COL + half * 64, v[0]);
         tmem_ld_32x32b_x32(t_lane + ACC_COL + half * 64 + 32, v[1]);
         tmem_ld_32x32b_x32(t_lane + ACC_COL + 128 + half * 64, v[2]);
@@ -246,40 +385,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->acc_empty);
       acc_phase ^= 1;
-      if (row_in_tile >= mb.rows) continue;
-      const size_t r = static_cast<size_t>(mb.row_begin + row_in_tile);
-      (void)r;
-      const float scale = args.alpha_a * __ldg(args.alpha_b + mb.expert);
-      if constexpr (EPI == kSwiGLU) {
-        const float alpha2 = args.alpha_a2;
-        const float six_alpha2 = __fmul_rn(6.0f, alpha2);
-        const int f0 = nt * 128 + half * 64;  // first feature of this thread's 64
-        uint32_t codes[8];
-        uint32_t scodes = 0;
+      const bool valid = row_in_tile < mb.rows;
+      if (!t.down) {
+        if (valid) {
+          const float scale = args.alpha_a1 * __ldg(args.w_gu_alpha + mb.expert);
+          const int f0 = t.nt * 128 + half * 64;  // first feature of this thread's 64
+          uint32_t codes[8];
+          uint32_t scodes = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          float h[16];
+          for (int b = 0; b < 4; ++b) {
+            float h[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c = b * 16 + i;
-            const float g = __uint_as_float(v[c >> 5][c & 31]) * scale;
-            const float u = __uint_as_float(v[2 + (c >> 5)][c & 31]) * scale;
-            h[i] = silu_times(g, u);
+            for (int i = 0; i < 16; ++i) {
+              const int c = b * 16 + i;
+              const float g = __uint_as_float(v[c >> 5][c & 31]) * scale;
+              const float u = __uint_as_float(v[2 + (c >> 5)][c & 31]) * scale;
+              h[i] = silu_times(g, u);
+            }
+            const uint32_t sc = quant_block16(h, alpha2, six_alpha2, codes[2 * b], codes[2 * b + 1]);
+            scodes |= sc << (8 * b);
           }
-          const uint32_t sc = quant_block16(h, alpha2, six_alpha2, codes[2 * b], codes[2 * b + 1]);
-          scodes |= sc << (8 * b);
+          // 64 features = 32 bytes = 16-byte chunks c0, c0 + 1 of K tile f0 / 256 of the A2 tile
+          const int a2_kt = f0 >> 8, c0 = (f0 & 255) >> 5;
+          *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.d_k_tiles, a2_kt, row_in_tile, c0)) =
+              make_uint4(codes[0], codes[1], codes[2], codes[3]);
+          *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.d_k_tiles, a2_kt, row_in_tile,
+                                                              c0 + 1)) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+          // the 4 scales of this K-group (features f0..f0+63) are 4 contiguous bytes
+          *reinterpret_cast<uint32_t*>(args.a2_sf + sf_atom_offset(mb.sf_block, args.d_k_tiles * 4, row_in_tile,
+                                                                   f0 / 16)) = scodes;
         }
-        // 64 features = 32 bytes = 16-byte chunks c0, c0 + 1 of K tile f0 / 256 of the A2 tile
-        const int a2_kt = f0 >> 8, c0 = (f0 & 255) >> 5;
-        *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.a2_k_tiles, a2_kt, row_in_tile, c0)) =
-            make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.a2_k_tiles, a2_kt, row_in_tile, c0 + 1)) =
-            make_uint4(codes[4], codes[5], codes[6], codes[7]);
-        // the 4 scales of this K-group (features f0..f0+63) are 4 contiguous bytes
-        *reinterpret_cast<uint32_t*>(args.a2_sf + sf_atom_offset(mb.sf_block, args.a2_kgroups, row_in_tile,
-                                                                 f0 / 16)) = scodes;
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(args.y + r * args.y_cols + nt * BN + half * 128);
+        // publish this warp's share of block t.block's A2 to the down-tile producers
+        fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(ready + t.block, 1u);
+        }
+      } else if (valid) {
+        const float scale = args.alpha_a2 * __ldg(args.w_d_alpha + mb.expert);
+        const size_t r = static_cast<size_t>(mb.row_begin + row_in_tile);
+        uint4* dst = reinterpret_cast<uint4*>(args.y + r * args.y_cols + t.nt * BN + half * 128);
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const int c = q * 8;
@@ -301,23 +447,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-template <int EPI, class R>
-static cudaError_t launch_ring(const GemmArgs& a, int grid, cudaStream_t s) {
+template <class R>
+static cudaError_t launch_ring(const ExpertGemmArgs& a, int grid, cudaStream_t s) {
   const size_t smem = ring_smem_bytes<R>();
-  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<EPI, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(gemm_experts_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(gemm_nvfp4_kernel<EPI, R>, dim3(grid), dim3(NUM_THREADS), smem, s, a);
+  return launch_pdl(gemm_experts_kernel<R>, dim3(grid), dim3(NUM_THREADS), smem, s, a);
 }
 
-template <int EPI>
-static cudaError_t launch_gemm(const GemmArgs& a, int grid, cudaStream_t s) {
+cudaError_t launch_gemm_experts(const ExpertGemmArgs& a, int grid, cudaStream_t s) {
   // With at most 32 tokens no expert has more than 32 rows.
-  if (a.max_rows_per_expert <= 32) return launch_ring<EPI, RingSmallM>(a, grid, s);
-  return launch_ring<EPI, RingFull>(a, grid, s);
+  if (a.max_rows_per_expert <= 32) return launch_ring<RingSmallM>(a, grid, s);
+  return launch_ring<RingFull>(a, grid, s);
 }
-
-cudaError_t launch_gemm_gate_up(const GemmArgs& a, int grid, cudaStream_t s) { return launch_gemm<kSwiGLU>(a, grid, s); }
-cudaError_t launch_gemm_down(const GemmArgs& a, int grid, cudaStream_t s) { return launch_gemm<kStoreBF16>(a, grid, s); }
 
 }  // namespace beam

@@ -27,7 +27,9 @@ cudaError_t launch_topk(const float* logits, int splits, int T, int E, int k, in
                         cudaStream_t s);
 
 // ---- router on the tensor cores for large batches (router_tc.cu)
-constexpr int kRouterTcMinTokens = 1024;
+// One CTA per 128 tokens, each streaming all of W_r: below ~32 CTAs the split-H SIMT
+// router (router.cu) fills more of the GPU and is faster (0.11 vs 0.32 ms at T = 1024).
+constexpr int kRouterTcMinTokens = 4096;
 bool router_tc_supported(int T, int H, int E, int k);
 size_t router_tc_smem_bytes(int E);
 cudaError_t launch_split_router(const float* w, int E, int H, uint16_t* out, cudaStream_t s);
@@ -38,20 +40,26 @@ cudaError_t launch_router_tc(const CUtensorMap& map_x, const uint16_t* w_tiles, 
 
 // ---- routing of a small batch in one launch (route_small.cu)
 bool route_small_supported(int T, int H, int E, int k);
-cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, int E, int k, float* logits,
+int64_t route_small_ws_floats(int T, int H, int E);  // partial logits [S][T][E]
+// part: [S][T][E] partial logits over S slices of H; *slices = S.
+cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, int E, int k, float* part,
                                int32_t* ids, float* wout, int32_t* offsets, int32_t* sf_block, MBlock* mblocks,
-                               int32_t* num_mblocks, int32_t* perm, int32_t* inv, unsigned int* done_counter,
+                               int32_t* num_mblocks, int32_t* perm, int32_t* inv, int32_t* tile_row,
+                               unsigned int* done_counter, uint32_t* sched, int sched_n, uint32_t* err, int* slices,
                                cudaStream_t s);
 
 // ---- permutation and activation quantisation (routing.cu)
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s);
+// Also zeroes sched[0, sched_n), the tile scheduler words of the expert GEMM launch.
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
-                        int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, cudaStream_t s);
-cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, int T, int k, int E, int32_t* perm_src,
-                           int32_t* inv, cudaStream_t s);
-cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* ids, const int32_t* inv, const int32_t* offsets,
-                            const int32_t* sf_block, int T, int H, int k, float alpha, uint8_t* a1, uint8_t* a1_sf,
-                            cudaStream_t s);
+                        int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
+                        cudaStream_t s);
+// tile_row[t][j] = 128 x activation block + row within it, for slot (t, j).
+cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,
+                           const int32_t* sf_block, int T, int k, int E, int32_t* perm_src, int32_t* inv,
+                           int32_t* tile_row, cudaStream_t s);
+cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, float alpha, uint8_t* a1,
+                            uint8_t* a1_sf, cudaStream_t s);
 
 // ---- weight quantiser and repacking (quant.cu)
 // Contiguous weight tiles of the grouped GEMMs: 256 rows x 256 K values of codes in the
@@ -67,37 +75,44 @@ cudaError_t launch_quantize_rows(const float* src, int64_t rows, int64_t cols, f
                                  uint8_t* codes, uint8_t* sf, cudaStream_t s);
 cudaError_t launch_amax(const float* src, int64_t n, float* amax_bits, cudaStream_t s);
 cudaError_t launch_amax_to_alpha(float* inout, cudaStream_t s);
-// ---- grouped NVFP4 GEMMs (gemm_nvfp4.cu)
-struct GemmArgs {
+// ---- grouped NVFP4 GEMMs, gate/up and down in one launch (gemm_nvfp4.cu)
+// Activation tiles are [blk][K/256][16384] (act_tile_offset), their scales [blk][K/64][512]
+// (sf_atom_offset); weight tiles are [E][n_tiles][K/256][kTileBytes].
+struct ExpertGemmArgs {
   const MBlock* mblocks;
   const int32_t* num_mblocks;
   int max_rows_per_expert;  // an upper bound (the number of tokens) used to pick the ring shape
-  int n_tiles;        // output tiles of 256 columns per 128-row block
-  int k_tiles;        // K / 256
-  const uint8_t* a_tiles;  // activation tiles [blk][k_tiles][16384] (act_tile_offset)
-  const uint8_t* b_tiles;  // weight tiles [E][n_tiles][k_tiles][kTileBytes]
-  const uint8_t* sfa; // activation scale blocks [blk][K/64][512]
-  const float* alpha_b;  // [E]
-  float alpha_a;
-  // gate/up epilogue: SwiGLU + NVFP4 of h
-  uint8_t* a2;        // activation tiles [blk][Ip/256][16384]
-  uint8_t* a2_sf;     // [blk][Ip/64][512]
-  int a2_k_tiles;     // Ip/256
-  int a2_kgroups;     // Ip/64
+  // gate/up: K = H, 256 B rows per output tile = 128 gate + 128 up features
+  int gu_n_tiles;           // I / 128
+  int gu_k_tiles;           // H / 256
+  const uint8_t* a1;
+  const uint8_t* a1_sf;
+  const uint8_t* w_gu;
+  const float* w_gu_alpha;  // [E]
+  float alpha_a1;
+  // SwiGLU + NVFP4 epilogue output, the down GEMM's A operand (K = Ip)
+  uint8_t* a2;
+  uint8_t* a2_sf;
   float alpha_a2;
-  // down epilogue: BF16 rows
-  uint16_t* y;        // [rows][H]
-  int y_cols;         // H
+  // down: K = Ip
+  int d_n_tiles;            // H / 256
+  int d_k_tiles;            // Ip / 256
+  const uint8_t* w_d;
+  const float* w_d_alpha;   // [E]
+  uint16_t* y;              // [rows][H] BF16
+  int y_cols;               // H
+  // [0]: next tile to claim; [1 + b]: gate/up epilogue warps done on block b.
+  // sched_words(nblk_max) words, zeroed by the routing kernel (two or more launches back).
+  uint32_t* sched;
   uint32_t* err;
 };
-cudaError_t launch_gemm_gate_up(const GemmArgs& a, int grid, cudaStream_t s);
-cudaError_t launch_gemm_down(const GemmArgs& a, int grid, cudaStream_t s);
-size_t gemm_smem_bytes();
+inline int64_t sched_words(int64_t nblk_max) { return 1 + nblk_max; }
+cudaError_t launch_gemm_experts(const ExpertGemmArgs& a, int grid, cudaStream_t s);
 
 // ---- finalize (finalize.cu)
 // next_x != nullptr also writes the next sublayer's pre-norm of out: bf16(out * rinv * next_gamma).
 cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
                             const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, uint16_t* next_x,
-                            const uint16_t* next_gamma, float next_eps, cudaStream_t s);
+                            const uint16_t* next_gamma, float next_eps, uint32_t* err, cudaStream_t s);
 
 }  // namespace beam

@@ -1,14 +1,18 @@
 // Routing of a small batch (T <= 16 tokens, E <= 256 experts) in one launch: router
 // logits, top-k + renormalise, histogram, scan, permutation and the 128-row work blocks.
 //
-// Phase 1 (every CTA): each CTA streams the rows W_r[e] of 4 experts (20 KB each at
-// H = 5120) into registers, stages x (T x H BF16) once in shared memory, and dots every
-// token with the 4 rows in FP32.  All loads are issued before any multiply; the step is
-// bound by reading W_r.
+// Phase 1 (every CTA): CTA (g, s) owns experts [8g, 8g + 8) (one warp each) and slice s of
+// the S slices of H.  Its W_r row slices (constant: loaded before the wait for the previous
+// kernel) and the x slice (T x H/S BF16) arrive in shared memory by bulk copies, one per
+// row; each warp dots every token with its row slice in FP32 and a warp reduction gives one
+// partial logit per (token, expert), stored to part[S][T][E].  Splitting H keeps each
+// CTA's share of W_r and of x small, so 128 CTAs (E = 256, S = 4) stream W_r at once.
 // Phase 2 (the last CTA to finish, found with an atomic counter after a release fence):
-// top-k per token (one warp per token), then the histogram, the prefix sums and the
-// stable permutation for the whole batch, as routing.cu does in three launches for large
-// batches.  The counter is reset by that CTA, ready for the next launch.
+// one bulk copy brings every partial; logit = sum of the S partials in slice order, top-k
+// per token (one warp per token), then
+// the histogram, the prefix sums and the stable permutation for the whole batch, as
+// routing.cu does in three launches for large batches.  The counter is reset by that CTA,
+// ready for the next launch, and so are the tile scheduler words of the expert GEMM.
 // Router (5120 -> 256 experts, FP32): vLLM PR "Day-0 support for Reflection's Beam-1.0",
 // section "Status"; news article "vLLM adds day-zero Reflection Beam serving", section
 // "Agents worked on the serving path".  8 of 256 experts: recipe
@@ -20,78 +24,97 @@
 namespace beam {
 
 constexpr int kSmallThreads = 256;
-constexpr int kExpertsPerCta = 4;       // x is staged once per CTA and reused for 4 experts
-constexpr int kMaxChunksPerThread = 8;  // H / 4 / 256 <= 8  ->  H <= 8192
+constexpr int kSmallExpertsPerCta = kSmallThreads / 32;  // one warp per expert
+constexpr int kSmallMaxF4 = 16;                          // 16-byte W pieces per lane: H / S <= 2048
 
+// Number of H slices: the largest S in {4, 2, 1} whose slice is a whole number of
+// 512-byte warp rows (32 lanes x 4 floats) and at most kSmallMaxF4 of them; 0 = unsupported.
+int route_small_slices(int H) {
+  for (int S = 4; S >= 1; S >>= 1)
+    if (H % (S * 128) == 0 && H / S / 128 <= kSmallMaxF4) return S;
+  return 0;
+}
+
+// Dynamic shared memory: phase 1 holds the CTA's W_r row slices and the x slice, phase 2
+// (last CTA) all partial logits.
+static size_t route_small_smem(int T, int H, int E) {
+  const int S = route_small_slices(H), Hs = H / S;
+  const size_t p1 = static_cast<size_t>(kSmallExpertsPerCta) * Hs * 4 + static_cast<size_t>(T) * Hs * 2;
+  const size_t p2 = static_cast<size_t>(S) * T * E * 4;
+  return p1 > p2 ? p1 : p2;
+}
+
+template <int MAXT>
 __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
-    const uint16_t* __restrict__ x, const float* __restrict__ w, int T, int H, int E, int k,
-    float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout, int32_t* __restrict__ offsets,
+    const uint16_t* __restrict__ x, const float* __restrict__ w, int T, int H, int E, int k, int S,
+    float* __restrict__ part, int32_t* __restrict__ ids, float* __restrict__ wout, int32_t* __restrict__ offsets,
     int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks, int32_t* __restrict__ num_mblocks,
-    int32_t* __restrict__ perm, int32_t* __restrict__ inv, unsigned int* __restrict__ done_counter) {
-  extern __shared__ __align__(16) uint16_t xs[];  // [T][H] BF16
-  const int e0 = blockIdx.x * kExpertsPerCta;
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, int32_t* __restrict__ tile_row,
+    unsigned int* __restrict__ done_counter, uint32_t* __restrict__ sched, int sched_n, uint32_t* __restrict__ err) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t bars[3];  // W slices, x slice, partial logits
+  __shared__ int s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int n4 = H / 4;
-  // ---------------------------------------------------------------- phase 1: logits
-  {
-    // The router weights are constant: stream this CTA's rows before waiting for the
-    // previous kernel in the stream.
-    float4 wv[kExpertsPerCta][kMaxChunksPerThread];
+  const int hs = blockIdx.x % S, g = blockIdx.x / S;
+  const int Hs = H / S, h0 = hs * Hs;
+  const int nf4 = Hs / 128;
+  const int e0 = g * kSmallExpertsPerCta, n_e = min(kSmallExpertsPerCta, E - e0);
+  float* ws = reinterpret_cast<float*>(smem);                                              // [8][Hs] FP32
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kSmallExpertsPerCta * Hs * 4);         // [T][Hs] BF16
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // ---------------------------------------------------------------- phase 1: partial logits
+  // Each slice row is one bulk copy.  The router weights are constant: they stream before
+  // the wait for the previous kernel in the stream; x after it.
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], static_cast<uint32_t>(n_e * Hs * 4));
+    for (int q = 0; q < n_e; ++q)
+      bulk_load(ws + q * Hs, w + static_cast<size_t>(e0 + q) * H + h0, Hs * 4, &bars[0]);
+  }
+  pdl_wait();
+  pdl_trigger();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[1], static_cast<uint32_t>(T * Hs * 2));
+    for (int t = 0; t < T; ++t) bulk_load(xs + t * Hs, x + static_cast<size_t>(t) * H + h0, Hs * 2, &bars[1]);
+  }
+  const bool ok_w = mbar_wait_bounded(&bars[0], 0, &s_abort);
+  const bool ok = mbar_wait_bounded(&bars[1], 0, &s_abort) && ok_w;
+  if (!ok) {
+    if (lane == 0) atomicOr(err, kErrTimeoutProducer);
+  } else if (warp < n_e) {
+    // All tokens at once: one W piece per step, then MAXT independent FMA chains (rows
+    // past T repeat row 0 and are dropped), so the smem loads and FMAs overlap.
+    const float4* wr = reinterpret_cast<const float4*>(ws + warp * Hs);
+    float acc[MAXT];
 #pragma unroll
-    for (int q = 0; q < kExpertsPerCta; ++q) {
-      const float4* wr = reinterpret_cast<const float4*>(w + static_cast<size_t>(min(e0 + q, E - 1)) * H);
+    for (int t = 0; t < MAXT; ++t) acc[t] = 0.0f;
+    for (int i = 0; i < nf4; ++i) {
+      const float4 wq = wr[lane + 32 * i];
 #pragma unroll
-      for (int i = 0; i < kMaxChunksPerThread; ++i) {
-        const int c = tid + i * kSmallThreads;
-        wv[q][i] = (c < n4 && e0 + q < E) ? __ldg(wr + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int t = 0; t < MAXT; ++t) {
+        const int tt = t < T ? t : 0;
+        const uint2 xv = reinterpret_cast<const uint2*>(xs + tt * Hs)[lane + 32 * i];
+        acc[t] = fmaf(bf16_bits_to_f32(xv.x & 0xFFFFu), wq.x, acc[t]);
+        acc[t] = fmaf(bf16_bits_to_f32(xv.x >> 16), wq.y, acc[t]);
+        acc[t] = fmaf(bf16_bits_to_f32(xv.y & 0xFFFFu), wq.z, acc[t]);
+        acc[t] = fmaf(bf16_bits_to_f32(xv.y >> 16), wq.w, acc[t]);
       }
     }
-    pdl_wait();
-    pdl_trigger();
-    {  // x -> shared memory: asynchronous 16-byte copies, all in flight at once
-      const int n16 = T * H / 8;
-      const uint4* xg = reinterpret_cast<const uint4*>(x);
-      for (int i = tid; i < n16; i += kSmallThreads)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(xs + 8 * i)), "l"(xg + i) : "memory");
-      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+    for (int t = 0; t < MAXT; ++t) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
     }
-    __syncthreads();
-    __shared__ float part[kSmallThreads / 32][kExpertsPerCta][kMaxSmallRouterTokens];
-    for (int t = 0; t < T; ++t) {
-      const uint2* xr = reinterpret_cast<const uint2*>(xs + static_cast<size_t>(t) * H);
-      float acc[kExpertsPerCta] = {};
+    if (lane < T) {  // lane t stores token t's partial (selected without dynamic indexing)
+      float mine = acc[0];
 #pragma unroll
-      for (int i = 0; i < kMaxChunksPerThread; ++i) {
-        const int c = tid + i * kSmallThreads;
-        if (c < n4) {
-          const uint2 xv = xr[c];
-          const float x0 = bf16_bits_to_f32(xv.x & 0xFFFFu), x1 = bf16_bits_to_f32(xv.x >> 16);
-          const float x2 = bf16_bits_to_f32(xv.y & 0xFFFFu), x3 = bf16_bits_to_f32(xv.y >> 16);
-#pragma unroll
-          for (int q = 0; q < kExpertsPerCta; ++q) {
-            acc[q] = fmaf(x0, wv[q][i].x, acc[q]);
-            acc[q] = fmaf(x1, wv[q][i].y, acc[q]);
-            acc[q] = fmaf(x2, wv[q][i].z, acc[q]);
-            acc[q] = fmaf(x3, wv[q][i].w, acc[q]);
-          }
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < kExpertsPerCta; ++q) {
-        float a = acc[q];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (lane == 0) part[warp][q][t] = a;
-      }
-    }
-    __syncthreads();
-    for (int i = tid; i < kExpertsPerCta * T; i += kSmallThreads) {
-      const int q = i / T, t = i % T;
-      if (e0 + q >= E) continue;
-      float v = 0.0f;
-#pragma unroll
-      for (int g = 0; g < kSmallThreads / 32; ++g) v += part[g][q][t];
-      logits[static_cast<size_t>(t) * E + e0 + q] = v;
+      for (int t = 1; t < MAXT; ++t)
+        if (lane == t) mine = acc[t];
+      part[(static_cast<size_t>(hs) * T + lane) * E + e0 + warp] = mine;
     }
   }
   // ---------------------------------------------------------------- elect the last CTA
@@ -104,25 +127,45 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
   __threadfence();
 
   // ---------------------------------------------------------------- phase 2: top-k
+  // All partial logits in one bulk copy (the other CTAs' stores were released before
+  // their counter increment; the proxy fence orders them before this copy).
+  float* ps = reinterpret_cast<float*>(smem);  // [S][T][E]
+  if (tid == 0) {
+    fence_proxy_async_global();
+    fence_proxy_async_smem();  // phase 1's reads of this shared memory are done (barrier above)
+    const uint32_t bytes = static_cast<uint32_t>(S * T * E * 4);
+    mbar_arrive_expect_tx(&bars[2], bytes);
+    bulk_load(ps, part, bytes, &bars[2]);
+  }
+  // the expert GEMM launch that follows starts from zeroed scheduler words
+  for (int i = tid; i < sched_n; i += kSmallThreads) sched[i] = 0u;
   __shared__ int s_ids[kMaxSmallRouterTokens * 16];
   __shared__ int s_cnt[256];
   __shared__ int s_off[256];
+  __shared__ int s_blk[256];
   __shared__ int warp_sums[33];
+  for (int i = tid; i < E; i += kSmallThreads) s_cnt[i] = 0;
+  if (!mbar_wait_bounded(&bars[2], 0, &s_abort)) {
+    if (tid == 0) atomicOr(err, kErrTimeoutProducer);
+  }
+  const int TE = T * E;
   for (int t = warp; t < T; t += kSmallThreads / 32) {
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int ee = lane + 32 * i;
-      v[i] = ee < E ? __ldcg(logits + static_cast<size_t>(t) * E + ee) : -INFINITY;
+      float sum = 0.0f;
+      for (int q = 0; q < S; ++q) sum += ee < E ? ps[q * TE + t * E + ee] : 0.0f;  // slice order
+      v[i] = ee < E ? sum : -INFINITY;
     }
-    warp_topk<8>(v, E, k, lane, ids + static_cast<size_t>(t) * k, wout + static_cast<size_t>(t) * k);
+    warp_topk<8>(v, E, k, lane, s_ids + t * k, wout + static_cast<size_t>(t) * k);
   }
-  __syncthreads();  // ids of this CTA's writes are visible to the CTA after the barrier
-  const int R = T * k;
-  for (int i = tid; i < R; i += kSmallThreads) s_ids[i] = ids[i];
-  for (int i = tid; i < E; i += kSmallThreads) s_cnt[i] = 0;
   __syncthreads();
-  for (int i = tid; i < R; i += kSmallThreads) atomicAdd(&s_cnt[s_ids[i]], 1);
+  const int R = T * k;
+  for (int i = tid; i < R; i += kSmallThreads) {
+    ids[i] = s_ids[i];
+    atomicAdd(&s_cnt[s_ids[i]], 1);
+  }
   __syncthreads();
   // ---------------------------------------------------------------- scan and work blocks
   const int cnt = tid < E ? s_cnt[tid] : 0;
@@ -134,6 +177,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     offsets[tid] = off;
     sf_block[tid] = blk;
     s_off[tid] = off;
+    s_blk[tid] = blk;
     for (int i = 0; i < nblk; ++i) {
       MBlock m;
       m.expert = tid;
@@ -158,26 +202,36 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     const int r = s_off[ee] + rank;
     perm[r] = t;
     inv[i] = r;
+    tile_row[i] = (s_blk[ee] + (rank >> 7)) * 128 + (rank & 127);
   }
   if (tid == 0) *done_counter = 0u;
 }
 
 bool route_small_supported(int T, int H, int E, int k) {
-  return T >= 1 && T <= kMaxSmallRouterTokens && E <= 256 && k <= 16 && H / 4 <= kMaxChunksPerThread * kSmallThreads &&
-         static_cast<size_t>(T) * H * 2 <= 160 * 1024;
+  // partial logits move as one bulk copy: S * T * E * 4 bytes, a multiple of 16
+  return T >= 1 && T <= kMaxSmallRouterTokens && E >= 1 && E <= 256 && E % 4 == 0 && k <= 16 &&
+         route_small_slices(H) > 0 && route_small_smem(T, H, E) <= 160 * 1024;
 }
 
-cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, int E, int k, float* logits,
+int64_t route_small_ws_floats(int T, int H, int E) {
+  return static_cast<int64_t>(route_small_slices(H)) * T * E;
+}
+
+cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, int E, int k, float* part,
                                int32_t* ids, float* wout, int32_t* offsets, int32_t* sf_block, MBlock* mblocks,
-                               int32_t* num_mblocks, int32_t* perm, int32_t* inv, unsigned int* done_counter,
+                               int32_t* num_mblocks, int32_t* perm, int32_t* inv, int32_t* tile_row,
+                               unsigned int* done_counter, uint32_t* sched, int sched_n, uint32_t* err, int* slices,
                                cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(T) * H * sizeof(uint16_t);
-  cudaError_t e = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  const int S = route_small_slices(H);
+  *slices = S;
+  const size_t smem = route_small_smem(T, H, E);
+  const int groups = (E + kSmallExpertsPerCta - 1) / kSmallExpertsPerCta;
+  auto kernel = T <= 8 ? route_small_kernel<8> : route_small_kernel<kMaxSmallRouterTokens>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(route_small_kernel, dim3((E + kExpertsPerCta - 1) / kExpertsPerCta), dim3(kSmallThreads), smem,
-                    s, x, w, T, H, E, k, logits, ids, wout, offsets, sf_block, mblocks, num_mblocks, perm, inv,
-                    done_counter);
+  return launch_pdl(kernel, dim3(groups * S), dim3(kSmallThreads), smem, s, x, w, T, H, E, k, S, part, ids, wout,
+                    offsets, sf_block, mblocks, num_mblocks, perm, inv, tile_row, done_counter, sched, sched_n,
+                    err);
 }
 
 }  // namespace beam

@@ -40,10 +40,12 @@ __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restri
 __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chunks, int E,
                             int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
                             int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks,
-                            int32_t* __restrict__ num_mblocks) {
+                            int32_t* __restrict__ num_mblocks, uint32_t* __restrict__ sched, int sched_n) {
   __shared__ int warp_sums[33];
   pdl_wait();
   pdl_trigger();
+  // the expert GEMM launch that follows starts from zeroed scheduler words
+  for (int i = threadIdx.x; i < sched_n; i += blockDim.x) sched[i] = 0u;
   const int e = threadIdx.x;
   int cnt = 0;
   if (e < E) {
@@ -78,10 +80,15 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
   }
 }
 
-// perm_src[r] = t and inv[t][j] = r for every (t, j) of one chunk of 256 tokens.
+// perm_src[r] = t, inv[t][j] = r and tile_row[t][j] (128 x activation block + row in the
+// block, the row's place in the activation tiles) for every (t, j) of one chunk of 256
+// tokens.
 __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ ids,
-                                                      const int32_t* __restrict__ chunk_base, int T, int k, int E,
-                                                      int32_t* __restrict__ perm_src, int32_t* __restrict__ inv) {
+                                                      const int32_t* __restrict__ chunk_base,
+                                                      const int32_t* __restrict__ offsets,
+                                                      const int32_t* __restrict__ sf_block, int T, int k, int E,
+                                                      int32_t* __restrict__ perm_src, int32_t* __restrict__ inv,
+                                                      int32_t* __restrict__ tile_row) {
   extern __shared__ uint32_t sm[];
   uint32_t* mask = sm;                                    // [8][E]
   int32_t* pre = reinterpret_cast<int32_t*>(sm + 8 * E);  // [8][E]
@@ -110,8 +117,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
       const int e = ids[static_cast<size_t>(t) * k + j];
       const int rank = pre[warp * E + e] + __popc(mask[warp * E + e] & below);
       const int r = chunk_base[static_cast<size_t>(chunk) * E + e] + rank;
+      const int li = r - offsets[e];  // row within the expert
       perm_src[r] = t;
       inv[static_cast<size_t>(t) * k + j] = r;
+      tile_row[static_cast<size_t>(t) * k + j] = (sf_block[e] + (li >> 7)) * 128 + (li & 127);
     }
   }
 }
@@ -120,10 +129,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
 // permuted rows.  The four threads of one 64-value group (one scale word of the
 // tensor-core layout) combine their scale bytes and one of them stores the 32-bit word.
 __global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restrict__ x,
-                                                       const int32_t* __restrict__ ids,
-                                                       const int32_t* __restrict__ inv,
-                                                       const int32_t* __restrict__ offsets,
-                                                       const int32_t* __restrict__ sf_block, int T, int H, int k,
+                                                       const int32_t* __restrict__ tile_row, int T, int H, int k,
                                                        float alpha, uint8_t* __restrict__ a1,
                                                        uint8_t* __restrict__ a1_sf) {
   const int nb = H / 16, kgroups = H / 64;
@@ -135,16 +141,13 @@ __global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restric
   pdl_wait();
   pdl_trigger();
   uint32_t lo = 0, hi = 0, sc = 0;
-  int r[16], e[16];
+  int dst[16];
   if (active) {
     const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
     const uint4 p0 = __ldg(xr + 2 * b), p1 = __ldg(xr + 2 * b + 1);
 #pragma unroll
-    for (int j = 0; j < 16; ++j)  // all slot indices in flight together
-      if (j < k) {
-        r[j] = __ldg(inv + static_cast<size_t>(t) * k + j);
-        e[j] = __ldg(ids + static_cast<size_t>(t) * k + j);
-      }
+    for (int j = 0; j < 16; ++j)  // all slot rows in flight together
+      dst[j] = j < k ? __ldg(tile_row + static_cast<size_t>(t) * k + j) : 0;
     const uint32_t u[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
     float v[16];
 #pragma unroll
@@ -163,8 +166,7 @@ __global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restric
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     if (j >= k) break;
-    const int li = r[j] - __ldg(offsets + e[j]);
-    const int blk = __ldg(sf_block + e[j]) + (li >> 7), m = li & 127;
+    const int blk = dst[j] >> 7, m = dst[j] & 127;
     // block b of 16 values: 8 bytes, half of 16-byte chunk (b % 16) / 2 of K tile b / 16
     *reinterpret_cast<uint2*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1) + (b & 1) * 8) =
         make_uint2(lo, hi);
@@ -174,11 +176,8 @@ __global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restric
 
 // Large batches: one warp per token, quantise x[t] once, write it to the token's k rows.
 __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __restrict__ x,
-                                                       const int32_t* __restrict__ ids,
-                                                       const int32_t* __restrict__ inv,
-                                                       const int32_t* __restrict__ offsets,
-                                                       const int32_t* __restrict__ sf_block, int T, int H, int k,
-                                                       float alpha, uint8_t* __restrict__ a1,
+                                                       const int32_t* __restrict__ tile_row, int T, int H,
+                                                       int k, float alpha, uint8_t* __restrict__ a1,
                                                        uint8_t* __restrict__ a1_sf) {
   __shared__ int s_blk[8][16], s_m[8][16];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -188,11 +187,9 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
   if (t >= T) return;
   // lane j < k: the permuted row of slot j and where its scales live
   if (lane < k) {
-    const int r = inv[static_cast<size_t>(t) * k + lane];
-    const int e = ids[static_cast<size_t>(t) * k + lane];
-    const int li = r - offsets[e];
-    s_blk[warp][lane] = sf_block[e] + (li >> 7);
-    s_m[warp][lane] = li & 127;
+    const int d = tile_row[static_cast<size_t>(t) * k + lane];
+    s_blk[warp][lane] = d >> 7;
+    s_m[warp][lane] = d & 127;
   }
   __syncwarp();
   const float six_alpha = __fmul_rn(6.0f, alpha);
@@ -225,14 +222,16 @@ cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* 
 }
 
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
-                        int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, cudaStream_t s) {
+                        int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
+                        cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
   return launch_pdl(scan_kernel, dim3(1), dim3(threads), 0, s, chunk_counts, n_chunks, E, chunk_base, offsets,
-                    sf_block, mblocks, num_mblocks);
+                    sf_block, mblocks, num_mblocks, sched, sched_n);
 }
 
-cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, int T, int k, int E, int32_t* perm_src,
-                           int32_t* inv, cudaStream_t s) {
+cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,
+                           const int32_t* sf_block, int T, int k, int E, int32_t* perm_src, int32_t* inv,
+                           int32_t* tile_row, cudaStream_t s) {
   const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
   const size_t smem = static_cast<size_t>(16) * E * sizeof(uint32_t);
   if (smem > 48 * 1024) {
@@ -240,18 +239,17 @@ cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, int T,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(scatter_kernel, dim3(n_chunks), dim3(256), smem, s, ids, chunk_base, T, k, E, perm_src, inv);
+  return launch_pdl(scatter_kernel, dim3(n_chunks), dim3(256), smem, s, ids, chunk_base, offsets, sf_block, T, k, E,
+                    perm_src, inv, tile_row);
 }
 
-cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* ids, const int32_t* inv, const int32_t* offsets,
-                            const int32_t* sf_block, int T, int H, int k, float alpha, uint8_t* a1, uint8_t* a1_sf,
-                            cudaStream_t s) {
+cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, float alpha, uint8_t* a1,
+                            uint8_t* a1_sf, cudaStream_t s) {
   if (T >= 256)
-    return launch_pdl(quant_a1_wide_kernel, dim3((T + 7) / 8), dim3(256), 0, s, x, ids, inv, offsets, sf_block, T, H,
-                      k, alpha, a1, a1_sf);
+    return launch_pdl(quant_a1_wide_kernel, dim3((T + 7) / 8), dim3(256), 0, s, x, tile_row, T, H, k, alpha, a1, a1_sf);
   const int64_t threads = static_cast<int64_t>(T) * (H / 16);
-  return launch_pdl(quant_a1_kernel, dim3(static_cast<unsigned>((threads + 127) / 128)), dim3(128), 0, s, x, ids, inv,
-                    offsets, sf_block, T, H, k, alpha, a1, a1_sf);
+  return launch_pdl(quant_a1_kernel, dim3(static_cast<unsigned>((threads + 127) / 128)), dim3(128), 0, s, x, tile_row,
+                    T, H, k, alpha, a1, a1_sf);
 }
 
 }  // namespace beam
