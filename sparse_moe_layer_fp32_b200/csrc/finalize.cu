@@ -147,8 +147,10 @@ __global__ void __launch_bounds__(kFinThreads) finalize_wide_kernel(const uint16
 // handful of CTAs must move each token's k rows of y, so the loads go through the copy
 // engine rather than per-thread loads).  The residual row and gamma (and the next gamma) do
 // not depend on the GEMM and are copied before the wait for it; inv and w come from the
-// routing, two launches back, and are read first.  Each thread owns 8-value chunks; the
-// weighted sums are recomputed from shared memory in each pass instead of being kept.
+// routing, two launches back, and are read first.  The last warp only issues the copies (a
+// thread that issues copies runs its warp's math several times slower afterwards); the
+// other threads own 8-value chunks, and the weighted sums are recomputed from shared
+// memory in each pass instead of being kept.
 template <bool PRE>
 __global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __restrict__ y,
                                                               const float* __restrict__ w,
@@ -167,6 +169,8 @@ __global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __
   __shared__ float s_red[32];
   __shared__ int s_abort;
   const int t = blockIdx.x;
+  const int nc = static_cast<int>(blockDim.x) - 32;  // compute threads; thread nc issues the copies
+  const bool copier = static_cast<int>(threadIdx.x) == nc;
   const uint32_t row_bytes = static_cast<uint32_t>(H) * 2;
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
@@ -179,7 +183,7 @@ __global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __
     s_w[threadIdx.x] = __ldcg(w + static_cast<size_t>(t) * k + threadIdx.x);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (copier) {
     mbar_arrive_expect_tx(&bars[0], (PRE ? 3u : 2u) * row_bytes);
     bulk_load(rs, residual + static_cast<size_t>(t) * H, row_bytes, &bars[0]);  // out may alias residual
     bulk_load(gs, gamma, row_bytes, &bars[0]);
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __
   }
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x == 0) {
+  if (copier) {
     mbar_arrive_expect_tx(&bars[1], static_cast<uint32_t>(k) * row_bytes);
     for (int j = 0; j < k; ++j)
       bulk_load(ys + static_cast<size_t>(j) * H, y + static_cast<size_t>(s_row[j]) * H, row_bytes, &bars[1]);
@@ -195,7 +199,9 @@ __global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __
   const bool ok0 = mbar_wait_bounded(&bars[0], 0, &s_abort);
   const bool ok1 = mbar_wait_bounded(&bars[1], 0, &s_abort);
   if (!(ok0 && ok1) && threadIdx.x == 0) atomicOr(err, kErrTimeoutEpilogue);
+  __syncwarp();  // every lane left the polling loop on its own: reconverge before the math
   const int nchunks = H / 8;
+  const int c0 = static_cast<int>(threadIdx.x) < nc ? static_cast<int>(threadIdx.x) : nchunks;  // copy warp: none
   // m[c] = sum_j w_j y_j over this chunk's 8 values, in slot order
   auto weighted = [&](int c, float (&m)[8]) {
 #pragma unroll
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __
     return make_uint4(o[0], o[1], o[2], o[3]);
   };
   float ss = 0.0f;
-  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+  for (int c = c0; c < nchunks; c += nc) {
     float m[8];
     weighted(c, m);
 #pragma unroll
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __
   }
   const float rinv = block_rinv(ss, H, eps, s_red);
   float ss2 = 0.0f;
-  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+  for (int c = c0; c < nchunks; c += nc) {
     float m[8];
     weighted(c, m);
     const uint4 ov = out_chunk(c, rinv, m);
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(1024) finalize_small_kernel(const uint16_t* __
   }
   if constexpr (PRE) {
     const float r2 = block_rinv(ss2, H, nn.eps, s_red);
-    for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+    for (int c = c0; c < nchunks; c += nc) {
       float m[8], f[8], g[8];
       weighted(c, m);
       unpack8(out_chunk(c, rinv, m), f);  // the same BF16 values as stored above
@@ -266,7 +272,7 @@ static cudaError_t launch_finalize_t(const uint16_t* y, const float* w, const in
     cudaError_t e = cudaFuncSetAttribute(finalize_small_kernel<PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(small));
     if (e != cudaSuccess) return e;
-    const int threads = std::min(1024, ((nchunks + 31) / 32) * 32);
+    const int threads = std::min(1024, ((nchunks + 31) / 32) * 32 + 32);  // + the copy warp
     return launch_pdl(finalize_small_kernel<PRE>, dim3(T), dim3(threads), small, s, y, w, inv, residual, gamma, H, k,
                       eps, out, nn, err);
   }

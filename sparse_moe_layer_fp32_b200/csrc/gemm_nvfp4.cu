@@ -19,7 +19,7 @@
 // waits on anything, so every awaited tile is held by a running CTA: no deadlock, and no
 // need for all CTAs to be resident at once.
 //
-// CTA layout (one persistent CTA per SM, 320 threads, warp-specialised):
+// CTA layout (one persistent CTA per SM, 576 threads, warp-specialised):
 //   warp 0      producer: claims tiles, publishes each tile id through a small shared
 //               ring, and per 256-wide K step bulk-copies the A tile (the valid rows of a
 //               128-row activation tile, <= 16 KB), the expert's weight tile with its
@@ -30,9 +30,11 @@
 //   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scales -> TMEM) and
 //               tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128, N=256, K=64) into a
 //               128x256 FP32 accumulator in TMEM, and tcgen05.commit to free stages.
-//   warps 2..9  epilogue: tcgen05.ld the accumulator (each warp its 32-lane quarter and
-//               one half of the columns), release it to the MMA warp at once, then do the
-//               FP32 math and the stores while the next tile accumulates.
+//   warps 2..17 epilogue: tcgen05.ld the accumulator (each warp its 32-lane quarter and
+//               a quarter of the columns), release it to the MMA warp at once, then do the
+//               FP32 math and the stores while the next tile accumulates.  The SwiGLU +
+//               NVFP4 epilogue is the longest per-tile step at prefill, so it gets four
+//               warps per SM sub-partition to hide its latencies.
 // Every wait is bounded (kWaitLimitNs): on expiry the CTA sets the device error word,
 // drains its own copies and MMAs, frees TMEM and exits.
 #include "common.cuh"
@@ -62,8 +64,10 @@ struct Ring {
 };
 using RingFull = Ring<4, A_TILE_BYTES>;
 using RingSmallM = Ring<5, 32 * BK_BYTES>;
-constexpr int NUM_THREADS = 320;
-constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_EPI_WARPS = 16;
+constexpr int NUM_THREADS = (2 + NUM_EPI_WARPS) * 32;
+constexpr int kEpiGroups = NUM_EPI_WARPS / 4;  // column groups: each warp owns a lane quarter x group
+static_assert(kEpiGroups * 64 == BN && kEpiGroups * 32 * 2 == BN, "down: 64 columns, gate/up: 32 + 32 per group");
 constexpr int kTileSlots = 4;       // tile ids the producer may publish ahead of the epilogue
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;     // 256 FP32 columns
@@ -346,8 +350,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;           // TMEM lanes this warp may access
-    const int half = (warp - 2) >> 2;       // which half of the 256 accumulator columns
+    const int quarter = warp & 3;            // TMEM lanes this warp may access
+    const int group = (warp - 2) >> 2;       // column group: gate/up 32 + 32 columns, down 64
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float alpha2 = args.alpha_a2;
@@ -370,15 +374,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       const MBlock mb = load_mblock(args.mblocks + t.block);
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->acc_full, acc_phase, abort_flag))) break;
       tc_fence_after();
-      uint32_t v[4][32];
-      if (!t.down) {  // gate columns [half*64, +64) and the matching up columns
-        tmem_ld_32x32b_x32(t_lane + ACC_COL + half * 64, v[0]);
-        tmem_ld_32x32b_x32(t_lane + ACC_COL + half * 64 + 32, v[1]);
-        tmem_ld_32x32b_x32(t_lane + ACC_COL + 128 + half * 64, v[2]);
-        tmem_ld_32x32b_x32(t_lane + ACC_COL + 128 + half * 64 + 32, v[3]);
+      uint32_t v[2][32];
+      if (!t.down) {  // gate columns [group*32, +32) and the matching up columns
+        tmem_ld_32x32b_x32(t_lane + ACC_COL + group * 32, v[0]);
+        tmem_ld_32x32b_x32(t_lane + ACC_COL + 128 + group * 32, v[1]);
       } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_lane + ACC_COL + half * 128 + c * 32, v[c]);
+        tmem_ld_32x32b_x32(t_lane + ACC_COL + group * 64, v[0]);
+        tmem_ld_32x32b_x32(t_lane + ACC_COL + group * 64 + 32, v[1]);
       }
       tmem_ld_wait();
       tc_fence_before();
@@ -389,31 +391,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       if (!t.down) {
         if (valid) {
           const float scale = args.alpha_a1 * __ldg(args.w_gu_alpha + mb.expert);
-          const int f0 = t.nt * 128 + half * 64;  // first feature of this thread's 64
-          uint32_t codes[8];
+          const int f0 = t.nt * 128 + group * 32;  // first feature of this thread's 32
+          uint32_t codes[4];
           uint32_t scodes = 0;
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
+          for (int b = 0; b < 2; ++b) {
             float h[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const int c = b * 16 + i;
-              const float g = __uint_as_float(v[c >> 5][c & 31]) * scale;
-              const float u = __uint_as_float(v[2 + (c >> 5)][c & 31]) * scale;
+              const float g = __uint_as_float(v[0][b * 16 + i]) * scale;
+              const float u = __uint_as_float(v[1][b * 16 + i]) * scale;
               h[i] = silu_times(g, u);
             }
             const uint32_t sc = quant_block16(h, alpha2, six_alpha2, codes[2 * b], codes[2 * b + 1]);
             scodes |= sc << (8 * b);
           }
-          // 64 features = 32 bytes = 16-byte chunks c0, c0 + 1 of K tile f0 / 256 of the A2 tile
-          const int a2_kt = f0 >> 8, c0 = (f0 & 255) >> 5;
-          *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.d_k_tiles, a2_kt, row_in_tile, c0)) =
+          // 32 features = one 16-byte chunk (f0 % 256) / 32 of K tile f0 / 256 of the A2 tile
+          *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.d_k_tiles, f0 >> 8, row_in_tile,
+                                                              (f0 & 255) >> 5)) =
               make_uint4(codes[0], codes[1], codes[2], codes[3]);
-          *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.d_k_tiles, a2_kt, row_in_tile,
-                                                              c0 + 1)) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-          // the 4 scales of this K-group (features f0..f0+63) are 4 contiguous bytes
-          *reinterpret_cast<uint32_t*>(args.a2_sf + sf_atom_offset(mb.sf_block, args.d_k_tiles * 4, row_in_tile,
-                                                                   f0 / 16)) = scodes;
+          // its 2 scales are 2 contiguous bytes of the K-group's 4 (f0 / 16 is even)
+          *reinterpret_cast<uint16_t*>(args.a2_sf + sf_atom_offset(mb.sf_block, args.d_k_tiles * 4, row_in_tile,
+                                                                   f0 / 16)) = static_cast<uint16_t>(scodes);
         }
         // publish this warp's share of block t.block's A2 to the down-tile producers
         fence_proxy_async_global();
@@ -425,15 +424,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       } else if (valid) {
         const float scale = args.alpha_a2 * __ldg(args.w_d_alpha + mb.expert);
         const size_t r = static_cast<size_t>(mb.row_begin + row_in_tile);
-        uint4* dst = reinterpret_cast<uint4*>(args.y + r * args.y_cols + t.nt * BN + half * 128);
+        uint4* dst = reinterpret_cast<uint4*>(args.y + r * args.y_cols + t.nt * BN + group * 64);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int c = q * 8;
+        for (int q = 0; q < 8; ++q) {
           uint32_t p[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            p[i] = bf16x2_bits(__uint_as_float(v[(c + 2 * i) >> 5][(c + 2 * i) & 31]) * scale,
-                               __uint_as_float(v[(c + 2 * i + 1) >> 5][(c + 2 * i + 1) & 31]) * scale);
+          for (int i = 0; i < 4; ++i) {
+            const int c = q * 8 + 2 * i;
+            p[i] = bf16x2_bits(__uint_as_float(v[c >> 5][c & 31]) * scale,
+                               __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31]) * scale);
+          }
           dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
         }
       }

@@ -23,8 +23,11 @@
 
 namespace beam {
 
-constexpr int kSmallThreads = 256;
-constexpr int kSmallExpertsPerCta = kSmallThreads / 32;  // one warp per expert
+constexpr int kSmallExpertsPerCta = 8;                   // one warp per expert
+// plus one warp whose lane 0 issues every bulk copy: a thread that issues copies runs its
+// warp's math several times slower afterwards, so the copy issuer computes nothing
+constexpr int kSmallThreads = (kSmallExpertsPerCta + 1) * 32;
+constexpr int kCopyThread = kSmallExpertsPerCta * 32;
 constexpr int kSmallMaxF4 = 16;                          // 16-byte W pieces per lane: H / S <= 2048
 
 // Number of H slices: the largest S in {4, 2, 1} whose slice is a whole number of
@@ -70,22 +73,25 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
   // ---------------------------------------------------------------- phase 1: partial logits
   // Each slice row is one bulk copy.  The router weights are constant: they stream before
   // the wait for the previous kernel in the stream; x after it.
-  if (tid == 0) {
+  if (tid == kCopyThread) {
     mbar_arrive_expect_tx(&bars[0], static_cast<uint32_t>(n_e * Hs * 4));
     for (int q = 0; q < n_e; ++q)
       bulk_load(ws + q * Hs, w + static_cast<size_t>(e0 + q) * H + h0, Hs * 4, &bars[0]);
   }
   pdl_wait();
   pdl_trigger();
-  if (tid == 0) {
+  if (tid == kCopyThread) {
     mbar_arrive_expect_tx(&bars[1], static_cast<uint32_t>(T * Hs * 2));
     for (int t = 0; t < T; ++t) bulk_load(xs + t * Hs, x + static_cast<size_t>(t) * H + h0, Hs * 2, &bars[1]);
   }
-  const bool ok_w = mbar_wait_bounded(&bars[0], 0, &s_abort);
-  const bool ok = mbar_wait_bounded(&bars[1], 0, &s_abort) && ok_w;
-  if (!ok) {
-    if (lane == 0) atomicOr(err, kErrTimeoutProducer);
-  } else if (warp < n_e) {
+  if (warp < n_e) {
+    // every lane leaves the polling loop on its own: reconverge before the warp-wide math
+    const bool ok_w = mbar_wait_bounded(&bars[0], 0, &s_abort);
+    const bool ok = mbar_wait_bounded(&bars[1], 0, &s_abort) && ok_w;
+    __syncwarp();
+    if (!ok) {
+      if (lane == 0) atomicOr(err, kErrTimeoutProducer);
+    } else {
     // All tokens at once: one W piece per step, then MAXT independent FMA chains (rows
     // past T repeat row 0 and are dropped), so the smem loads and FMAs overlap.
     const float4* wr = reinterpret_cast<const float4*>(ws + warp * Hs);
@@ -116,6 +122,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
         if (lane == t) mine = acc[t];
       part[(static_cast<size_t>(hs) * T + lane) * E + e0 + warp] = mine;
     }
+    }
   }
   // ---------------------------------------------------------------- elect the last CTA
   __shared__ int s_last;
@@ -130,13 +137,14 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
   // All partial logits in one bulk copy (the other CTAs' stores were released before
   // their counter increment; the proxy fence orders them before this copy).
   float* ps = reinterpret_cast<float*>(smem);  // [S][T][E]
-  if (tid == 0) {
+  if (tid == kCopyThread) {
     fence_proxy_async_global();
     fence_proxy_async_smem();  // phase 1's reads of this shared memory are done (barrier above)
     const uint32_t bytes = static_cast<uint32_t>(S * T * E * 4);
     mbar_arrive_expect_tx(&bars[2], bytes);
     bulk_load(ps, part, bytes, &bars[2]);
   }
+  __syncwarp();
   // the expert GEMM launch that follows starts from zeroed scheduler words
   for (int i = tid; i < sched_n; i += kSmallThreads) sched[i] = 0u;
   __shared__ int s_ids[kMaxSmallRouterTokens * 16];
@@ -148,8 +156,9 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
   if (!mbar_wait_bounded(&bars[2], 0, &s_abort)) {
     if (tid == 0) atomicOr(err, kErrTimeoutProducer);
   }
+  __syncwarp();
   const int TE = T * E;
-  for (int t = warp; t < T; t += kSmallThreads / 32) {
+  for (int t = warp; t < T && warp < kSmallExpertsPerCta; t += kSmallExpertsPerCta) {
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {

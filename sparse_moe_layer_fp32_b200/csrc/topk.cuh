@@ -16,37 +16,54 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 }
 
 // v: this lane's logits, expert e = lane + 32 i (entries with e >= E are ignored).
-// k rounds of a warp arg-max (larger logit first, equal logits -> lower expert index): a
-// warp max of the keys, then one ballot per register slot finds the lowest expert holding
-// it.  softmax is monotone, so these are the top-k of the softmax, and the renormalised
-// weights p_j / sum_chosen p equal a softmax over the chosen logits.  Lane j < k ends up
-// holding slot j and writes ids[j] / wout[j] (descending weight).
+// Each lane first sorts its EPL candidates (descending key, equal keys keep the lower
+// expert first); then k rounds take the warp maximum of the lanes' heads, the lowest
+// expert index among the heads equal to it wins (equal logits -> lower expert index), and
+// the winning lane pops its head.  softmax is monotone, so these are the top-k of the
+// softmax, and the renormalised weights p_j / sum_chosen p equal a softmax over the chosen
+// logits.  Lane j < k ends up holding slot j and writes ids[j] / wout[j] (descending
+// weight).
 template <int EPL>
 __device__ __forceinline__ void warp_topk(const float (&v)[EPL], int E, int k, int lane, int32_t* ids,
                                           float* wout) {
   uint32_t key[EPL];
+  int idx[EPL];
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) key[i] = lane + 32 * i < E ? order_key(v[i]) : 0u;
+  for (int i = 0; i < EPL; ++i) {
+    idx[i] = lane + 32 * i;
+    key[i] = idx[i] < E ? order_key(v[i]) : 0u;
+  }
+  // odd-even transposition sort; a swap needs a strictly larger key, so it is stable
+#pragma unroll
+  for (int p = 0; p < EPL; ++p) {
+#pragma unroll
+    for (int i = p & 1; i + 1 < EPL; i += 2) {
+      const bool sw = key[i + 1] > key[i];
+      const uint32_t ka = sw ? key[i + 1] : key[i], kb = sw ? key[i] : key[i + 1];
+      const int ia = sw ? idx[i + 1] : idx[i], ib = sw ? idx[i] : idx[i + 1];
+      key[i] = ka;
+      key[i + 1] = kb;
+      idx[i] = ia;
+      idx[i + 1] = ib;
+    }
+  }
   int my_e = 0;
   float my_v = 0.0f, v0 = 0.0f;
   for (int j = 0; j < k; ++j) {
-    uint32_t m = key[0];
+    const uint32_t top = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t best = __reduce_min_sync(0xffffffffu, key[0] == top ? static_cast<uint32_t>(idx[0]) : 0xffffffffu);
+    if (key[0] == top && static_cast<uint32_t>(idx[0]) == best) {  // pop the head
 #pragma unroll
-    for (int i = 1; i < EPL; ++i) m = max(m, key[i]);
-    const uint32_t top = __reduce_max_sync(0xffffffffu, m);
-    int best = 0;
-#pragma unroll
-    for (int i = EPL - 1; i >= 0; --i) {  // the lowest slot (then lane) that holds the maximum
-      const uint32_t b = __ballot_sync(0xffffffffu, key[i] == top);
-      if (b) best = 32 * i + __ffs(b) - 1;
+      for (int i = 0; i + 1 < EPL; ++i) {
+        key[i] = key[i + 1];
+        idx[i] = idx[i + 1];
+      }
+      key[EPL - 1] = 0u;
     }
-#pragma unroll
-    for (int i = 0; i < EPL; ++i)
-      if (best == lane + 32 * i) key[i] = 0u;
     const float val = key_value(top);
     if (j == 0) v0 = val;
     if (lane == j) {
-      my_e = best;
+      my_e = static_cast<int>(best);
       my_v = val;
     }
   }
