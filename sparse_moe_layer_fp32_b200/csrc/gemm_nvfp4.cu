@@ -19,7 +19,7 @@
 // waits on anything, so every awaited tile is held by a running CTA: no deadlock, and no
 // need for all CTAs to be resident at once.
 //
-// CTA layout (one persistent CTA per SM, 576 threads, warp-specialised):
+// CTA layout (one persistent CTA per SM, 704 threads, warp-specialised):
 //   warp 0      producer: claims tiles, publishes each tile id through a small shared
 //               ring, and per 256-wide K step bulk-copies the A tile (the valid rows of a
 //               128-row activation tile, <= 16 KB), the expert's weight tile with its
@@ -27,14 +27,18 @@
 //               landing on one mbarrier.  Activations and weights are both stored as
 //               contiguous tiles already in the swizzled shared-memory order, so every
 //               load is one sequential copy.
-//   warp 1      TMEM owner; lane 0 issues tcgen05.cp (scales -> TMEM) and
-//               tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128, N=256, K=64) into a
-//               128x256 FP32 accumulator in TMEM, and tcgen05.commit to free stages.
+//   warp 1      TMEM owner; lane 0 issues tcgen05.mma.kind::mxf4nvf4.block_scale.block16
+//               (M=128, N=256, K=64) into a 128x256 FP32 accumulator in TMEM and
+//               tcgen05.commit to free stages.
 //   warps 2..17 epilogue: tcgen05.ld the accumulator (each warp its 32-lane quarter and
 //               a quarter of the columns), release it to the MMA warp at once, then do the
 //               FP32 math and the stores while the next tile accumulates.  The SwiGLU +
 //               NVFP4 epilogue is the longest per-tile step at prefill, so it gets four
 //               warps per SM sub-partition to hide its latencies.
+//   warps 18-21 scale factors: per stage, copy the A and B scales from shared memory to that
+//               stage's TMEM columns with tcgen05.st (one warp per lane quarter).  Done with
+//               tcgen05.cp by the MMA thread, the 12 copies per K step took the tensor pipe
+//               about as long as the 4 MMAs.
 // Every wait is bounded (kWaitLimitNs): on expiry the CTA sets the device error word,
 // drains its own copies and MMAs, frees TMEM and exits.
 #include "common.cuh"
@@ -65,25 +69,30 @@ struct Ring {
 using RingFull = Ring<4, A_TILE_BYTES>;
 using RingSmallM = Ring<5, 32 * BK_BYTES>;
 constexpr int NUM_EPI_WARPS = 16;
-constexpr int NUM_THREADS = (2 + NUM_EPI_WARPS) * 32;
+constexpr int NUM_SF_WARPS = 4;                      // one per TMEM lane quarter
+constexpr int FIRST_SF_WARP = 2 + NUM_EPI_WARPS;
+constexpr int NUM_THREADS = (2 + NUM_EPI_WARPS + NUM_SF_WARPS) * 32;
 constexpr int kEpiGroups = NUM_EPI_WARPS / 4;  // column groups: each warp owns a lane quarter x group
 static_assert(kEpiGroups * 64 == BN && kEpiGroups * 32 * 2 == BN, "down: 64 columns, gate/up: 32 + 32 per group");
 constexpr int kTileSlots = 4;       // tile ids the producer may publish ahead of the epilogue
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0;     // 256 FP32 columns
-constexpr uint32_t SFA_COL = 256;   // 4 K-groups x 4 columns
-constexpr uint32_t SFB_COL = 288;   // 4 K-groups x 8 columns
+constexpr uint32_t ACC_COL = 0;            // 256 FP32 columns
+constexpr uint32_t SF_COL = 256;           // scale factors, one column set per ring stage:
+constexpr uint32_t SF_STAGE_COLS = 48;     //   A: 4 K-groups x 4 columns, then B: 4 K-groups x 8
+constexpr uint32_t SFB_OFF = 16;
 
 // Instruction descriptor: E2M1 A and B (format 1), E4M3 scales (format 0), K-major
 // operands, N = 256 (n_dim = N/8 at bit 17), M = 128 (m_dim = M/16 at bit 24).
 constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((BM >> 4) << 24);
 
 constexpr int kMaxStages = 5;
+static_assert(SF_COL + kMaxStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor stages must fit in TMEM");
 struct __align__(8) GemmSmemTail {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t tile_full[kTileSlots];   // producer -> MMA + epilogue: tile id published
-  uint64_t tile_empty[kTileSlots];  // MMA + epilogue warps -> producer: slot read
+  uint64_t tile_empty[kTileSlots];  // MMA + epilogue + scale warps -> producer: slot read
+  uint64_t sf_full[kMaxStages];     // scale warps -> MMA: stage's scale factors are in TMEM
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
@@ -159,10 +168,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&tail->full[s], 1);
       mbar_init(&tail->empty[s], 1);
+      mbar_init(&tail->sf_full[s], NUM_SF_WARPS);
     }
     for (int j = 0; j < kTileSlots; ++j) {
       mbar_init(&tail->tile_full[j], 1);
-      mbar_init(&tail->tile_empty[j], 1 + NUM_EPI_WARPS);
+      mbar_init(&tail->tile_empty[j], 1 + NUM_EPI_WARPS + NUM_SF_WARPS);
     }
     mbar_init(&tail->acc_full, 1);
     mbar_init(&tail->acc_empty, NUM_EPI_WARPS);
@@ -312,25 +322,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
         tc_fence_after();
         bool ok = true;
         for (int kt = 0; kt < k_tiles; ++kt) {
-          if (!mbar_wait_bounded(&tail->full[stage], phase, abort_flag)) {
+          // the stage's operands have landed and its scale factors are in TMEM
+          if (!mbar_wait_bounded(&tail->sf_full[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t ssfb = sb + B_BYTES;
-          const uint32_t ssfa = ssfb + SFB_BYTES;
-#pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            tc_cp_32x128b_x4(tmem + SFA_COL + kb * 4, sdesc_sf(ssfa + kb * 512));
-            tc_cp_32x128b_x4(tmem + SFB_COL + kb * 8, sdesc_sf(ssfb + kb * 512));
-            tc_cp_32x128b_x4(tmem + SFB_COL + kb * 8 + 4, sdesc_sf(ssfb + SFA_BYTES + kb * 512));
-          }
+          const uint32_t sf = tmem + SF_COL + stage * SF_STAGE_COLS;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             tc_mma_nvfp4(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), kIdescNvfp4,
-                         tmem + SFA_COL + kb * 4, tmem + SFB_COL + kb * 8, (kt | kb) != 0 ? 1u : 0u);
+                         sf + kb * 4, sf + SFB_OFF + kb * 8, (kt | kb) != 0 ? 1u : 0u);
           }
           tc_commit(&tail->empty[stage]);
           if (++stage == STAGES) {
@@ -347,6 +351,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(&tail->drain, 0))
         if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+  } else if (warp >= FIRST_SF_WARP) {
+    // ------------------------------------------------------------ scale factors -> TMEM
+    // Each warp fills its own lane quarter of the stage's scale-factor columns from the
+    // 512-byte shared-memory atoms (row r of an atom holds the 4 scales of rows r, r + 32,
+    // r + 64, r + 96 of one 64-wide K-group), every quarter getting the same 4 columns per
+    // K-group, so the MMA finds the scales of row m at lane m, column + m / 32.  Doing it
+    // with tcgen05.st keeps these copies off the tensor pipe, which then only runs MMAs.
+    const int quarter = warp & 3;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    int stage = 0, slot = 0;
+    uint32_t phase = 0, slot_phase = 0;
+    for (;;) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->tile_full[slot], slot_phase, abort_flag))) break;
+      const int id = tail->tile_ids[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->tile_empty[slot]);
+      if (++slot == kTileSlots) {
+        slot = 0;
+        slot_phase ^= 1;
+      }
+      if (id < 0) break;
+      const int k_tiles = id >= total_gu ? args.d_k_tiles : args.gu_k_tiles;
+      bool ok = true;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->full[stage], phase, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const uint8_t* ssfb = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;  // [half][K-group][512]
+        const uint8_t* ssfa = ssfb + SFB_BYTES;                                // [K-group][512]
+        const uint32_t col = SF_COL + stage * SF_STAGE_COLS;
+        uint32_t r[16];
+        // A: K-group kb -> columns 4 kb .. 4 kb + 3
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512 + lane * 16);
+          r[kb * 4 + 0] = v.x; r[kb * 4 + 1] = v.y; r[kb * 4 + 2] = v.z; r[kb * 4 + 3] = v.w;
+        }
+        tmem_st_32x32b_x16(t_lane + col, r);
+        // B: K-group kb -> columns 8 kb .. 8 kb + 3 (rows 0-127), 8 kb + 4 .. 8 kb + 7 (rows 128-255)
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int kb = part * 2 + q;
+            const uint4 v0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512 + lane * 16);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(ssfb + SFA_BYTES + kb * 512 + lane * 16);
+            r[q * 8 + 0] = v0.x; r[q * 8 + 1] = v0.y; r[q * 8 + 2] = v0.z; r[q * 8 + 3] = v0.w;
+            r[q * 8 + 4] = v1.x; r[q * 8 + 5] = v1.y; r[q * 8 + 6] = v1.z; r[q * 8 + 7] = v1.w;
+          }
+          tmem_st_32x32b_x16(t_lane + col + SFB_OFF + part * 16, r);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tail->sf_full[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
     }
   } else {
     // ------------------------------------------------------------ epilogue
