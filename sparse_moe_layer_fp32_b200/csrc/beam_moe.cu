@@ -318,12 +318,13 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     return cudaEventRecord(h->events[launches + 1], s);
   };
   if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
+  const BlockScales bscales{h->w_gu_alpha, h->w_d_alpha, h->cfg.alpha_a1, h->cfg.alpha_a2};
   if (route_small_supported(T, H, E, k)) {
     // router + top-k + histogram + scan + permutation in one launch
     int slices = 1;
     BEAM_TRY(launch_route_small(xb, h->router_w, T, H, E, k, h->logits, h->ids, h->w, h->offsets, h->sf_block,
                                 h->mblocks, h->num_mblocks, h->perm, h->inv, h->tile_row, h->route_counter, h->sched,
-                                static_cast<int>(sched_words(h->nblk_max)), h->err, &slices, s));
+                                static_cast<int>(sched_words(h->nblk_max)), bscales, h->err, &slices, s));
     BEAM_TRY(mark("route_small"));
     ++launches;
     h->last_splits = slices;
@@ -349,7 +350,7 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     BEAM_TRY(mark("chunk_hist"));
     ++launches;
     BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
-                         h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), s));
+                         h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), bscales, s));
     BEAM_TRY(mark("scan"));
     ++launches;
     BEAM_TRY(launch_scatter(h->ids, h->chunk_base, h->offsets, h->sf_block, T, k, E, h->perm, h->inv, h->tile_row,
@@ -370,15 +371,12 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   g.a1 = h->a1;
   g.a1_sf = h->a1_sf;
   g.w_gu = h->w_gu_tiles;
-  g.w_gu_alpha = h->w_gu_alpha;
-  g.alpha_a1 = h->cfg.alpha_a1;
   g.a2 = h->a2;
   g.a2_sf = h->a2_sf;
   g.alpha_a2 = h->cfg.alpha_a2;
   g.d_n_tiles = H / 256;
   g.d_k_tiles = h->Ip / 256;
   g.w_d = h->w_d_tiles;
-  g.w_d_alpha = h->w_d_alpha;
   g.y = h->y;
   g.y_cols = H;
   g.sched = h->sched;

@@ -108,6 +108,13 @@ static size_t ring_smem_bytes() {
 
 __device__ __forceinline__ float silu_times(float g, float u) { return __fdiv_rn(g, 1.0f + expf(-g)) * u; }
 
+// One 32-byte store (8 x 32 bits) to a 32-byte aligned global address.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -135,7 +142,8 @@ __device__ __forceinline__ bool wait_counter_bounded(const uint32_t* counter, ui
 // Block-list entries are written by the routing kernels; read them from L2.
 __device__ __forceinline__ MBlock load_mblock(const MBlock* p) {
   const int4 v = __ldcg(reinterpret_cast<const int4*>(p));
-  return MBlock{v.x, v.y, v.z, v.w};
+  const int4 u = __ldcg(reinterpret_cast<const int4*>(p) + 1);
+  return MBlock{v.x, v.y, v.z, v.w, __int_as_float(u.x), __int_as_float(u.y), {0, 0}};
 }
 
 // Position of a tile id in the list [gate/up tiles of every block][down tiles of every block].
@@ -457,7 +465,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       const bool valid = row_in_tile < mb.rows;
       if (!t.down) {
         if (valid) {
-          const float scale = args.alpha_a1 * __ldg(args.w_gu_alpha + mb.expert);
+          const float scale = mb.scale_gu;
           const int f0 = t.nt * 128 + group * 32;  // first feature of this thread's 32
           uint32_t codes[4];
           uint32_t scodes = 0;
@@ -489,19 +497,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           atomicAdd(ready + t.block, 1u);
         }
       } else if (valid) {
-        const float scale = args.alpha_a2 * __ldg(args.w_d_alpha + mb.expert);
+        const float scale = mb.scale_d;
         const size_t r = static_cast<size_t>(mb.row_begin + row_in_tile);
-        uint4* dst = reinterpret_cast<uint4*>(args.y + r * args.y_cols + t.nt * BN + group * 64);
+        // 64 BF16 = 128 contiguous bytes of row r, written as 4 x 32-byte stores
+        uint16_t* dst = args.y + r * args.y_cols + t.nt * BN + group * 64;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint32_t p[4];
+        for (int q = 0; q < 4; ++q) {
+          uint32_t p[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = q * 8 + 2 * i;
+          for (int i = 0; i < 8; ++i) {
+            const int c = q * 16 + 2 * i;
             p[i] = bf16x2_bits(__uint_as_float(v[c >> 5][c & 31]) * scale,
                                __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31]) * scale);
           }
-          dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
+          st_global_v8(dst + q * 16, p);
         }
       }
     }

@@ -8,11 +8,20 @@
 namespace beam {
 
 // One 128-row work block of an expert for the grouped GEMMs.
-struct MBlock {
+struct alignas(32) MBlock {
   int32_t expert;     // expert index
   int32_t row_begin;  // first permuted row
   int32_t rows;       // valid rows, 1..128
   int32_t sf_block;   // scale block of these rows (see the scale-block layout in beam_moe.h)
+  float scale_gu;     // alpha_a1 * alpha_gu[expert]: dequantisation of the gate/up accumulators
+  float scale_d;      // alpha_a2 * alpha_d[expert]: dequantisation of the down accumulators
+  int32_t pad[2];
+};
+// What the block-list builders need to fill MBlock::scale_gu / scale_d.
+struct BlockScales {
+  const float* w_gu_alpha;  // [E]
+  const float* w_d_alpha;   // [E]
+  float alpha_a1, alpha_a2;
 };
 
 constexpr int kChunkTokens = 256;  // tokens per histogram / scatter chunk
@@ -45,15 +54,15 @@ int64_t route_small_ws_floats(int T, int H, int E);  // partial logits [S][T][E]
 cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, int E, int k, float* part,
                                int32_t* ids, float* wout, int32_t* offsets, int32_t* sf_block, MBlock* mblocks,
                                int32_t* num_mblocks, int32_t* perm, int32_t* inv, int32_t* tile_row,
-                               unsigned int* done_counter, uint32_t* sched, int sched_n, uint32_t* err, int* slices,
-                               cudaStream_t s);
+                               unsigned int* done_counter, uint32_t* sched, int sched_n, BlockScales bs, uint32_t* err,
+                               int* slices, cudaStream_t s);
 
 // ---- permutation and activation quantisation (routing.cu)
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s);
 // Also zeroes sched[0, sched_n), the tile scheduler words of the expert GEMM launch.
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
-                        cudaStream_t s);
+                        BlockScales bs, cudaStream_t s);
 // tile_row[t][j] = 128 x activation block + row within it, for slot (t, j).
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,
                            const int32_t* sf_block, int T, int k, int E, int32_t* perm_src, int32_t* inv,
@@ -88,8 +97,6 @@ struct ExpertGemmArgs {
   const uint8_t* a1;
   const uint8_t* a1_sf;
   const uint8_t* w_gu;
-  const float* w_gu_alpha;  // [E]
-  float alpha_a1;
   // SwiGLU + NVFP4 epilogue output, the down GEMM's A operand (K = Ip)
   uint8_t* a2;
   uint8_t* a2_sf;
@@ -98,7 +105,6 @@ struct ExpertGemmArgs {
   int d_n_tiles;            // H / 256
   int d_k_tiles;            // Ip / 256
   const uint8_t* w_d;
-  const float* w_d_alpha;   // [E]
   uint16_t* y;              // [rows][H] BF16
   int y_cols;               // H
   // [0]: next tile to claim; [1 + b]: gate/up epilogue warps done on block b.

@@ -53,7 +53,8 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     float* __restrict__ part, int32_t* __restrict__ ids, float* __restrict__ wout, int32_t* __restrict__ offsets,
     int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks, int32_t* __restrict__ num_mblocks,
     int32_t* __restrict__ perm, int32_t* __restrict__ inv, int32_t* __restrict__ tile_row,
-    unsigned int* __restrict__ done_counter, uint32_t* __restrict__ sched, int sched_n, uint32_t* __restrict__ err) {
+    unsigned int* __restrict__ done_counter, uint32_t* __restrict__ sched, int sched_n, BlockScales bs,
+    uint32_t* __restrict__ err) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t bars[3];  // W slices, x slice, partial logits
   __shared__ int s_abort;
@@ -193,6 +194,9 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
       m.row_begin = off + 128 * i;
       m.rows = min(128, cnt - 128 * i);
       m.sf_block = blk + i;
+      m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + tid);
+      m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + tid);
+      m.pad[0] = m.pad[1] = 0;
       mblocks[blk + i] = m;
     }
   }
@@ -229,8 +233,8 @@ int64_t route_small_ws_floats(int T, int H, int E) {
 cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, int E, int k, float* part,
                                int32_t* ids, float* wout, int32_t* offsets, int32_t* sf_block, MBlock* mblocks,
                                int32_t* num_mblocks, int32_t* perm, int32_t* inv, int32_t* tile_row,
-                               unsigned int* done_counter, uint32_t* sched, int sched_n, uint32_t* err, int* slices,
-                               cudaStream_t s) {
+                               unsigned int* done_counter, uint32_t* sched, int sched_n, BlockScales bs, uint32_t* err,
+                               int* slices, cudaStream_t s) {
   const int S = route_small_slices(H);
   *slices = S;
   const size_t smem = route_small_smem(T, H, E);
@@ -239,7 +243,7 @@ cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, 
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_pdl(kernel, dim3(groups * S), dim3(kSmallThreads), smem, s, x, w, T, H, E, k, S, part, ids, wout,
-                    offsets, sf_block, mblocks, num_mblocks, perm, inv, tile_row, done_counter, sched, sched_n,
+                    offsets, sf_block, mblocks, num_mblocks, perm, inv, tile_row, done_counter, sched, sched_n, bs,
                     err);
 }
 

@@ -40,7 +40,8 @@ __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restri
 __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chunks, int E,
                             int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
                             int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks,
-                            int32_t* __restrict__ num_mblocks, uint32_t* __restrict__ sched, int sched_n) {
+                            int32_t* __restrict__ num_mblocks, uint32_t* __restrict__ sched, int sched_n,
+                            BlockScales bs) {
   __shared__ int warp_sums[33];
   pdl_wait();
   pdl_trigger();
@@ -70,6 +71,9 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
       m.row_begin = off + 128 * i;
       m.rows = min(128, cnt - 128 * i);
       m.sf_block = blk + i;
+      m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + e);
+      m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + e);
+      m.pad[0] = m.pad[1] = 0;
       mblocks[blk + i] = m;
     }
   }
@@ -223,10 +227,10 @@ cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* 
 
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
-                        cudaStream_t s) {
+                        BlockScales bs, cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
   return launch_pdl(scan_kernel, dim3(1), dim3(threads), 0, s, chunk_counts, n_chunks, E, chunk_base, offsets,
-                    sf_block, mblocks, num_mblocks, sched, sched_n);
+                    sf_block, mblocks, num_mblocks, sched, sched_n, bs);
 }
 
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,
