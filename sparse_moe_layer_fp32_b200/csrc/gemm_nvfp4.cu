@@ -87,7 +87,7 @@ constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((
 
 constexpr int kMaxStages = 5;
 static_assert(SF_COL + kMaxStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor stages must fit in TMEM");
-struct __align__(8) GemmSmemTail {
+struct __align__(16) GemmSmemTail {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t tile_full[kTileSlots];   // producer -> MMA + epilogue: tile id published
@@ -97,6 +97,7 @@ struct __align__(8) GemmSmemTail {
   uint64_t acc_empty;
   uint64_t drain;
   int tile_ids[kTileSlots];         // claimed tile, -1 = no more work
+  int4 tile_mb[kTileSlots][2];      // its block-list entry (MBlock), read once by the producer
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -106,7 +107,10 @@ static size_t ring_smem_bytes() {
   return static_cast<size_t>(R::STAGES) * R::STAGE_BYTES + sizeof(GemmSmemTail) + 1024;
 }
 
-__device__ __forceinline__ float silu_times(float g, float u) { return __fdiv_rn(g, 1.0f + expf(-g)) * u; }
+// silu(g) * u in FP32 with the fast exponential and division (a few ulp; h is compared with
+// the FP64 oracle within its tolerance, unlike the quantiser steps, which stay exact).  For
+// g -> -inf, exp(-g) = inf and g / inf = -0.
+__device__ __forceinline__ float silu_times(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 // One 32-byte store (8 x 32 bits) to a 32-byte aligned global address.
 __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
@@ -227,15 +231,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       for (;;) {
         if (!mbar_wait_bounded(&tail->tile_empty[slot], slot_phase ^ 1, abort_flag)) break;
         int id = claim < static_cast<uint32_t>(total) ? static_cast<int>(claim) : -1;
+        // the tile's block entry travels with its id, so no consumer reads global memory for it
+        const TileRef t = tile_ref(id < 0 ? 0 : id, total_gu, n_gu, n_d);
+        const MBlock mb = id < 0 ? MBlock{} : load_mblock(args.mblocks + t.block);
         tail->tile_ids[slot] = id;
+        tail->tile_mb[slot][0] = make_int4(mb.expert, mb.row_begin, mb.rows, mb.sf_block);
+        tail->tile_mb[slot][1] = make_int4(__float_as_int(mb.scale_gu), __float_as_int(mb.scale_d), 0, 0);
         mbar_arrive(&tail->tile_full[slot]);
         if (++slot == kTileSlots) {
           slot = 0;
           slot_phase ^= 1;
         }
         if (id < 0) break;
-        const TileRef t = tile_ref(id, total_gu, n_gu, n_d);
-        const MBlock mb = load_mblock(args.mblocks + t.block);
         const int k_tiles = t.down ? args.d_k_tiles : args.gu_k_tiles;
         const int n_tiles = t.down ? n_d : n_gu;
         const uint8_t* a_src = (t.down ? args.a2 : args.a1) + static_cast<size_t>(mb.sf_block) * k_tiles * A_TILE_BYTES;
@@ -438,6 +445,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       // operations below never run with part of the warp gone
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->tile_full[slot], slot_phase, abort_flag))) break;
       const int id = tail->tile_ids[slot];
+      const int4 m0 = tail->tile_mb[slot][0], m1 = tail->tile_mb[slot][1];
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->tile_empty[slot]);
       if (++slot == kTileSlots) {
@@ -446,7 +454,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       }
       if (id < 0) break;
       const TileRef t = tile_ref(id, total_gu, n_gu, n_d);
-      const MBlock mb = load_mblock(args.mblocks + t.block);
+      const MBlock mb{m0.x, m0.y, m0.z, m0.w, __int_as_float(m1.x), __int_as_float(m1.y), {0, 0}};
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->acc_full, acc_phase, abort_flag))) break;
       tc_fence_after();
       uint32_t v[2][32];
