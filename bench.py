@@ -71,9 +71,10 @@ def kernel_work(shape: mi.LayerShape, T: int, counts: np.ndarray) -> dict:
     }
 
 
-def read_traffic(kernel: str, used_experts: int):
+def read_traffic(kernel: str, used_experts: int, tokens: int):
     """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json), scaled
-    by the experts that received tokens; None when the kernel's source changed since."""
+    by the experts that received tokens; None when the kernel's source changed since or the
+    batch is outside the regime the capture scales to."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -84,7 +85,7 @@ def read_traffic(kernel: str, used_experts: int):
     import hashlib
     src = os.path.join(ROOT, "sparse_moe_layer_fp32_b200", "csrc", ent["source"])
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if digest != ent["source_sha256_16"]:
+    if digest != ent["source_sha256_16"] or tokens > ent.get("applies_up_to_tokens", tokens):
         return None
     return ent["bytes_per_used_expert"] * used_experts
 
@@ -337,7 +338,7 @@ def run_ours(args, shape, rank, world, local_rank):
         bound, achieved, peak, unit = "hbm", wk["bytes"] / (kern[top] / 1e3) / 1e9, pk["hbm"], "GB/s"
         peak_note = f"{pk['src']} copy bandwidth"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": read_traffic(top, work["_used_experts"]), "kernel": top, "kernel_ms": kern[top],
+                "traffic": read_traffic(top, work["_used_experts"], T), "kernel": top, "kernel_ms": kern[top],
                 "peak_source": peak_note}
 
     # ---- end to end through the host-buffer entry point (copies inside the timed region)
