@@ -191,6 +191,17 @@ BEAM_MOE_API beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, vo
  * TIMEOUT or DEVICE. */
 BEAM_MOE_API beam_moe_status beam_moe_check(beam_moe_t h, void* stream);
 
+/* Expert GEMM variant for the batches that do not use the small-batch routing (more than
+ * 16 tokens).  SINGLE: one CTA per 128-row work block.  PAIR: CTA pairs (clusters of two
+ * SMs sharing one M = 256 MMA) over 256-row work blocks.  AUTO (the default at create)
+ * picks PAIR from BEAM_MOE_PAIR_MIN_TOKENS tokens on, SINGLE below; the threshold is set
+ * where PAIR measured faster (INT32_MAX: never).  Both compute the same result up to the
+ * FP32 rounding of the accumulation order.  Not from the source pages: an implementation
+ * choice exposed for testing and tuning.  Returns INVALID_ARG for an unknown mode. */
+enum { BEAM_MOE_GEMM_AUTO = 0, BEAM_MOE_GEMM_SINGLE = 1, BEAM_MOE_GEMM_PAIR = 2 };
+#define BEAM_MOE_PAIR_MIN_TOKENS 2147483647
+BEAM_MOE_API beam_moe_status beam_moe_set_gemm_mode(beam_moe_t h, int32_t mode);
+
 /* Per-kernel timing.  While enabled (enable != 0), beam_moe_forward records a CUDA event
  * on `stream` before its first kernel and after each kernel it enqueues.  Creating the
  * events is the only allocation; enable once, outside any timed region. */

@@ -36,6 +36,7 @@ struct beam_moe_ctx {
   uint32_t* err;
   unsigned int* route_counter;  // last-CTA election of the fused small-batch routing kernel
   uint32_t* sched;              // tile scheduler of the expert GEMM launch (sched_words(nblk_max))
+  int32_t gemm_mode;            // BEAM_MOE_GEMM_*: which expert GEMM large batches use
   uint16_t *stage_x, *stage_res, *stage_out;
   int last_T;
   int last_splits;  // logits layout of the last forward: [splits][T][E] partial sums
@@ -187,6 +188,7 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   h->last_splits = 1;
   h->last_launches = 0;
   h->profiling = false;
+  h->gemm_mode = BEAM_MOE_GEMM_AUTO;
   h->profiled_last = false;
   for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i) {
     h->events[i] = nullptr;
@@ -319,6 +321,9 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   };
   if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
   const BlockScales bscales{h->w_gu_alpha, h->w_d_alpha, h->cfg.alpha_a1, h->cfg.alpha_a2};
+  // CTA pairs for the expert GEMM when the average expert has a few hundred rows
+  const bool pair = !route_small_supported(T, H, E, k) &&
+                    (h->gemm_mode == BEAM_MOE_GEMM_PAIR || (h->gemm_mode == BEAM_MOE_GEMM_AUTO && T >= kPairMinTokens));
   if (route_small_supported(T, H, E, k)) {
     // router + top-k + histogram + scan + permutation in one launch
     int slices = 1;
@@ -350,7 +355,8 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     BEAM_TRY(mark("chunk_hist"));
     ++launches;
     BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
-                         h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), bscales, s));
+                         h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), bscales,
+                         pair ? 1 : 0, s));
     BEAM_TRY(mark("scan"));
     ++launches;
     BEAM_TRY(launch_scatter(h->ids, h->chunk_base, h->offsets, h->sf_block, T, k, E, h->perm, h->inv, h->tile_row,
@@ -381,7 +387,10 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   g.y_cols = H;
   g.sched = h->sched;
   g.err = h->err;
-  BEAM_TRY(launch_gemm_experts(g, h->num_sms, s));
+  if (pair)
+    BEAM_TRY(launch_gemm_experts_pair(g, h->num_sms, s));
+  else
+    BEAM_TRY(launch_gemm_experts(g, h->num_sms, s));
   BEAM_TRY(mark("gemm_experts"));
   ++launches;
   BEAM_TRY(launch_finalize(h->y, h->w, h->inv, static_cast<const uint16_t*>(residual), h->gamma, T, H, k,
@@ -496,6 +505,12 @@ beam_moe_status beam_moe_debug_wait_timeout(beam_moe_t h, int64_t limit_ns, void
   if (!h || limit_ns <= 0 || limit_ns > static_cast<int64_t>(kWaitLimitNs)) return BEAM_MOE_ERR_INVALID_ARG;
   wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns), h->err);
   BEAM_TRY(cudaGetLastError());
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_set_gemm_mode(beam_moe_t h, int32_t mode) {
+  if (!h || mode < BEAM_MOE_GEMM_AUTO || mode > BEAM_MOE_GEMM_PAIR) return BEAM_MOE_ERR_INVALID_ARG;
+  h->gemm_mode = mode;
   return BEAM_MOE_OK;
 }
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "beam_moe.h"
+
 namespace beam {
 
 // One 128-row work block of an expert for the grouped GEMMs.
@@ -60,9 +62,10 @@ cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, 
 // ---- permutation and activation quantisation (routing.cu)
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s);
 // Also zeroes sched[0, sched_n), the tile scheduler words of the expert GEMM launch.
+// pair != 0: the work list holds 256-row blocks for the CTA-pair GEMM.
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
-                        BlockScales bs, cudaStream_t s);
+                        BlockScales bs, int pair, cudaStream_t s);
 // tile_row[t][j] = 128 x activation block + row within it, for slot (t, j).
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,
                            const int32_t* sf_block, int T, int k, int E, int32_t* perm_src, int32_t* inv,
@@ -114,6 +117,9 @@ struct ExpertGemmArgs {
 };
 inline int64_t sched_words(int64_t nblk_max) { return 1 + nblk_max; }
 cudaError_t launch_gemm_experts(const ExpertGemmArgs& a, int grid, cudaStream_t s);
+// The CTA-pair version over 256-row blocks (grid rounded down to even).
+constexpr int kPairMinTokens = BEAM_MOE_PAIR_MIN_TOKENS;
+cudaError_t launch_gemm_experts_pair(const ExpertGemmArgs& a, int grid, cudaStream_t s);
 
 // ---- finalize (finalize.cu)
 // next_x != nullptr also writes the next sublayer's pre-norm of out: bf16(out * rinv * next_gamma).

@@ -41,7 +41,7 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
                             int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
                             int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks,
                             int32_t* __restrict__ num_mblocks, uint32_t* __restrict__ sched, int sched_n,
-                            BlockScales bs) {
+                            BlockScales bs, int pair) {
   __shared__ int warp_sums[33];
   pdl_wait();
   pdl_trigger();
@@ -57,30 +57,36 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
       cnt += v;
     }
   }
+  // Activations live in 128-row blocks (sf_block); the work list uses 128-row blocks, or
+  // 256-row blocks (two consecutive activation blocks, the second possibly empty) when a
+  // CTA pair computes each tile.
   const int nblk = (cnt + 127) / 128;
-  int total_rows, total_blk;
+  const int wrows = pair ? 256 : 128;
+  const int nwork = (cnt + wrows - 1) / wrows;
+  int total_rows, total_blk, total_work;
   const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
   const int blk = block_exclusive_scan(nblk, warp_sums, total_blk);
+  const int wbase = block_exclusive_scan(nwork, warp_sums, total_work);
   if (e < E) {
     offsets[e] = off;
     sf_block[e] = blk;
     for (int c = 0; c < n_chunks; ++c) chunk_base[static_cast<size_t>(c) * E + e] += off;
-    for (int i = 0; i < nblk; ++i) {
+    for (int i = 0; i < nwork; ++i) {
       MBlock m;
       m.expert = e;
-      m.row_begin = off + 128 * i;
-      m.rows = min(128, cnt - 128 * i);
-      m.sf_block = blk + i;
+      m.row_begin = off + wrows * i;
+      m.rows = min(wrows, cnt - wrows * i);
+      m.sf_block = blk + (wrows / 128) * i;
       m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + e);
       m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + e);
       m.pad[0] = m.pad[1] = 0;
-      mblocks[blk + i] = m;
+      mblocks[wbase + i] = m;
     }
   }
   if (e == 0) {
     offsets[E] = total_rows;
     sf_block[E] = total_blk;
-    *num_mblocks = total_blk;
+    *num_mblocks = total_work;
   }
 }
 
@@ -227,10 +233,10 @@ cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* 
 
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
-                        BlockScales bs, cudaStream_t s) {
+                        BlockScales bs, int pair, cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
   return launch_pdl(scan_kernel, dim3(1), dim3(threads), 0, s, chunk_counts, n_chunks, E, chunk_base, offsets,
-                    sf_block, mblocks, num_mblocks, sched, sched_n, bs);
+                    sf_block, mblocks, num_mblocks, sched, sched_n, bs, pair);
 }
 
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,

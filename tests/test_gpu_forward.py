@@ -202,3 +202,28 @@ def test_forward_with_fused_next_prenorm(bm, name, tokens, seed):
     with pytest.raises(bm.BeamMoeError):
         layer.forward_prenorm(xd, rd, g_next, 1e-6, next_x=rd)  # next_x may not alias residual
     layer.close()
+
+
+@pytest.mark.parametrize("name,tokens,seed", [("tiny", 1500, 3), ("mid", 2000, 11), ("mid", 300, 12)])
+def test_pair_gemm_matches_oracle_and_single_cta(bm, name, tokens, seed):
+    # The CTA-pair expert GEMM (256-row work blocks, one M = 256 MMA over two SMs) against the
+    # oracle and against the single-CTA GEMM on the same inputs.  ~190, ~250 and ~37 rows per
+    # expert: full pairs, pairs whose second half is partly filled, and empty second halves.
+    shape, layer, weights, out_single, ref, _ = _run(bm, SHAPES[name], tokens, seed)
+    from sparse_moe_layer_fp32_b200 import synthetic
+    xd, rd = synthetic.make_batch(shape, seed)
+    layer.set_gemm_mode(bm.GEMM_SINGLE)
+    out_s = layer.forward(xd, rd)
+    layer.check()
+    assert torch.equal(out_s, out_single)  # AUTO picks the single-CTA GEMM at this size
+    layer.set_gemm_mode(bm.GEMM_PAIR)
+    out_p = layer.forward(xd, rd)
+    layer.check()
+    torch.cuda.synchronize()
+    rel, mx = compare_outputs(bf16_to_f64(out_p), ref["out_pre"], skip=ref["near_tie"])
+    assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
+    d_rel, _ = compare_outputs(bf16_to_f64(out_p), bf16_to_f64(out_s))
+    assert d_rel < 1e-3, d_rel
+    with pytest.raises(bm.BeamMoeError):
+        layer.set_gemm_mode(7)
+    layer.close()
