@@ -337,8 +337,9 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     if (router_tc_supported(T, H, E, k)) {
       // FP32-class logits on the tensor cores (BF16 x 3-part split), top-k in the epilogue
       CUtensorMap map_x;
-      if (!make_map_bf16(&map_x, xb, H, T, 128)) return BEAM_MOE_ERR_CUDA;
-      BEAM_TRY(launch_router_tc(map_x, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s));
+      const int rt_tokens = router_tc_tokens_per_cta(T, h->num_sms);
+      if (!make_map_bf16(&map_x, xb, H, T, static_cast<uint32_t>(rt_tokens))) return BEAM_MOE_ERR_CUDA;
+      BEAM_TRY(launch_router_tc(map_x, rt_tokens, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s));
       BEAM_TRY(mark("router_tc"));
       ++launches;
       h->last_splits = 1;

@@ -46,8 +46,10 @@ size_t router_tc_smem_bytes(int E);
 cudaError_t launch_split_router(const float* w, int E, int H, uint16_t* out, cudaStream_t s);
 // map_x: x [T][H] BF16, boxes 32 x 128 with the 64-byte swizzle; w_tiles: the split router
 // weights from launch_split_router.  Writes logits [T][E], ids / w [T][k].
-cudaError_t launch_router_tc(const CUtensorMap& map_x, const uint16_t* w_tiles, int T, int H, int E, int k,
-                             float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s);
+// Tokens per CTA (128 or 256) for a batch of T; also the row count of the x tensor map's box.
+int router_tc_tokens_per_cta(int T, int num_sms);
+cudaError_t launch_router_tc(const CUtensorMap& map_x, int tokens_per_cta, const uint16_t* w_tiles, int T, int H,
+                             int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s);
 
 // ---- routing of a small batch in one launch (route_small.cu)
 bool route_small_supported(int T, int H, int E, int k);

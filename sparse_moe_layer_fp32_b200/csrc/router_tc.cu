@@ -11,13 +11,17 @@
 // tcgen05.mma.kind::f16 in TMEM.  The result differs from an FP32 FFMA GEMM only in the
 // order of the FP32 additions.
 //
-// One CTA per 128 tokens: warp 0 fills a 4-stage ring, per 32-wide K step with the x tile
-// (128 x 32 BF16, TMA, 64-byte swizzle) and the three weight tiles (3 x E x 32 BF16, one
-// bulk copy: the split weights are stored pre-tiled in that swizzled order); warp 1 owns
-// TMEM (E columns) and issues 2 x 3 MMAs (M = 128, N = E, K = 16) per stage; warps 2..5 read their token's E
-// logits from TMEM, keep a running top-k (larger logit first, equal logits -> lower
-// expert index), write the logits, the chosen ids and the renormalised weights (softmax
-// over the chosen logits = p_j / sum_chosen p).
+// One CTA per 128 x HALVES tokens (HALVES = 1 or 2): warp 0 fills a 4-stage (3-stage) ring,
+// per 32-wide K step with the x tile (128 HALVES x 32 BF16, TMA, 64-byte swizzle) and the
+// three weight tiles (3 x E x 32 BF16, one bulk copy: the split weights are stored
+// pre-tiled in that swizzled order); warp 1 owns TMEM (one accumulator of E columns per
+// 128 tokens) and issues 2 x 3 x HALVES MMAs (M = 128, N = E, K = 16) per stage.  Every CTA
+// streams the whole 7.9 MB weight split; two halves per CTA halve that traffic per token,
+// which pays once a batch needs more than one wave of 128-token CTAs (measured: 0.31 vs
+// 0.41 ms at 32K tokens, 0.41 vs 0.36 ms at 16K).  Warps 2..(4 HALVES + 1) read their
+// token's E logits from TMEM, keep a running top-k (larger logit first, equal logits ->
+// lower expert index), write the logits, the chosen ids and the renormalised weights
+// (softmax over the chosen logits = p_j / sum_chosen p).
 #include <algorithm>
 
 #include "common.cuh"
@@ -25,22 +29,31 @@
 
 namespace beam {
 
-constexpr int RT_BM = 128;
+constexpr int RT_MMA_M = 128;
 constexpr int RT_BK = 32;  // BF16 values per K step = one 64-byte swizzle row
-constexpr int RT_STAGES = 4;
-constexpr int RT_A_BYTES = RT_BM * 64;
-constexpr int RT_THREADS = 192;
+constexpr int RT_MAX_STAGES = 4;
+template <int HALVES>
+struct RtShape {
+  static constexpr int BM = HALVES * RT_MMA_M;  // tokens per CTA
+  static constexpr int STAGES = HALVES == 1 ? 4 : 3;
+  static constexpr int A_BYTES = BM * 64;
+  static constexpr int THREADS = (2 + 4 * HALVES) * 32;
+};
 
 struct __align__(8) RouterSmemTail {
-  uint64_t full[RT_STAGES];
-  uint64_t empty[RT_STAGES];
+  uint64_t full[RT_MAX_STAGES];
+  uint64_t empty[RT_MAX_STAGES];
   uint64_t acc_full;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-static size_t router_tc_stage_bytes(int E) { return RT_A_BYTES + 3 * static_cast<size_t>(E) * 64; }
-size_t router_tc_smem_bytes(int E) { return RT_STAGES * router_tc_stage_bytes(E) + sizeof(RouterSmemTail) + 1024; }
+template <int HALVES>
+static size_t router_tc_smem(int E) {
+  using S = RtShape<HALVES>;
+  return S::STAGES * (S::A_BYTES + 3 * static_cast<size_t>(E) * 64) + sizeof(RouterSmemTail) + 1024;
+}
+size_t router_tc_smem_bytes(int E) { return std::max(router_tc_smem<1>(E), router_tc_smem<2>(E)); }
 
 // E columns of TMEM rounded up to a power of two >= 32
 static __host__ __device__ uint32_t tmem_cols_for(int E) {
@@ -49,17 +62,19 @@ static __host__ __device__ uint32_t tmem_cols_for(int E) {
   return c;
 }
 
-__global__ void __launch_bounds__(RT_THREADS, 1)
+template <int HALVES>
+__global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ w_tiles, int T,
                      int H, int E, int k, float* __restrict__ logits, int32_t* __restrict__ ids,
                      float* __restrict__ wout, uint32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int RT_BM = RtShape<HALVES>::BM, RT_STAGES = RtShape<HALVES>::STAGES, RT_A_BYTES = RtShape<HALVES>::A_BYTES;
   const int stage_bytes = RT_A_BYTES + 3 * E * 64;
   RouterSmemTail* tail = reinterpret_cast<RouterSmemTail*>(smem + RT_STAGES * stage_bytes);
   volatile int* abort_flag = &tail->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t tcols = tmem_cols_for(E);
+  const uint32_t tcols = tmem_cols_for(E);  // per accumulator; two are allocated
   if (threadIdx.x == 0) {
     for (int s = 0; s < RT_STAGES; ++s) {
       mbar_init(&tail->full[s], 1);
@@ -70,7 +85,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tail->tmem_base, tcols);
+    tmem_alloc(&tail->tmem_base, HALVES * tcols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -116,7 +131,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     if (lane == 0) {
       // BF16 x BF16 -> FP32, K-major A and B, N = E, M = 128
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(E) >> 3) << 17) |
-                             ((RT_BM >> 4) << 24);
+                             ((RT_MMA_M >> 4) << 24);
       int stage = 0;
       uint32_t phase = 0;
       for (int kt = 0; kt < k_tiles; ++kt) {
@@ -126,9 +141,13 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-          for (int p = 0; p < 3; ++p)
-            tc_mma_bf16(tmem, sdesc_k_sw64(sa + kb * 32), sdesc_k_sw64(sa + RT_A_BYTES + p * E * 64 + kb * 32), idesc,
-                        (kt | kb | p) != 0);
+          for (int p = 0; p < 3; ++p) {
+            const uint64_t bdesc = sdesc_k_sw64(sa + RT_A_BYTES + p * E * 64 + kb * 32);
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h)  // tokens 128 h .. 128 h + 127: rows start 128 x 64 bytes in
+              tc_mma_bf16(tmem + h * tcols, sdesc_k_sw64(sa + h * RT_MMA_M * 64 + kb * 32), bdesc, idesc,
+                          (kt | kb | p) != 0);
+          }
         tc_commit(&tail->empty[stage]);
         if (++stage == RT_STAGES) {
           stage = 0;
@@ -144,7 +163,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int quarter = warp & 3;
-    const int t = m0 + quarter * 32 + lane;
+    const int half = (warp - 2) >> 2;  // which accumulator (128-token half)
+    const int t = m0 + half * RT_MMA_M + quarter * 32 + lane;
     const bool ok = mbar_wait_bounded(&tail->acc_full, 0, abort_flag);
     tc_fence_after();
     float best_v[16];
@@ -155,7 +175,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
       best_e[j] = 0x7fffffff;
     }
     float thr = -INFINITY;  // current k-th largest
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t t_lane = tmem + half * tcols + (static_cast<uint32_t>(quarter * 32) << 16);
     for (int c0 = 0; c0 < E; c0 += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(t_lane + c0, v);  // E % 16 == 0: columns past E are never used
@@ -212,7 +232,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (threadIdx.x == 0 && tail->abort_flag) atomicOr(err, kErrTimeoutMma);
-  if (warp == 1) tmem_dealloc(tmem, tcols);
+  if (warp == 1) tmem_dealloc(tmem, HALVES * tcols);
 }
 
 // W_r [E][H] FP32 -> BF16 parts hi, mid, lo (each rounded to nearest even), stored as
@@ -252,14 +272,29 @@ bool router_tc_supported(int T, int H, int E, int k) {
          router_tc_smem_bytes(E) <= 227 * 1024;
 }
 
-cudaError_t launch_router_tc(const CUtensorMap& map_x, const uint16_t* w_tiles, int T, int H, int E, int k,
-                             float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s) {
-  const size_t smem = router_tc_smem_bytes(E);
-  cudaError_t e =
-      cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+int router_tc_tokens_per_cta(int T, int num_sms) {
+  // two halves per CTA once 128-token CTAs would need more than one wave
+  return T > num_sms * RT_MMA_M ? 2 * RT_MMA_M : RT_MMA_M;
+}
+
+template <int HALVES>
+static cudaError_t launch_router_tc_t(const CUtensorMap& map_x, const uint16_t* w_tiles, int T, int H, int E, int k,
+                                      float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s) {
+  using S = RtShape<HALVES>;
+  const size_t smem = router_tc_smem<HALVES>(E);
+  cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<HALVES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(router_tc_kernel, dim3((T + RT_BM - 1) / RT_BM), dim3(RT_THREADS), smem, s, map_x,
+  return launch_pdl(router_tc_kernel<HALVES>, dim3((T + S::BM - 1) / S::BM), dim3(S::THREADS), smem, s, map_x,
                     reinterpret_cast<const uint8_t*>(w_tiles), T, H, E, k, logits, ids, wout, err);
+}
+
+cudaError_t launch_router_tc(const CUtensorMap& map_x, int tokens_per_cta, const uint16_t* w_tiles, int T, int H,
+                             int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s) {
+  if (tokens_per_cta == 2 * RT_MMA_M)
+    return launch_router_tc_t<2>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, s);
+  if (tokens_per_cta == RT_MMA_M) return launch_router_tc_t<1>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, s);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace beam

@@ -205,22 +205,35 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
   const float six_alpha = __fmul_rn(6.0f, alpha);
   const int nb = H / 16, kgroups = H / 64;
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
-  for (int b = lane; b < nb; b += 32) {
-    const uint4 p0 = __ldg(xr + 2 * b), p1 = __ldg(xr + 2 * b + 1);
-    const uint32_t u[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    float v[16];
+  // Lanes 2c, 2c + 1 hold the two halves of one 16-byte code chunk and lanes 4g..4g + 3 the
+  // four scale bytes of one K-group (nb is a multiple of 4): one 16-byte code store per lane
+  // pair and one 4-byte scale store per lane quad, per slot.
+  for (int b0 = 0; b0 < nb; b0 += 32) {
+    const int b = b0 + lane;
+    const bool active = b < nb;  // whole quads are active or not
+    uint32_t lo = 0, hi = 0, sc = 0;
+    if (active) {
+      const uint4 p0 = __ldg(xr + 2 * b), p1 = __ldg(xr + 2 * b + 1);
+      const uint32_t u[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      float v[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[2 * i] = bf16_bits_to_f32(u[i] & 0xFFFFu);
-      v[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16_bits_to_f32(u[i] & 0xFFFFu);
+        v[2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+      }
+      sc = quant_block16(v, alpha, six_alpha, lo, hi);
     }
-    uint32_t lo, hi;
-    const uint32_t sc = quant_block16(v, alpha, six_alpha, lo, hi);
+    const uint32_t lo1 = __shfl_down_sync(0xffffffffu, lo, 1), hi1 = __shfl_down_sync(0xffffffffu, hi, 1);
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc, 1);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
+    const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    if (!active || (lane & 1)) continue;
     for (int j = 0; j < k; ++j) {
       const int blk = s_blk[warp][j], m = s_m[warp][j];
-      *reinterpret_cast<uint2*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1) + (b & 1) * 8) =
-          make_uint2(lo, hi);
-      a1_sf[sf_atom_offset(blk, kgroups, m, b)] = static_cast<uint8_t>(sc);
+      *reinterpret_cast<uint4*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1)) =
+          make_uint4(lo, hi, lo1, hi1);
+      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, kgroups, m, b)) = word;
     }
   }
 }

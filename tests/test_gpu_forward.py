@@ -64,7 +64,8 @@ def _run(bm, shape, tokens, seed, max_tokens=None):
 
 
 @pytest.mark.parametrize("name,tokens,seed", [("tiny", 4, 0), ("tiny", 1, 1), ("tiny", 37, 2), ("tiny", 1500, 3),
-                                              ("mid", 200, 4), ("mid", 7, 5)])
+                                              ("mid", 200, 4), ("mid", 7, 5), ("mid", 4500, 13),
+                                              ("tiny", 19500, 14)])
 def test_forward_stages_and_end_to_end(bm, name, tokens, seed):
     shape, layer, weights, out, ref, (x, res, wr, g, cache, a1, a2) = _run(bm, SHAPES[name], tokens, seed)
     T, E, k, H, I = tokens, shape.experts, shape.top_k, shape.hidden, shape.inter
