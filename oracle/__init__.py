@@ -22,7 +22,9 @@ an FP32 tensor scale, post-RMSNorm with eps 1e-6) is the stated convention of th
 this repository implements.
 
 Precision: every floating-point step is FP64 except the NVFP4 quantiser, whose steps are
-IEEE FP32 operations by definition (so codes are reproducible bit for bit).
+IEEE FP32 operations by definition (so codes are reproducible bit for bit).  The MXFP8
+variant of the experts (``mxfp8.py``: E4M3 values, one power-of-two scale per 32 values)
+needs no FP32 step: its scaling is exact.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py`` (library
 routines for the rounding, closed forms, brute force and invariants).  No function is
@@ -40,6 +42,14 @@ from .nvfp4 import (  # noqa: F401
     dequantize_nvfp4,
     pack_nibbles,
     unpack_nibbles,
+)
+from .mxfp8 import (  # noqa: F401
+    e4m3_encode_signed,
+    e4m3_decode_signed,
+    scale_exponent,
+    ue8m0_decode,
+    quantize_mxfp8,
+    dequantize_mxfp8,
 )
 from .moe import (  # noqa: F401
     router_logits,

@@ -12,9 +12,10 @@ Steps, in order ([P1] "Status"/"Remaining work", [P2] "Overview"/"Variants", [P3
   5. token -> expert histogram, exclusive prefix sum (offsets), and the permutation
      that lists the rows of expert e in [offsets[e], offsets[e+1]) in ascending token order
   6. A1 = Q(x, alpha_a1)                              (NVFP4 activation, W4A4)
+     (MXFP8 variant: A1 = MX(x), no tensor scale; see mxfp8.py for the reading)
   7. G = deq(A1) deq(W_gate)^T, U = deq(A1) deq(W_up)^T  per expert (FP64)
   8. h = G * sigmoid(G) * U                           (SwiGLU), rounded to FP32
-  9. A2 = Q(h, alpha_a2)
+  9. A2 = Q(h, alpha_a2)                              (MXFP8 variant: A2 = MX(h))
  10. y = deq(A2) deq(W_down)^T                        (FP64)
  11. m = sum_j w_j y_j                                (weighted un-permute, MoE finalize)
  12. n = m / sqrt(mean(m^2) + eps) * gamma            (post-RMSNorm of the sandwich norm)
@@ -28,7 +29,10 @@ from __future__ import annotations
 
 import numpy as np
 
+from .mxfp8 import dequantize_mxfp8, quantize_mxfp8
 from .nvfp4 import dequantize_nvfp4, quantize_nvfp4, tensor_scale
+
+FORMATS = ("nvfp4", "mxfp8")
 
 
 # ----------------------------------------------------------------------------- routing
@@ -90,12 +94,20 @@ def permute(ids: np.ndarray, num_experts: int):
 
 
 # ----------------------------------------------------------------------------- experts
-def quantize_expert(w_gu: np.ndarray, w_d: np.ndarray):
-    """NVFP4 weights of one expert ([P2] "Variants": routed experts are NVFP4).
+def quantize_expert(w_gu: np.ndarray, w_d: np.ndarray, fmt: str = "nvfp4"):
+    """Quantised weights of one expert ([P2] "Variants": routed experts are NVFP4; the FP8
+    checkpoint is the second variant, MXFP8 here).
 
     w_gu: FP32 [2I, H] (rows 0..I-1 gate, I..2I-1 up); w_d: FP32 [H, I].
-    One tensor scale for gate+up together and one for down, each amax / 2688.
+    NVFP4: one tensor scale for gate+up together and one for down, each amax / 2688.
+    MXFP8: E4M3 codes with one UE8M0 scale per 32 values of a row, no tensor scale.
     """
+    if fmt == "mxfp8":
+        gu_c, gu_s = quantize_mxfp8(w_gu)
+        d_c, d_s = quantize_mxfp8(w_d)
+        return dict(fmt="mxfp8", w_gu=gu_c, w_gu_sf=gu_s, w_d=d_c, w_d_sf=d_s)
+    if fmt != "nvfp4":
+        raise ValueError(f"unknown expert format {fmt!r}")
     a_gu = tensor_scale(w_gu)
     a_d = tensor_scale(w_d)
     gu_p, gu_s = quantize_nvfp4(w_gu, a_gu)
@@ -105,6 +117,8 @@ def quantize_expert(w_gu: np.ndarray, w_d: np.ndarray):
 
 def dequantize_expert(q):
     """FP64 gate/up [2I, H] and down [H, I] of a quantised expert."""
+    if q.get("fmt") == "mxfp8":
+        return dequantize_mxfp8(q["w_gu"], q["w_gu_sf"]), dequantize_mxfp8(q["w_d"], q["w_d_sf"])
     return (
         dequantize_nvfp4(q["w_gu"], q["w_gu_sf"], q["w_gu_alpha"]),
         dequantize_nvfp4(q["w_d"], q["w_d_sf"], q["w_d_alpha"]),
@@ -116,20 +130,36 @@ def swiglu(g: np.ndarray, u: np.ndarray) -> np.ndarray:
     return g / (1.0 + np.exp(-g)) * u
 
 
-def expert_forward(a1_packed, a1_sf, alpha_a1, deq_w, alpha_a2):
+def quantize_act(v, alpha, fmt: str = "nvfp4"):
+    """Activation quantiser of steps 6 and 9: NVFP4 Q(v, alpha), or MXFP8 (alpha unused).
+    Returns (codes, scale codes): packed E2M1 [.., K/2] + E4M3 [.., K/16], or E4M3 [.., K]
+    + UE8M0 [.., K/32]."""
+    if fmt == "mxfp8":
+        return quantize_mxfp8(v)
+    return quantize_nvfp4(v, alpha)
+
+
+def dequantize_act(codes, sf, alpha, fmt: str = "nvfp4"):
+    if fmt == "mxfp8":
+        return dequantize_mxfp8(codes, sf)
+    return dequantize_nvfp4(codes, sf, alpha)
+
+
+def expert_forward(a1_packed, a1_sf, alpha_a1, deq_w, alpha_a2, fmt: str = "nvfp4"):
     """Steps 7-10 for the rows routed to one expert.
 
-    a1_packed/a1_sf: NVFP4 rows of that expert's inputs; deq_w: (gate/up, down) in FP64.
-    Returns dict(h32 [R, I] FP32, a2_packed, a2_sf, y [R, H] FP64).
+    a1_packed/a1_sf: quantised rows of that expert's inputs (format fmt); deq_w: (gate/up,
+    down) in FP64.  Returns dict(h32 [R, I] FP32, a2_packed, a2_sf, y [R, H] FP64); for
+    MXFP8 a2_packed holds one E4M3 code per value.
     """
     w_gu, w_d = deq_w
     inter = w_gu.shape[0] // 2
-    a1 = dequantize_nvfp4(a1_packed, a1_sf, alpha_a1)
+    a1 = dequantize_act(a1_packed, a1_sf, alpha_a1, fmt)
     g = a1 @ w_gu[:inter].T
     u = a1 @ w_gu[inter:].T
     h32 = swiglu(g, u).astype(np.float32)
-    a2_packed, a2_sf = quantize_nvfp4(h32, alpha_a2)
-    a2 = dequantize_nvfp4(a2_packed, a2_sf, alpha_a2)
+    a2_packed, a2_sf = quantize_act(h32, alpha_a2, fmt)
+    a2 = dequantize_act(a2_packed, a2_sf, alpha_a2, fmt)
     y = a2 @ w_d.T
     return dict(h32=h32, a2_packed=a2_packed, a2_sf=a2_sf, y=y)
 
@@ -179,19 +209,23 @@ def next_prenorm(out_bf16: np.ndarray, gamma_next: np.ndarray, eps: float):
 class ExpertCache:
     """Quantises (with this oracle's quantiser) and dequantises experts on first use.
 
-    get_fp32(e) must return the FP32 weights (w_gu [2I, H], w_d [H, I]) of expert e.
+    get_fp32(e) must return the FP32 weights (w_gu [2I, H], w_d [H, I]) of expert e;
+    fmt is the experts' format ("nvfp4" or "mxfp8").
     """
 
-    def __init__(self, get_fp32, keep: int = 64):
+    def __init__(self, get_fp32, keep: int = 64, fmt: str = "nvfp4"):
+        if fmt not in FORMATS:
+            raise ValueError(f"unknown expert format {fmt!r}")
         self.get_fp32 = get_fp32
         self.keep = keep
+        self.fmt = fmt
         self._deq = {}
         self._q = {}
 
     def quantized(self, e: int):
         if e not in self._q:
             w_gu, w_d = self.get_fp32(e)
-            self._q[e] = quantize_expert(w_gu, w_d)
+            self._q[e] = quantize_expert(w_gu, w_d, self.fmt)
         return self._q[e]
 
     def dequantized(self, e: int):
@@ -205,7 +239,8 @@ class ExpertCache:
 def moe_forward_tokens(x, residual, router_w, gamma, experts: ExpertCache, top_k, alpha_a1, alpha_a2,
                        eps=1e-6):
     """Steps 1-4 and 6-13 for a set of tokens (each token's output depends on that token
-    only, so any subset of a batch gives the same rows as the whole batch).
+    only, so any subset of a batch gives the same rows as the whole batch).  The
+    activations use the experts' format; alpha_a1 / alpha_a2 are unused for MXFP8.
 
     x, residual: FP64 [T, H] (exact BF16 values).  Returns dict with logits, ids, w,
     near_tie, a1 (packed, sf), h32 [T, k, I], y [T, k, H], out_pre, out (BF16 as FP64).
@@ -214,12 +249,13 @@ def moe_forward_tokens(x, residual, router_w, gamma, experts: ExpertCache, top_k
     t_count, hidden = x.shape
     logits = router_logits(x, router_w)
     ids, w, _ = route_topk(logits, top_k)
-    a1_packed, a1_sf = quantize_nvfp4(x.astype(np.float32), alpha_a1)
+    fmt = experts.fmt
+    a1_packed, a1_sf = quantize_act(x.astype(np.float32), alpha_a1, fmt)
     y = np.zeros((t_count, top_k, hidden), np.float64)
     h32 = None
     for e in np.unique(ids):
         tt, jj = np.nonzero(ids == e)
-        r = expert_forward(a1_packed[tt], a1_sf[tt], alpha_a1, experts.dequantized(int(e)), alpha_a2)
+        r = expert_forward(a1_packed[tt], a1_sf[tt], alpha_a1, experts.dequantized(int(e)), alpha_a2, fmt)
         if h32 is None:
             h32 = np.zeros((t_count, top_k, r["h32"].shape[1]), np.float32)
         h32[tt, jj] = r["h32"]
