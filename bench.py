@@ -46,15 +46,20 @@ def peaks():
 
 
 # ------------------------------------------------------------------ algorithmic work
-def kernel_work(shape: mi.LayerShape, T: int, counts: np.ndarray) -> dict:
+# bytes per quantised value: NVFP4 0.5 B + one scale byte per 16 values; MXFP8 1 B + one
+# scale byte per 32 values
+BYTES_PER_VALUE = {"nvfp4": 0.5625, "mxfp8": 1.03125}
+
+
+def kernel_work(shape: mi.LayerShape, T: int, counts: np.ndarray, fmt: str = "nvfp4") -> dict:
     """Algorithmic bytes and FLOPs of each kernel for one forward (T tokens).
 
-    NVFP4 costs 0.5 B per value plus one scale byte per 16 values (0.5625 B/value).  Only
-    the experts that received tokens have their weights read."""
+    Quantised operands cost BYTES_PER_VALUE[fmt] per value.  Only the experts that received
+    tokens have their weights read."""
     H, I, E, k = shape.hidden, shape.inter, shape.experts, shape.top_k
     R = T * k
     used = int((counts > 0).sum())
-    q = 0.5625
+    q = BYTES_PER_VALUE[fmt]
     return {
         "router": dict(bytes=E * H * 4 + T * H * 2 + T * E * 4, flops=2 * T * H * E),
         "topk": dict(bytes=T * E * 4 + R * 8, flops=0),
@@ -139,7 +144,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle leg
-def oracle_sample(shape: mi.LayerShape, tokens, seed=0):
+def oracle_sample(shape: mi.LayerShape, tokens, seed=0, fmt="nvfp4"):
     """Inputs and quantised experts the oracle needs for a token sample (prepared untimed)."""
     from oracle import moe
     xs, rs = [], []
@@ -152,17 +157,17 @@ def oracle_sample(shape: mi.LayerShape, tokens, seed=0):
     wr = mi.router_weight(shape, seed)
     g = mi.bf16_bits_to_f32(mi.gamma(shape, seed)).astype(np.float64)
     ids, _, _ = moe.route_topk(moe.router_logits(x, wr), shape.top_k)
-    quantised = {int(e): moe.quantize_expert(*mi.expert_weights(shape, seed, int(e))) for e in np.unique(ids)}
-    return x, res, wr, g, quantised
+    quantised = {int(e): moe.quantize_expert(*mi.expert_weights(shape, seed, int(e)), fmt) for e in np.unique(ids)}
+    return x, res, wr, g, quantised, fmt
 
 
 def oracle_step(shape, sample):
     """One oracle forward of the sample: routing, experts (dequantised from the stored
-    NVFP4 weights, FP64 matmuls), finalize.  Returns tokens processed."""
+    quantised weights, FP64 matmuls), finalize.  Returns tokens processed."""
     from oracle import moe
-    x, res, wr, g, quantised = sample
-    a1, a2 = mi.activation_scales(shape)
-    cache = moe.ExpertCache(lambda e: None, keep=2)
+    x, res, wr, g, quantised, fmt = sample
+    a1, a2 = mi.activation_scales(shape) if fmt == "nvfp4" else (None, None)
+    cache = moe.ExpertCache(lambda e: None, keep=2, fmt=fmt)
     cache._q = dict(quantised)
     moe.moe_forward_tokens(x, res, wr, g, cache, shape.top_k, a1, a2, shape.rms_eps)
     return x.shape[0]
@@ -181,9 +186,9 @@ def cpu_sample_tokens(shape):
     return [0] if shape.tokens <= 64 else [0, shape.tokens // 2]
 
 
-def cpu_baseline(shape, budget_s=25.0):
+def cpu_baseline(shape, budget_s=25.0, fmt="nvfp4"):
     toks = cpu_sample_tokens(shape)
-    sample = oracle_sample(shape, toks)
+    sample = oracle_sample(shape, toks, fmt=fmt)
     t0 = time.perf_counter()
     n = 0
     reps = 0
@@ -195,13 +200,13 @@ def cpu_baseline(shape, budget_s=25.0):
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
             "sample": f"{len(toks)} token(s) of the {shape.name} batch x {reps} repeats: FP64 router, "
-                      f"NVFP4 experts dequantised from stored codes, finalize; weights pre-quantised untimed"}
+                      f"{fmt.upper()} experts dequantised from stored codes, finalize; weights pre-quantised untimed"}
 
 
 def run_reference(args, shape, rank, world):
     if rank != 0:
         return
-    sample = oracle_sample(shape, cpu_sample_tokens(shape))
+    sample = oracle_sample(shape, cpu_sample_tokens(shape), fmt=args.experts_format)
     for _ in range(args.warmup):
         oracle_step(shape, sample)
     t0 = time.perf_counter()
@@ -213,7 +218,7 @@ def run_reference(args, shape, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(shape),
+        "config": workload_config(shape, fmt=args.experts_format),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{len(cpu_sample_tokens(shape))} token(s) of the {shape.name} batch per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -221,13 +226,13 @@ def run_reference(args, shape, rank, world):
     emit(line, rank)
 
 
-def workload_config(shape, l2_flush="write"):
+def workload_config(shape, l2_flush="write", fmt="nvfp4"):
     l2 = f"flushed: {L2_FLUSH_BYTES >> 20} MiB write between timed steps"
     if l2_flush == "write+read":
         l2 = f"flushed: {L2_FLUSH_BYTES >> 20} MiB write + {L2_FLUSH_BYTES >> 21} MiB read between timed steps"
     return {"workload": shape.name, "tokens": shape.tokens, "hidden": shape.hidden, "experts": shape.experts,
             "top_k": shape.top_k, "inter": shape.inter, "routing": "zipf-skewed" if shape.skew else "uniform",
-            "l2": l2}
+            "experts_format": fmt, "l2": l2}
 
 
 # ------------------------------------------------------------------ multi-rank plumbing
@@ -265,8 +270,9 @@ def run_ours(args, shape, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
-    weights = synthetic.make_weights(shape, 0, device=dev)
-    layer = synthetic.make_layer(shape, weights)
+    fmt = args.experts_format
+    weights = synthetic.make_weights(shape, 0, device=dev, fmt=fmt)
+    layer = synthetic.make_layer(shape, weights, fmt=fmt)
     del weights  # the handle holds its own repacked copy
     torch.cuda.empty_cache()
     x, res = synthetic.make_batch(shape, seed=rank)  # each replica its own batch
@@ -326,19 +332,23 @@ def run_ours(args, shape, rank, world, local_rank):
     kern = {n: sum(v) / len(v) for n, v in acc.items()}
     offsets = np.frombuffer(layer.debug(bm.BUF_OFFSETS).cpu().numpy().tobytes(), np.int32)
     counts = np.diff(offsets)
-    work = kernel_work(shape, T, counts)
+    work = kernel_work(shape, T, counts, fmt)
     top = max(kern, key=kern.get)
     pk = peaks()
     wk = work[top]
-    if wk["flops"] > 0 and wk["flops"] / max(wk["bytes"], 1) > (4 * pk["bf16_sus"] * 1e12) / (pk["hbm"] * 1e9):
-        bound, achieved, peak, unit = ("tensor", wk["flops"] / (kern[top] / 1e3) / 1e12, 4 * pk["bf16_sus"],
+    # the contraction's own dtype: NVFP4 = 4 x BF16 (nominal 9 / 2.25 PF), FP8 = 2 x (4.5 / 2.25)
+    ratio = 4 if fmt == "nvfp4" else 2
+    if wk["flops"] > 0 and wk["flops"] / max(wk["bytes"], 1) > (ratio * pk["bf16_sus"] * 1e12) / (pk["hbm"] * 1e9):
+        bound, achieved, peak, unit = ("tensor", wk["flops"] / (kern[top] / 1e3) / 1e12, ratio * pk["bf16_sus"],
                                        "TFLOP/s")
-        peak_note = f"NVFP4 dense = 4 x {pk['src']} sustained BF16 cuBLAS peak (nominal 9 / 2.25 PF ratio)"
+        peak_note = (f"{'NVFP4' if fmt == 'nvfp4' else 'FP8'} dense = {ratio} x {pk['src']} sustained BF16 cuBLAS "
+                     f"peak (nominal {'9' if fmt == 'nvfp4' else '4.5'} / 2.25 PF ratio)")
     else:
         bound, achieved, peak, unit = "hbm", wk["bytes"] / (kern[top] / 1e3) / 1e9, pk["hbm"], "GB/s"
         peak_note = f"{pk['src']} copy bandwidth"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": read_traffic(top, work["_used_experts"], T), "kernel": top, "kernel_ms": kern[top],
+                "traffic": read_traffic(top if fmt == "nvfp4" else f"{top}_{fmt}", work["_used_experts"], T),
+                "kernel": top, "kernel_ms": kern[top],
                 "peak_source": peak_note}
 
     # ---- end to end through the host-buffer entry point (copies inside the timed region)
@@ -366,9 +376,11 @@ def run_ours(args, shape, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) experts, fp32 router and accumulation",
+            "vs_baseline": None,
+            "dtype": ("nvfp4 (e2m1 x e4m3/16) experts" if fmt == "nvfp4" else "mxfp8 (e4m3 x ue8m0/32) experts")
+                     + ", fp32 router and accumulation",
             "data": "synthetic (seeded; random-init weights of the layer's shapes)",
-            "config": dict(workload_config(shape, args.l2_flush), parallelism=f"token-dp replicas x{world}"),
+            "config": dict(workload_config(shape, args.l2_flush, fmt), parallelism=f"token-dp replicas x{world}"),
             "roofline": roofline,
             "kernels_ms": kern,
             "used_experts": work["_used_experts"],
@@ -389,6 +401,8 @@ def main():
     ap.add_argument("--workload", default="decode8", choices=sorted(mi.SHAPES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts-format", default="nvfp4", choices=["nvfp4", "mxfp8"],
+                    help="routed experts in NVFP4 (default) or the block-scaled FP8 variant (MXFP8)")
     ap.add_argument("--l2-flush", default="write+read", choices=["write", "write+read"],
                     help="between timed steps: write 512 MiB, then (default) read 256 MiB so the step starts "
                          "with L2 cold and clean")
@@ -413,7 +427,7 @@ def main():
             import torch.distributed as dist
             dist.destroy_process_group()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(shape)
+        line["cpu_baseline"] = cpu_baseline(shape, fmt=args.experts_format)
     emit(line, rank)
 
 

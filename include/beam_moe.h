@@ -11,6 +11,8 @@
  *     "reflection/Beam-1.0-501B-A23B", section "Overview"), weights renormalised over
  *     the chosen 8;
  *   - routed experts in NVFP4, W4A4 on Blackwell (recipe, section "Variants"), SwiGLU;
+ *     or, as the second precision variant, block-scaled FP8 W8A8 experts (the recipe's FP8
+ *     checkpoint, same section), read as MXFP8 (beam_moe_create_mxfp8);
  *   - MoE finalize: weighted un-permute, post-RMSNorm of the sandwich norm (eps 1e-6)
  *     and residual add (PR, sections "Status" and "Remaining work").
  *
@@ -29,6 +31,9 @@
  *   - NVFP4 data: two 4-bit E2M1 codes per byte, element 2i in the low nibble; one
  *     unsigned E4M3 scale byte per 16 consecutive elements of a row; one FP32 tensor
  *     scale alpha per tensor; value = e2m1 * e4m3 * alpha.
+ *   - MXFP8 data (the block-scaled FP8 expert variant, beam_moe_create_mxfp8): one
+ *     signed E4M3 code per byte; one UE8M0 scale byte S per 32 consecutive elements of a
+ *     row (an exponent with bias 127); no tensor scale; value = e4m3 * 2^(S - 127).
  */
 #ifndef BEAM_MOE_H_
 #define BEAM_MOE_H_
@@ -91,6 +96,34 @@ typedef struct beam_moe_ctx* beam_moe_t;
  * beam_moe_destroy.  Returns INVALID_ARG / UNSUPPORTED / OOM / CUDA. */
 BEAM_MOE_API beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weights* weights, void* stream,
                                 beam_moe_t* out);
+
+/* Block-scaled FP8 (W8A8) experts, the second precision variant of the routed experts
+ * (recipe "reflection/Beam-1.0-501B-A23B", section "Variants": an FP8 checkpoint next to
+ * the NVFP4 one).  The pages do not give the FP8 block layout; this library reads it as
+ * the OCP microscaling format MXFP8, which the sm_100a tensor cores scale natively:
+ * E4M3 values, one power-of-two scale per 32 values along the contraction dimension,
+ * for the weights and for both activations (A1 = MX(x), A2 = MX(SwiGLU)).  Activation
+ * scales are chosen per 32-value block on the device: 2^e with e the smallest integer
+ * such that amax <= 448 * 2^e (e >= -127), so nothing saturates. */
+typedef struct {
+  const float* router_w;   /* [E][H] FP32, row e = expert e                              */
+  const uint8_t* w_gu;     /* [E][2I][H] E4M3 codes; rows 0..I-1 gate, I..2I-1 up       */
+  const uint8_t* w_gu_sf;  /* [E][2I][H/32] UE8M0 scales, row-major                     */
+  const uint8_t* w_d;      /* [E][H][I] E4M3 codes of the down projection              */
+  const uint8_t* w_d_sf;   /* [E][H][I/32] UE8M0 scales                                 */
+  const uint16_t* gamma;   /* [H] BF16 RMSNorm weight                                    */
+} beam_moe_weights_mxfp8;
+
+/* beam_moe_create for MXFP8 experts.  cfg->alpha_a1 and cfg->alpha_a2 are not used (MX
+ * activations have no tensor scale).  Same shape limits, ownership, synchronisation and
+ * errors as beam_moe_create.  Every other entry point takes the handle unchanged; the
+ * CTA-pair expert GEMM is NVFP4 only (beam_moe_set_gemm_mode(PAIR) returns UNSUPPORTED). */
+BEAM_MOE_API beam_moe_status beam_moe_create_mxfp8(const beam_moe_config* cfg, const beam_moe_weights_mxfp8* weights,
+                                                   void* stream, beam_moe_t* out);
+
+/* Expert format of a handle: BEAM_MOE_FMT_NVFP4 or BEAM_MOE_FMT_MXFP8 (-1 for NULL). */
+enum { BEAM_MOE_FMT_NVFP4 = 0, BEAM_MOE_FMT_MXFP8 = 1 };
+BEAM_MOE_API int32_t beam_moe_expert_format(beam_moe_t h);
 
 /* out[T][H] = residual + RMSNorm(sum_j w_j * expert_{id_j}(x)) * gamma, rounded to BF16.
  * x, residual, out: [num_tokens][H] BF16 row-major, caller-owned, device memory.
@@ -159,6 +192,12 @@ BEAM_MOE_API beam_moe_status beam_moe_route_static(const void* x, const float* r
 BEAM_MOE_API beam_moe_status beam_moe_quantize_nvfp4(const float* src, int64_t rows, int64_t cols, float alpha, uint8_t* codes,
                                         uint8_t* sf, float* alpha_out, void* stream);
 
+/* MXFP8 quantiser (weights or activations), the rule of beam_moe_create_mxfp8:
+ * src [rows][cols] FP32 row-major, finite, cols % 32 == 0.  codes [rows][cols] E4M3,
+ * sf [rows][cols/32] UE8M0 (row-major scale bytes).  codes must be 16-byte aligned. */
+BEAM_MOE_API beam_moe_status beam_moe_quantize_mxfp8(const float* src, int64_t rows, int64_t cols, uint8_t* codes,
+                                                     uint8_t* sf, void* stream);
+
 /* Internal buffers of the last forward, for tests (layouts in the comment of each id). */
 typedef enum {
   BEAM_MOE_BUF_LOGITS = 0,   /* [S][T][E] FP32 partial sums over S slices of H (S = size/(4TE)) */
@@ -179,7 +218,11 @@ typedef enum {
  * Scale blocks: scale s of that row is the byte at
  * ((blk * (K/64) + s/4) * 512) + (m%32)*16 + (m/32)*4 + s%4.
  * Activation tiles: codes byte j of that row (values 2j, 2j+1) is at
- * ((blk * (K/256) + j/128) * 16384) + m*128 + ((((j%128)/16) ^ (m%8)) * 16) + j%16. */
+ * ((blk * (K/256) + j/128) * 16384) + m*128 + ((((j%128)/16) ^ (m%8)) * 16) + j%16.
+ * MXFP8 handles: the same formulas with one value per code byte, one scale per 32 values
+ * and K tiles of 128 values: scale s at ((blk * (K/128) + s/4) * 512) + (m%32)*16 +
+ * (m/32)*4 + s%4, code j (value j) at ((blk * (K/128) + j/128) * 16384) + m*128 +
+ * ((((j%128)/16) ^ (m%8)) * 16) + j%16, and A2's K is I (no padding). */
 
 /* Copies min(bytes, size of the buffer) bytes of internal buffer `which` to dst (device),
  * enqueued on `stream`.  *size_out (host, may be NULL) receives the buffer's size for the
@@ -192,7 +235,7 @@ BEAM_MOE_API beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, vo
 BEAM_MOE_API beam_moe_status beam_moe_check(beam_moe_t h, void* stream);
 
 /* Expert GEMM variant for the batches that do not use the small-batch routing (more than
- * 16 tokens).  SINGLE: one CTA per 128-row work block.  PAIR: CTA pairs (clusters of two
+ * 16 tokens; NVFP4 handles).  SINGLE: one CTA per 128-row work block.  PAIR: CTA pairs (clusters of two
  * SMs sharing one M = 256 MMA) over 256-row work blocks.  AUTO (the default at create)
  * picks PAIR from BEAM_MOE_PAIR_MIN_TOKENS tokens on, SINGLE below; the threshold is set
  * where PAIR measured faster (INT32_MAX: never).  Both compute the same result up to the

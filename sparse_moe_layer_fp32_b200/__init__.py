@@ -25,8 +25,11 @@ EXPORTED = [
     "beam_moe_route_workspace_bytes", "beam_moe_quantize_nvfp4", "beam_moe_debug_copy", "beam_moe_check",
     "beam_moe_last_launch_count", "beam_moe_status_string", "beam_moe_destroy", "beam_moe_profile_enable",
     "beam_moe_profile_read", "beam_moe_kernel_name", "beam_moe_route_static", "beam_moe_debug_wait_timeout",
-    "beam_moe_forward_prenorm", "beam_moe_set_gemm_mode",
+    "beam_moe_forward_prenorm", "beam_moe_set_gemm_mode", "beam_moe_create_mxfp8", "beam_moe_quantize_mxfp8",
+    "beam_moe_expert_format",
 ]
+FMT_NVFP4, FMT_MXFP8 = 0, 1
+FORMATS = {"nvfp4": FMT_NVFP4, "mxfp8": FMT_MXFP8}
 
 
 class BeamMoeConfig(ctypes.Structure):
@@ -38,6 +41,10 @@ class BeamMoeConfig(ctypes.Structure):
 class BeamMoeWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("router_w", "w_gu", "w_gu_sf", "w_gu_alpha", "w_d", "w_d_sf", "w_d_alpha", "gamma")]
+
+
+class BeamMoeWeightsMxfp8(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("router_w", "w_gu", "w_gu_sf", "w_d", "w_d_sf", "gamma")]
 
 
 class BeamMoeError(RuntimeError):
@@ -72,6 +79,10 @@ def _load():
         "beam_moe_route_static": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
         "beam_moe_debug_wait_timeout": (i32, [vp, i64, vp]),
         "beam_moe_forward_prenorm": (i32, [vp, vp, vp, vp, vp, vp, f32, i32, vp]),
+        "beam_moe_create_mxfp8": (i32, [ctypes.POINTER(BeamMoeConfig), ctypes.POINTER(BeamMoeWeightsMxfp8), vp,
+                                        ctypes.POINTER(vp)]),
+        "beam_moe_quantize_mxfp8": (i32, [vp, i64, i64, vp, vp, vp]),
+        "beam_moe_expert_format": (i32, [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -111,6 +122,17 @@ def beam_moe_create(cfg: BeamMoeConfig, weights: BeamMoeWeights, stream=None) ->
     _check(_lib.beam_moe_create(ctypes.byref(cfg), ctypes.byref(weights), _stream(stream), ctypes.byref(h)),
            "beam_moe_create")
     return h
+
+
+def beam_moe_create_mxfp8(cfg: BeamMoeConfig, weights: BeamMoeWeightsMxfp8, stream=None) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_lib.beam_moe_create_mxfp8(ctypes.byref(cfg), ctypes.byref(weights), _stream(stream), ctypes.byref(h)),
+           "beam_moe_create_mxfp8")
+    return h
+
+
+def beam_moe_expert_format(h) -> int:
+    return int(_lib.beam_moe_expert_format(h))
 
 
 def beam_moe_forward(h, x, residual, out, num_tokens: int, stream=None):
@@ -158,6 +180,16 @@ def beam_moe_quantize_nvfp4(src, alpha: float | None = None, stream=None):
     return codes, sf, alpha_out
 
 
+def beam_moe_quantize_mxfp8(src, stream=None):
+    """MXFP8 of a 2-D FP32 CUDA tensor: (codes uint8 [r, c] E4M3, scales uint8 [r, c/32] UE8M0)."""
+    rows, cols = src.shape
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=src.device)
+    sf = torch.empty((rows, cols // 32), dtype=torch.uint8, device=src.device)
+    _check(_lib.beam_moe_quantize_mxfp8(_ptr(src.contiguous()), rows, cols, _ptr(codes), _ptr(sf), _stream(stream)),
+           "beam_moe_quantize_mxfp8")
+    return codes, sf
+
+
 def beam_moe_debug_copy(h, which: int, stream=None) -> torch.Tensor:
     size = ctypes.c_size_t(0)
     _check(_lib.beam_moe_debug_copy(h, which, None, 0, ctypes.byref(size), _stream(stream)), "beam_moe_debug_copy")
@@ -203,16 +235,29 @@ def beam_moe_profile_read(h):
 
 # ------------------------------------------------------------------ handle wrapper
 class MoELayer:
-    """Owns a beam_moe handle.  Weight tensors are CUDA tensors in the C-ABI layout."""
+    """Owns a beam_moe handle.  Weight tensors are CUDA tensors in the C-ABI layout.
 
-    def __init__(self, *, max_tokens, hidden, num_experts, top_k, inter, alpha_a1, alpha_a2, router_w, w_gu,
-                 w_gu_sf, w_gu_alpha, w_d, w_d_sf, w_d_alpha, gamma, rms_eps=1e-6, stream=None):
+    fmt="nvfp4" (beam_moe_create): NVFP4 experts with tensor scales w_gu_alpha / w_d_alpha
+    and the activation scales alpha_a1 / alpha_a2.  fmt="mxfp8" (beam_moe_create_mxfp8):
+    MXFP8 experts; the alphas are not used."""
+
+    def __init__(self, *, max_tokens, hidden, num_experts, top_k, inter, router_w, w_gu, w_gu_sf, w_d, w_d_sf,
+                 gamma, alpha_a1=1.0, alpha_a2=1.0, w_gu_alpha=None, w_d_alpha=None, rms_eps=1e-6, fmt="nvfp4",
+                 stream=None):
+        if fmt not in FORMATS:
+            raise ValueError(f"unknown expert format {fmt!r}")
+        self.fmt = fmt
         self.cfg = BeamMoeConfig(max_tokens, hidden, num_experts, top_k, inter, rms_eps, float(alpha_a1),
                                  float(alpha_a2))
-        ws = [router_w, w_gu, w_gu_sf, w_gu_alpha, w_d, w_d_sf, w_d_alpha, gamma]
-        wts = BeamMoeWeights(*[t.data_ptr() for t in ws])
         self.hidden, self.top_k = hidden, top_k
-        self.handle = beam_moe_create(self.cfg, wts, stream)
+        if fmt == "mxfp8":
+            ws = [router_w, w_gu, w_gu_sf, w_d, w_d_sf, gamma]
+            self.handle = beam_moe_create_mxfp8(self.cfg, BeamMoeWeightsMxfp8(*[t.data_ptr() for t in ws]), stream)
+        else:
+            if w_gu_alpha is None or w_d_alpha is None:
+                raise ValueError("NVFP4 experts need w_gu_alpha and w_d_alpha")
+            ws = [router_w, w_gu, w_gu_sf, w_gu_alpha, w_d, w_d_sf, w_d_alpha, gamma]
+            self.handle = beam_moe_create(self.cfg, BeamMoeWeights(*[t.data_ptr() for t in ws]), stream)
 
     def forward(self, x, residual, out=None, stream=None):
         out = torch.empty_like(residual) if out is None else out

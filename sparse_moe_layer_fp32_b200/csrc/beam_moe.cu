@@ -15,7 +15,7 @@ using namespace beam;
 
 struct beam_moe_ctx {
   beam_moe_config cfg;
-  int H, E, k, I, Ip, Tmax;
+  int H, E, k, I, Ip, Tmax;  // Ip: I rounded up to the K tile (the down GEMM's K)
   int64_t Rmax, nblk_max, n_chunks_max;
   int num_sms;
   // weights (owned, repacked)
@@ -37,6 +37,9 @@ struct beam_moe_ctx {
   unsigned int* route_counter;  // last-CTA election of the fused small-batch routing kernel
   uint32_t* sched;              // tile scheduler of the expert GEMM launch (sched_words(nblk_max))
   int32_t gemm_mode;            // BEAM_MOE_GEMM_*: which expert GEMM large batches use
+  int32_t fmt;                  // BEAM_MOE_FMT_*: expert weight and activation format
+  int kv;                       // K values per activation / weight tile: 256 (NVFP4), 128 (MXFP8)
+  int sfa_tile;                 // scale bytes per 128-row block per K tile: 2048 (NVFP4), 512
   uint16_t *stage_x, *stage_res, *stage_out;
   int last_T;
   int last_splits;  // logits layout of the last forward: [splits][T][E] partial sums
@@ -132,6 +135,14 @@ __global__ void wait_timeout_probe_kernel(uint64_t limit_ns, uint32_t* err) {
 // Kernels use 16-byte vector accesses on these pointers.
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Activation tiles and their scale blocks for a contraction of K values (multiple of kv).
+size_t act_bytes(const beam_moe_ctx* h, int K) {
+  return static_cast<size_t>(h->nblk_max) * (K / h->kv) * 16384u;
+}
+size_t act_sf_bytes(const beam_moe_ctx* h, int K) {
+  return static_cast<size_t>(h->nblk_max) * (K / h->kv) * static_cast<size_t>(h->sfa_tile);
+}
+
 }  // namespace
 
 extern "C" {
@@ -154,17 +165,27 @@ int64_t beam_moe_route_workspace_bytes(int32_t num_tokens, int32_t hidden, int32
   return route_ws_floats(num_tokens, hidden, num_experts) * static_cast<int64_t>(sizeof(float));
 }
 
-beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weights* wts, void* stream,
-                                beam_moe_t* out) {
-  if (!cfg || !wts || !out) return BEAM_MOE_ERR_INVALID_ARG;
-  *out = nullptr;
-  if (!wts->router_w || !wts->w_gu || !wts->w_gu_sf || !wts->w_gu_alpha || !wts->w_d || !wts->w_d_sf ||
-      !wts->w_d_alpha || !wts->gamma)
+}  // extern "C"
+
+namespace {
+
+// Weights of either format as create reads them (device pointers).
+struct ExpertWeightsIn {
+  const float* router_w;
+  const uint8_t *w_gu, *w_gu_sf, *w_d, *w_d_sf;
+  const float *w_gu_alpha, *w_d_alpha;  // NVFP4 only
+  const uint16_t* gamma;
+};
+
+beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& wts, int fmt, void* stream,
+                            beam_moe_t* out) {
+  const bool mx = fmt == BEAM_MOE_FMT_MXFP8;
+  if (!wts.router_w || !wts.w_gu || !wts.w_gu_sf || !wts.w_d || !wts.w_d_sf || !wts.gamma)
     return BEAM_MOE_ERR_INVALID_ARG;
-  if (!aligned(wts->w_gu, 16) || !aligned(wts->w_d, 16) || !aligned(wts->gamma, 16))
-    return BEAM_MOE_ERR_INVALID_ARG;
-  if (cfg->max_tokens <= 0 || !(cfg->alpha_a1 > 0.0f) || !(cfg->alpha_a2 > 0.0f) || !(cfg->rms_eps >= 0.0f))
-    return BEAM_MOE_ERR_INVALID_ARG;
+  if (!mx && (!wts.w_gu_alpha || !wts.w_d_alpha)) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned(wts.w_gu, 16) || !aligned(wts.w_d, 16) || !aligned(wts.gamma, 16)) return BEAM_MOE_ERR_INVALID_ARG;
+  if (cfg->max_tokens <= 0 || !(cfg->rms_eps >= 0.0f)) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!mx && (!(cfg->alpha_a1 > 0.0f) || !(cfg->alpha_a2 > 0.0f))) return BEAM_MOE_ERR_INVALID_ARG;
   beam_moe_status st = check_shape(cfg->hidden, cfg->num_experts, cfg->top_k);
   if (st != BEAM_MOE_OK) return st;
   if (cfg->inter <= 0) return BEAM_MOE_ERR_INVALID_ARG;
@@ -175,11 +196,15 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   beam_moe_ctx* h = new (std::nothrow) beam_moe_ctx();
   if (!h) return BEAM_MOE_ERR_OOM;
   h->cfg = *cfg;
+  if (mx) h->cfg.alpha_a1 = h->cfg.alpha_a2 = 1.0f;  // MX activations carry no tensor scale
+  h->fmt = fmt;
+  h->kv = mx ? 128 : 256;
+  h->sfa_tile = mx ? 512 : 4 * 512;
   h->H = cfg->hidden;
   h->E = cfg->num_experts;
   h->k = cfg->top_k;
   h->I = cfg->inter;
-  h->Ip = (cfg->inter + 255) / 256 * 256;
+  h->Ip = (cfg->inter + h->kv - 1) / h->kv * h->kv;
   h->Tmax = cfg->max_tokens;
   h->Rmax = static_cast<int64_t>(h->Tmax) * h->k;
   h->nblk_max = (h->Rmax + 127) / 128 + h->E;
@@ -216,20 +241,32 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   // ---- weights
   CREATE_TRY(dalloc(h, &h->router_w, sizeof(float) * E * H));
   CREATE_TRY(dalloc(h, &h->router_w3, sizeof(uint16_t) * 3 * E * H));
-  const size_t gu_tiles = static_cast<size_t>(E) * (2 * I / 256) * (H / 256);
-  const size_t d_tiles = static_cast<size_t>(E) * (H / 256) * (Ip / 256);
-  CREATE_TRY(dalloc(h, &h->w_gu_tiles, gu_tiles * kTileBytes));
-  CREATE_TRY(dalloc(h, &h->w_d_tiles, d_tiles * kTileBytes));
+  const size_t tile_bytes = mx ? kMxTileBytes : kTileBytes;
+  const size_t gu_tiles = static_cast<size_t>(E) * (2 * I / 256) * (H / h->kv);
+  const size_t d_tiles = static_cast<size_t>(E) * (H / 256) * (Ip / h->kv);
+  CREATE_TRY(dalloc(h, &h->w_gu_tiles, gu_tiles * tile_bytes));
+  CREATE_TRY(dalloc(h, &h->w_d_tiles, d_tiles * tile_bytes));
   CREATE_TRY(dalloc(h, &h->w_gu_alpha, sizeof(float) * E));
   CREATE_TRY(dalloc(h, &h->w_d_alpha, sizeof(float) * E));
   CREATE_TRY(dalloc(h, &h->gamma, sizeof(uint16_t) * H));
-  CREATE_TRY(cudaMemcpyAsync(h->router_w, wts->router_w, sizeof(float) * E * H, cudaMemcpyDeviceToDevice, s));
+  CREATE_TRY(cudaMemcpyAsync(h->router_w, wts.router_w, sizeof(float) * E * H, cudaMemcpyDeviceToDevice, s));
   CREATE_TRY(launch_split_router(h->router_w, E, H, h->router_w3, s));
-  CREATE_TRY(cudaMemcpyAsync(h->w_gu_alpha, wts->w_gu_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
-  CREATE_TRY(cudaMemcpyAsync(h->w_d_alpha, wts->w_d_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
-  CREATE_TRY(cudaMemcpyAsync(h->gamma, wts->gamma, sizeof(uint16_t) * H, cudaMemcpyDeviceToDevice, s));
-  CREATE_TRY(launch_repack_tiles(wts->w_gu, wts->w_gu_sf, E, 2 * I, H, H, I, h->w_gu_tiles, s));
-  CREATE_TRY(launch_repack_tiles(wts->w_d, wts->w_d_sf, E, H, I, Ip, 0, h->w_d_tiles, s));
+  if (mx) {  // the accumulators need no dequantisation: unit scales in the block list
+    const std::vector<float> ones(E, 1.0f);
+    CREATE_TRY(cudaMemcpy(h->w_gu_alpha, ones.data(), sizeof(float) * E, cudaMemcpyHostToDevice));
+    CREATE_TRY(cudaMemcpy(h->w_d_alpha, ones.data(), sizeof(float) * E, cudaMemcpyHostToDevice));
+  } else {
+    CREATE_TRY(cudaMemcpyAsync(h->w_gu_alpha, wts.w_gu_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
+    CREATE_TRY(cudaMemcpyAsync(h->w_d_alpha, wts.w_d_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
+  }
+  CREATE_TRY(cudaMemcpyAsync(h->gamma, wts.gamma, sizeof(uint16_t) * H, cudaMemcpyDeviceToDevice, s));
+  if (mx) {
+    CREATE_TRY(launch_repack_tiles_mx(wts.w_gu, wts.w_gu_sf, E, 2 * I, H, I, h->w_gu_tiles, s));
+    CREATE_TRY(launch_repack_tiles_mx(wts.w_d, wts.w_d_sf, E, H, I, 0, h->w_d_tiles, s));
+  } else {
+    CREATE_TRY(launch_repack_tiles(wts.w_gu, wts.w_gu_sf, E, 2 * I, H, H, I, h->w_gu_tiles, s));
+    CREATE_TRY(launch_repack_tiles(wts.w_d, wts.w_d_sf, E, H, I, Ip, 0, h->w_d_tiles, s));
+  }
 
   // ---- workspace
   int64_t lf = 0;
@@ -251,10 +288,10 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   CREATE_TRY(dalloc(h, &h->perm, sizeof(int32_t) * R));
   CREATE_TRY(dalloc(h, &h->inv, sizeof(int32_t) * R));
   CREATE_TRY(dalloc(h, &h->tile_row, sizeof(int32_t) * R));
-  CREATE_TRY(dalloc(h, &h->a1, static_cast<size_t>(h->nblk_max) * (H / 2) * 128));
-  CREATE_TRY(dalloc(h, &h->a1_sf, static_cast<size_t>(h->nblk_max) * (H / 64) * 512));
-  CREATE_TRY(dalloc(h, &h->a2, static_cast<size_t>(h->nblk_max) * (Ip / 2) * 128));
-  CREATE_TRY(dalloc(h, &h->a2_sf, static_cast<size_t>(h->nblk_max) * (Ip / 64) * 512));
+  CREATE_TRY(dalloc(h, &h->a1, act_bytes(h, H)));
+  CREATE_TRY(dalloc(h, &h->a1_sf, act_sf_bytes(h, H)));
+  CREATE_TRY(dalloc(h, &h->a2, act_bytes(h, Ip)));
+  CREATE_TRY(dalloc(h, &h->a2_sf, act_sf_bytes(h, Ip)));
   CREATE_TRY(dalloc(h, &h->y, sizeof(uint16_t) * static_cast<size_t>(R) * H));
   CREATE_TRY(dalloc(h, &h->err, sizeof(uint32_t)));
   CREATE_TRY(dalloc(h, &h->route_counter, sizeof(unsigned int)));
@@ -263,12 +300,12 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   CREATE_TRY(dalloc(h, &h->stage_x, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   CREATE_TRY(dalloc(h, &h->stage_res, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   CREATE_TRY(dalloc(h, &h->stage_out, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
-  // The SwiGLU outputs beyond I (when I is not a multiple of 256) are never written: their
-  // codes and scales must read as zero in the down GEMM.  Scale blocks of unused rows are
-  // also defined this way.
-  CREATE_TRY(cudaMemsetAsync(h->a2, 0, static_cast<size_t>(h->nblk_max) * (Ip / 2) * 128, s));
-  CREATE_TRY(cudaMemsetAsync(h->a2_sf, 0, static_cast<size_t>(h->nblk_max) * (Ip / 64) * 512, s));
-  CREATE_TRY(cudaMemsetAsync(h->a1_sf, 0, static_cast<size_t>(h->nblk_max) * (H / 64) * 512, s));
+  // The SwiGLU outputs beyond I (NVFP4 when I is not a multiple of 256) are never written:
+  // their codes and scales must read as zero in the down GEMM.  Scale blocks of unused rows
+  // are also defined this way.
+  CREATE_TRY(cudaMemsetAsync(h->a2, 0, act_bytes(h, Ip), s));
+  CREATE_TRY(cudaMemsetAsync(h->a2_sf, 0, act_sf_bytes(h, Ip), s));
+  CREATE_TRY(cudaMemsetAsync(h->a1_sf, 0, act_sf_bytes(h, H), s));
   CREATE_TRY(cudaMemsetAsync(h->err, 0, sizeof(uint32_t), s));
 
   CREATE_TRY(cudaStreamSynchronize(s));
@@ -277,6 +314,30 @@ beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weigh
   *out = h;
   return BEAM_MOE_OK;
 }
+
+}  // namespace
+
+extern "C" {
+
+beam_moe_status beam_moe_create(const beam_moe_config* cfg, const beam_moe_weights* wts, void* stream,
+                                beam_moe_t* out) {
+  if (!cfg || !wts || !out) return BEAM_MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const ExpertWeightsIn in{wts->router_w, wts->w_gu, wts->w_gu_sf, wts->w_d, wts->w_d_sf,
+                           wts->w_gu_alpha, wts->w_d_alpha, wts->gamma};
+  return create_impl(cfg, in, BEAM_MOE_FMT_NVFP4, stream, out);
+}
+
+beam_moe_status beam_moe_create_mxfp8(const beam_moe_config* cfg, const beam_moe_weights_mxfp8* wts, void* stream,
+                                      beam_moe_t* out) {
+  if (!cfg || !wts || !out) return BEAM_MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const ExpertWeightsIn in{wts->router_w, wts->w_gu, wts->w_gu_sf, wts->w_d, wts->w_d_sf, nullptr, nullptr,
+                           wts->gamma};
+  return create_impl(cfg, in, BEAM_MOE_FMT_MXFP8, stream, out);
+}
+
+int32_t beam_moe_expert_format(beam_moe_t h) { return h ? h->fmt : -1; }
 
 beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num_tokens, int32_t hidden,
                                int32_t num_experts, int32_t top_k, float* logits_ws, int32_t* ids, float* w,
@@ -322,7 +383,8 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
   const BlockScales bscales{h->w_gu_alpha, h->w_d_alpha, h->cfg.alpha_a1, h->cfg.alpha_a2};
   // CTA pairs for the expert GEMM when the average expert has a few hundred rows
-  const bool pair = !route_small_supported(T, H, E, k) &&
+  const bool mx = h->fmt == BEAM_MOE_FMT_MXFP8;
+  const bool pair = !mx && !route_small_supported(T, H, E, k) &&
                     (h->gemm_mode == BEAM_MOE_GEMM_PAIR || (h->gemm_mode == BEAM_MOE_GEMM_AUTO && T >= kPairMinTokens));
   if (route_small_supported(T, H, E, k)) {
     // router + top-k + histogram + scan + permutation in one launch
@@ -365,7 +427,10 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     BEAM_TRY(mark("scatter"));
     ++launches;
   }
-  BEAM_TRY(launch_quant_a1(xb, h->tile_row, T, H, k, h->cfg.alpha_a1, h->a1, h->a1_sf, s));
+  if (mx)
+    BEAM_TRY(launch_quant_a1_mx(xb, h->tile_row, T, H, k, h->a1, h->a1_sf, s));
+  else
+    BEAM_TRY(launch_quant_a1(xb, h->tile_row, T, H, k, h->cfg.alpha_a1, h->a1, h->a1_sf, s));
   BEAM_TRY(mark("quant_a1"));
   ++launches;
 
@@ -374,7 +439,7 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   g.num_mblocks = h->num_mblocks;
   g.max_rows_per_expert = T;  // a token chooses an expert at most once
   g.gu_n_tiles = h->I / 128;
-  g.gu_k_tiles = H / 256;
+  g.gu_k_tiles = H / h->kv;
   g.a1 = h->a1;
   g.a1_sf = h->a1_sf;
   g.w_gu = h->w_gu_tiles;
@@ -382,13 +447,15 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   g.a2_sf = h->a2_sf;
   g.alpha_a2 = h->cfg.alpha_a2;
   g.d_n_tiles = H / 256;
-  g.d_k_tiles = h->Ip / 256;
+  g.d_k_tiles = h->Ip / h->kv;
   g.w_d = h->w_d_tiles;
   g.y = h->y;
   g.y_cols = H;
   g.sched = h->sched;
   g.err = h->err;
-  if (pair)
+  if (mx)
+    BEAM_TRY(launch_gemm_experts_mx(g, h->num_sms, s));
+  else if (pair)
     BEAM_TRY(launch_gemm_experts_pair(g, h->num_sms, s));
   else
     BEAM_TRY(launch_gemm_experts(g, h->num_sms, s));
@@ -460,6 +527,16 @@ beam_moe_status beam_moe_quantize_nvfp4(const float* src, int64_t rows, int64_t 
   return BEAM_MOE_OK;
 }
 
+beam_moe_status beam_moe_quantize_mxfp8(const float* src, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* sf,
+                                        void* stream) {
+  if (rows < 0 || cols < 0 || cols % 32 != 0) return BEAM_MOE_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return BEAM_MOE_OK;
+  if (!src || !codes || !sf) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!aligned(src, 16) || !aligned(codes, 16)) return BEAM_MOE_ERR_INVALID_ARG;
+  BEAM_TRY(launch_quantize_rows_mx(src, rows, cols, codes, sf, static_cast<cudaStream_t>(stream)));
+  return BEAM_MOE_OK;
+}
+
 beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, void* dst, size_t bytes, size_t* size_out,
                                     void* stream) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;
@@ -474,10 +551,10 @@ beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, void* dst, size
     case BEAM_MOE_BUF_PERM: src = h->perm; n = sizeof(int32_t) * R; break;
     case BEAM_MOE_BUF_INV: src = h->inv; n = sizeof(int32_t) * R; break;
     case BEAM_MOE_BUF_SFBLOCK: src = h->sf_block; n = sizeof(int32_t) * (h->E + 1); break;
-    case BEAM_MOE_BUF_A1: src = h->a1; n = static_cast<size_t>(h->nblk_max) * (h->H / 2) * 128; break;
-    case BEAM_MOE_BUF_A1_SF: src = h->a1_sf; n = static_cast<size_t>(h->nblk_max) * (h->H / 64) * 512; break;
-    case BEAM_MOE_BUF_A2: src = h->a2; n = static_cast<size_t>(h->nblk_max) * (h->Ip / 2) * 128; break;
-    case BEAM_MOE_BUF_A2_SF: src = h->a2_sf; n = static_cast<size_t>(h->nblk_max) * (h->Ip / 64) * 512; break;
+    case BEAM_MOE_BUF_A1: src = h->a1; n = act_bytes(h, h->H); break;
+    case BEAM_MOE_BUF_A1_SF: src = h->a1_sf; n = act_sf_bytes(h, h->H); break;
+    case BEAM_MOE_BUF_A2: src = h->a2; n = act_bytes(h, h->Ip); break;
+    case BEAM_MOE_BUF_A2_SF: src = h->a2_sf; n = act_sf_bytes(h, h->Ip); break;
     case BEAM_MOE_BUF_Y: src = h->y; n = sizeof(uint16_t) * static_cast<size_t>(R) * h->H; break;
     default: return BEAM_MOE_ERR_INVALID_ARG;
   }
@@ -511,6 +588,7 @@ beam_moe_status beam_moe_debug_wait_timeout(beam_moe_t h, int64_t limit_ns, void
 
 beam_moe_status beam_moe_set_gemm_mode(beam_moe_t h, int32_t mode) {
   if (!h || mode < BEAM_MOE_GEMM_AUTO || mode > BEAM_MOE_GEMM_PAIR) return BEAM_MOE_ERR_INVALID_ARG;
+  if (mode == BEAM_MOE_GEMM_PAIR && h->fmt != BEAM_MOE_FMT_NVFP4) return BEAM_MOE_ERR_UNSUPPORTED;
   h->gemm_mode = mode;
   return BEAM_MOE_OK;
 }

@@ -295,6 +295,19 @@ __device__ __forceinline__ void tc_mma_nvfp4(uint32_t d_tmem, uint64_t adesc, ui
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// D(tmem) (+)= A(smem) * B(smem)^T, E4M3 operands (K = 32 per MMA) with one UE8M0 scale
+// per 32 values in TMEM; the scale byte within each 32-bit TMEM cell comes from the
+// instruction descriptor's scale-factor ids.
+__device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
 // D(tmem) (+)= A(smem) * B(smem)^T, BF16 operands, FP32 accumulation.
 __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -321,6 +334,16 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // Registers -> TMEM: lane i of the warp writes N consecutive 32-bit columns of TMEM lane
 // (taddr lane + i), starting at taddr's column (the warp's own lane quarter only).
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
                : "memory");
@@ -407,6 +430,46 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float al
   return sc;
 }
 
+// ---------------------------------------------------------------- MXFP8
+// Two FP32 -> two signed E4M3 codes in the low 16 bits (lo in the low byte),
+// round-to-nearest-even, saturating to +-448, sign of zero kept.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Scale exponent of an MX block: the smallest e with amax <= 448 * 2^e, clamped below at
+// -127.  With amax = m * 2^E, m in [1, 2): 448 = 1.75 * 2^8, so e = E - 8 when m <= 1.75
+// (mantissa bits <= 0x600000), else E - 7.  Zero and subnormal amax give -127.
+__device__ __forceinline__ int mx_scale_exp(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ef = static_cast<int>((b >> 23) & 0xFFu);
+  if (ef == 0) return -127;
+  const int e = ef - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return e < -127 ? -127 : e;
+}
+
+// MXFP8 of one block of 32 FP32 values: scale X = 2^e (mx_scale_exp of the block's amax),
+// codes E4M3(v_i / X).  v_i * 2^-e is exact (a power-of-two scaling that stays normal, or
+// falls below 2^-126 where it encodes to zero either way).  Writes the 32 code bytes as 8
+// little-endian words and returns the UE8M0 scale code e + 127.
+__device__ __forceinline__ uint32_t quant_block32_mx(const float (&v)[32], uint32_t (&c)[8]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int e = mx_scale_exp(amax);
+  // 2^-e as an FP32: e in [-127, 120], so -e + 127 is a normal biased exponent in [7, 254]
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t p0 = cvt_e4m3x2(__fmul_rn(v[4 * i], inv), __fmul_rn(v[4 * i + 1], inv));
+    const uint32_t p1 = cvt_e4m3x2(__fmul_rn(v[4 * i + 2], inv), __fmul_rn(v[4 * i + 3], inv));
+    c[i] = p0 | (p1 << 16);
+  }
+  return static_cast<uint32_t>(e + 127);
+}
+
 // Activation tiles: the codes of each 128-row block are stored as K/256 tiles of 128 rows x
 // 128 bytes (256 values), row m at m * 128 and its 16-byte chunk c at ((c ^ (m % 8)) * 16):
 // the 128-byte swizzle the tensor core reads, so a tile (or its first rows) is one
@@ -414,6 +477,28 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float al
 __device__ __forceinline__ size_t act_tile_offset(size_t block, int k_tiles, int kt, int m, int c) {
   return (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(kt)) * 16384u +
          static_cast<size_t>(m * 128 + ((c ^ (m & 7)) << 4));
+}
+
+// One 32-byte store (8 x 32 bits) to a 32-byte aligned global address.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
+// 32 code bytes = 16-byte chunks c and c + 1 (c even) of row m of activation tile
+// (block, kt).  Under the swizzle the two chunks fill one 32-byte aligned span
+// (c ^ (m % 8) and (c + 1) ^ (m % 8) differ only in bit 0), chunk c first when m is even
+// and second when m is odd; one 32-byte store writes both.
+__device__ __forceinline__ void st_act_pair(uint8_t* tiles, size_t block, int k_tiles, int kt, int m, int c,
+                                            const uint32_t (&w)[8]) {
+  uint8_t* p = tiles + (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(kt)) * 16384u +
+               static_cast<size_t>(m * 128 + ((c ^ (m & 6)) << 4));
+  const bool swap = (m & 1) != 0;
+  uint32_t s[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s[i] = swap ? w[(i + 4) & 7] : w[i];
+  st_global_v8(p, s);
 }
 
 // Byte offset of scale s of row m (0..127) in a 128-row scale block with K/64 groups.

@@ -59,15 +59,36 @@ static_assert(B_BYTES + SFB_BYTES == kTileBytes, "weight tile = B codes + B scal
 // expert has <= 32 rows): A holds 32 rows, which leaves room for a 5th stage of weights in
 // flight.  The MMA still reads 128 rows of A; rows past the region read the stage's B bytes
 // and only feed accumulator rows that are never stored.
-template <int kStages, int kABytes>
+//
+// Operand formats.  A K step is one 128-byte swizzle row per operand row in both: 256 E2M1
+// values (NVFP4: 4 MMAs of K = 64, 16 scales of 16 values per row) or 128 E4M3 values
+// (MXFP8: 4 MMAs of K = 32, 4 scales of 32 values per row).  Scale bytes per K step:
+struct FmtNvfp4 {
+  static constexpr bool kMx = false;
+  static constexpr int SFA = SFA_BYTES;    // 4 atoms: one per 64-value K-group
+  static constexpr int SFB = SFB_BYTES;    // 2 row halves x 4 atoms
+  static constexpr int TILE = kTileBytes;  // weight tile: B codes + B scales
+};
+struct FmtMxfp8 {
+  static constexpr bool kMx = true;
+  static constexpr int SFA = 512;          // 1 atom: the 4 scales of a row in one 32-bit word
+  static constexpr int SFB = 2 * 512;      // 2 row halves
+  static constexpr int TILE = kMxTileBytes;
+};
+static_assert(B_BYTES + FmtMxfp8::SFB == kMxTileBytes, "MXFP8 weight tile = B codes + B scales");
+template <int kStages, int kABytes, class F = FmtNvfp4>
 struct Ring {
+  using Fmt = F;
   static constexpr int STAGES = kStages;
   static constexpr int A_BYTES = kABytes;
-  static constexpr int STAGE_BYTES = kABytes + B_BYTES + SFB_BYTES + SFA_BYTES;
-  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for the swizzle");
+  // padded to 1024 bytes: every stage's operands keep the swizzle alignment
+  static constexpr int STAGE_BYTES = (kABytes + B_BYTES + F::SFB + F::SFA + 1023) / 1024 * 1024;
 };
 using RingFull = Ring<4, A_TILE_BYTES>;
 using RingSmallM = Ring<5, 32 * BK_BYTES>;
+using RingFullMx = Ring<4, A_TILE_BYTES, FmtMxfp8>;
+using RingSmallMMx = Ring<5, 32 * BK_BYTES, FmtMxfp8>;
+static_assert(RingFull::STAGE_BYTES == A_TILE_BYTES + kTileBytes + SFA_BYTES, "NVFP4 stages need no padding");
 constexpr int NUM_EPI_WARPS = 16;
 constexpr int NUM_SF_WARPS = 4;                      // one per TMEM lane quarter
 constexpr int FIRST_SF_WARP = 2 + NUM_EPI_WARPS;
@@ -84,6 +105,13 @@ constexpr uint32_t SFB_OFF = 16;
 // Instruction descriptor: E2M1 A and B (format 1), E4M3 scales (format 0), K-major
 // operands, N = 256 (n_dim = N/8 at bit 17), M = 128 (m_dim = M/16 at bit 24).
 constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((BM >> 4) << 24);
+// E4M3 A and B (format 0), UE8M0 scales (bit 23), K-major, N = 256, M = 128.  The scale
+// byte of MMA kb within each 32-bit TMEM scale cell is selected by the A and B
+// scale-factor ids (bits 29-30 and 4-5).
+constexpr uint32_t kIdescMxf8 = (1u << 23) | ((BN >> 3) << 17) | ((BM >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_mxf8(int kb) {
+  return kIdescMxf8 | (static_cast<uint32_t>(kb) << 29) | (static_cast<uint32_t>(kb) << 4);
+}
 
 constexpr int kMaxStages = 5;
 static_assert(SF_COL + kMaxStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor stages must fit in TMEM");
@@ -112,12 +140,6 @@ static size_t ring_smem_bytes() {
 // g -> -inf, exp(-g) = inf and g / inf = -0.
 __device__ __forceinline__ float silu_times(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
-// One 32-byte store (8 x 32 bits) to a 32-byte aligned global address.
-__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
-               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
-}
 
 __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -170,6 +192,7 @@ __device__ __forceinline__ TileRef tile_ref(int id, int total_gu, int n_gu, int 
 template <class R>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const ExpertGemmArgs args) {
   constexpr int STAGES = R::STAGES, A_BYTES = R::A_BYTES, STAGE_BYTES = R::STAGE_BYTES;
+  using F = typename R::Fmt;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmSmemTail* tail = reinterpret_cast<GemmSmemTail*>(smem + STAGES * STAGE_BYTES);
@@ -246,9 +269,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
         const int k_tiles = t.down ? args.d_k_tiles : args.gu_k_tiles;
         const int n_tiles = t.down ? n_d : n_gu;
         const uint8_t* a_src = (t.down ? args.a2 : args.a1) + static_cast<size_t>(mb.sf_block) * k_tiles * A_TILE_BYTES;
-        const uint8_t* sfa = (t.down ? args.a2_sf : args.a1_sf) + static_cast<size_t>(mb.sf_block) * k_tiles * SFA_BYTES;
+        const uint8_t* sfa = (t.down ? args.a2_sf : args.a1_sf) + static_cast<size_t>(mb.sf_block) * k_tiles * F::SFA;
         const uint8_t* btile = (t.down ? args.w_d : args.w_gu) +
-                               (static_cast<size_t>(mb.expert) * n_tiles + t.nt) * k_tiles * static_cast<size_t>(kTileBytes);
+                               (static_cast<size_t>(mb.expert) * n_tiles + t.nt) * k_tiles * static_cast<size_t>(F::TILE);
         if (t.down) {
           // this block's A2 is written by the gate/up epilogues (possibly of other CTAs)
           if (!wait_counter_bounded(ready + t.block, ready_target, abort_flag)) {
@@ -268,8 +291,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
         auto load_a = [&](int st, int kk) {
           uint8_t* sa = smem + st * STAGE_BYTES;
           bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, a_bytes, &tail->full[st]);
-          bulk_load(sa + A_BYTES + B_BYTES + SFB_BYTES, sfa + static_cast<size_t>(kk) * SFA_BYTES, SFA_BYTES,
-                    &tail->full[st]);
+          bulk_load(sa + A_BYTES + B_BYTES + F::SFB, sfa + static_cast<size_t>(kk) * F::SFA, F::SFA, &tail->full[st]);
         };
         // Before the wait only the weights are loaded; the first tile starts at stage 0, so
         // its deferred K steps kk < STAGES sit in stages kk.
@@ -289,10 +311,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&tail->full[stage], a_bytes + kTileBytes + SFA_BYTES);
+          mbar_arrive_expect_tx(&tail->full[stage], a_bytes + F::TILE + F::SFA);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          bulk_load(smem + stage * STAGE_BYTES + A_BYTES, btile + static_cast<size_t>(kt) * kTileBytes, kTileBytes,
+          bulk_load(smem + stage * STAGE_BYTES + A_BYTES, btile + static_cast<size_t>(kt) * F::TILE, F::TILE,
                     &tail->full[stage]);
           if (waited)
             load_a(stage, kt);
@@ -348,8 +370,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           const uint32_t sf = tmem + SF_COL + stage * SF_STAGE_COLS;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
-            tc_mma_nvfp4(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), kIdescNvfp4,
-                         sf + kb * 4, sf + SFB_OFF + kb * 8, (kt | kb) != 0 ? 1u : 0u);
+            if constexpr (F::kMx)  // the 4 MMAs share the stage's scale columns, byte kb of each cell
+              tc_mma_mxf8(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), idesc_mxf8(kb),
+                          sf, sf + SFB_OFF, (kt | kb) != 0 ? 1u : 0u);
+            else
+              tc_mma_nvfp4(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), kIdescNvfp4,
+                           sf + kb * 4, sf + SFB_OFF + kb * 8, (kt | kb) != 0 ? 1u : 0u);
           }
           tc_commit(&tail->empty[stage]);
           if (++stage == STAGES) {
@@ -396,8 +422,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           break;
         }
         const uint8_t* ssfb = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;  // [half][K-group][512]
-        const uint8_t* ssfa = ssfb + SFB_BYTES;                                // [K-group][512]
+        const uint8_t* ssfa = ssfb + F::SFB;                                   // [K-group][512]
         const uint32_t col = SF_COL + stage * SF_STAGE_COLS;
+        if constexpr (F::kMx) {
+          // one atom of A scales -> columns 0..3; B: rows 0-127 -> SFB_OFF + 0..3, rows 128-255 -> + 4..7
+          const uint4 a = *reinterpret_cast<const uint4*>(ssfa + lane * 16);
+          const uint32_t ra[4] = {a.x, a.y, a.z, a.w};
+          tmem_st_32x32b_x4(t_lane + col, ra);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + lane * 16);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 512 + lane * 16);
+          const uint32_t rb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+          tmem_st_32x32b_x8(t_lane + col + SFB_OFF, rb);
+        } else {
         uint32_t r[16];
         // A: K-group kb -> columns 4 kb .. 4 kb + 3
 #pragma unroll
@@ -418,6 +454,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
             r[q * 8 + 4] = v1.x; r[q * 8 + 5] = v1.y; r[q * 8 + 6] = v1.z; r[q * 8 + 7] = v1.w;
           }
           tmem_st_32x32b_x16(t_lane + col + SFB_OFF + part * 16, r);
+        }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -472,7 +509,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       acc_phase ^= 1;
       const bool valid = row_in_tile < mb.rows;
       if (!t.down) {
-        if (valid) {
+        if (valid && F::kMx) {
+          // 32 features = one MX block: 32 E4M3 codes (chunks c, c + 1 of K tile f0 / 128)
+          // and one scale byte (block f0 / 32 of the row: byte f0 / 32 % 4 of its K tile's word)
+          const float scale = mb.scale_gu;
+          const int f0 = t.nt * 128 + group * 32;
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            h[i] = silu_times(__uint_as_float(v[0][i]) * scale, __uint_as_float(v[1][i]) * scale);
+          uint32_t c[8];
+          const uint32_t sc = quant_block32_mx(h, c);
+          st_act_pair(args.a2, mb.sf_block, args.d_k_tiles, f0 >> 7, row_in_tile, (f0 & 127) >> 4, c);
+          args.a2_sf[sf_atom_offset(mb.sf_block, args.d_k_tiles, row_in_tile, f0 >> 5)] = static_cast<uint8_t>(sc);
+        } else if (valid) {
           const float scale = mb.scale_gu;
           const int f0 = t.nt * 128 + group * 32;  // first feature of this thread's 32
           uint32_t codes[4];
@@ -935,6 +985,11 @@ cudaError_t launch_gemm_experts(const ExpertGemmArgs& a, int grid, cudaStream_t 
   // With at most 32 tokens no expert has more than 32 rows.
   if (a.max_rows_per_expert <= 32) return launch_ring<RingSmallM>(a, grid, s);
   return launch_ring<RingFull>(a, grid, s);
+}
+
+cudaError_t launch_gemm_experts_mx(const ExpertGemmArgs& a, int grid, cudaStream_t s) {
+  if (a.max_rows_per_expert <= 32) return launch_ring<RingSmallMMx>(a, grid, s);
+  return launch_ring<RingFullMx>(a, grid, s);
 }
 
 cudaError_t launch_gemm_experts_pair(const ExpertGemmArgs& a, int grid, cudaStream_t s) {

@@ -89,6 +89,20 @@ cudaError_t launch_quantize_rows(const float* src, int64_t rows, int64_t cols, f
                                  uint8_t* codes, uint8_t* sf, cudaStream_t s);
 cudaError_t launch_amax(const float* src, int64_t n, float* amax_bits, cudaStream_t s);
 cudaError_t launch_amax_to_alpha(float* inout, cudaStream_t s);
+// ---- MXFP8 experts (quant.cu, routing.cu, gemm_nvfp4.cu)
+// Weight tiles: 256 rows x 128 K values (E4M3, one byte each) in the same swizzled order
+// as the NVFP4 code tiles, then 2 x 512 bytes of UE8M0 scales (4 per row: one per 32).
+constexpr int kMxTileSfBytes = 2 * 512;
+constexpr int kMxTileBytes = kTileCodeBytes + kMxTileSfBytes;  // 33792
+// K % 128 == 0 (no padding).
+cudaError_t launch_repack_tiles_mx(const uint8_t* codes, const uint8_t* sf, int E, int rows_per_e, int K,
+                                   int interleave_inter, uint8_t* dst, cudaStream_t s);
+cudaError_t launch_quantize_rows_mx(const float* src, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* sf,
+                                    cudaStream_t s);
+// A1 = MX(x) into the activation tiles: [blk][H/128][16384] codes, [blk][H/128][512] scales.
+cudaError_t launch_quant_a1_mx(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, uint8_t* a1,
+                               uint8_t* a1_sf, cudaStream_t s);
+
 // ---- grouped NVFP4 GEMMs, gate/up and down in one launch (gemm_nvfp4.cu)
 // Activation tiles are [blk][K/256][16384] (act_tile_offset), their scales [blk][K/64][512]
 // (sf_atom_offset); weight tiles are [E][n_tiles][K/256][kTileBytes].
@@ -119,6 +133,10 @@ struct ExpertGemmArgs {
 };
 inline int64_t sched_words(int64_t nblk_max) { return 1 + nblk_max; }
 cudaError_t launch_gemm_experts(const ExpertGemmArgs& a, int grid, cudaStream_t s);
+// The same GEMMs with MXFP8 operands: K tiles of 128 values (gu_k_tiles = H / 128,
+// d_k_tiles = I / 128), weight tiles of kMxTileBytes, scales [blk][K/128][512], and the
+// SwiGLU epilogue writes A2 = MX(h).  alpha_a2 is unused.
+cudaError_t launch_gemm_experts_mx(const ExpertGemmArgs& a, int grid, cudaStream_t s);
 // The CTA-pair version over 256-row blocks (grid rounded down to even).
 constexpr int kPairMinTokens = BEAM_MOE_PAIR_MIN_TOKENS;
 cudaError_t launch_gemm_experts_pair(const ExpertGemmArgs& a, int grid, cudaStream_t s);

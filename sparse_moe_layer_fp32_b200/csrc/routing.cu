@@ -12,7 +12,8 @@
 // A1 = Q(x, alpha_a1): x rows are quantised once per token (16-value blocks along H) and
 // the codes are written to the token's k permuted rows (the NVFP4 W4A4 experts of the
 // recipe "reflection/Beam-1.0-501B-A23B", section "Variants"), as activation tiles (see
-// act_tile_offset) of the row's 128-row block.
+// act_tile_offset) of the row's 128-row block.  For the block-scaled FP8 variant of the
+// experts (the recipe's FP8 checkpoint, read as MXFP8), A1 = MX(x) in 32-value blocks.
 #include "common.cuh"
 #include "internal.h"
 
@@ -236,6 +237,111 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
       if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, kgroups, m, b)) = word;
     }
   }
+}
+
+// ------------------------------------------------------------------ MXFP8
+// A1 = MX(x) for MXFP8 experts (E4M3 codes, one UE8M0 scale per 32 values): one thread per
+// 32-value block of x, quantised once and written to the token's k permuted rows.  A
+// block's 32 codes are chunks 2 (b % 4) and 2 (b % 4) + 1 of K tile b / 4 (one 32-byte
+// store); the four threads of one K tile combine their scale bytes into the row's 32-bit
+// scale word of that tile and one of them stores it.
+__device__ __forceinline__ void load_block32_bf16(const uint16_t* __restrict__ x, size_t t, int H, int b,
+                                                  float (&v)[32]) {
+  const uint4* xr = reinterpret_cast<const uint4*>(x + t * H) + 4 * b;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 p = __ldg(xr + q);
+    const uint32_t u[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * q + 2 * i] = bf16_bits_to_f32(u[i] & 0xFFFFu);
+      v[8 * q + 2 * i + 1] = bf16_bits_to_f32(u[i] >> 16);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(128) quant_a1_mx_kernel(const uint16_t* __restrict__ x,
+                                                          const int32_t* __restrict__ tile_row, int T, int H, int k,
+                                                          uint8_t* __restrict__ a1, uint8_t* __restrict__ a1_sf) {
+  const int nb = H / 32, k_tiles = H / 128;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const bool active = gid < static_cast<int64_t>(T) * nb;
+  const int t = active ? static_cast<int>(gid / nb) : 0;
+  const int b = active ? static_cast<int>(gid % nb) : 0;
+  pdl_wait();
+  pdl_trigger();
+  uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sc = 0;
+  int dst[16];
+  if (active) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) dst[j] = j < k ? __ldg(tile_row + static_cast<size_t>(t) * k + j) : 0;
+    float v[32];
+    load_block32_bf16(x, t, H, b, v);
+    sc = quant_block32_mx(v, c);
+  }
+  // lanes 4q..4q+3 hold blocks 4g..4g+3 of one token (nb is a multiple of 8)
+  const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc, 1);
+  const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
+  const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
+  const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  if (!active) return;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j >= k) break;
+    const int blk = dst[j] >> 7, m = dst[j] & 127;
+    st_act_pair(a1, blk, k_tiles, b >> 2, m, (b & 3) * 2, c);
+    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, k_tiles, m, b)) = word;
+  }
+}
+
+// Large batches: one warp per token, lane = 32-value block.
+__global__ void __launch_bounds__(256) quant_a1_mx_wide_kernel(const uint16_t* __restrict__ x,
+                                                               const int32_t* __restrict__ tile_row, int T, int H,
+                                                               int k, uint8_t* __restrict__ a1,
+                                                               uint8_t* __restrict__ a1_sf) {
+  __shared__ int s_blk[8][16], s_m[8][16];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * 8 + warp;
+  pdl_wait();
+  pdl_trigger();
+  if (t >= T) return;
+  if (lane < k) {
+    const int d = tile_row[static_cast<size_t>(t) * k + lane];
+    s_blk[warp][lane] = d >> 7;
+    s_m[warp][lane] = d & 127;
+  }
+  __syncwarp();
+  const int nb = H / 32, k_tiles = H / 128;
+  for (int b0 = 0; b0 < nb; b0 += 32) {
+    const int b = b0 + lane;
+    const bool active = b < nb;  // whole quads are active or not
+    uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sc = 0;
+    if (active) {
+      float v[32];
+      load_block32_bf16(x, t, H, b, v);
+      sc = quant_block32_mx(v, c);
+    }
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc, 1);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
+    const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    if (!active) continue;
+    for (int j = 0; j < k; ++j) {
+      const int blk = s_blk[warp][j], m = s_m[warp][j];
+      st_act_pair(a1, blk, k_tiles, b >> 2, m, (b & 3) * 2, c);
+      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, k_tiles, m, b)) = word;
+    }
+  }
+}
+
+cudaError_t launch_quant_a1_mx(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, uint8_t* a1,
+                               uint8_t* a1_sf, cudaStream_t s) {
+  if (T >= 256)
+    return launch_pdl(quant_a1_mx_wide_kernel, dim3((T + 7) / 8), dim3(256), 0, s, x, tile_row, T, H, k, a1, a1_sf);
+  const int64_t threads = static_cast<int64_t>(T) * (H / 32);
+  return launch_pdl(quant_a1_mx_kernel, dim3(static_cast<unsigned>((threads + 127) / 128)), dim3(128), 0, s, x,
+                    tile_row, T, H, k, a1, a1_sf);
 }
 
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s) {

@@ -26,13 +26,15 @@ def buf(layer, which, dtype):
     return to_np(layer.debug(which)).view(dtype)
 
 
-def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int) -> np.ndarray:
-    """Scale blocks (beam_moe.h layout) -> row-major scales [rows, kcols/16] in permuted row order."""
+def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int, block: int = 16) -> np.ndarray:
+    """Scale blocks (beam_moe.h layout) -> row-major scales [rows, kcols/block] in permuted row
+    order; block = 16 (NVFP4) or 32 (MXFP8): 4 scales per 32-bit word either way."""
     experts = len(offsets) - 1
     rows = int(offsets[-1])
-    kgroups = kcols // 64
-    out = np.zeros((rows, kcols // 16), np.uint8)
-    s = np.arange(kcols // 16)
+    n_sc = kcols // block
+    kgroups = n_sc // 4
+    out = np.zeros((rows, n_sc), np.uint8)
+    s = np.arange(n_sc)
     for e in range(experts):
         n = int(offsets[e + 1] - offsets[e])
         if n == 0:
@@ -46,13 +48,16 @@ def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols
     return out
 
 
-def tile_rows(tiles: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int) -> np.ndarray:
-    """Activation tiles (beam_moe.h layout) -> packed codes [rows, kcols/2] in permuted row order."""
+def tile_rows(tiles: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int,
+              values_per_byte: int = 2) -> np.ndarray:
+    """Activation tiles (beam_moe.h layout) -> codes [rows, kcols / values_per_byte] in permuted
+    row order (2: packed NVFP4; 1: MXFP8).  A tile holds 128 code bytes of each row."""
     experts = len(offsets) - 1
     rows = int(offsets[-1])
-    k_tiles = kcols // 256
-    out = np.zeros((rows, kcols // 2), np.uint8)
-    j = np.arange(kcols // 2)
+    row_bytes = kcols // values_per_byte
+    k_tiles = row_bytes // 128
+    out = np.zeros((rows, row_bytes), np.uint8)
+    j = np.arange(row_bytes)
     for e in range(experts):
         n = int(offsets[e + 1] - offsets[e])
         if n == 0:
@@ -104,7 +109,7 @@ def ids_match(gpu_ids: np.ndarray, ref_ids: np.ndarray, logits: np.ndarray, near
     return bad
 
 
-def oracle_layer_inputs(shape: mi.LayerShape, seed: int, weights_fp32=None, tokens=None):
+def oracle_layer_inputs(shape: mi.LayerShape, seed: int, weights_fp32=None, tokens=None, fmt: str = "nvfp4"):
     """Oracle-side inputs of a workload: x, residual (FP64 of BF16), W_r, gamma, expert cache."""
     xb, rb = mi.tokens(shape, seed) if tokens is None else tokens
     x = mi.bf16_bits_to_f32(xb).astype(np.float64)
@@ -112,4 +117,4 @@ def oracle_layer_inputs(shape: mi.LayerShape, seed: int, weights_fp32=None, toke
     wr = mi.router_weight(shape, seed)
     g = mi.bf16_bits_to_f32(mi.gamma(shape, seed)).astype(np.float64)
     getter = weights_fp32 or (lambda e: mi.expert_weights(shape, seed, e))
-    return x, res, wr, g, moe.ExpertCache(getter, keep=16)
+    return x, res, wr, g, moe.ExpertCache(getter, keep=16, fmt=fmt)

@@ -228,3 +228,77 @@ def test_pair_gemm_matches_oracle_and_single_cta(bm, name, tokens, seed):
     with pytest.raises(bm.BeamMoeError):
         layer.set_gemm_mode(7)
     layer.close()
+
+
+# ---------------------------------------------------------------- MXFP8 experts
+# The block-scaled FP8 variant (the recipe's FP8 checkpoint, section "Variants", read as
+# MXFP8: E4M3 values and one power-of-two scale per 32 values for weights, A1 and A2),
+# created with beam_moe_create_mxfp8.  Stages as above: routing and permutation are the
+# format-independent kernels; A1 is bit-exact (codes and scales, sign of zero included);
+# A2 codes may differ where the GPU's FP32 SwiGLU and the oracle's FP64 one straddle a
+# rounding boundary; y, finalize and the end-to-end output at the layer's tolerances.
+@pytest.mark.parametrize("name,tokens,seed", [("tiny", 4, 20), ("tiny", 37, 21), ("tiny", 1500, 22), ("mid", 7, 23),
+                                              ("mid", 200, 24), ("mid", 4500, 25)])
+def test_forward_mxfp8_stages_and_end_to_end(bm, name, tokens, seed):
+    from oracle import mxfp8
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(SHAPES[name], tokens=tokens)
+    x, res, wr, g, cache = oracle_layer_inputs(shape, seed, fmt="mxfp8")
+    weights = synthetic.make_weights(shape, seed, threads=4, fmt="mxfp8")
+    layer = bm.MoELayer(max_tokens=tokens, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                        inter=shape.inter, fmt="mxfp8", **weights)
+    assert bm.beam_moe_expert_format(layer.handle) == bm.FMT_MXFP8
+    xd, rd = synthetic.make_batch(shape, seed)
+    out = layer.forward(xd, rd)
+    layer.check()
+    ref = moe.moe_forward(x, res, wr, g, cache, shape.experts, shape.top_k, None, None, shape.rms_eps)
+    T, E, k, H, I = tokens, shape.experts, shape.top_k, shape.hidden, shape.inter
+    ids = buf(layer, bm.BUF_IDS, np.int32).reshape(T, k)
+    w = buf(layer, bm.BUF_WEIGHTS, np.float32).reshape(T, k)
+    near = ref["near_tie"]
+    assert not ids_match(ids, ref["ids"], ref["logits"], near)
+    pm = moe.permute(ids.astype(np.int64), E)
+    offsets = buf(layer, bm.BUF_OFFSETS, np.int32)
+    perm = buf(layer, bm.BUF_PERM, np.int32)
+    inv = buf(layer, bm.BUF_INV, np.int32).reshape(T, k)
+    sfb = buf(layer, bm.BUF_SFBLOCK, np.int32)
+    np.testing.assert_array_equal(offsets, pm["offsets"])
+    np.testing.assert_array_equal(perm, pm["perm_src"])
+    np.testing.assert_array_equal(inv, pm["inv"])
+    # ---- A1 = MX(x rows): bit-exact
+    a1c = tile_rows(buf(layer, bm.BUF_A1, np.uint8), sfb, offsets, H, values_per_byte=1)
+    a1s = sf_rows(buf(layer, bm.BUF_A1_SF, np.uint8), sfb, offsets, H, block=32)
+    rc, rs = mxfp8.quantize_mxfp8(x[perm].astype(np.float32))
+    np.testing.assert_array_equal(a1s, rs)
+    np.testing.assert_array_equal(a1c, rc)
+    # ---- A2 and y from the GPU's own A1
+    a2c = tile_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, I, values_per_byte=1)
+    a2s = sf_rows(buf(layer, bm.BUF_A2_SF, np.uint8), sfb, offsets, I, block=32)
+    y = to_np(layer.debug(bm.BUF_Y).view(torch.bfloat16).float()).reshape(T * k, H).astype(np.float64)
+    mism, n_codes = 0, 0
+    y_ref = np.zeros_like(y)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if lo == hi:
+            continue
+        deq = cache.dequantized(e)
+        r = moe.expert_forward(a1c[lo:hi], a1s[lo:hi], None, deq, None, "mxfp8")
+        mism += int((a2c[lo:hi] != r["a2_packed"]).sum()) + int((a2s[lo:hi] != r["a2_sf"]).sum())
+        n_codes += a2c[lo:hi].size
+        d_gpu = mxfp8.dequantize_mxfp8(a2c[lo:hi], a2s[lo:hi])
+        d_ref = mxfp8.dequantize_mxfp8(r["a2_packed"], r["a2_sf"])
+        assert np.linalg.norm(d_gpu - d_ref) <= 1e-2 * max(np.linalg.norm(d_ref), 1e-30)
+        y_ref[lo:hi] = d_gpu @ deq[1].T
+    assert mism <= max(2, 5e-3 * n_codes), f"A2 mismatches {mism} of {n_codes}"
+    rel_y = np.linalg.norm(y - y_ref) / max(np.linalg.norm(y_ref), 1e-30)
+    assert rel_y < 5e-3, rel_y
+    out_np = bf16_to_f64(out)
+    pre, _, _ = moe.finalize(y[inv], w.astype(np.float64), res, g, shape.rms_eps)
+    assert np.all(np.abs(out_np - pre) <= 2.0 ** -8 * np.maximum(np.abs(pre), 1.0))
+    rel, mx = compare_outputs(out_np, ref["out_pre"], skip=near)
+    assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
+    # the CTA-pair GEMM is NVFP4 only
+    with pytest.raises(bm.BeamMoeError) as ei:
+        layer.set_gemm_mode(bm.GEMM_PAIR)
+    assert ei.value.status == bm.ERR_UNSUPPORTED
+    layer.close()

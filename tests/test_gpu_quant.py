@@ -78,3 +78,46 @@ def test_e2m1_e4m3_conversion_sweep(bm):
         rc, rs = nvfp4.quantize_nvfp4(v, alpha)
         np.testing.assert_array_equal(sf, rs)
         np.testing.assert_array_equal(_norm(codes), _norm(rc))
+
+
+# ---------------------------------------------------------------- MXFP8 (beam_moe_quantize_mxfp8)
+# The block-scaled FP8 variant of the experts (the recipe's FP8 checkpoint, read as MXFP8:
+# E4M3 codes, one UE8M0 scale per 32 values).  Codes are compared bit for bit, the sign of
+# zero included: both sides keep the input's sign.
+def _gpu_mx(bm, v):
+    codes, sf = bm.beam_moe_quantize_mxfp8(torch.from_numpy(v).cuda())
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), sf.cpu().numpy()
+
+
+@pytest.mark.parametrize("rows,cols,scale", [(1, 32, 1.0), (7, 96, 0.02), (64, 5120, 0.02), (300, 1536, 3e5)])
+def test_quantize_mxfp8_matches_oracle(bm, rows, cols, scale):
+    from oracle import mxfp8
+    rng = np.random.default_rng(rows * 11 + cols)
+    v = (rng.standard_normal((rows, cols)) * scale).astype(np.float32)
+    codes, sf = _gpu_mx(bm, v)
+    rc, rs = mxfp8.quantize_mxfp8(v)
+    np.testing.assert_array_equal(sf, rs)
+    np.testing.assert_array_equal(codes, rc)
+
+
+def test_quantize_mxfp8_edge_blocks(bm):
+    from oracle import mxfp8
+    e4 = mxfp8.e4m3_decode_signed(np.arange(0x7F, dtype=np.uint8))
+    mids = (e4[:-1] + e4[1:]) / 2
+    blocks = [np.zeros(32),                                   # amax 0 -> scale code 0
+              np.full(32, 1e-42),                             # subnormal amax
+              np.linspace(-3e38, 3e38, 32),                   # largest exponents
+              np.array([448.0] + [-0.0] * 31) * 2.0 ** -20,   # exactly on a scale boundary, -0
+              np.array([np.nextafter(np.float32(448.0), np.float32(1e9))] + [1.0] * 31),  # one ulp above
+              np.concatenate([mids[-32:-1], [448.0]]),        # E4M3 midpoints with scale 2^0: ties to even
+              np.concatenate([-mids[40:71], [-448.0]]) * 2.0 ** 7,
+              np.array([1.0, -1e-30] * 16)]                   # negatives that round to zero
+    v = np.stack(blocks).astype(np.float32)
+    codes, sf = _gpu_mx(bm, v)
+    rc, rs = mxfp8.quantize_mxfp8(v)
+    np.testing.assert_array_equal(sf, rs)
+    np.testing.assert_array_equal(codes, rc)
+    assert sf[0, 0] == 0 and sf[3, 0] == 127 - 20 and sf[5, 0] == 127
+    with pytest.raises(bm.BeamMoeError):
+        bm.beam_moe_quantize_mxfp8(torch.zeros((2, 48), device="cuda"))
