@@ -7,6 +7,9 @@
 // K-major):
 //   gate/up: D[r][n] = A1[r] . Wgu[e][n],  K = H; epilogue h = silu(g) * u, A2 = Q(h)
 //   down:    D[r][n] = A2[r] . Wd[e][n],   K = I; epilogue y = bf16(D * scale)
+// The single-CTA kernel is also built for the recipe's second precision variant, FP8
+// experts (same section), read as MXFP8: E4M3 operands with one UE8M0 scale per 32 values,
+// tcgen05.mma.kind::mxf8f6f4, and A2 = MX(h) in the epilogue (template parameter FmtMxfp8).
 //
 // Work items are (128-row block of one expert) x (256-column tile).  The tile list holds
 // every gate/up tile, then every down tile; CTAs claim tiles in that order from a global

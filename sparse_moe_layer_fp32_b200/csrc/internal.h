@@ -89,7 +89,7 @@ cudaError_t launch_quantize_rows(const float* src, int64_t rows, int64_t cols, f
                                  uint8_t* codes, uint8_t* sf, cudaStream_t s);
 cudaError_t launch_amax(const float* src, int64_t n, float* amax_bits, cudaStream_t s);
 cudaError_t launch_amax_to_alpha(float* inout, cudaStream_t s);
-// ---- MXFP8 experts (quant.cu, routing.cu, gemm_nvfp4.cu)
+// ---- MXFP8 experts (quant.cu, routing.cu, gemm_experts.cu)
 // Weight tiles: 256 rows x 128 K values (E4M3, one byte each) in the same swizzled order
 // as the NVFP4 code tiles, then 2 x 512 bytes of UE8M0 scales (4 per row: one per 32).
 constexpr int kMxTileSfBytes = 2 * 512;
@@ -103,7 +103,7 @@ cudaError_t launch_quantize_rows_mx(const float* src, int64_t rows, int64_t cols
 cudaError_t launch_quant_a1_mx(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, uint8_t* a1,
                                uint8_t* a1_sf, cudaStream_t s);
 
-// ---- grouped NVFP4 GEMMs, gate/up and down in one launch (gemm_nvfp4.cu)
+// ---- grouped NVFP4 GEMMs, gate/up and down in one launch (gemm_experts.cu)
 // Activation tiles are [blk][K/256][16384] (act_tile_offset), their scales [blk][K/64][512]
 // (sf_atom_offset); weight tiles are [E][n_tiles][K/256][kTileBytes].
 struct ExpertGemmArgs {
