@@ -61,4 +61,6 @@ from .moe import (  # noqa: F401
     next_prenorm,
     moe_forward,
     moe_forward_tokens,
+    shard_dequantized,
+    moe_forward_tp,
 )

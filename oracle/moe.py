@@ -271,3 +271,51 @@ def moe_forward(x, residual, router_w, gamma, experts: ExpertCache, num_experts,
     r = moe_forward_tokens(x, residual, router_w, gamma, experts, top_k, alpha_a1, alpha_a2, eps)
     r.update(permute(r["ids"], num_experts))
     return r
+
+
+# ----------------------------------------------------------------------------- tensor parallel
+def shard_dequantized(deq_w, rank: int, world: int):
+    """Rank `rank`'s slice of one expert under tensor parallelism over the intermediate size:
+    the gate and up rows of features [r s, (r+1) s) and the same columns of down, s = I / world
+    ([PR] "Status": Beam's TP all-reduce; [RECIPE] "Launching the server": NVFP4 with TP4).
+    deq_w: (gate/up [2I, H], down [H, I]) FP64.  Returns the shard's (gate/up [2s, H], down [H, s])."""
+    w_gu, w_d = deq_w
+    inter = w_gu.shape[0] // 2
+    if inter % world:
+        raise ValueError("the intermediate size must split evenly over the ranks")
+    s = inter // world
+    lo, hi = rank * s, (rank + 1) * s
+    return np.concatenate([w_gu[lo:hi], w_gu[inter + lo:inter + hi]]), w_d[:, lo:hi]
+
+
+def moe_forward_tp(x, residual, router_w, gamma, experts: ExpertCache, top_k, alpha_a1, alpha_a2, world: int,
+                   eps=1e-6):
+    """The layer with its experts split over `world` tensor-parallel ranks ([PR] "Status": the
+    TP all-reduce fused with the sandwich norms and the MoE finalize).  Every rank routes
+    the same tokens and quantises the same A1; rank r runs its shard of every expert and
+    forms its partial m_r = sum_j w_j y_r; the all-reduce gives m = sum_r m_r (ranks in
+    order), then the post-RMSNorm and the residual add as in finalize.  The activation
+    quantisation blocks (16 or 32 values along I) never straddle a shard boundary when
+    I / world is a multiple of them, so each rank's A2 is the matching slice of the
+    unsharded A2.  Returns dict(ids, w, m_parts [world, T, H], m, out_pre, out)."""
+    x = np.asarray(x, np.float64)
+    t_count, hidden = x.shape
+    logits = router_logits(x, router_w)
+    ids, w, _ = route_topk(logits, top_k)
+    fmt = experts.fmt
+    a1_packed, a1_sf = quantize_act(x.astype(np.float32), alpha_a1, fmt)
+    m_parts = np.zeros((world, t_count, hidden), np.float64)
+    for r in range(world):
+        y = np.zeros((t_count, top_k, hidden), np.float64)
+        for e in np.unique(ids):
+            tt, jj = np.nonzero(ids == e)
+            shard = shard_dequantized(experts.dequantized(int(e)), r, world)
+            y[tt, jj] = expert_forward(a1_packed[tt], a1_sf[tt], alpha_a1, shard, alpha_a2, fmt)["y"]
+        m_parts[r] = np.einsum("tk,tkh->th", w, y)
+    m = np.zeros((t_count, hidden), np.float64)
+    for r in range(world):
+        m = m + m_parts[r]
+    rms = np.sqrt(np.mean(m * m, axis=1, keepdims=True) + eps)
+    out_pre = np.asarray(residual, np.float64) + m / rms * np.asarray(gamma, np.float64)[None, :]
+    return dict(ids=ids, w=w, near_tie=near_tie_mask(logits, top_k), m_parts=m_parts, m=m, out_pre=out_pre,
+                out=bf16_round(out_pre))

@@ -250,3 +250,36 @@ def test_generator_bf16_matches_torch():
     v = np.random.default_rng(4).standard_normal(50_000).astype(np.float32)
     ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     np.testing.assert_array_equal(mi.f32_to_bf16_bits(v), ref)
+
+
+def test_tensor_parallel_partials_sum_to_the_unsharded_layer():
+    # Splitting every expert's intermediate features over W ranks partitions the sums of
+    # the gate/up and down GEMMs; A2's quantisation blocks never straddle a shard.  So the
+    # ranks' partial m add up to the unsharded m (FP64 rounding only), for both formats,
+    # and W = 1 is the unsharded layer itself.
+    shape, x, res, wr, g, cache = _tiny()
+    a1s, a2s = np.float32(5.0 / 2688), np.float32(3.0 / 2688)
+    full = moe.moe_forward(x, res, wr, g, cache, shape.experts, shape.top_k, a1s, a2s)
+    for world in (1, 2, 4):
+        tp = moe.moe_forward_tp(x, res, wr, g, cache, shape.top_k, a1s, a2s, world)
+        np.testing.assert_array_equal(tp["ids"], full["ids"])
+        np.testing.assert_allclose(tp["m"], full["m"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(tp["out_pre"], full["out_pre"], rtol=0, atol=1e-12)
+        assert tp["m_parts"].shape == (world,) + full["m"].shape
+        if world > 1:  # every rank contributes
+            assert all(np.abs(tp["m_parts"][r]).max() > 0 for r in range(world))
+    one = moe.moe_forward_tp(x, res, wr, g, cache, shape.top_k, a1s, a2s, 1)
+    np.testing.assert_array_equal(one["m"], full["m"])
+    cache8 = moe.ExpertCache(lambda e: mi.expert_weights(shape, 0, e), fmt="mxfp8")
+    full8 = moe.moe_forward(x, res, wr, g, cache8, shape.experts, shape.top_k, None, None)
+    tp8 = moe.moe_forward_tp(x, res, wr, g, cache8, shape.top_k, None, None, 4)
+    np.testing.assert_allclose(tp8["m"], full8["m"], rtol=0, atol=1e-12)
+    # the shard slices: gate rows, matching up rows, matching down columns
+    w_gu, w_d = cache.dequantized(0)
+    gu1, d1 = moe.shard_dequantized((w_gu, w_d), 1, 4)
+    inter = w_gu.shape[0] // 2
+    np.testing.assert_array_equal(gu1[: inter // 4], w_gu[inter // 4: inter // 2])
+    np.testing.assert_array_equal(gu1[inter // 4:], w_gu[inter + inter // 4: inter + inter // 2])
+    np.testing.assert_array_equal(d1, w_d[:, inter // 4: inter // 2])
+    with pytest.raises(ValueError):
+        moe.shard_dequantized((w_gu, w_d), 0, 3)
