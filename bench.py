@@ -393,6 +393,104 @@ def run_ours(args, shape, rank, world, local_rank):
     return line
 
 
+# ------------------------------------------------------------------ tensor parallel, one GPU
+def run_tp_shared(args, shape):
+    """Tensor-parallel layer (experts split over W ranks along I, finalize fused with its
+    all-reduce) with all W ranks on one GPU, run in turn: every rank's phase 0 (routing,
+    its slice of the expert GEMMs, its partial m and their publication), then every rank's
+    phase 1 (the exchange, sum, norm, residual).  Each phase is timed with CUDA events on
+    the launching stream; a rank's step = its phase 0 + phase 1.  `value` estimates the
+    group's tokens/s if each rank had its own GPU: T / the slowest rank's step.  The
+    partials that rank r reads from its peers sit in this GPU's memory here, so the NVLink
+    transfer of the exchange (W x T x H x 4 B per rank) is not in the estimate."""
+    import dataclasses
+    import torch
+    import sparse_moe_layer_fp32_b200 as bm
+    from sparse_moe_layer_fp32_b200 import synthetic, tp
+
+    W, fmt = args.tp_shared_gpu, args.experts_format
+    torch.cuda.set_device(0)
+    full = synthetic.make_weights(shape, 0, fmt=fmt)
+    a1, a2 = mi.activation_scales(shape) if fmt == "nvfp4" else (1.0, 1.0)
+    layers = []
+    for r in range(W):
+        sh = tp.shard_weights(full, r, W, shape.inter)
+        layers.append(bm.MoELayer(max_tokens=shape.tokens, hidden=shape.hidden, num_experts=shape.experts,
+                                  top_k=shape.top_k, inter=shape.inter // W, alpha_a1=float(a1), alpha_a2=float(a2),
+                                  rms_eps=shape.rms_eps, fmt=fmt, **sh))
+        del sh
+    del full
+    torch.cuda.empty_cache()
+    grp = tp.SharedGpuGroup(layers)
+    x, res = synthetic.make_batch(shape, 0)
+    outs = [torch.empty_like(res) for _ in range(W)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    clean = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        flush.zero_()
+        clean.sum()
+
+    for _ in range(max(args.warmup, 3)):
+        grp.forward(x, res, outs)
+        flush_l2()
+    for lay in layers:
+        lay.check()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ph = [[[], []] for _ in range(W)]
+    kern = {}
+    with ClockSampler(0) as clk:
+        for step in range(args.steps + 1):
+            prof = step == args.steps  # one extra pass with the library's per-kernel events
+            for lay in layers:
+                lay.profile(prof)
+            for phase in (0, 1):
+                for r, lay in enumerate(layers):
+                    flush_l2()  # each rank starts cold, as on its own GPU
+                    a, b = ev(), ev()
+                    a.record(stream)
+                    lay.forward_tp_phase(x, res, outs[r], phase)
+                    b.record(stream)
+                    if prof:
+                        for name, kms in lay.kernel_times():
+                            kern.setdefault(name, []).append(kms)
+                    else:
+                        ph[r][phase].append((a, b))
+        torch.cuda.synchronize()
+    for lay in layers:
+        lay.check()
+    assert all(torch.equal(o, outs[0]) for o in outs[1:]), "ranks disagree"
+    p0 = [sum(a.elapsed_time(b) for a, b in ph[r][0]) / args.steps for r in range(W)]
+    p1 = [sum(a.elapsed_time(b) for a, b in ph[r][1]) / args.steps for r in range(W)]
+    rank_ms = [p0[r] + p1[r] for r in range(W)]
+    kms = {n: sum(v) / len(v) for n, v in kern.items()}
+    T, H = shape.tokens, shape.hidden
+    pk = peaks()
+    red_bytes = W * T * H * 4 + 2 * T * H * 2 + H * 2
+    part_bytes = T * shape.top_k * H * 2 + W * T * H * 4 / W  # its y rows, its own partial m
+    roof = {"bound": "hbm", "kernel": "tp_reduce", "kernel_ms": kms.get("tp_reduce"),
+            "achieved": red_bytes / (kms["tp_reduce"] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s",
+            "traffic": None, "peak_source": f"{pk['src']} copy bandwidth"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    line = {
+        "metric": METRIC, "value": T / (max(rank_ms) / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": max(rank_ms), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": ("nvfp4" if fmt == "nvfp4" else "mxfp8") + " experts, fp32 router, accumulation and all-reduce",
+        "data": "synthetic (seeded; random-init weights of the layer's shapes)",
+        "config": dict(workload_config(shape, "write+read", fmt), parallelism=f"tp{W}, ranks sharing one GPU in turn"),
+        "estimate": "value = T / slowest rank's (phase 0 + phase 1); peers' partials read from this GPU's memory, "
+                    "so the NVLink transfer of the exchange is not included",
+        "tp": {"world": W, "rank_ms": rank_ms, "phase0_ms": p0, "phase1_ms": p1,
+               "exchange_bytes_per_rank": W * T * H * 4, "tp_partial_bytes": part_bytes},
+        "kernels_ms": kms, "roofline": roof, "gpu_launches": sum(lay.launches() for lay in layers),
+        "clocks": clk.summary(),
+    }
+    grp.close()
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -401,6 +499,8 @@ def main():
     ap.add_argument("--workload", default="decode8", choices=sorted(mi.SHAPES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tp-shared-gpu", type=int, default=0, metavar="W",
+                    help="tensor-parallel layer with W ranks sharing this one GPU, run in turn (per-rank timing)")
     ap.add_argument("--experts-format", default="nvfp4", choices=["nvfp4", "mxfp8"],
                     help="routed experts in NVFP4 (default) or the block-scaled FP8 variant (MXFP8)")
     ap.add_argument("--l2-flush", default="write+read", choices=["write", "write+read"],
@@ -413,6 +513,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, shape, rank, world)
+        return
+    if args.tp_shared_gpu:
+        emit(run_tp_shared(args, shape), 0)
         return
     if world > 1:
         import datetime

@@ -143,12 +143,63 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_prenorm(beam_moe_t h, const void* 
                                                       void* next_x, const void* next_gamma, float next_eps,
                                                       int32_t num_tokens, void* stream);
 
-/* Same as beam_moe_forward with HOST buffers: copies x and residual to the handle's
- * device staging buffers, runs the forward, copies out back, all enqueued on `stream`
- * (cudaMemcpyAsync; pinned host memory makes the copies asynchronous).  The caller
+/* Same as beam_moe_forward with HOST buffers: copies x to the handle's device staging
+ * buffer on `stream`, runs the forward, copies out back on `stream`; the residual's copy
+ * starts once x has landed and runs on a second stream of the handle, overlapping the
+ * routing and the expert GEMMs; only the finalize waits for it (the first call creates that
+ * stream and two events).
+ * All copies are cudaMemcpyAsync; pinned host memory makes them asynchronous.  The caller
  * synchronises `stream` before reading out_host. */
 BEAM_MOE_API beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const void* residual_host, void* out_host,
                                       int32_t num_tokens, void* stream);
+
+/* ---- Tensor parallelism over the experts' intermediate size, with the finalize fused to
+ * its all-reduce (vLLM PR "Day-0 support for Reflection's Beam-1.0", section "Status":
+ * Beam's TP all-reduce fused with the sandwich norms and the MoE finalize; recipe
+ * "reflection/Beam-1.0-501B-A23B": NVFP4 with TP4 on Blackwell).
+ *
+ * Each of W ranks (one process per GPU) creates an ordinary handle (beam_moe_create or
+ * beam_moe_create_mxfp8) from its slice of the experts: cfg->inter = I / W, the gate rows
+ * and the up rows of features [r I/W, (r+1) I/W) and the same columns of the down weights
+ * (the tensor scales of the whole tensors unchanged; I / W must meet create's limits).
+ * Router weights and gamma are the full ones on every rank.  Then, once per group:
+ *   1. beam_moe_tp_region: the handle allocates its exchange region (device memory it owns:
+ *      a flag header plus two [max_tokens][H] FP32 buffers) and returns its address;
+ *   2. the ranks exchange the regions (beam_moe_ipc_export / beam_moe_ipc_import across
+ *      processes, or plain pointers when the ranks share a process and a GPU);
+ *   3. beam_moe_tp_attach with every rank's region, in rank order.
+ * beam_moe_forward_tp then computes out on every rank (identical bits on all ranks): the
+ * routing, A1 and the expert GEMMs of the rank's slice, its partial m, the exchange, and
+ * the post-RMSNorm + residual of the summed m.  Every rank must call it the same number of
+ * times, with the same num_tokens, like a collective.  A rank that waits more than 2 s for
+ * its peers gives up: beam_moe_check then returns BEAM_MOE_ERR_TIMEOUT. */
+#define BEAM_MOE_IPC_HANDLE_BYTES 64
+BEAM_MOE_API int64_t beam_moe_tp_region_bytes(beam_moe_t h);
+/* Allocates the region on the first call (synchronises the device); *region gets its
+ * device address (256-byte aligned). */
+BEAM_MOE_API beam_moe_status beam_moe_tp_region(beam_moe_t h, void** region);
+/* regions: host array of `world` device addresses (regions[rank] must be this handle's own
+ * region); 1 <= world <= 16.  Synchronises `stream` and the device, clears this rank's
+ * flags.  Call on every rank before the group's first forward. */
+BEAM_MOE_API beam_moe_status beam_moe_tp_attach(beam_moe_t h, int32_t rank, int32_t world, void* const* regions,
+                                                void* stream);
+/* x, residual, out, num_tokens as beam_moe_forward (out on every rank; out may equal
+ * residual).  Enqueued on `stream`; the exchange waits on the device, not the host. */
+BEAM_MOE_API beam_moe_status beam_moe_forward_tp(beam_moe_t h, const void* x, const void* residual, void* out,
+                                                 int32_t num_tokens, void* stream);
+/* beam_moe_forward_tp in two halves: phase 0 = routing, GEMMs, this rank's partial m and its
+ * publication; phase 1 = the wait for every rank's partials, their sum, norm and residual.
+ * Phases alternate (0, 1, 0, 1, ...) with the same num_tokens.  Splitting lets ranks that
+ * share one GPU run every rank's phase 0 before any phase 1, so no kernel waits on a kernel
+ * that has not run. */
+BEAM_MOE_API beam_moe_status beam_moe_forward_tp_phase(beam_moe_t h, const void* x, const void* residual, void* out,
+                                                       int32_t num_tokens, int32_t phase, void* stream);
+/* cudaIpcGetMemHandle / cudaIpcOpenMemHandle / cudaIpcCloseMemHandle of a region, as
+ * BEAM_MOE_IPC_HANDLE_BYTES opaque bytes (host memory), so that callers need no CUDA
+ * headers. */
+BEAM_MOE_API beam_moe_status beam_moe_ipc_export(const void* dev_ptr, void* handle_out);
+BEAM_MOE_API beam_moe_status beam_moe_ipc_import(const void* handle, void** dev_ptr);
+BEAM_MOE_API beam_moe_status beam_moe_ipc_close(void* dev_ptr);
 
 /* Bytes of logits_ws that beam_moe_route needs for this shape (the logits may be held as
  * partial sums over slices of H).  0 for empty shapes. */

@@ -26,8 +26,11 @@ EXPORTED = [
     "beam_moe_last_launch_count", "beam_moe_status_string", "beam_moe_destroy", "beam_moe_profile_enable",
     "beam_moe_profile_read", "beam_moe_kernel_name", "beam_moe_route_static", "beam_moe_debug_wait_timeout",
     "beam_moe_forward_prenorm", "beam_moe_set_gemm_mode", "beam_moe_create_mxfp8", "beam_moe_quantize_mxfp8",
-    "beam_moe_expert_format",
+    "beam_moe_expert_format", "beam_moe_tp_region_bytes", "beam_moe_tp_region", "beam_moe_tp_attach",
+    "beam_moe_forward_tp", "beam_moe_forward_tp_phase", "beam_moe_ipc_export", "beam_moe_ipc_import",
+    "beam_moe_ipc_close",
 ]
+IPC_HANDLE_BYTES = 64
 FMT_NVFP4, FMT_MXFP8 = 0, 1
 FORMATS = {"nvfp4": FMT_NVFP4, "mxfp8": FMT_MXFP8}
 
@@ -83,6 +86,14 @@ def _load():
                                         ctypes.POINTER(vp)]),
         "beam_moe_quantize_mxfp8": (i32, [vp, i64, i64, vp, vp, vp]),
         "beam_moe_expert_format": (i32, [vp]),
+        "beam_moe_tp_region_bytes": (i64, [vp]),
+        "beam_moe_tp_region": (i32, [vp, ctypes.POINTER(vp)]),
+        "beam_moe_tp_attach": (i32, [vp, i32, i32, ctypes.POINTER(vp), vp]),
+        "beam_moe_forward_tp": (i32, [vp, vp, vp, vp, i32, vp]),
+        "beam_moe_forward_tp_phase": (i32, [vp, vp, vp, vp, i32, i32, vp]),
+        "beam_moe_ipc_export": (i32, [vp, vp]),
+        "beam_moe_ipc_import": (i32, [vp, ctypes.POINTER(vp)]),
+        "beam_moe_ipc_close": (i32, [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -133,6 +144,49 @@ def beam_moe_create_mxfp8(cfg: BeamMoeConfig, weights: BeamMoeWeightsMxfp8, stre
 
 def beam_moe_expert_format(h) -> int:
     return int(_lib.beam_moe_expert_format(h))
+
+
+def beam_moe_tp_region_bytes(h) -> int:
+    return int(_lib.beam_moe_tp_region_bytes(h))
+
+
+def beam_moe_tp_region(h) -> int:
+    """Device address of the handle's tensor-parallel exchange region (allocated on first use)."""
+    p = ctypes.c_void_p()
+    _check(_lib.beam_moe_tp_region(h, ctypes.byref(p)), "beam_moe_tp_region")
+    return int(p.value)
+
+
+def beam_moe_tp_attach(h, rank: int, world: int, regions, stream=None):
+    arr = (ctypes.c_void_p * world)(*[int(r) for r in regions])
+    _check(_lib.beam_moe_tp_attach(h, int(rank), int(world), arr, _stream(stream)), "beam_moe_tp_attach")
+
+
+def beam_moe_forward_tp(h, x, residual, out, num_tokens: int, stream=None):
+    _check(_lib.beam_moe_forward_tp(h, _ptr(x), _ptr(residual), _ptr(out), int(num_tokens), _stream(stream)),
+           "beam_moe_forward_tp")
+
+
+def beam_moe_forward_tp_phase(h, x, residual, out, num_tokens: int, phase: int, stream=None):
+    _check(_lib.beam_moe_forward_tp_phase(h, _ptr(x), _ptr(residual), _ptr(out), int(num_tokens), int(phase),
+                                          _stream(stream)), "beam_moe_forward_tp_phase")
+
+
+def beam_moe_ipc_export(dev_ptr: int) -> bytes:
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(_lib.beam_moe_ipc_export(ctypes.c_void_p(int(dev_ptr)), buf), "beam_moe_ipc_export")
+    return buf.raw
+
+
+def beam_moe_ipc_import(handle: bytes) -> int:
+    p = ctypes.c_void_p()
+    _check(_lib.beam_moe_ipc_import(ctypes.create_string_buffer(bytes(handle), IPC_HANDLE_BYTES), ctypes.byref(p)),
+           "beam_moe_ipc_import")
+    return int(p.value)
+
+
+def beam_moe_ipc_close(dev_ptr: int):
+    _check(_lib.beam_moe_ipc_close(ctypes.c_void_p(int(dev_ptr))), "beam_moe_ipc_close")
 
 
 def beam_moe_forward(h, x, residual, out, num_tokens: int, stream=None):
@@ -286,6 +340,22 @@ class MoELayer:
 
     def profile(self, enable: bool = True):
         beam_moe_profile_enable(self.handle, enable)
+
+    # ---- tensor parallelism (this layer holds one rank's slice of the experts; see tp.py)
+    def tp_region(self) -> int:
+        return beam_moe_tp_region(self.handle)
+
+    def tp_attach(self, rank: int, world: int, regions, stream=None):
+        beam_moe_tp_attach(self.handle, rank, world, regions, stream)
+
+    def forward_tp(self, x, residual, out=None, stream=None):
+        out = torch.empty_like(residual) if out is None else out
+        beam_moe_forward_tp(self.handle, x, residual, out, x.shape[0], stream)
+        return out
+
+    def forward_tp_phase(self, x, residual, out, phase: int, stream=None):
+        beam_moe_forward_tp_phase(self.handle, x, residual, out, x.shape[0], phase, stream)
+        return out
 
     def set_gemm_mode(self, mode: int):
         beam_moe_set_gemm_mode(self.handle, mode)

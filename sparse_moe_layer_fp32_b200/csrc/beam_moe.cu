@@ -41,6 +41,19 @@ struct beam_moe_ctx {
   int kv;                       // K values per activation / weight tile: 256 (NVFP4), 128 (MXFP8)
   int sfa_tile;                 // scale bytes per 128-row block per K tile: 2048 (NVFP4), 512
   uint16_t *stage_x, *stage_res, *stage_out;
+  // beam_moe_forward_host: the residual's upload runs on a second stream while the forward
+  // computes; the finalize waits for it (created on the first host-buffer forward)
+  cudaStream_t copy_stream;
+  cudaEvent_t ev_start, ev_res;
+  // tensor parallelism (beam_moe_tp_*): this handle holds one rank's slice of the experts
+  uint8_t* tp_region;           // this rank's exchange region (owned), or null
+  uint8_t** tp_regions_dev;     // device array [kMaxTpRanks]: every rank's region
+  TpGroup tp;                   // every rank's region, this rank, the group size
+  bool tp_attached;
+  bool tp_pending;              // phase 0 ran, phase 1 not yet
+  uint32_t tp_epoch;            // forwards so far in this group (the flag value of the last one)
+  unsigned int* tp_counter;     // CTA arrivals of tp_partial
+  int tp_last_T;
   int last_T;
   int last_splits;  // logits layout of the last forward: [splits][T][E] partial sums
   int last_launches;
@@ -357,9 +370,18 @@ beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num
   return BEAM_MOE_OK;
 }
 
+// tp_phase: -1 the single-GPU forward; 0 the tensor-parallel forward up to the partial sums
+// and their publication (tp_partial instead of finalize); 1 only the all-reduce + finalize
+// (tp_reduce) of the last phase 0.
 static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* residual, void* out, void* next_x,
-                                    const void* next_gamma, float next_eps, int32_t num_tokens, void* stream) {
+                                    const void* next_gamma, float next_eps, int32_t num_tokens, void* stream,
+                                    int tp_phase = -1, cudaEvent_t residual_ready = nullptr) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;
+  if (tp_phase >= 0) {
+    if (!h->tp_attached) return BEAM_MOE_ERR_INVALID_ARG;
+    if (tp_phase == 1 && (!h->tp_pending || num_tokens != h->tp_last_T)) return BEAM_MOE_ERR_INVALID_ARG;
+    if (tp_phase == 0 && h->tp_pending) return BEAM_MOE_ERR_INVALID_ARG;  // phases must alternate
+  }
   if (num_tokens < 0 || num_tokens > h->Tmax) return BEAM_MOE_ERR_INVALID_ARG;
   if (num_tokens == 0) {
     h->last_T = 0;
@@ -381,6 +403,16 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     return cudaEventRecord(h->events[launches + 1], s);
   };
   if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
+  if (tp_phase == 1) {
+    BEAM_TRY(launch_tp_reduce(static_cast<const uint16_t*>(residual), h->gamma, T, H, h->cfg.rms_eps, h->tp,
+                              h->tp_epoch, static_cast<uint16_t*>(out), h->err, s));
+    BEAM_TRY(mark("tp_reduce"));
+    ++launches;
+    h->tp_pending = false;
+    h->last_launches = launches;
+    h->profiled_last = prof;
+    return BEAM_MOE_OK;
+  }
   const BlockScales bscales{h->w_gu_alpha, h->w_d_alpha, h->cfg.alpha_a1, h->cfg.alpha_a2};
   // CTA pairs for the expert GEMM when the average expert has a few hundred rows
   const bool mx = h->fmt == BEAM_MOE_FMT_MXFP8;
@@ -461,11 +493,21 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     BEAM_TRY(launch_gemm_experts(g, h->num_sms, s));
   BEAM_TRY(mark("gemm_experts"));
   ++launches;
-  BEAM_TRY(launch_finalize(h->y, h->w, h->inv, static_cast<const uint16_t*>(residual), h->gamma, T, H, k,
-                           h->cfg.rms_eps, static_cast<uint16_t*>(out), static_cast<uint16_t*>(next_x),
-                           static_cast<const uint16_t*>(next_gamma), next_eps, h->err, s));
-  BEAM_TRY(mark("finalize"));
-  ++launches;
+  if (tp_phase == 0) {
+    BEAM_TRY(launch_tp_partial(h->y, h->w, h->inv, T, H, k, h->tp, h->tp_epoch + 1, h->tp_counter, s));
+    BEAM_TRY(mark("tp_partial"));
+    ++launches;
+    ++h->tp_epoch;
+    h->tp_pending = true;
+    h->tp_last_T = T;
+  } else {
+    if (residual_ready) BEAM_TRY(cudaStreamWaitEvent(s, residual_ready, 0));
+    BEAM_TRY(launch_finalize(h->y, h->w, h->inv, static_cast<const uint16_t*>(residual), h->gamma, T, H, k,
+                             h->cfg.rms_eps, static_cast<uint16_t*>(out), static_cast<uint16_t*>(next_x),
+                             static_cast<const uint16_t*>(next_gamma), next_eps, h->err, s));
+    BEAM_TRY(mark("finalize"));
+    ++launches;
+  }
   h->last_T = T;
   h->last_launches = launches;
   h->profiled_last = prof;
@@ -488,6 +530,88 @@ beam_moe_status beam_moe_forward_prenorm(beam_moe_t h, const void* x, const void
   return forward_impl(h, x, residual, out, next_x, next_gamma, next_eps, num_tokens, stream);
 }
 
+int64_t beam_moe_tp_region_bytes(beam_moe_t h) {
+  if (!h) return 0;
+  return static_cast<int64_t>(kTpHeaderBytes) + 2ll * h->Tmax * h->H * static_cast<int64_t>(sizeof(float));
+}
+
+beam_moe_status beam_moe_tp_region(beam_moe_t h, void** region) {
+  if (!h || !region) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!h->tp_region) {
+    const size_t bytes = static_cast<size_t>(beam_moe_tp_region_bytes(h));
+    BEAM_TRY(dalloc(h, &h->tp_region, bytes));
+    BEAM_TRY(dalloc(h, &h->tp_counter, sizeof(unsigned int)));
+    BEAM_TRY(dalloc(h, &h->tp_regions_dev, sizeof(uint8_t*) * kMaxTpRanks));
+    BEAM_TRY(cudaMemset(h->tp_region, 0, kTpHeaderBytes));
+    BEAM_TRY(cudaMemset(h->tp_counter, 0, sizeof(unsigned int)));
+  }
+  *region = h->tp_region;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_tp_attach(beam_moe_t h, int32_t rank, int32_t world, void* const* regions, void* stream) {
+  if (!h || !regions || world < 1 || world > kMaxTpRanks || rank < 0 || rank >= world) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!h->tp_region || regions[rank] != h->tp_region) return BEAM_MOE_ERR_INVALID_ARG;
+  for (int q = 0; q < world; ++q)
+    if (!regions[q] || !aligned(regions[q], 256)) return BEAM_MOE_ERR_INVALID_ARG;
+  BEAM_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  BEAM_TRY(cudaMemset(h->tp_region, 0, kTpHeaderBytes));  // no epoch published yet in this group
+  BEAM_TRY(cudaDeviceSynchronize());
+  uint8_t* table[kMaxTpRanks] = {};
+  for (int q = 0; q < world; ++q) table[q] = static_cast<uint8_t*>(regions[q]);
+  BEAM_TRY(cudaMemcpy(h->tp_regions_dev, table, sizeof(table), cudaMemcpyHostToDevice));
+  TpGroup g{};
+  g.regions = h->tp_regions_dev;
+  g.own = h->tp_region;
+  g.rank = rank;
+  g.world = world;
+  g.buf_floats = static_cast<size_t>(h->Tmax) * h->H;
+  h->tp = g;
+  h->tp_epoch = 0;
+  h->tp_pending = false;
+  h->tp_attached = true;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_forward_tp_phase(beam_moe_t h, const void* x, const void* residual, void* out,
+                                          int32_t num_tokens, int32_t phase, void* stream) {
+  if (phase != 0 && phase != 1) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!h || num_tokens <= 0) return num_tokens == 0 && h ? BEAM_MOE_OK : BEAM_MOE_ERR_INVALID_ARG;
+  if (phase == 1 && (!residual || !out || !aligned(residual, 16) || !aligned(out, 16)))
+    return BEAM_MOE_ERR_INVALID_ARG;
+  return forward_impl(h, x, residual, out, nullptr, nullptr, 0.0f, num_tokens, stream, phase);
+}
+
+beam_moe_status beam_moe_forward_tp(beam_moe_t h, const void* x, const void* residual, void* out,
+                                    int32_t num_tokens, void* stream) {
+  beam_moe_status st = beam_moe_forward_tp_phase(h, x, residual, out, num_tokens, 0, stream);
+  if (st != BEAM_MOE_OK || num_tokens == 0) return st;
+  return beam_moe_forward_tp_phase(h, x, residual, out, num_tokens, 1, stream);
+}
+
+beam_moe_status beam_moe_ipc_export(const void* dev_ptr, void* handle_out) {
+  if (!dev_ptr || !handle_out) return BEAM_MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t hd;
+  BEAM_TRY(cudaIpcGetMemHandle(&hd, const_cast<void*>(dev_ptr)));
+  static_assert(sizeof(hd) == BEAM_MOE_IPC_HANDLE_BYTES, "IPC handle size");
+  std::memcpy(handle_out, &hd, sizeof(hd));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_ipc_import(const void* handle, void** dev_ptr) {
+  if (!handle || !dev_ptr) return BEAM_MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t hd;
+  std::memcpy(&hd, handle, sizeof(hd));
+  BEAM_TRY(cudaIpcOpenMemHandle(dev_ptr, hd, cudaIpcMemLazyEnablePeerAccess));
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_ipc_close(void* dev_ptr) {
+  if (!dev_ptr) return BEAM_MOE_ERR_INVALID_ARG;
+  BEAM_TRY(cudaIpcCloseMemHandle(dev_ptr));
+  return BEAM_MOE_OK;
+}
+
 beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const void* residual_host, void* out_host,
                                       int32_t num_tokens, void* stream) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;
@@ -496,9 +620,22 @@ beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const vo
   if (!x_host || !residual_host || !out_host) return BEAM_MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t bytes = sizeof(uint16_t) * static_cast<size_t>(num_tokens) * h->H;
+  if (!h->copy_stream) {
+    BEAM_TRY(cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking));
+    BEAM_TRY(cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming));
+    BEAM_TRY(cudaEventCreateWithFlags(&h->ev_res, cudaEventDisableTiming));
+  }
+  // x first, at the full host-to-device bandwidth; the residual upload then starts (after
+  // everything before it on `stream`, including the previous forward's finalize, which
+  // read the staging buffer) and overlaps the routing and the expert GEMMs; only the
+  // finalize waits for it
   BEAM_TRY(cudaMemcpyAsync(h->stage_x, x_host, bytes, cudaMemcpyHostToDevice, s));
-  BEAM_TRY(cudaMemcpyAsync(h->stage_res, residual_host, bytes, cudaMemcpyHostToDevice, s));
-  beam_moe_status st = beam_moe_forward(h, h->stage_x, h->stage_res, h->stage_out, num_tokens, stream);
+  BEAM_TRY(cudaEventRecord(h->ev_start, s));
+  BEAM_TRY(cudaStreamWaitEvent(h->copy_stream, h->ev_start, 0));
+  BEAM_TRY(cudaMemcpyAsync(h->stage_res, residual_host, bytes, cudaMemcpyHostToDevice, h->copy_stream));
+  BEAM_TRY(cudaEventRecord(h->ev_res, h->copy_stream));
+  beam_moe_status st = forward_impl(h, h->stage_x, h->stage_res, h->stage_out, nullptr, nullptr, 0.0f, num_tokens,
+                                    stream, -1, h->ev_res);
   if (st != BEAM_MOE_OK) return st;
   BEAM_TRY(cudaMemcpyAsync(out_host, h->stage_out, bytes, cudaMemcpyDeviceToHost, s));
   return BEAM_MOE_OK;
@@ -621,6 +758,11 @@ void beam_moe_destroy(beam_moe_t h) {
   cudaDeviceSynchronize();
   for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i)
     if (h->events[i]) cudaEventDestroy(h->events[i]);
+  if (h->copy_stream) {
+    cudaEventDestroy(h->ev_start);
+    cudaEventDestroy(h->ev_res);
+    cudaStreamDestroy(h->copy_stream);
+  }
   free_all(h);
   delete h;
 }

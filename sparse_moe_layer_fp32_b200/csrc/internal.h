@@ -141,6 +141,22 @@ cudaError_t launch_gemm_experts_mx(const ExpertGemmArgs& a, int grid, cudaStream
 constexpr int kPairMinTokens = BEAM_MOE_PAIR_MIN_TOKENS;
 cudaError_t launch_gemm_experts_pair(const ExpertGemmArgs& a, int grid, cudaStream_t s);
 
+// ---- tensor-parallel finalize fused with its all-reduce (finalize_tp.cu)
+// Exchange region of one rank: kTpHeaderBytes of flags (u32 slot q = the last epoch rank q
+// published), then two buffers of [max_tokens][H] FP32 partial m (epoch parity).
+constexpr int kMaxTpRanks = 16;
+constexpr size_t kTpHeaderBytes = 1024;
+struct TpGroup {
+  uint8_t* const* regions;  // device array: every rank's region as mapped in this process
+  uint8_t* own;             // this rank's region (regions[rank])
+  int rank, world;
+  size_t buf_floats;        // floats per partial buffer: max_tokens * H
+};
+cudaError_t launch_tp_partial(const uint16_t* y, const float* w, const int32_t* inv, int T, int H, int k,
+                              const TpGroup& g, uint32_t epoch, unsigned int* counter, cudaStream_t s);
+cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, int H, float eps,
+                             const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, cudaStream_t s);
+
 // ---- finalize (finalize.cu)
 // next_x != nullptr also writes the next sublayer's pre-norm of out: bf16(out * rinv * next_gamma).
 cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,

@@ -1,0 +1,99 @@
+"""Host side of the tensor-parallel layer: weight shards, the exchange of the ranks' regions,
+and ranks that share one GPU.
+
+Tensor parallelism over the experts' intermediate size with the finalize fused to its
+all-reduce (vLLM PR "Day-0 support for Reflection's Beam-1.0", section "Status"; recipe
+"reflection/Beam-1.0-501B-A23B": NVFP4 with TP4 on Blackwell).  Rank r holds features
+[r I/W, (r+1) I/W) of every expert: those gate rows, the matching up rows and the same
+columns of down.  The device work is beam_moe_forward_tp (C ABI); this module only slices
+tensors and moves region addresses between processes.
+"""
+
+from __future__ import annotations
+
+from . import MoELayer, beam_moe_ipc_export, beam_moe_ipc_import
+
+WEIGHT_KEYS = ("w_gu", "w_gu_sf", "w_d", "w_d_sf")
+
+
+def shard_weights(weights: dict, rank: int, world: int, inter: int) -> dict:
+    """This rank's slice of layer weights in the C-ABI layout (either expert format).
+
+    w_gu / w_gu_sf [E][2I][..]: gate rows [r s, (r+1) s) then up rows [I + r s, I + (r+1) s),
+    s = I / world; w_d / w_d_sf [E][H][cols]: the r-th of `world` equal column ranges (the
+    same features, packed codes and scales alike).  Tensor scales, router weights and gamma
+    are shared unchanged."""
+    if world < 1 or not 0 <= rank < world or inter % world:
+        raise ValueError(f"cannot take shard {rank} of {world} of an intermediate size {inter}")
+    s = inter // world
+    out = {k: v for k, v in weights.items() if k not in WEIGHT_KEYS}
+    for key in ("w_gu", "w_gu_sf"):
+        t = weights[key]
+        if t.shape[1] != 2 * inter:
+            raise ValueError(f"{key} must have 2 * inter rows")
+        gate = t[:, rank * s:(rank + 1) * s]
+        up = t[:, inter + rank * s:inter + (rank + 1) * s]
+        out[key] = _cat_rows(gate, up)
+    for key in ("w_d", "w_d_sf"):
+        t = weights[key]
+        cols = t.shape[-1]
+        if cols % world:
+            raise ValueError(f"{key} columns do not split over {world} ranks")
+        c = cols // world
+        out[key] = t[..., rank * c:(rank + 1) * c].contiguous()
+    return out
+
+
+def _cat_rows(a, b):
+    import torch
+    return torch.cat([a, b], dim=1).contiguous()
+
+
+def connect(layer: MoELayer, rank: int, world: int, group=None, export=None, import_=None):
+    """Exchanges exchange-region addresses across processes (one per GPU) and attaches the
+    layer.  Every rank exports its region as an IPC handle, all handles are gathered over
+    torch.distributed (any backend), and each peer's handle is opened in this process.
+    Returns the addresses this process opened (close them with beam_moe_ipc_close after
+    the layer is destroyed)."""
+    import torch.distributed as dist
+    export = export or beam_moe_ipc_export
+    import_ = import_ or beam_moe_ipc_import
+    own = layer.tp_region()
+    handles = [None] * world
+    dist.all_gather_object(handles, bytes(export(own)), group=group)
+    regions, opened = [], []
+    for q, hd in enumerate(handles):
+        if q == rank:
+            regions.append(own)
+        else:
+            p = import_(hd)
+            regions.append(p)
+            opened.append(p)
+    layer.tp_attach(rank, world, regions)
+    return opened
+
+
+class SharedGpuGroup:
+    """W ranks of one tensor-parallel group in one process on one GPU (tests and
+    measurement when fewer GPUs than ranks are available).  The ranks run one after the
+    other: every rank's phase 0 (GEMMs, partial m, publication), then every rank's phase 1
+    (all-reduce + finalize), so no kernel waits on a kernel that has not run."""
+
+    def __init__(self, layers):
+        self.layers = list(layers)
+        regions = [lay.tp_region() for lay in self.layers]
+        for r, lay in enumerate(self.layers):
+            lay.tp_attach(r, len(self.layers), regions)
+
+    def forward(self, x, residual, outs=None):
+        import torch
+        outs = outs or [torch.empty_like(residual) for _ in self.layers]
+        for lay, o in zip(self.layers, outs):
+            lay.forward_tp_phase(x, residual, o, 0)
+        for lay, o in zip(self.layers, outs):
+            lay.forward_tp_phase(x, residual, o, 1)
+        return outs
+
+    def close(self):
+        for lay in self.layers:
+            lay.close()

@@ -66,3 +66,82 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.reduce_max(4.25, 1) == 4.25
     assert bench.whole_job_rate(8, 1, 0.25) == pytest.approx(32000.0)
+
+
+# ---------------------------------------------------------------- tensor-parallel host logic
+# The TP layer (experts split over ranks along the intermediate size, finalize fused to its
+# all-reduce) exchanges the ranks' exchange-region addresses as IPC handles over the process
+# group.  Two CPU ranks run sparse_moe_layer_fp32_b200.tp.connect with a stand-in layer and
+# stand-in IPC calls (no GPU): every rank must attach with all regions in rank order, its
+# own address in its own slot and each peer's address opened from that peer's handle.
+class _FakeLayer:
+    def __init__(self, rank):
+        self.rank = rank
+        self.attached = None
+
+    def tp_region(self):
+        return 0x10000 * (self.rank + 1)
+
+    def tp_attach(self, rank, world, regions):
+        self.attached = (rank, world, list(regions))
+
+
+def _tp_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        from sparse_moe_layer_fp32_b200 import tp
+        layer = _FakeLayer(rank)
+        export = lambda p: p.to_bytes(8, "little") + bytes(56)  # noqa: E731
+        import_ = lambda hd: int.from_bytes(hd[:8], "little") + 0x1  # noqa: E731  (a mapping differs from the owner's address)
+        opened = tp.connect(layer, rank, world, export=export, import_=import_)
+        q.put((rank, layer.attached, opened))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tp_connect_exchanges_regions_in_rank_order(repo_root):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 2
+    procs = [ctx.Process(target=_tp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, a0, o0), (r1, a1, o1) = res
+    assert a0 == (0, 2, [0x10000, 0x20001]) and o0 == [0x20001]
+    assert a1 == (1, 2, [0x10001, 0x20000]) and o1 == [0x10001]
+
+
+def test_tp_shard_weights_partition_the_experts():
+    from sparse_moe_layer_fp32_b200 import tp
+    E, H, inter, world = 3, 64, 256, 4
+    g = torch.Generator().manual_seed(0)
+    full = dict(router_w=torch.randn(E, H, generator=g), gamma=torch.ones(H),
+                w_gu=torch.randint(0, 255, (E, 2 * inter, H // 2), dtype=torch.uint8, generator=g),
+                w_gu_sf=torch.randint(0, 255, (E, 2 * inter, H // 16), dtype=torch.uint8, generator=g),
+                w_gu_alpha=torch.rand(E, generator=g),
+                w_d=torch.randint(0, 255, (E, H, inter // 2), dtype=torch.uint8, generator=g),
+                w_d_sf=torch.randint(0, 255, (E, H, inter // 16), dtype=torch.uint8, generator=g),
+                w_d_alpha=torch.rand(E, generator=g))
+    shards = [tp.shard_weights(full, r, world, inter) for r in range(world)]
+    s = inter // world
+    for key in ("w_gu", "w_gu_sf"):
+        gate = torch.cat([sh[key][:, :s] for sh in shards], dim=1)
+        up = torch.cat([sh[key][:, s:] for sh in shards], dim=1)
+        assert torch.equal(torch.cat([gate, up], dim=1), full[key])
+        assert all(sh[key].is_contiguous() and sh[key].shape[1] == 2 * s for sh in shards)
+    for key in ("w_d", "w_d_sf"):
+        assert torch.equal(torch.cat([sh[key] for sh in shards], dim=-1), full[key])
+        assert all(sh[key].is_contiguous() for sh in shards)
+    for key in ("router_w", "gamma", "w_gu_alpha", "w_d_alpha"):
+        assert all(sh[key] is full[key] for sh in shards)
+    with pytest.raises(ValueError):
+        tp.shard_weights(full, 0, 3, inter)
+    with pytest.raises(ValueError):
+        tp.shard_weights(full, 4, 4, inter)

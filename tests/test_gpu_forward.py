@@ -302,3 +302,33 @@ def test_forward_mxfp8_stages_and_end_to_end(bm, name, tokens, seed):
         layer.set_gemm_mode(bm.GEMM_PAIR)
     assert ei.value.status == bm.ERR_UNSUPPORTED
     layer.close()
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
+def test_forward_host_buffers_match_device_path(bm, fmt):
+    # beam_moe_forward_host: x uploads on the caller's stream, the residual on the handle's
+    # copy stream (overlapping routing and GEMMs, the finalize waits for it), out comes back
+    # on the caller's stream.  Same bits as the device-buffer forward, call after call with
+    # changing batch sizes (the staging buffers are reused), pinned or pageable host memory.
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(SHAPES["mid"], tokens=300)
+    weights = synthetic.make_weights(shape, 3, threads=4, fmt=fmt)
+    if fmt == "nvfp4":
+        layer = bm.MoELayer(max_tokens=300, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                            inter=shape.inter, alpha_a1=0.002, alpha_a2=0.0002, **weights)
+    else:
+        layer = bm.MoELayer(max_tokens=300, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                            inter=shape.inter, fmt="mxfp8", **weights)
+    xd, rd = synthetic.make_batch(shape, 3)
+    for T, pinned in [(300, True), (7, True), (300, False), (64, True), (1, False)]:
+        xh, rh = xd[:T].cpu(), rd[:T].cpu()
+        oh = torch.empty_like(rh)
+        if pinned:
+            xh, rh, oh = xh.pin_memory(), rh.pin_memory(), oh.pin_memory()
+        layer.forward_host(xh, rh, oh)
+        torch.cuda.synchronize()
+        ref = layer.forward(xd[:T], rd[:T])
+        torch.cuda.synchronize()
+        assert torch.equal(oh, ref.cpu()), (T, pinned)
+    layer.check()
+    layer.close()

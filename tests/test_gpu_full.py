@@ -40,10 +40,12 @@ def weights_i1536():
     return synthetic.make_weights(mi.SHAPES["decode8"], 0)
 
 
-def _check_workload(bm, shape, weights):
+def _check_workload(bm, shape, weights, fmt="nvfp4"):
     from sparse_moe_layer_fp32_b200 import synthetic
-    gold = np.load(os.path.join(GOLDEN, f"full_{shape.name}.npz"))
-    layer = synthetic.make_layer(shape, weights)
+    suffix = "" if fmt == "nvfp4" else f"_{fmt}"
+    gold = np.load(os.path.join(GOLDEN, f"full_{shape.name}{suffix}.npz"))
+    assert str(gold["experts_format"]) == fmt if "experts_format" in gold else fmt == "nvfp4"
+    layer = synthetic.make_layer(shape, weights, fmt=fmt)
     x, res = synthetic.make_batch(shape, 0)
     out = layer.forward(x, res)
     layer.check()
@@ -91,3 +93,15 @@ def test_full_size_page_implied_intermediate(bm):
     weights = synthetic.make_weights(shape, 0)
     near, rel, mx, used = _check_workload(bm, shape, weights)
     print(f"decode8_i2560: rel-L2 {rel:.2e}, max abs {mx:.2e}, experts used {used}")
+
+
+@pytest.mark.parametrize("name", ["decode8", "prefill16k"])
+def test_full_size_workload_mxfp8_experts(bm, name):
+    # the block-scaled FP8 variant of the experts (MXFP8), same routing and finalize
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = mi.SHAPES[name]
+    weights = synthetic.make_weights(shape, 0, fmt="mxfp8")
+    near, rel, mx, used = _check_workload(bm, shape, weights, fmt="mxfp8")
+    del weights
+    torch.cuda.empty_cache()
+    print(f"{name} mxfp8: sampled near-ties {near}, rel-L2 {rel:.2e}, max abs {mx:.2e}, experts used {used}")
