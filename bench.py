@@ -5,6 +5,11 @@ One step = one whole layer forward (router, top-k, permutation, NVFP4 quantisati
 two grouped NVFP4 GEMMs, finalize) over one synthetic batch of the chosen workload.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode8] [--impl ours|reference]
+                  [--experts-format nvfp4|mxfp8] [--tp-shared-gpu W]
+
+--experts-format mxfp8 measures the block-scaled FP8 variant of the experts (E4M3 values,
+one power-of-two scale per 32).  --tp-shared-gpu W measures the tensor-parallel layer with
+W ranks sharing this GPU, run in turn (per-rank phase timings; see run_tp_shared).
 
 N > 1 runs under torchrun, one rank per GPU: token data parallel replicas (each rank a
 full copy of the layer and its own batch, no collective on the data path; the process
