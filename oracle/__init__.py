@@ -63,4 +63,5 @@ from .moe import (  # noqa: F401
     moe_forward_tokens,
     shard_dequantized,
     moe_forward_tp,
+    moe_forward_ep,
 )

@@ -319,3 +319,47 @@ def moe_forward_tp(x, residual, router_w, gamma, experts: ExpertCache, top_k, al
     out_pre = np.asarray(residual, np.float64) + m / rms * np.asarray(gamma, np.float64)[None, :]
     return dict(ids=ids, w=w, near_tie=near_tie_mask(logits, top_k), m_parts=m_parts, m=m, out_pre=out_pre,
                 out=bf16_round(out_pre))
+
+
+# ----------------------------------------------------------------------------- expert parallel
+def moe_forward_ep(x_ranks, residual_ranks, router_w, gamma, experts: ExpertCache, num_experts, top_k, alpha_a1,
+                   alpha_a2, world: int, eps=1e-6):
+    """The layer with its experts split over `world` expert-parallel ranks, each with its own
+    batch (attention data parallelism: [PR] "Status", Attention DP + MegaMoE; [RECIPE]
+    "Overview": 8 of 256 experts).  Rank q holds experts [q E/W, (q+1) E/W).  Dispatch: every
+    rank receives every rank's tokens (all-gather, rank order); rank q routes them all and
+    applies only its experts, giving partial m_q for every token; combine: rank r's output
+    rows are residual_r + RMSNorm(sum_q m_q[its tokens]) * gamma (reduce-scatter, ranks in
+    order).  Returns dict(ids, w, m_parts [world, sum T, H], m, out_pre per rank, out per
+    rank, near_tie)."""
+    if num_experts % world:
+        raise ValueError("the experts must split evenly over the ranks")
+    x = np.concatenate([np.asarray(v, np.float64) for v in x_ranks])
+    t_count, hidden = x.shape
+    logits = router_logits(x, router_w)
+    ids, w, _ = route_topk(logits, top_k)
+    fmt = experts.fmt
+    a1_packed, a1_sf = quantize_act(x.astype(np.float32), alpha_a1, fmt)
+    e_loc = num_experts // world
+    m_parts = np.zeros((world, t_count, hidden), np.float64)
+    for q in range(world):
+        for e in range(q * e_loc, (q + 1) * e_loc):
+            tt, jj = np.nonzero(ids == e)
+            if len(tt) == 0:
+                continue
+            y = expert_forward(a1_packed[tt], a1_sf[tt], alpha_a1, experts.dequantized(e), alpha_a2, fmt)["y"]
+            np.add.at(m_parts[q], tt, w[tt, jj][:, None] * y)
+    m = np.zeros((t_count, hidden), np.float64)
+    for q in range(world):
+        m = m + m_parts[q]
+    rms = np.sqrt(np.mean(m * m, axis=1, keepdims=True) + eps)
+    n = m / rms * np.asarray(gamma, np.float64)[None, :]
+    out_pre, out, begin = [], [], 0
+    for res in residual_ranks:
+        res = np.asarray(res, np.float64)
+        pre = res + n[begin:begin + res.shape[0]]
+        out_pre.append(pre)
+        out.append(bf16_round(pre))
+        begin += res.shape[0]
+    return dict(ids=ids, w=w, near_tie=near_tie_mask(logits, top_k), m_parts=m_parts, m=m, out_pre=out_pre,
+                out=out)

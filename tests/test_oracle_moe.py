@@ -283,3 +283,31 @@ def test_tensor_parallel_partials_sum_to_the_unsharded_layer():
     np.testing.assert_array_equal(d1, w_d[:, inter // 4: inter // 2])
     with pytest.raises(ValueError):
         moe.shard_dequantized((w_gu, w_d), 0, 3)
+
+
+def test_expert_parallel_partials_sum_to_the_unsharded_layer():
+    # Experts split over W ranks, each rank with its own batch: every token's slots fall in
+    # exactly one rank's expert range, so the ranks' partial m add up to the unsharded m of
+    # the concatenated batch, and each rank's output rows are that layer's rows of its
+    # tokens.  W = 1 is the unsharded layer itself.
+    shape, x, res, wr, g, cache = _tiny()
+    shape2, x2, res2, _, _, _ = _tiny(seed=5)
+    a1s, a2s = np.float32(5.0 / 2688), np.float32(3.0 / 2688)
+    xs, rs = [x, x2[:3]], [res, res2[:3]]
+    full = moe.moe_forward(np.concatenate(xs), np.concatenate(rs), wr, g, cache, shape.experts, shape.top_k, a1s,
+                           a2s)
+    for world in (1, 2, 4):
+        xw = xs if world == 2 else ([np.concatenate(xs)] if world == 1 else [x[:2], x[2:], x2[:1], x2[1:3]])
+        rw = rs if world == 2 else ([np.concatenate(rs)] if world == 1 else [res[:2], res[2:], res2[:1], res2[1:3]])
+        ep = moe.moe_forward_ep(xw, rw, wr, g, cache, shape.experts, shape.top_k, a1s, a2s, world)
+        np.testing.assert_array_equal(ep["ids"], full["ids"])
+        np.testing.assert_allclose(ep["m"], full["m"], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(np.concatenate(ep["out_pre"]), full["out_pre"], rtol=0, atol=1e-12)
+        # each rank's partial only holds its experts' slots
+        e_loc = shape.experts // world
+        for q in range(world):
+            own = (full["ids"] // e_loc) == q
+            idle = ~own.any(axis=1)
+            assert np.all(ep["m_parts"][q][idle] == 0)
+    with pytest.raises(ValueError):
+        moe.moe_forward_ep(xs, rs, wr, g, cache, shape.experts, shape.top_k, a1s, a2s, 3)
