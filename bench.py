@@ -404,31 +404,51 @@ def run_tp_shared(args, shape):
     all-reduce) with all W ranks on one GPU, run in turn: every rank's phase 0 (routing,
     its slice of the expert GEMMs, its partial m and their publication), then every rank's
     phase 1 (the exchange, sum, norm, residual).  Each phase is timed with CUDA events on
-    the launching stream; a rank's step = its phase 0 + phase 1.  `value` estimates the
-    group's tokens/s if each rank had its own GPU: T / the slowest rank's step.  The
-    partials that rank r reads from its peers sit in this GPU's memory here, so the NVLink
-    transfer of the exchange (W x T x H x 4 B per rank) is not in the estimate."""
+    the launching stream; a rank's step = the sum of its phases.  `value` estimates the
+    group's tokens/s if each rank had its own GPU: tokens / the slowest rank's step.  The
+    data that rank r reads from its peers sit in this GPU's memory here, so the NVLink
+    transfer of the exchange (W x T x H x 4 B per rank) is not in the estimate.
+
+    With --ep-shared-gpu W instead: the expert-parallel layer (rank r holds experts
+    [r E/W, (r+1) E/W) and its own batch of the workload's T tokens; three phases:
+    dispatch, the rank's experts on the gathered W T tokens, combine + finalize); `value` =
+    W T / the slowest rank's step (weak scaling of the batch)."""
     import dataclasses
     import torch
     import sparse_moe_layer_fp32_b200 as bm
     from sparse_moe_layer_fp32_b200 import synthetic, tp
 
-    W, fmt = args.tp_shared_gpu, args.experts_format
+    ep = bool(args.ep_shared_gpu)
+    W, fmt = (args.ep_shared_gpu if ep else args.tp_shared_gpu), args.experts_format
     torch.cuda.set_device(0)
     full = synthetic.make_weights(shape, 0, fmt=fmt)
     a1, a2 = mi.activation_scales(shape) if fmt == "nvfp4" else (1.0, 1.0)
     layers = []
     for r in range(W):
-        sh = tp.shard_weights(full, r, W, shape.inter)
-        layers.append(bm.MoELayer(max_tokens=shape.tokens, hidden=shape.hidden, num_experts=shape.experts,
-                                  top_k=shape.top_k, inter=shape.inter // W, alpha_a1=float(a1), alpha_a2=float(a2),
-                                  rms_eps=shape.rms_eps, fmt=fmt, **sh))
+        if ep:
+            sh = tp.shard_experts(full, r, W, shape.experts)
+            e_loc = shape.experts // W
+            layers.append(bm.MoELayer(max_tokens=W * shape.tokens, hidden=shape.hidden, num_experts=shape.experts,
+                                      top_k=shape.top_k, inter=shape.inter, alpha_a1=float(a1), alpha_a2=float(a2),
+                                      rms_eps=shape.rms_eps, fmt=fmt, expert_begin=r * e_loc, expert_count=e_loc,
+                                      **sh))
+        else:
+            sh = tp.shard_weights(full, r, W, shape.inter)
+            layers.append(bm.MoELayer(max_tokens=shape.tokens, hidden=shape.hidden, num_experts=shape.experts,
+                                      top_k=shape.top_k, inter=shape.inter // W, alpha_a1=float(a1),
+                                      alpha_a2=float(a2), rms_eps=shape.rms_eps, fmt=fmt, **sh))
         del sh
     del full
     torch.cuda.empty_cache()
     grp = tp.SharedGpuGroup(layers)
-    x, res = synthetic.make_batch(shape, 0)
-    outs = [torch.empty_like(res) for _ in range(W)]
+    if ep:  # each rank its own batch (seeds 0..W-1)
+        batches = [synthetic.make_batch(shape, r) for r in range(W)]
+        xs, rs = [b[0] for b in batches], [b[1] for b in batches]
+    else:
+        x, res = synthetic.make_batch(shape, 0)
+        xs, rs = [x] * W, [res] * W
+    outs = [torch.empty_like(rs[r]) for r in range(W)]
+    nphase = 3 if ep else 2
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     clean = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -437,25 +457,33 @@ def run_tp_shared(args, shape):
         flush.zero_()
         clean.sum()
 
+    def run_phase(lay, r, phase):
+        if ep:
+            lay.forward_ep_phase(xs[r], rs[r], outs[r], phase)
+        else:
+            lay.forward_tp_phase(xs[r], rs[r], outs[r], phase)
+
     for _ in range(max(args.warmup, 3)):
-        grp.forward(x, res, outs)
+        for phase in range(nphase):
+            for r, lay in enumerate(layers):
+                run_phase(lay, r, phase)
         flush_l2()
     for lay in layers:
         lay.check()
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    ph = [[[], []] for _ in range(W)]
+    ph = [[[] for _ in range(nphase)] for _ in range(W)]
     kern = {}
     with ClockSampler(0) as clk:
         for step in range(args.steps + 1):
             prof = step == args.steps  # one extra pass with the library's per-kernel events
             for lay in layers:
                 lay.profile(prof)
-            for phase in (0, 1):
+            for phase in range(nphase):
                 for r, lay in enumerate(layers):
                     flush_l2()  # each rank starts cold, as on its own GPU
                     a, b = ev(), ev()
                     a.record(stream)
-                    lay.forward_tp_phase(x, res, outs[r], phase)
+                    run_phase(lay, r, phase)
                     b.record(stream)
                     if prof:
                         for name, kms in lay.kernel_times():
@@ -465,29 +493,33 @@ def run_tp_shared(args, shape):
         torch.cuda.synchronize()
     for lay in layers:
         lay.check()
-    assert all(torch.equal(o, outs[0]) for o in outs[1:]), "ranks disagree"
-    p0 = [sum(a.elapsed_time(b) for a, b in ph[r][0]) / args.steps for r in range(W)]
-    p1 = [sum(a.elapsed_time(b) for a, b in ph[r][1]) / args.steps for r in range(W)]
-    rank_ms = [p0[r] + p1[r] for r in range(W)]
+    if not ep:
+        assert all(torch.equal(o, outs[0]) for o in outs[1:]), "ranks disagree"
+    pms = [[sum(a.elapsed_time(b) for a, b in ph[r][p]) / args.steps for r in range(W)] for p in range(nphase)]
+    rank_ms = [sum(pms[p][r] for p in range(nphase)) for r in range(W)]
     kms = {n: sum(v) / len(v) for n, v in kern.items()}
     T, H = shape.tokens, shape.hidden
     pk = peaks()
-    red_bytes = W * T * H * 4 + 2 * T * H * 2 + H * 2
-    part_bytes = T * shape.top_k * H * 2 + W * T * H * 4 / W  # its y rows, its own partial m
+    red_bytes = W * T * H * 4 + 2 * T * H * 2 + H * 2  # per rank: W partials of its T tokens, residual, out
+    part_bytes = T * shape.top_k * H * 2 + (W * T if ep else T) * H * 4  # y rows it holds, its partial m
     roof = {"bound": "hbm", "kernel": "tp_reduce", "kernel_ms": kms.get("tp_reduce"),
             "achieved": red_bytes / (kms["tp_reduce"] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s",
             "traffic": None, "peak_source": f"{pk['src']} copy bandwidth"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     line = {
-        "metric": METRIC, "value": T / (max(rank_ms) / 1e3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-        "warmup": max(args.warmup, 3), "ms_per_step": max(rank_ms), "higher_is_better": True, "scaling": "strong",
+        "metric": METRIC, "value": (W * T if ep else T) / (max(rank_ms) / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": max(rank_ms), "higher_is_better": True,
+        "scaling": "weak" if ep else "strong",
         "vs_baseline": None,
         "dtype": ("nvfp4" if fmt == "nvfp4" else "mxfp8") + " experts, fp32 router, accumulation and all-reduce",
         "data": "synthetic (seeded; random-init weights of the layer's shapes)",
-        "config": dict(workload_config(shape, "write+read", fmt), parallelism=f"tp{W}, ranks sharing one GPU in turn"),
-        "estimate": "value = T / slowest rank's (phase 0 + phase 1); peers' partials read from this GPU's memory, "
+        "config": dict(workload_config(shape, "write+read", fmt),
+                       parallelism=f"{'ep' if ep else 'tp'}{W}, ranks sharing one GPU in turn"
+                                   + (f", {T} tokens per rank" if ep else "")),
+        "estimate": "value = tokens / slowest rank's sum of phases; peers' data read from this GPU's memory, "
                     "so the NVLink transfer of the exchange is not included",
-        "tp": {"world": W, "rank_ms": rank_ms, "phase0_ms": p0, "phase1_ms": p1,
+        "tp": {"world": W, "mode": "ep" if ep else "tp", "rank_ms": rank_ms, "phase_ms": pms,
+               "phase0_ms": pms[0], "phase1_ms": pms[1],
                "exchange_bytes_per_rank": W * T * H * 4, "tp_partial_bytes": part_bytes},
         "kernels_ms": kms, "roofline": roof, "gpu_launches": sum(lay.launches() for lay in layers),
         "clocks": clk.summary(),
@@ -506,6 +538,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tp-shared-gpu", type=int, default=0, metavar="W",
                     help="tensor-parallel layer with W ranks sharing this one GPU, run in turn (per-rank timing)")
+    ap.add_argument("--ep-shared-gpu", type=int, default=0, metavar="W",
+                    help="expert-parallel layer with W ranks (each its own batch) sharing this one GPU, run in turn")
     ap.add_argument("--experts-format", default="nvfp4", choices=["nvfp4", "mxfp8"],
                     help="routed experts in NVFP4 (default) or the block-scaled FP8 variant (MXFP8)")
     ap.add_argument("--l2-flush", default="write+read", choices=["write", "write+read"],
@@ -519,7 +553,7 @@ def main():
     if args.impl == "reference":
         run_reference(args, shape, rank, world)
         return
-    if args.tp_shared_gpu:
+    if args.tp_shared_gpu or args.ep_shared_gpu:
         emit(run_tp_shared(args, shape), 0)
         return
     if world > 1:

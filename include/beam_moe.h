@@ -201,6 +201,39 @@ BEAM_MOE_API beam_moe_status beam_moe_ipc_export(const void* dev_ptr, void* hand
 BEAM_MOE_API beam_moe_status beam_moe_ipc_import(const void* handle, void** dev_ptr);
 BEAM_MOE_API beam_moe_status beam_moe_ipc_close(void* dev_ptr);
 
+/* ---- Expert parallelism with attention data parallelism (vLLM PR "Day-0 support for
+ * Reflection's Beam-1.0", section "Status": Attention DP with the MegaMoE kernels; recipe,
+ * "Overview": 8 of 256 experts).  Each of W ranks holds experts [expert_begin,
+ * expert_begin + expert_count) (cfg->num_experts = all E, used for routing; the weight
+ * arrays and the tensor scales hold only the rank's experts, in order) and its own batch of
+ * num_tokens tokens, the same num_tokens on every rank.  cfg->max_tokens bounds the
+ * gathered batch: W * num_tokens.  beam_moe_forward_ep:
+ *   phase 0, dispatch: the rank's x rows go to every rank (peer stores into the ranks'
+ *            regions, rank order), then a delivery flag;
+ *   phase 1: wait for every rank's tokens, route all W * num_tokens of them (the same
+ *            result on every rank), run this rank's experts on the rows routed to them,
+ *            publish the partial m of every token;
+ *   phase 2, combine: out = residual + RMSNorm(sum over ranks of the partial m of this
+ *            rank's tokens) * gamma, for this rank's num_tokens rows.
+ * Regions, exchange and attach as for tensor parallelism (beam_moe_tp_region /
+ * beam_moe_ipc_* / beam_moe_tp_attach); beam_moe_forward and beam_moe_forward_tp refuse
+ * these handles (INVALID_ARG).  Dispatch moves whole BF16 rows to every rank (an all-gather)
+ * rather than only the k routed rows to their experts' ranks. */
+BEAM_MOE_API beam_moe_status beam_moe_create_ep(const beam_moe_config* cfg, const beam_moe_weights* weights,
+                                                int32_t expert_begin, int32_t expert_count, void* stream,
+                                                beam_moe_t* out);
+BEAM_MOE_API beam_moe_status beam_moe_create_ep_mxfp8(const beam_moe_config* cfg, const beam_moe_weights_mxfp8* weights,
+                                                      int32_t expert_begin, int32_t expert_count, void* stream,
+                                                      beam_moe_t* out);
+/* x, residual, out: this rank's [num_tokens][H] BF16 (device).  Like a collective: every
+ * rank calls it the same number of times with the same num_tokens. */
+BEAM_MOE_API beam_moe_status beam_moe_forward_ep(beam_moe_t h, const void* x, const void* residual, void* out,
+                                                 int32_t num_tokens, void* stream);
+/* One phase (0, 1, 2, in turn) of beam_moe_forward_ep, so that ranks sharing one GPU can run
+ * every rank's phase p before any rank's phase p + 1. */
+BEAM_MOE_API beam_moe_status beam_moe_forward_ep_phase(beam_moe_t h, const void* x, const void* residual, void* out,
+                                                       int32_t num_tokens, int32_t phase, void* stream);
+
 /* Bytes of logits_ws that beam_moe_route needs for this shape (the logits may be held as
  * partial sums over slices of H).  0 for empty shapes. */
 BEAM_MOE_API int64_t beam_moe_route_workspace_bytes(int32_t num_tokens, int32_t hidden, int32_t num_experts);

@@ -28,7 +28,8 @@ EXPORTED = [
     "beam_moe_forward_prenorm", "beam_moe_set_gemm_mode", "beam_moe_create_mxfp8", "beam_moe_quantize_mxfp8",
     "beam_moe_expert_format", "beam_moe_tp_region_bytes", "beam_moe_tp_region", "beam_moe_tp_attach",
     "beam_moe_forward_tp", "beam_moe_forward_tp_phase", "beam_moe_ipc_export", "beam_moe_ipc_import",
-    "beam_moe_ipc_close",
+    "beam_moe_ipc_close", "beam_moe_create_ep", "beam_moe_create_ep_mxfp8", "beam_moe_forward_ep",
+    "beam_moe_forward_ep_phase",
 ]
 IPC_HANDLE_BYTES = 64
 FMT_NVFP4, FMT_MXFP8 = 0, 1
@@ -94,6 +95,12 @@ def _load():
         "beam_moe_ipc_export": (i32, [vp, vp]),
         "beam_moe_ipc_import": (i32, [vp, ctypes.POINTER(vp)]),
         "beam_moe_ipc_close": (i32, [vp]),
+        "beam_moe_create_ep": (i32, [ctypes.POINTER(BeamMoeConfig), ctypes.POINTER(BeamMoeWeights), i32, i32, vp,
+                                     ctypes.POINTER(vp)]),
+        "beam_moe_create_ep_mxfp8": (i32, [ctypes.POINTER(BeamMoeConfig), ctypes.POINTER(BeamMoeWeightsMxfp8), i32,
+                                           i32, vp, ctypes.POINTER(vp)]),
+        "beam_moe_forward_ep": (i32, [vp, vp, vp, vp, i32, vp]),
+        "beam_moe_forward_ep_phase": (i32, [vp, vp, vp, vp, i32, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -140,6 +147,26 @@ def beam_moe_create_mxfp8(cfg: BeamMoeConfig, weights: BeamMoeWeightsMxfp8, stre
     _check(_lib.beam_moe_create_mxfp8(ctypes.byref(cfg), ctypes.byref(weights), _stream(stream), ctypes.byref(h)),
            "beam_moe_create_mxfp8")
     return h
+
+
+def beam_moe_create_ep(cfg: BeamMoeConfig, weights, expert_begin: int, expert_count: int, stream=None):
+    """Expert-parallel handle: weights (BeamMoeWeights or BeamMoeWeightsMxfp8) of experts
+    [expert_begin, expert_begin + expert_count) of cfg.num_experts."""
+    h = ctypes.c_void_p()
+    fn = _lib.beam_moe_create_ep_mxfp8 if isinstance(weights, BeamMoeWeightsMxfp8) else _lib.beam_moe_create_ep
+    _check(fn(ctypes.byref(cfg), ctypes.byref(weights), int(expert_begin), int(expert_count), _stream(stream),
+              ctypes.byref(h)), "beam_moe_create_ep")
+    return h
+
+
+def beam_moe_forward_ep(h, x, residual, out, num_tokens: int, stream=None):
+    _check(_lib.beam_moe_forward_ep(h, _ptr(x), _ptr(residual), _ptr(out), int(num_tokens), _stream(stream)),
+           "beam_moe_forward_ep")
+
+
+def beam_moe_forward_ep_phase(h, x, residual, out, num_tokens: int, phase: int, stream=None):
+    _check(_lib.beam_moe_forward_ep_phase(h, _ptr(x), _ptr(residual), _ptr(out), int(num_tokens), int(phase),
+                                          _stream(stream)), "beam_moe_forward_ep_phase")
 
 
 def beam_moe_expert_format(h) -> int:
@@ -297,7 +324,7 @@ class MoELayer:
 
     def __init__(self, *, max_tokens, hidden, num_experts, top_k, inter, router_w, w_gu, w_gu_sf, w_d, w_d_sf,
                  gamma, alpha_a1=1.0, alpha_a2=1.0, w_gu_alpha=None, w_d_alpha=None, rms_eps=1e-6, fmt="nvfp4",
-                 stream=None):
+                 expert_begin=None, expert_count=None, stream=None):
         if fmt not in FORMATS:
             raise ValueError(f"unknown expert format {fmt!r}")
         self.fmt = fmt
@@ -306,12 +333,19 @@ class MoELayer:
         self.hidden, self.top_k = hidden, top_k
         if fmt == "mxfp8":
             ws = [router_w, w_gu, w_gu_sf, w_d, w_d_sf, gamma]
-            self.handle = beam_moe_create_mxfp8(self.cfg, BeamMoeWeightsMxfp8(*[t.data_ptr() for t in ws]), stream)
+            wts = BeamMoeWeightsMxfp8(*[t.data_ptr() for t in ws])
         else:
             if w_gu_alpha is None or w_d_alpha is None:
                 raise ValueError("NVFP4 experts need w_gu_alpha and w_d_alpha")
             ws = [router_w, w_gu, w_gu_sf, w_gu_alpha, w_d, w_d_sf, w_d_alpha, gamma]
-            self.handle = beam_moe_create(self.cfg, BeamMoeWeights(*[t.data_ptr() for t in ws]), stream)
+            wts = BeamMoeWeights(*[t.data_ptr() for t in ws])
+        self.expert_parallel = expert_count is not None
+        if self.expert_parallel:  # this layer holds experts [expert_begin, expert_begin + expert_count)
+            self.handle = beam_moe_create_ep(self.cfg, wts, expert_begin or 0, expert_count, stream)
+        elif fmt == "mxfp8":
+            self.handle = beam_moe_create_mxfp8(self.cfg, wts, stream)
+        else:
+            self.handle = beam_moe_create(self.cfg, wts, stream)
 
     def forward(self, x, residual, out=None, stream=None):
         out = torch.empty_like(residual) if out is None else out
@@ -355,6 +389,15 @@ class MoELayer:
 
     def forward_tp_phase(self, x, residual, out, phase: int, stream=None):
         beam_moe_forward_tp_phase(self.handle, x, residual, out, x.shape[0], phase, stream)
+        return out
+
+    def forward_ep(self, x, residual, out=None, stream=None):
+        out = torch.empty_like(residual) if out is None else out
+        beam_moe_forward_ep(self.handle, x, residual, out, x.shape[0], stream)
+        return out
+
+    def forward_ep_phase(self, x, residual, out, phase: int, stream=None):
+        beam_moe_forward_ep_phase(self.handle, x, residual, out, x.shape[0], phase, stream)
         return out
 
     def set_gemm_mode(self, mode: int):

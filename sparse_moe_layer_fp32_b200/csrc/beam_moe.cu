@@ -54,6 +54,12 @@ struct beam_moe_ctx {
   uint32_t tp_epoch;            // forwards so far in this group (the flag value of the last one)
   unsigned int* tp_counter;     // CTA arrivals of tp_partial
   int tp_last_T;
+  // expert parallelism (beam_moe_create_ep*): this handle holds experts [e_begin, e_begin + e_count)
+  int e_begin, e_count;
+  bool ep;
+  bool ep_dispatched;           // phase 0 ran, phase 1 not yet
+  int ep_T;                     // this rank's tokens in the current forward
+  unsigned int* ep_counter;     // CTA arrivals of ep_dispatch
   int last_T;
   int last_splits;  // logits layout of the last forward: [splits][T][E] partial sums
   int last_launches;
@@ -190,9 +196,14 @@ struct ExpertWeightsIn {
   const uint16_t* gamma;
 };
 
+// e_count < 0: the handle holds every expert; else experts [e_begin, e_begin + e_count) of
+// cfg->num_experts, whose weights (and tensor scales) are the arrays of wts.
 beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& wts, int fmt, void* stream,
-                            beam_moe_t* out) {
+                            beam_moe_t* out, int e_begin = 0, int e_count = -1) {
   const bool mx = fmt == BEAM_MOE_FMT_MXFP8;
+  const bool ep = e_count >= 0;
+  if (!ep) e_count = cfg->num_experts;
+  if (e_begin < 0 || e_count < 1 || e_begin > cfg->num_experts - e_count) return BEAM_MOE_ERR_INVALID_ARG;
   if (!wts.router_w || !wts.w_gu || !wts.w_gu_sf || !wts.w_d || !wts.w_d_sf || !wts.gamma)
     return BEAM_MOE_ERR_INVALID_ARG;
   if (!mx && (!wts.w_gu_alpha || !wts.w_d_alpha)) return BEAM_MOE_ERR_INVALID_ARG;
@@ -211,6 +222,9 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   h->cfg = *cfg;
   if (mx) h->cfg.alpha_a1 = h->cfg.alpha_a2 = 1.0f;  // MX activations carry no tensor scale
   h->fmt = fmt;
+  h->ep = ep;
+  h->e_begin = e_begin;
+  h->e_count = e_count;
   h->kv = mx ? 128 : 256;
   h->sfa_tile = mx ? 512 : 4 * 512;
   h->H = cfg->hidden;
@@ -254,31 +268,32 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   // ---- weights
   CREATE_TRY(dalloc(h, &h->router_w, sizeof(float) * E * H));
   CREATE_TRY(dalloc(h, &h->router_w3, sizeof(uint16_t) * 3 * E * H));
+  const int Ew = e_count;  // experts whose weights this handle holds
   const size_t tile_bytes = mx ? kMxTileBytes : kTileBytes;
-  const size_t gu_tiles = static_cast<size_t>(E) * (2 * I / 256) * (H / h->kv);
-  const size_t d_tiles = static_cast<size_t>(E) * (H / 256) * (Ip / h->kv);
+  const size_t gu_tiles = static_cast<size_t>(Ew) * (2 * I / 256) * (H / h->kv);
+  const size_t d_tiles = static_cast<size_t>(Ew) * (H / 256) * (Ip / h->kv);
   CREATE_TRY(dalloc(h, &h->w_gu_tiles, gu_tiles * tile_bytes));
   CREATE_TRY(dalloc(h, &h->w_d_tiles, d_tiles * tile_bytes));
-  CREATE_TRY(dalloc(h, &h->w_gu_alpha, sizeof(float) * E));
-  CREATE_TRY(dalloc(h, &h->w_d_alpha, sizeof(float) * E));
+  CREATE_TRY(dalloc(h, &h->w_gu_alpha, sizeof(float) * Ew));
+  CREATE_TRY(dalloc(h, &h->w_d_alpha, sizeof(float) * Ew));
   CREATE_TRY(dalloc(h, &h->gamma, sizeof(uint16_t) * H));
   CREATE_TRY(cudaMemcpyAsync(h->router_w, wts.router_w, sizeof(float) * E * H, cudaMemcpyDeviceToDevice, s));
   CREATE_TRY(launch_split_router(h->router_w, E, H, h->router_w3, s));
   if (mx) {  // the accumulators need no dequantisation: unit scales in the block list
-    const std::vector<float> ones(E, 1.0f);
-    CREATE_TRY(cudaMemcpy(h->w_gu_alpha, ones.data(), sizeof(float) * E, cudaMemcpyHostToDevice));
-    CREATE_TRY(cudaMemcpy(h->w_d_alpha, ones.data(), sizeof(float) * E, cudaMemcpyHostToDevice));
+    const std::vector<float> ones(Ew, 1.0f);
+    CREATE_TRY(cudaMemcpy(h->w_gu_alpha, ones.data(), sizeof(float) * Ew, cudaMemcpyHostToDevice));
+    CREATE_TRY(cudaMemcpy(h->w_d_alpha, ones.data(), sizeof(float) * Ew, cudaMemcpyHostToDevice));
   } else {
-    CREATE_TRY(cudaMemcpyAsync(h->w_gu_alpha, wts.w_gu_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
-    CREATE_TRY(cudaMemcpyAsync(h->w_d_alpha, wts.w_d_alpha, sizeof(float) * E, cudaMemcpyDeviceToDevice, s));
+    CREATE_TRY(cudaMemcpyAsync(h->w_gu_alpha, wts.w_gu_alpha, sizeof(float) * Ew, cudaMemcpyDeviceToDevice, s));
+    CREATE_TRY(cudaMemcpyAsync(h->w_d_alpha, wts.w_d_alpha, sizeof(float) * Ew, cudaMemcpyDeviceToDevice, s));
   }
   CREATE_TRY(cudaMemcpyAsync(h->gamma, wts.gamma, sizeof(uint16_t) * H, cudaMemcpyDeviceToDevice, s));
   if (mx) {
-    CREATE_TRY(launch_repack_tiles_mx(wts.w_gu, wts.w_gu_sf, E, 2 * I, H, I, h->w_gu_tiles, s));
-    CREATE_TRY(launch_repack_tiles_mx(wts.w_d, wts.w_d_sf, E, H, I, 0, h->w_d_tiles, s));
+    CREATE_TRY(launch_repack_tiles_mx(wts.w_gu, wts.w_gu_sf, Ew, 2 * I, H, I, h->w_gu_tiles, s));
+    CREATE_TRY(launch_repack_tiles_mx(wts.w_d, wts.w_d_sf, Ew, H, I, 0, h->w_d_tiles, s));
   } else {
-    CREATE_TRY(launch_repack_tiles(wts.w_gu, wts.w_gu_sf, E, 2 * I, H, H, I, h->w_gu_tiles, s));
-    CREATE_TRY(launch_repack_tiles(wts.w_d, wts.w_d_sf, E, H, I, Ip, 0, h->w_d_tiles, s));
+    CREATE_TRY(launch_repack_tiles(wts.w_gu, wts.w_gu_sf, Ew, 2 * I, H, H, I, h->w_gu_tiles, s));
+    CREATE_TRY(launch_repack_tiles(wts.w_d, wts.w_d_sf, Ew, H, I, Ip, 0, h->w_d_tiles, s));
   }
 
   // ---- workspace
@@ -350,6 +365,24 @@ beam_moe_status beam_moe_create_mxfp8(const beam_moe_config* cfg, const beam_moe
   return create_impl(cfg, in, BEAM_MOE_FMT_MXFP8, stream, out);
 }
 
+beam_moe_status beam_moe_create_ep(const beam_moe_config* cfg, const beam_moe_weights* wts, int32_t expert_begin,
+                                   int32_t expert_count, void* stream, beam_moe_t* out) {
+  if (!cfg || !wts || !out || expert_count < 1) return BEAM_MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const ExpertWeightsIn in{wts->router_w, wts->w_gu, wts->w_gu_sf, wts->w_d, wts->w_d_sf,
+                           wts->w_gu_alpha, wts->w_d_alpha, wts->gamma};
+  return create_impl(cfg, in, BEAM_MOE_FMT_NVFP4, stream, out, expert_begin, expert_count);
+}
+
+beam_moe_status beam_moe_create_ep_mxfp8(const beam_moe_config* cfg, const beam_moe_weights_mxfp8* wts,
+                                         int32_t expert_begin, int32_t expert_count, void* stream, beam_moe_t* out) {
+  if (!cfg || !wts || !out || expert_count < 1) return BEAM_MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const ExpertWeightsIn in{wts->router_w, wts->w_gu, wts->w_gu_sf, wts->w_d, wts->w_d_sf, nullptr, nullptr,
+                           wts->gamma};
+  return create_impl(cfg, in, BEAM_MOE_FMT_MXFP8, stream, out, expert_begin, expert_count);
+}
+
 int32_t beam_moe_expert_format(beam_moe_t h) { return h ? h->fmt : -1; }
 
 beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num_tokens, int32_t hidden,
@@ -375,11 +408,15 @@ beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num
 // (tp_reduce) of the last phase 0.
 static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* residual, void* out, void* next_x,
                                     const void* next_gamma, float next_eps, int32_t num_tokens, void* stream,
-                                    int tp_phase = -1, cudaEvent_t residual_ready = nullptr) {
+                                    int tp_phase = -1, cudaEvent_t residual_ready = nullptr, int tok_off = 0,
+                                    bool ep_gathered = false) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;
+  if (tp_phase < 0 && h->ep) return BEAM_MOE_ERR_INVALID_ARG;  // holds only some experts: beam_moe_forward_ep
   if (tp_phase >= 0) {
     if (!h->tp_attached) return BEAM_MOE_ERR_INVALID_ARG;
-    if (tp_phase == 1 && (!h->tp_pending || num_tokens != h->tp_last_T)) return BEAM_MOE_ERR_INVALID_ARG;
+    if (tp_phase == 1 && (!h->tp_pending || tok_off < 0 || tok_off + num_tokens > h->tp_last_T ||
+                          (!h->ep && num_tokens != h->tp_last_T)))
+      return BEAM_MOE_ERR_INVALID_ARG;
     if (tp_phase == 0 && h->tp_pending) return BEAM_MOE_ERR_INVALID_ARG;  // phases must alternate
   }
   if (num_tokens < 0 || num_tokens > h->Tmax) return BEAM_MOE_ERR_INVALID_ARG;
@@ -404,7 +441,7 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   };
   if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
   if (tp_phase == 1) {
-    BEAM_TRY(launch_tp_reduce(static_cast<const uint16_t*>(residual), h->gamma, T, H, h->cfg.rms_eps, h->tp,
+    BEAM_TRY(launch_tp_reduce(static_cast<const uint16_t*>(residual), h->gamma, T, tok_off, H, h->cfg.rms_eps, h->tp,
                               h->tp_epoch, static_cast<uint16_t*>(out), h->err, s));
     BEAM_TRY(mark("tp_reduce"));
     ++launches;
@@ -413,7 +450,13 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     h->profiled_last = prof;
     return BEAM_MOE_OK;
   }
-  const BlockScales bscales{h->w_gu_alpha, h->w_d_alpha, h->cfg.alpha_a1, h->cfg.alpha_a2};
+  const BlockScales bscales{h->w_gu_alpha, h->w_d_alpha, h->cfg.alpha_a1, h->cfg.alpha_a2, h->e_begin,
+                            h->e_begin + h->e_count};
+  if (ep_gathered) {  // x is the gathered-token buffer: wait until every rank delivered
+    BEAM_TRY(launch_ep_wait(h->tp, h->tp_epoch + 1, h->err, s));
+    BEAM_TRY(mark("ep_wait"));
+    ++launches;
+  }
   // CTA pairs for the expert GEMM when the average expert has a few hundred rows
   const bool mx = h->fmt == BEAM_MOE_FMT_MXFP8;
   const bool pair = !mx && !route_small_supported(T, H, E, k) &&
@@ -494,7 +537,8 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   BEAM_TRY(mark("gemm_experts"));
   ++launches;
   if (tp_phase == 0) {
-    BEAM_TRY(launch_tp_partial(h->y, h->w, h->inv, T, H, k, h->tp, h->tp_epoch + 1, h->tp_counter, s));
+    BEAM_TRY(launch_tp_partial(h->y, h->w, h->inv, h->ids, h->e_begin, h->e_begin + h->e_count, T, H, k, h->tp,
+                               h->tp_epoch + 1, h->tp_counter, s));
     BEAM_TRY(mark("tp_partial"));
     ++launches;
     ++h->tp_epoch;
@@ -532,7 +576,9 @@ beam_moe_status beam_moe_forward_prenorm(beam_moe_t h, const void* x, const void
 
 int64_t beam_moe_tp_region_bytes(beam_moe_t h) {
   if (!h) return 0;
-  return static_cast<int64_t>(kTpHeaderBytes) + 2ll * h->Tmax * h->H * static_cast<int64_t>(sizeof(float));
+  const int64_t part = 2ll * h->Tmax * h->H * static_cast<int64_t>(sizeof(float));
+  const int64_t gathered = h->ep ? 2ll * h->Tmax * h->H * static_cast<int64_t>(sizeof(uint16_t)) : 0;
+  return static_cast<int64_t>(kTpHeaderBytes) + part + gathered;
 }
 
 beam_moe_status beam_moe_tp_region(beam_moe_t h, void** region) {
@@ -542,6 +588,8 @@ beam_moe_status beam_moe_tp_region(beam_moe_t h, void** region) {
     BEAM_TRY(dalloc(h, &h->tp_region, bytes));
     BEAM_TRY(dalloc(h, &h->tp_counter, sizeof(unsigned int)));
     BEAM_TRY(dalloc(h, &h->tp_regions_dev, sizeof(uint8_t*) * kMaxTpRanks));
+    BEAM_TRY(dalloc(h, &h->ep_counter, sizeof(unsigned int)));
+    BEAM_TRY(cudaMemset(h->ep_counter, 0, sizeof(unsigned int)));
     BEAM_TRY(cudaMemset(h->tp_region, 0, kTpHeaderBytes));
     BEAM_TRY(cudaMemset(h->tp_counter, 0, sizeof(unsigned int)));
   }
@@ -569,13 +617,56 @@ beam_moe_status beam_moe_tp_attach(beam_moe_t h, int32_t rank, int32_t world, vo
   h->tp = g;
   h->tp_epoch = 0;
   h->tp_pending = false;
+  h->ep_dispatched = false;
   h->tp_attached = true;
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_forward_ep_phase(beam_moe_t h, const void* x, const void* residual, void* out,
+                                          int32_t num_tokens, int32_t phase, void* stream) {
+  if (!h || !h->ep || !h->tp_attached || phase < 0 || phase > 2) return BEAM_MOE_ERR_INVALID_ARG;
+  if (num_tokens <= 0 || static_cast<int64_t>(num_tokens) * h->tp.world > h->Tmax) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!x || !residual || !out || !aligned(x, 16) || !aligned(residual, 16) || !aligned(out, 16))
+    return BEAM_MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint32_t epoch = h->tp_epoch + 1;  // the forward in flight (published by phases 0 and 1)
+  const size_t x_off = kTpHeaderBytes + 2 * static_cast<size_t>(h->Tmax) * h->H * sizeof(float);
+  if (phase == 0) {
+    if (h->ep_dispatched || h->tp_pending) return BEAM_MOE_ERR_INVALID_ARG;  // phases run 0, 1, 2 in turn
+    BEAM_TRY(launch_ep_dispatch(static_cast<const uint16_t*>(x), num_tokens, h->H, h->tp, x_off, epoch,
+                                h->ep_counter, s));
+    h->ep_dispatched = true;
+    h->ep_T = num_tokens;
+    h->last_launches = 1;
+    h->profiled_last = false;
+    return BEAM_MOE_OK;
+  }
+  if (phase == 1) {
+    if (!h->ep_dispatched || num_tokens != h->ep_T) return BEAM_MOE_ERR_INVALID_ARG;
+    const uint16_t* gathered = reinterpret_cast<const uint16_t*>(h->tp_region + x_off) +
+                               static_cast<size_t>(epoch & 1u) * h->Tmax * h->H;
+    h->ep_dispatched = false;
+    return forward_impl(h, gathered, residual, out, nullptr, nullptr, 0.0f, num_tokens * h->tp.world, stream, 0,
+                        nullptr, 0, true);
+  }
+  if (num_tokens != h->ep_T) return BEAM_MOE_ERR_INVALID_ARG;
+  return forward_impl(h, x, residual, out, nullptr, nullptr, 0.0f, num_tokens, stream, 1, nullptr,
+                      h->tp.rank * num_tokens);
+}
+
+beam_moe_status beam_moe_forward_ep(beam_moe_t h, const void* x, const void* residual, void* out,
+                                    int32_t num_tokens, void* stream) {
+  for (int phase = 0; phase < 3; ++phase) {
+    beam_moe_status st = beam_moe_forward_ep_phase(h, x, residual, out, num_tokens, phase, stream);
+    if (st != BEAM_MOE_OK) return st;
+  }
   return BEAM_MOE_OK;
 }
 
 beam_moe_status beam_moe_forward_tp_phase(beam_moe_t h, const void* x, const void* residual, void* out,
                                           int32_t num_tokens, int32_t phase, void* stream) {
   if (phase != 0 && phase != 1) return BEAM_MOE_ERR_INVALID_ARG;
+  if (h && h->ep) return BEAM_MOE_ERR_INVALID_ARG;  // expert-parallel handles: beam_moe_forward_ep
   if (!h || num_tokens <= 0) return num_tokens == 0 && h ? BEAM_MOE_OK : BEAM_MOE_ERR_INVALID_ARG;
   if (phase == 1 && (!residual || !out || !aligned(residual, 16) || !aligned(out, 16)))
     return BEAM_MOE_ERR_INVALID_ARG;

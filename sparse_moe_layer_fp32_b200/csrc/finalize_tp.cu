@@ -70,8 +70,9 @@ __device__ __forceinline__ uint32_t* tp_flags(uint8_t* region) { return reinterp
 
 __global__ void __launch_bounds__(kTpMaxThreads) tp_partial_kernel(const uint16_t* __restrict__ y,
                                                                    const float* __restrict__ w,
-                                                                   const int32_t* __restrict__ inv, int H, int k,
-                                                                   TpGroup g, uint32_t epoch,
+                                                                   const int32_t* __restrict__ inv,
+                                                                   const int32_t* __restrict__ ids, int e_begin,
+                                                                   int e_end, int H, int k, TpGroup g, uint32_t epoch,
                                                                    uint32_t* __restrict__ counter) {
   __shared__ int s_row[kTpMaxK];
   __shared__ float s_w[kTpMaxK];
@@ -79,8 +80,13 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_partial_kernel(const uint16_
   pdl_wait();
   pdl_trigger();
   if (threadIdx.x < k) {
-    s_row[threadIdx.x] = inv[static_cast<size_t>(t) * k + threadIdx.x];
-    s_w[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
+    // a slot whose expert this rank does not hold contributes nothing here (weight 0, any
+    // valid row: its y row is not written by this rank)
+    const size_t i = static_cast<size_t>(t) * k + threadIdx.x;
+    const int e = ids[i];
+    const bool held = e >= e_begin && e < e_end;
+    s_row[threadIdx.x] = held ? inv[i] : 0;
+    s_w[threadIdx.x] = held ? w[i] : 0.0f;
   }
   __syncthreads();
   float* part = tp_part(g.own, static_cast<int>(epoch & 1u), g.buf_floats) + static_cast<size_t>(t) * H;
@@ -94,11 +100,11 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_partial_kernel(const uint16_
                            : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float wj = j0 + j < k ? s_w[j0 + j] : 0.0f;
+        if (j0 + j >= k || s_w[j0 + j] == 0.0f) continue;  // unheld slots: the row may hold anything
         float f[8];
         unpack8_bf16(yv[j], f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(s_w[j0 + j], f[i], acc[i]);
       }
     }
     reinterpret_cast<float4*>(part)[2 * c] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -118,9 +124,9 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_partial_kernel(const uint16_
 }
 
 __global__ void __launch_bounds__(kTpMaxThreads) tp_reduce_kernel(const uint16_t* residual,
-                                                                  const uint16_t* __restrict__ gamma, int H,
-                                                                  float eps, TpGroup g, uint32_t epoch, uint16_t* out,
-                                                                  uint32_t* err) {
+                                                                  const uint16_t* __restrict__ gamma, int tok_off,
+                                                                  int H, float eps, TpGroup g, uint32_t epoch,
+                                                                  uint16_t* out, uint32_t* err) {
   extern __shared__ float m_s[];  // [H]
   __shared__ float s_red[kTpMaxThreads / 32];
   __shared__ const float* s_part[kMaxTpRanks];  // this token's row in every rank's buffer
@@ -130,7 +136,7 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_reduce_kernel(const uint16_t
   pdl_wait();
   pdl_trigger();
   if (threadIdx.x < g.world)
-    s_part[threadIdx.x] = tp_part(g.regions[threadIdx.x], buf, g.buf_floats) + static_cast<size_t>(t) * H;
+    s_part[threadIdx.x] = tp_part(g.regions[threadIdx.x], buf, g.buf_floats) + static_cast<size_t>(tok_off + t) * H;
   if (threadIdx.x == 0) s_ok = 1;
   __syncthreads();
   if (threadIdx.x < g.world) {  // thread q waits for rank q's flag
@@ -198,12 +204,14 @@ static int tp_threads(int H) {
   return want < kTpMaxThreads ? want : kTpMaxThreads;
 }
 
-cudaError_t launch_tp_partial(const uint16_t* y, const float* w, const int32_t* inv, int T, int H, int k,
-                              const TpGroup& g, uint32_t epoch, unsigned int* counter, cudaStream_t s) {
-  return launch_pdl(tp_partial_kernel, dim3(T), dim3(tp_threads(H)), 0, s, y, w, inv, H, k, g, epoch, counter);
+cudaError_t launch_tp_partial(const uint16_t* y, const float* w, const int32_t* inv, const int32_t* ids, int e_begin,
+                              int e_end, int T, int H, int k, const TpGroup& g, uint32_t epoch, unsigned int* counter,
+                              cudaStream_t s) {
+  return launch_pdl(tp_partial_kernel, dim3(T), dim3(tp_threads(H)), 0, s, y, w, inv, ids, e_begin, e_end, H, k, g,
+                    epoch, counter);
 }
 
-cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, int H, float eps,
+cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, int tok_off, int H, float eps,
                              const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(H) * sizeof(float);
   if (smem > 48 * 1024) {
@@ -211,8 +219,67 @@ cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, in
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(tp_reduce_kernel, dim3(T), dim3(tp_threads(H)), smem, s, residual, gamma, H, eps, g, epoch, out,
-                    err);
+  return launch_pdl(tp_reduce_kernel, dim3(T), dim3(tp_threads(H)), smem, s, residual, gamma, tok_off, H, eps, g,
+                    epoch, out, err);
+}
+
+// ------------------------------------------------------------------ expert parallel
+// Dispatch by all-gather: CTA t copies token t's row (16-byte chunks) into row rank T + t of
+// every rank's gathered buffer (peer stores over NVLink), then the same arrival / publish
+// as tp_partial, into the delivery slots.
+__global__ void __launch_bounds__(kTpMaxThreads) ep_dispatch_kernel(const uint16_t* __restrict__ x, int T, int H,
+                                                                    TpGroup g, size_t x_offset, uint32_t epoch,
+                                                                    uint32_t* __restrict__ counter) {
+  __shared__ uint16_t* s_dst[kMaxTpRanks];
+  const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  // buffer (epoch & 1) of g.buf_floats elements ([max_tokens][H]), row rank T + t
+  if (threadIdx.x < g.world)
+    s_dst[threadIdx.x] = reinterpret_cast<uint16_t*>(g.regions[threadIdx.x] + x_offset) +
+                         static_cast<size_t>(epoch & 1u) * g.buf_floats +
+                         (static_cast<size_t>(g.rank) * T + t) * static_cast<size_t>(H);
+  __syncthreads();
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    const uint4 v = __ldg(src + c);
+    for (int q = 0; q < g.world; ++q) reinterpret_cast<uint4*>(s_dst[q])[c] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t done = atom_add_acq_rel_gpu(counter, 1u);
+    if (done == gridDim.x - 1) {
+      *counter = 0u;
+      for (int q = 0; q < g.world; ++q) st_release_sys(tp_flags(g.regions[q]) + kMaxTpRanks + g.rank, epoch);
+    }
+  }
+}
+
+// Waits (bounded) until every rank delivered this epoch's tokens.  It never triggers its
+// dependents early: the kernels after it (which read the gathered tokens, some before their
+// own grid-dependency wait) start only once it has ended.
+__global__ void ep_wait_kernel(TpGroup g, uint32_t epoch, uint32_t* err) {
+  pdl_wait();
+  if (threadIdx.x < g.world) {
+    const uint32_t* flag = tp_flags(g.own) + kMaxTpRanks + threadIdx.x;
+    const uint64_t t0 = globaltimer_ns();
+    while (static_cast<int32_t>(ld_acquire_sys(flag) - epoch) < 0) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(err, kErrTimeoutEpilogue);
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+}
+
+cudaError_t launch_ep_dispatch(const uint16_t* x, int T, int H, const TpGroup& g, size_t x_offset, uint32_t epoch,
+                               unsigned int* counter, cudaStream_t s) {
+  return launch_pdl(ep_dispatch_kernel, dim3(T), dim3(tp_threads(H)), 0, s, x, T, H, g, x_offset, epoch, counter);
+}
+
+cudaError_t launch_ep_wait(const TpGroup& g, uint32_t epoch, uint32_t* err, cudaStream_t s) {
+  return launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s, g, epoch, err);
 }
 
 }  // namespace beam

@@ -19,11 +19,15 @@ struct alignas(32) MBlock {
   float scale_d;      // alpha_a2 * alpha_d[expert]: dequantisation of the down accumulators
   int32_t pad[2];
 };
-// What the block-list builders need to fill MBlock::scale_gu / scale_d.
+// What the block-list builders need: the experts whose weights this handle holds (all of
+// them, or one expert-parallel rank's range [e_begin, e_end); blocks of other experts are
+// left out of the work list, their rows keep their places in the activations), and what
+// fills MBlock::scale_gu / scale_d.  MBlock::expert is the index within the range.
 struct BlockScales {
-  const float* w_gu_alpha;  // [E]
-  const float* w_d_alpha;   // [E]
+  const float* w_gu_alpha;  // [e_end - e_begin]
+  const float* w_d_alpha;   // [e_end - e_begin]
   float alpha_a1, alpha_a2;
+  int e_begin, e_end;
 };
 
 constexpr int kChunkTokens = 256;  // tokens per histogram / scatter chunk
@@ -141,9 +145,11 @@ cudaError_t launch_gemm_experts_mx(const ExpertGemmArgs& a, int grid, cudaStream
 constexpr int kPairMinTokens = BEAM_MOE_PAIR_MIN_TOKENS;
 cudaError_t launch_gemm_experts_pair(const ExpertGemmArgs& a, int grid, cudaStream_t s);
 
-// ---- tensor-parallel finalize fused with its all-reduce (finalize_tp.cu)
+// ---- tensor / expert parallel finalize fused with its all-reduce (finalize_tp.cu)
 // Exchange region of one rank: kTpHeaderBytes of flags (u32 slot q = the last epoch rank q
-// published), then two buffers of [max_tokens][H] FP32 partial m (epoch parity).
+// published its partial m; slot kMaxTpRanks + q = the last epoch rank q delivered its
+// tokens), two buffers of [max_tokens][H] FP32 partial m (epoch parity), and for expert
+// parallelism two buffers of [max_tokens][H] BF16 gathered tokens.
 constexpr int kMaxTpRanks = 16;
 constexpr size_t kTpHeaderBytes = 1024;
 struct TpGroup {
@@ -152,10 +158,20 @@ struct TpGroup {
   int rank, world;
   size_t buf_floats;        // floats per partial buffer: max_tokens * H
 };
-cudaError_t launch_tp_partial(const uint16_t* y, const float* w, const int32_t* inv, int T, int H, int k,
-                              const TpGroup& g, uint32_t epoch, unsigned int* counter, cudaStream_t s);
-cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, int H, float eps,
+// Partial m over the slots whose expert lies in [e_begin, e_end) (all of them under TP).
+cudaError_t launch_tp_partial(const uint16_t* y, const float* w, const int32_t* inv, const int32_t* ids, int e_begin,
+                              int e_end, int T, int H, int k, const TpGroup& g, uint32_t epoch, unsigned int* counter,
+                              cudaStream_t s);
+// out[t] for t < T from partial rows tok_off + t (tok_off = 0 under TP).
+cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, int tok_off, int H, float eps,
                              const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, cudaStream_t s);
+// Expert parallelism: this rank's T tokens into rows [rank T, rank T + T) of every rank's
+// gathered-token buffer (x_offset: its byte offset in a region; buffer epoch & 1), then the
+// delivery flag; and the wait for every rank's delivery (one CTA that lets its dependents
+// start only when it ends).
+cudaError_t launch_ep_dispatch(const uint16_t* x, int T, int H, const TpGroup& g, size_t x_offset, uint32_t epoch,
+                               unsigned int* counter, cudaStream_t s);
+cudaError_t launch_ep_wait(const TpGroup& g, uint32_t epoch, uint32_t* err, cudaStream_t s);
 
 // ---- finalize (finalize.cu)
 // next_x != nullptr also writes the next sublayer's pre-norm of out: bf16(out * rinv * next_gamma).

@@ -180,30 +180,32 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
   // ---------------------------------------------------------------- scan and work blocks
   const int cnt = tid < E ? s_cnt[tid] : 0;
   const int nblk = (cnt + 127) / 128;
-  int total_rows, total_blk;
+  const bool held = tid >= bs.e_begin && tid < bs.e_end;  // this handle has the expert's weights
+  int total_rows, total_blk, total_work;
   const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
   const int blk = block_exclusive_scan(nblk, warp_sums, total_blk);
+  const int wbase = block_exclusive_scan(held ? nblk : 0, warp_sums, total_work);
   if (tid < E) {
     offsets[tid] = off;
     sf_block[tid] = blk;
     s_off[tid] = off;
     s_blk[tid] = blk;
-    for (int i = 0; i < nblk; ++i) {
+    for (int i = 0; held && i < nblk; ++i) {
       MBlock m;
-      m.expert = tid;
+      m.expert = tid - bs.e_begin;
       m.row_begin = off + 128 * i;
       m.rows = min(128, cnt - 128 * i);
       m.sf_block = blk + i;
-      m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + tid);
-      m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + tid);
+      m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + m.expert);
+      m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + m.expert);
       m.pad[0] = m.pad[1] = 0;
-      mblocks[blk + i] = m;
+      mblocks[wbase + i] = m;
     }
   }
   if (tid == 0) {
     offsets[E] = total_rows;
     sf_block[E] = total_blk;
-    *num_mblocks = total_blk;
+    *num_mblocks = total_work;
   }
   __syncthreads();
   // ---------------------------------------------------------------- permutation

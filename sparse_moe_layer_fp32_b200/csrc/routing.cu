@@ -63,7 +63,8 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
   // CTA pair computes each tile.
   const int nblk = (cnt + 127) / 128;
   const int wrows = pair ? 256 : 128;
-  const int nwork = (cnt + wrows - 1) / wrows;
+  const bool held = e >= bs.e_begin && e < bs.e_end;  // this handle has the expert's weights
+  const int nwork = held ? (cnt + wrows - 1) / wrows : 0;
   int total_rows, total_blk, total_work;
   const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
   const int blk = block_exclusive_scan(nblk, warp_sums, total_blk);
@@ -74,12 +75,12 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
     for (int c = 0; c < n_chunks; ++c) chunk_base[static_cast<size_t>(c) * E + e] += off;
     for (int i = 0; i < nwork; ++i) {
       MBlock m;
-      m.expert = e;
+      m.expert = e - bs.e_begin;
       m.row_begin = off + wrows * i;
       m.rows = min(wrows, cnt - wrows * i);
       m.sf_block = blk + (wrows / 128) * i;
-      m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + e);
-      m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + e);
+      m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + m.expert);
+      m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + m.expert);
       m.pad[0] = m.pad[1] = 0;
       mblocks[wbase + i] = m;
     }

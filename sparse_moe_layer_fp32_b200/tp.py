@@ -1,12 +1,14 @@
-"""Host side of the tensor-parallel layer: weight shards, the exchange of the ranks' regions,
-and ranks that share one GPU.
+"""Host side of the tensor- and expert-parallel layers: weight shards, the exchange of the
+ranks' regions, and ranks that share one GPU.
 
 Tensor parallelism over the experts' intermediate size with the finalize fused to its
 all-reduce (vLLM PR "Day-0 support for Reflection's Beam-1.0", section "Status"; recipe
 "reflection/Beam-1.0-501B-A23B": NVFP4 with TP4 on Blackwell).  Rank r holds features
 [r I/W, (r+1) I/W) of every expert: those gate rows, the matching up rows and the same
-columns of down.  The device work is beam_moe_forward_tp (C ABI); this module only slices
-tensors and moves region addresses between processes.
+columns of down.  Expert parallelism with attention data parallelism (the PR's Attention DP
++ MegaMoE): rank r holds experts [r E/W, (r+1) E/W) and its own batch.  The device work is
+beam_moe_forward_tp / beam_moe_forward_ep (C ABI); this module only slices tensors and moves
+region addresses between processes.
 """
 
 from __future__ import annotations
@@ -44,6 +46,23 @@ def shard_weights(weights: dict, rank: int, world: int, inter: int) -> dict:
     return out
 
 
+def shard_experts(weights: dict, rank: int, world: int, num_experts: int) -> dict:
+    """Expert parallelism: this rank's experts [r E/W, (r+1) E/W) of layer weights in the C-ABI
+    layout (either format): the expert-major arrays sliced along their first dimension,
+    router weights and gamma unchanged."""
+    if world < 1 or not 0 <= rank < world or num_experts % world:
+        raise ValueError(f"cannot take expert shard {rank} of {world} of {num_experts} experts")
+    e = num_experts // world
+    out = dict(weights)
+    for key in WEIGHT_KEYS + ("w_gu_alpha", "w_d_alpha"):
+        if key in weights:
+            t = weights[key]
+            if t.shape[0] != num_experts:
+                raise ValueError(f"{key} must have num_experts rows")
+            out[key] = t[rank * e:(rank + 1) * e].contiguous()
+    return out
+
+
 def _cat_rows(a, b):
     import torch
     return torch.cat([a, b], dim=1).contiguous()
@@ -74,19 +93,32 @@ def connect(layer: MoELayer, rank: int, world: int, group=None, export=None, imp
 
 
 class SharedGpuGroup:
-    """W ranks of one tensor-parallel group in one process on one GPU (tests and
+    """W ranks of one tensor- or expert-parallel group in one process on one GPU (tests and
     measurement when fewer GPUs than ranks are available).  The ranks run one after the
-    other: every rank's phase 0 (GEMMs, partial m, publication), then every rank's phase 1
-    (all-reduce + finalize), so no kernel waits on a kernel that has not run."""
+    other, phase by phase: every rank's phase p before any rank's phase p + 1, so no kernel
+    waits on a kernel that has not run.  Tensor parallel: phase 0 (GEMMs, partial m,
+    publication), phase 1 (all-reduce + finalize); every rank gets the same x.  Expert
+    parallel (layers created with an expert range): phase 0 (dispatch), 1 (routing of the
+    gathered batch, the rank's experts, partial m), 2 (combine + finalize); each rank its own
+    x and residual."""
 
     def __init__(self, layers):
         self.layers = list(layers)
+        self.expert_parallel = bool(getattr(self.layers[0], "expert_parallel", False))
         regions = [lay.tp_region() for lay in self.layers]
         for r, lay in enumerate(self.layers):
             lay.tp_attach(r, len(self.layers), regions)
 
     def forward(self, x, residual, outs=None):
+        """Tensor parallel: x, residual tensors (the same on every rank).  Expert parallel:
+        lists of each rank's x and residual."""
         import torch
+        if self.expert_parallel:
+            outs = outs or [torch.empty_like(r) for r in residual]
+            for phase in range(3):
+                for lay, xr, rr, o in zip(self.layers, x, residual, outs):
+                    lay.forward_ep_phase(xr, rr, o, phase)
+            return outs
         outs = outs or [torch.empty_like(residual) for _ in self.layers]
         for lay, o in zip(self.layers, outs):
             lay.forward_tp_phase(x, residual, o, 0)

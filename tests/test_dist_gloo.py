@@ -145,3 +145,21 @@ def test_tp_shard_weights_partition_the_experts():
         tp.shard_weights(full, 0, 3, inter)
     with pytest.raises(ValueError):
         tp.shard_weights(full, 4, 4, inter)
+
+
+def test_ep_shard_experts_partition_the_expert_arrays():
+    from sparse_moe_layer_fp32_b200 import tp
+    E, H, inter, world = 8, 64, 128, 4
+    g = torch.Generator().manual_seed(1)
+    full = dict(router_w=torch.randn(E, H, generator=g), gamma=torch.ones(H),
+                w_gu=torch.randint(0, 255, (E, 2 * inter, H), dtype=torch.uint8, generator=g),
+                w_gu_sf=torch.randint(0, 255, (E, 2 * inter, H // 32), dtype=torch.uint8, generator=g),
+                w_d=torch.randint(0, 255, (E, H, inter), dtype=torch.uint8, generator=g),
+                w_d_sf=torch.randint(0, 255, (E, H, inter // 32), dtype=torch.uint8, generator=g))
+    shards = [tp.shard_experts(full, r, world, E) for r in range(world)]
+    for key in ("w_gu", "w_gu_sf", "w_d", "w_d_sf"):
+        assert torch.equal(torch.cat([sh[key] for sh in shards]), full[key])
+        assert all(sh[key].shape[0] == E // world and sh[key].is_contiguous() for sh in shards)
+    assert all(sh["router_w"] is full["router_w"] and sh["gamma"] is full["gamma"] for sh in shards)
+    with pytest.raises(ValueError):
+        tp.shard_experts(full, 0, 3, E)
