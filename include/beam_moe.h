@@ -329,6 +329,20 @@ enum { BEAM_MOE_GEMM_AUTO = 0, BEAM_MOE_GEMM_SINGLE = 1, BEAM_MOE_GEMM_PAIR = 2 
 #define BEAM_MOE_PAIR_MIN_TOKENS 2147483647
 BEAM_MOE_API beam_moe_status beam_moe_set_gemm_mode(beam_moe_t h, int32_t mode);
 
+/* Router for batches of more than 16 tokens (16 or fewer use the fused small-batch routing
+ * kernel).  SIMT: FP32 FFMA over slices of H, then a top-k kernel that sums the slices.
+ * TENSOR: the tensor cores on the exact three-part BF16 split of the FP32 weights, over
+ * (128-token tiles) x (slices of H) with partial logits summed by the top-k kernel (about
+ * one wave of CTAs below 4096 tokens, two from there); once a single slice fills two waves
+ * (about 37,900 tokens on 148 SMs), one 256-token tile per CTA with the top-k in its
+ * epilogue.  AUTO (the default) is TENSOR from BEAM_MOE_ROUTER_TC_SPLIT_MIN_TOKENS tokens
+ * on.  All compute FP32-accurate logits and differ only in the order of the FP32 additions.
+ * Not from the source pages: an implementation choice exposed for testing and tuning.
+ * Returns INVALID_ARG for an unknown mode. */
+enum { BEAM_MOE_ROUTER_AUTO = 0, BEAM_MOE_ROUTER_SIMT = 1, BEAM_MOE_ROUTER_TENSOR = 2 };
+#define BEAM_MOE_ROUTER_TC_SPLIT_MIN_TOKENS 17
+BEAM_MOE_API beam_moe_status beam_moe_set_router_mode(beam_moe_t h, int32_t mode);
+
 /* Per-kernel timing.  While enabled (enable != 0), beam_moe_forward records a CUDA event
  * on `stream` before its first kernel and after each kernel it enqueues.  Creating the
  * events is the only allocation; enable once, outside any timed region. */

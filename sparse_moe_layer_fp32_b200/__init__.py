@@ -29,7 +29,7 @@ EXPORTED = [
     "beam_moe_expert_format", "beam_moe_tp_region_bytes", "beam_moe_tp_region", "beam_moe_tp_attach",
     "beam_moe_forward_tp", "beam_moe_forward_tp_phase", "beam_moe_ipc_export", "beam_moe_ipc_import",
     "beam_moe_ipc_close", "beam_moe_create_ep", "beam_moe_create_ep_mxfp8", "beam_moe_forward_ep",
-    "beam_moe_forward_ep_phase",
+    "beam_moe_forward_ep_phase", "beam_moe_set_router_mode",
 ]
 IPC_HANDLE_BYTES = 64
 FMT_NVFP4, FMT_MXFP8 = 0, 1
@@ -78,6 +78,7 @@ def _load():
         "beam_moe_destroy": (None, [vp]),
         "beam_moe_profile_enable": (i32, [vp, i32]),
         "beam_moe_set_gemm_mode": (i32, [vp, i32]),
+        "beam_moe_set_router_mode": (i32, [vp, i32]),
         "beam_moe_profile_read": (i32, [vp, ctypes.POINTER(f32), i32, ctypes.POINTER(i32)]),
         "beam_moe_kernel_name": (ctypes.c_char_p, [vp, i32]),
         "beam_moe_route_static": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
@@ -298,6 +299,13 @@ def beam_moe_debug_wait_timeout(h, limit_ns: int, stream=None):
 GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
 
 
+ROUTER_AUTO, ROUTER_SIMT, ROUTER_TENSOR = 0, 1, 2
+
+
+def beam_moe_set_router_mode(h, mode: int):
+    _check(_lib.beam_moe_set_router_mode(h, int(mode)), "beam_moe_set_router_mode")
+
+
 def beam_moe_set_gemm_mode(h, mode: int):
     _check(_lib.beam_moe_set_gemm_mode(h, int(mode)), "beam_moe_set_gemm_mode")
 
@@ -399,6 +407,9 @@ class MoELayer:
     def forward_ep_phase(self, x, residual, out, phase: int, stream=None):
         beam_moe_forward_ep_phase(self.handle, x, residual, out, x.shape[0], phase, stream)
         return out
+
+    def set_router_mode(self, mode: int):
+        beam_moe_set_router_mode(self.handle, mode)
 
     def set_gemm_mode(self, mode: int):
         beam_moe_set_gemm_mode(self.handle, mode)

@@ -37,6 +37,7 @@ struct beam_moe_ctx {
   unsigned int* route_counter;  // last-CTA election of the fused small-batch routing kernel
   uint32_t* sched;              // tile scheduler of the expert GEMM launch (sched_words(nblk_max))
   int32_t gemm_mode;            // BEAM_MOE_GEMM_*: which expert GEMM large batches use
+  int32_t router_mode;          // BEAM_MOE_ROUTER_*: which router batches of more than 16 tokens use
   int32_t fmt;                  // BEAM_MOE_FMT_*: expert weight and activation format
   int kv;                       // K values per activation / weight tile: 256 (NVFP4), 128 (MXFP8)
   int sfa_tile;                 // scale bytes per 128-row block per K tile: 2048 (NVFP4), 512
@@ -241,6 +242,7 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   h->last_launches = 0;
   h->profiling = false;
   h->gemm_mode = BEAM_MOE_GEMM_AUTO;
+  h->router_mode = BEAM_MOE_ROUTER_AUTO;
   h->profiled_last = false;
   for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i) {
     h->events[i] = nullptr;
@@ -300,6 +302,9 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   int64_t lf = 0;
   for (int T = 1; T <= h->Tmax; T = (T < 64 ? T + 1 : T + 64)) lf = std::max(lf, route_ws_floats(T, H, E));
   lf = std::max(lf, route_ws_floats(h->Tmax, H, E));
+  // the tensor-core router's partial logits: [splits][T][E] (every T: the split count steps)
+  for (int T = 1; T <= h->Tmax; ++T)
+    lf = std::max(lf, static_cast<int64_t>(router_tc_split_count(T, H, h->num_sms)) * T * E);
   for (int T = 1; T <= std::min(h->Tmax, kMaxSmallRouterTokens); ++T)
     if (route_small_supported(T, H, h->E, h->k)) lf = std::max(lf, route_small_ws_floats(T, H, h->E));
   h->logits_floats = lf;
@@ -471,7 +476,25 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     ++launches;
     h->last_splits = slices;
   } else {
-    if (router_tc_supported(T, H, E, k)) {
+    const bool simt_only = h->router_mode == BEAM_MOE_ROUTER_SIMT;
+    // AUTO and TENSOR: slices of H whenever the split count is above one (measured faster than
+    // one tile per CTA at every batch up to 32K tokens, and than the SIMT router from 17)
+    const bool tc_split = !simt_only && router_tc_split_supported(H, E, k) && T >= kRouterTcSplitMinTokens &&
+                          router_tc_split_count(T, H, h->num_sms) > 1;
+    if (tc_split) {
+      // tensor cores over (token tiles) x (slices of H), partial logits; the top-k kernel
+      // sums the slices in order
+      CUtensorMap map_x;
+      if (!make_map_bf16(&map_x, xb, H, T, 128u)) return BEAM_MOE_ERR_CUDA;
+      const int splits = router_tc_split_count(T, H, h->num_sms);
+      BEAM_TRY(launch_router_tc(map_x, 128, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s, splits));
+      BEAM_TRY(mark("router_tc"));
+      ++launches;
+      h->last_splits = splits;
+      BEAM_TRY(launch_topk(h->logits, splits, T, E, k, h->ids, h->w, s));
+      BEAM_TRY(mark("topk"));
+      ++launches;
+    } else if (!simt_only && router_tc_supported(T, H, E, k)) {
       // FP32-class logits on the tensor cores (BF16 x 3-part split), top-k in the epilogue
       CUtensorMap map_x;
       const int rt_tokens = router_tc_tokens_per_cta(T, h->num_sms);
@@ -811,6 +834,12 @@ beam_moe_status beam_moe_debug_wait_timeout(beam_moe_t h, int64_t limit_ns, void
   if (!h || limit_ns <= 0 || limit_ns > static_cast<int64_t>(kWaitLimitNs)) return BEAM_MOE_ERR_INVALID_ARG;
   wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns), h->err);
   BEAM_TRY(cudaGetLastError());
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_set_router_mode(beam_moe_t h, int32_t mode) {
+  if (!h || mode < BEAM_MOE_ROUTER_AUTO || mode > BEAM_MOE_ROUTER_TENSOR) return BEAM_MOE_ERR_INVALID_ARG;
+  h->router_mode = mode;
   return BEAM_MOE_OK;
 }
 

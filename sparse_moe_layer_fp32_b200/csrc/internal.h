@@ -45,6 +45,9 @@ cudaError_t launch_topk(const float* logits, int splits, int T, int E, int k, in
 // One CTA per 128 tokens, each streaming all of W_r: below ~32 CTAs the split-H SIMT
 // router (router.cu) fills more of the GPU and is faster (0.11 vs 0.32 ms at T = 1024).
 constexpr int kRouterTcMinTokens = 4096;
+// From this many tokens up to kRouterTcMinTokens the tensor-core router runs over
+// (token tiles) x (slices of H) with partial logits (BEAM_MOE_ROUTER_AUTO).
+constexpr int kRouterTcSplitMinTokens = BEAM_MOE_ROUTER_TC_SPLIT_MIN_TOKENS;
 bool router_tc_supported(int T, int H, int E, int k);
 size_t router_tc_smem_bytes(int E);
 cudaError_t launch_split_router(const float* w, int E, int H, uint16_t* out, cudaStream_t s);
@@ -52,8 +55,13 @@ cudaError_t launch_split_router(const float* w, int E, int H, uint16_t* out, cud
 // weights from launch_split_router.  Writes logits [T][E], ids / w [T][k].
 // Tokens per CTA (128 or 256) for a batch of T; also the row count of the x tensor map's box.
 int router_tc_tokens_per_cta(int T, int num_sms);
+// splits > 1 (128-token CTAs only): grid (token tiles) x (splits slices of H), partial
+// logits [splits][T][E] into `logits`, no top-k (launch_topk sums the slices and selects).
 cudaError_t launch_router_tc(const CUtensorMap& map_x, int tokens_per_cta, const uint16_t* w_tiles, int T, int H,
-                             int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s);
+                             int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s,
+                             int splits = 1);
+bool router_tc_split_supported(int H, int E, int k);
+int router_tc_split_count(int T, int H, int num_sms);
 
 // ---- routing of a small batch in one launch (route_small.cu)
 bool route_small_supported(int T, int H, int E, int k);

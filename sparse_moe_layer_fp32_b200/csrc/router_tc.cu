@@ -22,6 +22,11 @@
 // token's E logits from TMEM, keep a running top-k (larger logit first, equal logits ->
 // lower expert index), write the logits, the chosen ids and the renormalised weights
 // (softmax over the chosen logits = p_j / sum_chosen p).
+//
+// Batches below two waves of 128-token tiles would leave most SMs idle with every CTA
+// streaming all of W: there the grid is (token tiles) x (S slices of H), each CTA runs its
+// slice's K steps only and writes its FP32 partial logits to [S][T][E]; the top-k kernel of
+// the SIMT router then sums the S slices in order and selects.
 #include <algorithm>
 
 #include "common.cuh"
@@ -66,7 +71,7 @@ template <int HALVES>
 __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ w_tiles, int T,
                      int H, int E, int k, float* __restrict__ logits, int32_t* __restrict__ ids,
-                     float* __restrict__ wout, uint32_t* __restrict__ err) {
+                     float* __restrict__ wout, uint32_t* __restrict__ err, int splits) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int RT_BM = RtShape<HALVES>::BM, RT_STAGES = RtShape<HALVES>::STAGES, RT_A_BYTES = RtShape<HALVES>::A_BYTES;
@@ -95,11 +100,15 @@ __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
   pdl_wait();
   pdl_trigger();
   const int m0 = blockIdx.x * RT_BM;
-  const int k_tiles = H / RT_BK;
+  // this CTA's K steps: [k_lo, k_lo + k_tiles) of H / RT_BK (all of them when splits == 1)
+  const int k_all = H / RT_BK;
+  const int k_per = (k_all + splits - 1) / splits;
+  const int k_lo = static_cast<int>(blockIdx.y) * k_per;
+  const int k_tiles = max(0, min(k_per, k_all - k_lo));
   // Every CTA reads the same weight tiles; starting each CTA at a different K step keeps
   // them from all hitting the same L2 lines at once.  (Only the FP32 summation order
   // changes with the start.)
-  const int k_start = static_cast<int>(blockIdx.x % static_cast<unsigned>(k_tiles));
+  const int k_start = k_tiles > 0 ? static_cast<int>(blockIdx.x % static_cast<unsigned>(k_tiles)) : 0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -112,7 +121,7 @@ __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
         mbar_arrive_expect_tx(&tail->full[stage], static_cast<uint32_t>(stage_bytes));
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        const int kk = (kt + k_start) % k_tiles;
+        const int kk = k_lo + (kt + k_start) % k_tiles;
         tma_load_2d(sa, &map_x, &tail->full[stage], kk * RT_BK, m0);
         bulk_load(sa + RT_A_BYTES, w_tiles + static_cast<size_t>(kk) * 3 * E * 64, 3 * E * 64, &tail->full[stage]);
         if (++stage == RT_STAGES) {
@@ -154,6 +163,9 @@ __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
           phase ^= 1;
         }
       }
+      if (k_tiles == 0) {  // an empty slice (H not divisible into the splits): zero partials
+        // nothing was issued; the epilogue writes zeros for this slice
+      }
       tc_commit(&tail->acc_full);  // also fires after an abort, once the issued MMAs finish
       // every issued MMA has finished before TMEM can be freed (bounded)
       const uint64_t t0 = globaltimer_ns();
@@ -176,13 +188,18 @@ __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
     }
     float thr = -INFINITY;  // current k-th largest
     const uint32_t t_lane = tmem + half * tcols + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool partial = splits > 1;  // write this slice's partial logits only
     for (int c0 = 0; c0 < E; c0 += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(t_lane + c0, v);  // E % 16 == 0: columns past E are never used
       tmem_ld_wait();
       if (!ok || t >= T) continue;
+      if (k_tiles == 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0u;  // the accumulator was never written
+      }
       const int ncols = min(32, E - c0);
-      float* lrow = logits + static_cast<size_t>(t) * E + c0;
+      float* lrow = logits + (static_cast<size_t>(blockIdx.y) * T + t) * E + c0;
       if (ncols == 32) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
@@ -192,6 +209,7 @@ __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
       } else {
         for (int i = 0; i < ncols; ++i) lrow[i] = __uint_as_float(v[i]);
       }
+      if (partial) continue;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         float cv = __uint_as_float(v[i]);
@@ -213,7 +231,7 @@ __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
           if (j == k - 1) thr = best_v[j];
       }
     }
-    if (ok && t < T) {
+    if (ok && t < T && !partial) {
       float z[16], sum = 0.0f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -272,6 +290,19 @@ bool router_tc_supported(int T, int H, int E, int k) {
          router_tc_smem_bytes(E) <= 227 * 1024;
 }
 
+bool router_tc_split_supported(int H, int E, int k) {
+  return H % RT_BK == 0 && E % 16 == 0 && E >= 16 && E <= 256 && k <= 16 && router_tc_smem_bytes(E) <= 227 * 1024;
+}
+
+int router_tc_split_count(int T, int H, int num_sms) {
+  // (token tiles) x (slices of H), each slice at least 4 K steps: about one wave of CTAs
+  // below kRouterTcMinTokens tokens, about two from there on
+  const int tiles = (T + RT_MMA_M - 1) / RT_MMA_M;
+  const int max_splits = std::max(1, H / RT_BK / 4);
+  const int want = T < kRouterTcMinTokens ? num_sms / tiles : (2 * num_sms + tiles - 1) / tiles;
+  return std::max(1, std::min(want, max_splits));
+}
+
 int router_tc_tokens_per_cta(int T, int num_sms) {
   // two halves per CTA once 128-token CTAs would need more than one wave
   return T > num_sms * RT_MMA_M ? 2 * RT_MMA_M : RT_MMA_M;
@@ -279,21 +310,25 @@ int router_tc_tokens_per_cta(int T, int num_sms) {
 
 template <int HALVES>
 static cudaError_t launch_router_tc_t(const CUtensorMap& map_x, const uint16_t* w_tiles, int T, int H, int E, int k,
-                                      float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s) {
+                                      float* logits, int32_t* ids, float* wout, uint32_t* err, int splits,
+                                      cudaStream_t s) {
   using S = RtShape<HALVES>;
   const size_t smem = router_tc_smem<HALVES>(E);
   cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<HALVES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return launch_pdl(router_tc_kernel<HALVES>, dim3((T + S::BM - 1) / S::BM), dim3(S::THREADS), smem, s, map_x,
-                    reinterpret_cast<const uint8_t*>(w_tiles), T, H, E, k, logits, ids, wout, err);
+  return launch_pdl(router_tc_kernel<HALVES>, dim3((T + S::BM - 1) / S::BM, splits), dim3(S::THREADS), smem, s,
+                    map_x, reinterpret_cast<const uint8_t*>(w_tiles), T, H, E, k, logits, ids, wout, err, splits);
 }
 
 cudaError_t launch_router_tc(const CUtensorMap& map_x, int tokens_per_cta, const uint16_t* w_tiles, int T, int H,
-                             int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s) {
-  if (tokens_per_cta == 2 * RT_MMA_M)
-    return launch_router_tc_t<2>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, s);
-  if (tokens_per_cta == RT_MMA_M) return launch_router_tc_t<1>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, s);
+                             int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s,
+                             int splits) {
+  if (splits < 1) return cudaErrorInvalidValue;
+  if (tokens_per_cta == 2 * RT_MMA_M && splits == 1)
+    return launch_router_tc_t<2>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, 1, s);
+  if (tokens_per_cta == RT_MMA_M)
+    return launch_router_tc_t<1>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, splits, s);
   return cudaErrorInvalidValue;
 }
 

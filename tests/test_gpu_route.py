@@ -58,3 +58,48 @@ def test_route_zero_router_ties(bm):
     torch.cuda.synchronize()
     assert ids.cpu().numpy().tolist() == [list(range(8))] * 8
     np.testing.assert_allclose(w.cpu().numpy(), 1 / 8, rtol=1e-6)
+
+
+@pytest.fixture(scope="module")
+def router_layer(bm):
+    # the full router shape (H 5120 -> 256, top-8) with small experts (I = 128): only the
+    # routing buffers are read here
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(mi.SHAPES["decode8"], inter=128, tokens=5000)
+    weights = synthetic.make_weights(shape, 5, threads=8)
+    layer = bm.MoELayer(max_tokens=5000, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                        inter=shape.inter, alpha_a1=0.002, alpha_a2=0.0002, **weights)
+    yield shape, layer
+    layer.close()
+
+
+@pytest.mark.parametrize("tokens", [17, 32, 100, 640, 1024, 2500, 4095, 4096, 5000])
+def test_router_modes_match_oracle(bm, router_layer, tokens):
+    # SIMT FFMA over slices of H, and the tensor cores on the three-part BF16 split (below
+    # 4096 tokens over token tiles x slices of H with partial logits; from 4096 one tile per
+    # CTA with the top-k in the epilogue): both exact against the oracle except near-ties
+    shape, layer = router_layer
+    shape = dataclasses.replace(shape, tokens=tokens)
+    xb, rb = mi.tokens(shape, 6)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+    r = torch.from_numpy(rb.view(np.int16)).view(torch.bfloat16).cuda()
+    logits = moe.router_logits(mi.bf16_bits_to_f32(xb).astype(np.float64), mi.router_weight(shape, 5))
+    rid, rw, _ = moe.route_topk(logits, shape.top_k)
+    near = moe.near_tie_mask(logits, shape.top_k)
+    got = {}
+    for mode in (bm.ROUTER_SIMT, bm.ROUTER_TENSOR, bm.ROUTER_AUTO):
+        layer.set_router_mode(mode)
+        layer.forward(x, r)
+        layer.check()
+        ids = layer.debug(bm.BUF_IDS).cpu().numpy().view(np.int32).reshape(tokens, shape.top_k)
+        w = layer.debug(bm.BUF_WEIGHTS).cpu().numpy().view(np.float32).reshape(tokens, shape.top_k)
+        assert not ids_match(ids, rid, logits, near), mode
+        # neighbours with near-equal logits may swap slots: compare sorted weights.  The
+        # logits are FP32-accurate (~1e-5 absolute at |l| ~ 3 after 5120 terms, the scale of
+        # the near-tie margin), so the renormalised weights agree to ~1e-5
+        keep = ~near
+        np.testing.assert_allclose(np.sort(w[keep], 1), np.sort(rw[keep], 1), rtol=1e-4, atol=1e-5)
+        got[mode] = ids
+    layer.set_router_mode(bm.ROUTER_AUTO)
+    with pytest.raises(bm.BeamMoeError):
+        layer.set_router_mode(7)
