@@ -41,12 +41,12 @@ int router_split_count(int T, int H, int E);
 cudaError_t launch_topk(const float* logits, int splits, int T, int E, int k, int32_t* ids, float* w,
                         cudaStream_t s);
 
-// ---- router on the tensor cores for large batches (router_tc.cu)
-// One CTA per 128 tokens, each streaming all of W_r: below ~32 CTAs the split-H SIMT
-// router (router.cu) fills more of the GPU and is faster (0.11 vs 0.32 ms at T = 1024).
+// ---- router on the tensor cores (router_tc.cu)
+// Over (128-token tiles) x (slices of H) with partial logits that launch_topk sums: the
+// default for batches of kRouterTcSplitMinTokens or more.  One tile per CTA with the top-k
+// in its epilogue (router_tc_supported, from kRouterTcMinTokens tokens) is used once the
+// split count falls to one (router_tc_split_count).
 constexpr int kRouterTcMinTokens = 4096;
-// From this many tokens up to kRouterTcMinTokens the tensor-core router runs over
-// (token tiles) x (slices of H) with partial logits (BEAM_MOE_ROUTER_AUTO).
 constexpr int kRouterTcSplitMinTokens = BEAM_MOE_ROUTER_TC_SPLIT_MIN_TOKENS;
 bool router_tc_supported(int T, int H, int E, int k);
 size_t router_tc_smem_bytes(int E);

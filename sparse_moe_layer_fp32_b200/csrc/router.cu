@@ -12,6 +12,9 @@
 //  * many tokens: a 64x64-tiled SGEMM, split along H when there are too few tiles to
 //    fill the GPU; the split partial sums are added in a fixed order by the top-k
 //    kernel, so results are deterministic.
+// These serve beam_moe_route and BEAM_MOE_ROUTER_SIMT; the layer's default router for
+// batches above 16 tokens is the tensor-core one (router_tc.cu), whose partial logits the
+// same top-k kernel sums.
 // Top-k: one warp per token, E/32 logits per lane, k rounds of a warp arg-max
 // (larger logit first, equal logits -> lower expert index).  Since softmax is monotone
 // the top-k of p is the top-k of the logits, and p_j / sum_chosen p = softmax over the
@@ -159,16 +162,19 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
   pdl_wait();
   pdl_trigger();
   if (t >= T) return;
+  // slices outer, experts inner: the EPL loads of one slice are in flight together (the
+  // partials are read once: streaming loads); each expert's sum still runs over the slices
+  // in order
   float v[EPL];
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    float a = -INFINITY;
-    if (e < E) {
-      a = 0.0f;
-      for (int sp = 0; sp < splits; ++sp) a += partial[(static_cast<size_t>(sp) * T + t) * E + e];
-    }
-    v[i] = a;
+  for (int i = 0; i < EPL; ++i) v[i] = lane + 32 * i < E ? 0.0f : -INFINITY;
+  for (int sp = 0; sp < splits; ++sp) {
+    const float* row = partial + (static_cast<size_t>(sp) * T + t) * E;
+    float p[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) p[i] = lane + 32 * i < E ? __ldcs(row + lane + 32 * i) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) v[i] += p[i];
   }
   warp_topk<EPL>(v, E, k, lane, ids + static_cast<size_t>(t) * k, wout + static_cast<size_t>(t) * k);
 }
