@@ -48,3 +48,38 @@ def test_host_side_validation_without_gpu():
     assert lib.beam_moe_route_workspace_bytes(8, 5120, 256) == 8 * 256 * 4
     assert lib.beam_moe_route_workspace_bytes(0, 5120, 256) == 0
     assert lib.beam_moe_route_workspace_bytes(1024, 5120, 256) % (1024 * 256 * 4) == 0
+
+
+def test_host_side_validation_of_the_variant_and_parallel_entry_points():
+    # MXFP8 experts, tensor and expert parallelism, router mode: argument errors are answered
+    # on the host, before any CUDA call
+    import sparse_moe_layer_fp32_b200 as pkg
+    lib = pkg.lib()
+    h = ctypes.c_void_p()
+    bad = pkg.ERR_INVALID_ARG
+    assert lib.beam_moe_create_mxfp8(None, None, None, ctypes.byref(h)) == bad
+    assert lib.beam_moe_create_ep(None, None, 0, 8, None, ctypes.byref(h)) == bad
+    assert lib.beam_moe_create_ep_mxfp8(None, None, 0, 8, None, ctypes.byref(h)) == bad
+    cfg = pkg.BeamMoeConfig(8, 5120, 256, 8, 1536, 1e-6, 1.0, 1.0)
+    w = pkg.BeamMoeWeights()  # all null
+    assert lib.beam_moe_create_ep(ctypes.byref(cfg), ctypes.byref(w), 0, 0, None, ctypes.byref(h)) == bad
+    assert lib.beam_moe_create_mxfp8(ctypes.byref(cfg), ctypes.byref(pkg.BeamMoeWeightsMxfp8()), None,
+                                     ctypes.byref(h)) == bad
+    assert lib.beam_moe_quantize_mxfp8(None, 4, 48, None, None, None) == bad      # cols % 32
+    assert lib.beam_moe_quantize_mxfp8(None, -1, 64, None, None, None) == bad
+    assert lib.beam_moe_quantize_mxfp8(None, 0, 64, None, None, None) == pkg.OK  # empty: nothing to do
+    assert lib.beam_moe_quantize_mxfp8(None, 4, 64, None, None, None) == bad      # null buffers
+    assert lib.beam_moe_expert_format(None) == -1
+    assert lib.beam_moe_set_router_mode(None, pkg.ROUTER_AUTO) == bad
+    assert lib.beam_moe_set_gemm_mode(None, pkg.GEMM_AUTO) == bad
+    assert lib.beam_moe_tp_region_bytes(None) == 0
+    p = ctypes.c_void_p()
+    assert lib.beam_moe_tp_region(None, ctypes.byref(p)) == bad
+    assert lib.beam_moe_tp_attach(None, 0, 2, None, None) == bad
+    assert lib.beam_moe_forward_tp(None, None, None, None, 4, None) == bad
+    assert lib.beam_moe_forward_tp_phase(None, None, None, None, 4, 2, None) == bad  # phase 0 or 1
+    assert lib.beam_moe_forward_ep(None, None, None, None, 4, None) == bad
+    assert lib.beam_moe_forward_ep_phase(None, None, None, None, 4, 3, None) == bad  # phase 0, 1 or 2
+    assert lib.beam_moe_ipc_export(None, None) == bad
+    assert lib.beam_moe_ipc_import(None, ctypes.byref(p)) == bad
+    assert lib.beam_moe_ipc_close(None) == bad
