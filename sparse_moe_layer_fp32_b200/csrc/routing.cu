@@ -209,13 +209,23 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
   // Lanes 2c, 2c + 1 hold the two halves of one 16-byte code chunk and lanes 4g..4g + 3 the
   // four scale bytes of one K-group (nb is a multiple of 4): one 16-byte code store per lane
-  // pair and one 4-byte scale store per lane quad, per slot.
+  // pair and one 4-byte scale store per lane quad, per slot.  The next iteration's 32 bytes
+  // are loaded before this one's quantisation (its divisions hide the load latency).
+  uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+  if (lane < nb) {
+    n0 = __ldg(xr + 2 * lane);
+    n1 = __ldg(xr + 2 * lane + 1);
+  }
   for (int b0 = 0; b0 < nb; b0 += 32) {
     const int b = b0 + lane;
     const bool active = b < nb;  // whole quads are active or not
+    const uint4 p0 = n0, p1 = n1;
+    if (b + 32 < nb) {
+      n0 = __ldg(xr + 2 * (b + 32));
+      n1 = __ldg(xr + 2 * (b + 32) + 1);
+    }
     uint32_t lo = 0, hi = 0, sc = 0;
     if (active) {
-      const uint4 p0 = __ldg(xr + 2 * b), p1 = __ldg(xr + 2 * b + 1);
       const uint32_t u[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
       float v[16];
 #pragma unroll
