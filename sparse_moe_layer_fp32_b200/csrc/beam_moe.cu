@@ -607,14 +607,24 @@ int64_t beam_moe_tp_region_bytes(beam_moe_t h) {
 beam_moe_status beam_moe_tp_region(beam_moe_t h, void** region) {
   if (!h || !region) return BEAM_MOE_ERR_INVALID_ARG;
   if (!h->tp_region) {
+    // built into locals and published only when every step succeeded (a failed call leaves
+    // the handle without a region; what it allocated is freed with the handle)
     const size_t bytes = static_cast<size_t>(beam_moe_tp_region_bytes(h));
-    BEAM_TRY(dalloc(h, &h->tp_region, bytes));
-    BEAM_TRY(dalloc(h, &h->tp_counter, sizeof(unsigned int)));
-    BEAM_TRY(dalloc(h, &h->tp_regions_dev, sizeof(uint8_t*) * kMaxTpRanks));
-    BEAM_TRY(dalloc(h, &h->ep_counter, sizeof(unsigned int)));
-    BEAM_TRY(cudaMemset(h->ep_counter, 0, sizeof(unsigned int)));
-    BEAM_TRY(cudaMemset(h->tp_region, 0, kTpHeaderBytes));
-    BEAM_TRY(cudaMemset(h->tp_counter, 0, sizeof(unsigned int)));
+    uint8_t* region = nullptr;
+    uint8_t** table = nullptr;
+    unsigned int *tp_counter = nullptr, *ep_counter = nullptr;
+    BEAM_TRY(dalloc(h, &region, bytes));
+    BEAM_TRY(dalloc(h, &tp_counter, sizeof(unsigned int)));
+    BEAM_TRY(dalloc(h, &table, sizeof(uint8_t*) * kMaxTpRanks));
+    BEAM_TRY(dalloc(h, &ep_counter, sizeof(unsigned int)));
+    BEAM_TRY(cudaMemset(ep_counter, 0, sizeof(unsigned int)));
+    BEAM_TRY(cudaMemset(region, 0, kTpHeaderBytes));
+    BEAM_TRY(cudaMemset(tp_counter, 0, sizeof(unsigned int)));
+    BEAM_TRY(cudaDeviceSynchronize());
+    h->tp_region = region;
+    h->tp_counter = tp_counter;
+    h->tp_regions_dev = table;
+    h->ep_counter = ep_counter;
   }
   *region = h->tp_region;
   return BEAM_MOE_OK;
