@@ -163,3 +163,32 @@ def test_ep_shard_experts_partition_the_expert_arrays():
     assert all(sh["router_w"] is full["router_w"] and sh["gamma"] is full["gamma"] for sh in shards)
     with pytest.raises(ValueError):
         tp.shard_experts(full, 0, 3, E)
+
+
+def test_bench_host_logic_for_the_expert_formats(repo_root, capsys):
+    # algorithmic bytes per quantised value (NVFP4 0.5 + 1/16, MXFP8 1 + 1/32), the expert
+    # GEMM's bytes and FLOPs, and the reference arm's JSON line for the MXFP8 variant on the
+    # tiny workload (the CPU oracle, bounded sample)
+    import json
+
+    import numpy as np
+
+    import bench
+    import moe_inputs as mi
+    shape = mi.SHAPES["decode8"]
+    counts = np.zeros(shape.experts, np.int64)
+    counts[:58] = 1
+    w4 = bench.kernel_work(shape, 8, counts, "nvfp4")["gemm_experts"]
+    w8 = bench.kernel_work(shape, 8, counts, "mxfp8")["gemm_experts"]
+    assert w4["flops"] == w8["flops"] == 2 * 64 * 3 * 1536 * 5120
+    weights4 = 58 * 3 * 1536 * 5120 * 0.5625
+    weights8 = 58 * 3 * 1536 * 5120 * 1.03125
+    assert weights4 < w4["bytes"] < weights4 * 1.01
+    assert weights8 < w8["bytes"] < weights8 * 1.01
+
+    class A:
+        steps, warmup, gpus, experts_format = 1, 0, 1, "mxfp8"
+    bench.run_reference(A, mi.SHAPES["tiny"], 0, 1)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["config"]["experts_format"] == "mxfp8"
+    assert line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
