@@ -76,13 +76,13 @@ __global__ void __launch_bounds__(kFinThreads) finalize_wide_kernel(const uint16
   float ss = 0.0f;
   for (int c = threadIdx.x; c < nchunks; c += kFinThreads) {
     float acc[8] = {};
-    for (int j0 = 0; j0 < k; j0 += 4) {
-      uint4 yv[4];
+    for (int j0 = 0; j0 < k; j0 += 8) {  // up to 8 rows' chunks in flight (top-8: all of them)
+      uint4 yv[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < 8; ++j)
         if (j0 + j < k) yv[j] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j0 + j]) * H) + c);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         if (j0 + j >= k) break;
         float f[8];
         unpack8(yv[j], f);
