@@ -121,3 +121,37 @@ def test_quantize_mxfp8_edge_blocks(bm):
     assert sf[0, 0] == 0 and sf[3, 0] == 127 - 20 and sf[5, 0] == 127
     with pytest.raises(bm.BeamMoeError):
         bm.beam_moe_quantize_mxfp8(torch.zeros((2, 48), device="cuda"))
+
+
+def test_hardware_conversions_swept_against_the_oracle_rounding(bm):
+    # The quantisers expose the raw conversions when the block scale is one: an MXFP8 block
+    # holding 448 (the E4M3 maximum) has scale 2^0, so its codes are E4M3(v); an NVFP4 block
+    # with amax 6 and alpha 1 has d = E4M3(6 / 6) = 1, so its codes are E2M1(v).  Every code,
+    # every midpoint between neighbours and the FP32 neighbours of each midpoint, both signs.
+    from oracle import mxfp8
+    e4 = mxfp8.e4m3_decode_signed(np.arange(0x7F, dtype=np.uint8))
+    mids = ((e4[:-1] + e4[1:]) / 2).astype(np.float32)
+    pos = np.concatenate([e4.astype(np.float32), mids, np.nextafter(mids, np.float32(0)),
+                          np.nextafter(mids, np.float32(1e9))])
+    vals = np.concatenate([pos, -pos]).astype(np.float32)
+    n = (len(vals) + 30) // 31
+    v = np.zeros((n, 32), np.float32)
+    v[:, 0] = 448.0  # fixes the scale at 2^0
+    v[:, 1:].reshape(-1)[: len(vals)] = vals
+    codes, sf = _gpu_mx(bm, v)
+    assert np.all(sf == 127)
+    np.testing.assert_array_equal(codes, mxfp8.e4m3_encode_signed(v))
+    # E2M1 through NVFP4 with d = 1
+    e2 = nvfp4.E2M1_VALUES.astype(np.float32)
+    m2 = ((e2[:-1] + e2[1:]) / 2).astype(np.float32)
+    p2 = np.concatenate([e2, m2, np.nextafter(m2, np.float32(0)), np.nextafter(m2, np.float32(10))])
+    vals2 = np.concatenate([p2, -p2]).astype(np.float32)
+    n2 = (len(vals2) + 14) // 15
+    w = np.zeros((n2, 16), np.float32)
+    w[:, 0] = 6.0  # amax 6 with alpha 1: scale E4M3(1) = 1, d = 1
+    w[:, 1:].reshape(-1)[: len(vals2)] = vals2
+    c2, s2, a = _gpu_q(bm, w, 1.0)
+    assert a == 1.0 and np.all(nvfp4.e4m3_decode(s2) == 1.0)
+    np.testing.assert_array_equal(_norm(c2), _norm(nvfp4.quantize_nvfp4(w, np.float32(1.0))[0]))
+    np.testing.assert_array_equal(_norm(c2).reshape(n2, 16), np.where(nvfp4.e2m1_encode(w) == 8, 0,
+                                                                      nvfp4.e2m1_encode(w)))
