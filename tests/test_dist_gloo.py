@@ -192,3 +192,39 @@ def test_bench_host_logic_for_the_expert_formats(repo_root, capsys):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["config"]["experts_format"] == "mxfp8"
     assert line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+class _PhaseLayer:
+    def __init__(self, log, rank, ep):
+        self.log, self.rank, self.expert_parallel = log, rank, ep
+        self.attached = None
+
+    def tp_region(self):
+        return 0x1000 * (self.rank + 1)
+
+    def tp_attach(self, rank, world, regions):
+        self.attached = (rank, world, list(regions))
+
+    def forward_tp_phase(self, x, residual, out, phase):
+        self.log.append(("tp", self.rank, phase))
+
+    def forward_ep_phase(self, x, residual, out, phase):
+        self.log.append(("ep", self.rank, phase))
+
+
+@pytest.mark.parametrize("ep", [False, True])
+def test_shared_gpu_group_runs_every_rank_phase_by_phase(ep):
+    # Ranks sharing one GPU must never have a kernel wait on a kernel that has not run: every
+    # rank's phase p is enqueued before any rank's phase p + 1 (TP: 2 phases, EP: 3).
+    from sparse_moe_layer_fp32_b200 import tp
+    log = []
+    layers = [_PhaseLayer(log, r, ep) for r in range(3)]
+    grp = tp.SharedGpuGroup(layers)
+    assert [lay.attached for lay in layers] == [(r, 3, [0x1000, 0x2000, 0x3000]) for r in range(3)]
+    xs = [torch.zeros(2, 8) for _ in range(3)]
+    if ep:
+        grp.forward(xs, xs, outs=[torch.zeros(2, 8) for _ in range(3)])
+    else:
+        grp.forward(xs[0], xs[0], outs=[torch.zeros(2, 8) for _ in range(3)])
+    phases = 3 if ep else 2
+    assert log == [("ep" if ep else "tp", r, p) for p in range(phases) for r in range(3)]
