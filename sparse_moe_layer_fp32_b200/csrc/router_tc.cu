@@ -166,9 +166,8 @@ __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
           phase ^= 1;
         }
       }
-      if (k_tiles == 0) {  // an empty slice (H not divisible into the splits): zero partials
-        // nothing was issued; the epilogue writes zeros for this slice
-      }
+      // an empty slice (k_tiles == 0: the splits do not divide H evenly) issued nothing; its
+      // epilogue writes zeros
       tc_commit(&tail->acc_full);  // also fires after an abort, once the issued MMAs finish
       // every issued MMA has finished before TMEM can be freed (bounded)
       const uint64_t t0 = globaltimer_ns();
