@@ -10,8 +10,9 @@ other than themselves.
 * Quantisation: each code is the nearest E4M3 of v / 2^e (torch again), values already on
   the grid round-trip exactly, and the error stays within half an E4M3 step.
 * The layer with MXFP8 experts: dense evaluation of every expert masked by the routing
-  equals the sparse forward, and grid-exact operands reduce the expert GEMMs to plain
-  FP64 matmuls.
+  equals the sparse forward, grid-exact operands reduce the expert GEMMs to plain FP64
+  matmuls, and a hand-worked two-expert example matches every intermediate written as a
+  literal (scales, codes, SwiGLU values, A2 roundings, m, the RMS and the BF16 output).
 The FP8 checkpoint is the second variant of the routed experts (vLLM recipe
 "reflection/Beam-1.0-501B-A23B", section "Variants"); MXFP8 is the reading of its block
 format (E4M3 values, one power-of-two scale per 32 values).
@@ -194,3 +195,46 @@ def test_mxfp8_grid_exact_expert_gemms_equal_fp64_matmul():
     np.testing.assert_array_equal(r["h32"], (gg / (1 + np.exp(-gg)) * uu).astype(np.float32))
     a2 = mx.dequantize_mxfp8(r["a2_packed"], r["a2_sf"])
     np.testing.assert_allclose(r["y"], a2 @ w_d.T.astype(np.float64), rtol=1e-15, atol=0)
+
+
+def test_hand_worked_two_expert_example_mxfp8():
+    # T = 1, H = I = 32 (one MX block), E = 2, k = 2, residual 0, gamma 1.  x = 2 e0, router
+    # rows +-0.5 e0 (logits +-1); expert 0: gate row 0 = up row 0 = e0, down[0, 0] = 1;
+    # expert 1: gate row 0 = -e0, up row 0 = e0, down[1, 0] = 1.  Worked by hand:
+    #   A1: amax 2 -> e = -7 (2 <= 448 * 2^-7 = 3.5, 2 > 448 * 2^-8), 2 / 2^-7 = 256 exact
+    #   weights: amax 1 -> e = -8, 1 / 2^-8 = 256 exact: every operand is exact
+    #   h0 = silu(2) * 2 = 4 sigmoid(2) = 3.52318831; e = -6; 3.5232 * 64 = 225.48 -> E4M3 224
+    #        (step 16 in [128, 256)) -> 3.5
+    #   h1 = silu(-2) * 2 = -4 sigmoid(-2) = -0.47681169; e = -9; * 512 = -244.13 -> -240 -> -0.46875
+    #   m = (sigmoid(2) * 3.5, sigmoid(-2) * -0.46875) = (3.08278977, -0.05587637)
+    #   rms = sqrt((m0^2 + m1^2) / 32 + 1e-6) = 0.54505582; out = (5.65591575, -0.10251495)
+    #   BF16: 5.65625 (181 * 2^-5), -0.1025390625 (-210 * 2^-11)
+    H = I = 32
+    x = np.zeros((1, H)); x[0, 0] = 2.0
+    wr = np.zeros((2, H), np.float32); wr[0, 0] = 0.5; wr[1, 0] = -0.5
+    experts = {}
+    for e, sign in ((0, 1.0), (1, -1.0)):
+        w_gu = np.zeros((2 * I, H), np.float32)
+        w_gu[0, 0] = sign
+        w_gu[I, 0] = 1.0
+        w_d = np.zeros((H, I), np.float32)
+        w_d[e, 0] = 1.0
+        experts[e] = (w_gu, w_d)
+    cache = moe.ExpertCache(lambda e: experts[e], fmt="mxfp8")
+    r = moe.moe_forward(x, np.zeros_like(x), wr, np.ones(H), cache, num_experts=2, top_k=2, alpha_a1=None,
+                        alpha_a2=None)
+    assert r["ids"].tolist() == [[0, 1]]
+    np.testing.assert_allclose(r["w"][0], [0.8807970779778823, 0.11920292202211755], rtol=1e-15)
+    assert r["a1_sf"][0, 0] == 127 - 7 and r["a1_packed"][0, 0] == 0x78  # 256 = 2^8: E4M3 (15 << 3) | 0
+    assert not r["a1_packed"][0, 1:].any()
+    q0 = cache.quantized(0)
+    assert q0["w_gu_sf"][0, 0] == 127 - 8 and q0["w_gu"][0, 0] == 0x78 and q0["w_gu"][I, 0] == 0x78
+    assert q0["w_gu"][0, 1:].sum() == 0 and q0["w_d_sf"][0, 0] == 127 - 8
+    h0, h1 = r["h32"][0, 0, 0], r["h32"][0, 1, 0]
+    assert abs(h0 - 3.52318831) < 1e-6 and abs(h1 - (-0.47681169)) < 1e-6
+    y = r["y"][0]
+    assert y[0, 0] == 3.5 and y[1, 1] == -0.46875 and not y[0, 1:].any() and y[1, 0] == 0
+    m = r["m"][0]
+    assert abs(m[0] - 3.08278977) < 1e-7 and abs(m[1] - (-0.05587637)) < 1e-7 and not m[2:].any()
+    assert abs(r["out_pre"][0, 0] - 5.65591575) < 1e-7 and abs(r["out_pre"][0, 1] - (-0.10251495)) < 1e-7
+    assert r["out"][0, 0] == 181 * 2.0 ** -5 and r["out"][0, 1] == -210 * 2.0 ** -11
