@@ -254,11 +254,17 @@ BEAM_MOE_API beam_moe_status beam_moe_route(const void* x, const float* router_w
  * imply) is not allowed after start-up.  Same result as beam_moe_route (same kernels),
  * but the logits scratch is a fixed 8 MiB array compiled into this library: every GPU
  * that loads the library holds it until the process exits.
- *   - Accepts exactly the shapes whose beam_moe_route_workspace_bytes(T, H, E) is at
- *     most 8 MiB (at H = 5120, E = 256: T <= 4096 and 4736 <= T <= 8192); larger shapes
+ *   - Accepts exactly the shapes whose logits fit the array: S(T, H, E) * T * E <= 2^21
+ *     floats, where S is the number of slices of H the router sums (the rule of
+ *     beam_moe_route_workspace_bytes(T, H, E) <= 8 MiB).  S falls as T grows (8, 4, 2, 1
+ *     at H = 5120, E = 256), so the accepted T are not one interval: at H = 5120,
+ *     E = 256 they are 1..1024, 1153..2048, 2305..4096 and 4673..8192.  Other shapes
  *     return BEAM_MOE_ERR_UNSUPPORTED before anything is enqueued.
  *   - The first call on each device looks up the array's device address (with that
  *     device current) and caches it; make that first call before any stream capture.
+ *     The address is looked up again only when the device's CUDA context has changed
+ *     (a device reset): the first call after such a change should also come before any
+ *     stream capture.
  *   - All calls on a device share the one array, which keeps the last call's contents
  *     (every element a call reads it first writes, so nothing needs clearing).  Calls
  *     that overlap on the GPU (different streams, or different host threads) race on it:

@@ -21,21 +21,53 @@ static __device__ __align__(256) float g_route_scratch[kStaticScratchFloats];
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 float* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context the address belongs to
 
-// Device address of the scratch array on the current device, looked up once per device.
-// In host code `g_route_scratch` names a host-side stand-in, not device memory, so the
-// kernels must receive the address that cudaGetSymbolAddress returns.
+// Unique id of the current CUDA context (never reused within a process), or false when no
+// context is current.  A device reset destroys the context the module was loaded into; the
+// next context gets a new id, and the array a new address.
+bool current_context_id(unsigned long long* id) {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess)
+      return false;
+    get_current = reinterpret_cast<GetCurrent>(a);
+    get_id = reinterpret_cast<GetId>(b);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array on the current device.  It is looked up the first
+// time a device is used, and again only if the device's context has changed since (after a
+// device reset, say), so a stale address is never handed to a kernel.  In host code
+// `g_route_scratch` names a host-side stand-in, not device memory, so the kernels must
+// receive the address that cudaGetSymbolAddress returns.
 cudaError_t scratch_on_current_device(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_addr[dev]) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  if (!g_scratch_addr[dev] || !have_ctx || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    e = cudaGetSymbolAddress(&p, g_route_scratch);  // makes the device's context current if none was
     if (e != cudaSuccess) return e;
+    if (!current_context_id(&ctx)) return cudaErrorDeviceUninitialized;  // no context after the lookup
     g_scratch_addr[dev] = static_cast<float*>(p);
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_addr[dev];
   return cudaSuccess;

@@ -7,9 +7,11 @@ allocation can bring) once it is running.  beam_moe_route_static serves them: it
 scratch is a fixed array compiled into the library, so the caller passes only x, the
 router weights and the outputs.  The pages have no counterpart of this entry point.
 
-The test calls it through the C ABI twice in a row, on two different shapes, and checks
-each result against the allocating entry point beam_moe_route at the routing tolerance of
-the other GPU tests (ids equal, weights within 2e-5).  This file is collected last.
+The test calls it through the C ABI several times in a row, on different shapes (among
+them the two that fill the array exactly with 2 and 1 slices of H), and checks each result
+against the allocating entry point beam_moe_route at the routing tolerance of the other GPU
+tests (ids equal, weights within 2e-5).  Shapes whose logits do not fit the array, including
+those between the accepted token ranges, must be rejected.  This file is collected last.
 """
 
 import ctypes
@@ -46,7 +48,8 @@ def test_route_static_matches_route_on_consecutive_calls():
     import sparse_moe_layer_fp32_b200 as bm
 
     results = []
-    for name, tokens, seed in (("decode8", 8, 11), ("spec1024", 1024, 12)):
+    for name, tokens, seed in (("decode8", 8, 11), ("spec1024", 1024, 12), ("prefill16k", 4096, 14),
+                               ("prefill16k", 8192, 15)):
         shape, x, wr = _inputs(name, tokens, seed)
         st, ids, w = _route_static(bm, x, wr, shape.top_k)
         assert st == bm.OK, bm.status_string(st)
@@ -70,3 +73,13 @@ def test_route_static_rejects_shapes_beyond_its_array():
                                         None)
     assert st == bm.ERR_UNSUPPORTED
     assert bm.beam_moe_route_workspace_bytes(16384, 5120, 256) > 8 << 20
+    # between the accepted ranges: 1025..1152 tokens are summed over 8 slices of H, 4097..4672
+    # over 2, so their logits need more than the array holds although 4096 and 8192 fit
+    for tokens in (1025, 1100, 1152, 2049, 2304, 4097, 4672, 8193):
+        st = bm.lib().beam_moe_route_static(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(wr.data_ptr()), tokens,
+                                            5120, 256, 8, ctypes.c_void_p(x.data_ptr()),
+                                            ctypes.c_void_p(x.data_ptr()), None)
+        assert st == bm.ERR_UNSUPPORTED, tokens
+        assert bm.beam_moe_route_workspace_bytes(tokens, 5120, 256) > 8 << 20, tokens
+    for tokens in (1024, 1153, 2048, 2305, 4096, 4673, 8192):
+        assert bm.beam_moe_route_workspace_bytes(tokens, 5120, 256) <= 8 << 20, tokens
