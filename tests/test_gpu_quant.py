@@ -65,11 +65,40 @@ def test_quantize_edge_blocks(bm):
         np.testing.assert_array_equal(_norm(codes), _norm(rc))
 
 
+def test_quotients_near_every_e2m1_midpoint(bm):
+    # v / d within a few ulp of each E2M1 rounding midpoint (and exactly on it where fl32
+    # allows), for many block scales d: the quotients whose rounding the quantiser must
+    # settle with an IEEE division rather than its reciprocal product.
+    rng = np.random.default_rng(77)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    rows = []
+    for alpha in (np.float32(1.0), np.float32(0.37), np.float32(1e-3), np.float32(3.1e-5)):
+        for sc in rng.choice(np.arange(8, 127), 12, replace=False):
+            d = np.float32(nvfp4.e4m3_decode(np.uint8(sc)) * alpha)
+            for m in mids:
+                base = np.float32(m * d)
+                cand = [base, np.nextafter(base, np.float32(0)), np.nextafter(base, np.float32(np.inf))]
+                cand += [np.nextafter(cand[1], np.float32(0)), np.nextafter(cand[2], np.float32(np.inf))]
+                row = np.zeros(16, np.float32)
+                row[0] = np.float32(6.0 * d)  # amax: the block's scale code is sc again
+                row[1:6] = cand
+                row[6:11] = -np.array(cand, np.float32)
+                row[11:] = rng.uniform(-6, 6, 5).astype(np.float32) * d
+                rows.append((row, alpha))
+    for alpha in sorted({a for _, a in rows}):
+        v = np.stack([r for r, a in rows if a == alpha])
+        codes, sf, _ = _gpu_q(bm, v, float(alpha))
+        rc, rs = nvfp4.quantize_nvfp4(v, alpha)
+        np.testing.assert_array_equal(sf, rs)
+        np.testing.assert_array_equal(_norm(codes), _norm(rc))
+
+
 def test_e2m1_e4m3_conversion_sweep(bm):
-    # 2^24 values per call spread over every block scale and every E2M1 interval: the
-    # hardware conversions (cvt.rn.satfinite e2m1x2 / e4m3x2) against the oracle rounding.
+    # 7 x 2^24 (1.17e8) values spread over every block scale and every E2M1 interval: the
+    # hardware conversions (cvt.rn.satfinite e2m1x2 / e4m3x2) and the quotient rounding
+    # against the oracle rounding.
     rng = np.random.default_rng(2024)
-    for _ in range(2):
+    for _ in range(7):
         n = 1 << 24
         mag = np.exp(rng.uniform(np.log(1e-3), np.log(5e3), n // 16)).astype(np.float32)
         v = (rng.uniform(-1, 1, (n // 16, 16)) * mag[:, None]).astype(np.float32)
