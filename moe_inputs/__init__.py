@@ -61,6 +61,9 @@ SHAPES = {
         LayerShape("decode8_e32", 8, 5120, 32, 8, 1536),
         # profiling case: the 8 x 2K prefill's rows per expert (512) with 32 experts
         LayerShape("prefill2k_e32", 2048, 5120, 32, 8, 1536),
+        # profiling case: the 8 x 2K prefill's token count (per-token kernels see the full
+        # batch: x 168 MB, A1 377 MB, y 1.34 GB, all larger than L2) with 32 experts' weights
+        LayerShape("prefill16k_e32", 16384, 5120, 32, 8, 1536),
     ]
 }
 

@@ -109,6 +109,40 @@ def ids_match(gpu_ids: np.ndarray, ref_ids: np.ndarray, logits: np.ndarray, near
     return bad
 
 
+def ids_match_sel(gpu_ids: np.ndarray, ref_ids: np.ndarray, logits_sel: np.ndarray, near: np.ndarray, rel=1e-5):
+    """ids_match with the oracle's logits of its chosen experts only (logits_sel[t, j] is the
+    logit of ref_ids[t, j]), which is all the order check needs."""
+    t_count, k = ref_ids.shape
+    dense = np.zeros((t_count, int(max(ref_ids.max(), gpu_ids.max())) + 1), np.float64)
+    np.put_along_axis(dense, ref_ids.astype(np.int64), logits_sel, axis=1)
+    return ids_match(gpu_ids, ref_ids, dense, near, rel)
+
+
+def oracle_batch_routing(x_bits: np.ndarray, router_w: np.ndarray, k: int, chunk: int = 4096):
+    """The oracle's routing of a whole batch (FP64 logits, computed in chunks of tokens):
+    ids [T, k], w [T, k], the chosen logits [T, k] and the near-tie mask [T]."""
+    t_count = x_bits.shape[0]
+    ids = np.empty((t_count, k), np.int64)
+    w = np.empty((t_count, k), np.float64)
+    lsel = np.empty((t_count, k), np.float64)
+    near = np.empty(t_count, bool)
+    for t0 in range(0, t_count, chunk):
+        t1 = min(t_count, t0 + chunk)
+        logits = moe.router_logits(mi.bf16_bits_to_f32(x_bits[t0:t1]), router_w)
+        i, ww, _ = moe.route_topk(logits, k)
+        ids[t0:t1], w[t0:t1] = i, ww
+        lsel[t0:t1] = np.take_along_axis(logits, i, axis=1)
+        near[t0:t1] = moe.near_tie_mask(logits, k)
+    return ids, w, lsel, near
+
+
+def weights_by_expert(ids: np.ndarray, w: np.ndarray, rows) -> tuple:
+    """(ids, w) of the given rows with each row's slots sorted by expert id, so routing
+    weights compare per (token, expert) whatever the slot order."""
+    o = np.argsort(ids[rows], axis=1, kind="stable")
+    return np.take_along_axis(ids[rows], o, 1), np.take_along_axis(w[rows], o, 1)
+
+
 def oracle_layer_inputs(shape: mi.LayerShape, seed: int, weights_fp32=None, tokens=None, fmt: str = "nvfp4"):
     """Oracle-side inputs of a workload: x, residual (FP64 of BF16), W_r, gamma, expert cache."""
     xb, rb = mi.tokens(shape, seed) if tokens is None else tokens
