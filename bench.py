@@ -4,9 +4,13 @@
 One step = one whole layer forward (router, top-k, permutation, NVFP4 quantisation, the
 two grouped NVFP4 GEMMs, finalize) over one synthetic batch of the chosen workload.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode8] [--impl ours|reference]
-                  [--experts-format nvfp4|mxfp8] [--tp-shared-gpu W]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload default|<name>]
+                  [--impl ours|reference] [--experts-format nvfp4|mxfp8] [--tp-shared-gpu W]
 
+The default run measures the metric's three batch sizes on one layer: the 8 x 2K prefill
+(T = 16384, the headline of the JSON line), the decode verify step (T = 8) and the batched
+verify (T = 1024) under "workloads", each with its own roofline, e2e, clocks, CPU baseline
+and parity against the oracle.  --workload <name> measures one workload alone.
 --experts-format mxfp8 measures the block-scaled FP8 variant of the experts (E4M3 values,
 one power-of-two scale per 32).  --tp-shared-gpu W measures the tensor-parallel layer with
 W ranks sharing this GPU, run in turn (per-rank phase timings; see run_tp_shared).
@@ -101,88 +105,127 @@ def read_traffic(kernel: str, used_experts: int, tokens: int):
 
 
 # ------------------------------------------------------------------ clocks
+REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
+
+
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during a region."""
+    """SM clock, power and clock-event (throttle) reasons of one GPU, sampled while a region
+    runs: NVML polled every 2 ms from a thread (the timed regions last tens of ms), else
+    nvidia-smi at its 200 ms period."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, pci_bus_id: str | None = None, period_s: float = 0.002):
         self.gpu = gpu_index
+        self.pci = pci_bus_id
+        self.period = period_s
+        self.rows = []  # (sm_mhz, max_mhz, power_w, reasons bitmask)
         self.proc = None
         self.path = None
+        self.thread = None
+        self.stop = False
+        self.source = None
+
+    def _nvml_loop(self, nvml, handle):
+        mx = float(nvml.nvmlDeviceGetMaxClockInfo(handle, nvml.NVML_CLOCK_SM))
+        while not self.stop:
+            try:
+                sm = float(nvml.nvmlDeviceGetClockInfo(handle, nvml.NVML_CLOCK_SM))
+                pw = nvml.nvmlDeviceGetPowerUsage(handle) / 1000.0
+                rs = int(nvml.nvmlDeviceGetCurrentClocksEventReasons(handle))
+                self.rows.append((sm, mx, pw, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def __enter__(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
-        time.sleep(0.3)
+            import threading
+
+            import pynvml as nvml
+            nvml.nvmlInit()
+            handle = (nvml.nvmlDeviceGetHandleByPciBusId(self.pci) if self.pci
+                      else nvml.nvmlDeviceGetHandleByIndex(self.gpu))
+            self.source = "nvml 2 ms"
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nvml, handle), daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                              "--format=csv,noheader,nounits", "-lms", "200"],
+                                             stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                self.source = "nvidia-smi 200 ms"
+            except (OSError, FileNotFoundError):
+                self.proc = None
+        time.sleep(0.05)
         return self
 
     def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=5)
         if self.proc:
             self.proc.terminate()
             self.proc.wait(timeout=10)
 
     def summary(self):
-        rows = []
-        try:
-            for line in open(self.path):
-                f = [c.strip() for c in line.split(",")]
-                if len(f) >= 9 and f[1].replace(".", "").isdigit():
-                    rows.append(f)
-        finally:
-            os.unlink(self.path)
+        rows = list(self.rows)
+        if self.path:
+            try:
+                names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+                for line in open(self.path):
+                    f = [c.strip() for c in line.split(",")]
+                    if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                        bits = sum(REASON_BITS[n] for n, v in zip(names, f[5:9]) if v.lower() == "active")
+                        pw = float(f[3]) if f[3].replace(".", "").isdigit() else 0.0
+                        rows.append((float(f[1]), float(f[2]), pw, bits))
+            finally:
+                os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        sm = [float(r[1]) for r in rows]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+        reasons = sorted({n for r in rows for n, b in REASON_BITS.items() if r[3] & b})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1], "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(r[2] for r in rows), "source": self.source}
 
 
 # ------------------------------------------------------------------ CPU oracle leg
 def oracle_sample(shape: mi.LayerShape, tokens, seed=0, fmt="nvfp4"):
-    """Inputs and quantised experts the oracle needs for a token sample (prepared untimed)."""
+    """Inputs of the oracle for a token sample, drawn untimed: the tokens' BF16 rows, the
+    router, gamma and the FP32 weights of the experts they route to."""
     from oracle import moe
     xs, rs = [], []
     for t in tokens:
         xb, rb = mi.tokens(shape, seed, t, t + 1)
         xs.append(xb[0])
         rs.append(rb[0])
-    x = mi.bf16_bits_to_f32(np.stack(xs)).astype(np.float64)
-    res = mi.bf16_bits_to_f32(np.stack(rs)).astype(np.float64)
+    xb, rb = np.stack(xs), np.stack(rs)
     wr = mi.router_weight(shape, seed)
-    g = mi.bf16_bits_to_f32(mi.gamma(shape, seed)).astype(np.float64)
-    ids, _, _ = moe.route_topk(moe.router_logits(x, wr), shape.top_k)
-    quantised = {int(e): moe.quantize_expert(*mi.expert_weights(shape, seed, int(e)), fmt) for e in np.unique(ids)}
-    return x, res, wr, g, quantised, fmt
+    ids, _, _ = moe.route_topk(moe.router_logits(mi.bf16_bits_to_f32(xb), wr), shape.top_k)
+    experts = {int(e): mi.expert_weights(shape, seed, int(e)) for e in np.unique(ids)}
+    return xb, rb, wr, mi.gamma(shape, seed), experts, fmt
 
 
 def oracle_step(shape, sample):
-    """One oracle forward of the sample: routing, experts (dequantised from the stored
-    quantised weights, FP64 matmuls), finalize.  Returns tokens processed."""
-    from oracle import moe
-    x, res, wr, g, quantised, fmt = sample
-    a1, a2 = mi.activation_scales(shape) if fmt == "nvfp4" else (None, None)
-    cache = moe.ExpertCache(lambda e: None, keep=2, fmt=fmt)
-    cache._q = dict(quantised)
-    moe.moe_forward_tokens(x, res, wr, g, cache, shape.top_k, a1, a2, shape.rms_eps)
-    return x.shape[0]
+    """One forward of the sample by the C++ FP64 oracle (OpenMP over the host cores): routing,
+    each expert quantised by the oracle's own quantiser and dequantised to FP64, the FP64
+    expert GEMMs, finalize.  Returns (tokens processed, its result)."""
+    from oracle import cpp
+    xb, rb, wr, gb, experts, fmt = sample
+    a1, a2 = mi.activation_scales(shape) if fmt == "nvfp4" else (1.0, 1.0)
+    r = cpp.moe_forward(xb, rb, wr, gb, experts.__getitem__, shape.top_k, shape.inter, alpha_a1=a1, alpha_a2=a2,
+                        eps=shape.rms_eps, fmt=fmt)
+    return xb.shape[0], r
 
 
 def cpu_cores() -> int:
+    """Threads the C++ oracle runs on (OpenMP uses every core the process may run on)."""
     try:
-        from threadpoolctl import threadpool_info
-        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-        return int(n)
+        return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count() or 1
 
@@ -191,31 +234,66 @@ def cpu_sample_tokens(shape):
     return [0] if shape.tokens <= 64 else [0, shape.tokens // 2]
 
 
-def cpu_baseline(shape, budget_s=25.0, fmt="nvfp4"):
+def cpu_baseline(shape, budget_s=8.0, fmt="nvfp4", gpu=None):
+    """The oracle timed on the host cores over a bounded sample of the workload.  With gpu =
+    (ids [T, k], out [T, H] as FP64) of the same batch on the GPU, also the parity of that
+    batch: the oracle's routing of every token (FP64 logits) against the GPU's ids, with the
+    near-tie count, and the GPU's output rows of the sampled tokens against the oracle's."""
     toks = cpu_sample_tokens(shape)
     sample = oracle_sample(shape, toks, fmt=fmt)
     t0 = time.perf_counter()
     n = 0
     reps = 0
+    r = None
     while True:
-        n += oracle_step(shape, sample)
+        dn, r = oracle_step(shape, sample)
+        n += dn
         reps += 1
-        if time.perf_counter() - t0 > budget_s or reps >= 3:
+        if time.perf_counter() - t0 > budget_s or reps >= 2:
             break
     dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"{len(toks)} token(s) of the {shape.name} batch x {reps} repeats: FP64 router, "
-                      f"{fmt.upper()} experts dequantised from stored codes, finalize; weights pre-quantised untimed"}
+    base = {"value": n / dt, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{len(toks)} token(s) of the {shape.name} batch x {reps} repeats through the C++ FP64 oracle: "
+                      f"router, top-k, {fmt.upper()} quantisation of x and of each routed expert's FP32 weights, "
+                      f"FP64 expert GEMMs, finalize; FP32 weights drawn untimed"}
+    if gpu is None:
+        return base, None
+    return base, oracle_parity(shape, toks, r, *gpu)
+
+
+def oracle_parity(shape, toks, ref, gpu_ids, gpu_out, seed=0):
+    """Parity of the GPU's forward of a batch (routing of every token, outputs of the sampled
+    tokens) against the oracle; see cpu_baseline."""
+    from oracle import moe
+    k = shape.top_k
+    wr = mi.router_weight(shape, seed)
+    near = np.zeros(shape.tokens, bool)
+    differ = 0
+    for t0 in range(0, shape.tokens, 4096):
+        t1 = min(shape.tokens, t0 + 4096)
+        xb, _ = mi.tokens(shape, seed, t0, t1)
+        logits = moe.router_logits(mi.bf16_bits_to_f32(xb), wr)
+        ids = moe.route_topk(logits, k)[0]
+        near[t0:t1] = moe.near_tie_mask(logits, k)
+        same = np.sort(ids, 1) == np.sort(gpu_ids[t0:t1], 1)
+        differ += int((~same.all(1) & ~near[t0:t1]).sum())
+    keep = ~near[toks]
+    g, o = gpu_out[toks][keep], ref["out_pre"][keep]
+    rel = float(np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-30)) if g.size else 0.0
+    mx = float(np.abs(g - o).max()) if g.size else 0.0
+    return {"near_ties": int(near.sum()), "tokens": shape.tokens, "ids_differ_outside_near_ties": differ,
+            "sampled_tokens": len(toks), "rel_l2": rel, "max_abs": mx, "tol": {"rel_l2": 1e-2, "max_abs": 5e-2}}
 
 
 def run_reference(args, shape, rank, world):
     if rank != 0:
         return
-    sample = oracle_sample(shape, cpu_sample_tokens(shape), fmt=args.experts_format)
+    fmt = getattr(args, "experts_format", "nvfp4")
+    sample = oracle_sample(shape, cpu_sample_tokens(shape), fmt=fmt)
     for _ in range(args.warmup):
         oracle_step(shape, sample)
     t0 = time.perf_counter()
-    n = sum(oracle_step(shape, sample) for _ in range(args.steps))
+    n = sum(oracle_step(shape, sample)[0] for _ in range(args.steps))
     dt = time.perf_counter() - t0
     value = n / dt
     cores = cpu_cores()
@@ -223,7 +301,7 @@ def run_reference(args, shape, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(shape, fmt=args.experts_format),
+        "config": workload_config(shape, fmt=fmt, world=world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{len(cpu_sample_tokens(shape))} token(s) of the {shape.name} batch per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -231,13 +309,13 @@ def run_reference(args, shape, rank, world):
     emit(line, rank)
 
 
-def workload_config(shape, l2_flush="write", fmt="nvfp4"):
-    l2 = f"flushed: {L2_FLUSH_BYTES >> 20} MiB write between timed steps"
-    if l2_flush == "write+read":
-        l2 = f"flushed: {L2_FLUSH_BYTES >> 20} MiB write + {L2_FLUSH_BYTES >> 21} MiB read between timed steps"
+def workload_config(shape, fmt="nvfp4", world=1):
+    """The workload's config keys; the same for both arms of the measurement."""
     return {"workload": shape.name, "tokens": shape.tokens, "hidden": shape.hidden, "experts": shape.experts,
             "top_k": shape.top_k, "inter": shape.inter, "routing": "zipf-skewed" if shape.skew else "uniform",
-            "experts_format": fmt, "l2": l2}
+            "experts_format": fmt,
+            "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MiB write + {L2_FLUSH_BYTES >> 21} MiB read between timed steps",
+            "parallelism": f"token-dp replicas x{world}"}
 
 
 # ------------------------------------------------------------------ multi-rank plumbing
@@ -266,38 +344,53 @@ def emit(line: dict, rank: int, stream=None) -> bool:
 
 
 # ------------------------------------------------------------------ GPU leg
-def run_ours(args, shape, rank, world, local_rank):
+# The workloads of the metric (T = 16384 / 8 / 1024); the first is the headline of the line.
+DEFAULT_WORKLOADS = ("prefill16k", "decode8", "spec1024")
+
+
+def roofline_of(kern: dict, work: dict, fmt: str, T: int) -> dict:
+    """Roofline of the dominant kernel: algorithmic bytes or FLOPs per launch over its live
+    CUDA-event duration, against the measured (or fallback) peaks."""
+    top = max(kern, key=kern.get)
+    pk = peaks()
+    wk = work[top]
+    # the contraction's own dtype: NVFP4 = 4 x BF16 (nominal 9 / 2.25 PF), FP8 = 2 x (4.5 / 2.25)
+    ratio = 4 if fmt == "nvfp4" else 2
+    name = "NVFP4" if fmt == "nvfp4" else "FP8"
+    if wk["flops"] > 0 and wk["flops"] / max(wk["bytes"], 1) > (ratio * pk["bf16_sus"] * 1e12) / (pk["hbm"] * 1e9):
+        achieved = wk["flops"] / (kern[top] / 1e3) / 1e12
+        burst, sus = ratio * pk["bf16"], ratio * pk["bf16_sus"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s", "frac": achieved / burst,
+                "peak_sustained": sus, "frac_sustained": achieved / sus,
+                "peak_source": f"{name} dense = {ratio} x the {pk['src']} BF16 cuBLAS peak (nominal "
+                               f"{'9' if fmt == 'nvfp4' else '4.5'} / 2.25 PF ratio); burst applies: the kernel runs "
+                               f"ms-long stretches between L2 flushes, not a seconds-long loop at the power cap"}
+    else:
+        achieved = wk["bytes"] / (kern[top] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
+                "peak_source": f"{pk['src']} copy bandwidth"}
+    roof.update(traffic=read_traffic(top if fmt == "nvfp4" else f"{top}_{fmt}", work["_used_experts"], T),
+                kernel=top, kernel_ms=kern[top], algorithmic_bytes=wk["bytes"], algorithmic_flops=wk["flops"])
+    return roof
+
+
+def measure_workload(args, layer, shape, rank, world, dev, flush_l2, want_parity):
+    """Times one workload on an existing layer: K steps with CUDA events on the launching
+    stream (L2 flushed between steps, outside the events), the max over ranks; then the
+    library's per-kernel events in a separate pass, and the host-buffer (e2e) path."""
     import torch
-    import torch.distributed as dist
     import sparse_moe_layer_fp32_b200 as bm
     from sparse_moe_layer_fp32_b200 import synthetic
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
     fmt = args.experts_format
-    weights = synthetic.make_weights(shape, 0, device=dev, fmt=fmt)
-    layer = synthetic.make_layer(shape, weights, fmt=fmt)
-    del weights  # the handle holds its own repacked copy
-    torch.cuda.empty_cache()
+    T = shape.tokens
     x, res = synthetic.make_batch(shape, seed=rank)  # each replica its own batch
     x, res = x.to(dev), res.to(dev)
     out = torch.empty_like(res)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    clean = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.float32, device=dev) if args.l2_flush == "write+read" \
-        else None
-    T = shape.tokens
-
-    def flush_l2():
-        """Between steps, outside the timed region: write a buffer 4x the L2; with
-        write+read, then read another 2x the L2 so the step starts with L2 clean as well
-        as cold (the write-back of the flush's dirty lines is not charged to the step)."""
-        flush.zero_()
-        if clean is not None:
-            clean.sum()
 
     def barrier():
         if world > 1:
+            import torch.distributed as dist
             dist.barrier()
 
     for _ in range(max(args.warmup, 3)):
@@ -308,7 +401,9 @@ def run_ours(args, shape, rank, world, local_rank):
     barrier()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    with ClockSampler(local_rank) as clk:
+    props = torch.cuda.get_device_properties(dev)
+    pci = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    with ClockSampler(dev.index or 0, pci) as clk:
         torch.cuda.synchronize()
         barrier()
         for i in range(args.steps):
@@ -319,16 +414,14 @@ def run_ours(args, shape, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
     launches = layer.launches() * args.steps
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     ms = reduce_max(sum(step_ms) / args.steps, world, dev)
-    value = whole_job_rate(T, world, ms)
     layer.check()
 
     # ---- per-kernel durations (CUDA events inside the library, same stream), separate pass
     layer.profile(True)
     acc = {}
-    reps = max(args.steps, 5)
-    for _ in range(reps):
+    for _ in range(max(args.steps, 5)):
         layer.forward(x, res, out)
         for name, kms in layer.kernel_times():
             acc.setdefault(name, []).append(kms)
@@ -336,25 +429,7 @@ def run_ours(args, shape, rank, world, local_rank):
     layer.profile(False)
     kern = {n: sum(v) / len(v) for n, v in acc.items()}
     offsets = np.frombuffer(layer.debug(bm.BUF_OFFSETS).cpu().numpy().tobytes(), np.int32)
-    counts = np.diff(offsets)
-    work = kernel_work(shape, T, counts, fmt)
-    top = max(kern, key=kern.get)
-    pk = peaks()
-    wk = work[top]
-    # the contraction's own dtype: NVFP4 = 4 x BF16 (nominal 9 / 2.25 PF), FP8 = 2 x (4.5 / 2.25)
-    ratio = 4 if fmt == "nvfp4" else 2
-    if wk["flops"] > 0 and wk["flops"] / max(wk["bytes"], 1) > (ratio * pk["bf16_sus"] * 1e12) / (pk["hbm"] * 1e9):
-        bound, achieved, peak, unit = ("tensor", wk["flops"] / (kern[top] / 1e3) / 1e12, ratio * pk["bf16_sus"],
-                                       "TFLOP/s")
-        peak_note = (f"{'NVFP4' if fmt == 'nvfp4' else 'FP8'} dense = {ratio} x {pk['src']} sustained BF16 cuBLAS "
-                     f"peak (nominal {'9' if fmt == 'nvfp4' else '4.5'} / 2.25 PF ratio)")
-    else:
-        bound, achieved, peak, unit = "hbm", wk["bytes"] / (kern[top] / 1e3) / 1e9, pk["hbm"], "GB/s"
-        peak_note = f"{pk['src']} copy bandwidth"
-    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": read_traffic(top if fmt == "nvfp4" else f"{top}_{fmt}", work["_used_experts"], T),
-                "kernel": top, "kernel_ms": kern[top],
-                "peak_source": peak_note}
+    work = kernel_work(shape, T, np.diff(offsets), fmt)
 
     # ---- end to end through the host-buffer entry point (copies inside the timed region)
     xh = x.cpu().pin_memory()
@@ -374,27 +449,71 @@ def run_ours(args, shape, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)) / args.steps, world, dev)
-    assert torch.equal(oh.to(dev), layer.forward(x, res)), "host-buffer path differs from device path"
+    ref_out = layer.forward(x, res)
+    assert torch.equal(oh.to(dev), ref_out), "host-buffer path differs from device path"
+    gpu = None
+    if want_parity:
+        ids = layer.debug(bm.BUF_IDS).cpu().numpy().view(np.int32).reshape(T, shape.top_k).astype(np.int64)
+        gpu = (ids, ref_out.float().cpu().numpy().astype(np.float64))
+    return {
+        "value": whole_job_rate(T, world, ms), "unit": UNIT, "ms_per_step": ms, "us_per_layer": ms * 1e3,
+        "steps": args.steps, "config": workload_config(shape, fmt, world),
+        "roofline": roofline_of(kern, work, fmt, T), "kernels_ms": kern, "used_experts": work["_used_experts"],
+        "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * T * shape.hidden * 2,
+                "d2h_bytes_per_step": T * shape.hidden * 2},
+        "gpu_launches": launches, "clocks": clk.summary(),
+    }, gpu
 
-    line = None
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": ("nvfp4 (e2m1 x e4m3/16) experts" if fmt == "nvfp4" else "mxfp8 (e4m3 x ue8m0/32) experts")
-                     + ", fp32 router and accumulation",
-            "data": "synthetic (seeded; random-init weights of the layer's shapes)",
-            "config": dict(workload_config(shape, args.l2_flush, fmt), parallelism=f"token-dp replicas x{world}"),
-            "roofline": roofline,
-            "kernels_ms": kern,
-            "used_experts": work["_used_experts"],
-            "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * T * shape.hidden * 2,
-                    "d2h_bytes_per_step": T * shape.hidden * 2},
-            "gpu_launches": launches,
-            "clocks": clk.summary(),
-        }
+
+def run_ours(args, shapes, rank, world, local_rank):
+    """Every workload of `shapes` on one layer (one set of weights, workspace for the
+    largest batch); returns {name: measurement}, each with its parity inputs."""
+    import torch
+    from sparse_moe_layer_fp32_b200 import synthetic
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    fmt = args.experts_format
+    base = shapes[0]
+    key = lambda s: (s.hidden, s.experts, s.top_k, s.inter, s.skew)  # noqa: E731
+    assert all(key(s) == key(base) for s in shapes), "workloads of one run share the layer's shape"
+    weights = synthetic.make_weights(base, 0, device=dev, fmt=fmt)
+    layer = synthetic.make_layer(base, weights, max_tokens=max(s.tokens for s in shapes), fmt=fmt)
+    del weights  # the handle holds its own repacked copy
+    torch.cuda.empty_cache()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        """Between steps, outside the timed region: write a buffer 4x the L2, then read
+        another 2x the L2 so the step starts with L2 cold and clean (the write-back of the
+        flush's dirty lines is not charged to the step)."""
+        flush.zero_()
+        clean.sum()
+
+    want_parity = rank == 0 and world == 1 and not args.no_cpu_baseline
+    results = {}
+    for shape in shapes:
+        results[shape.name] = measure_workload(args, layer, shape, rank, world, dev, flush_l2, want_parity)
     layer.close()
+    return results
+
+
+def compose_line(args, shapes, results, world):
+    """The one JSON line: the headline workload's numbers at the top level, the others under
+    "workloads" with the same keys."""
+    fmt = args.experts_format
+    head = shapes[0].name
+    line = {
+        "metric": METRIC, "n_gpus": world, "warmup": max(args.warmup, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": ("nvfp4 (e2m1 x e4m3/16) experts" if fmt == "nvfp4" else "mxfp8 (e4m3 x ue8m0/32) experts")
+                 + ", fp32 router and accumulation",
+        "data": "synthetic (seeded; random-init weights of the layer's shapes)",
+    }
+    line.update(results[head])
+    if len(shapes) > 1:
+        line["workloads"] = {s.name: results[s.name] for s in shapes[1:]}
     return line
 
 
@@ -513,7 +632,7 @@ def run_tp_shared(args, shape):
         "vs_baseline": None,
         "dtype": ("nvfp4" if fmt == "nvfp4" else "mxfp8") + " experts, fp32 router, accumulation and all-reduce",
         "data": "synthetic (seeded; random-init weights of the layer's shapes)",
-        "config": dict(workload_config(shape, "write+read", fmt),
+        "config": dict(workload_config(shape, fmt),
                        parallelism=f"{'ep' if ep else 'tp'}{W}, ranks sharing one GPU in turn"
                                    + (f", {T} tokens per rank" if ep else "")),
         "estimate": "value = tokens / slowest rank's sum of phases; peers' data read from this GPU's memory, "
@@ -533,7 +652,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode8", choices=sorted(mi.SHAPES))
+    ap.add_argument("--workload", default="default", choices=["default"] + sorted(mi.SHAPES),
+                    help="default: prefill16k (the headline), decode8 and spec1024 in one line")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tp-shared-gpu", type=int, default=0, metavar="W",
@@ -542,19 +662,17 @@ def main():
                     help="expert-parallel layer with W ranks (each its own batch) sharing this one GPU, run in turn")
     ap.add_argument("--experts-format", default="nvfp4", choices=["nvfp4", "mxfp8"],
                     help="routed experts in NVFP4 (default) or the block-scaled FP8 variant (MXFP8)")
-    ap.add_argument("--l2-flush", default="write+read", choices=["write", "write+read"],
-                    help="between timed steps: write 512 MiB, then (default) read 256 MiB so the step starts "
-                         "with L2 cold and clean")
     args = ap.parse_args()
-    shape = mi.SHAPES[args.workload]
+    names = DEFAULT_WORKLOADS if args.workload == "default" else (args.workload,)
+    shapes = [mi.SHAPES[n] for n in names]
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
-        run_reference(args, shape, rank, world)
+        run_reference(args, shapes[0], rank, world)
         return
     if args.tp_shared_gpu or args.ep_shared_gpu:
-        emit(run_tp_shared(args, shape), 0)
+        emit(run_tp_shared(args, shapes[0]), 0)
         return
     if world > 1:
         import datetime
@@ -563,14 +681,17 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, shape, rank, world, local_rank)
+        results = run_ours(args, shapes, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(shape, fmt=args.experts_format)
-    emit(line, rank)
+        for shape in shapes:
+            meas, gpu = results[shape.name]
+            meas["cpu_baseline"], meas["parity"] = cpu_baseline(shape, fmt=args.experts_format, gpu=gpu)
+    results = {n: m for n, (m, _) in results.items()}
+    emit(compose_line(args, shapes, results, world), rank)
 
 
 if __name__ == "__main__":
