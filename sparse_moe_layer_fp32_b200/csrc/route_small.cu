@@ -146,6 +146,10 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     bulk_load(ps, part, bytes, &bars[2]);
   }
   __syncwarp();
+  // thread e's tensor scales of expert e, loaded while the partial logits are in flight
+  const bool held = tid >= bs.e_begin && tid < bs.e_end;  // this handle has the expert's weights
+  const float a_gu = held ? __ldg(bs.w_gu_alpha + (tid - bs.e_begin)) : 0.0f;
+  const float a_d = held ? __ldg(bs.w_d_alpha + (tid - bs.e_begin)) : 0.0f;
   // the expert GEMM launch that follows starts from zeroed scheduler words
   for (int i = tid; i < sched_n; i += kSmallThreads) sched[i] = 0u;
   __shared__ int s_ids[kMaxSmallRouterTokens * 16];
@@ -180,7 +184,6 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
   // ---------------------------------------------------------------- scan and work blocks
   const int cnt = tid < E ? s_cnt[tid] : 0;
   const int nblk = (cnt + 127) / 128;
-  const bool held = tid >= bs.e_begin && tid < bs.e_end;  // this handle has the expert's weights
   int total_rows, total_blk, total_work;
   const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
   const int blk = block_exclusive_scan(nblk, warp_sums, total_blk);
@@ -196,8 +199,8 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
       m.row_begin = off + 128 * i;
       m.rows = min(128, cnt - 128 * i);
       m.sf_block = blk + i;
-      m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + m.expert);
-      m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + m.expert);
+      m.scale_gu = bs.alpha_a1 * a_gu;
+      m.scale_d = bs.alpha_a2 * a_d;
       m.pad[0] = m.pad[1] = 0;
       mblocks[wbase + i] = m;
     }
