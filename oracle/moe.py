@@ -326,40 +326,50 @@ def moe_forward_ep(x_ranks, residual_ranks, router_w, gamma, experts: ExpertCach
                    alpha_a2, world: int, eps=1e-6):
     """The layer with its experts split over `world` expert-parallel ranks, each with its own
     batch (attention data parallelism: [PR] "Status", Attention DP + MegaMoE; [RECIPE]
-    "Overview": 8 of 256 experts).  Rank q holds experts [q E/W, (q+1) E/W).  Dispatch: every
-    rank receives every rank's tokens (all-gather, rank order); rank q routes them all and
-    applies only its experts, giving partial m_q for every token; combine: rank r's output
-    rows are residual_r + RMSNorm(sum_q m_q[its tokens]) * gamma (reduce-scatter, ranks in
-    order).  Returns dict(ids, w, m_parts [world, sum T, H], m, out_pre per rank, out per
-    rank, near_tie)."""
-    if num_experts % world:
-        raise ValueError("the experts must split evenly over the ranks")
-    x = np.concatenate([np.asarray(v, np.float64) for v in x_ranks])
-    t_count, hidden = x.shape
-    logits = router_logits(x, router_w)
-    ids, w, _ = route_topk(logits, top_k)
+    "Overview": 8 of 256 experts).  Rank q holds experts [q E/W, (q+1) E/W).  In order:
+      1. every rank routes its own tokens (steps 1-4) and quantises each of them once (step 6);
+      2. dispatch: the quantised row of slot (t, j) of rank s goes to the rank that holds
+         expert ids_s[t, j]; rank q's rows of expert e are ordered by (source rank, token);
+      3. every rank runs its experts on the rows it received (steps 7-10);
+      4. combine: each output row y goes back to its source rank, into slot (t, j);
+      5. every rank finalizes its own tokens from the returned rows (steps 11-13).
+    Only routed rows travel: no rank routes or quantises another rank's tokens.  Returns dict
+    with, per rank: ids, w, near_tie, y (returned rows [T, k, H]), m, out_pre, out; and
+    counts [world][E] (rows each rank sends to each expert) and received [world] (rows
+    each rank computes)."""
+    if num_experts % world or len(x_ranks) != world:
+        raise ValueError("one batch per rank, and the experts must split evenly over the ranks")
     fmt = experts.fmt
-    a1_packed, a1_sf = quantize_act(x.astype(np.float32), alpha_a1, fmt)
     e_loc = num_experts // world
-    m_parts = np.zeros((world, t_count, hidden), np.float64)
-    for q in range(world):
+    routed = []
+    for xs in x_ranks:  # step 1 on every rank, its own tokens only
+        xs = np.asarray(xs, np.float64)
+        logits = router_logits(xs, router_w)
+        ids, w, _ = route_topk(logits, top_k)
+        a1p, a1s = quantize_act(xs.astype(np.float32), alpha_a1, fmt)
+        routed.append(dict(ids=ids, w=w, near_tie=near_tie_mask(logits, top_k), a1p=a1p, a1s=a1s,
+                           y=np.zeros((xs.shape[0], top_k, xs.shape[1]), np.float64)))
+    counts = np.array([np.bincount(r["ids"].reshape(-1), minlength=num_experts) for r in routed], np.int64)
+    received = np.zeros(world, np.int64)
+    for q in range(world):  # steps 2-4: rank q computes the rows of its experts
         for e in range(q * e_loc, (q + 1) * e_loc):
-            tt, jj = np.nonzero(ids == e)
-            if len(tt) == 0:
+            src, tok, slot = [], [], []
+            for sr, r in enumerate(routed):  # rows ordered by (source rank, token)
+                tt, jj = np.nonzero(r["ids"] == e)
+                src += [sr] * len(tt)
+                tok += list(tt)
+                slot += list(jj)
+            if not src:
                 continue
-            y = expert_forward(a1_packed[tt], a1_sf[tt], alpha_a1, experts.dequantized(e), alpha_a2, fmt)["y"]
-            np.add.at(m_parts[q], tt, w[tt, jj][:, None] * y)
-    m = np.zeros((t_count, hidden), np.float64)
-    for q in range(world):
-        m = m + m_parts[q]
-    rms = np.sqrt(np.mean(m * m, axis=1, keepdims=True) + eps)
-    n = m / rms * np.asarray(gamma, np.float64)[None, :]
-    out_pre, out, begin = [], [], 0
-    for res in residual_ranks:
-        res = np.asarray(res, np.float64)
-        pre = res + n[begin:begin + res.shape[0]]
-        out_pre.append(pre)
-        out.append(bf16_round(pre))
-        begin += res.shape[0]
-    return dict(ids=ids, w=w, near_tie=near_tie_mask(logits, top_k), m_parts=m_parts, m=m, out_pre=out_pre,
-                out=out)
+            a1p = np.concatenate([routed[sr]["a1p"][t][None] for sr, t in zip(src, tok)])
+            a1s = np.concatenate([routed[sr]["a1s"][t][None] for sr, t in zip(src, tok)])
+            y = expert_forward(a1p, a1s, alpha_a1, experts.dequantized(e), alpha_a2, fmt)["y"]
+            received[q] += len(src)
+            for i, (sr, t, j) in enumerate(zip(src, tok, slot)):
+                routed[sr]["y"][t, j] = y[i]
+    ranks = []
+    for r, res in zip(routed, residual_ranks):  # step 5 on every rank
+        pre, out, m = finalize(r["y"], r["w"], res, gamma, eps)
+        ranks.append(dict(ids=r["ids"], w=r["w"], near_tie=r["near_tie"], y=r["y"], m=m, out_pre=pre, out=out))
+    return dict(ranks=ranks, counts=counts, received=received, out_pre=[q["out_pre"] for q in ranks],
+                out=[q["out"] for q in ranks], near_tie=np.concatenate([q["near_tie"] for q in ranks]))

@@ -285,11 +285,13 @@ def test_tensor_parallel_partials_sum_to_the_unsharded_layer():
         moe.shard_dequantized((w_gu, w_d), 0, 3)
 
 
-def test_expert_parallel_partials_sum_to_the_unsharded_layer():
-    # Experts split over W ranks, each rank with its own batch: every token's slots fall in
-    # exactly one rank's expert range, so the ranks' partial m add up to the unsharded m of
-    # the concatenated batch, and each rank's output rows are that layer's rows of its
-    # tokens.  W = 1 is the unsharded layer itself.
+def test_expert_parallel_routed_rows_reproduce_the_unsharded_layer():
+    # Experts split over W ranks, each rank with its own batch; only routed rows travel: each
+    # rank routes and quantises its own tokens, sends each slot's row to the expert's owner
+    # and finalizes its tokens from the rows that come back.  Every token's output is then
+    # the unsharded layer's output for that token (W = 1 is the unsharded layer itself), the
+    # rows each rank computes are its experts' share of all slots, and every rank sends
+    # exactly its tokens' k slots.
     shape, x, res, wr, g, cache = _tiny()
     shape2, x2, res2, _, _, _ = _tiny(seed=5)
     a1s, a2s = np.float32(5.0 / 2688), np.float32(3.0 / 2688)
@@ -300,14 +302,14 @@ def test_expert_parallel_partials_sum_to_the_unsharded_layer():
         xw = xs if world == 2 else ([np.concatenate(xs)] if world == 1 else [x[:2], x[2:], x2[:1], x2[1:3]])
         rw = rs if world == 2 else ([np.concatenate(rs)] if world == 1 else [res[:2], res[2:], res2[:1], res2[1:3]])
         ep = moe.moe_forward_ep(xw, rw, wr, g, cache, shape.experts, shape.top_k, a1s, a2s, world)
-        np.testing.assert_array_equal(ep["ids"], full["ids"])
-        np.testing.assert_allclose(ep["m"], full["m"], rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(np.concatenate([q["ids"] for q in ep["ranks"]]), full["ids"])
+        np.testing.assert_allclose(np.concatenate([q["m"] for q in ep["ranks"]]), full["m"], rtol=0, atol=1e-12)
         np.testing.assert_allclose(np.concatenate(ep["out_pre"]), full["out_pre"], rtol=0, atol=1e-12)
-        # each rank's partial only holds its experts' slots
+        np.testing.assert_array_equal(np.concatenate(ep["out"]), full["out"])
         e_loc = shape.experts // world
-        for q in range(world):
-            own = (full["ids"] // e_loc) == q
-            idle = ~own.any(axis=1)
-            assert np.all(ep["m_parts"][q][idle] == 0)
+        hist = np.bincount(full["ids"].reshape(-1), minlength=shape.experts)
+        np.testing.assert_array_equal(ep["received"], hist.reshape(world, e_loc).sum(1))
+        np.testing.assert_array_equal(ep["counts"].sum(1), [len(v) * shape.top_k for v in xw])
+        np.testing.assert_array_equal(ep["counts"].sum(0), hist)
     with pytest.raises(ValueError):
         moe.moe_forward_ep(xs, rs, wr, g, cache, shape.experts, shape.top_k, a1s, a2s, 3)
