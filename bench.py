@@ -43,6 +43,7 @@ import moe_inputs as mi  # noqa: E402
 METRIC = "moe_layer_tokens_per_s"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 512 << 20  # written between timed steps (L2 is 126 MB)
+TP_TWO_SHOT_MIN_TOKENS = 256  # the library reduces in two steps from this batch on
 
 
 def peaks():
@@ -85,10 +86,12 @@ def kernel_work(shape: mi.LayerShape, T: int, counts: np.ndarray, fmt: str = "nv
     }
 
 
-def read_traffic(kernel: str, used_experts: int, tokens: int):
-    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json), scaled
-    by the experts that received tokens; None when the kernel's source changed since or the
-    batch is outside the regime the capture scales to."""
+def read_traffic(kernel: str, used_experts: int, tokens: int, top_k: int = 8):
+    """DRAM bytes per launch from the committed ncu captures (profiles/traffic.json): for the
+    expert GEMM, weights per used expert (decode capture) plus, above 32 tokens, bytes per
+    routed row (prefill capture); for the per-token kernels, bytes per token (batches of 256
+    tokens or more).  None when the kernel's source changed since the capture or no capture
+    covers the batch."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -99,9 +102,15 @@ def read_traffic(kernel: str, used_experts: int, tokens: int):
     import hashlib
     src = os.path.join(ROOT, "sparse_moe_layer_fp32_b200", "csrc", ent["source"])
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if digest != ent["source_sha256_16"] or tokens > ent.get("applies_up_to_tokens", tokens):
+    if digest != ent["source_sha256_16"]:
         return None
-    return ent["bytes_per_used_expert"] * used_experts
+    if "bytes_per_token" in ent:
+        return ent["bytes_per_token"] * tokens if tokens >= 256 else None
+    if tokens <= ent.get("applies_up_to_tokens", tokens):
+        return ent["bytes_per_used_expert"] * used_experts
+    if "prefill" in ent:
+        return ent["bytes_per_used_expert"] * used_experts + ent["prefill"]["bytes_per_row"] * tokens * top_k
+    return None
 
 
 # ------------------------------------------------------------------ clocks
@@ -370,6 +379,8 @@ def roofline_of(kern: dict, work: dict, fmt: str, T: int) -> dict:
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
                 "peak_source": f"{pk['src']} copy bandwidth"}
     roof.update(traffic=read_traffic(top if fmt == "nvfp4" else f"{top}_{fmt}", work["_used_experts"], T),
+                traffic_source="ncu dram__bytes_read.sum + dram__bytes_write.sum, profiles/traffic.json "
+                               "(captured on a smaller case and scaled by experts used and routed rows)",
                 kernel=top, kernel_ms=kern[top], algorithmic_bytes=wk["bytes"], algorithmic_flops=wk["flops"])
     return roof
 
@@ -529,9 +540,10 @@ def run_tp_shared(args, shape):
     transfer of the exchange (W x T x H x 4 B per rank) is not in the estimate.
 
     With --ep-shared-gpu W instead: the expert-parallel layer (rank r holds experts
-    [r E/W, (r+1) E/W) and its own batch of the workload's T tokens; three phases:
-    dispatch, the rank's experts on the gathered W T tokens, combine + finalize); `value` =
-    W T / the slowest rank's step (weak scaling of the batch)."""
+    [r E/W, (r+1) E/W) and its own batch of the workload's T tokens; four phases: routing of
+    its tokens + count publication, layout + dispatch of the routed rows, its experts on the
+    rows it received + return of the outputs, finalize of its tokens); `value` = W T / the
+    slowest rank's step (weak scaling of the batch)."""
     import dataclasses
     import torch
     import sparse_moe_layer_fp32_b200 as bm
@@ -567,7 +579,7 @@ def run_tp_shared(args, shape):
         x, res = synthetic.make_batch(shape, 0)
         xs, rs = [x] * W, [res] * W
     outs = [torch.empty_like(rs[r]) for r in range(W)]
-    nphase = 3 if ep else 2
+    nphase = tp.EP_PHASES if ep else tp.TP_PHASES
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     clean = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -617,12 +629,21 @@ def run_tp_shared(args, shape):
     pms = [[sum(a.elapsed_time(b) for a, b in ph[r][p]) / args.steps for r in range(W)] for p in range(nphase)]
     rank_ms = [sum(pms[p][r] for p in range(nphase)) for r in range(W)]
     kms = {n: sum(v) / len(v) for n, v in kern.items()}
-    T, H = shape.tokens, shape.hidden
+    T, H, k = shape.tokens, shape.hidden, shape.top_k
     pk = peaks()
-    red_bytes = W * T * H * 4 + 2 * T * H * 2 + H * 2  # per rank: W partials of its T tokens, residual, out
-    part_bytes = T * shape.top_k * H * 2 + (W * T if ep else T) * H * 4  # y rows it holds, its partial m
-    roof = {"bound": "hbm", "kernel": "tp_reduce", "kernel_ms": kms.get("tp_reduce"),
-            "achieved": red_bytes / (kms["tp_reduce"] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s",
+    q = BYTES_PER_VALUE[fmt]
+    if ep:  # dispatch: x read once, each slot's quantised row stored at its expert's rank
+        top, nbytes = "ep_dispatch", T * H * 2 + T * k * H * q
+        exchange = T * k * H * q + T * k * H * 2  # per rank: its rows out, their outputs back
+    elif T >= TP_TWO_SHOT_MIN_TOKENS:  # two-shot: the W partials of the rank's slice, residual, out and row buffer
+        S = -(-T // W)
+        top, nbytes = "tp_reduce", T * H * 4 + 3 * S * H * 2 + H * 2
+        exchange = (W - 1) * S * H * 4 + (T - S) * H * 2  # peers' partials of the slice, peers' rows
+    else:  # one-shot: the W partials of every token, residual, out
+        top, nbytes = "tp_reduce", W * T * H * 4 + 2 * T * H * 2 + H * 2
+        exchange = (W - 1) * T * H * 4
+    roof = {"bound": "hbm", "kernel": top, "kernel_ms": kms.get(top),
+            "achieved": nbytes / (kms[top] / 1e3) / 1e9, "peak": pk["hbm"], "unit": "GB/s",
             "traffic": None, "peak_source": f"{pk['src']} copy bandwidth"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     line = {
@@ -638,8 +659,7 @@ def run_tp_shared(args, shape):
         "estimate": "value = tokens / slowest rank's sum of phases; peers' data read from this GPU's memory, "
                     "so the NVLink transfer of the exchange is not included",
         "tp": {"world": W, "mode": "ep" if ep else "tp", "rank_ms": rank_ms, "phase_ms": pms,
-               "phase0_ms": pms[0], "phase1_ms": pms[1],
-               "exchange_bytes_per_rank": W * T * H * 4, "tp_partial_bytes": part_bytes},
+               "exchange_bytes_per_rank": exchange},
         "kernels_ms": kms, "roofline": roof, "gpu_launches": sum(lay.launches() for lay in layers),
         "clocks": clk.summary(),
     }

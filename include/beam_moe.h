@@ -116,8 +116,7 @@ typedef struct {
 
 /* beam_moe_create for MXFP8 experts.  cfg->alpha_a1 and cfg->alpha_a2 are not used (MX
  * activations have no tensor scale).  Same shape limits, ownership, synchronisation and
- * errors as beam_moe_create.  Every other entry point takes the handle unchanged; the
- * CTA-pair expert GEMM is NVFP4 only (beam_moe_set_gemm_mode(PAIR) returns UNSUPPORTED). */
+ * errors as beam_moe_create.  Every other entry point takes the handle unchanged. */
 BEAM_MOE_API beam_moe_status beam_moe_create_mxfp8(const beam_moe_config* cfg, const beam_moe_weights_mxfp8* weights,
                                                    void* stream, beam_moe_t* out);
 
@@ -164,15 +163,20 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_h
  * (the tensor scales of the whole tensors unchanged; I / W must meet create's limits).
  * Router weights and gamma are the full ones on every rank.  Then, once per group:
  *   1. beam_moe_tp_region: the handle allocates its exchange region (device memory it owns:
- *      a flag header plus two [max_tokens][H] FP32 buffers) and returns its address;
+ *      a flag header, two [max_tokens][H] FP32 buffers and one [max_tokens][H] BF16 buffer)
+ *      and returns its address;
  *   2. the ranks exchange the regions (beam_moe_ipc_export / beam_moe_ipc_import across
  *      processes, or plain pointers when the ranks share a process and a GPU);
  *   3. beam_moe_tp_attach with every rank's region, in rank order.
  * beam_moe_forward_tp then computes out on every rank (identical bits on all ranks): the
  * routing, A1 and the expert GEMMs of the rank's slice, its partial m, the exchange, and
- * the post-RMSNorm + residual of the summed m.  Every rank must call it the same number of
- * times, with the same num_tokens, like a collective.  A rank that waits more than 2 s for
- * its peers gives up: beam_moe_check then returns BEAM_MOE_ERR_TIMEOUT. */
+ * the post-RMSNorm + residual of the summed m.  Below 256 tokens the all-reduce is one-shot
+ * (every rank reads all W partials of every token); from 256 tokens on it is two-shot: rank r
+ * reduces and finishes only tokens [r S, (r + 1) S), S = ceil(T / W), publishes those BF16
+ * rows in its region, and then copies the other ranks' rows into out (T H 4 + T H 2 bytes
+ * read per rank instead of W T H 4).  Both forms give the same bits.  Every rank must call it
+ * the same number of times, with the same num_tokens, like a collective.  A rank that waits
+ * more than 2 s for its peers gives up: beam_moe_check then returns BEAM_MOE_ERR_TIMEOUT. */
 #define BEAM_MOE_IPC_HANDLE_BYTES 64
 BEAM_MOE_API int64_t beam_moe_tp_region_bytes(beam_moe_t h);
 /* Allocates the region on the first call (synchronises the device); *region gets its
@@ -187,11 +191,14 @@ BEAM_MOE_API beam_moe_status beam_moe_tp_attach(beam_moe_t h, int32_t rank, int3
  * residual).  Enqueued on `stream`; the exchange waits on the device, not the host. */
 BEAM_MOE_API beam_moe_status beam_moe_forward_tp(beam_moe_t h, const void* x, const void* residual, void* out,
                                                  int32_t num_tokens, void* stream);
-/* beam_moe_forward_tp in two halves: phase 0 = routing, GEMMs, this rank's partial m and its
- * publication; phase 1 = the wait for every rank's partials, their sum, norm and residual.
- * Phases alternate (0, 1, 0, 1, ...) with the same num_tokens.  Splitting lets ranks that
- * share one GPU run every rank's phase 0 before any phase 1, so no kernel waits on a kernel
- * that has not run. */
+/* beam_moe_forward_tp in three parts: phase 0 = routing, GEMMs, this rank's partial m and
+ * its publication; phase 1 = the wait for every rank's partials, their sum, norm and residual
+ * (of every token, or of this rank's slice in the two-shot form, then published); phase 2 =
+ * the two-shot form's wait for every rank's rows and their copy into out (nothing is
+ * enqueued in the one-shot form).  Phases run in order (0, 1, 2, 0, ...) with the same
+ * num_tokens; phase 1 and 2 need residual and out.  Splitting lets ranks that share one GPU
+ * run every rank's phase p before any phase p + 1, so no kernel waits on a kernel that has
+ * not run. */
 BEAM_MOE_API beam_moe_status beam_moe_forward_tp_phase(beam_moe_t h, const void* x, const void* residual, void* out,
                                                        int32_t num_tokens, int32_t phase, void* stream);
 /* cudaIpcGetMemHandle / cudaIpcOpenMemHandle / cudaIpcCloseMemHandle of a region, as
@@ -203,22 +210,28 @@ BEAM_MOE_API beam_moe_status beam_moe_ipc_close(void* dev_ptr);
 
 /* ---- Expert parallelism with attention data parallelism (vLLM PR "Day-0 support for
  * Reflection's Beam-1.0", section "Status": Attention DP with the MegaMoE kernels; recipe,
- * "Overview": 8 of 256 experts).  Each of W ranks holds experts [expert_begin,
- * expert_begin + expert_count) (cfg->num_experts = all E, used for routing; the weight
- * arrays and the tensor scales hold only the rank's experts, in order) and its own batch of
- * num_tokens tokens, the same num_tokens on every rank.  cfg->max_tokens bounds the
- * gathered batch: W * num_tokens.  beam_moe_forward_ep:
- *   phase 0, dispatch: the rank's x rows go to every rank (peer stores into the ranks'
- *            regions, rank order), then a delivery flag;
- *   phase 1: wait for every rank's tokens, route all W * num_tokens of them (the same
- *            result on every rank), run this rank's experts on the rows routed to them,
- *            publish the partial m of every token;
- *   phase 2, combine: out = residual + RMSNorm(sum over ranks of the partial m of this
- *            rank's tokens) * gamma, for this rank's num_tokens rows.
+ * "Overview": 8 of 256 experts; "Launching the server": expert parallel with data-parallel
+ * attention).  Each of W ranks holds experts [expert_begin, expert_begin + expert_count)
+ * with expert_begin = rank * expert_count and expert_count * W = E (cfg->num_experts = all
+ * E, used for routing; the weight arrays and the tensor scales hold only the rank's
+ * experts, in order) and its own batch of num_tokens tokens, the same num_tokens on every
+ * rank; cfg->max_tokens bounds W * num_tokens.  Only routed rows travel.
+ * beam_moe_forward_ep, in four phases:
+ *   0  route the rank's own tokens; publish its per-expert row counts to every rank;
+ *   1  wait for every rank's counts and derive the common layout (each rank's received rows,
+ *      expert-major, within an expert by source rank then token); quantise each own token
+ *      once and store each slot's row into the activation tiles of its expert's rank (peer
+ *      stores), adding it to that block's arrival count;
+ *   2  the expert GEMMs over the rows this rank received (a block's gate/up tiles start as
+ *      soon as all its rows have arrived), then every output row back to its source slot
+ *      (peer stores) and a return flag;
+ *   3  wait for every rank's return flag; finalize the rank's own tokens from the returned
+ *      rows (slot order, this rank's routing weights).
+ * Each token's output is bit-identical to the single-GPU forward of the same tokens.
  * Regions, exchange and attach as for tensor parallelism (beam_moe_tp_region /
- * beam_moe_ipc_* / beam_moe_tp_attach); beam_moe_forward and beam_moe_forward_tp refuse
- * these handles (INVALID_ARG).  Dispatch moves whole BF16 rows to every rank (an all-gather)
- * rather than only the k routed rows to their experts' ranks. */
+ * beam_moe_ipc_* / beam_moe_tp_attach; attach checks the expert ranges);
+ * beam_moe_forward and beam_moe_forward_tp refuse these handles (INVALID_ARG).  A rank that
+ * waits more than 2 s for its peers gives up: beam_moe_check then returns TIMEOUT. */
 BEAM_MOE_API beam_moe_status beam_moe_create_ep(const beam_moe_config* cfg, const beam_moe_weights* weights,
                                                 int32_t expert_begin, int32_t expert_count, void* stream,
                                                 beam_moe_t* out);
@@ -229,8 +242,9 @@ BEAM_MOE_API beam_moe_status beam_moe_create_ep_mxfp8(const beam_moe_config* cfg
  * rank calls it the same number of times with the same num_tokens. */
 BEAM_MOE_API beam_moe_status beam_moe_forward_ep(beam_moe_t h, const void* x, const void* residual, void* out,
                                                  int32_t num_tokens, void* stream);
-/* One phase (0, 1, 2, in turn) of beam_moe_forward_ep, so that ranks sharing one GPU can run
- * every rank's phase p before any rank's phase p + 1. */
+/* One phase (0, 1, 2, 3, in turn, the same num_tokens) of beam_moe_forward_ep, so that ranks
+ * sharing one GPU can run every rank's phase p before any rank's phase p + 1; any other
+ * order returns INVALID_ARG. */
 BEAM_MOE_API beam_moe_status beam_moe_forward_ep_phase(beam_moe_t h, const void* x, const void* residual, void* out,
                                                        int32_t num_tokens, int32_t phase, void* stream);
 
@@ -323,17 +337,6 @@ BEAM_MOE_API beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, vo
 /* Synchronises `stream`, then reads and clears the device error word.  Returns OK,
  * TIMEOUT or DEVICE. */
 BEAM_MOE_API beam_moe_status beam_moe_check(beam_moe_t h, void* stream);
-
-/* Expert GEMM variant for the batches that do not use the small-batch routing (more than
- * 16 tokens; NVFP4 handles).  SINGLE: one CTA per 128-row work block.  PAIR: CTA pairs (clusters of two
- * SMs sharing one M = 256 MMA) over 256-row work blocks.  AUTO (the default at create)
- * picks PAIR from BEAM_MOE_PAIR_MIN_TOKENS tokens on, SINGLE below; the threshold is set
- * where PAIR measured faster (INT32_MAX: never).  Both compute the same result up to the
- * FP32 rounding of the accumulation order.  Not from the source pages: an implementation
- * choice exposed for testing and tuning.  Returns INVALID_ARG for an unknown mode. */
-enum { BEAM_MOE_GEMM_AUTO = 0, BEAM_MOE_GEMM_SINGLE = 1, BEAM_MOE_GEMM_PAIR = 2 };
-#define BEAM_MOE_PAIR_MIN_TOKENS 2147483647
-BEAM_MOE_API beam_moe_status beam_moe_set_gemm_mode(beam_moe_t h, int32_t mode);
 
 /* Router for batches of more than 16 tokens (16 or fewer use the fused small-batch routing
  * kernel).  SIMT: FP32 FFMA over slices of H, then a top-k kernel that sums the slices.

@@ -25,7 +25,7 @@ EXPORTED = [
     "beam_moe_route_workspace_bytes", "beam_moe_quantize_nvfp4", "beam_moe_debug_copy", "beam_moe_check",
     "beam_moe_last_launch_count", "beam_moe_status_string", "beam_moe_destroy", "beam_moe_profile_enable",
     "beam_moe_profile_read", "beam_moe_kernel_name", "beam_moe_route_static", "beam_moe_debug_wait_timeout",
-    "beam_moe_forward_prenorm", "beam_moe_set_gemm_mode", "beam_moe_create_mxfp8", "beam_moe_quantize_mxfp8",
+    "beam_moe_forward_prenorm", "beam_moe_create_mxfp8", "beam_moe_quantize_mxfp8",
     "beam_moe_expert_format", "beam_moe_tp_region_bytes", "beam_moe_tp_region", "beam_moe_tp_attach",
     "beam_moe_forward_tp", "beam_moe_forward_tp_phase", "beam_moe_ipc_export", "beam_moe_ipc_import",
     "beam_moe_ipc_close", "beam_moe_create_ep", "beam_moe_create_ep_mxfp8", "beam_moe_forward_ep",
@@ -77,7 +77,6 @@ def _load():
         "beam_moe_status_string": (ctypes.c_char_p, [i32]),
         "beam_moe_destroy": (None, [vp]),
         "beam_moe_profile_enable": (i32, [vp, i32]),
-        "beam_moe_set_gemm_mode": (i32, [vp, i32]),
         "beam_moe_set_router_mode": (i32, [vp, i32]),
         "beam_moe_profile_read": (i32, [vp, ctypes.POINTER(f32), i32, ctypes.POINTER(i32)]),
         "beam_moe_kernel_name": (ctypes.c_char_p, [vp, i32]),
@@ -296,18 +295,11 @@ def beam_moe_debug_wait_timeout(h, limit_ns: int, stream=None):
     _check(_lib.beam_moe_debug_wait_timeout(h, int(limit_ns), _stream(stream)), "beam_moe_debug_wait_timeout")
 
 
-GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
-
-
 ROUTER_AUTO, ROUTER_SIMT, ROUTER_TENSOR = 0, 1, 2
 
 
 def beam_moe_set_router_mode(h, mode: int):
     _check(_lib.beam_moe_set_router_mode(h, int(mode)), "beam_moe_set_router_mode")
-
-
-def beam_moe_set_gemm_mode(h, mode: int):
-    _check(_lib.beam_moe_set_gemm_mode(h, int(mode)), "beam_moe_set_gemm_mode")
 
 
 def beam_moe_profile_enable(h, enable: bool = True):
@@ -410,9 +402,6 @@ class MoELayer:
 
     def set_router_mode(self, mode: int):
         beam_moe_set_router_mode(self.handle, mode)
-
-    def set_gemm_mode(self, mode: int):
-        beam_moe_set_gemm_mode(self.handle, mode)
 
     def kernel_times(self):
         return beam_moe_profile_read(self.handle)

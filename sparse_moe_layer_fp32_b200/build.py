@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbeam_moe.so")
-SOURCES = ["beam_moe.cu", "router.cu", "routing.cu", "quant.cu", "gemm_experts.cu", "finalize.cu", "route_static.cu", "route_small.cu", "router_tc.cu", "finalize_tp.cu"]
+SOURCES = ["beam_moe.cu", "router.cu", "routing.cu", "quant.cu", "gemm_experts.cu", "finalize.cu", "route_static.cu", "route_small.cu", "router_tc.cu", "finalize_tp.cu", "expert_parallel.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

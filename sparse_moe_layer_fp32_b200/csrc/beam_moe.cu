@@ -36,7 +36,6 @@ struct beam_moe_ctx {
   uint32_t* err;
   unsigned int* route_counter;  // last-CTA election of the fused small-batch routing kernel
   uint32_t* sched;              // tile scheduler of the expert GEMM launch (sched_words(nblk_max))
-  int32_t gemm_mode;            // BEAM_MOE_GEMM_*: which expert GEMM large batches use
   int32_t router_mode;          // BEAM_MOE_ROUTER_*: which router batches of more than 16 tokens use
   int32_t fmt;                  // BEAM_MOE_FMT_*: expert weight and activation format
   int kv;                       // K values per activation / weight tile: 256 (NVFP4), 128 (MXFP8)
@@ -51,16 +50,21 @@ struct beam_moe_ctx {
   uint8_t** tp_regions_dev;     // device array [kMaxTpRanks]: every rank's region
   TpGroup tp;                   // every rank's region, this rank, the group size
   bool tp_attached;
-  bool tp_pending;              // phase 0 ran, phase 1 not yet
+  int tp_next_phase;            // the phase of beam_moe_forward_tp_phase that may run next (0..2)
+  bool tp_two_shot;             // the forward in flight reduces in two steps (its T >= kTpTwoShotMinTokens)
   uint32_t tp_epoch;            // forwards so far in this group (the flag value of the last one)
-  unsigned int* tp_counter;     // CTA arrivals of tp_partial
+  unsigned int* tp_counter;     // CTA arrivals of tp_partial [0] and of the two-shot tp_reduce [1]
   int tp_last_T;
   // expert parallelism (beam_moe_create_ep*): this handle holds experts [e_begin, e_begin + e_count)
   int e_begin, e_count;
   bool ep;
-  bool ep_dispatched;           // phase 0 ran, phase 1 not yet
+  int ep_next_phase;            // the phase of beam_moe_forward_ep_phase that may run next (0..3)
   int ep_T;                     // this rank's tokens in the current forward
-  unsigned int* ep_counter;     // CTA arrivals of ep_dispatch
+  unsigned int* ep_counter;     // CTA arrivals of ep_combine
+  EpLayout ep_lay;              // this rank's region (the same layout on every rank)
+  EpDest* ep_dst;               // [E]: where this rank's rows of each expert go
+  int32_t* ep_own_rows;         // rows this rank received in the current forward
+  int32_t* inv_identity;        // [max_tokens k]: i, the returned rows' slot order
   int last_T;
   int last_splits;  // logits layout of the last forward: [splits][T][E] partial sums
   int last_launches;
@@ -241,7 +245,6 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   h->last_splits = 1;
   h->last_launches = 0;
   h->profiling = false;
-  h->gemm_mode = BEAM_MOE_GEMM_AUTO;
   h->router_mode = BEAM_MOE_ROUTER_AUTO;
   h->profiled_last = false;
   for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i) {
@@ -340,6 +343,34 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   CREATE_TRY(cudaMemsetAsync(h->a2_sf, 0, act_sf_bytes(h, Ip), s));
   CREATE_TRY(cudaMemsetAsync(h->a1_sf, 0, act_sf_bytes(h, H), s));
   CREATE_TRY(cudaMemsetAsync(h->err, 0, sizeof(uint32_t), s));
+  if (ep) {
+    if (E > 1024 || R >= (1ll << 24)) return fail(cudaErrorInvalidValue);  // the layout's limits
+    CREATE_TRY(dalloc(h, &h->ep_dst, sizeof(EpDest) * E));
+    CREATE_TRY(dalloc(h, &h->ep_own_rows, sizeof(int32_t)));
+    CREATE_TRY(dalloc(h, &h->inv_identity, sizeof(int32_t) * R));
+    std::vector<int32_t> iota(static_cast<size_t>(R));
+    for (int64_t i = 0; i < R; ++i) iota[i] = static_cast<int32_t>(i);
+    CREATE_TRY(cudaMemcpy(h->inv_identity, iota.data(), sizeof(int32_t) * R, cudaMemcpyHostToDevice));
+    // the region: flag header, count matrix, arrival counters, origins, received activation
+    // tiles and scales, returned rows
+    size_t off = kTpHeaderBytes;
+    auto take = [&](size_t bytes, size_t align) {
+      off = (off + align - 1) / align * align;
+      const size_t at = off;
+      off += bytes;
+      return at;
+    };
+    EpLayout& lay = h->ep_lay;
+    lay.nblk = static_cast<int>(h->nblk_max);
+    lay.rows = static_cast<int>(R);
+    lay.counts = take(sizeof(int32_t) * kMaxTpRanks * E, 256);
+    lay.arrivals = take(sizeof(uint32_t) * lay.nblk, 256);
+    lay.origin = take(sizeof(int32_t) * R, 256);
+    lay.a1 = take(act_bytes(h, H), 1024);
+    lay.a1_sf = take(act_sf_bytes(h, H), 1024);
+    lay.ret = take(sizeof(uint16_t) * static_cast<size_t>(R) * H, 1024);
+    lay.bytes = (off + 255) / 256 * 256;
+  }
 
   CREATE_TRY(cudaStreamSynchronize(s));
   CREATE_TRY(cudaGetLastError());
@@ -409,20 +440,21 @@ beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num
 }
 
 // tp_phase: -1 the single-GPU forward; 0 the tensor-parallel forward up to the partial sums
-// and their publication (tp_partial instead of finalize); 1 only the all-reduce + finalize
-// (tp_reduce) of the last phase 0.
+// and their publication (tp_partial instead of finalize); 1 the all-reduce + finalize
+// (tp_reduce) of the last phase 0: of every token (one-shot) or of this rank's slice
+// (two-shot); 2 the gather of the other slices (two-shot; nothing in the one-shot form).  ep_phase (expert-parallel handles, tp_phase -1): 0 the
+// routing of this rank's tokens and the count publication; 1 the layout and the dispatch; 2
+// the expert GEMMs over the received rows and the combine; 3 the finalize of the returned
+// rows (see expert_parallel.cu).
 static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* residual, void* out, void* next_x,
                                     const void* next_gamma, float next_eps, int32_t num_tokens, void* stream,
-                                    int tp_phase = -1, cudaEvent_t residual_ready = nullptr, int tok_off = 0,
-                                    bool ep_gathered = false) {
+                                    int tp_phase = -1, cudaEvent_t residual_ready = nullptr, int ep_phase = -1) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;
-  if (tp_phase < 0 && h->ep) return BEAM_MOE_ERR_INVALID_ARG;  // holds only some experts: beam_moe_forward_ep
+  if (tp_phase < 0 && h->ep && ep_phase < 0) return BEAM_MOE_ERR_INVALID_ARG;  // holds only some experts
   if (tp_phase >= 0) {
-    if (!h->tp_attached) return BEAM_MOE_ERR_INVALID_ARG;
-    if (tp_phase == 1 && (!h->tp_pending || tok_off < 0 || tok_off + num_tokens > h->tp_last_T ||
-                          (!h->ep && num_tokens != h->tp_last_T)))
-      return BEAM_MOE_ERR_INVALID_ARG;
-    if (tp_phase == 0 && h->tp_pending) return BEAM_MOE_ERR_INVALID_ARG;  // phases must alternate
+    if (!h->tp_attached || h->ep) return BEAM_MOE_ERR_INVALID_ARG;
+    if (tp_phase != h->tp_next_phase) return BEAM_MOE_ERR_INVALID_ARG;  // phases in order
+    if (tp_phase > 0 && num_tokens != h->tp_last_T) return BEAM_MOE_ERR_INVALID_ARG;
   }
   if (num_tokens < 0 || num_tokens > h->Tmax) return BEAM_MOE_ERR_INVALID_ARG;
   if (num_tokens == 0) {
@@ -445,27 +477,97 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     return cudaEventRecord(h->events[launches + 1], s);
   };
   if (prof) BEAM_TRY(cudaEventRecord(h->events[0], s));
-  if (tp_phase == 1) {
-    BEAM_TRY(launch_tp_reduce(static_cast<const uint16_t*>(residual), h->gamma, T, tok_off, H, h->cfg.rms_eps, h->tp,
-                              h->tp_epoch, static_cast<uint16_t*>(out), h->err, s));
-    BEAM_TRY(mark("tp_reduce"));
-    ++launches;
-    h->tp_pending = false;
+  auto finish = [&]() {
+    h->last_T = T;
     h->last_launches = launches;
     h->profiled_last = prof;
     return BEAM_MOE_OK;
+  };
+  if (tp_phase == 1) {
+    BEAM_TRY(launch_tp_reduce(static_cast<const uint16_t*>(residual), h->gamma, T, h->tp_two_shot, H, h->cfg.rms_eps,
+                              h->tp, h->tp_epoch, static_cast<uint16_t*>(out), h->err, h->tp_counter + 1, s));
+    BEAM_TRY(mark("tp_reduce"));
+    ++launches;
+    h->tp_next_phase = 2;
+    return finish();
+  }
+  if (tp_phase == 2) {
+    if (h->tp_two_shot) {
+      BEAM_TRY(launch_tp_gather(T, H, h->tp, h->tp_epoch, static_cast<uint16_t*>(out), h->err, 4 * h->num_sms, s));
+      BEAM_TRY(mark("tp_gather"));
+      ++launches;
+    }
+    h->tp_next_phase = 0;
+    return finish();
   }
   const BlockScales bscales{h->w_gu_alpha, h->w_d_alpha, h->cfg.alpha_a1, h->cfg.alpha_a2, h->e_begin,
                             h->e_begin + h->e_count};
-  if (ep_gathered) {  // x is the gathered-token buffer: wait until every rank delivered
-    BEAM_TRY(launch_ep_wait(h->tp, h->tp_epoch + 1, h->err, s));
+  const bool mx = h->fmt == BEAM_MOE_FMT_MXFP8;
+  // The expert GEMMs' arguments over a block list (this forward's, or the received rows')
+  auto gemm_args = [&](const uint8_t* a1, const uint8_t* a1_sf, int max_rows, const uint32_t* arrivals) {
+    ExpertGemmArgs g{};
+    g.mblocks = h->mblocks;
+    g.num_mblocks = h->num_mblocks;
+    g.max_rows_per_expert = max_rows;
+    g.gu_n_tiles = h->I / 128;
+    g.gu_k_tiles = H / h->kv;
+    g.a1 = a1;
+    g.a1_sf = a1_sf;
+    g.w_gu = h->w_gu_tiles;
+    g.a2 = h->a2;
+    g.a2_sf = h->a2_sf;
+    g.alpha_a2 = h->cfg.alpha_a2;
+    g.d_n_tiles = H / 256;
+    g.d_k_tiles = h->Ip / h->kv;
+    g.w_d = h->w_d_tiles;
+    g.y = h->y;
+    g.y_cols = H;
+    g.sched = h->sched;
+    g.err = h->err;
+    g.arrivals = arrivals;
+    return g;
+  };
+  if (ep_phase >= 1) {
+    const uint32_t epoch = h->tp_epoch + 1;  // the forward in flight
+    uint8_t* region = h->tp_region;
+    if (ep_phase == 1) {
+      BEAM_TRY(launch_ep_layout(h->tp, h->ep_lay, E, bscales, h->mblocks, h->num_mblocks, h->sched,
+                                static_cast<int>(sched_words(h->nblk_max)), h->ep_dst, h->ep_own_rows, epoch, h->err,
+                                s));
+      BEAM_TRY(mark("ep_layout"));
+      ++launches;
+      BEAM_TRY(launch_ep_dispatch(xb, h->ids, h->inv, h->offsets, h->ep_dst, T, H, k, h->fmt, h->cfg.alpha_a1, h->tp,
+                                  h->ep_lay, s));
+      BEAM_TRY(mark("ep_dispatch"));
+      ++launches;
+      return finish();
+    }
+    if (ep_phase == 2) {
+      const ExpertGemmArgs g = gemm_args(region + h->ep_lay.a1, region + h->ep_lay.a1_sf, T * h->tp.world,
+                                         reinterpret_cast<const uint32_t*>(region + h->ep_lay.arrivals));
+      if (mx)
+        BEAM_TRY(launch_gemm_experts_mx(g, h->num_sms, s));
+      else
+        BEAM_TRY(launch_gemm_experts(g, h->num_sms, s));
+      BEAM_TRY(mark("gemm_experts"));
+      ++launches;
+      BEAM_TRY(launch_ep_combine(h->y, h->ep_own_rows, H, h->tp, h->ep_lay, epoch, h->ep_counter, 4 * h->num_sms, s));
+      BEAM_TRY(mark("ep_combine"));
+      ++launches;
+      return finish();
+    }
+    // phase 3: this rank's tokens from their returned rows, in slot order
+    BEAM_TRY(launch_ep_wait_returned(h->tp, epoch, h->err, s));
     BEAM_TRY(mark("ep_wait"));
     ++launches;
+    BEAM_TRY(launch_finalize(reinterpret_cast<const uint16_t*>(region + h->ep_lay.ret), h->w, h->inv_identity,
+                             static_cast<const uint16_t*>(residual), h->gamma, T, H, k, h->cfg.rms_eps,
+                             static_cast<uint16_t*>(out), nullptr, nullptr, 0.0f, h->err, s));
+    BEAM_TRY(mark("finalize"));
+    ++launches;
+    h->tp_epoch = epoch;
+    return finish();
   }
-  // CTA pairs for the expert GEMM when the average expert has a few hundred rows
-  const bool mx = h->fmt == BEAM_MOE_FMT_MXFP8;
-  const bool pair = !mx && !route_small_supported(T, H, E, k) &&
-                    (h->gemm_mode == BEAM_MOE_GEMM_PAIR || (h->gemm_mode == BEAM_MOE_GEMM_AUTO && T >= kPairMinTokens));
   if (route_small_supported(T, H, E, k)) {
     // router + top-k + histogram + scan + permutation in one launch
     int slices = 1;
@@ -516,14 +618,19 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     BEAM_TRY(mark("chunk_hist"));
     ++launches;
     BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
-                         h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), bscales,
-                         pair ? 1 : 0, s));
+                         h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), bscales, s));
     BEAM_TRY(mark("scan"));
     ++launches;
     BEAM_TRY(launch_scatter(h->ids, h->chunk_base, h->offsets, h->sf_block, T, k, E, h->perm, h->inv, h->tile_row,
                             s));
     BEAM_TRY(mark("scatter"));
     ++launches;
+  }
+  if (ep_phase == 0) {  // this rank's per-expert row counts to every rank
+    BEAM_TRY(launch_ep_counts(h->offsets, E, h->tp, h->ep_lay, h->tp_epoch + 1, s));
+    BEAM_TRY(mark("ep_counts"));
+    ++launches;
+    return finish();
   }
   if (mx)
     BEAM_TRY(launch_quant_a1_mx(xb, h->tile_row, T, H, k, h->a1, h->a1_sf, s));
@@ -532,29 +639,10 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   BEAM_TRY(mark("quant_a1"));
   ++launches;
 
-  ExpertGemmArgs g{};
-  g.mblocks = h->mblocks;
-  g.num_mblocks = h->num_mblocks;
-  g.max_rows_per_expert = T;  // a token chooses an expert at most once
-  g.gu_n_tiles = h->I / 128;
-  g.gu_k_tiles = H / h->kv;
-  g.a1 = h->a1;
-  g.a1_sf = h->a1_sf;
-  g.w_gu = h->w_gu_tiles;
-  g.a2 = h->a2;
-  g.a2_sf = h->a2_sf;
-  g.alpha_a2 = h->cfg.alpha_a2;
-  g.d_n_tiles = H / 256;
-  g.d_k_tiles = h->Ip / h->kv;
-  g.w_d = h->w_d_tiles;
-  g.y = h->y;
-  g.y_cols = H;
-  g.sched = h->sched;
-  g.err = h->err;
+  // a token chooses an expert at most once: at most T rows per expert
+  const ExpertGemmArgs g = gemm_args(h->a1, h->a1_sf, T, nullptr);
   if (mx)
     BEAM_TRY(launch_gemm_experts_mx(g, h->num_sms, s));
-  else if (pair)
-    BEAM_TRY(launch_gemm_experts_pair(g, h->num_sms, s));
   else
     BEAM_TRY(launch_gemm_experts(g, h->num_sms, s));
   BEAM_TRY(mark("gemm_experts"));
@@ -565,7 +653,8 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     BEAM_TRY(mark("tp_partial"));
     ++launches;
     ++h->tp_epoch;
-    h->tp_pending = true;
+    h->tp_next_phase = 1;
+    h->tp_two_shot = h->tp.world > 1 && T >= kTpTwoShotMinTokens;
     h->tp_last_T = T;
   } else {
     if (residual_ready) BEAM_TRY(cudaStreamWaitEvent(s, residual_ready, 0));
@@ -599,9 +688,10 @@ beam_moe_status beam_moe_forward_prenorm(beam_moe_t h, const void* x, const void
 
 int64_t beam_moe_tp_region_bytes(beam_moe_t h) {
   if (!h) return 0;
+  if (h->ep) return static_cast<int64_t>(h->ep_lay.bytes);
   const int64_t part = 2ll * h->Tmax * h->H * static_cast<int64_t>(sizeof(float));
-  const int64_t gathered = h->ep ? 2ll * h->Tmax * h->H * static_cast<int64_t>(sizeof(uint16_t)) : 0;
-  return static_cast<int64_t>(kTpHeaderBytes) + part + gathered;
+  const int64_t rows = static_cast<int64_t>(h->Tmax) * h->H * static_cast<int64_t>(sizeof(uint16_t));
+  return static_cast<int64_t>(kTpHeaderBytes) + part + rows;
 }
 
 beam_moe_status beam_moe_tp_region(beam_moe_t h, void** region) {
@@ -614,12 +704,17 @@ beam_moe_status beam_moe_tp_region(beam_moe_t h, void** region) {
     uint8_t** table = nullptr;
     unsigned int *tp_counter = nullptr, *ep_counter = nullptr;
     BEAM_TRY(dalloc(h, &region, bytes));
-    BEAM_TRY(dalloc(h, &tp_counter, sizeof(unsigned int)));
+    BEAM_TRY(dalloc(h, &tp_counter, 2 * sizeof(unsigned int)));
     BEAM_TRY(dalloc(h, &table, sizeof(uint8_t*) * kMaxTpRanks));
     BEAM_TRY(dalloc(h, &ep_counter, sizeof(unsigned int)));
     BEAM_TRY(cudaMemset(ep_counter, 0, sizeof(unsigned int)));
     BEAM_TRY(cudaMemset(region, 0, kTpHeaderBytes));
-    BEAM_TRY(cudaMemset(tp_counter, 0, sizeof(unsigned int)));
+    if (h->ep) {  // the scales of received blocks' unused rows read as zero
+      BEAM_TRY(cudaMemset(region + h->ep_lay.a1_sf, 0, act_sf_bytes(h, h->H)));
+      BEAM_TRY(cudaMemset(region + h->ep_lay.arrivals, 0, sizeof(uint32_t) * h->ep_lay.nblk));
+      BEAM_TRY(cudaMemset(region + h->ep_lay.origin, 0xFF, sizeof(int32_t) * h->ep_lay.rows));  // no source yet
+    }
+    BEAM_TRY(cudaMemset(tp_counter, 0, 2 * sizeof(unsigned int)));
     BEAM_TRY(cudaDeviceSynchronize());
     h->tp_region = region;
     h->tp_counter = tp_counter;
@@ -635,8 +730,13 @@ beam_moe_status beam_moe_tp_attach(beam_moe_t h, int32_t rank, int32_t world, vo
   if (!h->tp_region || regions[rank] != h->tp_region) return BEAM_MOE_ERR_INVALID_ARG;
   for (int q = 0; q < world; ++q)
     if (!regions[q] || !aligned(regions[q], 256)) return BEAM_MOE_ERR_INVALID_ARG;
+  // expert parallelism: rank r holds experts [r E / W, (r + 1) E / W), every rank as many
+  if (h->ep && (h->e_count * world != h->E || h->e_begin != rank * h->e_count)) return BEAM_MOE_ERR_INVALID_ARG;
   BEAM_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   BEAM_TRY(cudaMemset(h->tp_region, 0, kTpHeaderBytes));  // no epoch published yet in this group
+  // CTA arrival counters restart (a forward that gave up on a wait may have left a count)
+  BEAM_TRY(cudaMemset(h->tp_counter, 0, 2 * sizeof(unsigned int)));
+  BEAM_TRY(cudaMemset(h->ep_counter, 0, sizeof(unsigned int)));
   BEAM_TRY(cudaDeviceSynchronize());
   uint8_t* table[kMaxTpRanks] = {};
   for (int q = 0; q < world; ++q) table[q] = static_cast<uint8_t*>(regions[q]);
@@ -649,47 +749,31 @@ beam_moe_status beam_moe_tp_attach(beam_moe_t h, int32_t rank, int32_t world, vo
   g.buf_floats = static_cast<size_t>(h->Tmax) * h->H;
   h->tp = g;
   h->tp_epoch = 0;
-  h->tp_pending = false;
-  h->ep_dispatched = false;
+  h->tp_next_phase = 0;
+  h->tp_two_shot = false;
+  h->ep_next_phase = 0;
   h->tp_attached = true;
   return BEAM_MOE_OK;
 }
 
 beam_moe_status beam_moe_forward_ep_phase(beam_moe_t h, const void* x, const void* residual, void* out,
                                           int32_t num_tokens, int32_t phase, void* stream) {
-  if (!h || !h->ep || !h->tp_attached || phase < 0 || phase > 2) return BEAM_MOE_ERR_INVALID_ARG;
+  if (!h || !h->ep || !h->tp_attached || phase < 0 || phase > 3) return BEAM_MOE_ERR_INVALID_ARG;
   if (num_tokens <= 0 || static_cast<int64_t>(num_tokens) * h->tp.world > h->Tmax) return BEAM_MOE_ERR_INVALID_ARG;
   if (!x || !residual || !out || !aligned(x, 16) || !aligned(residual, 16) || !aligned(out, 16))
     return BEAM_MOE_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const uint32_t epoch = h->tp_epoch + 1;  // the forward in flight (published by phases 0 and 1)
-  const size_t x_off = kTpHeaderBytes + 2 * static_cast<size_t>(h->Tmax) * h->H * sizeof(float);
-  if (phase == 0) {
-    if (h->ep_dispatched || h->tp_pending) return BEAM_MOE_ERR_INVALID_ARG;  // phases run 0, 1, 2 in turn
-    BEAM_TRY(launch_ep_dispatch(static_cast<const uint16_t*>(x), num_tokens, h->H, h->tp, x_off, epoch,
-                                h->ep_counter, s));
-    h->ep_dispatched = true;
-    h->ep_T = num_tokens;
-    h->last_launches = 1;
-    h->profiled_last = false;
-    return BEAM_MOE_OK;
-  }
-  if (phase == 1) {
-    if (!h->ep_dispatched || num_tokens != h->ep_T) return BEAM_MOE_ERR_INVALID_ARG;
-    const uint16_t* gathered = reinterpret_cast<const uint16_t*>(h->tp_region + x_off) +
-                               static_cast<size_t>(epoch & 1u) * h->Tmax * h->H;
-    h->ep_dispatched = false;
-    return forward_impl(h, gathered, residual, out, nullptr, nullptr, 0.0f, num_tokens * h->tp.world, stream, 0,
-                        nullptr, 0, true);
-  }
-  if (num_tokens != h->ep_T) return BEAM_MOE_ERR_INVALID_ARG;
-  return forward_impl(h, x, residual, out, nullptr, nullptr, 0.0f, num_tokens, stream, 1, nullptr,
-                      h->tp.rank * num_tokens);
+  if (phase != h->ep_next_phase || (phase > 0 && num_tokens != h->ep_T)) return BEAM_MOE_ERR_INVALID_ARG;
+  beam_moe_status st = forward_impl(h, x, residual, out, nullptr, nullptr, 0.0f, num_tokens, stream, -1, nullptr,
+                                    phase);
+  if (st != BEAM_MOE_OK) return st;
+  h->ep_T = num_tokens;
+  h->ep_next_phase = (phase + 1) % 4;
+  return BEAM_MOE_OK;
 }
 
 beam_moe_status beam_moe_forward_ep(beam_moe_t h, const void* x, const void* residual, void* out,
                                     int32_t num_tokens, void* stream) {
-  for (int phase = 0; phase < 3; ++phase) {
+  for (int phase = 0; phase < 4; ++phase) {
     beam_moe_status st = beam_moe_forward_ep_phase(h, x, residual, out, num_tokens, phase, stream);
     if (st != BEAM_MOE_OK) return st;
   }
@@ -698,19 +782,21 @@ beam_moe_status beam_moe_forward_ep(beam_moe_t h, const void* x, const void* res
 
 beam_moe_status beam_moe_forward_tp_phase(beam_moe_t h, const void* x, const void* residual, void* out,
                                           int32_t num_tokens, int32_t phase, void* stream) {
-  if (phase != 0 && phase != 1) return BEAM_MOE_ERR_INVALID_ARG;
+  if (phase < 0 || phase > 2) return BEAM_MOE_ERR_INVALID_ARG;
   if (h && h->ep) return BEAM_MOE_ERR_INVALID_ARG;  // expert-parallel handles: beam_moe_forward_ep
   if (!h || num_tokens <= 0) return num_tokens == 0 && h ? BEAM_MOE_OK : BEAM_MOE_ERR_INVALID_ARG;
-  if (phase == 1 && (!residual || !out || !aligned(residual, 16) || !aligned(out, 16)))
+  if (phase >= 1 && (!residual || !out || !aligned(residual, 16) || !aligned(out, 16)))
     return BEAM_MOE_ERR_INVALID_ARG;
   return forward_impl(h, x, residual, out, nullptr, nullptr, 0.0f, num_tokens, stream, phase);
 }
 
 beam_moe_status beam_moe_forward_tp(beam_moe_t h, const void* x, const void* residual, void* out,
                                     int32_t num_tokens, void* stream) {
-  beam_moe_status st = beam_moe_forward_tp_phase(h, x, residual, out, num_tokens, 0, stream);
-  if (st != BEAM_MOE_OK || num_tokens == 0) return st;
-  return beam_moe_forward_tp_phase(h, x, residual, out, num_tokens, 1, stream);
+  for (int phase = 0; phase < 3; ++phase) {
+    beam_moe_status st = beam_moe_forward_tp_phase(h, x, residual, out, num_tokens, phase, stream);
+    if (st != BEAM_MOE_OK || num_tokens == 0) return st;
+  }
+  return BEAM_MOE_OK;
 }
 
 beam_moe_status beam_moe_ipc_export(const void* dev_ptr, void* handle_out) {
@@ -850,13 +936,6 @@ beam_moe_status beam_moe_debug_wait_timeout(beam_moe_t h, int64_t limit_ns, void
 beam_moe_status beam_moe_set_router_mode(beam_moe_t h, int32_t mode) {
   if (!h || mode < BEAM_MOE_ROUTER_AUTO || mode > BEAM_MOE_ROUTER_TENSOR) return BEAM_MOE_ERR_INVALID_ARG;
   h->router_mode = mode;
-  return BEAM_MOE_OK;
-}
-
-beam_moe_status beam_moe_set_gemm_mode(beam_moe_t h, int32_t mode) {
-  if (!h || mode < BEAM_MOE_GEMM_AUTO || mode > BEAM_MOE_GEMM_PAIR) return BEAM_MOE_ERR_INVALID_ARG;
-  if (mode == BEAM_MOE_GEMM_PAIR && h->fmt != BEAM_MOE_FMT_NVFP4) return BEAM_MOE_ERR_UNSUPPORTED;
-  h->gemm_mode = mode;
   return BEAM_MOE_OK;
 }
 

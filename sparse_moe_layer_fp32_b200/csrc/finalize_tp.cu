@@ -14,14 +14,22 @@
 //               so every rank computes the same bits), then the same FP32 arithmetic as the
 //               single-GPU finalize: out = bf16(residual + m / sqrt(mean(m^2) + eps) * gamma).
 //
-// One-shot all-reduce: every rank reads all W partials of every token (the decode case,
-// where latency rules).  Exchange regions are double-buffered by epoch parity: a rank
-// overwrites buffer b only in epoch e + 2, after it has seen every peer's epoch e + 1 flag,
-// which a peer sets only after it finished reading buffer b in epoch e.
+// One-shot all-reduce (small batches, where latency rules): every rank's tp_reduce reads all
+// W partials of every token, W T H 4 bytes per rank.  Two-shot (large batches): rank r's
+// tp_reduce covers only its slice of the tokens, [r S, (r + 1) S) with S = ceil(T / W), so
+// it reads T H 4 bytes; it writes the finished BF16 rows to its own output and to its
+// region's row buffer, and its last CTA publishes them (second flag set); then tp_gather
+// waits for every rank's rows and copies the other slices into the output (T H 2 bytes
+// read over the links).  Both forms do the same arithmetic per token, so their bits agree.
+// Partial buffers are double-buffered by epoch parity: a rank overwrites buffer b only in
+// epoch e + 2, after it has seen every peer's epoch e + 1 flag, which a peer sets only after
+// it finished reading buffer b in epoch e.  The row buffer is single: a rank writes it in
+// epoch e + 1 only after every peer published its epoch e + 1 partials, which a peer does
+// only after its tp_gather of epoch e has completed (stream order).
 //
 // On one GPU the ranks can run one after the other: every rank's tp_partial first, then
-// every rank's tp_reduce, whose waits are then already satisfied; nothing waits on a
-// kernel that is not running.
+// every rank's tp_reduce, then every rank's tp_gather, whose waits are then already
+// satisfied; nothing waits on a kernel that is not running.
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,21 +41,6 @@ namespace beam {
 constexpr int kTpMaxThreads = 1024;
 constexpr int kTpMaxK = 16;
 
-__device__ __forceinline__ void st_release_sys(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// CTA arrival: release of this CTA's stores (ordered before it by the barrier) and acquire
-// of every earlier arrival's, at GPU scope (all CTAs of the grid share the GPU).
-__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 
 __device__ __forceinline__ void unpack8_bf16(const uint4 v, float (&f)[8]) {
   const uint32_t u[4] = {v.x, v.y, v.z, v.w};
@@ -67,6 +60,34 @@ __device__ __forceinline__ float* tp_part(uint8_t* region, int buf, size_t buf_f
   return reinterpret_cast<float*>(region + kTpHeaderBytes) + static_cast<size_t>(buf) * buf_floats;
 }
 __device__ __forceinline__ uint32_t* tp_flags(uint8_t* region) { return reinterpret_cast<uint32_t*>(region); }
+// The finished BF16 rows of the two-shot form, after the two partial buffers.
+__device__ __forceinline__ uint16_t* tp_rows(uint8_t* region, size_t buf_floats) {
+  return reinterpret_cast<uint16_t*>(tp_part(region, 2, buf_floats));
+}
+
+// Bounded acquire wait (thread q < W: rank q's flag in slot base + q of this rank's region)
+// until every flag holds the epoch; false (and the error word set) when a wait ran out.
+// Every thread of the CTA calls it; the barrier orders every thread's later loads.
+__device__ __forceinline__ bool tp_wait_flags(const TpGroup& g, int base, uint32_t epoch, uint32_t* err,
+                                              int* s_ok) {
+  if (threadIdx.x == 0) *s_ok = 1;
+  __syncthreads();
+  if (threadIdx.x < g.world) {
+    const uint32_t* flag = tp_flags(g.own) + base + threadIdx.x;
+    const uint64_t t0 = globaltimer_ns();
+    // epochs only grow; compare modulo 2^32
+    while (static_cast<int32_t>(ld_acquire_sys(flag) - epoch) < 0) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(err, kErrTimeoutEpilogue);
+        *s_ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
 
 __global__ void __launch_bounds__(kTpMaxThreads) tp_partial_kernel(const uint16_t* __restrict__ y,
                                                                    const float* __restrict__ w,
@@ -123,37 +144,26 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_partial_kernel(const uint16_
   }
 }
 
+// Token t = tok_begin + blockIdx.x.  publish (two-shot): also store the row into this rank's
+// row buffer, and the last CTA publishes the epoch in flag slot kTpRowSlot + rank of every
+// rank's region.
 __global__ void __launch_bounds__(kTpMaxThreads) tp_reduce_kernel(const uint16_t* residual,
-                                                                  const uint16_t* __restrict__ gamma, int tok_off,
+                                                                  const uint16_t* __restrict__ gamma, int tok_begin,
                                                                   int H, float eps, TpGroup g, uint32_t epoch,
-                                                                  uint16_t* out, uint32_t* err) {
+                                                                  uint16_t* out, uint32_t* err, int publish,
+                                                                  uint32_t* __restrict__ counter) {
   extern __shared__ float m_s[];  // [H]
   __shared__ float s_red[kTpMaxThreads / 32];
   __shared__ const float* s_part[kMaxTpRanks];  // this token's row in every rank's buffer
   __shared__ int s_ok;
-  const int t = blockIdx.x;
+  const int t = tok_begin + static_cast<int>(blockIdx.x);
   const int buf = static_cast<int>(epoch & 1u);
   pdl_wait();
   pdl_trigger();
   if (threadIdx.x < g.world)
-    s_part[threadIdx.x] = tp_part(g.regions[threadIdx.x], buf, g.buf_floats) + static_cast<size_t>(tok_off + t) * H;
-  if (threadIdx.x == 0) s_ok = 1;
-  __syncthreads();
-  if (threadIdx.x < g.world) {  // thread q waits for rank q's flag
-    const uint32_t* flag = tp_flags(g.own) + threadIdx.x;
-    const uint64_t t0 = globaltimer_ns();
-    // epochs only grow; compare modulo 2^32
-    while (static_cast<int32_t>(ld_acquire_sys(flag) - epoch) < 0) {
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(err, kErrTimeoutEpilogue);
-        s_ok = 0;
-        break;
-      }
-      __nanosleep(64);
-    }
-  }
-  __syncthreads();  // the waiting threads' acquires order every thread's partial loads below
-  if (!s_ok) return;
+    s_part[threadIdx.x] = tp_part(g.regions[threadIdx.x], buf, g.buf_floats) + static_cast<size_t>(t) * H;
+  // the waiting threads' acquires order every thread's partial loads below
+  if (!tp_wait_flags(g, 0, epoch, err, &s_ok)) return;
   float ss = 0.0f;
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
     float m[8] = {};
@@ -195,7 +205,43 @@ __global__ void __launch_bounds__(kTpMaxThreads) tp_reduce_kernel(const uint16_t
     for (int i = 0; i < 4; ++i)
       o[i] = bf16x2(r[2 * i] + m_s[c * 8 + 2 * i] * rinv * gm[2 * i],
                     r[2 * i + 1] + m_s[c * 8 + 2 * i + 1] * rinv * gm[2 * i + 1]);
-    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    const uint4 row = make_uint4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = row;
+    if (publish) reinterpret_cast<uint4*>(tp_rows(g.own, g.buf_floats) + static_cast<size_t>(t) * H)[c] = row;
+  }
+  if (publish) {  // same publication pattern as tp_partial
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const uint32_t done = atom_add_acq_rel_gpu(counter, 1u);
+      if (done == gridDim.x - 1) {
+        *counter = 0u;
+        for (int q = 0; q < g.world; ++q) st_release_sys(tp_flags(g.regions[q]) + kTpRowSlot + g.rank, epoch);
+      }
+    }
+  }
+}
+
+// Two-shot, second step: once every rank published its rows (bounded wait), copy the rows
+// of the other ranks' slices (rank q: [q S, min(T, (q + 1) S))) from their row buffers into
+// this rank's output, 16 bytes per thread, grid-stride.
+__global__ void __launch_bounds__(256) tp_gather_kernel(int T, int S, int H, TpGroup g, uint32_t epoch,
+                                                        uint16_t* out, uint32_t* err) {
+  __shared__ int s_ok;
+  pdl_wait();
+  pdl_trigger();
+  if (!tp_wait_flags(g, kTpRowSlot, epoch, err, &s_ok)) return;
+  const int own_begin = g.rank * S, own_end = min(T, own_begin + S);
+  const int own_rows = own_end - own_begin;
+  const int chunks = H / 8;
+  const size_t total = static_cast<size_t>(T - own_rows) * chunks;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    int t = static_cast<int>(i / chunks);
+    const int c = static_cast<int>(i - static_cast<size_t>(t) * chunks);
+    if (t >= own_begin) t += own_rows;  // skip this rank's own slice
+    const int q = t / S;
+    const uint4* src = reinterpret_cast<const uint4*>(tp_rows(g.regions[q], g.buf_floats) + static_cast<size_t>(t) * H);
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[c] = __ldcv(src + c);  // peers' memory: not cached
   }
 }
 
@@ -211,75 +257,32 @@ cudaError_t launch_tp_partial(const uint16_t* y, const float* w, const int32_t* 
                     epoch, counter);
 }
 
-cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, int tok_off, int H, float eps,
-                             const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, cudaStream_t s) {
+int tp_slice_tokens(int T, int world) { return (T + world - 1) / world; }
+
+cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, bool two_shot, int H, float eps,
+                             const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, unsigned int* counter,
+                             cudaStream_t s) {
   const size_t smem = static_cast<size_t>(H) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(tp_reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(tp_reduce_kernel, dim3(T), dim3(tp_threads(H)), smem, s, residual, gamma, tok_off, H, eps, g,
-                    epoch, out, err);
-}
-
-// ------------------------------------------------------------------ expert parallel
-// Dispatch by all-gather: CTA t copies token t's row (16-byte chunks) into row rank T + t of
-// every rank's gathered buffer (peer stores over NVLink), then the same arrival / publish
-// as tp_partial, into the delivery slots.
-__global__ void __launch_bounds__(kTpMaxThreads) ep_dispatch_kernel(const uint16_t* __restrict__ x, int T, int H,
-                                                                    TpGroup g, size_t x_offset, uint32_t epoch,
-                                                                    uint32_t* __restrict__ counter) {
-  __shared__ uint16_t* s_dst[kMaxTpRanks];
-  const int t = blockIdx.x;
-  pdl_wait();
-  pdl_trigger();
-  // buffer (epoch & 1) of g.buf_floats elements ([max_tokens][H]), row rank T + t
-  if (threadIdx.x < g.world)
-    s_dst[threadIdx.x] = reinterpret_cast<uint16_t*>(g.regions[threadIdx.x] + x_offset) +
-                         static_cast<size_t>(epoch & 1u) * g.buf_floats +
-                         (static_cast<size_t>(g.rank) * T + t) * static_cast<size_t>(H);
-  __syncthreads();
-  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
-  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
-    const uint4 v = __ldg(src + c);
-    for (int q = 0; q < g.world; ++q) reinterpret_cast<uint4*>(s_dst[q])[c] = v;
+  int begin = 0, count = T;
+  if (two_shot) {  // this rank's slice; the host only picks the two-shot form when every slice is non-empty
+    const int S = tp_slice_tokens(T, g.world);
+    begin = g.rank * S;
+    count = min(T, begin + S) - begin;
+    if (count <= 0) return cudaErrorInvalidValue;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t done = atom_add_acq_rel_gpu(counter, 1u);
-    if (done == gridDim.x - 1) {
-      *counter = 0u;
-      for (int q = 0; q < g.world; ++q) st_release_sys(tp_flags(g.regions[q]) + kMaxTpRanks + g.rank, epoch);
-    }
-  }
+  return launch_pdl(tp_reduce_kernel, dim3(count), dim3(tp_threads(H)), smem, s, residual, gamma, begin, H, eps, g,
+                    epoch, out, err, two_shot ? 1 : 0, counter);
 }
 
-// Waits (bounded) until every rank delivered this epoch's tokens.  It never triggers its
-// dependents early: the kernels after it (which read the gathered tokens, some before their
-// own grid-dependency wait) start only once it has ended.
-__global__ void ep_wait_kernel(TpGroup g, uint32_t epoch, uint32_t* err) {
-  pdl_wait();
-  if (threadIdx.x < g.world) {
-    const uint32_t* flag = tp_flags(g.own) + kMaxTpRanks + threadIdx.x;
-    const uint64_t t0 = globaltimer_ns();
-    while (static_cast<int32_t>(ld_acquire_sys(flag) - epoch) < 0) {
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(err, kErrTimeoutEpilogue);
-        break;
-      }
-      __nanosleep(64);
-    }
-  }
-}
-
-cudaError_t launch_ep_dispatch(const uint16_t* x, int T, int H, const TpGroup& g, size_t x_offset, uint32_t epoch,
-                               unsigned int* counter, cudaStream_t s) {
-  return launch_pdl(ep_dispatch_kernel, dim3(T), dim3(tp_threads(H)), 0, s, x, T, H, g, x_offset, epoch, counter);
-}
-
-cudaError_t launch_ep_wait(const TpGroup& g, uint32_t epoch, uint32_t* err, cudaStream_t s) {
-  return launch_pdl(ep_wait_kernel, dim3(1), dim3(32), 0, s, g, epoch, err);
+cudaError_t launch_tp_gather(int T, int H, const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, int grid,
+                             cudaStream_t s) {
+  return launch_pdl(tp_gather_kernel, dim3(grid), dim3(256), 0, s, T, tp_slice_tokens(T, g.world), H, g, epoch, out,
+                    err);
 }
 
 }  // namespace beam

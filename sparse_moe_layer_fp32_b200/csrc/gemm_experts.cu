@@ -79,19 +79,35 @@ struct FmtMxfp8 {
   static constexpr int TILE = kMxTileBytes;
 };
 static_assert(B_BYTES + FmtMxfp8::SFB == kMxTileBytes, "MXFP8 weight tile = B codes + B scales");
-template <int kStages, int kABytes, class F = FmtNvfp4>
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;            // 256 FP32 columns
+constexpr uint32_t SF_COL = 256;           // scale factors, one column set per K step of a stage:
+constexpr uint32_t SF_STAGE_COLS = 48;     //   A: 4 K-groups x 4 columns, then B: 4 K-groups x 8
+constexpr uint32_t SFB_OFF = 16;
+constexpr int kMaxStages = 5;
+// A stage may hold KPS consecutive K steps: their A regions, then their weight tiles (which
+// lie back to back in global memory, so one copy brings all of them), then their A scales
+// (also contiguous: one copy).  Fewer, larger copies per K step; coarser ring granularity.
+template <int kStages, int kABytes, class F = FmtNvfp4, int kKps = 1>
 struct Ring {
   using Fmt = F;
   static constexpr int STAGES = kStages;
-  static constexpr int A_BYTES = kABytes;
+  static constexpr int KPS = kKps;
+  static constexpr int A_BYTES = kABytes;                    // one K step's A region
+  static constexpr int B_OFF = kKps * kABytes;               // weight tiles of the stage's K steps
+  static constexpr int SFA_OFF = B_OFF + kKps * F::TILE;     // A scales of the stage's K steps
   // padded to 1024 bytes: every stage's operands keep the swizzle alignment
-  static constexpr int STAGE_BYTES = (kABytes + B_BYTES + F::SFB + F::SFA + 1023) / 1024 * 1024;
+  static constexpr int STAGE_BYTES = (SFA_OFF + kKps * F::SFA + 1023) / 1024 * 1024;
+  static constexpr uint32_t SF_COLS = kKps * SF_STAGE_COLS;  // TMEM scale columns per stage
+  static_assert(kABytes % 1024 == 0 && F::TILE % 1024 == 0, "operand regions keep the swizzle alignment");
+  static_assert(SF_COL + kStages * SF_COLS <= TMEM_COLS, "scale-factor stages must fit in TMEM");
+  static_assert(kStages <= kMaxStages, "barrier arrays");
 };
-using RingFull = Ring<4, A_TILE_BYTES>;
+using RingFull = Ring<2, A_TILE_BYTES, FmtNvfp4, 2>;
 using RingSmallM = Ring<5, 32 * BK_BYTES>;
-using RingFullMx = Ring<4, A_TILE_BYTES, FmtMxfp8>;
+using RingFullMx = Ring<2, A_TILE_BYTES, FmtMxfp8, 2>;
 using RingSmallMMx = Ring<5, 32 * BK_BYTES, FmtMxfp8>;
-static_assert(RingFull::STAGE_BYTES == A_TILE_BYTES + kTileBytes + SFA_BYTES, "NVFP4 stages need no padding");
+static_assert(RingFull::STAGE_BYTES == 2 * (A_TILE_BYTES + kTileBytes + SFA_BYTES), "NVFP4 stages need no padding");
 constexpr int NUM_EPI_WARPS = 16;
 constexpr int NUM_SF_WARPS = 4;                      // one per TMEM lane quarter
 constexpr int FIRST_SF_WARP = 2 + NUM_EPI_WARPS;
@@ -99,11 +115,6 @@ constexpr int NUM_THREADS = (2 + NUM_EPI_WARPS + NUM_SF_WARPS) * 32;
 constexpr int kEpiGroups = NUM_EPI_WARPS / 4;  // column groups: each warp owns a lane quarter x group
 static_assert(kEpiGroups * 64 == BN && kEpiGroups * 32 * 2 == BN, "down: 64 columns, gate/up: 32 + 32 per group");
 constexpr int kTileSlots = 4;       // tile ids the producer may publish ahead of the epilogue
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0;            // 256 FP32 columns
-constexpr uint32_t SF_COL = 256;           // scale factors, one column set per ring stage:
-constexpr uint32_t SF_STAGE_COLS = 48;     //   A: 4 K-groups x 4 columns, then B: 4 K-groups x 8
-constexpr uint32_t SFB_OFF = 16;
 
 // Instruction descriptor: E2M1 A and B (format 1), E4M3 scales (format 0), K-major
 // operands, N = 256 (n_dim = N/8 at bit 17), M = 128 (m_dim = M/16 at bit 24).
@@ -116,8 +127,6 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(int kb) {
   return kIdescMxf8 | (static_cast<uint32_t>(kb) << 29) | (static_cast<uint32_t>(kb) << 4);
 }
 
-constexpr int kMaxStages = 5;
-static_assert(SF_COL + kMaxStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor stages must fit in TMEM");
 struct __align__(16) GemmSmemTail {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
@@ -149,15 +158,18 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Waits until *counter >= target (acquire).  Returns false (and sets *abort) when the
-// wait ran past kWaitLimitNs or another role already aborted.
+// Waits until *counter >= target (acquire at GPU scope, or at system scope for counters
+// that other GPUs add to).  Returns false (and sets *abort) when the wait ran past
+// kWaitLimitNs or another role already aborted.
+template <bool kSys = false>
 __device__ __forceinline__ bool wait_counter_bounded(const uint32_t* counter, uint32_t target,
                                                      volatile int* abort_flag) {
-  if (ld_acquire_gpu(counter) >= target) return true;
+  auto load = [&]() { return kSys ? ld_acquire_sys(counter) : ld_acquire_gpu(counter); };
+  if (load() >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     __nanosleep(64);
-    if (ld_acquire_gpu(counter) >= target) return true;
+    if (load() >= target) return true;
     if ((i & 15u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -194,7 +206,7 @@ __device__ __forceinline__ TileRef tile_ref(int id, int total_gu, int n_gu, int 
 
 template <class R>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const ExpertGemmArgs args) {
-  constexpr int STAGES = R::STAGES, A_BYTES = R::A_BYTES, STAGE_BYTES = R::STAGE_BYTES;
+  constexpr int STAGES = R::STAGES, A_BYTES = R::A_BYTES, STAGE_BYTES = R::STAGE_BYTES, KPS = R::KPS;
   using F = typename R::Fmt;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -282,6 +294,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
             break;
           }
           fence_proxy_async_global();
+        } else if (args.arrivals) {
+          // expert parallelism: this block's A1 rows are stored by the ranks that route them
+          if (!wait_counter_bounded<true>(args.arrivals + t.block, static_cast<uint32_t>(mb.rows), abort_flag)) {
+            atomicOr(args.err, kErrTimeoutProducer);
+            break;
+          }
+          fence_proxy_async_global();
         }
         // rows past the block's valid rows are not copied: their stale shared-memory
         // contents only reach accumulator rows that are never stored
@@ -290,37 +309,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           atomicOr(args.err, kErrRange);
           a_bytes = A_BYTES;
         }
-        // A and its scales of K step kk into stage st
-        auto load_a = [&](int st, int kk) {
+        // Stage c of the tile holds K steps [c KPS, c KPS + nk): their weight tiles in one
+        // copy, their A scales in one copy, and their A tiles in one copy when whole
+        // 128-row tiles are copied (else one copy per K step).
+        const int n_chunks = (k_tiles + KPS - 1) / KPS;
+        auto chunk_steps = [&](int c) { return min(KPS, k_tiles - c * KPS); };
+        auto load_a = [&](int st, int c) {
           uint8_t* sa = smem + st * STAGE_BYTES;
-          bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, a_bytes, &tail->full[st]);
-          bulk_load(sa + A_BYTES + B_BYTES + F::SFB, sfa + static_cast<size_t>(kk) * F::SFA, F::SFA, &tail->full[st]);
+          const int kk = c * KPS, nk = chunk_steps(c);
+          if (KPS > 1 && A_BYTES == A_TILE_BYTES && a_bytes == static_cast<uint32_t>(A_TILE_BYTES)) {
+            bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, nk * A_TILE_BYTES, &tail->full[st]);
+          } else {
+            for (int j = 0; j < nk; ++j)
+              bulk_load(sa + j * A_BYTES, a_src + static_cast<size_t>(kk + j) * A_TILE_BYTES, a_bytes,
+                        &tail->full[st]);
+          }
+          bulk_load(sa + R::SFA_OFF, sfa + static_cast<size_t>(kk) * F::SFA, nk * F::SFA, &tail->full[st]);
         };
         // Before the wait only the weights are loaded; the first tile starts at stage 0, so
-        // its deferred K steps kk < STAGES sit in stages kk.
+        // its deferred chunks c < STAGES sit in stages c.
         int deferred = 0;
         auto resolve = [&]() {
           pdl_wait();
           pdl_trigger();
           waited = true;
-          for (int kk = 0; kk < deferred; ++kk) load_a(kk, kk);
+          for (int c = 0; c < deferred; ++c) load_a(c, c);
         };
         bool ok = true;
-        const int claim_at = max(0, k_tiles - STAGES);
-        for (int kt = 0; kt < k_tiles; ++kt) {
-          if (kt == claim_at) claim = atomicAdd(args.sched, 1u);
-          if (!waited && kt == STAGES) resolve();
+        const int claim_at = max(0, n_chunks - STAGES);
+        for (int c = 0; c < n_chunks; ++c) {
+          if (c == claim_at) claim = atomicAdd(args.sched, 1u);
+          if (!waited && c == STAGES) resolve();
           if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&tail->full[stage], a_bytes + F::TILE + F::SFA);
+          const int nk = chunk_steps(c);
+          mbar_arrive_expect_tx(&tail->full[stage], static_cast<uint32_t>(nk) * (a_bytes + F::TILE + F::SFA));
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          bulk_load(smem + stage * STAGE_BYTES + A_BYTES, btile + static_cast<size_t>(kt) * F::TILE, F::TILE,
-                    &tail->full[stage]);
+          bulk_load(smem + stage * STAGE_BYTES + R::B_OFF, btile + static_cast<size_t>(c * KPS) * F::TILE,
+                    nk * F::TILE, &tail->full[stage]);
           if (waited)
-            load_a(stage, kt);
+            load_a(stage, c);
           else
             ++deferred;
           if (++stage == STAGES) {
@@ -358,27 +389,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
         }
         if (id < 0) break;
         const int k_tiles = id >= total_gu ? args.d_k_tiles : args.gu_k_tiles;
+        const int n_chunks = (k_tiles + KPS - 1) / KPS;
         if (!mbar_wait_bounded(&tail->acc_empty, acc_phase ^ 1, abort_flag)) break;
         tc_fence_after();
         bool ok = true;
-        for (int kt = 0; kt < k_tiles; ++kt) {
+        for (int c = 0; c < n_chunks; ++c) {
           // the stage's operands have landed and its scale factors are in TMEM
           if (!mbar_wait_bounded(&tail->sf_full[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
-          const uint32_t sf = tmem + SF_COL + stage * SF_STAGE_COLS;
+          const int nk = min(KPS, k_tiles - c * KPS);
+          for (int j = 0; j < nk; ++j) {
+            const int kt = c * KPS + j;
+            const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES) + j * A_BYTES;
+            const uint32_t sb = smem_u32(smem + stage * STAGE_BYTES) + R::B_OFF + j * F::TILE;
+            const uint32_t sf = tmem + SF_COL + stage * R::SF_COLS + j * SF_STAGE_COLS;
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            if constexpr (F::kMx)  // the 4 MMAs share the stage's scale columns, byte kb of each cell
-              tc_mma_mxf8(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), idesc_mxf8(kb),
-                          sf, sf + SFB_OFF, (kt | kb) != 0 ? 1u : 0u);
-            else
-              tc_mma_nvfp4(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), kIdescNvfp4,
-                           sf + kb * 4, sf + SFB_OFF + kb * 8, (kt | kb) != 0 ? 1u : 0u);
+            for (int kb = 0; kb < 4; ++kb) {
+              if constexpr (F::kMx)  // the 4 MMAs share the step's scale columns, byte kb of each cell
+                tc_mma_mxf8(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), idesc_mxf8(kb),
+                            sf, sf + SFB_OFF, (kt | kb) != 0 ? 1u : 0u);
+              else
+                tc_mma_nvfp4(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), kIdescNvfp4,
+                             sf + kb * 4, sf + SFB_OFF + kb * 8, (kt | kb) != 0 ? 1u : 0u);
+            }
           }
           tc_commit(&tail->empty[stage]);
           if (++stage == STAGES) {
@@ -418,46 +454,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       }
       if (id < 0) break;
       const int k_tiles = id >= total_gu ? args.d_k_tiles : args.gu_k_tiles;
+      const int n_chunks = (k_tiles + KPS - 1) / KPS;
       bool ok = true;
-      for (int kt = 0; kt < k_tiles; ++kt) {
+      for (int c = 0; c < n_chunks; ++c) {
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->full[stage], phase, abort_flag))) {
           ok = false;
           break;
         }
-        const uint8_t* ssfb = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;  // [half][K-group][512]
-        const uint8_t* ssfa = ssfb + F::SFB;                                   // [K-group][512]
-        const uint32_t col = SF_COL + stage * SF_STAGE_COLS;
-        if constexpr (F::kMx) {
-          // one atom of A scales -> columns 0..3; B: rows 0-127 -> SFB_OFF + 0..3, rows 128-255 -> + 4..7
-          const uint4 a = *reinterpret_cast<const uint4*>(ssfa + lane * 16);
-          const uint32_t ra[4] = {a.x, a.y, a.z, a.w};
-          tmem_st_32x32b_x4(t_lane + col, ra);
-          const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + lane * 16);
-          const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 512 + lane * 16);
-          const uint32_t rb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-          tmem_st_32x32b_x8(t_lane + col + SFB_OFF, rb);
-        } else {
-        uint32_t r[16];
-        // A: K-group kb -> columns 4 kb .. 4 kb + 3
+        const int nk = min(KPS, k_tiles - c * KPS);
+        for (int j = 0; j < nk; ++j) {
+          const uint8_t* ssfb = smem + stage * STAGE_BYTES + R::B_OFF + j * F::TILE + B_BYTES;  // [half][K-group][512]
+          const uint8_t* ssfa = smem + stage * STAGE_BYTES + R::SFA_OFF + j * F::SFA;           // [K-group][512]
+          const uint32_t col = SF_COL + stage * R::SF_COLS + j * SF_STAGE_COLS;
+          if constexpr (F::kMx) {
+            // one atom of A scales -> columns 0..3; B: rows 0-127 -> SFB_OFF + 0..3, rows 128-255 -> + 4..7
+            const uint4 a = *reinterpret_cast<const uint4*>(ssfa + lane * 16);
+            const uint32_t ra[4] = {a.x, a.y, a.z, a.w};
+            tmem_st_32x32b_x4(t_lane + col, ra);
+            const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + lane * 16);
+            const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 512 + lane * 16);
+            const uint32_t rb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            tmem_st_32x32b_x8(t_lane + col + SFB_OFF, rb);
+          } else {
+            uint32_t r[16];
+            // A: K-group kb -> columns 4 kb .. 4 kb + 3
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512 + lane * 16);
-          r[kb * 4 + 0] = v.x; r[kb * 4 + 1] = v.y; r[kb * 4 + 2] = v.z; r[kb * 4 + 3] = v.w;
-        }
-        tmem_st_32x32b_x16(t_lane + col, r);
-        // B: K-group kb -> columns 8 kb .. 8 kb + 3 (rows 0-127), 8 kb + 4 .. 8 kb + 7 (rows 128-255)
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512 + lane * 16);
+              r[kb * 4 + 0] = v.x; r[kb * 4 + 1] = v.y; r[kb * 4 + 2] = v.z; r[kb * 4 + 3] = v.w;
+            }
+            tmem_st_32x32b_x16(t_lane + col, r);
+            // B: K-group kb -> columns 8 kb .. 8 kb + 3 (rows 0-127), 8 kb + 4 .. 8 kb + 7 (rows 128-255)
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+            for (int part = 0; part < 2; ++part) {
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int kb = part * 2 + q;
-            const uint4 v0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512 + lane * 16);
-            const uint4 v1 = *reinterpret_cast<const uint4*>(ssfb + SFA_BYTES + kb * 512 + lane * 16);
-            r[q * 8 + 0] = v0.x; r[q * 8 + 1] = v0.y; r[q * 8 + 2] = v0.z; r[q * 8 + 3] = v0.w;
-            r[q * 8 + 4] = v1.x; r[q * 8 + 5] = v1.y; r[q * 8 + 6] = v1.z; r[q * 8 + 7] = v1.w;
+              for (int q = 0; q < 2; ++q) {
+                const int kb = part * 2 + q;
+                const uint4 v0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512 + lane * 16);
+                const uint4 v1 = *reinterpret_cast<const uint4*>(ssfb + SFA_BYTES + kb * 512 + lane * 16);
+                r[q * 8 + 0] = v0.x; r[q * 8 + 1] = v0.y; r[q * 8 + 2] = v0.z; r[q * 8 + 3] = v0.w;
+                r[q * 8 + 4] = v1.x; r[q * 8 + 5] = v1.y; r[q * 8 + 6] = v1.z; r[q * 8 + 7] = v1.w;
+              }
+              tmem_st_32x32b_x16(t_lane + col + SFB_OFF + part * 16, r);
+            }
           }
-          tmem_st_32x32b_x16(t_lane + col + SFB_OFF + part * 16, r);
-        }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -584,397 +624,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-// ------------------------------------------------------------------ CTA pairs
-// Large batches: the same tile list over 256-row blocks, each tile computed by a pair of CTAs
-// (a cluster of 2) with one MMA spanning both SMs (tcgen05.mma.cta_group::2, M = 256).  CTA c
-// of the pair holds rows [128c, 128c + 128) of the block's activations and accumulator, and
-// rows [128c, 128c + 128) of each 256-row weight tile (the MMA reads B from both CTAs); both
-// hold all 256 rows of the weight scales.  A K step then moves 38 KB into each CTA (A 16 KB,
-// its half of B 16 KB, B scales 4 KB, A scales 2 KB) instead of 54 KB, and a 5th stage fits.
-// At prefill sizes the single-CTA ring is bound by those loads (bytes in flight / L2 latency).
-// CTA 0 claims the tiles and publishes each id and block entry to both CTAs' rings, issues
-// the MMAs and commits them to both CTAs' barriers; CTA 1 runs its producer, scale and
-// epilogue warps and reports to CTA 0's barriers.  Every wait stays bounded; the cluster
-// barriers at entry and exit are reached on every path.
-constexpr int PAIR_STAGES = 5;
-constexpr int PAIR_B_BYTES = B_BYTES / 2;
-constexpr int PAIR_STAGE_BYTES = A_TILE_BYTES + PAIR_B_BYTES + SFB_BYTES + SFA_BYTES;
-static_assert(PAIR_STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for the swizzle");
-static_assert(PAIR_STAGES <= kMaxStages, "barrier arrays");
-constexpr int kRingConsumers = 1 + NUM_EPI_WARPS + NUM_SF_WARPS;  // per CTA: MMA thread or producer, epilogue, scales
-// M = 256 across the pair
-constexpr uint32_t kIdescNvfp4Pair = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((2 * BM >> 4) << 24);
-
-static size_t pair_smem_bytes() {
-  return static_cast<size_t>(PAIR_STAGES) * PAIR_STAGE_BYTES + sizeof(GemmSmemTail) + 1024;
-}
-
-__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_pair_kernel(const ExpertGemmArgs args) {
-  constexpr int STAGES = PAIR_STAGES, STAGE_BYTES = PAIR_STAGE_BYTES, A_BYTES = A_TILE_BYTES;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  GemmSmemTail* tail = reinterpret_cast<GemmSmemTail*>(smem + STAGES * STAGE_BYTES);
-  volatile int* abort_flag = &tail->abort_flag;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();  // 0 leads the pair
-  const bool lead = rank == 0;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&tail->full[s], 1);
-      mbar_init(&tail->empty[s], 1);
-      mbar_init(&tail->sf_full[s], 2 * NUM_SF_WARPS);
-    }
-    for (int j = 0; j < kTileSlots; ++j) {
-      mbar_init(&tail->tile_full[j], 1);
-      mbar_init(&tail->tile_empty[j], 2 * kRingConsumers);
-    }
-    mbar_init(&tail->acc_full, 1);
-    mbar_init(&tail->acc_empty, 2 * NUM_EPI_WARPS);
-    mbar_init(&tail->drain, 1);
-    tail->abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(&tail->tmem_base, TMEM_COLS);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();  // both CTAs' barriers exist before any arrives from the other
-  tc_fence_after();
-  const uint32_t tmem = tail->tmem_base;
-  // rank 0's barriers that both CTAs report to, and rank 1's tile ring that rank 0 fills
-  const uint32_t lead_tile_empty = mapa_shared(smem_u32(&tail->tile_empty[0]), 0);
-  const uint32_t lead_sf_full = mapa_shared(smem_u32(&tail->sf_full[0]), 0);
-  const uint32_t lead_acc_empty = mapa_shared(smem_u32(&tail->acc_empty), 0);
-  const bool producer = warp == 0 && lane == 0;
-  if (!producer) {
-    pdl_wait();
-    pdl_trigger();
-  }
-
-  const int n_gu = args.gu_n_tiles, n_d = args.d_n_tiles;
-  const int num_blocks = __ldcg(args.num_mblocks);  // 256-row blocks
-  const int total_gu = num_blocks * n_gu;
-  const int total = total_gu + num_blocks * n_d;
-  uint32_t* const ready = args.sched + 1;
-  const uint32_t ready_target = static_cast<uint32_t>(n_gu) * 2 * NUM_EPI_WARPS;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      const uint32_t peer_tile_full = mapa_shared(smem_u32(&tail->tile_full[0]), 1);
-      const uint32_t peer_tile_ids = mapa_shared(smem_u32(&tail->tile_ids[0]), 1);
-      const uint32_t peer_tile_mb = mapa_shared(smem_u32(&tail->tile_mb[0][0]), 1);
-      int stage = 0, slot = 0;
-      uint32_t phase = 0, slot_phase = 0;
-      uint32_t armed = 0, armed_parity = 0;
-      uint32_t claim = lead ? atomicAdd(args.sched, 1u) : 0u;
-      bool waited = false;
-      for (;;) {
-        int id;
-        MBlock mb{};
-        if (lead) {
-          if (!mbar_wait_bounded_cluster(&tail->tile_empty[slot], slot_phase ^ 1, abort_flag)) break;
-          id = claim < static_cast<uint32_t>(total) ? static_cast<int>(claim) : -1;
-          if (id >= 0) mb = load_mblock(args.mblocks + tile_ref(id, total_gu, n_gu, n_d).block);
-          const int4 m0 = make_int4(mb.expert, mb.row_begin, mb.rows, mb.sf_block);
-          const int4 m1 = make_int4(__float_as_int(mb.scale_gu), __float_as_int(mb.scale_d), 0, 0);
-          tail->tile_ids[slot] = id;
-          tail->tile_mb[slot][0] = m0;
-          tail->tile_mb[slot][1] = m1;
-          st_cluster_s32(peer_tile_ids + 4 * slot, id);
-          st_cluster_v4(peer_tile_mb + 32 * slot, m0);
-          st_cluster_v4(peer_tile_mb + 32 * slot + 16, m1);
-          mbar_arrive(&tail->tile_full[slot]);
-          mbar_arrive_cluster(peer_tile_full + 8 * slot);  // release: the stores above come first
-        } else {
-          if (!mbar_wait_bounded_cluster(&tail->tile_full[slot], slot_phase, abort_flag)) break;
-          id = tail->tile_ids[slot];
-          const int4 m0 = tail->tile_mb[slot][0], m1 = tail->tile_mb[slot][1];
-          mb = MBlock{m0.x, m0.y, m0.z, m0.w, __int_as_float(m1.x), __int_as_float(m1.y), {0, 0}};
-          mbar_arrive_cluster(lead_tile_empty + 8 * slot);
-        }
-        if (++slot == kTileSlots) {
-          slot = 0;
-          slot_phase ^= 1;
-        }
-        if (id < 0) break;
-        const TileRef t = tile_ref(id, total_gu, n_gu, n_d);
-        const int k_tiles = t.down ? args.d_k_tiles : args.gu_k_tiles;
-        const int n_tiles = t.down ? n_d : n_gu;
-        const int half_rows = min(max(mb.rows - 128 * static_cast<int>(rank), 0), BM);
-        const size_t act_block = static_cast<size_t>(mb.sf_block) + rank;  // this CTA's 128-row activation block
-        const uint8_t* a_src = (t.down ? args.a2 : args.a1) + act_block * k_tiles * A_TILE_BYTES;
-        const uint8_t* sfa = (t.down ? args.a2_sf : args.a1_sf) + act_block * k_tiles * SFA_BYTES;
-        const uint8_t* btile = (t.down ? args.w_d : args.w_gu) +
-                               (static_cast<size_t>(mb.expert) * n_tiles + t.nt) * k_tiles * static_cast<size_t>(kTileBytes);
-        if (t.down && half_rows > 0) {
-          if (!wait_counter_bounded(ready + t.block, ready_target, abort_flag)) {
-            atomicOr(args.err, kErrTimeoutProducer);
-            break;
-          }
-          fence_proxy_async_global();
-        }
-        // an empty half copies no activations: its accumulator rows are never stored
-        const uint32_t a_bytes = half_rows > 0 ? static_cast<uint32_t>((half_rows + 7) & ~7) * BK_BYTES : 0u;
-        const uint32_t sfa_bytes = half_rows > 0 ? static_cast<uint32_t>(SFA_BYTES) : 0u;
-        auto load_a = [&](int st, int kk) {
-          if (a_bytes == 0) return;
-          uint8_t* sa = smem + st * STAGE_BYTES;
-          bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, a_bytes, &tail->full[st]);
-          bulk_load(sa + A_BYTES + PAIR_B_BYTES + SFB_BYTES, sfa + static_cast<size_t>(kk) * SFA_BYTES, sfa_bytes,
-                    &tail->full[st]);
-        };
-        int deferred = 0;
-        auto resolve = [&]() {
-          pdl_wait();
-          pdl_trigger();
-          waited = true;
-          for (int kk = 0; kk < deferred; ++kk) load_a(kk, kk);
-        };
-        bool ok = true;
-        const int claim_at = max(0, k_tiles - STAGES);
-        for (int kt = 0; kt < k_tiles; ++kt) {
-          if (lead && kt == claim_at) claim = atomicAdd(args.sched, 1u);
-          if (!waited && kt == STAGES) resolve();
-          if (!mbar_wait_bounded_cluster(&tail->empty[stage], phase ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&tail->full[stage], a_bytes + PAIR_B_BYTES + SFB_BYTES + sfa_bytes);
-          armed |= 1u << stage;
-          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          const uint8_t* wk = btile + static_cast<size_t>(kt) * kTileBytes;
-          uint8_t* sb = smem + stage * STAGE_BYTES + A_BYTES;
-          bulk_load(sb, wk + rank * PAIR_B_BYTES, PAIR_B_BYTES, &tail->full[stage]);  // this CTA's 128 B rows
-          bulk_load(sb + PAIR_B_BYTES, wk + B_BYTES, SFB_BYTES, &tail->full[stage]);  // all 256 rows' scales
-          if (waited)
-            load_a(stage, kt);
-          else
-            ++deferred;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (!waited) resolve();
-        if (!ok) break;
-      }
-      if (!waited) {
-        pdl_wait();
-        pdl_trigger();
-      }
-      for (int s = 0; s < STAGES; ++s)
-        if ((armed >> s) & 1u) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&tail->full[s], (armed_parity >> s) & 1u))
-            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-        }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (rank 0 only)
-    if (lane == 0 && lead) {
-      int stage = 0, slot = 0;
-      uint32_t phase = 0, acc_phase = 0, slot_phase = 0;
-      for (;;) {
-        if (!mbar_wait_bounded_cluster(&tail->tile_full[slot], slot_phase, abort_flag)) break;
-        const int id = tail->tile_ids[slot];
-        mbar_arrive(&tail->tile_empty[slot]);
-        if (++slot == kTileSlots) {
-          slot = 0;
-          slot_phase ^= 1;
-        }
-        if (id < 0) break;
-        const int k_tiles = id >= total_gu ? args.d_k_tiles : args.gu_k_tiles;
-        if (!mbar_wait_bounded_cluster(&tail->acc_empty, acc_phase ^ 1, abort_flag)) break;
-        tc_fence_after();
-        bool ok = true;
-        for (int kt = 0; kt < k_tiles; ++kt) {
-          // both CTAs' operands have landed and both CTAs' scales are in TMEM
-          if (!mbar_wait_bounded_cluster(&tail->sf_full[stage], phase, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
-          const uint32_t sf = tmem + SF_COL + stage * SF_STAGE_COLS;
-#pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            tc_mma_nvfp4_pair(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32),
-                              kIdescNvfp4Pair, sf + kb * 4, sf + SFB_OFF + kb * 8, (kt | kb) != 0 ? 1u : 0u);
-          }
-          tc_commit_pair_multicast(&tail->empty[stage], 0x3);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (!ok) break;
-        tc_commit_pair_multicast(&tail->acc_full, 0x3);
-        acc_phase ^= 1;
-      }
-      tc_commit_pair(&tail->drain);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(&tail->drain, 0))
-        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-    }
-  } else if (warp >= FIRST_SF_WARP) {
-    // ------------------------------------------------------------ scale factors -> TMEM (both CTAs)
-    const int quarter = warp & 3;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    int stage = 0, slot = 0;
-    uint32_t phase = 0, slot_phase = 0;
-    for (;;) {
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded_cluster(&tail->tile_full[slot], slot_phase, abort_flag))) break;
-      const int id = tail->tile_ids[slot];
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_tile_empty + 8 * slot);
-      if (++slot == kTileSlots) {
-        slot = 0;
-        slot_phase ^= 1;
-      }
-      if (id < 0) break;
-      const int k_tiles = id >= total_gu ? args.d_k_tiles : args.gu_k_tiles;
-      bool ok = true;
-      for (int kt = 0; kt < k_tiles; ++kt) {
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded_cluster(&tail->full[stage], phase, abort_flag))) {
-          ok = false;
-          break;
-        }
-        const uint8_t* ssfb = smem + stage * STAGE_BYTES + A_BYTES + PAIR_B_BYTES;
-        const uint8_t* ssfa = ssfb + SFB_BYTES;
-        const uint32_t col = SF_COL + stage * SF_STAGE_COLS;
-        uint32_t r[16];
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512 + lane * 16);
-          r[kb * 4 + 0] = v.x; r[kb * 4 + 1] = v.y; r[kb * 4 + 2] = v.z; r[kb * 4 + 3] = v.w;
-        }
-        tmem_st_32x32b_x16(t_lane + col, r);
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int kb = part * 2 + q;
-            const uint4 v0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512 + lane * 16);
-            const uint4 v1 = *reinterpret_cast<const uint4*>(ssfb + SFA_BYTES + kb * 512 + lane * 16);
-            r[q * 8 + 0] = v0.x; r[q * 8 + 1] = v0.y; r[q * 8 + 2] = v0.z; r[q * 8 + 3] = v0.w;
-            r[q * 8 + 4] = v1.x; r[q * 8 + 5] = v1.y; r[q * 8 + 6] = v1.z; r[q * 8 + 7] = v1.w;
-          }
-          tmem_st_32x32b_x16(t_lane + col + SFB_OFF + part * 16, r);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead_sf_full + 8 * stage);
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      if (!ok) break;
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue (both CTAs, own rows)
-    const int quarter = warp & 3;
-    const int group = (warp - 2) >> 2;
-    const int row_in_tile = quarter * 32 + lane;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const float alpha2 = args.alpha_a2;
-    const float six_alpha2 = __fmul_rn(6.0f, alpha2);
-    int slot = 0;
-    uint32_t acc_phase = 0, slot_phase = 0;
-    for (;;) {
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded_cluster(&tail->tile_full[slot], slot_phase, abort_flag))) break;
-      const int id = tail->tile_ids[slot];
-      const int4 m0 = tail->tile_mb[slot][0], m1 = tail->tile_mb[slot][1];
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_tile_empty + 8 * slot);
-      if (++slot == kTileSlots) {
-        slot = 0;
-        slot_phase ^= 1;
-      }
-      if (id < 0) break;
-      const TileRef t = tile_ref(id, total_gu, n_gu, n_d);
-      const MBlock mb{m0.x, m0.y, m0.z, m0.w, __int_as_float(m1.x), __int_as_float(m1.y), {0, 0}};
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded_cluster(&tail->acc_full, acc_phase, abort_flag))) break;
-      tc_fence_after();
-      uint32_t v[2][32];
-      if (!t.down) {
-        tmem_ld_32x32b_x32(t_lane + ACC_COL + group * 32, v[0]);
-        tmem_ld_32x32b_x32(t_lane + ACC_COL + 128 + group * 32, v[1]);
-      } else {
-        tmem_ld_32x32b_x32(t_lane + ACC_COL + group * 64, v[0]);
-        tmem_ld_32x32b_x32(t_lane + ACC_COL + group * 64 + 32, v[1]);
-      }
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
-      acc_phase ^= 1;
-      const int half_rows = min(max(mb.rows - 128 * static_cast<int>(rank), 0), BM);
-      const size_t act_block = static_cast<size_t>(mb.sf_block) + rank;
-      const bool valid = row_in_tile < half_rows;
-      if (!t.down) {
-        if (valid) {
-          const float scale = mb.scale_gu;
-          const int f0 = t.nt * 128 + group * 32;
-          uint32_t codes[4];
-          uint32_t scodes = 0;
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            float h[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g = __uint_as_float(v[0][b * 16 + i]) * scale;
-              const float u = __uint_as_float(v[1][b * 16 + i]) * scale;
-              h[i] = silu_times(g, u);
-            }
-            const uint32_t sc = quant_block16(h, alpha2, six_alpha2, codes[2 * b], codes[2 * b + 1]);
-            scodes |= sc << (8 * b);
-          }
-          *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(act_block, args.d_k_tiles, f0 >> 8, row_in_tile,
-                                                              (f0 & 255) >> 5)) =
-              make_uint4(codes[0], codes[1], codes[2], codes[3]);
-          *reinterpret_cast<uint16_t*>(args.a2_sf + sf_atom_offset(act_block, args.d_k_tiles * 4, row_in_tile,
-                                                                   f0 / 16)) = static_cast<uint16_t>(scodes);
-        }
-        fence_proxy_async_global();
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence();
-          atomicAdd(ready + t.block, 1u);
-        }
-      } else if (valid) {
-        const float scale = mb.scale_d;
-        const size_t r = static_cast<size_t>(mb.row_begin + 128 * static_cast<int>(rank) + row_in_tile);
-        uint16_t* dst = args.y + r * args.y_cols + t.nt * BN + group * 64;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t p[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int c = q * 16 + 2 * i;
-            p[i] = bf16x2_bits(__uint_as_float(v[c >> 5][c & 31]) * scale,
-                               __uint_as_float(v[(c + 1) >> 5][(c + 1) & 31]) * scale);
-          }
-          st_global_v8(dst + q * 16, p);
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync();  // rank 0's MMAs (which write both CTAs' TMEM) have drained; no arrives remain
-  tc_fence_after();
-  if (threadIdx.x == 0 && tail->abort_flag) atomicOr(args.err, kErrTimeoutMma);
-  if (warp == 1) tmem_dealloc_pair(tmem, TMEM_COLS);
-}
-
 template <class R>
 static cudaError_t launch_ring(const ExpertGemmArgs& a, int grid, cudaStream_t s) {
   const size_t smem = ring_smem_bytes<R>();
@@ -993,14 +642,6 @@ cudaError_t launch_gemm_experts(const ExpertGemmArgs& a, int grid, cudaStream_t 
 cudaError_t launch_gemm_experts_mx(const ExpertGemmArgs& a, int grid, cudaStream_t s) {
   if (a.max_rows_per_expert <= 32) return launch_ring<RingSmallMMx>(a, grid, s);
   return launch_ring<RingFullMx>(a, grid, s);
-}
-
-cudaError_t launch_gemm_experts_pair(const ExpertGemmArgs& a, int grid, cudaStream_t s) {
-  const size_t smem = pair_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gemm_experts_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  return launch_pdl_cluster(gemm_experts_pair_kernel, dim3(grid & ~1), dim3(NUM_THREADS), smem, 2u, s, a);
 }
 
 }  // namespace beam

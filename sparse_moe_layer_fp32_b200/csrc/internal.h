@@ -76,10 +76,9 @@ cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, 
 // ---- permutation and activation quantisation (routing.cu)
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s);
 // Also zeroes sched[0, sched_n), the tile scheduler words of the expert GEMM launch.
-// pair != 0: the work list holds 256-row blocks for the CTA-pair GEMM.
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
-                        BlockScales bs, int pair, cudaStream_t s);
+                        BlockScales bs, cudaStream_t s);
 // tile_row[t][j] = 128 x activation block + row within it, for slot (t, j).
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,
                            const int32_t* sf_block, int T, int k, int E, int32_t* perm_src, int32_t* inv,
@@ -142,6 +141,10 @@ struct ExpertGemmArgs {
   // sched_words(nblk_max) words, zeroed by the routing kernel (two or more launches back).
   uint32_t* sched;
   uint32_t* err;
+  // Expert parallelism: rows delivered into each block by the ranks (release, system scope);
+  // a gate/up tile's activations are read once its block's count reaches the block's rows.
+  // Null otherwise.
+  const uint32_t* arrivals;
 };
 inline int64_t sched_words(int64_t nblk_max) { return 1 + nblk_max; }
 cudaError_t launch_gemm_experts(const ExpertGemmArgs& a, int grid, cudaStream_t s);
@@ -149,17 +152,19 @@ cudaError_t launch_gemm_experts(const ExpertGemmArgs& a, int grid, cudaStream_t 
 // d_k_tiles = I / 128), weight tiles of kMxTileBytes, scales [blk][K/128][512], and the
 // SwiGLU epilogue writes A2 = MX(h).  alpha_a2 is unused.
 cudaError_t launch_gemm_experts_mx(const ExpertGemmArgs& a, int grid, cudaStream_t s);
-// The CTA-pair version over 256-row blocks (grid rounded down to even).
-constexpr int kPairMinTokens = BEAM_MOE_PAIR_MIN_TOKENS;
-cudaError_t launch_gemm_experts_pair(const ExpertGemmArgs& a, int grid, cudaStream_t s);
 
-// ---- tensor / expert parallel finalize fused with its all-reduce (finalize_tp.cu)
-// Exchange region of one rank: kTpHeaderBytes of flags (u32 slot q = the last epoch rank q
-// published its partial m; slot kMaxTpRanks + q = the last epoch rank q delivered its
-// tokens), two buffers of [max_tokens][H] FP32 partial m (epoch parity), and for expert
-// parallelism two buffers of [max_tokens][H] BF16 gathered tokens.
+// ---- tensor parallel finalize fused with its all-reduce (finalize_tp.cu)
+// Exchange region of a tensor-parallel rank: kTpHeaderBytes of flags (u32 slot q = the last
+// epoch rank q published its partial m; slot kTpRowSlot + q = the last epoch rank q
+// published its finished rows), two buffers of [max_tokens][H] FP32 partial m (epoch
+// parity), then [max_tokens][H] BF16 finished rows (the two-shot form).  Expert-parallel
+// regions share the header and TpGroup; their body is EpLayout below.
 constexpr int kMaxTpRanks = 16;
 constexpr size_t kTpHeaderBytes = 1024;
+constexpr int kTpRowSlot = 4 * kMaxTpRanks;
+// The two-shot all-reduce from this many tokens on (every rank's slice is then non-empty
+// for any world <= kMaxTpRanks, since T >= world^2).
+constexpr int kTpTwoShotMinTokens = 256;
 struct TpGroup {
   uint8_t* const* regions;  // device array: every rank's region as mapped in this process
   uint8_t* own;             // this rank's region (regions[rank])
@@ -170,16 +175,63 @@ struct TpGroup {
 cudaError_t launch_tp_partial(const uint16_t* y, const float* w, const int32_t* inv, const int32_t* ids, int e_begin,
                               int e_end, int T, int H, int k, const TpGroup& g, uint32_t epoch, unsigned int* counter,
                               cudaStream_t s);
-// out[t] for t < T from partial rows tok_off + t (tok_off = 0 under TP).
-cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, int tok_off, int H, float eps,
-                             const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, cudaStream_t s);
-// Expert parallelism: this rank's T tokens into rows [rank T, rank T + T) of every rank's
-// gathered-token buffer (x_offset: its byte offset in a region; buffer epoch & 1), then the
-// delivery flag; and the wait for every rank's delivery (one CTA that lets its dependents
-// start only when it ends).
-cudaError_t launch_ep_dispatch(const uint16_t* x, int T, int H, const TpGroup& g, size_t x_offset, uint32_t epoch,
-                               unsigned int* counter, cudaStream_t s);
-cudaError_t launch_ep_wait(const TpGroup& g, uint32_t epoch, uint32_t* err, cudaStream_t s);
+// Tokens of a rank's slice in the two-shot form: ceil(T / world).
+int tp_slice_tokens(int T, int world);
+// One-shot: out[t] for every t < T.  Two-shot: out[t] for this rank's slice only, also stored
+// into its row buffer and published (counter: the CTA arrivals of this step).
+cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, int T, bool two_shot, int H, float eps,
+                             const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, unsigned int* counter,
+                             cudaStream_t s);
+// Two-shot: the other ranks' finished rows into out, after a bounded wait for their flags.
+cudaError_t launch_tp_gather(int T, int H, const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, int grid,
+                             cudaStream_t s);
+
+// ---- expert parallelism: dispatch of routed rows, combine of expert outputs (expert_parallel.cu)
+// Flag slots of the region header: rank q's counts of the epoch published / its expert
+// outputs for the epoch returned.
+constexpr int kEpCountSlot = 2 * kMaxTpRanks;
+constexpr int kEpReturnSlot = 3 * kMaxTpRanks;
+// Byte offsets in an expert-parallel rank's region (after the 1 KB flag header).
+struct EpLayout {
+  size_t counts;    // int32 [kMaxTpRanks][E]: rows source rank s routes to expert e
+  size_t arrivals;  // u32 [nblk]: rows delivered into each 128-row block of this rank's experts
+  size_t origin;    // int32 [rows]: source rank << 24 | source slot t k + j of each received row
+  size_t a1;        // activation tiles of the received rows (the GEMM layout)
+  size_t a1_sf;     // their scale blocks
+  size_t ret;       // BF16 [max_tokens][k][H]: this rank's slots' expert outputs, returned
+  size_t bytes;     // the whole region
+  int nblk;         // blocks the arrival counters cover
+  int rows;         // rows of origin and of the returned rows (max_tokens k)
+};
+// Where source-rank rows of expert e go: destination rank, its permuted row of this rank's
+// first row of e, the block of the destination's first row of e, and the rows of e that
+// lower ranks send (this rank's rows of e start after them).
+struct EpDest {
+  int32_t rank, row0, blk0, pre;
+};
+// Zeroes this rank's arrival counters, then publishes its expert counts (offsets[e + 1] -
+// offsets[e]) into every rank's count matrix and sets its count flag (release, system scope).
+cudaError_t launch_ep_counts(const int32_t* offsets, int E, const TpGroup& g, const EpLayout& lay, uint32_t epoch,
+                             cudaStream_t s);
+// Waits (bounded) for every rank's counts, then: this rank's block list over its experts
+// (mblocks, num_mblocks, scheduler words zeroed), its received row count, and dst[e] for
+// every expert (where this rank's rows of e go).
+cudaError_t launch_ep_layout(const TpGroup& g, const EpLayout& lay, int E, BlockScales bs, MBlock* mblocks,
+                             int32_t* num_mblocks, uint32_t* sched, int sched_n, EpDest* dst, int32_t* own_rows,
+                             uint32_t epoch, uint32_t* err, cudaStream_t s);
+// Quantises this rank's tokens once (A1 = Q(x), NVFP4 or MXFP8) and stores each slot's row
+// into the activation tiles of its expert's rank (peer stores), its origin, then adds the
+// row to that block's arrival counter (release, system scope).
+cudaError_t launch_ep_dispatch(const uint16_t* x, const int32_t* ids, const int32_t* inv, const int32_t* offsets,
+                               const EpDest* dst, int T, int H, int k, int fmt, float alpha, const TpGroup& g,
+                               const EpLayout& lay, cudaStream_t s);
+// Returns every received row's expert output to its source slot (peer stores), then sets
+// this rank's return flag in every rank's region (release, system scope).
+cudaError_t launch_ep_combine(const uint16_t* y, const int32_t* own_rows, int H, const TpGroup& g,
+                              const EpLayout& lay, uint32_t epoch, unsigned int* counter, int grid, cudaStream_t s);
+// Waits (bounded) until every rank returned this epoch's rows; lets its dependents start
+// only when it ends.
+cudaError_t launch_ep_wait_returned(const TpGroup& g, uint32_t epoch, uint32_t* err, cudaStream_t s);
 
 // ---- finalize (finalize.cu)
 // next_x != nullptr also writes the next sublayer's pre-norm of out: bf16(out * rinv * next_gamma).

@@ -42,7 +42,7 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
                             int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
                             int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks,
                             int32_t* __restrict__ num_mblocks, uint32_t* __restrict__ sched, int sched_n,
-                            BlockScales bs, int pair) {
+                            BlockScales bs) {
   __shared__ int warp_sums[33];
   pdl_wait();
   pdl_trigger();
@@ -58,13 +58,10 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
       cnt += v;
     }
   }
-  // Activations live in 128-row blocks (sf_block); the work list uses 128-row blocks, or
-  // 256-row blocks (two consecutive activation blocks, the second possibly empty) when a
-  // CTA pair computes each tile.
+  // Activations live in 128-row blocks (sf_block), and so does the work list.
   const int nblk = (cnt + 127) / 128;
-  const int wrows = pair ? 256 : 128;
   const bool held = e >= bs.e_begin && e < bs.e_end;  // this handle has the expert's weights
-  const int nwork = held ? (cnt + wrows - 1) / wrows : 0;
+  const int nwork = held ? nblk : 0;
   int total_rows, total_blk, total_work;
   const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
   const int blk = block_exclusive_scan(nblk, warp_sums, total_blk);
@@ -76,9 +73,9 @@ __global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chun
     for (int i = 0; i < nwork; ++i) {
       MBlock m;
       m.expert = e - bs.e_begin;
-      m.row_begin = off + wrows * i;
-      m.rows = min(wrows, cnt - wrows * i);
-      m.sf_block = blk + (wrows / 128) * i;
+      m.row_begin = off + 128 * i;
+      m.rows = min(128, cnt - 128 * i);
+      m.sf_block = blk + i;
       m.scale_gu = bs.alpha_a1 * __ldg(bs.w_gu_alpha + m.expert);
       m.scale_d = bs.alpha_a2 * __ldg(bs.w_d_alpha + m.expert);
       m.pad[0] = m.pad[1] = 0;
@@ -209,20 +206,27 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
   // Lanes 2c, 2c + 1 hold the two halves of one 16-byte code chunk and lanes 4g..4g + 3 the
   // four scale bytes of one K-group (nb is a multiple of 4): one 16-byte code store per lane
-  // pair and one 4-byte scale store per lane quad, per slot.  The next iteration's 32 bytes
-  // are loaded before this one's quantisation (its divisions hide the load latency).
-  uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+  // pair and one 4-byte scale store per lane quad, per slot.  The next two iterations' 32
+  // bytes per lane are in flight during this one's quantisation (more bytes in flight per
+  // warp: the loads' latency, not their issue, bounds this kernel).
+  uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0, f0 = n0, f1 = n0;
   if (lane < nb) {
     n0 = __ldg(xr + 2 * lane);
     n1 = __ldg(xr + 2 * lane + 1);
+  }
+  if (lane + 32 < nb) {
+    f0 = __ldg(xr + 2 * (lane + 32));
+    f1 = __ldg(xr + 2 * (lane + 32) + 1);
   }
   for (int b0 = 0; b0 < nb; b0 += 32) {
     const int b = b0 + lane;
     const bool active = b < nb;  // whole quads are active or not
     const uint4 p0 = n0, p1 = n1;
-    if (b + 32 < nb) {
-      n0 = __ldg(xr + 2 * (b + 32));
-      n1 = __ldg(xr + 2 * (b + 32) + 1);
+    n0 = f0;
+    n1 = f1;
+    if (b + 64 < nb) {
+      f0 = __ldg(xr + 2 * (b + 64));
+      f1 = __ldg(xr + 2 * (b + 64) + 1);
     }
     uint32_t lo = 0, hi = 0, sc = 0;
     if (active) {
@@ -363,10 +367,10 @@ cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* 
 
 cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
-                        BlockScales bs, int pair, cudaStream_t s) {
+                        BlockScales bs, cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
   return launch_pdl(scan_kernel, dim3(1), dim3(threads), 0, s, chunk_counts, n_chunks, E, chunk_base, offsets,
-                    sf_block, mblocks, num_mblocks, sched, sched_n, bs, pair);
+                    sf_block, mblocks, num_mblocks, sched, sched_n, bs);
 }
 
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,

@@ -16,6 +16,8 @@ from __future__ import annotations
 from . import MoELayer, beam_moe_ipc_export, beam_moe_ipc_import
 
 WEIGHT_KEYS = ("w_gu", "w_gu_sf", "w_d", "w_d_sf")
+TP_PHASES = 3  # phases of beam_moe_forward_tp_phase
+EP_PHASES = 4  # phases of beam_moe_forward_ep_phase
 
 
 def shard_weights(weights: dict, rank: int, world: int, inter: int) -> dict:
@@ -97,10 +99,12 @@ class SharedGpuGroup:
     measurement when fewer GPUs than ranks are available).  The ranks run one after the
     other, phase by phase: every rank's phase p before any rank's phase p + 1, so no kernel
     waits on a kernel that has not run.  Tensor parallel: phase 0 (GEMMs, partial m,
-    publication), phase 1 (all-reduce + finalize); every rank gets the same x.  Expert
-    parallel (layers created with an expert range): phase 0 (dispatch), 1 (routing of the
-    gathered batch, the rank's experts, partial m), 2 (combine + finalize); each rank its own
-    x and residual."""
+    publication), phase 1 (all-reduce + finalize, of the rank's slice from 256 tokens on),
+    phase 2 (the other slices' rows, from 256 tokens on); every rank gets the same x.  Expert
+    parallel (layers created with an expert range): phase 0 (routing of the rank's own
+    tokens, count publication), 1 (layout, dispatch of the routed rows), 2 (the rank's
+    experts on the rows it received, return of the outputs), 3 (finalize of the rank's own
+    tokens); each rank its own x and residual."""
 
     def __init__(self, layers):
         self.layers = list(layers)
@@ -115,15 +119,14 @@ class SharedGpuGroup:
         import torch
         if self.expert_parallel:
             outs = outs or [torch.empty_like(r) for r in residual]
-            for phase in range(3):
+            for phase in range(EP_PHASES):
                 for lay, xr, rr, o in zip(self.layers, x, residual, outs):
                     lay.forward_ep_phase(xr, rr, o, phase)
             return outs
         outs = outs or [torch.empty_like(residual) for _ in self.layers]
-        for lay, o in zip(self.layers, outs):
-            lay.forward_tp_phase(x, residual, o, 0)
-        for lay, o in zip(self.layers, outs):
-            lay.forward_tp_phase(x, residual, o, 1)
+        for phase in range(TP_PHASES):
+            for lay, o in zip(self.layers, outs):
+                lay.forward_tp_phase(x, residual, o, phase)
         return outs
 
     def close(self):

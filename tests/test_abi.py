@@ -71,15 +71,14 @@ def test_host_side_validation_of_the_variant_and_parallel_entry_points():
     assert lib.beam_moe_quantize_mxfp8(None, 4, 64, None, None, None) == bad      # null buffers
     assert lib.beam_moe_expert_format(None) == -1
     assert lib.beam_moe_set_router_mode(None, pkg.ROUTER_AUTO) == bad
-    assert lib.beam_moe_set_gemm_mode(None, pkg.GEMM_AUTO) == bad
     assert lib.beam_moe_tp_region_bytes(None) == 0
     p = ctypes.c_void_p()
     assert lib.beam_moe_tp_region(None, ctypes.byref(p)) == bad
     assert lib.beam_moe_tp_attach(None, 0, 2, None, None) == bad
     assert lib.beam_moe_forward_tp(None, None, None, None, 4, None) == bad
-    assert lib.beam_moe_forward_tp_phase(None, None, None, None, 4, 2, None) == bad  # phase 0 or 1
+    assert lib.beam_moe_forward_tp_phase(None, None, None, None, 4, 3, None) == bad  # phase 0, 1 or 2
     assert lib.beam_moe_forward_ep(None, None, None, None, 4, None) == bad
-    assert lib.beam_moe_forward_ep_phase(None, None, None, None, 4, 3, None) == bad  # phase 0, 1 or 2
+    assert lib.beam_moe_forward_ep_phase(None, None, None, None, 4, 4, None) == bad  # phase 0 .. 3
     assert lib.beam_moe_ipc_export(None, None) == bad
     assert lib.beam_moe_ipc_import(None, ctypes.byref(p)) == bad
     assert lib.beam_moe_ipc_close(None) == bad

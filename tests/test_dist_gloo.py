@@ -215,7 +215,7 @@ class _PhaseLayer:
 @pytest.mark.parametrize("ep", [False, True])
 def test_shared_gpu_group_runs_every_rank_phase_by_phase(ep):
     # Ranks sharing one GPU must never have a kernel wait on a kernel that has not run: every
-    # rank's phase p is enqueued before any rank's phase p + 1 (TP: 2 phases, EP: 3).
+    # rank's phase p is enqueued before any rank's phase p + 1 (TP: 2 phases, EP: 4).
     from sparse_moe_layer_fp32_b200 import tp
     log = []
     layers = [_PhaseLayer(log, r, ep) for r in range(3)]
@@ -226,5 +226,5 @@ def test_shared_gpu_group_runs_every_rank_phase_by_phase(ep):
         grp.forward(xs, xs, outs=[torch.zeros(2, 8) for _ in range(3)])
     else:
         grp.forward(xs[0], xs[0], outs=[torch.zeros(2, 8) for _ in range(3)])
-    phases = 3 if ep else 2
+    phases = tp.EP_PHASES if ep else tp.TP_PHASES
     assert log == [("ep" if ep else "tp", r, p) for p in range(phases) for r in range(3)]

@@ -3,13 +3,15 @@ beam_moe_forward_ep through the C ABI) on one GPU.
 
 The vLLM PR "Day-0 support for Reflection's Beam-1.0" (section "Status") pairs attention
 data parallelism with the MegaMoE expert kernels; each rank owns E / W of the experts and
-its own batch.  One GPU holds every rank here (SharedGpuGroup): each phase (dispatch;
-routing of the gathered batch + the rank's experts + partial m; combine + finalize) runs
-for every rank before the next phase, so the exchange waits are satisfied when they run.
-Checks: each rank's output matches the oracle's expert-parallel layer (= the unsharded
-layer on the concatenated batch) at the layer's tolerances and a single handle with all
-experts closely; repeated forwards repeat the bits; handles holding part of the experts
-refuse the single-GPU and tensor-parallel forwards.
+its own batch, and only routed rows travel: each rank routes and quantises its own tokens,
+stores each slot's row into the activation tiles of its expert's rank, the rank computes the
+rows it received and returns each output row to its source slot, and each rank finalizes
+its own tokens.  One GPU holds every rank here (SharedGpuGroup): each of the four phases
+runs for every rank before the next phase, so the exchange waits are satisfied when they
+run.  Checks: each rank's output matches the oracle's expert-parallel layer at the layer's
+tolerances and is bit-identical to a handle with all experts run on that rank's tokens;
+repeated forwards repeat the bits; phases out of order, unequal expert ranges and the
+single-GPU and tensor-parallel forwards are refused.
 """
 
 import dataclasses
@@ -33,12 +35,24 @@ def bm():
     return m
 
 
+def _ep_layers(bm, shape, full, world, max_tokens, a1, a2, fmt):
+    from sparse_moe_layer_fp32_b200 import tp
+    E, e_loc = shape.experts, shape.experts // world
+    layers = []
+    for r in range(world):
+        sh = tp.shard_experts(full, r, world, E)
+        layers.append(bm.MoELayer(max_tokens=max_tokens, hidden=shape.hidden, num_experts=E, top_k=shape.top_k,
+                                  inter=shape.inter, alpha_a1=float(a1), alpha_a2=float(a2), fmt=fmt,
+                                  expert_begin=r * e_loc, expert_count=e_loc, **sh))
+    return layers
+
+
 @pytest.mark.parametrize("name,fmt,world,tokens,seed", [("tiny", "nvfp4", 2, 3, 40), ("mid", "nvfp4", 4, 2, 41),
                                                         ("mid", "nvfp4", 4, 80, 42), ("tiny", "mxfp8", 4, 70, 43),
-                                                        ("mid", "mxfp8", 2, 300, 44)])
-def test_ep_matches_oracle(bm, name, fmt, world, tokens, seed):
+                                                        ("mid", "mxfp8", 2, 300, 44), ("mid", "nvfp4", 2, 600, 45)])
+def test_ep_matches_oracle_and_single_gpu_bits(bm, name, fmt, world, tokens, seed):
     from sparse_moe_layer_fp32_b200 import synthetic, tp
-    shape = dataclasses.replace(SHAPES[name], tokens=world * tokens)  # the gathered batch
+    shape = dataclasses.replace(SHAPES[name], tokens=world * tokens)  # every rank's batch together
     x, res, wr, g, cache = oracle_layer_inputs(shape, seed, fmt=fmt)
     if fmt == "nvfp4":
         a1 = np.float32(np.float32(np.abs(x).max()) / np.float32(2688))
@@ -47,13 +61,7 @@ def test_ep_matches_oracle(bm, name, fmt, world, tokens, seed):
     else:
         a1 = a2 = np.float32(1.0)
     full = synthetic.make_weights(shape, seed, threads=4, fmt=fmt)
-    E, e_loc = shape.experts, shape.experts // world
-    layers = []
-    for r in range(world):
-        sh = tp.shard_experts(full, r, world, E)
-        layers.append(bm.MoELayer(max_tokens=world * tokens, hidden=shape.hidden, num_experts=E,
-                                  top_k=shape.top_k, inter=shape.inter, alpha_a1=float(a1), alpha_a2=float(a2),
-                                  fmt=fmt, expert_begin=r * e_loc, expert_count=e_loc, **sh))
+    layers = _ep_layers(bm, shape, full, world, world * tokens, a1, a2, fmt)
     grp = tp.SharedGpuGroup(layers)
     xd, rd = synthetic.make_batch(shape, seed)
     xs = [xd[r * tokens:(r + 1) * tokens].contiguous() for r in range(world)]
@@ -63,26 +71,51 @@ def test_ep_matches_oracle(bm, name, fmt, world, tokens, seed):
         lay.check()
     torch.cuda.synchronize()
     ref = moe.moe_forward_ep([x[r * tokens:(r + 1) * tokens] for r in range(world)],
-                             [res[r * tokens:(r + 1) * tokens] for r in range(world)], wr, g, cache, E, shape.top_k,
-                             a1 if fmt == "nvfp4" else None, a2 if fmt == "nvfp4" else None, world, shape.rms_eps)
+                             [res[r * tokens:(r + 1) * tokens] for r in range(world)], wr, g, cache, shape.experts,
+                             shape.top_k, a1 if fmt == "nvfp4" else None, a2 if fmt == "nvfp4" else None, world,
+                             shape.rms_eps)
     got = np.concatenate([bf16_to_f64(o) for o in outs])
     rel, mx = compare_outputs(got, np.concatenate(ref["out_pre"]), skip=ref["near_tie"])
     assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
-    whole = bm.MoELayer(max_tokens=world * tokens, hidden=shape.hidden, num_experts=E, top_k=shape.top_k,
+    # the same bits as one handle with every expert, run on each rank's own tokens
+    whole = bm.MoELayer(max_tokens=world * tokens, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
                         inter=shape.inter, alpha_a1=float(a1), alpha_a2=float(a2), fmt=fmt, **full)
-    rel1, _ = compare_outputs(got, bf16_to_f64(whole.forward(xd, rd)))
-    assert rel1 < 5e-3, rel1
+    for r in range(world):
+        assert torch.equal(outs[r], whole.forward(xs[r], rs[r])), r
     whole.close()
-    for _ in range(2):  # the gathered and partial buffers alternate by epoch
+    for _ in range(2):  # the regions are reused forward after forward
         again = grp.forward(xs, rs)
         for o, a in zip(outs, again):
             assert torch.equal(o, a)
     for lay in layers:
         lay.check()
-    # a handle that holds part of the experts runs only the expert-parallel forward
+    # a handle that holds part of the experts runs only the expert-parallel forward, its
+    # phases in order
     with pytest.raises(bm.BeamMoeError) as ei:
         layers[0].forward(xs[0], rs[0])
     assert ei.value.status == bm.ERR_INVALID_ARG
     with pytest.raises(bm.BeamMoeError):
         layers[0].forward_tp(xs[0], rs[0])
+    with pytest.raises(bm.BeamMoeError):
+        layers[0].forward_ep_phase(xs[0], rs[0], outs[0], 2)
     grp.close()
+
+
+def test_ep_attach_refuses_unequal_expert_ranges(bm):
+    from sparse_moe_layer_fp32_b200 import synthetic, tp
+    shape = dataclasses.replace(SHAPES["tiny"], tokens=4)
+    full = synthetic.make_weights(shape, 3, threads=2)
+    # 16 experts over 2 ranks as 4 + 12: not the equal ranges the layout needs
+    layers = []
+    for begin, count in ((0, 4), (4, 12)):
+        sh = dict(full)
+        for key in ("w_gu", "w_gu_sf", "w_d", "w_d_sf", "w_gu_alpha", "w_d_alpha"):
+            sh[key] = full[key][begin:begin + count].contiguous()
+        layers.append(bm.MoELayer(max_tokens=8, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                                  inter=shape.inter, alpha_a1=0.001, alpha_a2=0.0001, expert_begin=begin,
+                                  expert_count=count, **sh))
+    with pytest.raises(bm.BeamMoeError) as ei:
+        tp.SharedGpuGroup(layers)
+    assert ei.value.status == bm.ERR_INVALID_ARG
+    for lay in layers:
+        lay.close()

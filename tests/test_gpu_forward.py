@@ -205,31 +205,6 @@ def test_forward_with_fused_next_prenorm(bm, name, tokens, seed):
     layer.close()
 
 
-@pytest.mark.parametrize("name,tokens,seed", [("tiny", 1500, 3), ("mid", 2000, 11), ("mid", 300, 12)])
-def test_pair_gemm_matches_oracle_and_single_cta(bm, name, tokens, seed):
-    # The CTA-pair expert GEMM (256-row work blocks, one M = 256 MMA over two SMs) against the
-    # oracle and against the single-CTA GEMM on the same inputs.  ~190, ~250 and ~37 rows per
-    # expert: full pairs, pairs whose second half is partly filled, and empty second halves.
-    shape, layer, weights, out_single, ref, _ = _run(bm, SHAPES[name], tokens, seed)
-    from sparse_moe_layer_fp32_b200 import synthetic
-    xd, rd = synthetic.make_batch(shape, seed)
-    layer.set_gemm_mode(bm.GEMM_SINGLE)
-    out_s = layer.forward(xd, rd)
-    layer.check()
-    assert torch.equal(out_s, out_single)  # AUTO picks the single-CTA GEMM at this size
-    layer.set_gemm_mode(bm.GEMM_PAIR)
-    out_p = layer.forward(xd, rd)
-    layer.check()
-    torch.cuda.synchronize()
-    rel, mx = compare_outputs(bf16_to_f64(out_p), ref["out_pre"], skip=ref["near_tie"])
-    assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
-    d_rel, _ = compare_outputs(bf16_to_f64(out_p), bf16_to_f64(out_s))
-    assert d_rel < 1e-3, d_rel
-    with pytest.raises(bm.BeamMoeError):
-        layer.set_gemm_mode(7)
-    layer.close()
-
-
 # ---------------------------------------------------------------- MXFP8 experts
 # The block-scaled FP8 variant (the recipe's FP8 checkpoint, section "Variants", read as
 # MXFP8: E4M3 values and one power-of-two scale per 32 values for weights, A1 and A2),
@@ -297,10 +272,6 @@ def test_forward_mxfp8_stages_and_end_to_end(bm, name, tokens, seed):
     assert np.all(np.abs(out_np - pre) <= 2.0 ** -8 * np.maximum(np.abs(pre), 1.0))
     rel, mx = compare_outputs(out_np, ref["out_pre"], skip=near)
     assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
-    # the CTA-pair GEMM is NVFP4 only
-    with pytest.raises(bm.BeamMoeError) as ei:
-        layer.set_gemm_mode(bm.GEMM_PAIR)
-    assert ei.value.status == bm.ERR_UNSUPPORTED
     layer.close()
 
 

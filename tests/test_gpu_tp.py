@@ -7,9 +7,12 @@ all-reduce with the sandwich norms and the MoE finalize; the recipe
 here (SharedGpuGroup): every rank's phase 0 runs before any rank's phase 1, so the exchange
 waits are satisfied when they run.  Checks: all ranks produce identical bits; the output
 matches the oracle's tensor-parallel layer (= the unsharded layer) at the layer's
-tolerances and a single handle holding all experts closely; repeated forwards (the
-exchange buffers alternate by epoch) repeat the bits; a peer that never publishes makes
-the wait give up with a TIMEOUT status and the group recovers after a re-attach.
+tolerances and a single handle holding all experts closely; from 256 tokens on the
+all-reduce is two-shot (each rank finishes its slice of the tokens, then gathers the
+others'), and its bits equal the one-shot form's (the same batch in halves below 256
+tokens: every token's result is independent of the rest of the batch); repeated forwards
+(the exchange buffers alternate by epoch) repeat the bits; a peer that never publishes
+makes the wait give up with a TIMEOUT status and the group recovers after a re-attach.
 """
 
 import dataclasses
@@ -52,7 +55,8 @@ def _group(bm, shape, full, world, tokens, fmt, a1, a2):
 
 
 @pytest.mark.parametrize("fmt,world,tokens,seed", [("nvfp4", 2, 5, 30), ("nvfp4", 4, 40, 31), ("nvfp4", 4, 300, 32),
-                                                   ("mxfp8", 2, 7, 33), ("mxfp8", 4, 260, 34)])
+                                                   ("mxfp8", 2, 7, 33), ("mxfp8", 4, 260, 34),
+                                                   ("nvfp4", 2, 301, 35), ("nvfp4", 4, 257, 36)])
 def test_tp_matches_oracle_and_ranks_agree(bm, fmt, world, tokens, seed):
     from sparse_moe_layer_fp32_b200 import synthetic
     shape = dataclasses.replace(SHAPE, tokens=tokens)
@@ -67,6 +71,13 @@ def test_tp_matches_oracle_and_ranks_agree(bm, fmt, world, tokens, seed):
     torch.cuda.synchronize()
     for o in outs[1:]:
         assert torch.equal(o, outs[0])  # every rank holds the same output
+    if tokens >= 256:  # two-shot; the same tokens in two one-shot batches give the same bits
+        h = tokens // 2
+        halves = [grp.forward(xd[:h].contiguous(), rd[:h].contiguous()),
+                  grp.forward(xd[h:].contiguous(), rd[h:].contiguous())]
+        for lay in grp.layers:
+            lay.check()
+        assert torch.equal(torch.cat([halves[0][0], halves[1][0]]), outs[0])
     ref = moe.moe_forward_tp(x, res, wr, g, cache, shape.top_k, a1 if fmt == "nvfp4" else None,
                              a2 if fmt == "nvfp4" else None, world, shape.rms_eps)
     got = bf16_to_f64(outs[0])
