@@ -43,7 +43,6 @@ import moe_inputs as mi  # noqa: E402
 METRIC = "moe_layer_tokens_per_s"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 512 << 20  # written between timed steps (L2 is 126 MB)
-TP_TWO_SHOT_MIN_TOKENS = 256  # the library reduces in two steps from this batch on
 
 
 def peaks():
@@ -635,7 +634,7 @@ def run_tp_shared(args, shape):
     if ep:  # dispatch: x read once, each slot's quantised row stored at its expert's rank
         top, nbytes = "ep_dispatch", T * H * 2 + T * k * H * q
         exchange = T * k * H * q + T * k * H * 2  # per rank: its rows out, their outputs back
-    elif T >= TP_TWO_SHOT_MIN_TOKENS:  # two-shot: the W partials of the rank's slice, residual, out and row buffer
+    elif T >= bm.TP_TWO_SHOT_MIN_TOKENS:  # two-shot: the W partials of the rank's slice, residual, out and row buffer
         S = -(-T // W)
         top, nbytes = "tp_reduce", T * H * 4 + 3 * S * H * 2 + H * 2
         exchange = (W - 1) * S * H * 4 + (T - S) * H * 2  # peers' partials of the slice, peers' rows

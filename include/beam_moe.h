@@ -201,6 +201,14 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_tp(beam_moe_t h, const void* x, co
  * not run. */
 BEAM_MOE_API beam_moe_status beam_moe_forward_tp_phase(beam_moe_t h, const void* x, const void* residual, void* out,
                                                        int32_t num_tokens, int32_t phase, void* stream);
+/* The batch size from which beam_moe_forward_tp reduces in two steps (default
+ * BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS; INT32_MAX keeps the one-shot form for every batch).  A
+ * batch whose slices would not all hold a token (T < W^2 can do that) stays one-shot.  Both
+ * forms give the same bits; the choice only moves the exchange's bytes and latency.  Takes
+ * effect at the next phase 0; all ranks of a group must use the same value.  Not from the
+ * source pages: exposed for tuning and testing.  INVALID_ARG for min_tokens < 1. */
+#define BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS 256
+BEAM_MOE_API beam_moe_status beam_moe_set_tp_two_shot_tokens(beam_moe_t h, int32_t min_tokens);
 /* cudaIpcGetMemHandle / cudaIpcOpenMemHandle / cudaIpcCloseMemHandle of a region, as
  * BEAM_MOE_IPC_HANDLE_BYTES opaque bytes (host memory), so that callers need no CUDA
  * headers. */

@@ -51,7 +51,8 @@ struct beam_moe_ctx {
   TpGroup tp;                   // every rank's region, this rank, the group size
   bool tp_attached;
   int tp_next_phase;            // the phase of beam_moe_forward_tp_phase that may run next (0..2)
-  bool tp_two_shot;             // the forward in flight reduces in two steps (its T >= kTpTwoShotMinTokens)
+  bool tp_two_shot;             // the forward in flight reduces in two steps
+  int32_t tp_two_shot_min;      // from this batch size on (beam_moe_set_tp_two_shot_tokens)
   uint32_t tp_epoch;            // forwards so far in this group (the flag value of the last one)
   unsigned int* tp_counter;     // CTA arrivals of tp_partial [0] and of the two-shot tp_reduce [1]
   int tp_last_T;
@@ -246,6 +247,7 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   h->last_launches = 0;
   h->profiling = false;
   h->router_mode = BEAM_MOE_ROUTER_AUTO;
+  h->tp_two_shot_min = BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS;
   h->profiled_last = false;
   for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i) {
     h->events[i] = nullptr;
@@ -587,9 +589,11 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
       // tensor cores over (token tiles) x (slices of H), partial logits; the top-k kernel
       // sums the slices in order
       CUtensorMap map_x;
-      if (!make_map_bf16(&map_x, xb, H, T, 128u)) return BEAM_MOE_ERR_CUDA;
-      const int splits = router_tc_split_count(T, H, h->num_sms);
-      BEAM_TRY(launch_router_tc(map_x, 128, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s, splits));
+      const RouterTcPlan plan = router_tc_split_plan(T, H, h->num_sms);
+      if (!make_map_bf16(&map_x, xb, H, T, static_cast<uint32_t>(plan.tokens))) return BEAM_MOE_ERR_CUDA;
+      const int splits = plan.splits;
+      BEAM_TRY(launch_router_tc(map_x, plan.tokens, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s,
+                                splits));
       BEAM_TRY(mark("router_tc"));
       ++launches;
       h->last_splits = splits;
@@ -654,7 +658,9 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     ++launches;
     ++h->tp_epoch;
     h->tp_next_phase = 1;
-    h->tp_two_shot = h->tp.world > 1 && T >= kTpTwoShotMinTokens;
+    // two-shot only when every rank's slice of ceil(T / W) tokens holds one
+    h->tp_two_shot = h->tp.world > 1 && T >= h->tp_two_shot_min &&
+                     static_cast<int64_t>(tp_slice_tokens(T, h->tp.world)) * (h->tp.world - 1) < T;
     h->tp_last_T = T;
   } else {
     if (residual_ready) BEAM_TRY(cudaStreamWaitEvent(s, residual_ready, 0));
@@ -930,6 +936,12 @@ beam_moe_status beam_moe_debug_wait_timeout(beam_moe_t h, int64_t limit_ns, void
   if (!h || limit_ns <= 0 || limit_ns > static_cast<int64_t>(kWaitLimitNs)) return BEAM_MOE_ERR_INVALID_ARG;
   wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns), h->err);
   BEAM_TRY(cudaGetLastError());
+  return BEAM_MOE_OK;
+}
+
+beam_moe_status beam_moe_set_tp_two_shot_tokens(beam_moe_t h, int32_t min_tokens) {
+  if (!h || min_tokens < 1) return BEAM_MOE_ERR_INVALID_ARG;
+  h->tp_two_shot_min = min_tokens;
   return BEAM_MOE_OK;
 }
 

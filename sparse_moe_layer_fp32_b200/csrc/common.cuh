@@ -315,25 +315,9 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
   return __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-// E2M1 codes of fl32(v0 / d) and fl32(v1 / d) (IEEE division, round-to-nearest-even), as
-// cvt_e2m1x2 of the two quotients, without dividing in the common case.  r = v * fl32(1/d)
-// is within 1.5 * 2^-23 (relative) of v / d, and fl32(v / d) within 2^-24 of it, so both lie
-// in the band r (1 -+ 2^-20).  E2M1 rounding is monotone: when both ends of the band give
-// the same code, every value inside the band (the exact quotient among them) gives it too.
-// Only a quotient within about 2^-20 of one of the format's rounding midpoints (0.25, 0.75,
-// 1.25, 1.75, 2.5, 3.5, 5) can give different ends; those few take the IEEE divisions.
-__device__ __forceinline__ uint32_t e2m1x2_of_quotients(float v0, float v1, float d, float inv_d) {
-  constexpr float kBandLo = 1.0f - 0x1p-20f, kBandHi = 1.0f + 0x1p-20f;
-  const float r0 = __fmul_rn(v0, inv_d), r1 = __fmul_rn(v1, inv_d);
-  const uint32_t c_lo = cvt_e2m1x2(__fmul_rn(r0, kBandLo), __fmul_rn(r1, kBandLo));
-  const uint32_t c_hi = cvt_e2m1x2(__fmul_rn(r0, kBandHi), __fmul_rn(r1, kBandHi));
-  if (c_lo == c_hi) return c_lo;
-  return cvt_e2m1x2(__fdiv_rn(v0, d), __fdiv_rn(v1, d));
-}
-
 // NVFP4 quantisation of one block of 16 FP32 values with tensor scale alpha:
 // s = amax / (6 alpha), S = E4M3(s), d = S alpha, q_i = E2M1(v_i / d); S == 0 -> all 0
-// (every step an IEEE FP32 operation; the 16 quotients as in e2m1x2_of_quotients).
+// (every step an IEEE FP32 operation).
 // Writes 8 code bytes (little-endian in two uint32) and returns the scale code.
 __device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float alpha, float six_alpha, uint32_t& lo,
                                                   uint32_t& hi) {
@@ -346,15 +330,9 @@ __device__ __forceinline__ uint32_t quant_block16(const float (&v)[16], float al
     return 0;
   }
   const float d = __fmul_rn(e4m3_value(sc), alpha);
-  const float inv_d = __frcp_rn(d);
   uint32_t b[8];
-  if (inv_d < 0x1p126f) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = e2m1x2_of_quotients(v[2 * i], v[2 * i + 1], d, inv_d);
-  } else {  // d below 2^-126 (a subnormal tensor scale): the bound above does not hold
-#pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = cvt_e2m1x2(__fdiv_rn(v[2 * i], d), __fdiv_rn(v[2 * i + 1], d));
-  }
+  for (int i = 0; i < 8; ++i) b[i] = cvt_e2m1x2(__fdiv_rn(v[2 * i], d), __fdiv_rn(v[2 * i + 1], d));
   lo = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
   hi = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
   return sc;

@@ -30,6 +30,8 @@
 // phase (every rank's phase p before any rank's phase p + 1); every wait is then already
 // satisfied when it runs.  Every wait is bounded (kWaitLimitNs) and reports a timeout in the
 // error word.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -127,26 +129,29 @@ __global__ void __launch_bounds__(1024) ep_layout_kernel(TpGroup g, EpLayout lay
 }
 
 // ------------------------------------------------------------------ phase 1: dispatch
-// One warp per token: the token's row is quantised once, 16 (NVFP4) or 32 (MXFP8) values per
-// lane per step, and each 16-byte chunk / scale word stored into every slot's destination.
+// One CTA per token, one lane per 16-value (NVFP4) or 32-value (MXFP8) block of its row (a
+// single step at H = 5120: every load of the row is in flight at once): the row is quantised
+// once and each 16-byte chunk / scale word stored into every slot's destination; after a
+// barrier, thread j publishes slot j (its origin, then a release add on its block's arrival
+// counter, which covers the whole CTA's stores).
+constexpr int kEpMaxK = 16;
+constexpr int kEpDispatchThreads = 512;
 template <bool kMx>
-__global__ void __launch_bounds__(256) ep_dispatch_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ ids,
-                                                          const int32_t* __restrict__ inv,
-                                                          const int32_t* __restrict__ offsets,
-                                                          const EpDest* __restrict__ dst, int T, int H, int k,
-                                                          float alpha, TpGroup g, EpLayout lay) {
-  __shared__ uint8_t* s_a1[8][16];
-  __shared__ uint8_t* s_sf[8][16];
-  __shared__ int s_blk[8][16], s_m[8][16];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int t = blockIdx.x * 8 + warp;
+__global__ void __launch_bounds__(kEpDispatchThreads) ep_dispatch_kernel(
+    const uint16_t* __restrict__ x, const int32_t* __restrict__ ids, const int32_t* __restrict__ inv,
+    const int32_t* __restrict__ offsets, const EpDest* __restrict__ dst, int T, int H, int k, float alpha, TpGroup g,
+    EpLayout lay) {
+  __shared__ uint8_t* s_a1[kEpMaxK];
+  __shared__ uint8_t* s_sf[kEpMaxK];
+  __shared__ int s_blk[kEpMaxK], s_m[kEpMaxK];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (t >= T) return;
   int row = 0, blk = 0, dr = 0;
-  bool in_range = true;
-  if (lane < k) {
-    const size_t i = static_cast<size_t>(t) * k + lane;
+  bool in_range = false;
+  if (tid < k) {
+    const size_t i = static_cast<size_t>(t) * k + tid;
     const int e = ids[i];
     const EpDest o = dst[e];
     const int li = inv[i] - offsets[e];  // this token's rank among this rank's rows of e
@@ -154,19 +159,21 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(const uint16_t* __rest
     row = o.row0 + li;
     blk = o.blk0 + (pos >> 7);
     dr = o.rank;
-    in_range = blk < lay.nblk && dr < g.world;
-    s_a1[warp][lane] = g.regions[in_range ? dr : g.rank] + lay.a1;
-    s_sf[warp][lane] = g.regions[in_range ? dr : g.rank] + lay.a1_sf;
-    s_blk[warp][lane] = in_range ? blk : -1;
-    s_m[warp][lane] = pos & 127;
+    in_range = blk < lay.nblk && dr < g.world && row < lay.rows;
+    s_a1[tid] = g.regions[in_range ? dr : g.rank] + lay.a1;
+    s_sf[tid] = g.regions[in_range ? dr : g.rank] + lay.a1_sf;
+    s_blk[tid] = in_range ? blk : -1;
+    s_m[tid] = pos & 127;
   }
-  __syncwarp();
+  __syncthreads();
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
   if constexpr (!kMx) {
     const float six_alpha = __fmul_rn(6.0f, alpha);
     const int nb = H / 16, kgroups = H / 64;
-    for (int b0 = 0; b0 < nb; b0 += 32) {
-      const int b = b0 + lane;
+    // the loop bound is the same for the whole warp (blockDim is a multiple of 32): shuffles
+    // below always see every lane
+    for (int b0 = 0; b0 < nb; b0 += blockDim.x) {
+      const int b = b0 + tid;
       const bool active = b < nb;  // whole quads are active or not (nb % 4 == 0)
       uint32_t lo = 0, hi = 0, sc = 0;
       if (active) {
@@ -187,17 +194,17 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(const uint16_t* __rest
       const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
       if (!active || (lane & 1)) continue;
       for (int j = 0; j < k; ++j) {
-        const int bj = s_blk[warp][j], m = s_m[warp][j];
+        const int bj = s_blk[j], m = s_m[j];
         if (bj < 0) continue;
-        *reinterpret_cast<uint4*>(s_a1[warp][j] + act_tile_offset(bj, H / 256, b >> 4, m, (b & 15) >> 1)) =
+        *reinterpret_cast<uint4*>(s_a1[j] + act_tile_offset(bj, H / 256, b >> 4, m, (b & 15) >> 1)) =
             make_uint4(lo, hi, lo1, hi1);
-        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_sf[warp][j] + sf_atom_offset(bj, kgroups, m, b)) = word;
+        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_sf[j] + sf_atom_offset(bj, kgroups, m, b)) = word;
       }
     }
   } else {
     const int nb = H / 32, k_tiles = H / 128;
-    for (int b0 = 0; b0 < nb; b0 += 32) {
-      const int b = b0 + lane;
+    for (int b0 = 0; b0 < nb; b0 += blockDim.x) {
+      const int b = b0 + tid;
       const bool active = b < nb;
       uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0}, sc = 0;
       if (active) {
@@ -220,17 +227,18 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(const uint16_t* __rest
       const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
       if (!active) continue;
       for (int j = 0; j < k; ++j) {
-        const int bj = s_blk[warp][j], m = s_m[warp][j];
+        const int bj = s_blk[j], m = s_m[j];
         if (bj < 0) continue;
-        st_act_pair(s_a1[warp][j], bj, k_tiles, b >> 2, m, (b & 3) * 2, c);
-        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_sf[warp][j] + sf_atom_offset(bj, k_tiles, m, b)) = word;
+        st_act_pair(s_a1[j], bj, k_tiles, b >> 2, m, (b & 3) * 2, c);
+        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_sf[j] + sf_atom_offset(bj, k_tiles, m, b)) = word;
       }
     }
   }
-  // every lane's stores of the k rows come before each slot's origin and arrival (release)
-  __syncwarp();
-  if (lane < k && in_range) {
-    reinterpret_cast<int32_t*>(g.regions[dr] + lay.origin)[row] = (g.rank << 24) | (t * k + lane);
+  // every thread's stores of the k rows come before each slot's origin and arrival: the
+  // barrier orders them before thread j, whose release add is cumulative over them
+  __syncthreads();
+  if (tid < k && in_range) {
+    reinterpret_cast<int32_t*>(g.regions[dr] + lay.origin)[row] = (g.rank << 24) | (t * k + tid);
     red_add_release_sys(reinterpret_cast<uint32_t*>(g.regions[dr] + lay.arrivals) + blk, 1u);
   }
 }
@@ -292,12 +300,15 @@ cudaError_t launch_ep_layout(const TpGroup& g, const EpLayout& lay, int E, Block
 cudaError_t launch_ep_dispatch(const uint16_t* x, const int32_t* ids, const int32_t* inv, const int32_t* offsets,
                                const EpDest* dst, int T, int H, int k, int fmt, float alpha, const TpGroup& g,
                                const EpLayout& lay, cudaStream_t s) {
-  const dim3 grid((T + 7) / 8);
-  if (fmt == BEAM_MOE_FMT_MXFP8)
-    return launch_pdl(ep_dispatch_kernel<true>, grid, dim3(256), 0, s, x, ids, inv, offsets, dst, T, H, k, alpha, g,
-                      lay);
-  return launch_pdl(ep_dispatch_kernel<false>, grid, dim3(256), 0, s, x, ids, inv, offsets, dst, T, H, k, alpha, g,
-                    lay);
+  if (k > kEpMaxK) return cudaErrorInvalidValue;
+  const bool mx = fmt == BEAM_MOE_FMT_MXFP8;
+  const int lanes = H / (mx ? 32 : 16);  // one lane per block of the row, whole warps, at most kEpDispatchThreads
+  const int threads = std::min(kEpDispatchThreads, (lanes + 31) / 32 * 32);
+  if (mx)
+    return launch_pdl(ep_dispatch_kernel<true>, dim3(T), dim3(threads), 0, s, x, ids, inv, offsets, dst, T, H, k,
+                      alpha, g, lay);
+  return launch_pdl(ep_dispatch_kernel<false>, dim3(T), dim3(threads), 0, s, x, ids, inv, offsets, dst, T, H, k, alpha,
+                    g, lay);
 }
 
 cudaError_t launch_ep_combine(const uint16_t* y, const int32_t* own_rows, int H, const TpGroup& g,

@@ -81,33 +81,28 @@ struct FmtMxfp8 {
 static_assert(B_BYTES + FmtMxfp8::SFB == kMxTileBytes, "MXFP8 weight tile = B codes + B scales");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;            // 256 FP32 columns
-constexpr uint32_t SF_COL = 256;           // scale factors, one column set per K step of a stage:
+constexpr uint32_t SF_COL = 256;           // scale factors, one column set per ring stage:
 constexpr uint32_t SF_STAGE_COLS = 48;     //   A: 4 K-groups x 4 columns, then B: 4 K-groups x 8
 constexpr uint32_t SFB_OFF = 16;
 constexpr int kMaxStages = 5;
-// A stage may hold KPS consecutive K steps: their A regions, then their weight tiles (which
-// lie back to back in global memory, so one copy brings all of them), then their A scales
-// (also contiguous: one copy).  Fewer, larger copies per K step; coarser ring granularity.
-template <int kStages, int kABytes, class F = FmtNvfp4, int kKps = 1>
+// One K step per stage (measured against two K steps per stage, whose operands arrive in
+// fewer, larger copies: 2.21 vs 1.99-2.04 ms at prefill16k, the coarser ring leaves the MMA
+// waiting longer).
+template <int kStages, int kABytes, class F = FmtNvfp4>
 struct Ring {
   using Fmt = F;
   static constexpr int STAGES = kStages;
-  static constexpr int KPS = kKps;
-  static constexpr int A_BYTES = kABytes;                    // one K step's A region
-  static constexpr int B_OFF = kKps * kABytes;               // weight tiles of the stage's K steps
-  static constexpr int SFA_OFF = B_OFF + kKps * F::TILE;     // A scales of the stage's K steps
+  static constexpr int A_BYTES = kABytes;
   // padded to 1024 bytes: every stage's operands keep the swizzle alignment
-  static constexpr int STAGE_BYTES = (SFA_OFF + kKps * F::SFA + 1023) / 1024 * 1024;
-  static constexpr uint32_t SF_COLS = kKps * SF_STAGE_COLS;  // TMEM scale columns per stage
-  static_assert(kABytes % 1024 == 0 && F::TILE % 1024 == 0, "operand regions keep the swizzle alignment");
-  static_assert(SF_COL + kStages * SF_COLS <= TMEM_COLS, "scale-factor stages must fit in TMEM");
+  static constexpr int STAGE_BYTES = (kABytes + B_BYTES + F::SFB + F::SFA + 1023) / 1024 * 1024;
+  static_assert(SF_COL + kStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor stages must fit in TMEM");
   static_assert(kStages <= kMaxStages, "barrier arrays");
 };
-using RingFull = Ring<2, A_TILE_BYTES, FmtNvfp4, 2>;
+using RingFull = Ring<4, A_TILE_BYTES>;
 using RingSmallM = Ring<5, 32 * BK_BYTES>;
-using RingFullMx = Ring<2, A_TILE_BYTES, FmtMxfp8, 2>;
+using RingFullMx = Ring<4, A_TILE_BYTES, FmtMxfp8>;
 using RingSmallMMx = Ring<5, 32 * BK_BYTES, FmtMxfp8>;
-static_assert(RingFull::STAGE_BYTES == 2 * (A_TILE_BYTES + kTileBytes + SFA_BYTES), "NVFP4 stages need no padding");
+static_assert(RingFull::STAGE_BYTES == A_TILE_BYTES + kTileBytes + SFA_BYTES, "NVFP4 stages need no padding");
 constexpr int NUM_EPI_WARPS = 16;
 constexpr int NUM_SF_WARPS = 4;                      // one per TMEM lane quarter
 constexpr int FIRST_SF_WARP = 2 + NUM_EPI_WARPS;
@@ -206,7 +201,7 @@ __device__ __forceinline__ TileRef tile_ref(int id, int total_gu, int n_gu, int 
 
 template <class R>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const ExpertGemmArgs args) {
-  constexpr int STAGES = R::STAGES, A_BYTES = R::A_BYTES, STAGE_BYTES = R::STAGE_BYTES, KPS = R::KPS;
+  constexpr int STAGES = R::STAGES, A_BYTES = R::A_BYTES, STAGE_BYTES = R::STAGE_BYTES;
   using F = typename R::Fmt;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -309,49 +304,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           atomicOr(args.err, kErrRange);
           a_bytes = A_BYTES;
         }
-        // Stage c of the tile holds K steps [c KPS, c KPS + nk): their weight tiles in one
-        // copy, their A scales in one copy, and their A tiles in one copy when whole
-        // 128-row tiles are copied (else one copy per K step).
-        const int n_chunks = (k_tiles + KPS - 1) / KPS;
-        auto chunk_steps = [&](int c) { return min(KPS, k_tiles - c * KPS); };
-        auto load_a = [&](int st, int c) {
+        // A and its scales of K step kk into stage st
+        auto load_a = [&](int st, int kk) {
           uint8_t* sa = smem + st * STAGE_BYTES;
-          const int kk = c * KPS, nk = chunk_steps(c);
-          if (KPS > 1 && A_BYTES == A_TILE_BYTES && a_bytes == static_cast<uint32_t>(A_TILE_BYTES)) {
-            bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, nk * A_TILE_BYTES, &tail->full[st]);
-          } else {
-            for (int j = 0; j < nk; ++j)
-              bulk_load(sa + j * A_BYTES, a_src + static_cast<size_t>(kk + j) * A_TILE_BYTES, a_bytes,
-                        &tail->full[st]);
-          }
-          bulk_load(sa + R::SFA_OFF, sfa + static_cast<size_t>(kk) * F::SFA, nk * F::SFA, &tail->full[st]);
+          bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, a_bytes, &tail->full[st]);
+          bulk_load(sa + A_BYTES + B_BYTES + F::SFB, sfa + static_cast<size_t>(kk) * F::SFA, F::SFA, &tail->full[st]);
         };
         // Before the wait only the weights are loaded; the first tile starts at stage 0, so
-        // its deferred chunks c < STAGES sit in stages c.
+        // its deferred K steps kk < STAGES sit in stages kk.
         int deferred = 0;
         auto resolve = [&]() {
           pdl_wait();
           pdl_trigger();
           waited = true;
-          for (int c = 0; c < deferred; ++c) load_a(c, c);
+          for (int kk = 0; kk < deferred; ++kk) load_a(kk, kk);
         };
         bool ok = true;
-        const int claim_at = max(0, n_chunks - STAGES);
-        for (int c = 0; c < n_chunks; ++c) {
-          if (c == claim_at) claim = atomicAdd(args.sched, 1u);
-          if (!waited && c == STAGES) resolve();
+        const int claim_at = max(0, k_tiles - STAGES);
+        for (int kt = 0; kt < k_tiles; ++kt) {
+          if (kt == claim_at) claim = atomicAdd(args.sched, 1u);
+          if (!waited && kt == STAGES) resolve();
           if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          const int nk = chunk_steps(c);
-          mbar_arrive_expect_tx(&tail->full[stage], static_cast<uint32_t>(nk) * (a_bytes + F::TILE + F::SFA));
+          mbar_arrive_expect_tx(&tail->full[stage], a_bytes + F::TILE + F::SFA);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          bulk_load(smem + stage * STAGE_BYTES + R::B_OFF, btile + static_cast<size_t>(c * KPS) * F::TILE,
-                    nk * F::TILE, &tail->full[stage]);
+          bulk_load(smem + stage * STAGE_BYTES + A_BYTES, btile + static_cast<size_t>(kt) * F::TILE, F::TILE,
+                    &tail->full[stage]);
           if (waited)
-            load_a(stage, c);
+            load_a(stage, kt);
           else
             ++deferred;
           if (++stage == STAGES) {
@@ -389,32 +372,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
         }
         if (id < 0) break;
         const int k_tiles = id >= total_gu ? args.d_k_tiles : args.gu_k_tiles;
-        const int n_chunks = (k_tiles + KPS - 1) / KPS;
         if (!mbar_wait_bounded(&tail->acc_empty, acc_phase ^ 1, abort_flag)) break;
         tc_fence_after();
         bool ok = true;
-        for (int c = 0; c < n_chunks; ++c) {
+        for (int kt = 0; kt < k_tiles; ++kt) {
           // the stage's operands have landed and its scale factors are in TMEM
           if (!mbar_wait_bounded(&tail->sf_full[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nk = min(KPS, k_tiles - c * KPS);
-          for (int j = 0; j < nk; ++j) {
-            const int kt = c * KPS + j;
-            const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES) + j * A_BYTES;
-            const uint32_t sb = smem_u32(smem + stage * STAGE_BYTES) + R::B_OFF + j * F::TILE;
-            const uint32_t sf = tmem + SF_COL + stage * R::SF_COLS + j * SF_STAGE_COLS;
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          const uint32_t sf = tmem + SF_COL + stage * SF_STAGE_COLS;
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-              if constexpr (F::kMx)  // the 4 MMAs share the step's scale columns, byte kb of each cell
-                tc_mma_mxf8(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), idesc_mxf8(kb),
-                            sf, sf + SFB_OFF, (kt | kb) != 0 ? 1u : 0u);
-              else
-                tc_mma_nvfp4(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), kIdescNvfp4,
-                             sf + kb * 4, sf + SFB_OFF + kb * 8, (kt | kb) != 0 ? 1u : 0u);
-            }
+          for (int kb = 0; kb < 4; ++kb) {
+            if constexpr (F::kMx)  // the 4 MMAs share the stage's scale columns, byte kb of each cell
+              tc_mma_mxf8(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), idesc_mxf8(kb),
+                          sf, sf + SFB_OFF, (kt | kb) != 0 ? 1u : 0u);
+            else
+              tc_mma_nvfp4(tmem + ACC_COL, sdesc_k_sw128(sa + kb * 32), sdesc_k_sw128(sb + kb * 32), kIdescNvfp4,
+                           sf + kb * 4, sf + SFB_OFF + kb * 8, (kt | kb) != 0 ? 1u : 0u);
           }
           tc_commit(&tail->empty[stage]);
           if (++stage == STAGES) {
@@ -454,49 +432,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
       }
       if (id < 0) break;
       const int k_tiles = id >= total_gu ? args.d_k_tiles : args.gu_k_tiles;
-      const int n_chunks = (k_tiles + KPS - 1) / KPS;
       bool ok = true;
-      for (int c = 0; c < n_chunks; ++c) {
+      for (int kt = 0; kt < k_tiles; ++kt) {
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tail->full[stage], phase, abort_flag))) {
           ok = false;
           break;
         }
-        const int nk = min(KPS, k_tiles - c * KPS);
-        for (int j = 0; j < nk; ++j) {
-          const uint8_t* ssfb = smem + stage * STAGE_BYTES + R::B_OFF + j * F::TILE + B_BYTES;  // [half][K-group][512]
-          const uint8_t* ssfa = smem + stage * STAGE_BYTES + R::SFA_OFF + j * F::SFA;           // [K-group][512]
-          const uint32_t col = SF_COL + stage * R::SF_COLS + j * SF_STAGE_COLS;
-          if constexpr (F::kMx) {
-            // one atom of A scales -> columns 0..3; B: rows 0-127 -> SFB_OFF + 0..3, rows 128-255 -> + 4..7
-            const uint4 a = *reinterpret_cast<const uint4*>(ssfa + lane * 16);
-            const uint32_t ra[4] = {a.x, a.y, a.z, a.w};
-            tmem_st_32x32b_x4(t_lane + col, ra);
-            const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + lane * 16);
-            const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 512 + lane * 16);
-            const uint32_t rb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            tmem_st_32x32b_x8(t_lane + col + SFB_OFF, rb);
-          } else {
-            uint32_t r[16];
-            // A: K-group kb -> columns 4 kb .. 4 kb + 3
+        const uint8_t* ssfb = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;  // [half][K-group][512]
+        const uint8_t* ssfa = ssfb + F::SFB;                                   // [K-group][512]
+        const uint32_t col = SF_COL + stage * SF_STAGE_COLS;
+        if constexpr (F::kMx) {
+          // one atom of A scales -> columns 0..3; B: rows 0-127 -> SFB_OFF + 0..3, rows 128-255 -> + 4..7
+          const uint4 a = *reinterpret_cast<const uint4*>(ssfa + lane * 16);
+          const uint32_t ra[4] = {a.x, a.y, a.z, a.w};
+          tmem_st_32x32b_x4(t_lane + col, ra);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(ssfb + lane * 16);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(ssfb + 512 + lane * 16);
+          const uint32_t rb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+          tmem_st_32x32b_x8(t_lane + col + SFB_OFF, rb);
+        } else {
+          uint32_t r[16];
+          // A: K-group kb -> columns 4 kb .. 4 kb + 3
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-              const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512 + lane * 16);
-              r[kb * 4 + 0] = v.x; r[kb * 4 + 1] = v.y; r[kb * 4 + 2] = v.z; r[kb * 4 + 3] = v.w;
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512 + lane * 16);
+            r[kb * 4 + 0] = v.x; r[kb * 4 + 1] = v.y; r[kb * 4 + 2] = v.z; r[kb * 4 + 3] = v.w;
+          }
+          tmem_st_32x32b_x16(t_lane + col, r);
+          // B: K-group kb -> columns 8 kb .. 8 kb + 3 (rows 0-127), 8 kb + 4 .. 8 kb + 7 (rows 128-255)
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int kb = part * 2 + q;
+              const uint4 v0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512 + lane * 16);
+              const uint4 v1 = *reinterpret_cast<const uint4*>(ssfb + SFA_BYTES + kb * 512 + lane * 16);
+              r[q * 8 + 0] = v0.x; r[q * 8 + 1] = v0.y; r[q * 8 + 2] = v0.z; r[q * 8 + 3] = v0.w;
+              r[q * 8 + 4] = v1.x; r[q * 8 + 5] = v1.y; r[q * 8 + 6] = v1.z; r[q * 8 + 7] = v1.w;
             }
-            tmem_st_32x32b_x16(t_lane + col, r);
-            // B: K-group kb -> columns 8 kb .. 8 kb + 3 (rows 0-127), 8 kb + 4 .. 8 kb + 7 (rows 128-255)
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const int kb = part * 2 + q;
-                const uint4 v0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512 + lane * 16);
-                const uint4 v1 = *reinterpret_cast<const uint4*>(ssfb + SFA_BYTES + kb * 512 + lane * 16);
-                r[q * 8 + 0] = v0.x; r[q * 8 + 1] = v0.y; r[q * 8 + 2] = v0.z; r[q * 8 + 3] = v0.w;
-                r[q * 8 + 4] = v1.x; r[q * 8 + 5] = v1.y; r[q * 8 + 6] = v1.z; r[q * 8 + 7] = v1.w;
-              }
-              tmem_st_32x32b_x16(t_lane + col + SFB_OFF + part * 16, r);
-            }
+            tmem_st_32x32b_x16(t_lane + col + SFB_OFF + part * 16, r);
           }
         }
         tmem_st_wait();

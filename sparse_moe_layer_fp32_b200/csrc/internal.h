@@ -55,12 +55,17 @@ cudaError_t launch_split_router(const float* w, int E, int H, uint16_t* out, cud
 // weights from launch_split_router.  Writes logits [T][E], ids / w [T][k].
 // Tokens per CTA (128 or 256) for a batch of T; also the row count of the x tensor map's box.
 int router_tc_tokens_per_cta(int T, int num_sms);
-// splits > 1 (128-token CTAs only): grid (token tiles) x (splits slices of H), partial
-// logits [splits][T][E] into `logits`, no top-k (launch_topk sums the slices and selects).
+// splits > 1: grid (token tiles) x (splits slices of H), partial logits [splits][T][E] into
+// `logits`, no top-k (launch_topk sums the slices and selects).
 cudaError_t launch_router_tc(const CUtensorMap& map_x, int tokens_per_cta, const uint16_t* w_tiles, int T, int H,
                              int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s,
                              int splits = 1);
 bool router_tc_split_supported(int H, int E, int k);
+// The sliced form for a batch of T: tokens per CTA (128 or 256) and slices of H.
+struct RouterTcPlan {
+  int tokens, splits;
+};
+RouterTcPlan router_tc_split_plan(int T, int H, int num_sms);
 int router_tc_split_count(int T, int H, int num_sms);
 
 // ---- routing of a small batch in one launch (route_small.cu)
@@ -162,9 +167,8 @@ cudaError_t launch_gemm_experts_mx(const ExpertGemmArgs& a, int grid, cudaStream
 constexpr int kMaxTpRanks = 16;
 constexpr size_t kTpHeaderBytes = 1024;
 constexpr int kTpRowSlot = 4 * kMaxTpRanks;
-// The two-shot all-reduce from this many tokens on (every rank's slice is then non-empty
-// for any world <= kMaxTpRanks, since T >= world^2).
-constexpr int kTpTwoShotMinTokens = 256;
+// The two-shot all-reduce from BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS tokens on by default (every
+// rank's slice is then non-empty for any world <= kMaxTpRanks, since T >= world^2).
 struct TpGroup {
   uint8_t* const* regions;  // device array: every rank's region as mapped in this process
   uint8_t* own;             // this rank's region (regions[rank])

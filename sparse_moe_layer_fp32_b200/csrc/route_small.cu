@@ -182,12 +182,14 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
   }
   __syncthreads();
   // ---------------------------------------------------------------- scan and work blocks
+  // One scan of three 10-bit fields (rows, blocks, blocks of held experts): every prefix of
+  // each field is at most T k <= 256 rows or E + T k / 128 <= 258 blocks, below 2^10.
   const int cnt = tid < E ? s_cnt[tid] : 0;
   const int nblk = (cnt + 127) / 128;
-  int total_rows, total_blk, total_work;
-  const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
-  const int blk = block_exclusive_scan(nblk, warp_sums, total_blk);
-  const int wbase = block_exclusive_scan(held ? nblk : 0, warp_sums, total_work);
+  int total_packed;
+  const int packed = block_exclusive_scan(cnt | (nblk << 10) | ((held ? nblk : 0) << 20), warp_sums, total_packed);
+  const int off = packed & 1023, blk = (packed >> 10) & 1023, wbase = packed >> 20;
+  const int total_rows = total_packed & 1023, total_blk = (total_packed >> 10) & 1023, total_work = total_packed >> 20;
   if (tid < E) {
     offsets[tid] = off;
     sf_block[tid] = blk;
@@ -210,17 +212,29 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     sf_block[E] = total_blk;
     *num_mblocks = total_work;
   }
+  if (tid < E) s_cnt[tid] = 0;  // from here: rows of each expert placed so far
   __syncthreads();
   // ---------------------------------------------------------------- permutation
-  // rank of (t, j) = number of earlier tokens that chose the same expert
-  for (int i = tid; i < R; i += kSmallThreads) {
-    const int t = i / k, ee = s_ids[i];
-    int rank = 0;
-    for (int q = 0; q < t * k; ++q) rank += s_ids[q] == ee;
-    const int r = s_off[ee] + rank;
-    perm[r] = t;
-    inv[i] = r;
-    tile_row[i] = (s_blk[ee] + (rank >> 7)) * 128 + (rank & 127);
+  // rank of slot i = t k + j = earlier slots (a token chooses an expert once: earlier tokens)
+  // with the same expert.  One warp walks the slots 32 at a time in order: lanes holding the
+  // same expert rank among themselves by lane, after the count of the chunks before.
+  if (warp == 0) {
+    for (int i0 = 0; i0 < R; i0 += 32) {
+      const int i = i0 + lane;
+      const int ee = i < R ? s_ids[i] : -1 - lane;  // past R: a key no other lane holds
+      const unsigned peers = __match_any_sync(0xffffffffu, ee);
+      const int before = __popc(peers & ((1u << lane) - 1u));
+      const int rank = (i < R ? s_cnt[ee] : 0) + before;
+      __syncwarp();
+      if (i < R && before == 0) s_cnt[ee] += __popc(peers);  // the lowest lane of each expert
+      __syncwarp();
+      if (i < R) {
+        const int r = s_off[ee] + rank;
+        perm[r] = i / k;
+        inv[i] = r;
+        tile_row[i] = (s_blk[ee] + (rank >> 7)) * 128 + (rank & 127);
+      }
+    }
   }
   if (tid == 0) *done_counter = 0u;
 }

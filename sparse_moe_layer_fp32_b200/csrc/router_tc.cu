@@ -296,14 +296,16 @@ bool router_tc_split_supported(int H, int E, int k) {
   return H % RT_BK == 0 && E % 16 == 0 && E >= 16 && E <= 256 && k <= 16 && router_tc_smem_bytes(E) <= 227 * 1024;
 }
 
-int router_tc_split_count(int T, int H, int num_sms) {
+RouterTcPlan router_tc_split_plan(int T, int H, int num_sms) {
   // (token tiles) x (slices of H), each slice at least 4 K steps: about one wave of CTAs
   // below kRouterTcMinTokens tokens, about two from there on
   const int tiles = (T + RT_MMA_M - 1) / RT_MMA_M;
   const int max_splits = std::max(1, H / RT_BK / 4);
   const int want = T < kRouterTcMinTokens ? num_sms / tiles : (2 * num_sms + tiles - 1) / tiles;
-  return std::max(1, std::min(want, max_splits));
+  return RouterTcPlan{RT_MMA_M, std::max(1, std::min(want, max_splits))};
 }
+
+int router_tc_split_count(int T, int H, int num_sms) { return router_tc_split_plan(T, H, num_sms).splits; }
 
 int router_tc_tokens_per_cta(int T, int num_sms) {
   // two halves per CTA once 128-token CTAs would need more than one wave
@@ -327,8 +329,8 @@ cudaError_t launch_router_tc(const CUtensorMap& map_x, int tokens_per_cta, const
                              int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s,
                              int splits) {
   if (splits < 1) return cudaErrorInvalidValue;
-  if (tokens_per_cta == 2 * RT_MMA_M && splits == 1)
-    return launch_router_tc_t<2>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, 1, s);
+  if (tokens_per_cta == 2 * RT_MMA_M)
+    return launch_router_tc_t<2>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, splits, s);
   if (tokens_per_cta == RT_MMA_M)
     return launch_router_tc_t<1>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, splits, s);
   return cudaErrorInvalidValue;

@@ -206,27 +206,20 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
   // Lanes 2c, 2c + 1 hold the two halves of one 16-byte code chunk and lanes 4g..4g + 3 the
   // four scale bytes of one K-group (nb is a multiple of 4): one 16-byte code store per lane
-  // pair and one 4-byte scale store per lane quad, per slot.  The next two iterations' 32
-  // bytes per lane are in flight during this one's quantisation (more bytes in flight per
-  // warp: the loads' latency, not their issue, bounds this kernel).
-  uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0, f0 = n0, f1 = n0;
+  // pair and one 4-byte scale store per lane quad, per slot.  The next iteration's 32 bytes
+  // are loaded before this one's quantisation (its divisions hide the load latency).
+  uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
   if (lane < nb) {
     n0 = __ldg(xr + 2 * lane);
     n1 = __ldg(xr + 2 * lane + 1);
-  }
-  if (lane + 32 < nb) {
-    f0 = __ldg(xr + 2 * (lane + 32));
-    f1 = __ldg(xr + 2 * (lane + 32) + 1);
   }
   for (int b0 = 0; b0 < nb; b0 += 32) {
     const int b = b0 + lane;
     const bool active = b < nb;  // whole quads are active or not
     const uint4 p0 = n0, p1 = n1;
-    n0 = f0;
-    n1 = f1;
-    if (b + 64 < nb) {
-      f0 = __ldg(xr + 2 * (b + 64));
-      f1 = __ldg(xr + 2 * (b + 64) + 1);
+    if (b + 32 < nb) {
+      n0 = __ldg(xr + 2 * (b + 32));
+      n1 = __ldg(xr + 2 * (b + 32) + 1);
     }
     uint32_t lo = 0, hi = 0, sc = 0;
     if (active) {

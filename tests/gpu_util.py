@@ -6,7 +6,7 @@ import torch
 
 import moe_inputs as mi
 import sparse_moe_layer_fp32_b200 as bm
-from oracle import moe, nvfp4
+from oracle import moe, mxfp8, nvfp4
 
 # Output tolerance of the layer against the oracle: relative L2 1e-2 and per-element
 # absolute 5e-2 (tokens whose 8th/9th logit gap is a near-tie are excluded and counted).
@@ -152,3 +152,73 @@ def oracle_layer_inputs(shape: mi.LayerShape, seed: int, weights_fp32=None, toke
     g = mi.bf16_bits_to_f32(mi.gamma(shape, seed)).astype(np.float64)
     getter = weights_fp32 or (lambda e: mi.expert_weights(shape, seed, e))
     return x, res, wr, g, moe.ExpertCache(getter, keep=16, fmt=fmt)
+
+
+# Relative width of the band around a rounding boundary inside which the GPU and the oracle
+# may decide an A2 code or scale differently: the GPU's h comes from FP32 tensor-core sums of
+# up to H exact products and an FP32 SiLU, the oracle's from FP64 (typically ~1e-6 apart).
+A2_BOUNDARY_DELTA = 1e-4
+
+
+def _boundary(encode, v, delta=A2_BOUNDARY_DELTA):
+    """True where v scaled by (1 - delta) and by (1 + delta) encode differently."""
+    v = np.asarray(v, np.float64)
+    return encode((v * (1 - delta)).astype(np.float32)) != encode((v * (1 + delta)).astype(np.float32))
+
+
+def a2_boundary_rows(gpu_codes, gpu_sf, h32, alpha2, fmt, delta=A2_BOUNDARY_DELTA):
+    """Rows whose GPU A2 differs from the oracle's quantisation of the oracle's own h.
+
+    gpu_codes / gpu_sf: the GPU's A2 of those rows (packed NVFP4 nibbles or E4M3 bytes, and
+    scale codes); h32: the oracle's FP32 h [R, I].  Every difference must be a decision at a
+    rounding boundary: a differing scale where the block's scale input moved by +-delta
+    (relative) encodes to two codes, a differing code (in a block whose scales agree) where
+    its quotient moved by +-delta does; both decisions are then valid at FP32 precision.
+    Any other difference fails.  Returns a bool mask [R] of the rows that differ."""
+    h = np.asarray(h32, np.float32)
+    R, I = h.shape
+    if fmt == "mxfp8":
+        oc, osf = mxfp8.quantize_mxfp8(h)
+        blocks = h.reshape(R, I // 32, 32).astype(np.float64)
+        amax = np.abs(blocks).max(axis=-1)
+        sb = (mxfp8.scale_exponent(amax * (1 - delta)) != mxfp8.scale_exponent(amax * (1 + delta)))
+        q = np.ldexp(blocks, -mxfp8.scale_exponent(amax)[..., None]).reshape(R, I)
+        cb = _boundary(mxfp8.e4m3_encode_signed, q, delta)
+        gc, oc2, blk = np.asarray(gpu_codes), oc, 32
+    else:
+        pc, osf = nvfp4.quantize_nvfp4(h, alpha2)
+        blocks = h.reshape(R, I // 16, 16)
+        six_alpha = np.float32(np.float32(6.0) * np.float32(alpha2))
+        s_in = (np.abs(blocks).max(axis=-1) / six_alpha).astype(np.float32)
+        sb = _boundary(nvfp4.e4m3_encode, s_in, delta)
+        d = (nvfp4.e4m3_decode(osf).astype(np.float32) * np.float32(alpha2)).astype(np.float32)
+        q = (blocks / np.where(d == 0, np.float32(1), d)[..., None]).astype(np.float32).reshape(R, I)
+        cb = _boundary(lambda v: nvfp4.e2m1_encode(np.abs(v)), q, delta)
+        # +-0 compare equal; a nonzero code's sign is the value's sign on both sides
+        gc, oc2, blk = nvfp4.unpack_nibbles(norm_zero(gpu_codes)), nvfp4.unpack_nibbles(norm_zero(pc)), 16
+    s_diff = np.asarray(gpu_sf) != osf
+    assert np.all(sb[s_diff]), "an A2 scale differs away from a rounding boundary"
+    c_diff = (gc != oc2) & ~np.repeat(s_diff, blk, axis=1)
+    assert np.all(cb[c_diff]), "an A2 code differs away from a rounding boundary"
+    return s_diff.any(axis=1) | c_diff.any(axis=1)
+
+
+def a2_boundary_tokens(layer, T, k, I, h32_tok, alpha2, fmt, skip=None):
+    """Tokens of the layer's last forward (T tokens) whose A2 rows differ from the oracle's at
+    rounding boundaries only (a2_boundary_rows; other differences fail).  h32_tok: the
+    oracle's h [T, k, I] in slot order; tokens in skip (routing near-ties) are not compared."""
+    mx = fmt == "mxfp8"
+    kv, vpb, blk = (128, 1, 32) if mx else (256, 2, 16)
+    Ip = (I + kv - 1) // kv * kv
+    offsets = buf(layer, bm.BUF_OFFSETS, np.int32)
+    sfb = buf(layer, bm.BUF_SFBLOCK, np.int32)
+    inv = buf(layer, bm.BUF_INV, np.int32).reshape(-1, k)[:T]
+    codes = tile_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, Ip, values_per_byte=vpb)[:, : I // vpb]
+    sf = sf_rows(buf(layer, bm.BUF_A2_SF, np.uint8), sfb, offsets, Ip, block=blk)[:, : I // blk]
+    keep = np.ones(T, bool) if skip is None else ~np.asarray(skip, bool)
+    tok = np.nonzero(keep)[0]
+    rows = inv[tok].reshape(-1)
+    diff = a2_boundary_rows(codes[rows], sf[rows], np.asarray(h32_tok)[tok].reshape(-1, I), alpha2, fmt)
+    out = np.zeros(T, bool)
+    out[tok] = diff.reshape(-1, k).any(axis=1)
+    return out

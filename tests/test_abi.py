@@ -18,6 +18,13 @@ def test_header_declares_the_binding_names(repo_root):
     assert _declared(repo_root) == sorted(pkg.EXPORTED)
 
 
+def test_header_constants_match_the_binding(repo_root):
+    import sparse_moe_layer_fp32_b200 as pkg
+    text = open(os.path.join(repo_root, "include", "beam_moe.h")).read()
+    m = re.search(r"#define BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS (\d+)", text)
+    assert m and int(m.group(1)) == pkg.TP_TWO_SHOT_MIN_TOKENS
+
+
 def test_library_exports_every_declared_symbol(repo_root):
     import sparse_moe_layer_fp32_b200 as pkg
     lib = ctypes.CDLL(pkg.LIB_PATH)
@@ -71,6 +78,7 @@ def test_host_side_validation_of_the_variant_and_parallel_entry_points():
     assert lib.beam_moe_quantize_mxfp8(None, 4, 64, None, None, None) == bad      # null buffers
     assert lib.beam_moe_expert_format(None) == -1
     assert lib.beam_moe_set_router_mode(None, pkg.ROUTER_AUTO) == bad
+    assert lib.beam_moe_set_tp_two_shot_tokens(None, 256) == bad
     assert lib.beam_moe_tp_region_bytes(None) == 0
     p = ctypes.c_void_p()
     assert lib.beam_moe_tp_region(None, ctypes.byref(p)) == bad

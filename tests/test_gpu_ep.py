@@ -24,7 +24,8 @@ pytestmark = pytest.mark.gpu
 
 import moe_inputs as mi  # noqa: E402
 from oracle import moe  # noqa: E402
-from tests.gpu_util import ABS_MAX, REL_L2, bf16_to_f64, compare_outputs, oracle_layer_inputs  # noqa: E402
+from tests.gpu_util import (ABS_MAX, REL_L2, a2_boundary_tokens, bf16_to_f64, compare_outputs,  # noqa: E402
+                            oracle_layer_inputs)
 
 SHAPES = {"tiny": mi.SHAPES["tiny"], "mid": mi.LayerShape("mid", 0, 512, 32, 4, 384)}
 
@@ -74,15 +75,26 @@ def test_ep_matches_oracle_and_single_gpu_bits(bm, name, fmt, world, tokens, see
                              [res[r * tokens:(r + 1) * tokens] for r in range(world)], wr, g, cache, shape.experts,
                              shape.top_k, a1 if fmt == "nvfp4" else None, a2 if fmt == "nvfp4" else None, world,
                              shape.rms_eps)
-    got = np.concatenate([bf16_to_f64(o) for o in outs])
-    rel, mx = compare_outputs(got, np.concatenate(ref["out_pre"]), skip=ref["near_tie"])
-    assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
-    # the same bits as one handle with every expert, run on each rank's own tokens
+    # the same bits as one handle with every expert, run on each rank's own tokens; its A2
+    # buffers show which tokens' A2 codes or scales sit on a rounding boundary, where the
+    # GPU's FP32 h and the oracle's FP64 h may decide differently (both valid): like routing
+    # near-ties, those tokens are counted and held to the relative-L2 bound only
     whole = bm.MoELayer(max_tokens=world * tokens, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
                         inter=shape.inter, alpha_a1=float(a1), alpha_a2=float(a2), fmt=fmt, **full)
+    edge = np.zeros(world * tokens, bool)
     for r in range(world):
         assert torch.equal(outs[r], whole.forward(xs[r], rs[r])), r
+        whole.check()
+        sl = slice(r * tokens, (r + 1) * tokens)
+        o = moe.moe_forward_tokens(x[sl], res[sl], wr, g, cache, shape.top_k, a1 if fmt == "nvfp4" else None,
+                                   a2 if fmt == "nvfp4" else None, shape.rms_eps)
+        edge[sl] = a2_boundary_tokens(whole, tokens, shape.top_k, shape.inter, o["h32"], a2, fmt, skip=o["near_tie"])
     whole.close()
+    got = np.concatenate([bf16_to_f64(o) for o in outs])
+    rel, _ = compare_outputs(got, np.concatenate(ref["out_pre"]), skip=ref["near_tie"])
+    _, mx = compare_outputs(got, np.concatenate(ref["out_pre"]), skip=ref["near_tie"] | edge)
+    assert rel <= REL_L2 and mx <= ABS_MAX, (rel, mx)
+    assert edge.sum() <= max(2, 0.01 * world * tokens), int(edge.sum())
     for _ in range(2):  # the regions are reused forward after forward
         again = grp.forward(xs, rs)
         for o, a in zip(outs, again):

@@ -67,8 +67,8 @@ def test_quantize_edge_blocks(bm):
 
 def test_quotients_near_every_e2m1_midpoint(bm):
     # v / d within a few ulp of each E2M1 rounding midpoint (and exactly on it where fl32
-    # allows), for many block scales d: the quotients whose rounding the quantiser must
-    # settle with an IEEE division rather than its reciprocal product.
+    # allows), for many block scales d: the quotients whose code depends on the last bit of
+    # the IEEE quotient.
     rng = np.random.default_rng(77)
     mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
     rows = []

@@ -9,8 +9,7 @@ waits are satisfied when they run.  Checks: all ranks produce identical bits; th
 matches the oracle's tensor-parallel layer (= the unsharded layer) at the layer's
 tolerances and a single handle holding all experts closely; from 256 tokens on the
 all-reduce is two-shot (each rank finishes its slice of the tokens, then gathers the
-others'), and its bits equal the one-shot form's (the same batch in halves below 256
-tokens: every token's result is independent of the rest of the batch); repeated forwards
+others'), and its bits equal the one-shot form's on the same batch; repeated forwards
 (the exchange buffers alternate by epoch) repeat the bits; a peer that never publishes
 makes the wait give up with a TIMEOUT status and the group recovers after a re-attach.
 """
@@ -71,13 +70,15 @@ def test_tp_matches_oracle_and_ranks_agree(bm, fmt, world, tokens, seed):
     torch.cuda.synchronize()
     for o in outs[1:]:
         assert torch.equal(o, outs[0])  # every rank holds the same output
-    if tokens >= 256:  # two-shot; the same tokens in two one-shot batches give the same bits
-        h = tokens // 2
-        halves = [grp.forward(xd[:h].contiguous(), rd[:h].contiguous()),
-                  grp.forward(xd[h:].contiguous(), rd[h:].contiguous())]
+    if tokens >= bm.TP_TWO_SHOT_MIN_TOKENS:  # two-shot; the one-shot form of the same batch: the same bits
+        for lay in grp.layers:
+            lay.set_tp_two_shot_tokens(2 ** 31 - 1)
+        one = grp.forward(xd, rd)
         for lay in grp.layers:
             lay.check()
-        assert torch.equal(torch.cat([halves[0][0], halves[1][0]]), outs[0])
+            lay.set_tp_two_shot_tokens(bm.TP_TWO_SHOT_MIN_TOKENS)
+        for o in one:
+            assert torch.equal(o, outs[0])
     ref = moe.moe_forward_tp(x, res, wr, g, cache, shape.top_k, a1 if fmt == "nvfp4" else None,
                              a2 if fmt == "nvfp4" else None, world, shape.rms_eps)
     got = bf16_to_f64(outs[0])
