@@ -359,7 +359,9 @@ DEFAULT_WORKLOADS = ("prefill16k", "decode8", "spec1024")
 def roofline_of(kern: dict, work: dict, fmt: str, T: int) -> dict:
     """Roofline of the dominant kernel: algorithmic bytes or FLOPs per launch over its live
     CUDA-event duration, against the measured (or fallback) peaks."""
-    top = max(kern, key=kern.get)
+    # the longest kernel whose algorithmic work is known (the expert GEMM in every workload;
+    # a profiler's serialised, cold launches can reorder the short ones)
+    top = max((n for n in kern if n in work), key=kern.get)
     pk = peaks()
     wk = work[top]
     # the contraction's own dtype: NVFP4 = 4 x BF16 (nominal 9 / 2.25 PF), FP8 = 2 x (4.5 / 2.25)

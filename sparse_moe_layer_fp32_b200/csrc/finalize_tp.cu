@@ -35,9 +35,8 @@
 
 namespace beam {
 
-// Both kernels: one CTA per token, one thread per 8-value chunk of the row (H / 8 threads,
-// rounded up to whole warps, at most kTpMaxThreads; wider rows loop), so the k (or W) row
-// loads of a chunk are all in flight at once: at decode sizes these kernels are latency-bound.
+// Both kernels: one CTA per token; a thread's k (or W) row loads of one 8-value chunk are all
+// in flight at once (tp_threads: how many threads share a row).
 constexpr int kTpMaxThreads = 1024;
 constexpr int kTpMaxK = 16;
 
@@ -245,7 +244,12 @@ __global__ void __launch_bounds__(256) tp_gather_kernel(int T, int S, int H, TpG
   }
 }
 
-static int tp_threads(int H) {
+// One thread per 8-value chunk for small batches (few CTAs: the latency of one token's
+// loads decides); 128 threads looping over the chunks once there are many tokens (many CTAs
+// per SM keep more loads in flight; the wide finalize measured 96% of HBM this way).
+constexpr int kTpWideTokens = 256, kTpWideThreads = 128;
+static int tp_threads(int H, int tokens) {
+  if (tokens >= kTpWideTokens) return kTpWideThreads;
   const int want = (H / 8 + 31) / 32 * 32;
   return want < kTpMaxThreads ? want : kTpMaxThreads;
 }
@@ -253,7 +257,7 @@ static int tp_threads(int H) {
 cudaError_t launch_tp_partial(const uint16_t* y, const float* w, const int32_t* inv, const int32_t* ids, int e_begin,
                               int e_end, int T, int H, int k, const TpGroup& g, uint32_t epoch, unsigned int* counter,
                               cudaStream_t s) {
-  return launch_pdl(tp_partial_kernel, dim3(T), dim3(tp_threads(H)), 0, s, y, w, inv, ids, e_begin, e_end, H, k, g,
+  return launch_pdl(tp_partial_kernel, dim3(T), dim3(tp_threads(H, T)), 0, s, y, w, inv, ids, e_begin, e_end, H, k, g,
                     epoch, counter);
 }
 
@@ -275,8 +279,8 @@ cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, in
     count = min(T, begin + S) - begin;
     if (count <= 0) return cudaErrorInvalidValue;
   }
-  return launch_pdl(tp_reduce_kernel, dim3(count), dim3(tp_threads(H)), smem, s, residual, gamma, begin, H, eps, g,
-                    epoch, out, err, two_shot ? 1 : 0, counter);
+  return launch_pdl(tp_reduce_kernel, dim3(count), dim3(tp_threads(H, count)), smem, s, residual, gamma, begin, H, eps,
+                    g, epoch, out, err, two_shot ? 1 : 0, counter);
 }
 
 cudaError_t launch_tp_gather(int T, int H, const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, int grid,
