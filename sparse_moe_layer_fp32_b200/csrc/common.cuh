@@ -409,7 +409,19 @@ __device__ __forceinline__ void st_act_pair(uint8_t* tiles, size_t block, int k_
   st_global_v8(p, s);
 }
 
-// Byte offset of scale s of row m (0..127) in a 128-row scale block with K/64 groups.
+// NVFP4 activation scales in K-step chunks: the 16 scales of one K step (256 values) of the
+// 128 rows of a block are one 2 KB chunk, row m's 16 bytes at m 16, so a K step's scales are
+// one contiguous copy for the GEMM and a row's 16 bytes are one contiguous store for the
+// writers.  (The 512-byte-atom order of the tensor cores scattered a row's scales in 4-byte
+// pieces 512 bytes apart, whose partial-sector writes held the A1 writer at ~3.4 TB/s where
+// 16-byte pieces reach ~4.5 TB/s; the scale warps gather the atom order from the chunk.)
+__device__ __forceinline__ size_t sf_chunk_offset(size_t block, int k_tiles, int m, int s) {
+  return ((block * static_cast<size_t>(k_tiles) + static_cast<size_t>(s >> 4)) * 128u + static_cast<size_t>(m)) * 16u +
+         static_cast<size_t>(s & 15);
+}
+
+// MXFP8 activation scales: byte offset of scale s of row m (0..127) in a 128-row scale block
+// with K/128 four-scale groups (the tcgen05 scale-factor atom order).
 __device__ __forceinline__ size_t sf_atom_offset(size_t block, int kgroups, int m, int s) {
   return (block * static_cast<size_t>(kgroups) + static_cast<size_t>(s >> 2)) * 512u +
          static_cast<size_t>((m & 31) * 16 + (m >> 5) * 4 + (s & 3));

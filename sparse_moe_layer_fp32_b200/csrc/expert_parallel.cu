@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kEpDispatchThreads) ep_dispatch_kernel(
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
   if constexpr (!kMx) {
     const float six_alpha = __fmul_rn(6.0f, alpha);
-    const int nb = H / 16, kgroups = H / 64;
+    const int nb = H / 16;
     // the loop bound is the same for the whole warp (blockDim is a multiple of 32): shuffles
     // below always see every lane
     for (int b0 = 0; b0 < nb; b0 += blockDim.x) {
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(kEpDispatchThreads) ep_dispatch_kernel(
         if (bj < 0) continue;
         *reinterpret_cast<uint4*>(s_a1[j] + act_tile_offset(bj, H / 256, b >> 4, m, (b & 15) >> 1)) =
             make_uint4(lo, hi, lo1, hi1);
-        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_sf[j] + sf_atom_offset(bj, kgroups, m, b)) = word;
+        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_sf[j] + sf_chunk_offset(bj, H / 256, m, b)) = word;
       }
     }
   } else {

@@ -26,7 +26,8 @@
 //   warp 0      producer: claims tiles, publishes each tile id through a small shared
 //               ring, and per 256-wide K step bulk-copies the A tile (the valid rows of a
 //               128-row activation tile, <= 16 KB), the expert's weight tile with its
-//               scales (32 KB + 4 KB) and the A scales (2 KB) into the stage ring, all
+//               scales (32 KB + 4 KB) and the A scales (2 KB: the K step's chunk of 128
+//               rows x 16 scale bytes; MXFP8: one 512-byte atom) into the stage ring, all
 //               landing on one mbarrier.  Activations and weights are both stored as
 //               contiguous tiles already in the swizzled shared-memory order, so every
 //               load is one sequential copy.
@@ -54,7 +55,7 @@ constexpr int BN = 256;
 constexpr int BK_BYTES = 128;  // 256 FP4 values per K step (one 128-byte swizzle row)
 constexpr int A_TILE_BYTES = BM * BK_BYTES;  // 16384: one activation tile in global memory
 constexpr int B_BYTES = BN * BK_BYTES;       // 32768
-constexpr int SFA_BYTES = 4 * 512;           // 4 K-groups of 64 values x 128 rows
+constexpr int SFA_BYTES = 128 * 16;          // 128 rows x 16 scales (the K step's 256 values)
 constexpr int SFB_BYTES = 2 * 4 * 512;       // 2 row blocks of 128
 static_assert(B_BYTES + SFB_BYTES == kTileBytes, "weight tile = B codes + B scales");
 // Two ring shapes.  Stage layout: A | B | SFB | SFA (B and SFB are one contiguous weight
@@ -68,7 +69,7 @@ static_assert(B_BYTES + SFB_BYTES == kTileBytes, "weight tile = B codes + B scal
 // (MXFP8: 4 MMAs of K = 32, 4 scales of 32 values per row).  Scale bytes per K step:
 struct FmtNvfp4 {
   static constexpr bool kMx = false;
-  static constexpr int SFA = SFA_BYTES;    // 4 atoms: one per 64-value K-group
+  static constexpr int SFA = SFA_BYTES;    // one K-step chunk: [128 rows][16 scales]
   static constexpr int SFB = SFB_BYTES;    // 2 row halves x 4 atoms
   static constexpr int TILE = kTileBytes;  // weight tile: B codes + B scales
 };
@@ -308,6 +309,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
         auto load_a = [&](int st, int kk) {
           uint8_t* sa = smem + st * STAGE_BYTES;
           bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, a_bytes, &tail->full[st]);
+          // one contiguous chunk per K step (NVFP4: 128 rows x 16 scales; MXFP8: one atom)
           bulk_load(sa + A_BYTES + B_BYTES + F::SFB, sfa + static_cast<size_t>(kk) * F::SFA, F::SFA, &tail->full[st]);
         };
         // Before the wait only the weights are loaded; the first tile starts at stage 0, so
@@ -412,10 +414,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
     }
   } else if (warp >= FIRST_SF_WARP) {
     // ------------------------------------------------------------ scale factors -> TMEM
-    // Each warp fills its own lane quarter of the stage's scale-factor columns from the
-    // 512-byte shared-memory atoms (row r of an atom holds the 4 scales of rows r, r + 32,
-    // r + 64, r + 96 of one 64-wide K-group), every quarter getting the same 4 columns per
-    // K-group, so the MMA finds the scales of row m at lane m, column + m / 32.  Doing it
+    // Each warp fills its own lane quarter of the stage's scale-factor columns: per K-group,
+    // lane l writes the 4 scales of rows l, l + 32, l + 64, l + 96 into 4 columns (B: from
+    // the weight tile's 512-byte atoms, which hold them in that order; NVFP4 A: gathered
+    // from the stage's [128 rows][16 scales]), every quarter getting the same columns, so
+    // the MMA finds the scales of row m at lane m, column + m / 32.  Doing it
     // with tcgen05.st keeps these copies off the tensor pipe, which then only runs MMAs.
     const int quarter = warp & 3;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -439,7 +442,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           break;
         }
         const uint8_t* ssfb = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;  // [half][K-group][512]
-        const uint8_t* ssfa = ssfb + F::SFB;                                   // [K-group][512]
+        const uint8_t* ssfa = ssfb + F::SFB;  // NVFP4 [128 rows][16 scales]; MXFP8 one 512-byte atom
         const uint32_t col = SF_COL + stage * SF_STAGE_COLS;
         if constexpr (F::kMx) {
           // one atom of A scales -> columns 0..3; B: rows 0-127 -> SFB_OFF + 0..3, rows 128-255 -> + 4..7
@@ -452,11 +455,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           tmem_st_32x32b_x8(t_lane + col + SFB_OFF, rb);
         } else {
           uint32_t r[16];
-          // A: K-group kb -> columns 4 kb .. 4 kb + 3
-#pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint4 v = *reinterpret_cast<const uint4*>(ssfa + kb * 512 + lane * 16);
-            r[kb * 4 + 0] = v.x; r[kb * 4 + 1] = v.y; r[kb * 4 + 2] = v.z; r[kb * 4 + 3] = v.w;
+          // A: the stage holds [128 rows][16 scales]; K-group kb -> columns 4 kb .. 4 kb + 3,
+          // column 4 kb + q of lane l = the 4 scales of row l + 32 q in that K-group
+          {
+            const uint4 q0 = *reinterpret_cast<const uint4*>(ssfa + lane * 16);
+            const uint4 q1 = *reinterpret_cast<const uint4*>(ssfa + (lane + 32) * 16);
+            const uint4 q2 = *reinterpret_cast<const uint4*>(ssfa + (lane + 64) * 16);
+            const uint4 q3 = *reinterpret_cast<const uint4*>(ssfa + (lane + 96) * 16);
+            r[0] = q0.x; r[1] = q1.x; r[2] = q2.x; r[3] = q3.x;
+            r[4] = q0.y; r[5] = q1.y; r[6] = q2.y; r[7] = q3.y;
+            r[8] = q0.z; r[9] = q1.z; r[10] = q2.z; r[11] = q3.z;
+            r[12] = q0.w; r[13] = q1.w; r[14] = q2.w; r[15] = q3.w;
           }
           tmem_st_32x32b_x16(t_lane + col, r);
           // B: K-group kb -> columns 8 kb .. 8 kb + 3 (rows 0-127), 8 kb + 4 .. 8 kb + 7 (rows 128-255)
@@ -560,9 +569,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           *reinterpret_cast<uint4*>(args.a2 + act_tile_offset(mb.sf_block, args.d_k_tiles, f0 >> 8, row_in_tile,
                                                               (f0 & 255) >> 5)) =
               make_uint4(codes[0], codes[1], codes[2], codes[3]);
-          // its 2 scales are 2 contiguous bytes of the K-group's 4 (f0 / 16 is even)
-          *reinterpret_cast<uint16_t*>(args.a2_sf + sf_atom_offset(mb.sf_block, args.d_k_tiles * 4, row_in_tile,
-                                                                   f0 / 16)) = static_cast<uint16_t>(scodes);
+          // its 2 scales are 2 contiguous bytes of the row's 16 in its K step (f0 / 16 is even)
+          *reinterpret_cast<uint16_t*>(args.a2_sf + sf_chunk_offset(mb.sf_block, args.d_k_tiles, row_in_tile,
+                                                                    f0 / 16)) = static_cast<uint16_t>(scodes);
         }
         // publish this warp's share of block t.block's A2 to the down-tile producers
         fence_proxy_async_global();

@@ -120,8 +120,8 @@ cudaError_t launch_quant_a1_mx(const uint16_t* x, const int32_t* tile_row, int T
                                uint8_t* a1_sf, cudaStream_t s);
 
 // ---- grouped NVFP4 GEMMs, gate/up and down in one launch (gemm_experts.cu)
-// Activation tiles are [blk][K/256][16384] (act_tile_offset), their scales [blk][K/64][512]
-// (sf_atom_offset); weight tiles are [E][n_tiles][K/256][kTileBytes].
+// Activation tiles are [blk][K/256][16384] (act_tile_offset), their scales [blk][K/256][128
+// rows][16] (sf_chunk_offset); weight tiles are [E][n_tiles][K/256][kTileBytes].
 struct ExpertGemmArgs {
   const MBlock* mblocks;
   const int32_t* num_mblocks;

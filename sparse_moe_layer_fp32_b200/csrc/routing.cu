@@ -12,7 +12,7 @@
 // A1 = Q(x, alpha_a1): x rows are quantised once per token (16-value blocks along H) and
 // the codes are written to the token's k permuted rows (the NVFP4 W4A4 experts of the
 // recipe "reflection/Beam-1.0-501B-A23B", section "Variants"), as activation tiles (see
-// act_tile_offset) of the row's 128-row block.  For the block-scaled FP8 variant of the
+// act_tile_offset) of the row's 128-row block, the scales in K-step chunks (sf_chunk_offset).  For the block-scaled FP8 variant of the
 // experts (the recipe's FP8 checkpoint, read as MXFP8), A1 = MX(x) in 32-value blocks.
 #include "common.cuh"
 #include "internal.h"
@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restric
                                                        const int32_t* __restrict__ tile_row, int T, int H, int k,
                                                        float alpha, uint8_t* __restrict__ a1,
                                                        uint8_t* __restrict__ a1_sf) {
-  const int nb = H / 16, kgroups = H / 64;
+  const int nb = H / 16;
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
   const bool active = gid < static_cast<int64_t>(T) * nb;
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restric
     // block b of 16 values: 8 bytes, half of 16-byte chunk (b % 16) / 2 of K tile b / 16
     *reinterpret_cast<uint2*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1) + (b & 1) * 8) =
         make_uint2(lo, hi);
-    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, kgroups, m, b)) = word;
+    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_chunk_offset(blk, H / 256, m, b)) = word;
   }
 }
 
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
   }
   __syncwarp();
   const float six_alpha = __fmul_rn(6.0f, alpha);
-  const int nb = H / 16, kgroups = H / 64;
+  const int nb = H / 16;
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H);
   // Lanes 2c, 2c + 1 hold the two halves of one 16-byte code chunk and lanes 4g..4g + 3 the
   // four scale bytes of one K-group (nb is a multiple of 4): one 16-byte code store per lane
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
       const int blk = s_blk[warp][j], m = s_m[warp][j];
       *reinterpret_cast<uint4*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1)) =
           make_uint4(lo, hi, lo1, hi1);
-      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, kgroups, m, b)) = word;
+      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_chunk_offset(blk, H / 256, m, b)) = word;
     }
   }
 }

@@ -27,8 +27,9 @@ def buf(layer, which, dtype):
 
 
 def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int, block: int = 16) -> np.ndarray:
-    """Scale blocks (beam_moe.h layout) -> row-major scales [rows, kcols/block] in permuted row
-    order; block = 16 (NVFP4) or 32 (MXFP8): 4 scales per 32-bit word either way."""
+    """Activation scales (beam_moe.h layouts) -> row-major scales [rows, kcols/block] in
+    permuted row order: block = 16 (NVFP4, stored in K-step chunks of 128 rows x 16 scales) or
+    32 (MXFP8, stored in 512-byte atoms of 4 scales per row)."""
     experts = len(offsets) - 1
     rows = int(offsets[-1])
     n_sc = kcols // block
@@ -42,8 +43,11 @@ def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols
         i = np.arange(n)
         blk = sf_block[e] + i // 128
         m = i % 128
-        off = ((blk[:, None] * kgroups + s[None, :] // 4) * 512 + (m[:, None] % 32) * 16 + (m[:, None] // 32) * 4
-               + s[None, :] % 4)
+        if block == 16:
+            off = ((blk[:, None] * (n_sc // 16) + s[None, :] // 16) * 128 + m[:, None]) * 16 + s[None, :] % 16
+        else:
+            off = ((blk[:, None] * kgroups + s[None, :] // 4) * 512 + (m[:, None] % 32) * 16 + (m[:, None] // 32) * 4
+                   + s[None, :] % 4)
         out[offsets[e]:offsets[e + 1]] = sf_buf[off]
     return out
 

@@ -131,3 +131,41 @@ def test_ep_attach_refuses_unequal_expert_ranges(bm):
     assert ei.value.status == bm.ERR_INVALID_ARG
     for lay in layers:
         lay.close()
+
+
+def test_ep_wait_gives_up_without_peer_and_group_recovers(bm):
+    # Failure detection without a GPU fault: rank 1 never publishes its expert counts, so
+    # rank 0's layout wait runs out (2 s): the error word says TIMEOUT, the layout leaves an
+    # empty block list and the context stays usable; after a re-attach the group computes
+    # the same bits as one handle with every expert.
+    from sparse_moe_layer_fp32_b200 import synthetic, tp
+    shape = dataclasses.replace(SHAPES["tiny"], tokens=2 * 4)
+    full = synthetic.make_weights(shape, 5, threads=2)
+    a1, a2 = 0.002, 0.0005
+    layers = _ep_layers(bm, shape, full, 2, 8, a1, a2, "nvfp4")
+    grp = tp.SharedGpuGroup(layers)
+    xd, rd = synthetic.make_batch(shape, 5)
+    xs = [xd[:4].contiguous(), xd[4:].contiguous()]
+    rs = [rd[:4].contiguous(), rd[4:].contiguous()]
+    out = torch.empty_like(rs[0])
+    layers[0].forward_ep_phase(xs[0], rs[0], out, 0)
+    layers[0].forward_ep_phase(xs[0], rs[0], out, 1)  # waits for rank 1's counts, which nothing sets
+    with pytest.raises(bm.BeamMoeError) as ei:
+        layers[0].check()
+    assert ei.value.status == bm.ERR_TIMEOUT
+    # phases run in order; rank 1 cannot start at phase 1
+    with pytest.raises(bm.BeamMoeError) as ei:
+        layers[1].forward_ep_phase(xs[1], rs[1], out, 1)
+    assert ei.value.status == bm.ERR_INVALID_ARG
+    regions = [lay.tp_region() for lay in layers]
+    for r, lay in enumerate(layers):
+        lay.tp_attach(r, 2, regions)
+    outs = grp.forward(xs, rs)
+    for lay in layers:
+        lay.check()
+    whole = bm.MoELayer(max_tokens=8, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                        inter=shape.inter, alpha_a1=a1, alpha_a2=a2, **full)
+    for r in range(2):
+        assert torch.equal(outs[r], whole.forward(xs[r], rs[r])), r
+    whole.close()
+    grp.close()
