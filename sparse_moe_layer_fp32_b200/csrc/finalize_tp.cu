@@ -279,8 +279,10 @@ cudaError_t launch_tp_reduce(const uint16_t* residual, const uint16_t* gamma, in
     count = min(T, begin + S) - begin;
     if (count <= 0) return cudaErrorInvalidValue;
   }
-  return launch_pdl(tp_reduce_kernel, dim3(count), dim3(tp_threads(H, count)), smem, s, residual, gamma, begin, H, eps,
-                    g, epoch, out, err, two_shot ? 1 : 0, counter);
+  // threads from the batch, not the slice: both forms then sum each row's squares in the
+  // same order and give the same bits
+  return launch_pdl(tp_reduce_kernel, dim3(count), dim3(tp_threads(H, T)), smem, s, residual, gamma, begin, H, eps, g,
+                    epoch, out, err, two_shot ? 1 : 0, counter);
 }
 
 cudaError_t launch_tp_gather(int T, int H, const TpGroup& g, uint32_t epoch, uint16_t* out, uint32_t* err, int grid,
