@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     float acc[MAXT];
 #pragma unroll
     for (int t = 0; t < MAXT; ++t) acc[t] = 0.0f;
+#pragma unroll 2
     for (int i = 0; i < nf4; ++i) {
       const float4 wq = wr[lane + 32 * i];
 #pragma unroll
@@ -126,13 +127,13 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     }
   }
   // ---------------------------------------------------------------- elect the last CTA
+  // The barrier orders every thread's partial stores before thread 0's arrival, a release
+  // at GPU scope (cumulative over them); the last arrival also acquires every earlier one's.
   __shared__ int s_last;
-  __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(done_counter, 1u) == gridDim.x - 1;
+  if (tid == 0) s_last = atom_add_acq_rel_gpu(done_counter, 1u) == gridDim.x - 1;
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
 
   // ---------------------------------------------------------------- phase 2: top-k
   // All partial logits in one bulk copy (the other CTAs' stores were released before
@@ -169,7 +170,11 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     for (int i = 0; i < 8; ++i) {
       const int ee = lane + 32 * i;
       float sum = 0.0f;
-      for (int q = 0; q < S; ++q) sum += ee < E ? ps[q * TE + t * E + ee] : 0.0f;  // slice order
+      // at most 4 slices (route_small_slices): unrolled, so the lane's 32 loads are in flight
+      // together; the sum still runs over the slices in order
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q < S) sum += ee < E ? ps[q * TE + t * E + ee] : 0.0f;
       v[i] = ee < E ? sum : -INFINITY;
     }
     warp_topk<8>(v, E, k, lane, s_ids + t * k, wout + static_cast<size_t>(t) * k);
