@@ -319,23 +319,23 @@ typedef enum {
   BEAM_MOE_BUF_PERM = 4,     /* [T*k] int32: token of permuted row r                        */
   BEAM_MOE_BUF_INV = 5,      /* [T][k] int32: permuted row of (token, slot)                */
   BEAM_MOE_BUF_SFBLOCK = 6,  /* [E+1] int32: first 128-row scale block of each expert      */
-  BEAM_MOE_BUF_A1 = 7,       /* activation tiles (below) of the permuted expert inputs, K = H */
-  BEAM_MOE_BUF_A1_SF = 8,    /* scales: [nblk][H/256][128][16] (MXFP8: atoms), see below   */
-  BEAM_MOE_BUF_A2 = 9,       /* activation tiles of the SwiGLU outputs, K = Ip = ceil(I/256)*256 */
-  BEAM_MOE_BUF_A2_SF = 10,   /* [nblk][Ip/256][128][16] (MXFP8: atoms)                      */
-  BEAM_MOE_BUF_Y = 11        /* [T*k][H] BF16 expert outputs in permuted row order          */
+  BEAM_MOE_BUF_A1 = 7,       /* activation units (below) of the permuted expert inputs, K = H */
+  BEAM_MOE_BUF_A2 = 8,       /* activation units of the SwiGLU outputs, K = Ip = ceil(I/256)*256 */
+  BEAM_MOE_BUF_Y = 9         /* [T*k][H] BF16 expert outputs in permuted row order          */
 } beam_moe_buffer;
 /* Blocks: the rows of expert e, local row i = r - off[e], live in block
  * blk = sfblock[e] + i/128, row m = i%128.
- * Scales (NVFP4): scale s of that row (values 16s .. 16s+15) is the byte at
- * ((blk * (K/256) + s/16) * 128 + m) * 16 + s%16: one chunk of 128 rows x 16 scales per
- * K step of 256 values, each row's 16 scales of a K step contiguous.
- * Activation tiles: codes byte j of that row (values 2j, 2j+1) is at
- * ((blk * (K/256) + j/128) * 16384) + m*128 + ((((j%128)/16) ^ (m%8)) * 16) + j%16.
- * MXFP8 handles: one value per code byte, one scale per 32 values and K tiles of 128
- * values: scale s at ((blk * (K/128) + s/4) * 512) + (m%32)*16 + (m/32)*4 + s%4 (512-byte
- * atoms, the tensor-core scale-factor order), code j (value j) at ((blk * (K/128) + j/128)
- * * 16384) + m*128 + ((((j%128)/16) ^ (m%8)) * 16) + j%16, and A2's K is I (no padding). */
+ * Activation units: one per block and K step of 256 values, U = 18432 bytes, the step's
+ * 16384 code bytes (128 rows x 128) followed by its 2048 scale bytes (128 rows x 16), so
+ * the expert GEMM loads a K step of codes and scales with one copy.  In unit
+ * u = blk * (K/256) + j/128, code byte j of that row (values 2j, 2j+1) is at
+ * u*U + m*128 + ((((j%128)/16) ^ (m%8)) * 16) + j%16, and scale s (values 16s .. 16s+15),
+ * in unit blk * (K/256) + s/16, at u*U + 16384 + m*16 + s%16.
+ * MXFP8 handles: one value per code byte, one scale per 32 values, K steps of 128 values
+ * and U = 16896 (16384 code bytes, then a 512-byte scale atom in the tensor cores'
+ * scale-factor order): code j (value j) in unit u = blk * (K/128) + j/128 at
+ * u*U + m*128 + ((((j%128)/16) ^ (m%8)) * 16) + j%16, scale s in unit blk * (K/128) + s/4
+ * at u*U + 16384 + (m%32)*16 + (m/32)*4 + s%4, and A2's K is I (no padding). */
 
 /* Copies min(bytes, size of the buffer) bytes of internal buffer `which` to dst (device),
  * enqueued on `stream`.  *size_out (host, may be NULL) receives the buffer's size for the

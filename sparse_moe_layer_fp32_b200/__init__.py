@@ -17,8 +17,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbeam_moe.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_OOM, ERR_TIMEOUT, ERR_DEVICE = range(7)
-(BUF_LOGITS, BUF_IDS, BUF_WEIGHTS, BUF_OFFSETS, BUF_PERM, BUF_INV, BUF_SFBLOCK, BUF_A1, BUF_A1_SF, BUF_A2,
- BUF_A2_SF, BUF_Y) = range(12)
+(BUF_LOGITS, BUF_IDS, BUF_WEIGHTS, BUF_OFFSETS, BUF_PERM, BUF_INV, BUF_SFBLOCK, BUF_A1, BUF_A2,
+ BUF_Y) = range(10)
 
 EXPORTED = [
     "beam_moe_create", "beam_moe_forward", "beam_moe_forward_host", "beam_moe_route",

@@ -31,7 +31,7 @@ struct beam_moe_ctx {
   int32_t* tile_row;  // [T][k]: 128 x activation block + row in it (where slot (t, j) goes in A1)
   float* w;
   MBlock* mblocks;
-  uint8_t *a1, *a1_sf, *a2, *a2_sf;
+  uint8_t *a1, *a2;  // activation units: per 128-row block and K step, codes then scales
   uint16_t* y;
   uint32_t* err;
   unsigned int* route_counter;  // last-CTA election of the fused small-batch routing kernel
@@ -39,7 +39,8 @@ struct beam_moe_ctx {
   int32_t router_mode;          // BEAM_MOE_ROUTER_*: which router batches of more than 16 tokens use
   int32_t fmt;                  // BEAM_MOE_FMT_*: expert weight and activation format
   int kv;                       // K values per activation / weight tile: 256 (NVFP4), 128 (MXFP8)
-  int sfa_tile;                 // scale bytes per 128-row block per K tile: 2048 (NVFP4), 512
+  int act_unit;                 // bytes per 128-row block per K step: 16384 codes + 2048 scales
+                                // (NVFP4) or + 512 (MXFP8)
   uint16_t *stage_x, *stage_res, *stage_out;
   // beam_moe_forward_host: the residual's upload runs on a second stream while the forward
   // computes; the finalize waits for it (created on the first host-buffer forward)
@@ -160,12 +161,9 @@ __global__ void wait_timeout_probe_kernel(uint64_t limit_ns, uint32_t* err) {
 // Kernels use 16-byte vector accesses on these pointers.
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// Activation tiles and their scale blocks for a contraction of K values (multiple of kv).
+// Activation units (codes and scales) for a contraction of K values (multiple of kv).
 size_t act_bytes(const beam_moe_ctx* h, int K) {
-  return static_cast<size_t>(h->nblk_max) * (K / h->kv) * 16384u;
-}
-size_t act_sf_bytes(const beam_moe_ctx* h, int K) {
-  return static_cast<size_t>(h->nblk_max) * (K / h->kv) * static_cast<size_t>(h->sfa_tile);
+  return static_cast<size_t>(h->nblk_max) * (K / h->kv) * static_cast<size_t>(h->act_unit);
 }
 
 }  // namespace
@@ -232,7 +230,7 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   h->e_begin = e_begin;
   h->e_count = e_count;
   h->kv = mx ? 128 : 256;
-  h->sfa_tile = mx ? 512 : 4 * 512;
+  h->act_unit = mx ? kActUnitMx : kActUnitNvfp4;
   h->H = cfg->hidden;
   h->E = cfg->num_experts;
   h->k = cfg->top_k;
@@ -327,9 +325,7 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   CREATE_TRY(dalloc(h, &h->inv, sizeof(int32_t) * R));
   CREATE_TRY(dalloc(h, &h->tile_row, sizeof(int32_t) * R));
   CREATE_TRY(dalloc(h, &h->a1, act_bytes(h, H)));
-  CREATE_TRY(dalloc(h, &h->a1_sf, act_sf_bytes(h, H)));
   CREATE_TRY(dalloc(h, &h->a2, act_bytes(h, Ip)));
-  CREATE_TRY(dalloc(h, &h->a2_sf, act_sf_bytes(h, Ip)));
   CREATE_TRY(dalloc(h, &h->y, sizeof(uint16_t) * static_cast<size_t>(R) * H));
   CREATE_TRY(dalloc(h, &h->err, sizeof(uint32_t)));
   CREATE_TRY(dalloc(h, &h->route_counter, sizeof(unsigned int)));
@@ -339,11 +335,10 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   CREATE_TRY(dalloc(h, &h->stage_res, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   CREATE_TRY(dalloc(h, &h->stage_out, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   // The SwiGLU outputs beyond I (NVFP4 when I is not a multiple of 256) are never written:
-  // their codes and scales must read as zero in the down GEMM.  Scale blocks of unused rows
-  // are also defined this way.
+  // their codes and scales must read as zero in the down GEMM.  The rows of a block past its
+  // valid rows are also defined this way (they feed only accumulator rows never stored).
   CREATE_TRY(cudaMemsetAsync(h->a2, 0, act_bytes(h, Ip), s));
-  CREATE_TRY(cudaMemsetAsync(h->a2_sf, 0, act_sf_bytes(h, Ip), s));
-  CREATE_TRY(cudaMemsetAsync(h->a1_sf, 0, act_sf_bytes(h, H), s));
+  CREATE_TRY(cudaMemsetAsync(h->a1, 0, act_bytes(h, H), s));
   CREATE_TRY(cudaMemsetAsync(h->err, 0, sizeof(uint32_t), s));
   if (ep) {
     if (E > 1024 || R >= (1ll << 24)) return fail(cudaErrorInvalidValue);  // the layout's limits
@@ -369,7 +364,6 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
     lay.arrivals = take(sizeof(uint32_t) * lay.nblk, 256);
     lay.origin = take(sizeof(int32_t) * R, 256);
     lay.a1 = take(act_bytes(h, H), 1024);
-    lay.a1_sf = take(act_sf_bytes(h, H), 1024);
     lay.ret = take(sizeof(uint16_t) * static_cast<size_t>(R) * H, 1024);
     lay.bytes = (off + 255) / 256 * 256;
   }
@@ -506,7 +500,7 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
                             h->e_begin + h->e_count};
   const bool mx = h->fmt == BEAM_MOE_FMT_MXFP8;
   // The expert GEMMs' arguments over a block list (this forward's, or the received rows')
-  auto gemm_args = [&](const uint8_t* a1, const uint8_t* a1_sf, int max_rows, const uint32_t* arrivals) {
+  auto gemm_args = [&](const uint8_t* a1, int max_rows, const uint32_t* arrivals) {
     ExpertGemmArgs g{};
     g.mblocks = h->mblocks;
     g.num_mblocks = h->num_mblocks;
@@ -514,10 +508,8 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     g.gu_n_tiles = h->I / 128;
     g.gu_k_tiles = H / h->kv;
     g.a1 = a1;
-    g.a1_sf = a1_sf;
     g.w_gu = h->w_gu_tiles;
     g.a2 = h->a2;
-    g.a2_sf = h->a2_sf;
     g.alpha_a2 = h->cfg.alpha_a2;
     g.d_n_tiles = H / 256;
     g.d_k_tiles = h->Ip / h->kv;
@@ -545,7 +537,7 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
       return finish();
     }
     if (ep_phase == 2) {
-      const ExpertGemmArgs g = gemm_args(region + h->ep_lay.a1, region + h->ep_lay.a1_sf, T * h->tp.world,
+      const ExpertGemmArgs g = gemm_args(region + h->ep_lay.a1, T * h->tp.world,
                                          reinterpret_cast<const uint32_t*>(region + h->ep_lay.arrivals));
       if (mx)
         BEAM_TRY(launch_gemm_experts_mx(g, h->num_sms, s));
@@ -637,14 +629,14 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     return finish();
   }
   if (mx)
-    BEAM_TRY(launch_quant_a1_mx(xb, h->tile_row, T, H, k, h->a1, h->a1_sf, s));
+    BEAM_TRY(launch_quant_a1_mx(xb, h->tile_row, T, H, k, h->a1, s));
   else
-    BEAM_TRY(launch_quant_a1(xb, h->tile_row, T, H, k, h->cfg.alpha_a1, h->a1, h->a1_sf, s));
+    BEAM_TRY(launch_quant_a1(xb, h->tile_row, T, H, k, h->cfg.alpha_a1, h->a1, s));
   BEAM_TRY(mark("quant_a1"));
   ++launches;
 
   // a token chooses an expert at most once: at most T rows per expert
-  const ExpertGemmArgs g = gemm_args(h->a1, h->a1_sf, T, nullptr);
+  const ExpertGemmArgs g = gemm_args(h->a1, T, nullptr);
   if (mx)
     BEAM_TRY(launch_gemm_experts_mx(g, h->num_sms, s));
   else
@@ -715,8 +707,8 @@ beam_moe_status beam_moe_tp_region(beam_moe_t h, void** region) {
     BEAM_TRY(dalloc(h, &ep_counter, sizeof(unsigned int)));
     BEAM_TRY(cudaMemset(ep_counter, 0, sizeof(unsigned int)));
     BEAM_TRY(cudaMemset(region, 0, kTpHeaderBytes));
-    if (h->ep) {  // the scales of received blocks' unused rows read as zero
-      BEAM_TRY(cudaMemset(region + h->ep_lay.a1_sf, 0, act_sf_bytes(h, h->H)));
+    if (h->ep) {  // received blocks' unused rows read as zero
+      BEAM_TRY(cudaMemset(region + h->ep_lay.a1, 0, act_bytes(h, h->H)));
       BEAM_TRY(cudaMemset(region + h->ep_lay.arrivals, 0, sizeof(uint32_t) * h->ep_lay.nblk));
       BEAM_TRY(cudaMemset(region + h->ep_lay.origin, 0xFF, sizeof(int32_t) * h->ep_lay.rows));  // no source yet
     }
@@ -905,9 +897,7 @@ beam_moe_status beam_moe_debug_copy(beam_moe_t h, int32_t which, void* dst, size
     case BEAM_MOE_BUF_INV: src = h->inv; n = sizeof(int32_t) * R; break;
     case BEAM_MOE_BUF_SFBLOCK: src = h->sf_block; n = sizeof(int32_t) * (h->E + 1); break;
     case BEAM_MOE_BUF_A1: src = h->a1; n = act_bytes(h, h->H); break;
-    case BEAM_MOE_BUF_A1_SF: src = h->a1_sf; n = act_sf_bytes(h, h->H); break;
     case BEAM_MOE_BUF_A2: src = h->a2; n = act_bytes(h, h->Ip); break;
-    case BEAM_MOE_BUF_A2_SF: src = h->a2_sf; n = act_sf_bytes(h, h->Ip); break;
     case BEAM_MOE_BUF_Y: src = h->y; n = sizeof(uint16_t) * static_cast<size_t>(R) * h->H; break;
     default: return BEAM_MOE_ERR_INVALID_ARG;
   }

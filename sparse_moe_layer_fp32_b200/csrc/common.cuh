@@ -378,12 +378,19 @@ __device__ __forceinline__ uint32_t quant_block32_mx(const float (&v)[32], uint3
   return static_cast<uint32_t>(e + 127);
 }
 
-// Activation tiles: the codes of each 128-row block are stored as K/256 tiles of 128 rows x
-// 128 bytes (256 values), row m at m * 128 and its 16-byte chunk c at ((c ^ (m % 8)) * 16):
-// the 128-byte swizzle the tensor core reads, so a tile (or its first rows) is one
-// contiguous copy.  Byte offset of 16-byte chunk c of row m of tile (block, kt):
+// Activation units.  The expert inputs (A1) and the SwiGLU outputs (A2) of each 128-row
+// block are stored K step by K step, one unit per K step: first the step's codes, a tile of
+// 128 rows x 128 bytes (NVFP4: 256 values, MXFP8: 128), row m at m * 128 and its 16-byte
+// chunk c at ((c ^ (m % 8)) * 16) (the 128-byte swizzle the tensor core reads), then the
+// step's scales (NVFP4: [128 rows][16] bytes; MXFP8: one 512-byte atom).  A K step of the
+// activations and its scales are therefore one contiguous copy for the GEMM.
+constexpr int kActCodeBytes = 16384;
+constexpr int kActUnitNvfp4 = kActCodeBytes + 128 * 16;
+constexpr int kActUnitMx = kActCodeBytes + 512;
+
+// NVFP4: byte offset of 16-byte code chunk c of row m in K step kt of `block`.
 __device__ __forceinline__ size_t act_tile_offset(size_t block, int k_tiles, int kt, int m, int c) {
-  return (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(kt)) * 16384u +
+  return (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(kt)) * kActUnitNvfp4 +
          static_cast<size_t>(m * 128 + ((c ^ (m & 7)) << 4));
 }
 
@@ -394,13 +401,13 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&v)[8]) {
                : "memory");
 }
 
-// 32 code bytes = 16-byte chunks c and c + 1 (c even) of row m of activation tile
-// (block, kt).  Under the swizzle the two chunks fill one 32-byte aligned span
+// MXFP8: 32 code bytes = 16-byte chunks c and c + 1 (c even) of row m in K step kt of
+// `block`.  Under the swizzle the two chunks fill one 32-byte aligned span
 // (c ^ (m % 8) and (c + 1) ^ (m % 8) differ only in bit 0), chunk c first when m is even
 // and second when m is odd; one 32-byte store writes both.
 __device__ __forceinline__ void st_act_pair(uint8_t* tiles, size_t block, int k_tiles, int kt, int m, int c,
                                             const uint32_t (&w)[8]) {
-  uint8_t* p = tiles + (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(kt)) * 16384u +
+  uint8_t* p = tiles + (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(kt)) * kActUnitMx +
                static_cast<size_t>(m * 128 + ((c ^ (m & 6)) << 4));
   const bool swap = (m & 1) != 0;
   uint32_t s[8];
@@ -409,21 +416,22 @@ __device__ __forceinline__ void st_act_pair(uint8_t* tiles, size_t block, int k_
   st_global_v8(p, s);
 }
 
-// NVFP4 activation scales in K-step chunks: the 16 scales of one K step (256 values) of the
-// 128 rows of a block are one 2 KB chunk, row m's 16 bytes at m 16, so a K step's scales are
-// one contiguous copy for the GEMM and a row's 16 bytes are one contiguous store for the
-// writers.  (The 512-byte-atom order of the tensor cores scattered a row's scales in 4-byte
-// pieces 512 bytes apart, whose partial-sector writes held the A1 writer at ~3.4 TB/s where
-// 16-byte pieces reach ~4.5 TB/s; the scale warps gather the atom order from the chunk.)
+// NVFP4 activation scales: the 16 scales of one K step (256 values) of the 128 rows of a
+// block follow the step's codes as a [128 rows][16] chunk, row m's 16 bytes at m * 16, so a
+// row's scales of a K step are one contiguous store for the writers.  (The 512-byte-atom
+// order of the tensor cores scattered a row's scales in 4-byte pieces 512 bytes apart, whose
+// partial-sector writes held the A1 writer at ~3.4 TB/s where 16-byte pieces reach ~4.5 TB/s;
+// the GEMM's scale warps gather the atom order from the chunk.)  Byte offset of scale s of
+// row m of `block`, in the same buffer as the codes:
 __device__ __forceinline__ size_t sf_chunk_offset(size_t block, int k_tiles, int m, int s) {
-  return ((block * static_cast<size_t>(k_tiles) + static_cast<size_t>(s >> 4)) * 128u + static_cast<size_t>(m)) * 16u +
-         static_cast<size_t>(s & 15);
+  return (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(s >> 4)) * kActUnitNvfp4 + kActCodeBytes +
+         static_cast<size_t>(m * 16 + (s & 15));
 }
 
-// MXFP8 activation scales: byte offset of scale s of row m (0..127) in a 128-row scale block
-// with K/128 four-scale groups (the tcgen05 scale-factor atom order).
-__device__ __forceinline__ size_t sf_atom_offset(size_t block, int kgroups, int m, int s) {
-  return (block * static_cast<size_t>(kgroups) + static_cast<size_t>(s >> 2)) * 512u +
+// MXFP8 activation scales: scale s of row m (0..127) of `block` (K/128 K steps of four
+// scales) in the 512-byte atom after its K step's codes (the tcgen05 scale-factor atom order).
+__device__ __forceinline__ size_t sf_atom_offset(size_t block, int k_tiles, int m, int s) {
+  return (block * static_cast<size_t>(k_tiles) + static_cast<size_t>(s >> 2)) * kActUnitMx + kActCodeBytes +
          static_cast<size_t>((m & 31) * 16 + (m >> 5) * 4 + (s & 3));
 }
 

@@ -142,7 +142,6 @@ __global__ void __launch_bounds__(kEpDispatchThreads) ep_dispatch_kernel(
     const int32_t* __restrict__ offsets, const EpDest* __restrict__ dst, int T, int H, int k, float alpha, TpGroup g,
     EpLayout lay) {
   __shared__ uint8_t* s_a1[kEpMaxK];
-  __shared__ uint8_t* s_sf[kEpMaxK];
   __shared__ int s_blk[kEpMaxK], s_m[kEpMaxK];
   const int tid = threadIdx.x, lane = tid & 31;
   const int t = blockIdx.x;
@@ -161,7 +160,6 @@ __global__ void __launch_bounds__(kEpDispatchThreads) ep_dispatch_kernel(
     dr = o.rank;
     in_range = blk < lay.nblk && dr < g.world && row < lay.rows;
     s_a1[tid] = g.regions[in_range ? dr : g.rank] + lay.a1;
-    s_sf[tid] = g.regions[in_range ? dr : g.rank] + lay.a1_sf;
     s_blk[tid] = in_range ? blk : -1;
     s_m[tid] = pos & 127;
   }
@@ -198,7 +196,7 @@ __global__ void __launch_bounds__(kEpDispatchThreads) ep_dispatch_kernel(
         if (bj < 0) continue;
         *reinterpret_cast<uint4*>(s_a1[j] + act_tile_offset(bj, H / 256, b >> 4, m, (b & 15) >> 1)) =
             make_uint4(lo, hi, lo1, hi1);
-        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_sf[j] + sf_chunk_offset(bj, H / 256, m, b)) = word;
+        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_a1[j] + sf_chunk_offset(bj, H / 256, m, b)) = word;
       }
     }
   } else {
@@ -230,7 +228,7 @@ __global__ void __launch_bounds__(kEpDispatchThreads) ep_dispatch_kernel(
         const int bj = s_blk[j], m = s_m[j];
         if (bj < 0) continue;
         st_act_pair(s_a1[j], bj, k_tiles, b >> 2, m, (b & 3) * 2, c);
-        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_sf[j] + sf_atom_offset(bj, k_tiles, m, b)) = word;
+        if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(s_a1[j] + sf_atom_offset(bj, k_tiles, m, b)) = word;
       }
     }
   }

@@ -53,16 +53,12 @@ namespace beam {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK_BYTES = 128;  // 256 FP4 values per K step (one 128-byte swizzle row)
-constexpr int A_TILE_BYTES = BM * BK_BYTES;  // 16384: one activation tile in global memory
+constexpr int A_TILE_BYTES = BM * BK_BYTES;  // 16384: the codes of one activation unit
 constexpr int B_BYTES = BN * BK_BYTES;       // 32768
 constexpr int SFA_BYTES = 128 * 16;          // 128 rows x 16 scales (the K step's 256 values)
 constexpr int SFB_BYTES = 2 * 4 * 512;       // 2 row blocks of 128
 static_assert(B_BYTES + SFB_BYTES == kTileBytes, "weight tile = B codes + B scales");
-// Two ring shapes.  Stage layout: A | B | SFB | SFA (B and SFB are one contiguous weight
-// tile).  Full: A holds 128 rows, 4 stages.  Small-M (batches of <= 32 tokens, so every
-// expert has <= 32 rows): A holds 32 rows, which leaves room for a 5th stage of weights in
-// flight.  The MMA still reads 128 rows of A; rows past the region read the stage's B bytes
-// and only feed accumulator rows that are never stored.
+static_assert(A_TILE_BYTES == kActCodeBytes, "activation unit codes");
 //
 // Operand formats.  A K step is one 128-byte swizzle row per operand row in both: 256 E2M1
 // values (NVFP4: 4 MMAs of K = 64, 16 scales of 16 values per row) or 128 E4M3 values
@@ -72,30 +68,47 @@ struct FmtNvfp4 {
   static constexpr int SFA = SFA_BYTES;    // one K-step chunk: [128 rows][16 scales]
   static constexpr int SFB = SFB_BYTES;    // 2 row halves x 4 atoms
   static constexpr int TILE = kTileBytes;  // weight tile: B codes + B scales
+  static constexpr int UNIT = kActUnitNvfp4;  // activation unit: A codes + A scales
 };
 struct FmtMxfp8 {
   static constexpr bool kMx = true;
   static constexpr int SFA = 512;          // 1 atom: the 4 scales of a row in one 32-bit word
   static constexpr int SFB = 2 * 512;      // 2 row halves
   static constexpr int TILE = kMxTileBytes;
+  static constexpr int UNIT = kActUnitMx;
 };
 static_assert(B_BYTES + FmtMxfp8::SFB == kMxTileBytes, "MXFP8 weight tile = B codes + B scales");
+static_assert(FmtNvfp4::UNIT == A_TILE_BYTES + FmtNvfp4::SFA && FmtMxfp8::UNIT == A_TILE_BYTES + FmtMxfp8::SFA,
+              "activation unit = codes + scales");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;            // 256 FP32 columns
 constexpr uint32_t SF_COL = 256;           // scale factors, one column set per ring stage:
 constexpr uint32_t SF_STAGE_COLS = 48;     //   A: 4 K-groups x 4 columns, then B: 4 K-groups x 8
 constexpr uint32_t SFB_OFF = 16;
 constexpr int kMaxStages = 5;
-// One K step per stage (measured against two K steps per stage, whose operands arrive in
-// fewer, larger copies: 2.21 vs 1.99-2.04 ms at prefill16k, the coarser ring leaves the MMA
-// waiting longer).
+// Two ring shapes, one K step per stage (measured against two K steps per stage, whose
+// operands arrive in fewer, larger copies: 2.21 vs 1.99-2.04 ms at prefill16k, the coarser
+// ring leaves the MMA waiting longer).
+//   Full (A holds 128 rows, 4 stages): the weight tile (B codes, B scales), then at the next
+//     1 KB boundary the activation unit (A codes, A scales): a K step of a 128-row block is
+//     two copies, one per operand (each copy has a fixed cost in the SM's copy path).  A
+//     block of fewer rows copies A's codes and scales of its rows only, as two copies.
+//   Small-M (batches of <= 32 tokens, so every expert has <= 32 rows; 5 stages): A holds 32
+//     rows and comes first, A | B | SFB | SFA, which leaves room for a 5th stage of weights in
+//     flight.  The MMA still reads 128 rows of A; rows past the region read the stage's own B
+//     bytes and only feed accumulator rows that are never stored.  A's codes and scales are
+//     two copies of only the rows present.
+// Offsets are 1 KB aligned where the swizzled operands start.
 template <int kStages, int kABytes, class F = FmtNvfp4>
 struct Ring {
   using Fmt = F;
   static constexpr int STAGES = kStages;
   static constexpr int A_BYTES = kABytes;
-  // padded to 1024 bytes: every stage's operands keep the swizzle alignment
-  static constexpr int STAGE_BYTES = (kABytes + B_BYTES + F::SFB + F::SFA + 1023) / 1024 * 1024;
+  static constexpr bool kFullA = kABytes == A_TILE_BYTES;
+  static constexpr int OFF_B = kFullA ? 0 : kABytes;  // B codes, then B scales
+  static constexpr int OFF_A = kFullA ? (F::TILE + 1023) / 1024 * 1024 : 0;
+  static constexpr int OFF_SFA = kFullA ? OFF_A + kABytes : kABytes + F::TILE;
+  static constexpr int STAGE_BYTES = (OFF_SFA + F::SFA + 1023) / 1024 * 1024;
   static_assert(SF_COL + kStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor stages must fit in TMEM");
   static_assert(kStages <= kMaxStages, "barrier arrays");
 };
@@ -279,8 +292,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
         if (id < 0) break;
         const int k_tiles = t.down ? args.d_k_tiles : args.gu_k_tiles;
         const int n_tiles = t.down ? n_d : n_gu;
-        const uint8_t* a_src = (t.down ? args.a2 : args.a1) + static_cast<size_t>(mb.sf_block) * k_tiles * A_TILE_BYTES;
-        const uint8_t* sfa = (t.down ? args.a2_sf : args.a1_sf) + static_cast<size_t>(mb.sf_block) * k_tiles * F::SFA;
+        const uint8_t* a_src = (t.down ? args.a2 : args.a1) + static_cast<size_t>(mb.sf_block) * k_tiles * F::UNIT;
         const uint8_t* btile = (t.down ? args.w_d : args.w_gu) +
                                (static_cast<size_t>(mb.expert) * n_tiles + t.nt) * k_tiles * static_cast<size_t>(F::TILE);
         if (t.down) {
@@ -298,19 +310,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           }
           fence_proxy_async_global();
         }
-        // rows past the block's valid rows are not copied: their stale shared-memory
-        // contents only reach accumulator rows that are never stored
+        // A block of 128 rows in the full ring: the whole unit, one copy.  Otherwise the
+        // codes and the scales of the block's valid rows (rounded up to 8; the MXFP8 atom
+        // holds all rows' scales), two copies: the stale shared-memory rows past them only
+        // reach accumulator rows never stored.
         uint32_t a_bytes = static_cast<uint32_t>(min(BM, (mb.rows + 7) & ~7)) * BK_BYTES;
         if (a_bytes > static_cast<uint32_t>(A_BYTES)) {  // cannot happen when the host picks the ring right
           atomicOr(args.err, kErrRange);
           a_bytes = A_BYTES;
         }
+        const bool whole = R::kFullA && a_bytes == static_cast<uint32_t>(A_TILE_BYTES);
+        const uint32_t sfa_bytes = F::kMx ? F::SFA : a_bytes / 8;  // NVFP4: 16 scale bytes per row
+        const uint32_t a_copy = whole ? F::UNIT : a_bytes + sfa_bytes;
         // A and its scales of K step kk into stage st
         auto load_a = [&](int st, int kk) {
-          uint8_t* sa = smem + st * STAGE_BYTES;
-          bulk_load(sa, a_src + static_cast<size_t>(kk) * A_TILE_BYTES, a_bytes, &tail->full[st]);
-          // one contiguous chunk per K step (NVFP4: 128 rows x 16 scales; MXFP8: one atom)
-          bulk_load(sa + A_BYTES + B_BYTES + F::SFB, sfa + static_cast<size_t>(kk) * F::SFA, F::SFA, &tail->full[st]);
+          uint8_t* sp = smem + st * STAGE_BYTES;
+          const uint8_t* unit = a_src + static_cast<size_t>(kk) * F::UNIT;
+          if (whole) {
+            bulk_load(sp + R::OFF_A, unit, F::UNIT, &tail->full[st]);
+          } else {
+            bulk_load(sp + R::OFF_A, unit, a_bytes, &tail->full[st]);
+            bulk_load(sp + R::OFF_SFA, unit + A_TILE_BYTES, sfa_bytes, &tail->full[st]);
+          }
         };
         // Before the wait only the weights are loaded; the first tile starts at stage 0, so
         // its deferred K steps kk < STAGES sit in stages kk.
@@ -330,10 +351,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&tail->full[stage], a_bytes + F::TILE + F::SFA);
+          mbar_arrive_expect_tx(&tail->full[stage], a_copy + F::TILE);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-          bulk_load(smem + stage * STAGE_BYTES + A_BYTES, btile + static_cast<size_t>(kt) * F::TILE, F::TILE,
+          bulk_load(smem + stage * STAGE_BYTES + R::OFF_B, btile + static_cast<size_t>(kt) * F::TILE, F::TILE,
                     &tail->full[stage]);
           if (waited)
             load_a(stage, kt);
@@ -384,8 +405,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES + R::OFF_A);
+          const uint32_t sb = smem_u32(smem + stage * STAGE_BYTES + R::OFF_B);
           const uint32_t sf = tmem + SF_COL + stage * SF_STAGE_COLS;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
@@ -441,8 +462,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           ok = false;
           break;
         }
-        const uint8_t* ssfb = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;  // [half][K-group][512]
-        const uint8_t* ssfa = ssfb + F::SFB;  // NVFP4 [128 rows][16 scales]; MXFP8 one 512-byte atom
+        const uint8_t* ssfb = smem + stage * STAGE_BYTES + R::OFF_B + B_BYTES;  // [half][K-group][512]
+        const uint8_t* ssfa = smem + stage * STAGE_BYTES + R::OFF_SFA;  // NVFP4 [128 rows][16]; MXFP8 one atom
         const uint32_t col = SF_COL + stage * SF_STAGE_COLS;
         if constexpr (F::kMx) {
           // one atom of A scales -> columns 0..3; B: rows 0-127 -> SFB_OFF + 0..3, rows 128-255 -> + 4..7
@@ -475,7 +496,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
             for (int q = 0; q < 2; ++q) {
               const int kb = part * 2 + q;
               const uint4 v0 = *reinterpret_cast<const uint4*>(ssfb + kb * 512 + lane * 16);
-              const uint4 v1 = *reinterpret_cast<const uint4*>(ssfb + SFA_BYTES + kb * 512 + lane * 16);
+              const uint4 v1 = *reinterpret_cast<const uint4*>(ssfb + SFB_BYTES / 2 + kb * 512 + lane * 16);
               r[q * 8 + 0] = v0.x; r[q * 8 + 1] = v0.y; r[q * 8 + 2] = v0.z; r[q * 8 + 3] = v0.w;
               r[q * 8 + 4] = v1.x; r[q * 8 + 5] = v1.y; r[q * 8 + 6] = v1.z; r[q * 8 + 7] = v1.w;
             }
@@ -547,7 +568,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
           uint32_t c[8];
           const uint32_t sc = quant_block32_mx(h, c);
           st_act_pair(args.a2, mb.sf_block, args.d_k_tiles, f0 >> 7, row_in_tile, (f0 & 127) >> 4, c);
-          args.a2_sf[sf_atom_offset(mb.sf_block, args.d_k_tiles, row_in_tile, f0 >> 5)] = static_cast<uint8_t>(sc);
+          args.a2[sf_atom_offset(mb.sf_block, args.d_k_tiles, row_in_tile, f0 >> 5)] = static_cast<uint8_t>(sc);
         } else if (valid) {
           const float scale = mb.scale_gu;
           const int f0 = t.nt * 128 + group * 32;  // first feature of this thread's 32
@@ -570,7 +591,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_experts_kernel(const Expe
                                                               (f0 & 255) >> 5)) =
               make_uint4(codes[0], codes[1], codes[2], codes[3]);
           // its 2 scales are 2 contiguous bytes of the row's 16 in its K step (f0 / 16 is even)
-          *reinterpret_cast<uint16_t*>(args.a2_sf + sf_chunk_offset(mb.sf_block, args.d_k_tiles, row_in_tile,
+          *reinterpret_cast<uint16_t*>(args.a2 + sf_chunk_offset(mb.sf_block, args.d_k_tiles, row_in_tile,
                                                                     f0 / 16)) = static_cast<uint16_t>(scodes);
         }
         // publish this warp's share of block t.block's A2 to the down-tile producers

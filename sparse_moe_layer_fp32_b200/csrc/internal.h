@@ -88,8 +88,9 @@ cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,
                            const int32_t* sf_block, int T, int k, int E, int32_t* perm_src, int32_t* inv,
                            int32_t* tile_row, cudaStream_t s);
+// A1 = Q(x) into the activation units: [blk][H/256][18432], codes then scales (common.cuh).
 cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, float alpha, uint8_t* a1,
-                            uint8_t* a1_sf, cudaStream_t s);
+                            cudaStream_t s);
 
 // ---- weight quantiser and repacking (quant.cu)
 // Contiguous weight tiles of the grouped GEMMs: 256 rows x 256 K values of codes in the
@@ -115,13 +116,14 @@ cudaError_t launch_repack_tiles_mx(const uint8_t* codes, const uint8_t* sf, int 
                                    int interleave_inter, uint8_t* dst, cudaStream_t s);
 cudaError_t launch_quantize_rows_mx(const float* src, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* sf,
                                     cudaStream_t s);
-// A1 = MX(x) into the activation tiles: [blk][H/128][16384] codes, [blk][H/128][512] scales.
+// A1 = MX(x) into the activation units: [blk][H/128][16896], 16384 code bytes then a
+// 512-byte scale atom per K step.
 cudaError_t launch_quant_a1_mx(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, uint8_t* a1,
-                               uint8_t* a1_sf, cudaStream_t s);
+                               cudaStream_t s);
 
 // ---- grouped NVFP4 GEMMs, gate/up and down in one launch (gemm_experts.cu)
-// Activation tiles are [blk][K/256][16384] (act_tile_offset), their scales [blk][K/256][128
-// rows][16] (sf_chunk_offset); weight tiles are [E][n_tiles][K/256][kTileBytes].
+// Activations are units of one K step, [blk][K/256][16384 code bytes, then 128 rows x 16
+// scales] (act_tile_offset, sf_chunk_offset); weight tiles are [E][n_tiles][K/256][kTileBytes].
 struct ExpertGemmArgs {
   const MBlock* mblocks;
   const int32_t* num_mblocks;
@@ -129,12 +131,10 @@ struct ExpertGemmArgs {
   // gate/up: K = H, 256 B rows per output tile = 128 gate + 128 up features
   int gu_n_tiles;           // I / 128
   int gu_k_tiles;           // H / 256
-  const uint8_t* a1;
-  const uint8_t* a1_sf;
+  const uint8_t* a1;        // activation units, codes and scales
   const uint8_t* w_gu;
   // SwiGLU + NVFP4 epilogue output, the down GEMM's A operand (K = Ip)
-  uint8_t* a2;
-  uint8_t* a2_sf;
+  uint8_t* a2;               // activation units, codes and scales
   float alpha_a2;
   // down: K = Ip
   int d_n_tiles;            // H / 256
@@ -200,8 +200,7 @@ struct EpLayout {
   size_t counts;    // int32 [kMaxTpRanks][E]: rows source rank s routes to expert e
   size_t arrivals;  // u32 [nblk]: rows delivered into each 128-row block of this rank's experts
   size_t origin;    // int32 [rows]: source rank << 24 | source slot t k + j of each received row
-  size_t a1;        // activation tiles of the received rows (the GEMM layout)
-  size_t a1_sf;     // their scale blocks
+  size_t a1;        // activation units (codes and scales) of the received rows, the GEMM layout
   size_t ret;       // BF16 [max_tokens][k][H]: this rank's slots' expert outputs, returned
   size_t bytes;     // the whole region
   int nblk;         // blocks the arrival counters cover

@@ -12,8 +12,9 @@
 // A1 = Q(x, alpha_a1): x rows are quantised once per token (16-value blocks along H) and
 // the codes are written to the token's k permuted rows (the NVFP4 W4A4 experts of the
 // recipe "reflection/Beam-1.0-501B-A23B", section "Variants"), as activation tiles (see
-// act_tile_offset) of the row's 128-row block, the scales in K-step chunks (sf_chunk_offset).  For the block-scaled FP8 variant of the
-// experts (the recipe's FP8 checkpoint, read as MXFP8), A1 = MX(x) in 32-value blocks.
+// act_tile_offset) of the row's 128-row block, each K step's scales after its codes
+// (sf_chunk_offset).  For the block-scaled FP8 variant of the experts (the recipe's FP8
+// checkpoint, read as MXFP8), A1 = MX(x) in 32-value blocks.
 #include "common.cuh"
 #include "internal.h"
 
@@ -139,8 +140,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
 // tensor-core layout) combine their scale bytes and one of them stores the 32-bit word.
 __global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restrict__ x,
                                                        const int32_t* __restrict__ tile_row, int T, int H, int k,
-                                                       float alpha, uint8_t* __restrict__ a1,
-                                                       uint8_t* __restrict__ a1_sf) {
+                                                       float alpha, uint8_t* __restrict__ a1) {
   const int nb = H / 16;
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
@@ -179,15 +179,14 @@ __global__ void __launch_bounds__(128) quant_a1_kernel(const uint16_t* __restric
     // block b of 16 values: 8 bytes, half of 16-byte chunk (b % 16) / 2 of K tile b / 16
     *reinterpret_cast<uint2*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1) + (b & 1) * 8) =
         make_uint2(lo, hi);
-    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_chunk_offset(blk, H / 256, m, b)) = word;
+    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1 + sf_chunk_offset(blk, H / 256, m, b)) = word;
   }
 }
 
 // Large batches: one warp per token, quantise x[t] once, write it to the token's k rows.
 __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __restrict__ x,
                                                        const int32_t* __restrict__ tile_row, int T, int H,
-                                                       int k, float alpha, uint8_t* __restrict__ a1,
-                                                       uint8_t* __restrict__ a1_sf) {
+                                                       int k, float alpha, uint8_t* __restrict__ a1) {
   __shared__ int s_blk[8][16], s_m[8][16];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * 8 + warp;
@@ -242,7 +241,7 @@ __global__ void __launch_bounds__(256) quant_a1_wide_kernel(const uint16_t* __re
       const int blk = s_blk[warp][j], m = s_m[warp][j];
       *reinterpret_cast<uint4*>(a1 + act_tile_offset(blk, H / 256, b >> 4, m, (b & 15) >> 1)) =
           make_uint4(lo, hi, lo1, hi1);
-      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_chunk_offset(blk, H / 256, m, b)) = word;
+      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1 + sf_chunk_offset(blk, H / 256, m, b)) = word;
     }
   }
 }
@@ -270,7 +269,7 @@ __device__ __forceinline__ void load_block32_bf16(const uint16_t* __restrict__ x
 
 __global__ void __launch_bounds__(128) quant_a1_mx_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ tile_row, int T, int H, int k,
-                                                          uint8_t* __restrict__ a1, uint8_t* __restrict__ a1_sf) {
+                                                          uint8_t* __restrict__ a1) {
   const int nb = H / 32, k_tiles = H / 128;
   const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
@@ -299,15 +298,14 @@ __global__ void __launch_bounds__(128) quant_a1_mx_kernel(const uint16_t* __rest
     if (j >= k) break;
     const int blk = dst[j] >> 7, m = dst[j] & 127;
     st_act_pair(a1, blk, k_tiles, b >> 2, m, (b & 3) * 2, c);
-    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, k_tiles, m, b)) = word;
+    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1 + sf_atom_offset(blk, k_tiles, m, b)) = word;
   }
 }
 
 // Large batches: one warp per token, lane = 32-value block.
 __global__ void __launch_bounds__(256) quant_a1_mx_wide_kernel(const uint16_t* __restrict__ x,
                                                                const int32_t* __restrict__ tile_row, int T, int H,
-                                                               int k, uint8_t* __restrict__ a1,
-                                                               uint8_t* __restrict__ a1_sf) {
+                                                               int k, uint8_t* __restrict__ a1) {
   __shared__ int s_blk[8][16], s_m[8][16];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * 8 + warp;
@@ -338,18 +336,18 @@ __global__ void __launch_bounds__(256) quant_a1_mx_wide_kernel(const uint16_t* _
     for (int j = 0; j < k; ++j) {
       const int blk = s_blk[warp][j], m = s_m[warp][j];
       st_act_pair(a1, blk, k_tiles, b >> 2, m, (b & 3) * 2, c);
-      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1_sf + sf_atom_offset(blk, k_tiles, m, b)) = word;
+      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(a1 + sf_atom_offset(blk, k_tiles, m, b)) = word;
     }
   }
 }
 
 cudaError_t launch_quant_a1_mx(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, uint8_t* a1,
-                               uint8_t* a1_sf, cudaStream_t s) {
+                               cudaStream_t s) {
   if (T >= 256)
-    return launch_pdl(quant_a1_mx_wide_kernel, dim3((T + 7) / 8), dim3(256), 0, s, x, tile_row, T, H, k, a1, a1_sf);
+    return launch_pdl(quant_a1_mx_wide_kernel, dim3((T + 7) / 8), dim3(256), 0, s, x, tile_row, T, H, k, a1);
   const int64_t threads = static_cast<int64_t>(T) * (H / 32);
   return launch_pdl(quant_a1_mx_kernel, dim3(static_cast<unsigned>((threads + 127) / 128)), dim3(128), 0, s, x,
-                    tile_row, T, H, k, a1, a1_sf);
+                    tile_row, T, H, k, a1);
 }
 
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s) {
@@ -381,12 +379,12 @@ cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const 
 }
 
 cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, float alpha, uint8_t* a1,
-                            uint8_t* a1_sf, cudaStream_t s) {
+                            cudaStream_t s) {
   if (T >= 256)
-    return launch_pdl(quant_a1_wide_kernel, dim3((T + 7) / 8), dim3(256), 0, s, x, tile_row, T, H, k, alpha, a1, a1_sf);
+    return launch_pdl(quant_a1_wide_kernel, dim3((T + 7) / 8), dim3(256), 0, s, x, tile_row, T, H, k, alpha, a1);
   const int64_t threads = static_cast<int64_t>(T) * (H / 16);
   return launch_pdl(quant_a1_kernel, dim3(static_cast<unsigned>((threads + 127) / 128)), dim3(128), 0, s, x, tile_row,
-                    T, H, k, alpha, a1, a1_sf);
+                    T, H, k, alpha, a1);
 }
 
 }  // namespace beam

@@ -26,16 +26,26 @@ def buf(layer, which, dtype):
     return to_np(layer.debug(which)).view(dtype)
 
 
-def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int, block: int = 16) -> np.ndarray:
-    """Activation scales (beam_moe.h layouts) -> row-major scales [rows, kcols/block] in
-    permuted row order: block = 16 (NVFP4, stored in K-step chunks of 128 rows x 16 scales) or
-    32 (MXFP8, stored in 512-byte atoms of 4 scales per row)."""
+ACT_CODE_BYTES = 16384  # codes of one activation unit (128 rows x 128 bytes)
+
+
+def act_unit_bytes(block: int) -> int:
+    """Bytes of one activation unit (one 128-row block, one K step): the codes, then the
+    scales (NVFP4, block 16: 128 rows x 16; MXFP8, block 32: one 512-byte atom)."""
+    return ACT_CODE_BYTES + (128 * 16 if block == 16 else 512)
+
+
+def sf_rows(units: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int, block: int = 16) -> np.ndarray:
+    """Activation units (beam_moe.h layouts) -> row-major scales [rows, kcols/block] in
+    permuted row order: block = 16 (NVFP4, each K step's 128 rows x 16 scales after its
+    codes) or 32 (MXFP8, a 512-byte atom of 4 scales per row after each K step's codes)."""
     experts = len(offsets) - 1
     rows = int(offsets[-1])
     n_sc = kcols // block
     kgroups = n_sc // 4
     out = np.zeros((rows, n_sc), np.uint8)
     s = np.arange(n_sc)
+    unit = act_unit_bytes(block)
     for e in range(experts):
         n = int(offsets[e + 1] - offsets[e])
         if n == 0:
@@ -44,24 +54,26 @@ def sf_rows(sf_buf: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols
         blk = sf_block[e] + i // 128
         m = i % 128
         if block == 16:
-            off = ((blk[:, None] * (n_sc // 16) + s[None, :] // 16) * 128 + m[:, None]) * 16 + s[None, :] % 16
+            off = ((blk[:, None] * (n_sc // 16) + s[None, :] // 16) * unit + ACT_CODE_BYTES + m[:, None] * 16
+                   + s[None, :] % 16)
         else:
-            off = ((blk[:, None] * kgroups + s[None, :] // 4) * 512 + (m[:, None] % 32) * 16 + (m[:, None] // 32) * 4
-                   + s[None, :] % 4)
-        out[offsets[e]:offsets[e + 1]] = sf_buf[off]
+            off = ((blk[:, None] * kgroups + s[None, :] // 4) * unit + ACT_CODE_BYTES + (m[:, None] % 32) * 16
+                   + (m[:, None] // 32) * 4 + s[None, :] % 4)
+        out[offsets[e]:offsets[e + 1]] = units[off]
     return out
 
 
-def tile_rows(tiles: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int,
+def tile_rows(units: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcols: int,
               values_per_byte: int = 2) -> np.ndarray:
-    """Activation tiles (beam_moe.h layout) -> codes [rows, kcols / values_per_byte] in permuted
-    row order (2: packed NVFP4; 1: MXFP8).  A tile holds 128 code bytes of each row."""
+    """Activation units (beam_moe.h layout) -> codes [rows, kcols / values_per_byte] in
+    permuted row order (2: packed NVFP4; 1: MXFP8).  A unit holds 128 code bytes of each row."""
     experts = len(offsets) - 1
     rows = int(offsets[-1])
     row_bytes = kcols // values_per_byte
     k_tiles = row_bytes // 128
     out = np.zeros((rows, row_bytes), np.uint8)
     j = np.arange(row_bytes)
+    unit = act_unit_bytes(16 if values_per_byte == 2 else 32)
     for e in range(experts):
         n = int(offsets[e + 1] - offsets[e])
         if n == 0:
@@ -69,9 +81,9 @@ def tile_rows(tiles: np.ndarray, sf_block: np.ndarray, offsets: np.ndarray, kcol
         i = np.arange(n)
         blk = (sf_block[e] + i // 128)[:, None]
         m = (i % 128)[:, None]
-        off = ((blk * k_tiles + j[None, :] // 128) * 16384 + m * 128 + ((((j[None, :] % 128) // 16) ^ (m % 8)) * 16)
+        off = ((blk * k_tiles + j[None, :] // 128) * unit + m * 128 + ((((j[None, :] % 128) // 16) ^ (m % 8)) * 16)
                + j[None, :] % 16)
-        out[offsets[e]:offsets[e + 1]] = tiles[off]
+        out[offsets[e]:offsets[e + 1]] = units[off]
     return out
 
 
@@ -218,7 +230,7 @@ def a2_boundary_tokens(layer, T, k, I, h32_tok, alpha2, fmt, skip=None):
     sfb = buf(layer, bm.BUF_SFBLOCK, np.int32)
     inv = buf(layer, bm.BUF_INV, np.int32).reshape(-1, k)[:T]
     codes = tile_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, Ip, values_per_byte=vpb)[:, : I // vpb]
-    sf = sf_rows(buf(layer, bm.BUF_A2_SF, np.uint8), sfb, offsets, Ip, block=blk)[:, : I // blk]
+    sf = sf_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, Ip, block=blk)[:, : I // blk]
     keep = np.ones(T, bool) if skip is None else ~np.asarray(skip, bool)
     tok = np.nonzero(keep)[0]
     rows = inv[tok].reshape(-1)

@@ -89,13 +89,13 @@ def test_forward_stages_and_end_to_end(bm, name, tokens, seed):
     np.testing.assert_array_equal(sfb, np.concatenate([[0], np.cumsum(nblk)]))
     # ---- A1: bit-exact
     a1p = tile_rows(buf(layer, bm.BUF_A1, np.uint8), sfb, offsets, H)
-    a1s = sf_rows(buf(layer, bm.BUF_A1_SF, np.uint8), sfb, offsets, H)
+    a1s = sf_rows(buf(layer, bm.BUF_A1, np.uint8), sfb, offsets, H)
     rp, rs = nvfp4.quantize_nvfp4(x[perm].astype(np.float32), a1)
     np.testing.assert_array_equal(a1s, rs)
     np.testing.assert_array_equal(norm_zero(a1p), norm_zero(rp))
     # ---- A2 and y from the GPU's own inputs
     a2p = tile_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, Ip)[:, : I // 2]
-    a2s = sf_rows(buf(layer, bm.BUF_A2_SF, np.uint8), sfb, offsets, Ip)[:, : I // 16]
+    a2s = sf_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, Ip)[:, : I // 16]
     y = to_np(layer.debug(bm.BUF_Y).view(torch.bfloat16).float()).reshape(T * k, H).astype(np.float64)
     mism, n_codes = 0, 0
     y_ref = np.zeros_like(y)
@@ -242,13 +242,13 @@ def test_forward_mxfp8_stages_and_end_to_end(bm, name, tokens, seed):
     np.testing.assert_array_equal(inv, pm["inv"])
     # ---- A1 = MX(x rows): bit-exact
     a1c = tile_rows(buf(layer, bm.BUF_A1, np.uint8), sfb, offsets, H, values_per_byte=1)
-    a1s = sf_rows(buf(layer, bm.BUF_A1_SF, np.uint8), sfb, offsets, H, block=32)
+    a1s = sf_rows(buf(layer, bm.BUF_A1, np.uint8), sfb, offsets, H, block=32)
     rc, rs = mxfp8.quantize_mxfp8(x[perm].astype(np.float32))
     np.testing.assert_array_equal(a1s, rs)
     np.testing.assert_array_equal(a1c, rc)
     # ---- A2 and y from the GPU's own A1
     a2c = tile_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, I, values_per_byte=1)
-    a2s = sf_rows(buf(layer, bm.BUF_A2_SF, np.uint8), sfb, offsets, I, block=32)
+    a2s = sf_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, I, block=32)
     y = to_np(layer.debug(bm.BUF_Y).view(torch.bfloat16).float()).reshape(T * k, H).astype(np.float64)
     mism, n_codes = 0, 0
     y_ref = np.zeros_like(y)

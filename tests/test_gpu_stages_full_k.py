@@ -80,7 +80,7 @@ def test_full_k_stages_on_every_row(bm, fmt, tokens, seed):
     # ---- A1: bit-exact on every row
     vpb, blk = (1, 32) if mx else (2, 16)
     a1c = tile_rows(buf(layer, bm.BUF_A1, np.uint8), sfb, offsets, H, values_per_byte=vpb)
-    a1s = sf_rows(buf(layer, bm.BUF_A1_SF, np.uint8), sfb, offsets, H, block=blk)
+    a1s = sf_rows(buf(layer, bm.BUF_A1, np.uint8), sfb, offsets, H, block=blk)
     if mx:
         rc, rs = mxfp8.quantize_mxfp8(x32[perm])
         np.testing.assert_array_equal(a1c, rc)
@@ -91,7 +91,7 @@ def test_full_k_stages_on_every_row(bm, fmt, tokens, seed):
     del rc, rs
     # ---- A2, y (from the GPU's own A1 / A2) and the oracle's own m, expert by expert
     a2c = tile_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, Ip, values_per_byte=vpb)[:, : I // vpb]
-    a2s = sf_rows(buf(layer, bm.BUF_A2_SF, np.uint8), sfb, offsets, Ip, block=blk)[:, : I // blk]
+    a2s = sf_rows(buf(layer, bm.BUF_A2, np.uint8), sfb, offsets, Ip, block=blk)[:, : I // blk]
     y = to_np(layer.debug(bm.BUF_Y).view(torch.bfloat16).float()).reshape(T * k, H)
     w_ref = np.zeros((T, E))
     np.put_along_axis(w_ref, r_ids, r_w, axis=1)
