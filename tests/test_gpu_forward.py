@@ -303,3 +303,30 @@ def test_forward_host_buffers_match_device_path(bm, fmt):
         assert torch.equal(oh, ref.cpu()), (T, pinned)
     layer.check()
     layer.close()
+
+
+def test_profiled_sections_and_launch_counts(bm):
+    """Per-kernel timing of a forward (beam_moe_profile_enable / _read): one named section per
+    kernel launched, in launch order, ending with the finalize; the output is the same bits
+    with timing on."""
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(SHAPES["mid"], tokens=300)
+    weights = synthetic.make_weights(shape, 31, threads=4)
+    layer = bm.MoELayer(max_tokens=300, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                        inter=shape.inter, alpha_a1=0.01, alpha_a2=0.01, **weights)
+    for T in (8, 40, 255, 256, 300):
+        x, r = synthetic.make_batch(dataclasses.replace(shape, tokens=T), T)
+        x, r = x.cuda(), r.cuda()
+        plain = layer.forward(x, r)
+        layer.check()
+        layer.profile(True)
+        timed = layer.forward(x, r)
+        sections = layer.kernel_times()
+        layer.profile(False)
+        layer.check()
+        assert torch.equal(plain, timed), T
+        names = [n for n, _ in sections]
+        assert names[-1] == "finalize" and names.count("quant_a1") == 1 and "gemm_experts" in names, names
+        assert all(ms >= 0 for _, ms in sections)
+        assert layer.launches() == len(names), (T, names)
+    layer.close()
