@@ -147,8 +147,16 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_prenorm(beam_moe_t h, const void* 
  * starts once x has landed and runs on a second stream of the handle, overlapping the
  * routing and the expert GEMMs; only the finalize waits for it (the first call creates that
  * stream and two events).
- * All copies are cudaMemcpyAsync; pinned host memory makes them asynchronous.  The caller
- * synchronises `stream` before reading out_host. */
+ * Batches of 2 x BEAM_MOE_HOST_CHUNK_TOKENS tokens or more (beam_moe_set_host_chunk_tokens)
+ * run in parts of that many tokens: the second stream uploads each part's x and residual in
+ * turn, `stream` runs each part's forward as its x lands, and a third stream of the handle
+ * copies each part's out back as soon as it is final, under the later parts' uploads.  The
+ * parts take the whole batch's router, finalize and GEMM forms, so out has the same bits as
+ * without parts.  Not with BEAM_MOE_ROUTER_SIMT.  After such a call the internal buffers
+ * (beam_moe_debug_copy) and the kernel timings hold the last part's.
+ * All copies are cudaMemcpyAsync; pinned host memory makes them asynchronous.  The work
+ * enqueued on `stream` ends with out_host complete: the caller synchronises `stream` before
+ * reading it. */
 BEAM_MOE_API beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const void* residual_host, void* out_host,
                                       int32_t num_tokens, void* stream);
 
@@ -209,6 +217,14 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_tp_phase(beam_moe_t h, const void*
  * source pages: exposed for tuning and testing.  INVALID_ARG for min_tokens < 1. */
 #define BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS 256
 BEAM_MOE_API beam_moe_status beam_moe_set_tp_two_shot_tokens(beam_moe_t h, int32_t min_tokens);
+/* Part size of beam_moe_forward_host (tokens, a multiple of 256, the router's largest token
+ * tile; default BEAM_MOE_HOST_CHUNK_TOKENS; 0 = a batch is never split).  Parts of 4096
+ * tokens keep each part's expert GEMMs compute-bound (every part reads the weights of the
+ * experts it routes to) while the host copies, 4 H bytes per token, set the pace.  Not from
+ * the source pages: an implementation choice exposed for tuning and testing.  INVALID_ARG
+ * for tokens < 0 or not a multiple of 256. */
+#define BEAM_MOE_HOST_CHUNK_TOKENS 4096
+BEAM_MOE_API beam_moe_status beam_moe_set_host_chunk_tokens(beam_moe_t h, int32_t tokens);
 /* cudaIpcGetMemHandle / cudaIpcOpenMemHandle / cudaIpcCloseMemHandle of a region, as
  * BEAM_MOE_IPC_HANDLE_BYTES opaque bytes (host memory), so that callers need no CUDA
  * headers. */

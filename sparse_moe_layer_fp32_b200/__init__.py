@@ -30,6 +30,7 @@ EXPORTED = [
     "beam_moe_forward_tp", "beam_moe_forward_tp_phase", "beam_moe_ipc_export", "beam_moe_ipc_import",
     "beam_moe_ipc_close", "beam_moe_create_ep", "beam_moe_create_ep_mxfp8", "beam_moe_forward_ep",
     "beam_moe_forward_ep_phase", "beam_moe_set_router_mode", "beam_moe_set_tp_two_shot_tokens",
+    "beam_moe_set_host_chunk_tokens",
 ]
 IPC_HANDLE_BYTES = 64
 FMT_NVFP4, FMT_MXFP8 = 0, 1
@@ -79,6 +80,7 @@ def _load():
         "beam_moe_profile_enable": (i32, [vp, i32]),
         "beam_moe_set_router_mode": (i32, [vp, i32]),
         "beam_moe_set_tp_two_shot_tokens": (i32, [vp, i32]),
+        "beam_moe_set_host_chunk_tokens": (i32, [vp, i32]),
         "beam_moe_profile_read": (i32, [vp, ctypes.POINTER(f32), i32, ctypes.POINTER(i32)]),
         "beam_moe_kernel_name": (ctypes.c_char_p, [vp, i32]),
         "beam_moe_route_static": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
@@ -304,10 +306,15 @@ def beam_moe_set_router_mode(h, mode: int):
 
 
 TP_TWO_SHOT_MIN_TOKENS = 256  # BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS
+HOST_CHUNK_TOKENS = 4096  # BEAM_MOE_HOST_CHUNK_TOKENS
 
 
 def beam_moe_set_tp_two_shot_tokens(h, min_tokens: int):
     _check(_lib.beam_moe_set_tp_two_shot_tokens(h, int(min_tokens)), "beam_moe_set_tp_two_shot_tokens")
+
+
+def beam_moe_set_host_chunk_tokens(h, tokens: int):
+    _check(_lib.beam_moe_set_host_chunk_tokens(h, int(tokens)), "beam_moe_set_host_chunk_tokens")
 
 
 def beam_moe_profile_enable(h, enable: bool = True):
@@ -413,6 +420,10 @@ class MoELayer:
 
     def set_tp_two_shot_tokens(self, min_tokens: int):
         beam_moe_set_tp_two_shot_tokens(self.handle, min_tokens)
+
+    def set_host_chunk_tokens(self, tokens: int):
+        """Part size of forward_host (0: never split a batch)."""
+        beam_moe_set_host_chunk_tokens(self.handle, tokens)
 
     def kernel_times(self):
         return beam_moe_profile_read(self.handle)

@@ -46,6 +46,12 @@ struct beam_moe_ctx {
   // computes; the finalize waits for it (created on the first host-buffer forward)
   cudaStream_t copy_stream;
   cudaEvent_t ev_start, ev_res;
+  // ... and batches of 2 x host_chunk_tokens or more run in parts of host_chunk_tokens: part
+  // c's output copies back on down_stream while later parts upload and compute
+  int32_t host_chunk_tokens;
+  cudaStream_t down_stream;
+  cudaEvent_t ev_down;
+  std::vector<cudaEvent_t> part_events;  // 3 per part: x landed, residual landed, finalized
   // tensor parallelism (beam_moe_tp_*): this handle holds one rank's slice of the experts
   uint8_t* tp_region;           // this rank's exchange region (owned), or null
   uint8_t** tp_regions_dev;     // device array [kMaxTpRanks]: every rank's region
@@ -246,6 +252,7 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   h->profiling = false;
   h->router_mode = BEAM_MOE_ROUTER_AUTO;
   h->tp_two_shot_min = BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS;
+  h->host_chunk_tokens = BEAM_MOE_HOST_CHUNK_TOKENS;
   h->profiled_last = false;
   for (int i = 0; i < beam_moe_ctx::kMaxEvents; ++i) {
     h->events[i] = nullptr;
@@ -444,7 +451,8 @@ beam_moe_status beam_moe_route(const void* x, const float* router_w, int32_t num
 // rows (see expert_parallel.cu).
 static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* residual, void* out, void* next_x,
                                     const void* next_gamma, float next_eps, int32_t num_tokens, void* stream,
-                                    int tp_phase = -1, cudaEvent_t residual_ready = nullptr, int ep_phase = -1) {
+                                    int tp_phase = -1, cudaEvent_t residual_ready = nullptr, int ep_phase = -1,
+                                    int plan_T = 0, int plan_first = 0) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;
   if (tp_phase < 0 && h->ep && ep_phase < 0) return BEAM_MOE_ERR_INVALID_ARG;  // holds only some experts
   if (tp_phase >= 0) {
@@ -463,6 +471,10 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   if (!aligned(x, 16) || !aligned(residual, 16) || !aligned(out, 16)) return BEAM_MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int T = num_tokens, H = h->H, E = h->E, k = h->k;
+  // Choices that change a row's arithmetic order (router form and slices, finalize form) and
+  // the GEMM ring follow PT: a part of a larger batch (plan_T tokens, this part from token
+  // plan_first on) computes that batch's bits.
+  const int PT = plan_T > 0 ? plan_T : T;
   const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   int launches = 0;
@@ -562,7 +574,7 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     h->tp_epoch = epoch;
     return finish();
   }
-  if (route_small_supported(T, H, E, k)) {
+  if (route_small_supported(PT, H, E, k)) {
     // router + top-k + histogram + scan + permutation in one launch
     int slices = 1;
     BEAM_TRY(launch_route_small(xb, h->router_w, T, H, E, k, h->logits, h->ids, h->w, h->offsets, h->sf_block,
@@ -575,29 +587,30 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     const bool simt_only = h->router_mode == BEAM_MOE_ROUTER_SIMT;
     // AUTO and TENSOR: slices of H whenever the split count is above one (measured faster than
     // one tile per CTA at every batch up to 32K tokens, and than the SIMT router from 17)
-    const bool tc_split = !simt_only && router_tc_split_supported(H, E, k) && T >= kRouterTcSplitMinTokens &&
-                          router_tc_split_count(T, H, h->num_sms) > 1;
+    const bool tc_split = !simt_only && router_tc_split_supported(H, E, k) && PT >= kRouterTcSplitMinTokens &&
+                          router_tc_split_count(PT, H, h->num_sms) > 1;
     if (tc_split) {
       // tensor cores over (token tiles) x (slices of H), partial logits; the top-k kernel
       // sums the slices in order
       CUtensorMap map_x;
-      const RouterTcPlan plan = router_tc_split_plan(T, H, h->num_sms);
+      const RouterTcPlan plan = router_tc_split_plan(PT, H, h->num_sms);
       if (!make_map_bf16(&map_x, xb, H, T, static_cast<uint32_t>(plan.tokens))) return BEAM_MOE_ERR_CUDA;
       const int splits = plan.splits;
       BEAM_TRY(launch_router_tc(map_x, plan.tokens, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s,
-                                splits));
+                                splits, plan_first));
       BEAM_TRY(mark("router_tc"));
       ++launches;
       h->last_splits = splits;
       BEAM_TRY(launch_topk(h->logits, splits, T, E, k, h->ids, h->w, s));
       BEAM_TRY(mark("topk"));
       ++launches;
-    } else if (!simt_only && router_tc_supported(T, H, E, k)) {
+    } else if (!simt_only && router_tc_supported(PT, H, E, k)) {
       // FP32-class logits on the tensor cores (BF16 x 3-part split), top-k in the epilogue
       CUtensorMap map_x;
-      const int rt_tokens = router_tc_tokens_per_cta(T, h->num_sms);
+      const int rt_tokens = router_tc_tokens_per_cta(PT, h->num_sms);
       if (!make_map_bf16(&map_x, xb, H, T, static_cast<uint32_t>(rt_tokens))) return BEAM_MOE_ERR_CUDA;
-      BEAM_TRY(launch_router_tc(map_x, rt_tokens, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s));
+      BEAM_TRY(launch_router_tc(map_x, rt_tokens, h->router_w3, T, H, E, k, h->logits, h->ids, h->w, h->err, s, 1,
+                                plan_first));
       BEAM_TRY(mark("router_tc"));
       ++launches;
       h->last_splits = 1;
@@ -636,7 +649,7 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
   ++launches;
 
   // a token chooses an expert at most once: at most T rows per expert
-  const ExpertGemmArgs g = gemm_args(h->a1, T, nullptr);
+  const ExpertGemmArgs g = gemm_args(h->a1, PT, nullptr);
   if (mx)
     BEAM_TRY(launch_gemm_experts_mx(g, h->num_sms, s));
   else
@@ -658,7 +671,7 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     if (residual_ready) BEAM_TRY(cudaStreamWaitEvent(s, residual_ready, 0));
     BEAM_TRY(launch_finalize(h->y, h->w, h->inv, static_cast<const uint16_t*>(residual), h->gamma, T, H, k,
                              h->cfg.rms_eps, static_cast<uint16_t*>(out), static_cast<uint16_t*>(next_x),
-                             static_cast<const uint16_t*>(next_gamma), next_eps, h->err, s));
+                             static_cast<const uint16_t*>(next_gamma), next_eps, h->err, s, PT));
     BEAM_TRY(mark("finalize"));
     ++launches;
   }
@@ -820,6 +833,63 @@ beam_moe_status beam_moe_ipc_close(void* dev_ptr) {
   return BEAM_MOE_OK;
 }
 
+// The host-buffer forward of a large batch in parts of host_chunk_tokens tokens.  The copy
+// stream uploads x and then the residual of part 0, 1, ... in order; the caller's stream runs
+// each part's forward once its x has landed (its finalize once its residual has); part c's
+// output goes back on down_stream as soon as it is final, while later parts upload and
+// compute.  Host-to-device copies are the bound at large batches (x and residual are 2 T H
+// bytes each way), so the device-to-host copies and the compute now hide under them.  Every
+// part runs with the whole batch's choices of router form and slices, finalize form and
+// GEMM ring (plan_T), so the output has the same bits as one forward of the whole batch.
+static beam_moe_status forward_host_parts(beam_moe_t h, const void* x_host, const void* residual_host,
+                                          void* out_host, int32_t T, cudaStream_t s) {
+  const int ct = h->host_chunk_tokens;
+  const int parts = (T + ct - 1) / ct;
+  if (!h->down_stream) {
+    BEAM_TRY(cudaStreamCreateWithFlags(&h->down_stream, cudaStreamNonBlocking));
+    BEAM_TRY(cudaEventCreateWithFlags(&h->ev_down, cudaEventDisableTiming));
+  }
+  while (h->part_events.size() < static_cast<size_t>(3 * parts)) {
+    cudaEvent_t e;
+    BEAM_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    h->part_events.push_back(e);
+  }
+  const size_t row = sizeof(uint16_t) * static_cast<size_t>(h->H);
+  // the staging buffers are free once everything before this call on `s` is done (the
+  // previous host forward's parts and copies back included: it ended by waiting for them)
+  BEAM_TRY(cudaEventRecord(h->ev_start, s));
+  BEAM_TRY(cudaStreamWaitEvent(h->copy_stream, h->ev_start, 0));
+  BEAM_TRY(cudaStreamWaitEvent(h->down_stream, h->ev_start, 0));
+  for (int c = 0; c < parts; ++c) {
+    const size_t off = row * static_cast<size_t>(c) * ct, n = row * static_cast<size_t>(std::min(ct, T - c * ct));
+    BEAM_TRY(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(h->stage_x) + off, static_cast<const uint8_t*>(x_host) + off,
+                             n, cudaMemcpyHostToDevice, h->copy_stream));
+    BEAM_TRY(cudaEventRecord(h->part_events[3 * c], h->copy_stream));
+    BEAM_TRY(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(h->stage_res) + off,
+                             static_cast<const uint8_t*>(residual_host) + off, n, cudaMemcpyHostToDevice,
+                             h->copy_stream));
+    BEAM_TRY(cudaEventRecord(h->part_events[3 * c + 1], h->copy_stream));
+  }
+  for (int c = 0; c < parts; ++c) {
+    const int Tc = std::min(ct, T - c * ct);
+    const size_t off = row * static_cast<size_t>(c) * ct, n = row * static_cast<size_t>(Tc);
+    BEAM_TRY(cudaStreamWaitEvent(s, h->part_events[3 * c], 0));
+    const beam_moe_status st = forward_impl(h, reinterpret_cast<uint8_t*>(h->stage_x) + off,
+                                            reinterpret_cast<uint8_t*>(h->stage_res) + off,
+                                            reinterpret_cast<uint8_t*>(h->stage_out) + off, nullptr, nullptr, 0.0f, Tc,
+                                            s, -1, h->part_events[3 * c + 1], -1, T, c * ct);
+    if (st != BEAM_MOE_OK) return st;
+    BEAM_TRY(cudaEventRecord(h->part_events[3 * c + 2], s));
+    BEAM_TRY(cudaStreamWaitEvent(h->down_stream, h->part_events[3 * c + 2], 0));
+    BEAM_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(out_host) + off, reinterpret_cast<uint8_t*>(h->stage_out) + off,
+                             n, cudaMemcpyDeviceToHost, h->down_stream));
+  }
+  // the call's work on `s` ends with out_host complete
+  BEAM_TRY(cudaEventRecord(h->ev_down, h->down_stream));
+  BEAM_TRY(cudaStreamWaitEvent(s, h->ev_down, 0));
+  return BEAM_MOE_OK;
+}
+
 beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const void* residual_host, void* out_host,
                                       int32_t num_tokens, void* stream) {
   if (!h) return BEAM_MOE_ERR_INVALID_ARG;
@@ -833,6 +903,9 @@ beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const vo
     BEAM_TRY(cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming));
     BEAM_TRY(cudaEventCreateWithFlags(&h->ev_res, cudaEventDisableTiming));
   }
+  const int ct = h->host_chunk_tokens;
+  if (ct > 0 && num_tokens >= 2 * ct && h->router_mode != BEAM_MOE_ROUTER_SIMT)
+    return forward_host_parts(h, x_host, residual_host, out_host, num_tokens, s);
   // x first, at the full host-to-device bandwidth; the residual upload then starts (after
   // everything before it on `stream`, including the previous forward's finalize, which
   // read the staging buffer) and overlaps the routing and the expert GEMMs; only the
@@ -929,6 +1002,12 @@ beam_moe_status beam_moe_debug_wait_timeout(beam_moe_t h, int64_t limit_ns, void
   return BEAM_MOE_OK;
 }
 
+beam_moe_status beam_moe_set_host_chunk_tokens(beam_moe_t h, int32_t tokens) {
+  if (!h || tokens < 0 || tokens % 256 != 0) return BEAM_MOE_ERR_INVALID_ARG;
+  h->host_chunk_tokens = tokens;
+  return BEAM_MOE_OK;
+}
+
 beam_moe_status beam_moe_set_tp_two_shot_tokens(beam_moe_t h, int32_t min_tokens) {
   if (!h || min_tokens < 1) return BEAM_MOE_ERR_INVALID_ARG;
   h->tp_two_shot_min = min_tokens;
@@ -974,6 +1053,11 @@ void beam_moe_destroy(beam_moe_t h) {
     cudaEventDestroy(h->ev_res);
     cudaStreamDestroy(h->copy_stream);
   }
+  if (h->down_stream) {
+    cudaEventDestroy(h->ev_down);
+    cudaStreamDestroy(h->down_stream);
+  }
+  for (cudaEvent_t e : h->part_events) cudaEventDestroy(e);
   free_all(h);
   delete h;
 }

@@ -265,10 +265,10 @@ static size_t finalize_small_smem(int H, int k) { return static_cast<size_t>(k +
 template <bool PRE>
 static cudaError_t launch_finalize_t(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
                                      const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out,
-                                     NextNorm nn, uint32_t* err, cudaStream_t s) {
+                                     NextNorm nn, uint32_t* err, cudaStream_t s, int form_T) {
   const int nchunks = H / 8;
   const size_t small = finalize_small_smem(H, k);
-  if (T < 256 && small <= 200 * 1024) {
+  if ((form_T > 0 ? form_T : T) < 256 && small <= 200 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(finalize_small_kernel<PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(small));
     if (e != cudaSuccess) return e;
@@ -288,10 +288,10 @@ static cudaError_t launch_finalize_t(const uint16_t* y, const float* w, const in
 
 cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
                             const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, uint16_t* next_x,
-                            const uint16_t* next_gamma, float next_eps, uint32_t* err, cudaStream_t s) {
+                            const uint16_t* next_gamma, float next_eps, uint32_t* err, cudaStream_t s, int form_T) {
   const NextNorm nn{next_x, next_gamma, next_eps};
-  if (next_x) return launch_finalize_t<true>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, err, s);
-  return launch_finalize_t<false>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, err, s);
+  if (next_x) return launch_finalize_t<true>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, err, s, form_T);
+  return launch_finalize_t<false>(y, w, inv, residual, gamma, T, H, k, eps, out, nn, err, s, form_T);
 }
 
 }  // namespace beam

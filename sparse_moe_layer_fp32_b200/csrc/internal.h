@@ -56,10 +56,12 @@ cudaError_t launch_split_router(const float* w, int E, int H, uint16_t* out, cud
 // Tokens per CTA (128 or 256) for a batch of T; also the row count of the x tensor map's box.
 int router_tc_tokens_per_cta(int T, int num_sms);
 // splits > 1: grid (token tiles) x (splits slices of H), partial logits [splits][T][E] into
-// `logits`, no top-k (launch_topk sums the slices and selects).
+// `logits`, no top-k (launch_topk sums the slices and selects).  first_token (a multiple of
+// tokens_per_cta): where these T tokens start in a batch routed in parts; the FP32
+// summation order of a token's logits depends only on its place in that batch.
 cudaError_t launch_router_tc(const CUtensorMap& map_x, int tokens_per_cta, const uint16_t* w_tiles, int T, int H,
                              int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s,
-                             int splits = 1);
+                             int splits = 1, int first_token = 0);
 bool router_tc_split_supported(int H, int E, int k);
 // The sliced form for a batch of T: tokens per CTA (128 or 256) and slices of H.
 struct RouterTcPlan {
@@ -238,8 +240,11 @@ cudaError_t launch_ep_wait_returned(const TpGroup& g, uint32_t epoch, uint32_t* 
 
 // ---- finalize (finalize.cu)
 // next_x != nullptr also writes the next sublayer's pre-norm of out: bf16(out * rinv * next_gamma).
+// form_T (> 0) picks the kernel form as for a batch of that many tokens (the forms sum a
+// row's squares in different orders), so a batch run in parts gives the whole batch's bits.
 cudaError_t launch_finalize(const uint16_t* y, const float* w, const int32_t* inv, const uint16_t* residual,
                             const uint16_t* gamma, int T, int H, int k, float eps, uint16_t* out, uint16_t* next_x,
-                            const uint16_t* next_gamma, float next_eps, uint32_t* err, cudaStream_t s);
+                            const uint16_t* next_gamma, float next_eps, uint32_t* err, cudaStream_t s,
+                            int form_T = 0);
 
 }  // namespace beam

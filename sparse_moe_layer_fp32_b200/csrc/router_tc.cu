@@ -74,7 +74,7 @@ template <int HALVES>
 __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap map_x, const uint8_t* __restrict__ w_tiles, int T,
                      int H, int E, int k, float* __restrict__ logits, int32_t* __restrict__ ids,
-                     float* __restrict__ wout, uint32_t* __restrict__ err, int splits) {
+                     float* __restrict__ wout, uint32_t* __restrict__ err, int splits, int tile_base) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int RT_BM = RtShape<HALVES>::BM, RT_STAGES = RtShape<HALVES>::STAGES, RT_A_BYTES = RtShape<HALVES>::A_BYTES;
@@ -109,9 +109,10 @@ __global__ void __launch_bounds__(RtShape<HALVES>::THREADS, 1)
   const int k_lo = static_cast<int>(blockIdx.y) * k_per;
   const int k_tiles = max(0, min(k_per, k_all - k_lo));
   // Every CTA reads the same weight tiles; starting each CTA at a different K step keeps
-  // them from all hitting the same L2 lines at once.  (Only the FP32 summation order
-  // changes with the start.)
-  const int k_start = k_tiles > 0 ? static_cast<int>(blockIdx.x % static_cast<unsigned>(k_tiles)) : 0;
+  // them from all hitting the same L2 lines at once.  Only the FP32 summation order changes
+  // with the start, which follows the tile's index in the whole batch (tile_base: this
+  // launch's first tile), so a batch routed in parts sums every token's logits alike.
+  const int k_start = k_tiles > 0 ? (tile_base + static_cast<int>(blockIdx.x)) % k_tiles : 0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -315,24 +316,26 @@ int router_tc_tokens_per_cta(int T, int num_sms) {
 template <int HALVES>
 static cudaError_t launch_router_tc_t(const CUtensorMap& map_x, const uint16_t* w_tiles, int T, int H, int E, int k,
                                       float* logits, int32_t* ids, float* wout, uint32_t* err, int splits,
-                                      cudaStream_t s) {
+                                      int tile_base, cudaStream_t s) {
   using S = RtShape<HALVES>;
   const size_t smem = router_tc_smem<HALVES>(E);
   cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<HALVES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_pdl(router_tc_kernel<HALVES>, dim3((T + S::BM - 1) / S::BM, splits), dim3(S::THREADS), smem, s,
-                    map_x, reinterpret_cast<const uint8_t*>(w_tiles), T, H, E, k, logits, ids, wout, err, splits);
+                    map_x, reinterpret_cast<const uint8_t*>(w_tiles), T, H, E, k, logits, ids, wout, err, splits,
+                    tile_base);
 }
 
 cudaError_t launch_router_tc(const CUtensorMap& map_x, int tokens_per_cta, const uint16_t* w_tiles, int T, int H,
                              int E, int k, float* logits, int32_t* ids, float* wout, uint32_t* err, cudaStream_t s,
-                             int splits) {
-  if (splits < 1) return cudaErrorInvalidValue;
+                             int splits, int first_token) {
+  if (splits < 1 || first_token % tokens_per_cta != 0) return cudaErrorInvalidValue;
+  const int tile_base = first_token / tokens_per_cta;
   if (tokens_per_cta == 2 * RT_MMA_M)
-    return launch_router_tc_t<2>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, splits, s);
+    return launch_router_tc_t<2>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, splits, tile_base, s);
   if (tokens_per_cta == RT_MMA_M)
-    return launch_router_tc_t<1>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, splits, s);
+    return launch_router_tc_t<1>(map_x, w_tiles, T, H, E, k, logits, ids, wout, err, splits, tile_base, s);
   return cudaErrorInvalidValue;
 }
 

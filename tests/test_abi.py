@@ -23,6 +23,8 @@ def test_header_constants_match_the_binding(repo_root):
     text = open(os.path.join(repo_root, "include", "beam_moe.h")).read()
     m = re.search(r"#define BEAM_MOE_TP_TWO_SHOT_MIN_TOKENS (\d+)", text)
     assert m and int(m.group(1)) == pkg.TP_TWO_SHOT_MIN_TOKENS
+    m = re.search(r"#define BEAM_MOE_HOST_CHUNK_TOKENS (\d+)", text)
+    assert m and int(m.group(1)) == pkg.HOST_CHUNK_TOKENS
 
 
 def test_library_exports_every_declared_symbol(repo_root):
@@ -79,6 +81,7 @@ def test_host_side_validation_of_the_variant_and_parallel_entry_points():
     assert lib.beam_moe_expert_format(None) == -1
     assert lib.beam_moe_set_router_mode(None, pkg.ROUTER_AUTO) == bad
     assert lib.beam_moe_set_tp_two_shot_tokens(None, 256) == bad
+    assert lib.beam_moe_set_host_chunk_tokens(None, 4096) == bad
     assert lib.beam_moe_tp_region_bytes(None) == 0
     p = ctypes.c_void_p()
     assert lib.beam_moe_tp_region(None, ctypes.byref(p)) == bad

@@ -305,6 +305,36 @@ def test_forward_host_buffers_match_device_path(bm, fmt):
     layer.close()
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
+def test_forward_host_in_parts_matches_device_path(bm, fmt):
+    # beam_moe_forward_host of a batch of 2 parts or more: each part uploads, computes and
+    # copies back on its own schedule, with the whole batch's router (forms, slices and the
+    # K order of each token tile), finalize and GEMM forms.  Same bits as the device-buffer
+    # forward of the whole batch, for parts of 256 and 512 tokens, ragged last parts (one of
+    # 188 tokens: the small-batch A1 writer inside it), call after call.
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(SHAPES["mid"], tokens=700)
+    weights = synthetic.make_weights(shape, 5, threads=4, fmt=fmt)
+    kw = dict(alpha_a1=0.002, alpha_a2=0.0002) if fmt == "nvfp4" else dict(fmt="mxfp8")
+    layer = bm.MoELayer(max_tokens=700, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                        inter=shape.inter, **kw, **weights)
+    xd, rd = synthetic.make_batch(shape, 5)
+    with pytest.raises(bm.BeamMoeError):
+        layer.set_host_chunk_tokens(100)  # parts align with the router's token tiles
+    for chunk, T in [(256, 700), (512, 700), (256, 512), (256, 511), (0, 700), (256, 700)]:
+        layer.set_host_chunk_tokens(chunk)
+        xh, rh = xd[:T].cpu().pin_memory(), rd[:T].cpu().pin_memory()
+        oh = torch.empty_like(rh).pin_memory()
+        layer.forward_host(xh, rh, oh)
+        torch.cuda.synchronize()
+        layer.check()
+        ref = layer.forward(xd[:T], rd[:T])
+        torch.cuda.synchronize()
+        assert torch.equal(oh, ref.cpu()), (chunk, T)
+    layer.check()
+    layer.close()
+
+
 def test_profiled_sections_and_launch_counts(bm):
     """Per-kernel timing of a forward (beam_moe_profile_enable / _read): one named section per
     kernel launched, in launch order, ending with the finalize; the output is the same bits
