@@ -463,6 +463,7 @@ def measure_workload(args, layer, shape, rank, world, dev, flush_l2, want_parity
     e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)) / args.steps, world, dev)
     ref_out = layer.forward(x, res)
     assert torch.equal(oh.to(dev), ref_out), "host-buffer path differs from device path"
+    graph = graph_replay(args, layer, x, res, ref_out, flush_l2, world, dev)
     gpu = None
     if want_parity:
         ids = layer.debug(bm.BUF_IDS).cpu().numpy().view(np.int32).reshape(T, shape.top_k).astype(np.int64)
@@ -473,8 +474,88 @@ def measure_workload(args, layer, shape, rank, world, dev, flush_l2, want_parity
         "roofline": roofline_of(kern, work, fmt, T), "kernels_ms": kern, "used_experts": work["_used_experts"],
         "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * T * shape.hidden * 2,
                 "d2h_bytes_per_step": T * shape.hidden * 2},
-        "gpu_launches": launches, "clocks": clk.summary(),
+        "gpu_launches": launches, "clocks": clk.summary(), "cuda_graph": graph,
     }, gpu
+
+
+def graph_replay(args, layer, x, res, ref_out, flush_l2, world, dev):
+    """The same step captured once in a CUDA graph and replayed (the plain stream above is the
+    headline): per-step time with the same flush protocol, and the replay's output against
+    the plain forward's bits."""
+    import torch
+    out = torch.empty_like(res)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer.forward(x, res, out)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(x, res, out)
+    for _ in range(max(args.warmup, 3)):
+        g.replay()
+        flush_l2()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        s_ev[i].record(stream)
+        g.replay()
+        e_ev[i].record(stream)
+        flush_l2()
+    torch.cuda.synchronize()
+    layer.check()
+    ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(s_ev, e_ev)) / args.steps, world, dev)
+    same = bool(torch.equal(out, ref_out))
+    assert same, "graph replay differs from the plain forward"
+    del g
+    return {"ms_per_step": ms, "same_bits_as_plain": same}
+
+
+def library_peaks(steps: int = 20):
+    """Dense GEMM rates of library kernels at 8192^3 on this GPU, as context for the
+    rooflines: cuBLAS BF16 (torch.mm) and the block-scaled NVFP4 GEMM behind
+    torch._scaled_mm (E2M1 operands, one E4M3 scale per 16 values).  L2 flushed before each
+    launch; median of `steps`."""
+    import statistics
+    import torch
+    M = N = K = 8192
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def rate(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.median(ts)
+        return {"ms": ms, "tflops": 2.0 * M * N * K / ms / 1e9}
+
+    g = torch.Generator(device="cuda").manual_seed(0)
+    xa = torch.randn(M, K, dtype=torch.bfloat16, device="cuda", generator=g)
+    xb = torch.randn(K, N, dtype=torch.bfloat16, device="cuda", generator=g)
+    out = {"shape": [M, N, K], "bf16_torch_mm": rate(lambda: torch.mm(xa, xb))}
+    del xa, xb
+    a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device="cuda", generator=g)
+    b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device="cuda", generator=g)
+    sa = torch.full((M, K // 16), 0x38, dtype=torch.uint8, device="cuda")  # E4M3 1.0
+    sb = torch.full((N, K // 16), 0x38, dtype=torch.uint8, device="cuda")
+    fa, fb = a.view(torch.float4_e2m1fn_x2), b.view(torch.float4_e2m1fn_x2)
+    ea, eb = sa.view(torch.float8_e4m3fn), sb.view(torch.float8_e4m3fn)
+    try:
+        out["nvfp4_torch_scaled_mm"] = rate(lambda: torch._scaled_mm(fa, fb.t(), ea, eb, out_dtype=torch.bfloat16))
+    except Exception as ex:  # a torch build without the FP4 GEMM
+        out["nvfp4_torch_scaled_mm"] = {"unavailable": f"{type(ex).__name__}: {str(ex)[:200]}"}
+    return out
 
 
 def run_ours(args, shapes, rank, world, local_rank):
@@ -683,7 +764,12 @@ def main():
                     help="expert-parallel layer with W ranks (each its own batch) sharing this one GPU, run in turn")
     ap.add_argument("--experts-format", default="nvfp4", choices=["nvfp4", "mxfp8"],
                     help="routed experts in NVFP4 (default) or the block-scaled FP8 variant (MXFP8)")
+    ap.add_argument("--library-peaks", action="store_true",
+                    help="print library GEMM rates at 8192^3 (cuBLAS BF16, NVFP4 scaled_mm) and exit")
     args = ap.parse_args()
+    if args.library_peaks:
+        print(json.dumps({"library_peaks": library_peaks()}))
+        return
     names = DEFAULT_WORKLOADS if args.workload == "default" else (args.workload,)
     shapes = [mi.SHAPES[n] for n in names]
     rank = int(os.environ.get("RANK", 0))

@@ -360,3 +360,36 @@ def test_profiled_sections_and_launch_counts(bm):
         assert all(ms >= 0 for _, ms in sections)
         assert layer.launches() == len(names), (T, names)
     layer.close()
+
+
+@pytest.mark.parametrize("tokens", [8, 300])
+def test_forward_replays_from_a_cuda_graph(bm, tokens):
+    # The forward enqueues only kernels on the caller's stream (no allocation, no host sync),
+    # so it can be captured in a CUDA graph once and replayed; each replay gives the eager
+    # forward's bits, and replays of new inputs copied into the captured buffers follow them.
+    from sparse_moe_layer_fp32_b200 import synthetic
+    shape = dataclasses.replace(SHAPES["mid"], tokens=tokens)
+    weights = synthetic.make_weights(shape, 9, threads=4)
+    layer = bm.MoELayer(max_tokens=tokens, hidden=shape.hidden, num_experts=shape.experts, top_k=shape.top_k,
+                        inter=shape.inter, alpha_a1=0.002, alpha_a2=0.0002, **weights)
+    x0, r0 = synthetic.make_batch(shape, 9)
+    x1, r1 = synthetic.make_batch(shape, 10)
+    x, r = x0.cuda().clone(), r0.cuda().clone()
+    out = torch.empty_like(r)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer.forward(x, r, out)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(x, r, out)
+    for xs, rs in [(x0, r0), (x1, r1), (x0, r0)]:
+        x.copy_(xs.cuda())
+        r.copy_(rs.cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        layer.check()
+        assert torch.equal(out, layer.forward(xs.cuda(), rs.cuda()))
+    del g
+    layer.close()
