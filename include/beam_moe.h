@@ -154,6 +154,10 @@ BEAM_MOE_API beam_moe_status beam_moe_forward_prenorm(beam_moe_t h, const void* 
  * parts take the whole batch's router, finalize and GEMM forms, so out has the same bits as
  * without parts.  Not with BEAM_MOE_ROUTER_SIMT.  After such a call the internal buffers
  * (beam_moe_debug_copy) and the kernel timings hold the last part's.
+ * An out of at most 2 MB in page-locked memory that the device can address (cudaHostAlloc,
+ * or registered with cudaHostRegisterMapped) is written by the finalize kernel directly, with
+ * no copy after it; larger outs and other host memory go through a staging buffer and a
+ * copy back.
  * All copies are cudaMemcpyAsync; pinned host memory makes them asynchronous.  The work
  * enqueued on `stream` ends with out_host complete: the caller synchronises `stream` before
  * reading it. */
