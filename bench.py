@@ -75,7 +75,6 @@ def kernel_work(shape: mi.LayerShape, T: int, counts: np.ndarray, fmt: str = "nv
         "chunk_hist": dict(bytes=R * 4, flops=0),
         "scan": dict(bytes=E * 16, flops=0),
         "scatter": dict(bytes=R * 12, flops=0),
-        "topk_route": dict(bytes=T * E * 4 + R * 8 + R * 12, flops=0),
         "quant_a1": dict(bytes=T * H * 2 + R * H * q, flops=0),
         # gate/up + down in one launch: both weight sets of the used experts, A1 read, the
         # NVFP4 intermediate A2 written and read back, y written (BF16)

@@ -35,7 +35,6 @@ struct beam_moe_ctx {
   uint16_t* y;
   uint32_t* err;
   unsigned int* route_counter;  // last-CTA election of the fused small-batch routing kernel
-  unsigned int* topk_counter;   // ... and of the fused top-k + permutation kernel
   uint32_t* sched;              // tile scheduler of the expert GEMM launch (sched_words(nblk_max))
   int32_t router_mode;          // BEAM_MOE_ROUTER_*: which router batches of more than 16 tokens use
   int32_t fmt;                  // BEAM_MOE_FMT_*: expert weight and activation format
@@ -338,9 +337,6 @@ beam_moe_status create_impl(const beam_moe_config* cfg, const ExpertWeightsIn& w
   CREATE_TRY(dalloc(h, &h->err, sizeof(uint32_t)));
   CREATE_TRY(dalloc(h, &h->route_counter, sizeof(unsigned int)));
   CREATE_TRY(cudaMemsetAsync(h->route_counter, 0, sizeof(unsigned int), s));
-  CREATE_TRY(dalloc(h, &h->topk_counter, sizeof(unsigned int)));
-  CREATE_TRY(cudaMemsetAsync(h->topk_counter, 0, sizeof(unsigned int), s));
-  CREATE_TRY(cudaMemsetAsync(h->chunk_counts, 0, sizeof(int32_t) * h->n_chunks_max * E, s));
   CREATE_TRY(dalloc(h, &h->sched, sizeof(uint32_t) * sched_words(h->nblk_max)));
   CREATE_TRY(dalloc(h, &h->stage_x, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
   CREATE_TRY(dalloc(h, &h->stage_res, sizeof(uint16_t) * static_cast<size_t>(h->Tmax) * H));
@@ -589,24 +585,6 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
     h->last_splits = slices;
   } else {
     const bool simt_only = h->router_mode == BEAM_MOE_ROUTER_SIMT;
-    // Top-k over the summed slices; up to kFusedRouteTokens tokens the same launch also
-    // builds the permutation (then chunk_hist, scan and scatter are skipped).
-    bool permuted = false;
-    auto topk_and_permute = [&](int splits) -> cudaError_t {
-      cudaError_t e;
-      if (topk_route_supported(T, E, k)) {
-        e = launch_topk_route(h->logits, splits, T, E, k, h->ids, h->w, h->chunk_counts, h->topk_counter,
-                              h->chunk_base, h->offsets, h->sf_block, h->mblocks, h->num_mblocks, h->sched,
-                              static_cast<int>(sched_words(h->nblk_max)), bscales, h->perm, h->inv, h->tile_row, s);
-        if (e == cudaSuccess) e = mark("topk_route");
-        permuted = true;
-      } else {
-        e = launch_topk(h->logits, splits, T, E, k, h->ids, h->w, s);
-        if (e == cudaSuccess) e = mark("topk");
-      }
-      ++launches;
-      return e;
-    };
     // AUTO and TENSOR: slices of H whenever the split count is above one (measured faster than
     // one tile per CTA at every batch up to 32K tokens, and than the SIMT router from 17)
     const bool tc_split = !simt_only && router_tc_split_supported(H, E, k) && PT >= kRouterTcSplitMinTokens &&
@@ -623,7 +601,9 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
       BEAM_TRY(mark("router_tc"));
       ++launches;
       h->last_splits = splits;
-      BEAM_TRY(topk_and_permute(splits));
+      BEAM_TRY(launch_topk(h->logits, splits, T, E, k, h->ids, h->w, s));
+      BEAM_TRY(mark("topk"));
+      ++launches;
     } else if (!simt_only && router_tc_supported(PT, H, E, k)) {
       // FP32-class logits on the tensor cores (BF16 x 3-part split), top-k in the epilogue
       CUtensorMap map_x;
@@ -639,21 +619,21 @@ static beam_moe_status forward_impl(beam_moe_t h, const void* x, const void* res
       BEAM_TRY(mark("router"));
       ++launches;
       h->last_splits = router_split_count(T, H, E);
-      BEAM_TRY(topk_and_permute(h->last_splits));
-    }
-    if (!permuted) {
-      BEAM_TRY(launch_chunk_hist(h->ids, T, k, E, h->chunk_counts, s));
-      BEAM_TRY(mark("chunk_hist"));
-      ++launches;
-      BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
-                           h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), bscales, s));
-      BEAM_TRY(mark("scan"));
-      ++launches;
-      BEAM_TRY(launch_scatter(h->ids, h->chunk_base, h->offsets, h->sf_block, T, k, E, h->perm, h->inv, h->tile_row,
-                              s));
-      BEAM_TRY(mark("scatter"));
+      BEAM_TRY(launch_topk(h->logits, h->last_splits, T, E, k, h->ids, h->w, s));
+      BEAM_TRY(mark("topk"));
       ++launches;
     }
+    BEAM_TRY(launch_chunk_hist(h->ids, T, k, E, h->chunk_counts, s));
+    BEAM_TRY(mark("chunk_hist"));
+    ++launches;
+    BEAM_TRY(launch_scan(h->chunk_counts, n_chunks, E, h->chunk_base, h->offsets, h->sf_block, h->mblocks,
+                         h->num_mblocks, h->sched, static_cast<int>(sched_words(h->nblk_max)), bscales, s));
+    BEAM_TRY(mark("scan"));
+    ++launches;
+    BEAM_TRY(launch_scatter(h->ids, h->chunk_base, h->offsets, h->sf_block, T, k, E, h->perm, h->inv, h->tile_row,
+                            s));
+    BEAM_TRY(mark("scatter"));
+    ++launches;
   }
   if (ep_phase == 0) {  // this rank's per-expert row counts to every rank
     BEAM_TRY(launch_ep_counts(h->offsets, E, h->tp, h->ep_lay, h->tp_epoch + 1, s));

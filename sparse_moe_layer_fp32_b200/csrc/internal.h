@@ -82,26 +82,14 @@ cudaError_t launch_route_small(const uint16_t* x, const float* w, int T, int H, 
 
 // ---- permutation and activation quantisation (routing.cu)
 cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* chunk_counts, cudaStream_t s);
-// Also zeroes sched[0, sched_n), the tile scheduler words of the expert GEMM launch, and the
-// chunk counts it read (the counting of launch_topk_route adds into zeroed counts).
-cudaError_t launch_scan(int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
+// Also zeroes sched[0, sched_n), the tile scheduler words of the expert GEMM launch.
+cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
                         BlockScales bs, cudaStream_t s);
 // tile_row[t][j] = 128 x activation block + row within it, for slot (t, j).
 cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const int32_t* offsets,
                            const int32_t* sf_block, int T, int k, int E, int32_t* perm_src, int32_t* inv,
                            int32_t* tile_row, cudaStream_t s);
-// launch_topk + launch_chunk_hist + launch_scan + launch_scatter in one launch, for batches
-// of up to kFusedRouteTokens tokens and E <= 256: the last CTA to finish its tokens runs the
-// scan and the scatter (elected through done_counter, which it resets).  chunk_counts must be
-// zero on entry (create zeroes them; every scan zeroes what it read).
-constexpr int kFusedRouteTokens = 1024;  // its last CTA scatters the chunks one after another
-bool topk_route_supported(int T, int E, int k);
-cudaError_t launch_topk_route(const float* logits, int splits, int T, int E, int k, int32_t* ids, float* w,
-                              int32_t* chunk_counts, unsigned int* done_counter, int32_t* chunk_base,
-                              int32_t* offsets, int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks,
-                              uint32_t* sched, int sched_n, BlockScales bs, int32_t* perm_src, int32_t* inv,
-                              int32_t* tile_row, cudaStream_t s);
 // A1 = Q(x) into the activation units: [blk][H/256][18432], codes then scales (common.cuh).
 cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, float alpha, uint8_t* a1,
                             cudaStream_t s);

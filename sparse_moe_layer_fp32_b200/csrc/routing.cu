@@ -17,7 +17,6 @@
 // checkpoint, read as MXFP8), A1 = MX(x) in 32-value blocks.
 #include "common.cuh"
 #include "internal.h"
-#include "topk.cuh"
 
 namespace beam {
 
@@ -39,13 +38,15 @@ __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restri
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[static_cast<size_t>(blockIdx.x) * E + e] = cnt[e];
 }
 
-// The scan over one CTA, one thread per expert (blockDim >= E, a multiple of 32).  It also
-// zeroes the counts it read, so the next forward's counting may accumulate into them.
-__device__ __forceinline__ void scan_blocks(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
-                                            int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
-                                            int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks,
-                                            int32_t* __restrict__ num_mblocks, uint32_t* __restrict__ sched,
-                                            int sched_n, const BlockScales& bs, int* warp_sums) {
+// One CTA, one thread per expert.
+__global__ void scan_kernel(const int32_t* __restrict__ chunk_counts, int n_chunks, int E,
+                            int32_t* __restrict__ chunk_base, int32_t* __restrict__ offsets,
+                            int32_t* __restrict__ sf_block, MBlock* __restrict__ mblocks,
+                            int32_t* __restrict__ num_mblocks, uint32_t* __restrict__ sched, int sched_n,
+                            BlockScales bs) {
+  __shared__ int warp_sums[33];
+  pdl_wait();
+  pdl_trigger();
   // the expert GEMM launch that follows starts from zeroed scheduler words
   for (int i = threadIdx.x; i < sched_n; i += blockDim.x) sched[i] = 0u;
   const int e = threadIdx.x;
@@ -53,8 +54,7 @@ __device__ __forceinline__ void scan_blocks(int32_t* __restrict__ chunk_counts, 
   if (e < E) {
     for (int c = 0; c < n_chunks; ++c) {
       const size_t i = static_cast<size_t>(c) * E + e;
-      const int v = __ldcg(chunk_counts + i);
-      chunk_counts[i] = 0;
+      const int v = chunk_counts[i];
       chunk_base[i] = cnt;
       cnt += v;
     }
@@ -90,31 +90,24 @@ __device__ __forceinline__ void scan_blocks(int32_t* __restrict__ chunk_counts, 
   }
 }
 
-// One CTA, one thread per expert.
-__global__ void scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E, int32_t* __restrict__ chunk_base,
-                            int32_t* __restrict__ offsets, int32_t* __restrict__ sf_block,
-                            MBlock* __restrict__ mblocks, int32_t* __restrict__ num_mblocks,
-                            uint32_t* __restrict__ sched, int sched_n, BlockScales bs) {
-  __shared__ int warp_sums[33];
-  pdl_wait();
-  pdl_trigger();
-  scan_blocks(chunk_counts, n_chunks, E, chunk_base, offsets, sf_block, mblocks, num_mblocks, sched, sched_n, bs,
-              warp_sums);
-}
-
 // perm_src[r] = t, inv[t][j] = r and tile_row[t][j] (128 x activation block + row in the
 // block, the row's place in the activation tiles) for every (t, j) of one chunk of 256
-// tokens, by one CTA of 256 threads; sm: 16 E words of shared memory.
-__device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ ids, const int32_t* __restrict__ chunk_base,
-                                              const int32_t* __restrict__ offsets,
-                                              const int32_t* __restrict__ sf_block, int T, int k, int E, int chunk,
-                                              int32_t* __restrict__ perm_src, int32_t* __restrict__ inv,
-                                              int32_t* __restrict__ tile_row, uint32_t* sm) {
+// tokens.
+__global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ ids,
+                                                      const int32_t* __restrict__ chunk_base,
+                                                      const int32_t* __restrict__ offsets,
+                                                      const int32_t* __restrict__ sf_block, int T, int k, int E,
+                                                      int32_t* __restrict__ perm_src, int32_t* __restrict__ inv,
+                                                      int32_t* __restrict__ tile_row) {
+  extern __shared__ uint32_t sm[];
   uint32_t* mask = sm;                                    // [8][E]
   int32_t* pre = reinterpret_cast<int32_t*>(sm + 8 * E);  // [8][E]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) mask[i] = 0;
   __syncthreads();
+  const int chunk = blockIdx.x;
   const int t = chunk * kChunkTokens + warp * 32 + lane;
   if (t < T)
     for (int j = 0; j < k; ++j) atomicOr(&mask[warp * E + ids[static_cast<size_t>(t) * k + j]], 1u << lane);
@@ -140,75 +133,6 @@ __device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ ids, c
       tile_row[static_cast<size_t>(t) * k + j] = (sf_block[e] + (li >> 7)) * 128 + (li & 127);
     }
   }
-  __syncthreads();  // the shared masks are free for the next chunk
-}
-
-__global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ ids,
-                                                      const int32_t* __restrict__ chunk_base,
-                                                      const int32_t* __restrict__ offsets,
-                                                      const int32_t* __restrict__ sf_block, int T, int k, int E,
-                                                      int32_t* __restrict__ perm_src, int32_t* __restrict__ inv,
-                                                      int32_t* __restrict__ tile_row) {
-  extern __shared__ uint32_t sm[];
-  pdl_wait();
-  pdl_trigger();
-  scatter_chunk(ids, chunk_base, offsets, sf_block, T, k, E, blockIdx.x, perm_src, inv, tile_row, sm);
-}
-
-// Batches of up to kFusedRouteTokens tokens: the top-k (warp per token, the slices of the
-// partial logits summed in order, as topk_kernel), the per-chunk expert counts (integer
-// atomics: their sums do not depend on order), then the last CTA to finish runs the scan and
-// the scatter of every chunk, in one launch instead of four.  The same ids, weights,
-// offsets, blocks and permutation as topk_kernel + chunk_hist + scan + scatter.
-template <int EPL>
-__global__ void __launch_bounds__(256) topk_route_kernel(const float* __restrict__ partial, int splits, int T, int E,
-                                                         int k, int32_t* __restrict__ ids, float* __restrict__ wout,
-                                                         int32_t* __restrict__ chunk_counts,
-                                                         unsigned int* __restrict__ done_counter,
-                                                         int32_t* __restrict__ chunk_base,
-                                                         int32_t* __restrict__ offsets, int32_t* __restrict__ sf_block,
-                                                         MBlock* __restrict__ mblocks,
-                                                         int32_t* __restrict__ num_mblocks,
-                                                         uint32_t* __restrict__ sched, int sched_n, BlockScales bs,
-                                                         int32_t* __restrict__ perm_src, int32_t* __restrict__ inv,
-                                                         int32_t* __restrict__ tile_row) {
-  extern __shared__ uint32_t sm[];  // the scatter's 16 E words
-  __shared__ int warp_sums[33];
-  __shared__ int s_last;
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  pdl_wait();
-  pdl_trigger();
-  if (t < T) {
-    float v[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) v[i] = lane + 32 * i < E ? 0.0f : -INFINITY;
-    for (int sp = 0; sp < splits; ++sp) {
-      const float* row = partial + (static_cast<size_t>(sp) * T + t) * E;
-      float p[EPL];
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) p[i] = lane + 32 * i < E ? __ldcs(row + lane + 32 * i) : 0.0f;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) v[i] += p[i];
-    }
-    int32_t* tid_row = ids + static_cast<size_t>(t) * k;
-    warp_topk<EPL>(v, E, k, lane, tid_row, wout + static_cast<size_t>(t) * k);
-    __syncwarp();
-    if (lane < k) atomicAdd(chunk_counts + static_cast<size_t>(t / kChunkTokens) * E + tid_row[lane], 1);
-  }
-  // The barrier orders every thread's ids, weights and counts before thread 0's release add;
-  // the last CTA's acquire then sees every CTA's.
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atom_add_acq_rel_gpu(done_counter, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!s_last) return;
-  if (threadIdx.x == 0) *done_counter = 0u;  // the next launch's election
-  const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
-  scan_blocks(chunk_counts, n_chunks, E, chunk_base, offsets, sf_block, mblocks, num_mblocks, sched, sched_n, bs,
-              warp_sums);
-  __syncthreads();
-  for (int c = 0; c < n_chunks; ++c)
-    scatter_chunk(ids, chunk_base, offsets, sf_block, T, k, E, c, perm_src, inv, tile_row, sm);
 }
 
 // One thread per 16-value block of x: quantise it once and write it to the token's k
@@ -432,7 +356,7 @@ cudaError_t launch_chunk_hist(const int32_t* ids, int T, int k, int E, int32_t* 
                     chunk_counts);
 }
 
-cudaError_t launch_scan(int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
+cudaError_t launch_scan(const int32_t* chunk_counts, int n_chunks, int E, int32_t* chunk_base, int32_t* offsets,
                         int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks, uint32_t* sched, int sched_n,
                         BlockScales bs, cudaStream_t s) {
   const int threads = ((E + 31) / 32) * 32;
@@ -452,30 +376,6 @@ cudaError_t launch_scatter(const int32_t* ids, const int32_t* chunk_base, const 
   }
   return launch_pdl(scatter_kernel, dim3(n_chunks), dim3(256), smem, s, ids, chunk_base, offsets, sf_block, T, k, E,
                     perm_src, inv, tile_row);
-}
-
-bool topk_route_supported(int T, int E, int k) {
-  return T >= 1 && T <= kFusedRouteTokens && E >= 1 && E <= 256 && k >= 1 && k <= 16 && k <= E;
-}
-
-cudaError_t launch_topk_route(const float* logits, int splits, int T, int E, int k, int32_t* ids, float* w,
-                              int32_t* chunk_counts, unsigned int* done_counter, int32_t* chunk_base,
-                              int32_t* offsets, int32_t* sf_block, MBlock* mblocks, int32_t* num_mblocks,
-                              uint32_t* sched, int sched_n, BlockScales bs, int32_t* perm_src, int32_t* inv,
-                              int32_t* tile_row, cudaStream_t s) {
-  if (!topk_route_supported(T, E, k)) return cudaErrorInvalidValue;
-  const dim3 grid((T + 7) / 8);
-  const size_t smem = static_cast<size_t>(16) * E * sizeof(uint32_t);
-  const int epl = (E + 31) / 32;
-#define TOPK_ROUTE(N)                                                                                                \
-  return launch_pdl(topk_route_kernel<N>, grid, dim3(256), smem, s, logits, splits, T, E, k, ids, w, chunk_counts, \
-                    done_counter, chunk_base, offsets, sf_block, mblocks, num_mblocks, sched, sched_n, bs, perm_src, \
-                    inv, tile_row)
-  if (epl <= 1) TOPK_ROUTE(1);
-  if (epl <= 2) TOPK_ROUTE(2);
-  if (epl <= 4) TOPK_ROUTE(4);
-  TOPK_ROUTE(8);
-#undef TOPK_ROUTE
 }
 
 cudaError_t launch_quant_a1(const uint16_t* x, const int32_t* tile_row, int T, int H, int k, float alpha, uint8_t* a1,
