@@ -923,12 +923,12 @@ beam_moe_status beam_moe_forward_host(beam_moe_t h, const void* x_host, const vo
   // engine, which moves them faster than the finalize's stores (spec1024: 1.038 vs 1.031 M);
   // pageable memory always does.
   void* out_dev = nullptr;
-  cudaPointerAttributes pa{};
-  if (bytes > kMaxDirectOutBytes) {
-  } else if (cudaPointerGetAttributes(&pa, out_host) == cudaSuccess) {
-    if (pa.type == cudaMemoryTypeHost && pa.devicePointer && aligned(pa.devicePointer, 16)) out_dev = pa.devicePointer;
-  } else {
-    (void)cudaGetLastError();  // an unknown pointer is pageable memory here: clear and copy
+  if (bytes <= kMaxDirectOutBytes) {
+    cudaPointerAttributes pa{};
+    if (cudaPointerGetAttributes(&pa, out_host) != cudaSuccess)
+      (void)cudaGetLastError();  // an unknown pointer is pageable memory here: clear and copy
+    else if (pa.type == cudaMemoryTypeHost && pa.devicePointer && aligned(pa.devicePointer, 16))
+      out_dev = pa.devicePointer;
   }
   beam_moe_status st = forward_impl(h, h->stage_x, h->stage_res, out_dev ? out_dev : h->stage_out, nullptr, nullptr,
                                     0.0f, num_tokens, stream, -1, h->ev_res);
