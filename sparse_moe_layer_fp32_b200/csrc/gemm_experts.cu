@@ -24,13 +24,13 @@
 //
 // CTA layout (one persistent CTA per SM, 704 threads, warp-specialised):
 //   warp 0      producer: claims tiles, publishes each tile id through a small shared
-//               ring, and per 256-wide K step bulk-copies the A tile (the valid rows of a
-//               128-row activation tile, <= 16 KB), the expert's weight tile with its
-//               scales (32 KB + 4 KB) and the A scales (2 KB: the K step's chunk of 128
-//               rows x 16 scale bytes; MXFP8: one 512-byte atom) into the stage ring, all
-//               landing on one mbarrier.  Activations and weights are both stored as
-//               contiguous tiles already in the swizzled shared-memory order, so every
-//               load is one sequential copy.
+//               ring, and per 256-wide K step bulk-copies the expert's weight tile with its
+//               scales (32 KB + 4 KB) and the block's activation unit (16 KB of codes, then
+//               the K step's 128 rows x 16 scale bytes; MXFP8: one 512-byte atom) into the
+//               stage ring, all landing on one mbarrier: two copies for a block of 128 rows,
+//               and for a block of fewer rows its valid rows' codes and scales (two copies).
+//               Activations and weights are both stored already in the swizzled
+//               shared-memory order, so every load is one sequential copy.
 //   warp 1      TMEM owner; lane 0 issues tcgen05.mma.kind::mxf4nvf4.block_scale.block16
 //               (M=128, N=256, K=64) into a 128x256 FP32 accumulator in TMEM and
 //               tcgen05.commit to free stages.
